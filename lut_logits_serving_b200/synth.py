@@ -1,0 +1,115 @@
+"""Seeded synthetic inputs for RQ-LUT logits serving.
+
+This module only draws random numbers in the shapes and distributions of
+the workloads; it holds none of the method's arithmetic.  Both the CUDA
+library's tests/benchmark and the CPU oracle's tests take their inputs from
+here.
+
+Seeds: one ``numpy.random.default_rng`` stream per tensor, derived from a
+base seed: codebooks = seed, codes = seed + 1, hidden states = seed + 2,
+token ids = seed + 3.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    V: int
+    D: int
+    M: int
+    L: int
+    K: int
+    B: int                      # tokens per logits call (0: decode-only)
+    sigmas: tuple               # codebook std per residual level
+    hidden_scale: float         # hidden ~ N(0, 1) * hidden_scale
+    softcap: float = 30.0
+    packed10: bool = False
+    argmax: bool = False
+    n_ids: int = 0              # input rows rebuilt per call
+    zipf_s: float = 1.1
+    decode_scale: float = 0.0   # embedding scale applied to rebuilt rows
+
+    @property
+    def ds(self) -> int:
+        return self.D // self.M
+
+    @property
+    def P(self) -> int:
+        return self.M * self.L
+
+
+# Shapes follow the pages' Gemma-2-2B tied embedding (V=256000, D=2304) with
+# the RQ artifact M=384, K=1024, L=2, plus one tiny case for quick checks.
+WORKLOADS = {
+    "tiny": Workload("tiny", V=4096, D=192, M=32, L=2, K=256, B=1,
+                     sigmas=(0.05, 0.01), hidden_scale=1.0),
+    "g2_b1": Workload("g2_b1", V=256000, D=2304, M=384, L=2, K=1024, B=1,
+                      sigmas=(0.02, 0.005), hidden_scale=40.0 / math.sqrt(2304.0),
+                      argmax=True, n_ids=1, decode_scale=math.sqrt(2304.0)),
+    "g2_b32": Workload("g2_b32", V=256000, D=2304, M=384, L=2, K=1024, B=32,
+                       sigmas=(0.02, 0.005), hidden_scale=0.83,
+                       argmax=True, n_ids=32, decode_scale=math.sqrt(2304.0)),
+    "decode512": Workload("decode512", V=256000, D=2304, M=384, L=2, K=1024, B=0,
+                          sigmas=(0.02, 0.005), hidden_scale=0.83,
+                          n_ids=512, decode_scale=math.sqrt(2304.0)),
+    "packed_b64": Workload("packed_b64", V=256000, D=2304, M=384, L=2, K=1024, B=64,
+                           sigmas=(0.02, 0.005), hidden_scale=0.83, packed10=True,
+                           argmax=True, n_ids=64, decode_scale=math.sqrt(2304.0)),
+}
+
+
+def codebooks(M: int, L: int, K: int, ds: int, sigmas, seed: int = 0) -> np.ndarray:
+    """float32 [M, L, K, ds]; level l ~ N(0, sigmas[l])."""
+    rng = np.random.default_rng(seed)
+    C = np.empty((M, L, K, ds), np.float32)
+    for l in range(L):
+        s = sigmas[min(l, len(sigmas) - 1)]
+        C[:, l] = rng.standard_normal((M, K, ds), dtype=np.float32) * np.float32(s)
+    return C
+
+
+def codes(V: int, M: int, L: int, K: int, seed: int = 1) -> np.ndarray:
+    """uint16 [V, M, L], uniform in [0, K)."""
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, K, size=(V, M, L), dtype=np.uint16)
+
+
+def hidden(B: int, D: int, scale: float, seed: int = 2) -> np.ndarray:
+    """float32 [B, D] ~ N(0, 1) * scale."""
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((B, D), dtype=np.float32) * np.float32(scale)
+
+
+def zipf_ids(N: int, V: int, s: float = 1.1, seed: int = 3) -> np.ndarray:
+    """int32 [N] token ids: rank r in 1..V drawn with P(r) ~ r^-s by inverse
+    CDF on the finite support, mapped through a seeded permutation of
+    [0, V) so frequent ids are spread over the vocabulary.  Repeats kept."""
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(V)
+    w = np.arange(1, V + 1, dtype=np.float64) ** (-s)
+    cdf = np.cumsum(w)
+    cdf /= cdf[-1]
+    u = rng.random(N)
+    r = np.minimum(np.searchsorted(cdf, u, side="right"), V - 1)
+    return perm[r].astype(np.int32)
+
+
+def make(w: Workload, seed: int = 0, V: int | None = None):
+    """All inputs of a workload: dict with C, codes, h, ids (V may be cut for
+    a smaller sample of the same distributions)."""
+    V = w.V if V is None else V
+    out = {
+        "C": codebooks(w.M, w.L, w.K, w.ds, w.sigmas, seed),
+        "codes": codes(V, w.M, w.L, w.K, seed + 1),
+    }
+    if w.B > 0:
+        out["h"] = hidden(w.B, w.D, w.hidden_scale, seed + 2)
+    if w.n_ids > 0:
+        out["ids"] = zipf_ids(w.n_ids, V, w.zipf_s, seed + 3)
+    return out

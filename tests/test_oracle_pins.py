@@ -1,0 +1,325 @@
+"""Pins for the CPU oracle: checks against facts that do not come from the
+oracle itself.
+
+* hand-derived golden values (bf16 rounding, 10-bit packing, row decode),
+* brute force on tiny inputs (pure Python, straight from the definition),
+* the pages' own check: LUT lookup+sum equals direct decode-then-matmul
+  ("Gemma-2 runtime compression: NF4 + LUT serving", correctness-check
+  table: LUT vs direct decode+matmul, both fp32, 4.8e-7 relative),
+* special cases that reduce to a library routine or a closed form,
+* digit-encoded codebooks whose exact sums reveal every index used,
+* artifact sizes the pages print (412 MB, 3.59 bits/param, 265 MB,
+  1,180 MB, the 768 MB idle-footprint drop).
+
+Each check is a plain function raising AssertionError, so the planted-
+mistake test below can run the same checks against mutated oracle builds.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from lut_logits_serving_b200 import synth
+
+
+def _read_rows(path):
+    out = []
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                out.append(line)
+    return out
+
+
+def _bits_to_f32(hexstr):
+    return np.array([int(hexstr, 16)], np.uint32).view(np.float32)[0]
+
+
+# ----------------------------------------------------------------- checks
+
+def check_bf16_golden(golden_dir):
+    for row in _read_rows(os.path.join(golden_dir, "bf16_rne.txt")):
+        f32, want = row.split()[:2]
+        got = oracle.f32_to_bf16_rne(_bits_to_f32(f32))
+        assert got == int(want, 16), (f32, hex(got), want)
+
+
+def check_pack10_golden(golden_dir):
+    for row in _read_rows(os.path.join(golden_dir, "pack10.txt")):
+        lhs, rhs = row.split("|")
+        codes = np.array([int(c, 16) for c in lhs.split(",")], np.uint16)[None, :]
+        want = np.array([int(b, 16) for b in rhs.split(",")], np.uint8)[None, :]
+        got = oracle.pack10(codes)
+        assert got.shape == want.shape and np.array_equal(got, want), (row, got)
+        back = oracle.unpack10(got, codes.shape[1])
+        assert np.array_equal(back, codes)
+
+
+def check_decode_golden(golden_dir):
+    for row in _read_rows(os.path.join(golden_dir, "decode_rows.txt")):
+        c0, c1, sc, want = row.split()[:4]
+        C = np.zeros((1, 2, 1, 1), np.float32)
+        C[0, 0, 0, 0] = _bits_to_f32(c0)
+        C[0, 1, 0, 0] = _bits_to_f32(c1)
+        codes = np.zeros((1, 1, 2), np.uint16)
+        out = oracle.decode_rows_bf16(np.array([0], np.int32), codes, C,
+                                      float(_bits_to_f32(sc)))
+        assert out.shape == (1, 1) and int(out[0, 0]) == int(want, 16), (row, hex(out[0, 0]))
+
+
+def _brute_force(codes, C, h, cap):
+    """Pure-Python fp64: decode every row, dot with h, softcap, argmax."""
+    V, M, L = codes.shape
+    _, _, K, ds = C.shape
+    B, D = h.shape
+    z = [[0.0] * V for _ in range(B)]
+    for v in range(V):
+        row = []
+        for i in range(D):
+            m, j = divmod(i, ds)
+            row.append(sum(float(C[m, l, int(codes[v, m, l]), j]) for l in range(L)))
+        for b in range(B):
+            z[b][v] = sum(float(h[b, i]) * row[i] for i in range(D))
+    y = [[cap * math.tanh(x / cap) for x in zb] for zb in z]
+    am = [max(range(V), key=lambda v: (yb[v], -v)) for yb in y]
+    return np.array(z), np.array(y), np.array(am)
+
+
+def check_brute_force_tiny():
+    rng = np.random.default_rng(11)
+    V, M, L, K, ds, B = 9, 3, 2, 5, 2, 2
+    C = rng.standard_normal((M, L, K, ds)).astype(np.float32)
+    codes = rng.integers(0, K, (V, M, L)).astype(np.uint16)
+    h = rng.standard_normal((B, M * ds)).astype(np.float32)
+    z_bf, y_bf, a_bf = _brute_force(codes, C, h, 30.0)
+    T = oracle.lut_build(h, C, "f64")
+    z_lut = oracle.logits_lut(codes, T)
+    z_dir = oracle.logits_direct(codes, C, h)
+    assert np.allclose(z_lut, z_bf, rtol=0, atol=1e-12), (z_lut, z_bf)
+    assert np.allclose(z_dir, z_bf, rtol=0, atol=1e-12)
+    y = oracle.softcap(z_lut, 30.0)
+    assert np.allclose(y, y_bf, rtol=0, atol=1e-12)
+    assert np.array_equal(oracle.argmax(y), a_bf)
+    # fp32 forms agree to fp32 rounding
+    z32 = oracle.logits_lut(codes, oracle.lut_build(h, C, "f32"))
+    assert np.allclose(z32, z_bf, rtol=0, atol=1e-5)
+    z32d = oracle.logits_direct(codes, C, h, precision="f32")
+    assert np.allclose(z32d, z_bf, rtol=0, atol=1e-5)
+
+
+def check_digit_encoded():
+    """Codebook values encode (k, m, j) for level 0 and k for level 1, all
+    small binary fractions so every sum is exact in fp32.  With a one-hot
+    hidden state at dim i = m*ds + j, z[v] = C[m,0,c0,j] + C[m,1,c1,j]
+    must decode back to exactly the codes stored for row v: a wrong
+    subspace split, a swapped level, a transposed code index or a dropped
+    level all change the digits."""
+    V, M, L, K, ds = 40, 4, 2, 8, 3
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, K, (V, M, L)).astype(np.uint16)
+    C = np.zeros((M, L, K, ds), np.float32)
+    for m in range(M):
+        for k in range(K):
+            for j in range(ds):
+                C[m, 0, k, j] = 64 * k + 4 * m + j
+                C[m, 1, k, j] = (k + 1) / 16.0
+    D = M * ds
+    for i in range(D):
+        m, j = divmod(i, ds)
+        h = np.zeros((1, D), np.float32)
+        h[0, i] = 1.0
+        for z in (oracle.logits_lut(codes, oracle.lut_build(h, C, "f64"))[0],
+                  oracle.logits_lut(codes, oracle.lut_build(h, C, "f32"))[0],
+                  oracle.logits_direct(codes, C, h)[0],
+                  oracle.logits_direct(codes, C, h, precision="f32")[0]):
+            ipart = np.floor(z)
+            frac = z - ipart
+            k0 = (ipart // 64).astype(int)
+            mm = ((ipart % 64) // 4).astype(int)
+            jj = (ipart % 4).astype(int)
+            k1 = np.rint(frac * 16).astype(int) - 1
+            assert np.all(mm == m) and np.all(jj == j), (i, mm, jj)
+            assert np.array_equal(k0, codes[:, m, 0].astype(int)), i
+            assert np.array_equal(k1, codes[:, m, 1].astype(int)), i
+        # the decoded input row holds the same digits (scale 1, exact in bf16
+        # only for small values, so compare the fp32 value via the row sum)
+    ids = np.arange(V, dtype=np.int32)
+    rows = oracle.decode_rows_bf16(ids, codes, C, 1.0)
+    f = (rows.astype(np.uint32) << 16).view(np.float32)
+    for v in range(V):
+        for m in range(M):
+            for j in range(ds):
+                exact = 64 * int(codes[v, m, 0]) + 4 * m + j + (int(codes[v, m, 1]) + 1) / 16.0
+                want = oracle.f32_to_bf16_rne(np.float32(exact))
+                assert rows[v, m * ds + j] == want
+                assert abs(f[v, m * ds + j] - exact) <= abs(exact) * 2.0 ** -8
+
+
+def check_special_cases():
+    rng = np.random.default_rng(7)
+    # M = 1, L = 1, codes = 0..K-1: logits are the codebook matvec C h
+    K, D = 37, 6
+    C = rng.standard_normal((1, 1, K, D)).astype(np.float32)
+    h = rng.standard_normal((2, D)).astype(np.float32)
+    codes = np.arange(K, dtype=np.uint16).reshape(K, 1, 1)
+    z = oracle.logits_lut(codes, oracle.lut_build(h, C, "f64"))
+    ref = (C[0, 0].astype(np.float64) @ h.astype(np.float64).T).T
+    assert np.allclose(z, ref, rtol=1e-13, atol=1e-13)
+    # a zero residual level reduces RQ to plain PQ (the L = 1 result)
+    M, K, ds, V = 4, 16, 3, 50
+    C2 = rng.standard_normal((M, 2, K, ds)).astype(np.float32)
+    C2[:, 1] = 0.0
+    codes2 = rng.integers(0, K, (V, M, 2)).astype(np.uint16)
+    h2 = rng.standard_normal((1, M * ds)).astype(np.float32)
+    z2 = oracle.logits_lut(codes2, oracle.lut_build(h2, C2, "f64"))
+    z1 = oracle.logits_lut(np.ascontiguousarray(codes2[:, :, :1]),
+                           oracle.lut_build(h2, np.ascontiguousarray(C2[:, :1]), "f64"))
+    assert np.array_equal(z2, z1)
+    # K = 1: every row is the same vector, every logit equal, argmax 0
+    C3 = rng.standard_normal((M, 2, 1, ds)).astype(np.float32)
+    codes3 = np.zeros((V, M, 2), np.uint16)
+    y3 = oracle.softcap(oracle.logits_lut(codes3, oracle.lut_build(h2, C3, "f64")), 30.0)
+    assert np.all(y3 == y3[0, 0])
+    assert oracle.argmax(y3)[0] == 0
+    assert oracle.argmax(y3.astype(np.float32))[0] == 0
+
+
+def check_softcap():
+    cap = 30.0
+    z = np.array([[0.0, 1e-3, -1e-3, 30.0 * math.atanh(0.5), -30.0 * math.atanh(0.5),
+                   1e6, -1e6, 2.0]])
+    y = oracle.softcap(z, cap)[0]
+    assert y[0] == 0.0
+    assert y[1] == -y[2]
+    assert abs(y[3] - 15.0) < 1e-12 and abs(y[4] + 15.0) < 1e-12
+    assert y[5] == 30.0 and y[6] == -30.0           # saturates, never exceeds
+    assert abs(y[7] - (2.0 - 8.0 / (3 * cap * cap))) < 1e-5   # tanh series
+    assert np.array_equal(oracle.softcap(z, 0.0), z)   # cap <= 0: off
+    assert np.array_equal(oracle.softcap(z, -1.0), z)
+
+
+def check_argmax():
+    rng = np.random.default_rng(3)
+    y = rng.standard_normal((4, 1000)).astype(np.float32)
+    assert np.array_equal(oracle.argmax(y), np.argmax(y, axis=1))
+    y[1, 10] = y[1, 500] = y[1].max() + 1           # tie: lowest index
+    assert oracle.argmax(y)[1] == 10
+    y64 = rng.standard_normal((2, 777))
+    assert np.array_equal(oracle.argmax(y64), np.argmax(y64, axis=1))
+
+
+def check_pages_fp32_identity(nrows=400):
+    """The pages' own gate at the Gemma-2 shape: LUT lookup+sum vs direct
+    decode+matmul, both fp32 (they report 4.8e-7 relative).  In fp64 the two
+    are the same number up to rounding (1e-12)."""
+    w = synth.WORKLOADS["g2_b1"]
+    C = synth.codebooks(w.M, w.L, w.K, w.ds, w.sigmas, 0)
+    codes = synth.codes(nrows, w.M, w.L, w.K, 1)
+    h = synth.hidden(1, w.D, w.hidden_scale, 2)
+    z_lut = oracle.logits_lut(codes, oracle.lut_build(h, C, "f32"))
+    z_dir = oracle.logits_direct(codes, C, h, precision="f32")
+    rel = np.linalg.norm(z_lut.astype(np.float64) - z_dir) / np.linalg.norm(z_dir.astype(np.float64))
+    assert 1e-9 < rel < 4.8e-6, rel          # same order as the pages' 4.8e-7
+    z64 = oracle.logits_lut(codes, oracle.lut_build(h, C, "f64"))
+    d64 = oracle.logits_direct(codes, C, h)
+    assert np.max(np.abs(z64 - d64)) <= 1e-12 * np.max(np.abs(d64))
+    return rel
+
+
+def check_sizes():
+    """Artifact sizes printed on the pages pin the layout we read:
+    u16 codes [V][M][L] + fp32 codebooks [M][L][K][ds]."""
+    V, D, M, L, K = 256000, 2304, 384, 2, 1024
+    ds = D // M
+    code_bytes = V * M * L * 2
+    cb_bytes = M * L * K * ds * 4
+    assert round((code_bytes + cb_bytes) / 1e6) == 412          # "412 MB"
+    assert round(V * D * 2 / 1e6) == 1180                           # "1,180 MB"
+    rb = oracle.packed10_row_bytes(M * L)
+    assert rb == 960
+    bpp = (V * rb * 8 + cb_bytes * 8) / (V * D)
+    assert round(bpp, 2) == 3.59                                    # "3.59 bits/param"
+    assert round((V * rb + cb_bytes) / 1e6) == 265                  # "265 MB"
+    # idle footprint drop 6,408 - 5,640 = 768 MB = bf16 matrix - RQ artifact
+    assert abs((V * D * 2 - code_bytes - cb_bytes) / 1e6 - 768) < 1.0
+
+
+# ------------------------------------------------------------------ tests
+
+def test_bf16_golden(golden_dir):
+    check_bf16_golden(golden_dir)
+
+
+def test_bf16_nan_is_quiet():
+    nan = np.array([0x7F800001], np.uint32).view(np.float32)[0]
+    out = oracle.f32_to_bf16_rne(nan)
+    assert (out & 0x7F80) == 0x7F80 and (out & 0x7F) != 0
+
+
+def test_pack10_golden(golden_dir):
+    check_pack10_golden(golden_dir)
+
+
+def test_pack10_roundtrip():
+    rng = np.random.default_rng(1)
+    for P in (1, 3, 64, 768, 13):
+        codes = rng.integers(0, 1024, (17, P)).astype(np.uint16)
+        packed = oracle.pack10(codes)
+        assert packed.shape == (17, (10 * P + 7) // 8)
+        assert np.array_equal(oracle.unpack10(packed, P), codes)
+
+
+def test_decode_golden(golden_dir):
+    check_decode_golden(golden_dir)
+
+
+def test_brute_force_tiny():
+    check_brute_force_tiny()
+
+
+def test_digit_encoded():
+    check_digit_encoded()
+
+
+def test_special_cases():
+    check_special_cases()
+
+
+def test_softcap():
+    check_softcap()
+
+
+def test_argmax():
+    check_argmax()
+
+
+def test_pages_fp32_identity():
+    rel = check_pages_fp32_identity()
+    print(f"LUT vs direct, both fp32, relative L2 diff = {rel:.3g} (pages: 4.8e-7)")
+
+
+def test_tiny_workload_lut_vs_direct():
+    w = synth.WORKLOADS["tiny"]
+    d = synth.make(w)
+    T = oracle.lut_build(d["h"], d["C"], "f64")
+    z = oracle.logits_lut(d["codes"], T)
+    zd = oracle.logits_direct(d["codes"], d["C"], d["h"])
+    assert np.max(np.abs(z - zd)) <= 1e-12 * np.max(np.abs(zd))
+    # every code value of every (m, l) table is used by some row
+    for m in range(w.M):
+        for l in range(w.L):
+            assert np.unique(d["codes"][:, m, l]).size == w.K
+
+
+def test_sizes():
+    check_sizes()
+
+
+def test_zipf_ids_shape_and_repeats():
+    ids = synth.zipf_ids(512, 256000, 1.1, 3)
+    assert ids.dtype == np.int32 and ids.shape == (512,)
+    assert ids.min() >= 0 and ids.max() < 256000
+    assert np.unique(ids).size < 512        # heavy head: repeats occur
