@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the RQ-LUT logits serving step on B200.
+
+One step = the whole hot path for one batch of B tokens on the Gemma-2
+shaped artifact (V=256000, D=2304, M=384, L=2, K=1024, uint16 codes):
+rebuild the B input rows (bf16), build the per-token lookup tables, stream
+the code matrix once with lookup + sum, Gemma-2 softcap, write the fp32
+logits and the argmax.  Default workload: decode batch 1.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  `value` = vocabulary rows scored per second
+over all ranks (V * B * steps / max-over-ranks device time); the code matrix
+(393 MB) is larger than L2, so every step streams it from HBM.
+Multi-GPU: independent replicas, one per rank (no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from lut_logits_serving_b200 import synth  # noqa: E402
+
+METRIC = "LUT logits vocab-rows/s & µs/call at V=256000 (1 B200), % of HBM roofline"
+UNIT = "vocab-rows/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="g2_b1", choices=["g2_b1", "g2_b32", "packed_b64"])
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def workload_config(w):
+    fmt = "packed10 (960 B/row)" if w.packed10 else "uint16 (1536 B/row)"
+    return {
+        "workload": f"{w.name}: V={w.V} D={w.D} M={w.M} L={w.L} K={w.K} B={w.B}, {fmt} codes, "
+                    f"softcap {w.softcap:g}, logits + argmax, {w.B} input rows rebuilt (bf16)",
+        "V": w.V, "D": w.D, "M": w.M, "L": w.L, "K": w.K, "B": w.B,
+        "codes": "packed10" if w.packed10 else "u16",
+        "l2": "inputs larger than L2: the 393 MB / 246 MB code matrix is streamed every step",
+    }
+
+
+def code_bytes(w):
+    return w.V * (w.P * 10 // 8 if w.packed10 else w.P * 2)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (median SM clock, reasons)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_step_fn(w, data):
+    """One pass of the whole path in the CPU oracle (fp64 tables and sums,
+    softcap, argmax, input-row decode), optionally on a subset of rows."""
+    import oracle
+
+    def step(rows=None):
+        T = oracle.lut_build(data["h"], data["C"], "f64")
+        z = oracle.logits_lut(data["codes"], T, rows)
+        y = oracle.softcap(z, w.softcap)
+        am = oracle.argmax(y.astype(np.float32))
+        oracle.decode_rows_bf16(data["ids"], data["codes"], data["C"], w.decode_scale)
+        return am
+    return step
+
+
+def cpu_baseline(w, data, seconds):
+    """Time the oracle as it stands on full-vocabulary steps until `seconds`."""
+    step = oracle_step_fn(w, data)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        step()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": w.V * w.B * n / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} full steps of {w.name} (all {w.V} rows x {w.B} tokens, fp64 tables, "
+                      f"softcap, argmax, row decode), single-threaded C, {el:.1f} s"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    data = synth.make(w)
+    step = oracle_step_fn(w, data)
+    # size each step's row sample so that warmup + steps end within ~2 minutes
+    probe = np.arange(min(w.V, 20000), dtype=np.int64)
+    t0 = time.perf_counter()
+    step(probe)
+    per_row = (time.perf_counter() - t0) / probe.size
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    nrows = int(max(1000, min(w.V, budget / max(per_row, 1e-9))))
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(w.V, nrows, replace=False)).astype(np.int64)
+    for _ in range(args.warmup):
+        step(rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(rows)
+    el = time.perf_counter() - t0
+    value = nrows * w.B * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{nrows} of {w.V} rows per step, {w.B} token(s)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------- our arm
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("logits_chunk.cu", "rq_common.cuh"):
+        with open(os.path.join(ROOT, "lut_logits_serving_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(kernel)
+    if not e or e.get("source_sha") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import lut_logits_serving_b200 as rq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    data = synth.make(w, seed=1000 * rank)
+    d = rq.dims(w.V, w.D, w.M, w.L, w.K)
+    fmt = rq.PACKED10 if w.packed10 else rq.U16
+    dC = torch.from_numpy(data["C"]).cuda()
+    c16 = torch.from_numpy(data["codes"].reshape(w.V, -1)).cuda()
+    dcodes = rq.rq_pack10(c16, d) if w.packed10 else c16
+    if w.packed10:
+        del c16
+    dh = torch.from_numpy(data["h"]).cuda()
+    dids = torch.from_numpy(data["ids"]).cuda()
+    logits = torch.empty((w.B, w.V), dtype=torch.float32, device="cuda")
+    am = torch.empty((w.B,), dtype=torch.int32, device="cuda")
+    rows = torch.empty((w.B, w.D), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
+                     device="cuda")
+
+    def step():
+        rq.rq_decode_rows(dids, dcodes, fmt, dC, d, w.decode_scale, out=rows)
+        rq.rq_logits_from_hidden(dh, dC, dcodes, fmt, d, w.softcap, logits=logits, argmax=am,
+                                 ws=ws)
+
+    # decode + (build, tiled pass, reduce) or (build + pass per token group) + argmax finalize
+    if w.B <= 4:
+        launches_per_step = 1 + 1 + 1 + 1 + 1
+    else:
+        launches_per_step = 1 + 2 * ((w.B + 31) // 32) + 1
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    graph = None
+    if not args.no_graph:
+        s2 = torch.cuda.Stream()
+        s2.wait_stream(stream)
+        with torch.cuda.stream(s2):
+            step()
+        stream.wait_stream(s2)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+    run = graph.replay if graph is not None else step
+
+    # ---- timed region: K steps, device time, max over ranks
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            run()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    t_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([t_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_ms = float(t.item())
+    sec = t_ms / 1e3
+    value = world * w.V * w.B * args.steps / sec
+
+    # ---- the dominant kernel alone (code-streaming pass), live CUDA events
+    nprof = min(args.steps, 2000)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(nprof)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(nprof)]
+    torch.cuda.synchronize()
+    for i in range(nprof):
+        rq.rq_set_profile_events(starts[i], stops[i])
+        step()
+    rq.rq_set_profile_events(None, None)
+    torch.cuda.synchronize()
+    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(starts, stops)]))
+    peak, peak_kind = load_peaks()
+    algo_bytes = code_bytes(w)
+    achieved = algo_bytes / (kern_ms / 1e3) / 1e9
+    kname = "logits_chunk_u16_kernel" if (w.B <= 4 and not w.packed10) else "logits_l2_kernel"
+
+    # ---- end to end through the public API with host buffers
+    h_host = torch.from_numpy(data["h"]).pin_memory()
+    ids_host = torch.from_numpy(data["ids"]).pin_memory()
+    out_host = torch.empty((w.B, w.V), dtype=torch.float32).pin_memory()
+    am_host = torch.empty((w.B,), dtype=torch.int32).pin_memory()
+    ne2e = min(args.steps, 2000)
+
+    def e2e_step():
+        dh.copy_(h_host, non_blocking=True)
+        dids.copy_(ids_host, non_blocking=True)
+        step()
+        out_host.copy_(logits, non_blocking=True)
+        am_host.copy_(am, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ne2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e_value = world * w.V * w.B * ne2e / (e_ms / 1e3)
+    h2d = data["h"].nbytes + data["ids"].nbytes
+    d2h = w.B * w.V * 4 + w.B * 4
+
+    # the argmax must agree with the logits it came from
+    assert torch.equal(am.long().cpu(), logits.argmax(dim=1).cpu()), "argmax/logits mismatch"
+    assert rq.rq_device_error() == 0
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, data, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        del graph
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+        "us_per_call": t_ms / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(w), parallelism=f"replicas x{world}",
+                       launch="cuda graph" if graph is not None else "eager"),
+        "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": profiled_traffic(kname), "algorithmic_bytes": algo_bytes,
+                     "kernel_us": kern_ms * 1e3},
+        "step_hbm_frac": code_bytes(w) / (sec / args.steps) / 1e9 / peak,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ne2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,214 @@
+/*
+ * rqlut.h -- C ABI of librqlut: LUT-based serving of a residual-product-
+ * quantized (RQ) tied embedding on one NVIDIA B200 (sm_100a).
+ *
+ * The method ("Gemma-2 runtime compression: NF4 + LUT serving" page, section
+ * on LUT-based serving; "Gemma-2-2B combined RQ+NF4" page, paragraph on the
+ * RQ reconstruction with M=384, K=1024, L=2):
+ *
+ *   A V x D embedding is stored as codes [V][M][L] into per-(subspace,
+ *   level) codebooks C[M][L][K][ds], ds = D/M, subspace m = dims
+ *   [m*ds, (m+1)*ds):  E[v, m*ds+j] = sum_l C[m][l][code[v][m][l]][j].
+ *   Output logits are computed without forming E: per token b a lookup
+ *   table T[b][m][l][k] = <h_b[m*ds : m*ds+ds], C[m][l][k]> is built, then
+ *   z[b][v] = sum_m sum_l T[b][m][l][code[v][m][l]]  (lookup + sum), and
+ *   Gemma-2's final softcap y = cap * tanh(z / cap) follows.  Input rows are
+ *   rebuilt on demand for the few ids of a step.
+ *
+ * Conventions shared by every call
+ *   - Pointers named device_* / "(device)" are CUDA device pointers; the
+ *     caller owns every buffer.  The library never allocates device memory.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Every call only enqueues work and never synchronizes.
+ *   - Return value: rq_status (0 = RQ_OK).  Argument errors are detected on
+ *     the host before anything is launched.  RQ_ERR_CUDA reports a launch
+ *     error (cudaGetLastError); kernel faults surface at the caller's next
+ *     synchronization, as usual for CUDA.
+ *   - Codes >= K are never read out of bounds: with K a power of two a code
+ *     is taken modulo K, otherwise it is clamped to K-1.  Ids outside
+ *     [0, V) in rq_decode_rows give zero rows and set RQ_DEVERR_BAD_ID in
+ *     the device error word (rq_device_error).
+ *   - Any wait inside a kernel is bounded (about one second); on expiry
+ *     the kernel sets RQ_DEVERR_TIMEOUT and returns.
+ *
+ * Layouts (row-major, little-endian)
+ *   h        float [B][D]
+ *   C        float [M][L][K][ds]
+ *   codes    RQ_CODES_U16:      uint16 [V][M*L], code of pair (m,l) at
+ *                               column p = m*L + l
+ *            RQ_CODES_PACKED10: uint8 [V][rb], rb = ceil(10*M*L/8); code
+ *                               p occupies bits [10p, 10p+10) of the row,
+ *                               bit i being bit (i%8) of byte i/8
+ *   lut      float [M*L][K][Bs], Bs = rq_lut_token_stride(B): token b of
+ *            table (p, k) at lut[(p*K + k)*Bs + b]
+ *   logits   float [B][V]
+ *   argmax   int32 [B]: lowest index of the largest softcapped logit
+ *   rows     uint16 bf16 bit patterns [N][D]
+ */
+#ifndef RQLUT_H
+#define RQLUT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RQ_API __attribute__((visibility("default")))
+#else
+#define RQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+    int64_t V;   /* vocabulary rows                                  */
+    int32_t D;   /* model dim; must be a multiple of M               */
+    int32_t M;   /* subspaces                                        */
+    int32_t L;   /* residual levels                                  */
+    int32_t K;   /* codewords per (subspace, level) codebook         */
+} rq_dims;
+
+enum rq_code_fmt {
+    RQ_CODES_U16 = 0,       /* one uint16 per code (K <= 65536)           */
+    RQ_CODES_PACKED10 = 1   /* 10-bit codes, bit stream per row (K<=1024) */
+};
+
+enum rq_status {
+    RQ_OK = 0,
+    RQ_ERR_INVALID_ARGUMENT = 1,   /* null pointer, bad shape or value      */
+    RQ_ERR_UNSUPPORTED = 2,        /* valid but not handled by this build   */
+    RQ_ERR_WORKSPACE_TOO_SMALL = 3,
+    RQ_ERR_CUDA = 4,               /* a CUDA runtime call failed            */
+    RQ_ERR_MISALIGNED = 5          /* a pointer breaks the stated alignment */
+};
+
+/* Bits of the device error word. */
+#define RQ_DEVERR_TIMEOUT 0x1u  /* a bounded wait inside a kernel expired */
+#define RQ_DEVERR_BAD_ID  0x2u  /* rq_decode_rows saw an id outside [0,V) */
+
+/* Human-readable name of a status code (static string, never NULL). */
+RQ_API const char *rq_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+RQ_API int rq_version(void);
+
+/* Bytes of the code matrix in format `fmt` (0 on invalid arguments). */
+RQ_API size_t rq_codes_bytes(rq_dims d, int fmt);
+
+/* Token stride Bs of the LUT layout: B for B <= 2, else B rounded up to a
+ * multiple of 4 (so a token group is a whole number of 16-byte vectors). */
+RQ_API int rq_lut_token_stride(int B);
+
+/* Bytes of the lookup table for B tokens: M*L*K*Bs*4 (0 on bad args). */
+RQ_API size_t rq_lut_bytes(rq_dims d, int B);
+
+/* Device workspace that rq_lut_logits needs for these arguments: partial
+ * sums of the vocabulary-tiled pass plus argmax partials.  0 is possible.
+ * `want_argmax` is 0 or 1. */
+RQ_API size_t rq_logits_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax);
+
+/* Device workspace of rq_logits_from_hidden (includes the lookup table of
+ * one token group). */
+RQ_API size_t rq_fused_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax);
+
+/*
+ * rq_lut_build -- per-token lookup tables (LUT serving section: the tables
+ * that replace the output matmul).
+ *   lut[(p*K + k)*Bs + b] = sum_{j<ds} h[b][m*ds + j] * C[m][l][k][j],
+ *   p = m*L + l, in fp32 (fused multiply-adds, j ascending).
+ *   h   (device) float [B][D], 4-byte aligned
+ *   C   (device) float [M][L][K][ds], 4-byte aligned
+ *   lut (device) float, rq_lut_bytes(d, B) bytes, 16-byte aligned; padding
+ *       tokens b in [B, Bs) are written as 0.
+ * Errors: RQ_ERR_INVALID_ARGUMENT (null, B < 1, bad dims),
+ *         RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ */
+RQ_API int rq_lut_build(const float *h, const float *C, rq_dims d, int B, float *lut,
+                 void *stream);
+
+/*
+ * rq_lut_logits -- logits by lookup and sum over each vocabulary row's codes,
+ * never forming the V x D matrix (LUT serving section and its correctness
+ * table: LUT vs direct decode+matmul), then Gemma-2's final softcap and an
+ * optional greedy argmax.
+ *   z[b][v] = sum_p lut[(p*K + code[v][p])*Bs + b]    (fp32 sums)
+ *   y = softcap > 0 ? softcap * tanhf(z / softcap) : z
+ *   codes  (device) code matrix in format `fmt`, 16-byte aligned
+ *   lut    (device) as written by rq_lut_build for the same B, 16-byte
+ *          aligned
+ *   logits (device) float [B][V] or NULL (then only argmax is produced)
+ *   argmax (device) int32 [B] or NULL; at least one of logits/argmax set
+ *   ws     (device) workspace of >= rq_logits_workspace_bytes(d, B, fmt,
+ *          argmax != NULL) bytes, 16-byte aligned (may be NULL if that is 0)
+ * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_MISALIGNED,
+ *         RQ_ERR_WORKSPACE_TOO_SMALL, RQ_ERR_UNSUPPORTED (PACKED10 with
+ *         K > 1024), RQ_ERR_CUDA.
+ */
+RQ_API int rq_lut_logits(const void *codes, int fmt, rq_dims d, const float *lut,
+                  int B, float softcap, float *logits, int32_t *argmax,
+                  void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * rq_logits_from_hidden -- rq_lut_build + rq_lut_logits in one call; large
+ * batches are processed in token groups so each group's table stays in L2.
+ * Same arguments and errors as the two calls; the table lives in `ws`
+ * (>= rq_fused_workspace_bytes(d, B, fmt, argmax != NULL) bytes).
+ */
+RQ_API int rq_logits_from_hidden(const float *h, const float *C, const void *codes,
+                          int fmt, rq_dims d, int B, float softcap,
+                          float *logits, int32_t *argmax, void *ws,
+                          size_t ws_bytes, void *stream);
+
+/*
+ * rq_decode_rows -- rebuild input-embedding rows on demand (LUT serving
+ * section: input token rows are reconstructed for the ids of a prompt, not
+ * for the whole vocabulary).
+ *   out[n][m*ds + j] = bf16_rne( fp32( fp32(sum_l C[m][l][c_l][j]) * scale ) ),
+ *   c_l = code[ids[n]][m*L + l]; the level sum runs l = 0..L-1 in fp32.
+ *   Gemma-2 uses scale = sqrt(D).
+ *   ids    (device) int32 [N]; ids outside [0, V) give zero rows and set
+ *          RQ_DEVERR_BAD_ID
+ *   codes  (device) as for rq_lut_logits; C (device) float [M][L][K][ds]
+ *   out    (device) uint16 [N][D] bf16 bit patterns, 4-byte aligned
+ *   N = 0 is a no-op.
+ * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ */
+RQ_API int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt,
+                   const float *C, rq_dims d, float scale, uint16_t *out,
+                   void *stream);
+
+/*
+ * rq_pack10 -- convert uint16 codes [V][M*L] (values < 1024) into the
+ * PACKED10 layout above (the 10-bit storage implied by the 3.59 bits/param
+ * figure of the combined RQ+NF4 page).  Codes >= 1024 keep their low 10
+ * bits.  packed (device) uint8 [V][rb], rb = ceil(10*M*L/8).
+ * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_CUDA.
+ */
+RQ_API int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed,
+              void *stream);
+
+/*
+ * rq_device_error -- read (and, if `clear`, reset) the device error word
+ * of the current device.  Synchronous: call after synchronizing the streams
+ * that ran the kernels of interest.  *out receives RQ_DEVERR_* bits.
+ */
+RQ_API int rq_device_error(uint32_t *out, int clear);
+
+/*
+ * rq_set_profile_events -- optional timing hook for benchmarks.  With both
+ * arguments non-NULL (cudaEvent_t handles passed as void*), each later
+ * rq_lut_logits / rq_logits_from_hidden call made from this host thread
+ * records `start` on its stream just before its first code-streaming kernel
+ * and `stop` just after its last one, so cudaEventElapsedTime(start, stop)
+ * is the device time of that pass alone (for token-grouped batches it spans
+ * the groups and the table builds between them).  NULL, NULL turns it off.
+ * The setting is thread-local; the events stay owned by the caller.
+ * Errors: RQ_ERR_INVALID_ARGUMENT if exactly one argument is NULL.
+ */
+RQ_API int rq_set_profile_events(void *start, void *stop);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RQLUT_H */

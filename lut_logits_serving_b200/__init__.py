@@ -1,0 +1,268 @@
+"""librqlut Python binding: LUT-based serving of a residual-product-quantized
+(RQ) tied embedding on one B200.
+
+Thin ctypes marshalling over the C ABI declared in ``include/rqlut.h``; every
+step of the computation runs in the library's sm_100a CUDA kernels.  PyTorch
+only provides device memory and the current stream.  The functions keep the C
+names:
+
+* ``rq_lut_build``  -- per-token tables T[p][k][b] = <h_b[m], C[m][l][k]>
+* ``rq_lut_logits`` -- z[b][v] = sum_p T[p][code[v][p]][b], softcap, argmax
+* ``rq_logits_from_hidden`` -- both, large batches in L2-sized token groups
+* ``rq_decode_rows`` -- bf16 input rows rebuilt on demand
+* ``rq_pack10`` -- uint16 codes -> 10-bit packed rows
+
+(method: "Gemma-2 runtime compression: NF4 + LUT serving", LUT section.)
+There is no CPU fallback: if the library or a GPU is missing, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "RqDims", "RqError", "U16", "PACKED10", "lib", "dims",
+    "rq_status_string", "rq_version", "rq_codes_bytes", "rq_lut_token_stride",
+    "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
+    "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
+    "rq_pack10", "rq_device_error", "rq_set_profile_events",
+]
+
+U16 = 0
+PACKED10 = 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librqlut.so")
+
+
+class RqDims(ctypes.Structure):
+    _fields_ = [("V", ctypes.c_int64), ("D", ctypes.c_int32), ("M", ctypes.c_int32),
+                ("L", ctypes.c_int32), ("K", ctypes.c_int32)]
+
+    def __repr__(self):
+        return f"RqDims(V={self.V}, D={self.D}, M={self.M}, L={self.L}, K={self.K})"
+
+
+def dims(V, D, M, L, K) -> RqDims:
+    return RqDims(int(V), int(D), int(M), int(L), int(K))
+
+
+class RqError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {rq_status_string(status)} ({status})")
+
+
+_lib = None
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+_f = ctypes.c_float
+
+_SIGNATURES = {
+    "rq_status_string": (ctypes.c_char_p, [_i]),
+    "rq_version": (_i, []),
+    "rq_codes_bytes": (_sz, [RqDims, _i]),
+    "rq_lut_token_stride": (_i, [_i]),
+    "rq_lut_bytes": (_sz, [RqDims, _i]),
+    "rq_logits_workspace_bytes": (_sz, [RqDims, _i, _i, _i]),
+    "rq_fused_workspace_bytes": (_sz, [RqDims, _i, _i, _i]),
+    "rq_lut_build": (_i, [_p, _p, RqDims, _i, _p, _p]),
+    "rq_lut_logits": (_i, [_p, _i, RqDims, _p, _i, _f, _p, _p, _p, _sz, _p]),
+    "rq_logits_from_hidden": (_i, [_p, _p, _p, _i, RqDims, _i, _f, _p, _p, _p, _sz, _p]),
+    "rq_decode_rows": (_i, [_p, _i64, _p, _i, _p, RqDims, _f, _p, _p]),
+    "rq_pack10": (_i, [_p, RqDims, _p, _p]),
+    "rq_device_error": (_i, [ctypes.POINTER(ctypes.c_uint32), _i]),
+    "rq_set_profile_events": (_i, [_p, _p]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load librqlut.so (built in-tree by ``lut_logits_serving_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"librqlut.so not found at {LIB_PATH}; build it with "
+                "`python -m lut_logits_serving_b200.build` (there is no CPU fallback)")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(l, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = l
+    return _lib
+
+
+# ------------------------------------------------------------ host queries
+
+def rq_status_string(status: int) -> str:
+    return lib().rq_status_string(int(status)).decode()
+
+
+def rq_version() -> int:
+    return lib().rq_version()
+
+
+def rq_codes_bytes(d: RqDims, fmt: int) -> int:
+    return lib().rq_codes_bytes(d, fmt)
+
+
+def rq_lut_token_stride(B: int) -> int:
+    return lib().rq_lut_token_stride(B)
+
+
+def rq_lut_bytes(d: RqDims, B: int) -> int:
+    return lib().rq_lut_bytes(d, B)
+
+
+def rq_logits_workspace_bytes(d: RqDims, B: int, fmt: int, want_argmax: bool) -> int:
+    return lib().rq_logits_workspace_bytes(d, B, fmt, int(bool(want_argmax)))
+
+
+def rq_fused_workspace_bytes(d: RqDims, B: int, fmt: int, want_argmax: bool) -> int:
+    return lib().rq_fused_workspace_bytes(d, B, fmt, int(bool(want_argmax)))
+
+
+# ------------------------------------------------------------ device calls
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda(t, dtype, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor (no CPU fallback)")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ptr_or_null(t, dtype, name):
+    return ctypes.c_void_p(None) if t is None else _cuda(t, dtype, name)
+
+
+def _check(fn, status):
+    if status != 0:
+        raise RqError(fn, status)
+
+
+def _codes_dtype(fmt):
+    torch = _torch()
+    return torch.uint16 if fmt == U16 else torch.uint8
+
+
+def _empty(shape, dtype, like):
+    torch = _torch()
+    return torch.empty(shape, dtype=dtype, device=like.device)
+
+
+def _workspace(nbytes, like, ws):
+    torch = _torch()
+    if nbytes == 0:
+        return ctypes.c_void_p(None), 0, ws
+    if ws is None or ws.numel() * ws.element_size() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=like.device)
+    return _cuda(ws, None, "ws"), ws.numel() * ws.element_size(), ws
+
+
+def rq_lut_build(h, C, d: RqDims, lut=None, stream=None):
+    """h float32 [B, D], C float32 [M, L, K, ds] -> lut float32 [P, K, Bs]."""
+    torch = _torch()
+    B = h.shape[0] if h.dim() == 2 else 1
+    Bs = rq_lut_token_stride(B)
+    if lut is None:
+        lut = _empty((d.M * d.L, d.K, Bs), torch.float32, h)
+    _check("rq_lut_build", lib().rq_lut_build(
+        _cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C"), d, B,
+        _cuda(lut, torch.float32, "lut"), _stream(stream)))
+    return lut
+
+
+def rq_lut_logits(codes, fmt: int, d: RqDims, lut, B: int, softcap: float = 30.0,
+                  want_logits: bool = True, want_argmax: bool = False, logits=None,
+                  argmax=None, ws=None, stream=None):
+    """Returns (logits float32 [B, V] or None, argmax int32 [B] or None, ws)."""
+    torch = _torch()
+    if want_logits and logits is None:
+        logits = _empty((B, d.V), torch.float32, lut)
+    if want_argmax and argmax is None:
+        argmax = _empty((B,), torch.int32, lut)
+    nbytes = rq_logits_workspace_bytes(d, B, fmt, argmax is not None)
+    wp, wn, ws = _workspace(nbytes, lut, ws)
+    _check("rq_lut_logits", lib().rq_lut_logits(
+        _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, _cuda(lut, torch.float32, "lut"), B,
+        float(softcap), _ptr_or_null(logits, torch.float32, "logits"),
+        _ptr_or_null(argmax, torch.int32, "argmax"), wp, wn, _stream(stream)))
+    return logits, argmax, ws
+
+
+def rq_logits_from_hidden(h, C, codes, fmt: int, d: RqDims, softcap: float = 30.0,
+                          want_logits: bool = True, want_argmax: bool = False, logits=None,
+                          argmax=None, ws=None, stream=None):
+    """Returns (logits float32 [B, V] or None, argmax int32 [B] or None, ws)."""
+    torch = _torch()
+    B = h.shape[0]
+    if want_logits and logits is None:
+        logits = _empty((B, d.V), torch.float32, h)
+    if want_argmax and argmax is None:
+        argmax = _empty((B,), torch.int32, h)
+    nbytes = rq_fused_workspace_bytes(d, B, fmt, argmax is not None)
+    wp, wn, ws = _workspace(nbytes, h, ws)
+    _check("rq_logits_from_hidden", lib().rq_logits_from_hidden(
+        _cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C"),
+        _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, B, float(softcap),
+        _ptr_or_null(logits, torch.float32, "logits"),
+        _ptr_or_null(argmax, torch.int32, "argmax"), wp, wn, _stream(stream)))
+    return logits, argmax, ws
+
+
+def rq_decode_rows(ids, codes, fmt: int, C, d: RqDims, scale: float, out=None, stream=None):
+    """ids int32 [N] -> bf16 rows [N, D] (returned as torch.bfloat16)."""
+    torch = _torch()
+    N = ids.numel()
+    if out is None:
+        out = _empty((N, d.D), torch.bfloat16, ids)
+    if out.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise ValueError("out: bf16 rows expected")
+    _check("rq_decode_rows", lib().rq_decode_rows(
+        _cuda(ids, torch.int32, "ids"), N, _cuda(codes, _codes_dtype(fmt), "codes"), fmt,
+        _cuda(C, torch.float32, "C"), d, float(scale), _cuda(out, None, "out"),
+        _stream(stream)))
+    return out
+
+
+def rq_pack10(codes_u16, d: RqDims, out=None, stream=None):
+    """uint16 [V, P] (or [V, M, L]) -> uint8 [V, ceil(10 P / 8)]."""
+    torch = _torch()
+    if out is None:
+        out = _empty((d.V, rq_codes_bytes(d, PACKED10) // d.V), torch.uint8, codes_u16)
+    _check("rq_pack10", lib().rq_pack10(_cuda(codes_u16, torch.uint16, "codes_u16"), d,
+                                        _cuda(out, torch.uint8, "packed"), _stream(stream)))
+    return out
+
+
+def rq_device_error(clear: bool = True) -> int:
+    v = ctypes.c_uint32(0)
+    _check("rq_device_error", lib().rq_device_error(ctypes.byref(v), int(bool(clear))))
+    return v.value
+
+
+def rq_set_profile_events(start=None, stop=None):
+    """start/stop: torch.cuda.Event (enable_timing=True) or None to switch off."""
+    sp = ctypes.c_void_p(start.cuda_event if start is not None else None)
+    tp = ctypes.c_void_p(stop.cuda_event if stop is not None else None)
+    _check("rq_set_profile_events", lib().rq_set_profile_events(sp, tp))

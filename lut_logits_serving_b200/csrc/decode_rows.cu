@@ -1,0 +1,93 @@
+// decode_rows.cu -- on-demand rebuild of input-embedding rows, and the
+// 10-bit code packer.
+//
+// "Gemma-2 runtime compression: NF4 + LUT serving", LUT section: input token
+// rows are reconstructed on demand (the ids of a prompt, not the whole
+// vocabulary).  Row element i = m*ds + j of id v:
+//   out = bf16_rne( fp32( fp32(sum_l C[m][l][code[v][m*L+l]][j]) * scale ) )
+// with the level sum in l order and explicit round-to-nearest fp32 ops, so
+// the bf16 result is reproducible bit for bit.
+//
+// Packing: the "Gemma-2-2B combined RQ+NF4" page stores the M=384, K=1024,
+// L=2 artifact at 3.59 bits/param, i.e. 10-bit codes; code p of a row sits
+// at bits [10p, 10p+10) of the row's little-endian bit string.
+#include <cuda_bf16.h>
+
+#include "rq_common.cuh"
+
+namespace rq {
+
+__global__ void __launch_bounds__(128) decode_rows_kernel(
+    const int32_t *__restrict__ ids, const void *__restrict__ codes, int fmt,
+    const float *__restrict__ C, int64_t V, int D, int M, int L, int K, float scale,
+    CodeFix fix, uint16_t *__restrict__ out, unsigned *err) {
+  const int64_t n = blockIdx.x;
+  const int ds = D / M;
+  const int P = M * L;
+  const int32_t id = ids[n];
+  uint16_t *orow = out + n * (int64_t)D;
+  if (id < 0 || (int64_t)id >= V) {
+    for (int i = threadIdx.x; i < D; i += blockDim.x) orow[i] = 0;
+    if (threadIdx.x == 0) atomicOr(err, RQ_DEVERR_BAD_ID);
+    return;
+  }
+  const int64_t rb = (10LL * P + 7) / 8;
+  const uint16_t *crow16 = (const uint16_t *)codes + (int64_t)id * P;
+  const uint8_t *crow10 = (const uint8_t *)codes + (int64_t)id * rb;
+  for (int m = threadIdx.x; m < M; m += blockDim.x) {
+    for (int j = 0; j < ds; ++j) {
+      float e = 0.f;
+      for (int l = 0; l < L; ++l) {
+        const int p = m * L + l;
+        uint32_t c = fmt == RQ_CODES_U16 ? (uint32_t)crow16[p] : packed10_code(crow10, p);
+        c = fix(c);
+        e = __fadd_rn(e, __ldg(C + (((size_t)p * K + c) * ds + j)));
+      }
+      const float s = __fmul_rn(e, scale);
+      orow[m * ds + j] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+    }
+  }
+}
+
+cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt,
+                               const float *C, int64_t V, int D, int M, int L, int K,
+                               float scale, uint16_t *out, unsigned *err, cudaStream_t s) {
+  if (N <= 0) return cudaSuccess;
+  if (N > 0x7fffffffLL) return cudaErrorInvalidValue;
+  decode_rows_kernel<<<(unsigned)N, 128, 0, s>>>(ids, codes, fmt, C, V, D, M, L, K, scale,
+                                                  make_codefix(K), out, err);
+  return cudaGetLastError();
+}
+
+// One thread per group of 4 codes = 5 output bytes.
+__global__ void pack10_kernel(const uint16_t *__restrict__ codes, int64_t V, int P,
+                              uint8_t *__restrict__ packed) {
+  const int groups = (P + 3) / 4;
+  const int64_t rb = (10LL * P + 7) / 8;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= V * groups) return;
+  const int64_t v = gid / groups;
+  const int g = (int)(gid % groups);
+  uint64_t bits = 0;
+  for (int q = 0; q < 4; ++q) {
+    const int p = 4 * g + q;
+    if (p < P) bits |= (uint64_t)(codes[v * P + p] & 0x3FFu) << (10 * q);
+  }
+  uint8_t *row = packed + v * rb;
+  for (int q = 0; q < 5; ++q) {
+    const int64_t byte = 5LL * g + q;
+    if (byte < rb) row[byte] = (uint8_t)(bits >> (8 * q));
+  }
+}
+
+cudaError_t launch_pack10(const uint16_t *codes, int64_t V, int P, uint8_t *packed,
+                          cudaStream_t s) {
+  const int64_t total = V * ((P + 3) / 4);
+  if (total == 0) return cudaSuccess;
+  const int64_t blocks = (total + 255) / 256;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  pack10_kernel<<<(unsigned)blocks, 256, 0, s>>>(codes, V, P, packed);
+  return cudaGetLastError();
+}
+
+}  // namespace rq

@@ -1,0 +1,208 @@
+// rq_common.cuh -- internal helpers shared by the librqlut kernels (sm_100a).
+// Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/rqlut.h"
+
+namespace rq {
+
+// Roughly one second at B200 clocks: every spin on an mbarrier gives up
+// after this many SM cycles, sets RQ_DEVERR_TIMEOUT and returns.
+constexpr long long kWaitLimitCycles = 2000000000LL;
+
+// Upper bound on the CTAs of any vocabulary-sweep grid.  Argmax partials are
+// sized from it so workspace sizes do not depend on the device.
+constexpr int kMaxSweepBlocks = 2048;
+
+// Tokens handled by one pass of the L2-served batched kernel.
+constexpr int kTokenGroup = 32;
+
+__host__ __device__ constexpr int64_t align_up(int64_t x, int64_t a) {
+  return (x + a - 1) / a * a;
+}
+
+// ----------------------------------------------------------------- codes
+
+// Keeps every table index in bounds whatever the code value: modulo K for a
+// power-of-two K (free: it is the extraction mask), else clamp to K-1.
+struct CodeFix {
+  uint32_t mask;   // K-1 when K is a power of two, else 0xFFFFFFFF
+  uint32_t kmax;   // K-1
+  __device__ __forceinline__ uint32_t operator()(uint32_t c) const {
+    c &= mask;
+    return c > kmax ? kmax : c;
+  }
+};
+
+inline CodeFix make_codefix(int K) {
+  CodeFix f;
+  f.kmax = (uint32_t)(K - 1);
+  f.mask = ((K & (K - 1)) == 0) ? (uint32_t)(K - 1) : 0xFFFFFFFFu;
+  return f;
+}
+
+// Code p of a 10-bit packed row: bits [10p, 10p+10), little-endian.
+__device__ __forceinline__ uint32_t packed10_code(const uint8_t *row, int p) {
+  const int bit = 10 * p;
+  const int byte = bit >> 3;
+  const uint32_t w = (uint32_t)row[byte] | ((uint32_t)row[byte + 1] << 8);
+  return (w >> (bit & 7)) & 0x3FFu;
+}
+
+// ---------------------------------------------------------- shared memory
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Spin until the phase with `parity` completes; false after the limit.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------- TMA
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 2-D tiled TMA load (no multicast) into this CTA's shared memory.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------- softcap
+
+__device__ __forceinline__ float softcap_f(float z, float cap) {
+  return cap > 0.f ? cap * tanhf(z / cap) : z;
+}
+
+// ---------------------------------------------------------------- argmax
+
+struct ArgBest {
+  float v;
+  int i;
+};
+
+// Larger value wins; equal values: lower index wins.  NaN never wins over a
+// number.  Order-independent, so any reduction tree gives the same answer.
+__device__ __forceinline__ ArgBest arg_better(ArgBest a, ArgBest b) {
+  bool a_nan = a.v != a.v, b_nan = b.v != b.v;
+  if (a_nan != b_nan) return a_nan ? b : a;
+  if (a.v > b.v) return a;
+  if (b.v > a.v) return b;
+  return a.i <= b.i ? a : b;
+}
+
+__device__ __forceinline__ ArgBest arg_shfl_xor(ArgBest a, int lane_mask) {
+  ArgBest o;
+  o.v = __shfl_xor_sync(0xffffffffu, a.v, lane_mask);
+  o.i = __shfl_xor_sync(0xffffffffu, a.i, lane_mask);
+  return o;
+}
+
+}  // namespace rq
+
+// Launchers implemented by the kernel translation units (host side).
+namespace rq {
+
+struct DevInfo {
+  int device;
+  int sms;
+  int max_smem_optin;
+  unsigned *err;   // device address of the error word
+};
+
+cudaError_t dev_info(DevInfo *out);
+
+cudaError_t launch_lut_build(const float *h, const float *C, int B, int b0, int nb, int D,
+                             int M, int L, int K, int Bs, float *lut, cudaStream_t s);
+
+cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt,
+                               const float *C, int64_t V, int D, int M, int L, int K,
+                               float scale, uint16_t *out, unsigned *err, cudaStream_t s);
+
+cudaError_t launch_pack10(const uint16_t *codes, int64_t V, int P, uint8_t *packed,
+                          cudaStream_t s);
+
+// Vocabulary-tiled pass with the LUT chunk resident in shared memory.
+struct ChunkPlan {
+  bool ok;      // this path applies
+  int TB;       // token stride of the LUT (1, 2 or 4)
+  int PC;       // pairs per chunk
+  int nch;      // chunks
+  int R;        // rows per tile
+  int variant;  // kernel instance
+  size_t smem;  // dynamic shared memory per CTA
+};
+ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di);
+size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V);
+cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
+                                int P, int K, int B, const float *lut, float *partial,
+                                const DevInfo &di, cudaStream_t s);
+cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
+                                   float *logits, float *am_val, int *am_idx, int nblk,
+                                   cudaStream_t s);
+
+// Batched pass with the LUT read through L2 (token groups of <= 32).
+cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K,
+                             const float *lut, int Bs, int lut_t0, int out_t0, int nb,
+                             float cap, float *logits, float *am_val, int *am_idx, int nblk,
+                             cudaStream_t s);
+int l2_grid_blocks(int64_t V, const DevInfo &di);
+
+cudaError_t launch_argmax_finalize(const float *am_val, const int *am_idx, int nblk, int B,
+                                   int32_t *argmax, cudaStream_t s);
+
+}  // namespace rq

@@ -1,0 +1,329 @@
+// rqlut_api.cu -- the C ABI of librqlut (see include/rqlut.h): argument
+// validation, workspace layout, path selection and launches.
+#include <mutex>
+
+#include "rq_common.cuh"
+
+// The device error word (RQ_DEVERR_* bits), one per device that loads the
+// library.  Kernels receive its device address; rq_device_error reads it.
+__device__ unsigned int g_rq_device_error = 0u;
+
+namespace rq {
+
+cudaError_t dev_info(DevInfo *out) {
+  static std::mutex mu;
+  static DevInfo cache[128];
+  static bool valid[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 128) {
+    std::lock_guard<std::mutex> g(mu);
+    if (valid[dev]) {
+      *out = cache[dev];
+      return cudaSuccess;
+    }
+  }
+  DevInfo d{};
+  d.device = dev;
+  if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  if ((e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                  dev)) != cudaSuccess)
+    return e;
+  void *p = nullptr;
+  if ((e = cudaGetSymbolAddress(&p, g_rq_device_error)) != cudaSuccess) return e;
+  d.err = static_cast<unsigned *>(p);
+  if (dev >= 0 && dev < 128) {
+    std::lock_guard<std::mutex> g(mu);
+    cache[dev] = d;
+    valid[dev] = true;
+  }
+  *out = d;
+  return cudaSuccess;
+}
+
+// Device-independent sizing: the B200 limits (148 SMs, 227 KB opt-in shared
+// memory per block) decide which kernel variant a workspace must cover.
+static DevInfo nominal_devinfo() {
+  DevInfo d{};
+  d.device = 0;
+  d.sms = 148;
+  d.max_smem_optin = 232448;
+  d.err = nullptr;
+  return d;
+}
+
+}  // namespace rq
+
+using namespace rq;
+
+namespace {
+
+constexpr int64_t kAlign = 256;
+
+// rq_set_profile_events state (per host thread).
+thread_local cudaEvent_t t_prof_start = nullptr;
+thread_local cudaEvent_t t_prof_stop = nullptr;
+
+cudaError_t prof_mark(cudaEvent_t ev, cudaStream_t s) {
+  return ev ? cudaEventRecord(ev, s) : cudaSuccess;
+}
+
+bool dims_ok(const rq_dims &d) {
+  if (d.V < 1 || d.V > (int64_t)0x7fffffff - 1024) return false;
+  if (d.D < 1 || d.M < 1 || d.L < 1 || d.K < 1) return false;
+  if (d.D % d.M != 0) return false;
+  if (d.K > 65536) return false;
+  if ((int64_t)d.M * d.L > (1 << 20)) return false;
+  return true;
+}
+
+bool fmt_ok(const rq_dims &d, int fmt) {
+  if (fmt == RQ_CODES_U16) return true;
+  if (fmt == RQ_CODES_PACKED10) return d.K <= 1024;
+  return false;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+
+// Workspace layout of rq_lut_logits:
+//   [partials: nch*B*V floats (small-batch path only)][am_val][am_idx]
+struct WsLayout {
+  bool chunk;
+  ChunkPlan cp;
+  size_t partial_off, partial_bytes;
+  size_t amv_off, ami_off, am_bytes;
+  size_t total;
+};
+
+WsLayout ws_layout(const rq_dims &d, int B, int fmt, bool want_argmax, const DevInfo &di) {
+  WsLayout w{};
+  const int P = d.M * d.L;
+  w.cp = plan_chunk(d.V, P, d.K, B, fmt, di);
+  w.chunk = w.cp.ok;
+  size_t off = 0;
+  if (w.chunk) {
+    w.partial_off = off;
+    w.partial_bytes = chunk_partial_bytes(w.cp, B, d.V);
+    off += (size_t)align_up((int64_t)w.partial_bytes, kAlign);
+  }
+  if (want_argmax) {
+    w.am_bytes = (size_t)B * kMaxSweepBlocks * 4;
+    w.amv_off = off;
+    off += (size_t)align_up((int64_t)w.am_bytes, kAlign);
+    w.ami_off = off;
+    off += (size_t)align_up((int64_t)w.am_bytes, kAlign);
+  }
+  w.total = off;
+  return w;
+}
+
+int sweep_blocks(const rq_dims &d, const DevInfo &di, bool chunk) {
+  (void)chunk;
+  return l2_grid_blocks(d.V, di);
+}
+
+// Path shared by rq_lut_logits and rq_logits_from_hidden.
+int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, int B, int Bs,
+               float cap, float *logits, int32_t *argmax, unsigned char *ws,
+               const WsLayout &w, const DevInfo &di, cudaStream_t s) {
+  const int P = d.M * d.L;
+  float *amv = argmax ? reinterpret_cast<float *>(ws + w.amv_off) : nullptr;
+  int *ami = argmax ? reinterpret_cast<int *>(ws + w.ami_off) : nullptr;
+  const int nblk = sweep_blocks(d, di, w.chunk);
+  cudaError_t e;
+  if (w.chunk) {
+    float *partial = reinterpret_cast<float *>(ws + w.partial_off);
+    if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
+    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, di, s);
+    if (e != cudaSuccess) return status_of(e);
+    if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
+    e = launch_reduce_partials(partial, w.cp.nch, B, d.V, cap, logits, amv, ami, nblk, s);
+    if (e != cudaSuccess) return status_of(e);
+  } else {
+    if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
+    for (int b0 = 0; b0 < B; b0 += kTokenGroup) {
+      const int nb = B - b0 < kTokenGroup ? B - b0 : kTokenGroup;
+      e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, b0, b0, nb, cap, logits, amv, ami,
+                           nblk, s);
+      if (e != cudaSuccess) return status_of(e);
+    }
+    if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
+  }
+  if (argmax) {
+    e = launch_argmax_finalize(amv, ami, nblk, B, argmax, s);
+    if (e != cudaSuccess) return status_of(e);
+  }
+  return RQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *rq_status_string(int status) {
+  switch (status) {
+    case RQ_OK: return "RQ_OK";
+    case RQ_ERR_INVALID_ARGUMENT: return "RQ_ERR_INVALID_ARGUMENT";
+    case RQ_ERR_UNSUPPORTED: return "RQ_ERR_UNSUPPORTED";
+    case RQ_ERR_WORKSPACE_TOO_SMALL: return "RQ_ERR_WORKSPACE_TOO_SMALL";
+    case RQ_ERR_CUDA: return "RQ_ERR_CUDA";
+    case RQ_ERR_MISALIGNED: return "RQ_ERR_MISALIGNED";
+    default: return "RQ_ERR_UNKNOWN";
+  }
+}
+
+int rq_version(void) { return 100; }
+
+size_t rq_codes_bytes(rq_dims d, int fmt) {
+  if (!dims_ok(d) || !fmt_ok(d, fmt)) return 0;
+  const int64_t P = (int64_t)d.M * d.L;
+  if (fmt == RQ_CODES_U16) return (size_t)(d.V * P * 2);
+  return (size_t)(d.V * ((10 * P + 7) / 8));
+}
+
+int rq_lut_token_stride(int B) {
+  if (B < 1) return 0;
+  if (B <= 2) return B;
+  return (B + 3) / 4 * 4;
+}
+
+size_t rq_lut_bytes(rq_dims d, int B) {
+  if (!dims_ok(d) || B < 1) return 0;
+  return (size_t)d.M * d.L * d.K * rq_lut_token_stride(B) * sizeof(float);
+}
+
+size_t rq_logits_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax) {
+  if (!dims_ok(d) || !fmt_ok(d, fmt) || B < 1) return 0;
+  return ws_layout(d, B, fmt, want_argmax != 0, nominal_devinfo()).total;
+}
+
+static int fused_group(int B) { return B <= 4 ? B : (B < kTokenGroup ? B : kTokenGroup); }
+
+size_t rq_fused_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax) {
+  if (!dims_ok(d) || !fmt_ok(d, fmt) || B < 1) return 0;
+  const int G = fused_group(B);
+  const size_t lut = (size_t)align_up((int64_t)rq_lut_bytes(d, G), kAlign);
+  return lut + ws_layout(d, B, fmt, want_argmax != 0, nominal_devinfo()).total;
+}
+
+int rq_lut_build(const float *h, const float *C, rq_dims d, int B, float *lut, void *stream) {
+  if (!h || !C || !lut || B < 1 || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(h, 4) || !aligned(C, 4) || !aligned(lut, 16)) return RQ_ERR_MISALIGNED;
+  const int Bs = rq_lut_token_stride(B);
+  if ((size_t)Bs * (d.D / d.M) * 4 > 48 * 1024) return RQ_ERR_UNSUPPORTED;
+  return status_of(launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int rq_lut_logits(const void *codes, int fmt, rq_dims d, const float *lut, int B, float softcap,
+                  float *logits, int32_t *argmax, void *ws, size_t ws_bytes, void *stream) {
+  if (!codes || !lut || B < 1 || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
+  if (!logits && !argmax) return RQ_ERR_INVALID_ARGUMENT;
+  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
+  if (!aligned(codes, 16) || !aligned(lut, 16) || (ws && !aligned(ws, 16)) ||
+      (logits && !aligned(logits, 4)) || (argmax && !aligned(argmax, 4)))
+    return RQ_ERR_MISALIGNED;
+  DevInfo di;
+  if (dev_info(&di) != cudaSuccess) return RQ_ERR_CUDA;
+  const WsLayout w = ws_layout(d, B, fmt, argmax != nullptr, di);
+  if (w.total > 0 && (!ws || ws_bytes < w.total)) return RQ_ERR_WORKSPACE_TOO_SMALL;
+  return run_logits(codes, fmt, d, lut, B, rq_lut_token_stride(B), softcap, logits, argmax,
+                    static_cast<unsigned char *>(ws), w, di, static_cast<cudaStream_t>(stream));
+}
+
+int rq_logits_from_hidden(const float *h, const float *C, const void *codes, int fmt, rq_dims d,
+                          int B, float softcap, float *logits, int32_t *argmax, void *ws,
+                          size_t ws_bytes, void *stream) {
+  if (!h || !C || !codes || B < 1 || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
+  if (!logits && !argmax) return RQ_ERR_INVALID_ARGUMENT;
+  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
+  if (!ws) return RQ_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned(h, 4) || !aligned(C, 4) || !aligned(codes, 16) || !aligned(ws, 16) ||
+      (logits && !aligned(logits, 4)) || (argmax && !aligned(argmax, 4)))
+    return RQ_ERR_MISALIGNED;
+  DevInfo di;
+  if (dev_info(&di) != cudaSuccess) return RQ_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int G = fused_group(B);
+  const int Bs = rq_lut_token_stride(G);
+  if ((size_t)Bs * (d.D / d.M) * 4 > 48 * 1024) return RQ_ERR_UNSUPPORTED;
+  const size_t lut_bytes = (size_t)align_up((int64_t)rq_lut_bytes(d, G), kAlign);
+  const WsLayout w = ws_layout(d, B, fmt, argmax != nullptr, di);
+  if (ws_bytes < lut_bytes + w.total) return RQ_ERR_WORKSPACE_TOO_SMALL;
+  float *lut = static_cast<float *>(ws);
+  unsigned char *rest = static_cast<unsigned char *>(ws) + lut_bytes;
+  if (w.chunk) {
+    // B <= 4: one table for all tokens, then the vocabulary-tiled pass
+    cudaError_t e = launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut, s);
+    if (e != cudaSuccess) return status_of(e);
+    return run_logits(codes, fmt, d, lut, B, Bs, softcap, logits, argmax, rest, w, di, s);
+  }
+  const int P = d.M * d.L;
+  float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
+  int *ami = argmax ? reinterpret_cast<int *>(rest + w.ami_off) : nullptr;
+  const int nblk = sweep_blocks(d, di, false);
+  for (int b0 = 0; b0 < B; b0 += G) {
+    const int nb = B - b0 < G ? B - b0 : G;
+    cudaError_t e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, s);
+    if (e != cudaSuccess) return status_of(e);
+    if (b0 == 0 && (e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
+    e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, 0, b0, nb, softcap, logits, amv, ami,
+                         nblk, s);
+    if (e != cudaSuccess) return status_of(e);
+  }
+  if (cudaError_t e = prof_mark(t_prof_stop, s)) return status_of(e);
+  if (argmax) return status_of(launch_argmax_finalize(amv, ami, nblk, B, argmax, s));
+  return RQ_OK;
+}
+
+int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt, const float *C,
+                   rq_dims d, float scale, uint16_t *out, void *stream) {
+  if (N < 0 || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
+  if (N == 0) return RQ_OK;
+  if (!ids || !codes || !C || !out) return RQ_ERR_INVALID_ARGUMENT;
+  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
+  if (!aligned(ids, 4) || !aligned(codes, 2) || !aligned(C, 4) || !aligned(out, 2))
+    return RQ_ERR_MISALIGNED;
+  DevInfo di;
+  if (dev_info(&di) != cudaSuccess) return RQ_ERR_CUDA;
+  return status_of(launch_decode_rows(ids, N, codes, fmt, C, d.V, d.D, d.M, d.L, d.K, scale, out,
+                                      di.err, static_cast<cudaStream_t>(stream)));
+}
+
+int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed, void *stream) {
+  if (!codes_u16 || !packed || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(codes_u16, 2)) return RQ_ERR_MISALIGNED;
+  return status_of(
+      launch_pack10(codes_u16, d.V, d.M * d.L, packed, static_cast<cudaStream_t>(stream)));
+}
+
+int rq_set_profile_events(void *start, void *stop) {
+  if ((start == nullptr) != (stop == nullptr)) return RQ_ERR_INVALID_ARGUMENT;
+  t_prof_start = static_cast<cudaEvent_t>(start);
+  t_prof_stop = static_cast<cudaEvent_t>(stop);
+  return RQ_OK;
+}
+
+int rq_device_error(uint32_t *out, int clear) {
+  if (!out) return RQ_ERR_INVALID_ARGUMENT;
+  DevInfo di;
+  if (dev_info(&di) != cudaSuccess) return RQ_ERR_CUDA;
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpy(&v, di.err, sizeof v, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return RQ_ERR_CUDA;
+  *out = v;
+  if (clear) {
+    e = cudaMemset(di.err, 0, sizeof(unsigned));
+    if (e != cudaSuccess) return RQ_ERR_CUDA;
+  }
+  return RQ_OK;
+}
+
+}  // extern "C"

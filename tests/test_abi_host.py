@@ -1,0 +1,130 @@
+"""Host-only checks of the C ABI (no GPU needed, no kernel launched):
+the library loads, exports every function ``include/rqlut.h`` declares, its
+size arithmetic matches the layouts the header states, and malformed
+arguments are rejected before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import lut_logits_serving_b200 as rq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rqlut.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RQ_API\s+[\w\s\*]*?\b(rq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("rq_lut_build", "rq_lut_logits", "rq_decode_rows", "rq_logits_from_hidden",
+              "rq_pack10", "rq_device_error", "rq_lut_bytes", "rq_logits_workspace_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = rq.lib()
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    # and only the ABI is visible (internal C++ symbols are hidden)
+    out = os.popen(f"nm -D --defined-only {rq.LIB_PATH}").read()
+    exported = set(re.findall(r" T (\w+)", out))
+    assert set(declared_functions()) <= exported
+    assert not [s for s in exported if s.startswith("_ZN2rq")]
+
+
+def test_binding_covers_every_declared_symbol():
+    for n in declared_functions():
+        assert callable(getattr(rq, n)), n
+
+
+G2 = rq.dims(256000, 2304, 384, 2, 1024)
+TINY = rq.dims(4096, 192, 32, 2, 256)
+
+
+def test_status_strings():
+    assert rq.rq_status_string(0) == "RQ_OK"
+    assert rq.rq_status_string(3) == "RQ_ERR_WORKSPACE_TOO_SMALL"
+    assert rq.rq_status_string(99) == "RQ_ERR_UNKNOWN"
+    assert rq.rq_version() >= 100
+
+
+def test_code_and_lut_sizes():
+    # u16 codes [V][M*L]: 393.216 MB; packed 10-bit rows of 960 bytes
+    assert rq.rq_codes_bytes(G2, rq.U16) == 256000 * 768 * 2
+    assert rq.rq_codes_bytes(G2, rq.PACKED10) == 256000 * 960
+    assert rq.rq_codes_bytes(TINY, rq.PACKED10) == 4096 * 80
+    assert rq.rq_codes_bytes(rq.dims(10, 3, 1, 1, 1024), rq.PACKED10) == 10 * 2   # ceil(10/8)
+    assert rq.rq_codes_bytes(rq.dims(10, 3, 1, 1, 2048), rq.PACKED10) == 0       # K > 1024
+    for B, Bs in ((1, 1), (2, 2), (3, 4), (4, 4), (5, 8), (32, 32), (33, 36), (64, 64)):
+        assert rq.rq_lut_token_stride(B) == Bs
+        assert rq.rq_lut_bytes(G2, B) == 768 * 1024 * Bs * 4
+    assert rq.rq_lut_bytes(G2, 1) == 3145728          # 3.1 MB per token
+
+
+def test_workspace_sizes():
+    # B <= 4 takes the vocabulary-tiled path: partial sums for every chunk
+    ws1 = rq.rq_logits_workspace_bytes(G2, 1, rq.U16, False)
+    assert ws1 > 0 and ws1 % (256000 * 4) == 0 and ws1 // (256000 * 4) <= 64
+    ws1a = rq.rq_logits_workspace_bytes(G2, 1, rq.U16, True)
+    assert ws1a > ws1
+    # B > 4 reads the table through L2: argmax partials only
+    assert rq.rq_logits_workspace_bytes(G2, 32, rq.U16, False) == 0
+    assert 0 < rq.rq_logits_workspace_bytes(G2, 32, rq.U16, True) < 1 << 20
+    # the fused call adds one token group's table (<= 32 tokens)
+    f64 = rq.rq_fused_workspace_bytes(G2, 64, rq.PACKED10, True)
+    assert f64 >= rq.rq_lut_bytes(G2, 32)
+    assert f64 < rq.rq_lut_bytes(G2, 64)
+    # never O(V*M*L) (the pages' naive gather index would be 1.57 GB)
+    for B in (1, 2, 3, 4, 5, 32, 64):
+        assert rq.rq_logits_workspace_bytes(G2, B, rq.U16, True) < 256000 * 768 * 8
+
+
+def test_invalid_dims_give_zero_sizes():
+    for d in (rq.dims(0, 2304, 384, 2, 1024), rq.dims(10, 2305, 384, 2, 1024),
+              rq.dims(10, 2304, 384, 0, 1024), rq.dims(10, 2304, 384, 2, 70000)):
+        assert rq.rq_lut_bytes(d, 1) == 0
+        assert rq.rq_codes_bytes(d, rq.U16) == 0
+    assert rq.rq_lut_bytes(G2, 0) == 0
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_argument_errors_return_before_any_launch():
+    lib = rq.lib()
+    s = _fake(None)
+    null = _fake(None)
+    a = _fake(0x10000)          # never dereferenced: every call below returns early
+    odd = _fake(0x10004)
+    INV, MIS, UNS, WS = 1, 5, 2, 3
+    assert lib.rq_lut_build(null, a, G2, 1, a, s) == INV
+    assert lib.rq_lut_build(a, a, G2, 0, a, s) == INV
+    assert lib.rq_lut_build(a, a, rq.dims(10, 7, 2, 1, 4), 1, a, s) == INV   # D % M != 0
+    assert lib.rq_lut_build(a, a, G2, 1, odd, s) == MIS                     # lut 16-B
+    assert lib.rq_lut_logits(a, 0, G2, a, 1, 30.0, null, null, null, 0, s) == INV
+    assert lib.rq_lut_logits(a, 7, G2, a, 1, 30.0, a, null, null, 0, s) == INV
+    assert lib.rq_lut_logits(a, 1, rq.dims(10, 8, 4, 2, 2048), a, 1, 30.0, a, null, null, 0,
+                             s) == UNS
+    assert lib.rq_lut_logits(odd, 0, G2, a, 1, 30.0, a, null, null, 0, s) == MIS
+    assert lib.rq_lut_logits(a, 0, G2, odd, 1, 30.0, a, null, null, 0, s) == MIS
+    assert lib.rq_logits_from_hidden(a, a, a, 0, G2, 1, 30.0, a, null, null, 0, s) == WS
+    assert lib.rq_decode_rows(null, 5, a, 0, a, G2, 48.0, a, s) == INV
+    assert lib.rq_decode_rows(a, -1, a, 0, a, G2, 48.0, a, s) == INV
+    assert lib.rq_decode_rows(null, 0, null, 0, null, G2, 48.0, null, s) == 0   # N = 0: no-op
+    assert lib.rq_decode_rows(_fake(0x10002), 5, a, 0, a, G2, 48.0, a, s) == MIS
+    assert lib.rq_pack10(null, G2, a, s) == INV
+    assert lib.rq_device_error(None, 0) == INV
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    h = torch.zeros(1, 192)
+    C = torch.zeros(32, 2, 256, 6)
+    with pytest.raises(ValueError):
+        rq.rq_lut_build(h, C, TINY, lut=torch.zeros(64, 256, 1))

@@ -1,0 +1,231 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU
+oracle on the same seeded inputs, element by element.  Small shapes that
+span several tiles and chunks with ragged tails, every kernel path (the
+shared-memory vocabulary-tiled pass for B <= 4, the L2-served token-group
+pass, the generic fallback), both code formats, and the degenerate cases."""
+import numpy as np
+import pytest
+
+import oracle
+from lut_logits_serving_b200 import synth
+from tests.parity import assert_logits_close, check_argmax
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import lut_logits_serving_b200 as rq  # noqa: E402
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def make_case(V, D, M, L, K, B, seed=0, sigmas=(0.05, 0.01), hscale=1.0):
+    C = synth.codebooks(M, L, K, D // M, sigmas, seed)
+    codes = synth.codes(V, M, L, K, seed + 1)
+    h = synth.hidden(B, D, hscale, seed + 2)
+    return C, codes, h
+
+
+def oracle_logits(C, codes, h, cap):
+    T = oracle.lut_build(h, C, "f64")
+    return oracle.softcap(oracle.logits_lut(codes, T), cap)
+
+
+def gpu_codes(codes, fmt, d):
+    c16 = dev(codes.reshape(codes.shape[0], -1))
+    if fmt == rq.U16:
+        return c16
+    return rq.rq_pack10(c16, d)
+
+
+# ------------------------------------------------------------- lut build
+
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 8, 32])
+def test_lut_build_matches_oracle(B):
+    V, D, M, L, K = 64, 192, 32, 2, 256
+    C, _, h = make_case(V, D, M, L, K, B)
+    d = rq.dims(V, D, M, L, K)
+    lut = rq.rq_lut_build(dev(h), dev(C), d).cpu().numpy()
+    Bs = rq.rq_lut_token_stride(B)
+    assert lut.shape == (M * L, K, Bs)
+    T = oracle.lut_build(h, C, "f64")                      # [B, M, L, K]
+    ref = T.reshape(B, M * L, K).transpose(1, 2, 0)        # [P, K, B]
+    scale = np.max(np.abs(ref))
+    assert np.max(np.abs(lut[:, :, :B] - ref)) <= 2e-6 * scale
+    assert np.all(lut[:, :, B:] == 0)                      # padding tokens are zero
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ the logits
+
+CASES = [
+    # V,    D,   M,  L, K,    note
+    (4096, 192, 32, 2, 256),   # the tiny workload
+    (4099, 192, 32, 2, 256),   # ragged last tile
+    (257, 48, 8, 2, 64),       # one row past a tile
+    (1, 48, 8, 2, 64),         # a single row
+    (3000, 288, 48, 2, 1024),  # K = 1024 instances, P = 96 -> 3 chunks (40, 40, 16)
+    (2000, 96, 16, 3, 100),    # L = 3, non-power-of-two K (clamped codes path)
+    (1500, 64, 64, 1, 32),     # ds = 1, L = 1
+    (700, 9, 3, 1, 7),         # P = 3: generic fallback
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "V%d_D%d_M%d_L%d_K%d" % c)
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 13, 32, 33])
+@pytest.mark.parametrize("fmt", [0, 1], ids=["u16", "packed10"])
+def test_logits_and_argmax(case, B, fmt):
+    V, D, M, L, K = case
+    if fmt == rq.PACKED10 and K > 1024:
+        pytest.skip("packed codes hold K <= 1024")
+    C, codes, h = make_case(V, D, M, L, K, B, seed=V + B)
+    d = rq.dims(V, D, M, L, K)
+    cap = 30.0
+    ref = oracle_logits(C, codes, h, cap)
+    dc = gpu_codes(codes, fmt, d)
+    dh, dC = dev(h), dev(C)
+    lut = rq.rq_lut_build(dh, dC, d)
+    logits, am, _ = rq.rq_lut_logits(dc, fmt, d, lut, B, cap, want_argmax=True)
+    got = logits.cpu().numpy()
+    assert got.shape == (B, V)
+    assert_logits_close(got, ref)
+    check_argmax(am.cpu().numpy(), ref)
+    # the fused call gives the same numbers
+    logits2, am2, _ = rq.rq_logits_from_hidden(dh, dC, dc, fmt, d, cap, want_argmax=True)
+    assert_logits_close(logits2.cpu().numpy(), ref)
+    assert np.array_equal(am2.cpu().numpy(), am.cpu().numpy())
+    # argmax alone (logits not written) agrees
+    _, am3, _ = rq.rq_lut_logits(dc, fmt, d, lut, B, cap, want_logits=False, want_argmax=True)
+    assert np.array_equal(am3.cpu().numpy(), am.cpu().numpy())
+    assert rq.rq_device_error() == 0
+
+
+def test_u16_and_packed_agree_bit_for_bit_on_the_generic_order():
+    """Both formats feed the same lookups in the same order in the L2-served
+    pass, so their logits are identical."""
+    V, D, M, L, K, B = 2048, 192, 32, 2, 256, 8
+    C, codes, h = make_case(V, D, M, L, K, B)
+    d = rq.dims(V, D, M, L, K)
+    lut = rq.rq_lut_build(dev(h), dev(C), d)
+    a, _, _ = rq.rq_lut_logits(gpu_codes(codes, 0, d), 0, d, lut, B, 30.0)
+    b, _, _ = rq.rq_lut_logits(gpu_codes(codes, 1, d), 1, d, lut, B, 30.0)
+    assert torch.equal(a, b)
+
+
+def test_softcap_off_gives_raw_sums():
+    V, D, M, L, K, B = 1024, 192, 32, 2, 256, 1
+    C, codes, h = make_case(V, D, M, L, K, B, hscale=20.0)   # large logits
+    d = rq.dims(V, D, M, L, K)
+    T = oracle.lut_build(h, C, "f64")
+    z = oracle.logits_lut(codes, T)
+    assert np.max(np.abs(z)) > 30.0        # the softcap would have bent these
+    lut = rq.rq_lut_build(dev(h), dev(C), d)
+    got, _, _ = rq.rq_lut_logits(dev(codes.reshape(V, -1)), 0, d, lut, B, 0.0)
+    assert_logits_close(got.cpu().numpy(), z)
+    capped, _, _ = rq.rq_lut_logits(dev(codes.reshape(V, -1)), 0, d, lut, B, 30.0)
+    assert float(capped.abs().max()) < 30.0
+
+
+def test_single_codeword_ties_go_to_index_zero():
+    """K = 1: every row is the same vector, all logits are bit-identical and
+    the argmax is row 0 on every path."""
+    V, D, M, L, K = 3000, 48, 8, 2, 1
+    for B in (1, 3, 8):
+        C, codes, h = make_case(V, D, M, L, K, B)
+        d = rq.dims(V, D, M, L, K)
+        lut = rq.rq_lut_build(dev(h), dev(C), d)
+        for fmt in (0, 1):
+            logits, am, _ = rq.rq_lut_logits(gpu_codes(codes, fmt, d), fmt, d, lut, B, 30.0,
+                                             want_argmax=True)
+            lg = logits.cpu().numpy()
+            assert np.all(lg == lg[:, :1])
+            assert np.all(am.cpu().numpy() == 0)
+
+
+def test_planted_maximum_is_found_at_every_position():
+    """One row holds a unique maximum; the argmax must find it wherever it
+    sits (first row, last row, tile and chunk boundaries)."""
+    V, D, M, L, K, B = 5000, 48, 8, 2, 16, 1
+    rng = np.random.default_rng(1)
+    C = synth.codebooks(M, L, K, D // M, (0.05, 0.01), 0)
+    h = synth.hidden(1, D, 1.0, 2)
+    T = oracle.lut_build(h, C, "f64")[0]                   # [M, L, K]
+    best = np.argmax(T, axis=2)                            # best code per table
+    worst = np.argmin(T, axis=2)
+    d = rq.dims(V, D, M, L, K)
+    lut = rq.rq_lut_build(dev(h), dev(C), d)
+    for pos in (0, 1, 255, 256, 2047, 4095, 4999):
+        codes = np.broadcast_to(worst, (V, M, L)).copy().astype(np.uint16)
+        codes[rng.integers(0, V, 50)] = rng.integers(0, K, (50, M, L))
+        codes[pos] = best
+        for fmt in (0, 1):
+            _, am, _ = rq.rq_lut_logits(gpu_codes(codes, fmt, d), fmt, d, lut, B, 30.0,
+                                        want_logits=False, want_argmax=True)
+            assert int(am.cpu()[0]) == pos
+
+
+def test_out_of_range_codes_stay_in_bounds():
+    """Codes >= K never index outside the tables: modulo K for a power of
+    two, clamped to K-1 otherwise (the header's stated behaviour)."""
+    V, D, M, L = 600, 48, 8, 2
+    for K, fix in ((64, lambda c: c % 64), (100, lambda c: np.minimum(c, 99))):
+        C, _, h = make_case(V, D, M, L, K, 1)
+        rng = np.random.default_rng(3)
+        raw = rng.integers(0, 65536, (V, M, L)).astype(np.uint16)
+        d = rq.dims(V, D, M, L, K)
+        lut = rq.rq_lut_build(dev(h), dev(C), d)
+        got, _, _ = rq.rq_lut_logits(dev(raw.reshape(V, -1)), 0, d, lut, 1, 30.0)
+        ref = oracle_logits(C, fix(raw.astype(np.int64)).astype(np.uint16), h, 30.0)
+        assert_logits_close(got.cpu().numpy(), ref)
+
+
+# ------------------------------------------------------------ row decode
+
+@pytest.mark.parametrize("fmt", [0, 1], ids=["u16", "packed10"])
+@pytest.mark.parametrize("shape", [(4096, 192, 32, 2, 256), (5000, 288, 48, 2, 1024),
+                                   (300, 96, 16, 3, 100), (50, 9, 3, 1, 7)])
+def test_decode_rows_bit_exact(shape, fmt):
+    V, D, M, L, K = shape
+    C, codes, _ = make_case(V, D, M, L, K, 1, sigmas=(0.02, 0.005))
+    ids = synth.zipf_ids(257, V, 1.1, 3)
+    d = rq.dims(V, D, M, L, K)
+    scale = float(np.sqrt(D))
+    out = rq.rq_decode_rows(dev(ids), gpu_codes(codes, fmt, d), fmt, dev(C), d, scale)
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    want = oracle.decode_rows_bf16(ids, codes, C, scale)
+    assert np.array_equal(got, want)
+
+
+def test_decode_rows_bad_ids_give_zero_rows_and_a_device_error():
+    V, D, M, L, K = 100, 48, 8, 2, 16
+    C, codes, _ = make_case(V, D, M, L, K, 1)
+    d = rq.dims(V, D, M, L, K)
+    rq.rq_device_error(clear=True)
+    ids = np.array([3, -1, 100, 99], np.int32)
+    out = rq.rq_decode_rows(dev(ids), dev(codes.reshape(V, -1)), 0, dev(C), d, 1.0)
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.all(got[1] == 0) and np.all(got[2] == 0)
+    want = oracle.decode_rows_bf16(np.array([3, 99], np.int32), codes, C, 1.0)
+    assert np.array_equal(got[[0, 3]], want)
+    assert rq.rq_device_error(clear=True) == 2
+    assert rq.rq_device_error() == 0
+
+
+def test_decode_rows_empty_is_a_noop():
+    d = rq.dims(10, 8, 4, 2, 4)
+    lib = rq.lib()
+    assert lib.rq_decode_rows(None, 0, None, 0, None, d, 1.0, None, None) == 0
+
+
+# ---------------------------------------------------------------- packing
+
+@pytest.mark.parametrize("P", [(32, 2), (3, 1), (7, 3), (384, 2)])
+def test_pack10_matches_oracle(P):
+    M, L = P
+    V = 777
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 1024, (V, M, L)).astype(np.uint16)
+    d = rq.dims(V, 8 * M, M, L, 1024)
+    got = rq.rq_pack10(dev(codes.reshape(V, -1)), d).cpu().numpy()
+    assert np.array_equal(got, oracle.pack10(codes))
