@@ -17,34 +17,54 @@
 
 namespace rq {
 
+// Grid (N, ceil(M / 128)): one thread per (row, subspace); the L code loads,
+// then all L*ds codeword loads of a subspace are independent, so a single
+// row costs two dependent memory round trips.
+template <int DS>
 __global__ void __launch_bounds__(128) decode_rows_kernel(
     const int32_t *__restrict__ ids, const void *__restrict__ codes, int fmt,
     const float *__restrict__ C, int64_t V, int D, int M, int L, int K, float scale,
     CodeFix fix, uint16_t *__restrict__ out, unsigned *err) {
   const int64_t n = blockIdx.x;
-  const int ds = D / M;
+  const int m = blockIdx.y * blockDim.x + threadIdx.x;
+  if (m >= M) return;
+  const int ds = DS > 0 ? DS : D / M;
   const int P = M * L;
   const int32_t id = ids[n];
-  uint16_t *orow = out + n * (int64_t)D;
+  uint16_t *o = out + n * (int64_t)D + (int64_t)m * ds;
   if (id < 0 || (int64_t)id >= V) {
-    for (int i = threadIdx.x; i < D; i += blockDim.x) orow[i] = 0;
-    if (threadIdx.x == 0) atomicOr(err, RQ_DEVERR_BAD_ID);
+    for (int j = 0; j < ds; ++j) o[j] = 0;
+    if (m == 0) atomicOr(err, RQ_DEVERR_BAD_ID);
     return;
   }
   const int64_t rb = (10LL * P + 7) / 8;
-  const uint16_t *crow16 = (const uint16_t *)codes + (int64_t)id * P;
-  const uint8_t *crow10 = (const uint8_t *)codes + (int64_t)id * rb;
-  for (int m = threadIdx.x; m < M; m += blockDim.x) {
+  const uint16_t *crow16 = static_cast<const uint16_t *>(codes) + (int64_t)id * P;
+  const uint8_t *crow10 = static_cast<const uint8_t *>(codes) + (int64_t)id * rb;
+  if (DS > 0) {
+    float e[DS > 0 ? DS : 1];
+#pragma unroll
+    for (int j = 0; j < DS; ++j) e[j] = 0.f;
+    for (int l = 0; l < L; ++l) {
+      const int p = m * L + l;
+      const uint32_t c =
+          fix(fmt == RQ_CODES_U16 ? (uint32_t)crow16[p] : packed10_code(crow10, p));
+      const float *cw = C + ((size_t)p * K + c) * DS;
+#pragma unroll
+      for (int j = 0; j < DS; ++j) e[j] = __fadd_rn(e[j], __ldg(cw + j));
+    }
+#pragma unroll
+    for (int j = 0; j < DS; ++j)
+      o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e[j], scale)));
+  } else {
     for (int j = 0; j < ds; ++j) {
       float e = 0.f;
       for (int l = 0; l < L; ++l) {
         const int p = m * L + l;
-        uint32_t c = fmt == RQ_CODES_U16 ? (uint32_t)crow16[p] : packed10_code(crow10, p);
-        c = fix(c);
-        e = __fadd_rn(e, __ldg(C + (((size_t)p * K + c) * ds + j)));
+        const uint32_t c =
+            fix(fmt == RQ_CODES_U16 ? (uint32_t)crow16[p] : packed10_code(crow10, p));
+        e = __fadd_rn(e, __ldg(C + ((size_t)p * K + c) * ds + j));
       }
-      const float s = __fmul_rn(e, scale);
-      orow[m * ds + j] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+      o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e, scale)));
     }
   }
 }
@@ -54,8 +74,14 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
                                float scale, uint16_t *out, unsigned *err, cudaStream_t s) {
   if (N <= 0) return cudaSuccess;
   if (N > 0x7fffffffLL) return cudaErrorInvalidValue;
-  decode_rows_kernel<<<(unsigned)N, 128, 0, s>>>(ids, codes, fmt, C, V, D, M, L, K, scale,
-                                                  make_codefix(K), out, err);
+  const dim3 grid((unsigned)N, (unsigned)((M + 127) / 128));
+  const CodeFix fix = make_codefix(K);
+  if (D / M == 6)
+    decode_rows_kernel<6><<<grid, 128, 0, s>>>(ids, codes, fmt, C, V, D, M, L, K, scale, fix,
+                                                 out, err);
+  else
+    decode_rows_kernel<0><<<grid, 128, 0, s>>>(ids, codes, fmt, C, V, D, M, L, K, scale, fix,
+                                                 out, err);
   return cudaGetLastError();
 }
 

@@ -8,22 +8,22 @@
 //
 // Design for sm_100a.  One token's tables are P*K*4 bytes (3.1 MB at the
 // Gemma-2 shape): far more than one SM's shared memory, but a chunk of PC
-// (m, l) pairs (PC*K*TB*4 bytes) fits.  Work units are (chunk, tile of R
-// vocabulary rows), ordered chunk-major and split evenly over a persistent
-// grid of one CTA per SM, so a CTA loads one or two table chunks into shared
-// memory (from L2, where the build kernel left them) and then streams its
-// code tiles:
-//   * each tile is a TMA 2-D box {PC codes, 256 rows} of the uint16 code
-//     matrix (a 2*PC-byte slice of every 2*P-byte row), landing in an
-//     NST-deep ring of shared-memory stages guarded by mbarriers; the code
-//     stream carries an L2 evict-first policy;
-//   * thread r owns row r of the tile: it reads its 2*PC code bytes with
-//     16-byte shared loads (row pitch = an odd multiple of 16 bytes, so the
-//     8 lanes of each load phase hit distinct bank groups) and performs PC
-//     table lookups, summing TB tokens in fp32 registers;
-//   * the per-chunk sums go to partial[c][b][v]; a second kernel adds the
-//     chunks in order, applies the softcap, writes logits and argmax
-//     partials.  Partials are 4*nch bytes per row and token (L2-resident).
+// (m, l) pairs (PC*K*TB*4 = 128 KB) fits.  The grid is nch x cpc CTAs, one
+// per SM: CTA (c, s) keeps table chunk c resident in shared memory for its
+// whole life and streams slice s of the vocabulary:
+//   * each tile of R rows arrives as TMA 2-D boxes {PC codes, 256 rows} of
+//     the uint16 code matrix -- a 2*PC-byte slice (16, 32 or 64 bytes,
+//     aligned to its own size) of every 2*P-byte row -- into an NST-deep
+//     ring of stages, with the TMA swizzle matching the slice width so the
+//     16-byte shared loads of consecutive rows fall in distinct bank groups;
+//     the code stream carries an L2 evict-first policy;
+//   * TPR threads own one row (PPT pairs each), do their table lookups from
+//     shared memory and sum TB tokens in fp32 registers; the TPR partial
+//     sums meet by a warp shuffle and land in partial[c][b][v];
+//   * there is no block barrier per tile: the last warp to finish a stage
+//     re-arms it with the TMA copy of the tile NST ahead;
+//   * a second kernel adds the nch chunk sums in order, applies the softcap,
+//     writes the logits and reduces the argmax (its last block finishes it).
 #include <cfloat>
 #include <climits>
 
@@ -34,13 +34,36 @@ namespace rq {
 struct ChunkArgs {
   const float *lut;   // [P][K][TB]
   float *partial;     // [nch][B][V]
+  unsigned *counter;  // reduce-kernel block counter, zeroed here
   int64_t V;
-  int64_t ntiles;     // tiles of THREADS rows
-  int64_t nunits;     // nch * ntiles
-  int P, K, B, nch;
+  int64_t ntiles;     // tiles of R rows
+  int P, K, B, nch, cpc;
   CodeFix fix;
   unsigned *err;
 };
+
+template <int TB>
+struct ChunkShape {
+  static constexpr int PC = TB == 1 ? 32 : (TB == 2 ? 16 : 8);  // pairs per chunk
+  static constexpr int PPT = TB == 4 ? 8 : 16;                  // pairs per thread
+  static constexpr int TPR = PC / PPT;                          // threads per row
+  static constexpr int THREADS = 1024;
+  static constexpr int WARPS = THREADS / 32;
+  static constexpr int R = THREADS / TPR;                       // rows per tile
+  static constexpr int ROWB = PC * 2;                           // code bytes per row slice
+  static constexpr int BOXES = R / 256;
+  static constexpr int BOX_BYTES = 256 * ROWB;
+  static constexpr int STAGE_BYTES = R * ROWB;
+};
+
+// 16-byte chunk j of row r (row index inside a 1024-byte-aligned TMA box) as
+// placed by the TMA swizzle whose span equals the row width.
+template <int ROWB>
+__device__ __forceinline__ int swz(int j, int r) {
+  if (ROWB == 64) return j ^ ((r >> 1) & 3);
+  if (ROWB == 32) return j ^ ((r >> 2) & 1);
+  return j;
+}
 
 template <int KT>
 __device__ __forceinline__ uint32_t fix_code(uint32_t c, const CodeFix &f) {
@@ -48,171 +71,299 @@ __device__ __forceinline__ uint32_t fix_code(uint32_t c, const CodeFix &f) {
   return f(c);
 }
 
-template <int TB>
-__device__ __forceinline__ void add_entry(const float *e, float (&acc)[TB]) {
+// Table entry at byte address `addr` (+ immediate OFF) of shared memory,
+// TB tokens wide.  Plain (non-volatile) asm: the table is written before a
+// __syncthreads and never again, so these loads may be scheduled freely.
+template <int TB, int OFF>
+__device__ __forceinline__ void add_entry(uint32_t addr, float (&acc)[TB]) {
   if (TB == 1) {
-    acc[0] += e[0];
+    float x;
+    asm("ld.shared.f32 %0, [%1+%2];" : "=f"(x) : "r"(addr), "n"(OFF));
+    acc[0] += x;
   } else if (TB == 2) {
-    const float2 t = *reinterpret_cast<const float2 *>(e);
-    acc[0] += t.x;
-    acc[1] += t.y;
+    float x, y;
+    asm("ld.shared.v2.f32 {%0, %1}, [%2+%3];" : "=f"(x), "=f"(y) : "r"(addr), "n"(OFF));
+    acc[0] += x;
+    acc[1] += y;
   } else {
-    const float4 t = *reinterpret_cast<const float4 *>(e);
-    acc[0] += t.x;
-    acc[1] += t.y;
-    acc[2] += t.z;
-    acc[3] += t.w;
+    float x, y, z, w;
+    asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4+%5];"
+        : "=f"(x), "=f"(y), "=f"(z), "=f"(w)
+        : "r"(addr), "n"(OFF));
+    acc[0] += x;
+    acc[1] += y;
+    acc[2] += z;
+    acc[3] += w;
   }
 }
 
-// 8 consecutive pairs (one 16-byte code vector) of one row.
+// Runtime-K variant: the pair offset is a register.
+template <int TB>
+__device__ __forceinline__ void add_entry_rt(uint32_t addr, float (&acc)[TB]) {
+  add_entry<TB, 0>(addr, acc);
+}
+
+// 8 consecutive pairs (one 16-byte code vector) of one row; `tbase` is the
+// shared byte address of the first of those 8 tables.
 template <int TB, int KT>
-__device__ __forceinline__ void lookup8(const float *Tg, int K, uint4 w, const CodeFix &f,
+__device__ __forceinline__ void lookup8(uint32_t tbase, int K, uint4 w, const CodeFix &f,
                                         float (&acc)[TB]) {
   const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  if (KT > 0) {
+    constexpr int PB = KT * TB * 4;  // bytes per table
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t c0 = fix_code<KT>(ws[q] & 0xFFFFu, f);
-    const uint32_t c1 = fix_code<KT>(ws[q] >> 16, f);
-    add_entry<TB>(Tg + ((size_t)(2 * q) * K + c0) * TB, acc);
-    add_entry<TB>(Tg + ((size_t)(2 * q + 1) * K + c1) * TB, acc);
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t c0 = fix_code<KT>(ws[q] & 0xFFFFu, f);
+      const uint32_t c1 = fix_code<KT>(ws[q] >> 16, f);
+      switch (q) {  // immediates must be literal constants per unrolled step
+        case 0:
+          add_entry<TB, 0 * PB>(tbase + c0 * (TB * 4), acc);
+          add_entry<TB, 1 * PB>(tbase + c1 * (TB * 4), acc);
+          break;
+        case 1:
+          add_entry<TB, 2 * PB>(tbase + c0 * (TB * 4), acc);
+          add_entry<TB, 3 * PB>(tbase + c1 * (TB * 4), acc);
+          break;
+        case 2:
+          add_entry<TB, 4 * PB>(tbase + c0 * (TB * 4), acc);
+          add_entry<TB, 5 * PB>(tbase + c1 * (TB * 4), acc);
+          break;
+        default:
+          add_entry<TB, 6 * PB>(tbase + c0 * (TB * 4), acc);
+          add_entry<TB, 7 * PB>(tbase + c1 * (TB * 4), acc);
+          break;
+      }
+    }
+  } else {
+    const uint32_t pb = (uint32_t)K * TB * 4;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t c0 = fix_code<KT>(ws[q] & 0xFFFFu, f);
+      const uint32_t c1 = fix_code<KT>(ws[q] >> 16, f);
+      add_entry_rt<TB>(tbase + (2 * q) * pb + c0 * (TB * 4), acc);
+      add_entry_rt<TB>(tbase + (2 * q + 1) * pb + c1 * (TB * 4), acc);
+    }
   }
 }
 
-template <int TB, int KT, int PC, int NST, int THREADS>
-__global__ void __launch_bounds__(THREADS, 1)
-    logits_chunk_u16_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
-  static_assert(PC % 8 == 0 && (PC / 8) % 2 == 1, "row pitch must be an odd multiple of 16 B");
-  static_assert(THREADS % 256 == 0, "tiles are whole TMA boxes of 256 rows");
-  constexpr int STAGE_BYTES = THREADS * PC * 2;
-  constexpr int BOX_BYTES = 256 * PC * 2;
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
 
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *smem = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int TB, int KT, int NST>
+__global__ void __launch_bounds__(1024, 1)
+    logits_chunk_u16_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
+  using S = ChunkShape<TB>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment (TMA swizzle atoms) by pointer arithmetic, so the
+  // compiler keeps the shared address space
+  unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int K = KT > 0 ? KT : a.K;
   float *Ts = reinterpret_cast<float *>(smem);
-  const size_t t_bytes = (size_t)align_up((int64_t)PC * K * TB * 4, 1024);
+  const size_t t_bytes = (size_t)align_up((int64_t)S::PC * K * TB * 4, 1024);
   unsigned char *stages = smem + t_bytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(stages + (size_t)NST * STAGE_BYTES);
+  uint64_t *full = reinterpret_cast<uint64_t *>(stages + (size_t)NST * S::STAGE_BYTES);
+  unsigned *released = reinterpret_cast<unsigned *>(full + NST);
+  int *abort_flag = reinterpret_cast<int *>(released + NST);
 
-  const int64_t per = a.nunits / gridDim.x, rem = a.nunits % gridDim.x;
-  const int64_t bx = blockIdx.x;
-  const int64_t u0 = bx * per + (bx < rem ? bx : rem);
-  const int64_t u1 = u0 + per + (bx < rem ? 1 : 0);
+  const int c = blockIdx.x / a.cpc;          // table chunk of this CTA
+  const int sl = blockIdx.x % a.cpc;         // vocabulary slice
+  const int64_t t0 = a.ntiles * sl / a.cpc;
+  const int64_t t1 = a.ntiles * (sl + 1) / a.cpc;
+  const int64_t n = t1 - t0;                 // tiles of this CTA
+  const int np = min(S::PC, a.P - c * S::PC);
 
-  if (threadIdx.x == 0) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid == 0) {
+    if (blockIdx.x == 0 && a.counter) *a.counter = 0u;
     prefetch_tmap(&tmap);
-    for (int s = 0; s < NST; ++s) mbar_init(smem_addr(&bars[s]), 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(smem_addr(&full[s]), 1);
+      released[s] = 0u;
+    }
+    *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
   const uint64_t pol = l2_policy_evict_first();
-  auto issue = [&](int64_t u, int s) {
-    const int c = (int)(u / a.ntiles);
-    const int64_t t = u % a.ntiles;
-    const uint32_t bar = smem_addr(&bars[s]);
-    mbar_arrive_expect_tx(bar, STAGE_BYTES);
+  auto issue = [&](int64_t i, int s) {   // tile t0 + i into stage s
+    const uint32_t bar = smem_addr(&full[s]);
+    mbar_arrive_expect_tx(bar, S::STAGE_BYTES);
+    const int y = (int)((t0 + i) * S::R);
 #pragma unroll
-    for (int q = 0; q < THREADS / 256; ++q)
-      tma_load_2d(smem_addr(stages + (size_t)s * STAGE_BYTES + q * BOX_BYTES), &tmap, c * PC,
-                  (int)(t * THREADS + q * 256), bar, pol);
+    for (int q = 0; q < S::BOXES; ++q)
+      tma_load_2d(smem_addr(stages + (size_t)s * S::STAGE_BYTES + q * S::BOX_BYTES), &tmap,
+                  c * S::PC, y + q * 256, bar, pol);
   };
+  if (tid == 0)
+    for (int s = 0; s < NST && s < n; ++s) issue(s, s);
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NST; ++s)
-      if (u0 + s < u1) issue(u0 + s, s);
+  // table chunk c -> shared memory (overlaps the first code tiles in flight)
+  {
+    const float4 *src = reinterpret_cast<const float4 *>(a.lut + (size_t)c * S::PC * K * TB);
+    float4 *dst = reinterpret_cast<float4 *>(Ts);
+    const int n4 = np * K * TB / 4;
+    for (int q = tid; q < n4; q += S::THREADS) dst[q] = __ldg(src + q);
   }
+  __syncthreads();
 
-  int cur = -1;
-  bool failed = false;
-  int64_t u = u0;
-  for (; u < u1; ++u) {
-    const int64_t i = u - u0;
-    const int c = (int)(u / a.ntiles);
-    const int64_t t = u % a.ntiles;
-    const int np = min(PC, a.P - c * PC);
-    if (c != cur) {
-      // Table chunk c -> shared memory (all threads finished the previous
-      // tile at the barrier that ended the last iteration).
-      const float4 *src = reinterpret_cast<const float4 *>(a.lut + (size_t)c * PC * K * TB);
-      float4 *dst = reinterpret_cast<float4 *>(Ts);
-      const int n4 = np * K * TB / 4;
-      for (int q = threadIdx.x; q < n4; q += THREADS) dst[q] = __ldg(src + q);
-      __syncthreads();
-      cur = c;
-    }
+  const int r = tid / S::TPR;                // row of the tile owned by this thread
+  const int hh = tid % S::TPR;               // which PPT pairs of the row
+  const int box = r >> 8, rr = r & 255;
+  const uint32_t tt = smem_addr(Ts) + (uint32_t)hh * S::PPT * K * TB * 4;
+  constexpr int NQ = S::PPT / 8;             // 16-byte code vectors per thread
+
+  for (int64_t i = 0; i < n; ++i) {
+    if (*reinterpret_cast<volatile int *>(abort_flag)) break;
     const int s = (int)(i % NST);
-    const uint32_t par = (uint32_t)((i / NST) & 1);
-    const bool ok = mbar_wait_bounded(smem_addr(&bars[s]), par);
-    if (ok) {
-      const int64_t v = t * THREADS + threadIdx.x;
-      const int ng = np / 8;
-      const uint4 *row =
-          reinterpret_cast<const uint4 *>(stages + (size_t)s * STAGE_BYTES + threadIdx.x * PC * 2);
-      float acc[TB];
-#pragma unroll
-      for (int b = 0; b < TB; ++b) acc[b] = 0.f;
-#pragma unroll
-      for (int g = 0; g < PC / 8; ++g) {
-        if (g < ng) lookup8<TB, KT>(Ts + (size_t)g * 8 * K * TB, K, row[g], a.fix, acc);
-      }
-      if (v < a.V) {
-#pragma unroll
-        for (int b = 0; b < TB; ++b)
-          if (b < a.B) a.partial[((size_t)c * a.B + b) * a.V + v] = acc[b];
-      }
-    }
-    if (__syncthreads_or(!ok)) {
-      failed = true;
+    if (!mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((i / NST) & 1))) {
+      *reinterpret_cast<volatile int *>(abort_flag) = 1;
       break;
     }
-    if (threadIdx.x == 0 && u + NST < u1) issue(u + NST, s);
+    const uint32_t rowp =
+        smem_addr(stages) + (uint32_t)(s * S::STAGE_BYTES + box * S::BOX_BYTES + rr * S::ROWB);
+    float acc[TB];
+#pragma unroll
+    for (int b = 0; b < TB; ++b) acc[b] = 0.f;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int j = hh * NQ + q;
+      if (j * 8 < np) {
+        const uint4 w = ld_shared_v4(rowp + 16 * swz<S::ROWB>(j, rr));
+        lookup8<TB, KT>(tt + (uint32_t)q * 8 * K * TB * 4, K, w, a.fix, acc);
+      }
+    }
+    if (S::TPR == 2) {
+#pragma unroll
+      for (int b = 0; b < TB; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], 1);
+    }
+    const int64_t v = (t0 + i) * S::R + r;
+    if (hh == 0 && v < a.V) {
+#pragma unroll
+      for (int b = 0; b < TB; ++b)
+        if (b < a.B) a.partial[((size_t)c * a.B + b) * a.V + v] = acc[b];
+    }
+    // release the stage; the last warp re-arms it with tile i + NST
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      const unsigned old = atomicAdd(&released[s], 1u);
+      if (old == S::WARPS - 1) {
+        released[s] = 0u;
+        if (i + NST < n && !*reinterpret_cast<volatile int *>(abort_flag)) {
+          fence_proxy_async_smem();
+          issue(i + NST, s);
+        }
+      }
+    }
   }
-  if (failed && threadIdx.x == 0) {
+  __syncthreads();
+  if (tid == 0 && *reinterpret_cast<volatile int *>(abort_flag)) {
     atomicOr(a.err, RQ_DEVERR_TIMEOUT);
-    // Let copies already in flight land before the CTA's shared memory goes.
-    for (int64_t w = u; w < u1 && w < u + NST; ++w) {
-      const int64_t i = w - u0;
-      mbar_wait_bounded(smem_addr(&bars[i % NST]), (uint32_t)((i / NST) & 1));
+    // let copies still in flight land before the CTA's shared memory goes
+    for (int s = 0; s < NST; ++s) {
+      for (int64_t i = s; i < n; i += NST) {
+        if (!mbar_try_wait(smem_addr(&full[s]), (uint32_t)((i / NST) & 1))) {
+          mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((i / NST) & 1));
+          break;
+        }
+      }
     }
   }
 }
 
 // ------------------------------------------------------------ reduction
 
-__global__ void __launch_bounds__(256) reduce_partials_kernel(const float *__restrict__ partial,
-                                                              int nch, int B, int64_t V,
-                                                              float cap, float *logits,
-                                                              float *am_val, int *am_idx) {
-  const int b = blockIdx.y;
-  ArgBest best{-FLT_MAX, INT_MAX};
-  bool any = false;
-  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < V;
-       v += (int64_t)gridDim.x * blockDim.x) {
-    float z = 0.f;
-    for (int c = 0; c < nch; ++c) z += __ldcs(partial + ((size_t)c * B + b) * V + v);
-    const float y = softcap_f(z, cap);
-    if (logits) logits[(size_t)b * V + v] = y;
-    const ArgBest cand{y, (int)v};
-    best = any ? arg_better(best, cand) : cand;
-    any = true;
-  }
-  if (am_val == nullptr) return;
-  if (!any) best = ArgBest{-FLT_MAX, INT_MAX};
+// Block-wide argmax of one (value, index) per thread; result in thread 0.
+__device__ __forceinline__ ArgBest block_argbest(ArgBest best, ArgBest *scratch) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) best = arg_better(best, arg_shfl_xor(best, o));
-  __shared__ ArgBest wbest[8];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (lane == 0) wbest[warp] = best;
   __syncthreads();
+  if (lane == 0) scratch[warp] = best;
+  __syncthreads();
+  ArgBest r = scratch[0];
+  if (threadIdx.x == 0)
+    for (int w = 1; w < (int)blockDim.x / 32; ++w) r = arg_better(r, scratch[w]);
+  return r;
+}
+
+// z = sum of the nch chunk sums in chunk order; softcap; logits; argmax.
+// Grid (nblk, B).  With `argmax` set, each block leaves its best (value,
+// index) in am_val/am_idx and the last block to finish reduces them.
+// Rows go 4 per thread (16-byte loads) when V is a multiple of 4.
+__global__ void __launch_bounds__(256) reduce_partials_kernel(
+    const float *__restrict__ partial, int nch, int B, int64_t V, float cap, float *logits,
+    float *am_val, int *am_idx, unsigned *counter, int32_t *argmax) {
+  __shared__ ArgBest scratch[8];
+  __shared__ bool last;
+  const int b = blockIdx.y;
+  ArgBest best{-FLT_MAX, INT_MAX};
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  if ((V & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0) {
+    const int64_t V4 = V / 4;
+    for (int64_t v4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v4 < V4; v4 += stride) {
+      float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 *src = reinterpret_cast<const float4 *>(partial + (size_t)b * V) + v4;
+      const size_t cstride = (size_t)B * V4;
+#pragma unroll 8
+      for (int c = 0; c < nch; ++c) {
+        const float4 t = __ldcs(src + c * cstride);
+        z.x += t.x;
+        z.y += t.y;
+        z.z += t.z;
+        z.w += t.w;
+      }
+      const float4 y = make_float4(softcap_f(z.x, cap), softcap_f(z.y, cap),
+                                   softcap_f(z.z, cap), softcap_f(z.w, cap));
+      if (logits) reinterpret_cast<float4 *>(logits + (size_t)b * V)[v4] = y;
+      const int v = (int)(4 * v4);
+      best = arg_better(best, ArgBest{y.x, v});
+      best = arg_better(best, ArgBest{y.y, v + 1});
+      best = arg_better(best, ArgBest{y.z, v + 2});
+      best = arg_better(best, ArgBest{y.w, v + 3});
+    }
+  } else {
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < V; v += stride) {
+      float z = 0.f;
+      for (int c = 0; c < nch; ++c) z += __ldcs(partial + ((size_t)c * B + b) * V + v);
+      const float y = softcap_f(z, cap);
+      if (logits) logits[(size_t)b * V + v] = y;
+      best = arg_better(best, ArgBest{y, (int)v});
+    }
+  }
+  if (argmax == nullptr) return;
+  const ArgBest r = block_argbest(best, scratch);
   if (threadIdx.x == 0) {
-    ArgBest r = wbest[0];
-    for (int w = 1; w < (int)blockDim.x / 32; ++w) r = arg_better(r, wbest[w]);
     am_val[(size_t)b * gridDim.x + blockIdx.x] = r.v;
     am_idx[(size_t)b * gridDim.x + blockIdx.x] = r.i;
+    __threadfence();
+    const unsigned ticket = atomicAdd(counter, 1u);
+    last = ticket == gridDim.x * gridDim.y - 1;
   }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const int nblk = gridDim.x;
+  for (int bb = 0; bb < B; ++bb) {
+    ArgBest t{-FLT_MAX, INT_MAX};
+    for (int k = threadIdx.x; k < nblk; k += blockDim.x)
+      t = arg_better(t, ArgBest{__ldcg(am_val + (size_t)bb * nblk + k),
+                                __ldcg(am_idx + (size_t)bb * nblk + k)});
+    const ArgBest rb = block_argbest(t, scratch);
+    if (threadIdx.x == 0) argmax[bb] = rb.i;
+  }
+  if (threadIdx.x == 0) *counter = 0u;
 }
 
 __global__ void __launch_bounds__(256) argmax_finalize_kernel(const float *__restrict__ am_val,
@@ -260,29 +411,38 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Variant {
-  int TB, KT, PC, NST, THREADS;
+  int TB, KT, NST;
   const void *fn;
+  size_t table_bytes_max;   // PC*K*TB*4 at the largest K served
 };
 
-#define RQ_CHUNK_VARIANT(TB, KT, PC, NST, TH)                                   \
-  Variant {                                                                     \
-    TB, KT, PC, NST, TH,                                                        \
-        reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, PC, NST, TH>) \
+#define RQ_CHUNK_VARIANT(TB, KT, NST)                                              \
+  Variant {                                                                        \
+    TB, KT, NST, reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, NST>), \
+        (size_t)ChunkShape<TB>::PC * 1024 * TB * 4                                 \
   }
 
-// Chosen so table chunk + NST stages fit in 227 KB with one CTA per SM.
+// 128 KB table chunk + NST stages (3 x 32 KB or 5 x 16 KB) per CTA, one CTA
+// per SM.  K = 1024 has its own instances (table offsets as immediates).
 const Variant kVariants[] = {
-    RQ_CHUNK_VARIANT(1, 1024, 40, 3, 256),   // 160 KB table + 3 x 20 KB
-    RQ_CHUNK_VARIANT(2, 1024, 24, 2, 256),   // 192 KB table + 2 x 12 KB
-    RQ_CHUNK_VARIANT(4, 1024, 8, 6, 256),    // 128 KB table + 6 x 4 KB
-    RQ_CHUNK_VARIANT(1, 0, 40, 3, 256),      // any K (runtime)
-    RQ_CHUNK_VARIANT(2, 0, 24, 3, 256),
-    RQ_CHUNK_VARIANT(4, 0, 8, 4, 256),
+    RQ_CHUNK_VARIANT(1, 1024, 3), RQ_CHUNK_VARIANT(2, 1024, 3), RQ_CHUNK_VARIANT(4, 1024, 5),
+    RQ_CHUNK_VARIANT(1, 0, 3),    RQ_CHUNK_VARIANT(2, 0, 3),    RQ_CHUNK_VARIANT(4, 0, 5),
 };
 
+int variant_pc(const Variant &v) {
+  return v.TB == 1 ? ChunkShape<1>::PC : (v.TB == 2 ? ChunkShape<2>::PC : ChunkShape<4>::PC);
+}
+int variant_rows(const Variant &v) {
+  return v.TB == 1 ? ChunkShape<1>::R : (v.TB == 2 ? ChunkShape<2>::R : ChunkShape<4>::R);
+}
+int variant_stage(const Variant &v) {
+  return v.TB == 1 ? ChunkShape<1>::STAGE_BYTES
+                   : (v.TB == 2 ? ChunkShape<2>::STAGE_BYTES : ChunkShape<4>::STAGE_BYTES);
+}
+
 size_t variant_smem(const Variant &v, int K) {
-  return 1024 + (size_t)align_up((int64_t)v.PC * K * v.TB * 4, 1024) +
-         (size_t)v.NST * v.THREADS * v.PC * 2 + 1024;
+  return 1024 + (size_t)align_up((int64_t)variant_pc(v) * K * v.TB * 4, 1024) +
+         (size_t)v.NST * variant_stage(v) + 1024;
 }
 
 }  // namespace
@@ -290,8 +450,8 @@ size_t variant_smem(const Variant &v, int K) {
 ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di) {
   ChunkPlan cp{};
   cp.ok = false;
-  if (fmt != RQ_CODES_U16 || B < 1 || B > 4 || P % 8 != 0) return cp;
-  if (V > (int64_t)INT_MAX - 512) return cp;
+  if (fmt != RQ_CODES_U16 || B < 1 || B > 4 || P % 8 != 0 || K > 1024) return cp;
+  if (V > (int64_t)INT_MAX - 2048) return cp;
   const int TB = rq_lut_token_stride(B);
   for (int i = 0; i < (int)(sizeof(kVariants) / sizeof(kVariants[0])); ++i) {
     const Variant &v = kVariants[i];
@@ -301,9 +461,9 @@ ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di)
     if (smem > (size_t)di.max_smem_optin) continue;
     cp.ok = true;
     cp.TB = TB;
-    cp.PC = v.PC;
-    cp.nch = (P + v.PC - 1) / v.PC;
-    cp.R = v.THREADS;
+    cp.PC = variant_pc(v);
+    cp.nch = (P + cp.PC - 1) / cp.PC;
+    cp.R = variant_rows(v);
     cp.variant = i;
     cp.smem = smem;
     return cp;
@@ -317,23 +477,26 @@ size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V) {
 
 cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
                                 int P, int K, int B, const float *lut, float *partial,
-                                const DevInfo &di, cudaStream_t s) {
+                                unsigned *counter, const DevInfo &di, cudaStream_t s) {
   (void)fmt;
   const Variant &var = kVariants[cp.variant];
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
+  const int rowb = cp.PC * 2;
   const cuuint64_t gdim[2] = {(cuuint64_t)P, (cuuint64_t)V};
   const cuuint64_t gstride[1] = {(cuuint64_t)P * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)var.PC, 256u};
+  const cuuint32_t box[2] = {(cuuint32_t)cp.PC, 256u};
   const cuuint32_t estride[2] = {1u, 1u};
+  const CUtensorMapSwizzle swz = rowb == 64   ? CU_TENSOR_MAP_SWIZZLE_64B
+                                 : rowb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                              : CU_TENSOR_MAP_SWIZZLE_NONE;
   CUresult r = encode_fn()(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(codes),
-                           gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
-  static bool attr_set[64][sizeof(kVariants) / sizeof(kVariants[0])] = {};
-  if (di.device < 64 && !attr_set[di.device][cp.variant]) {
+  static bool attr_set[128][sizeof(kVariants) / sizeof(kVariants[0])] = {};
+  if (di.device < 128 && !attr_set[di.device][cp.variant]) {
     cudaError_t e = cudaFuncSetAttribute(var.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cp.smem);
     if (e != cudaSuccess) return e;
@@ -343,27 +506,29 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   ChunkArgs a;
   a.lut = lut;
   a.partial = partial;
+  a.counter = counter;
   a.V = V;
-  a.ntiles = (V + var.THREADS - 1) / var.THREADS;
-  a.nunits = a.ntiles * cp.nch;
+  a.ntiles = (V + cp.R - 1) / cp.R;
   a.P = P;
   a.K = K;
   a.B = B;
   a.nch = cp.nch;
+  int64_t cpc = di.sms / cp.nch;
+  if (cpc < 1) cpc = 1;
+  if (cpc > a.ntiles) cpc = a.ntiles;
+  a.cpc = (int)cpc;
   a.fix = make_codefix(K);
   a.err = di.err;
-  int64_t grid = di.sms;
-  if (grid > a.nunits) grid = a.nunits;
-  if (grid < 1) grid = 1;
+  const int64_t grid = (int64_t)cp.nch * cpc;
   void *args[] = {&tmap, &a};
-  return cudaLaunchKernel(var.fn, dim3((unsigned)grid), dim3(var.THREADS), args, cp.smem, s);
+  return cudaLaunchKernel(var.fn, dim3((unsigned)grid), dim3(1024), args, cp.smem, s);
 }
 
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
                                    float *logits, float *am_val, int *am_idx, int nblk,
-                                   cudaStream_t s) {
+                                   unsigned *counter, int32_t *argmax, cudaStream_t s) {
   reduce_partials_kernel<<<dim3((unsigned)nblk, (unsigned)B), 256, 0, s>>>(
-      partial, nch, B, V, cap, logits, am_val, am_idx);
+      partial, nch, B, V, cap, logits, am_val, am_idx, counter, argmax);
   return cudaGetLastError();
 }
 

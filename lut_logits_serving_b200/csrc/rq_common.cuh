@@ -190,10 +190,12 @@ ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di)
 size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V);
 cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
                                 int P, int K, int B, const float *lut, float *partial,
-                                const DevInfo &di, cudaStream_t s);
+                                unsigned *counter, const DevInfo &di, cudaStream_t s);
+// Sums the chunk partials, softcap, logits; with `argmax` set also the
+// argmax (block partials in am_val/am_idx, finished by the last block).
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
                                    float *logits, float *am_val, int *am_idx, int nblk,
-                                   cudaStream_t s);
+                                   unsigned *counter, int32_t *argmax, cudaStream_t s);
 
 // Batched pass with the LUT read through L2 (token groups of <= 32).
 cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K,

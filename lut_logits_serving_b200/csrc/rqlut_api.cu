@@ -96,6 +96,7 @@ struct WsLayout {
   ChunkPlan cp;
   size_t partial_off, partial_bytes;
   size_t amv_off, ami_off, am_bytes;
+  size_t counter_off;
   size_t total;
 };
 
@@ -116,13 +117,23 @@ WsLayout ws_layout(const rq_dims &d, int B, int fmt, bool want_argmax, const Dev
     off += (size_t)align_up((int64_t)w.am_bytes, kAlign);
     w.ami_off = off;
     off += (size_t)align_up((int64_t)w.am_bytes, kAlign);
+    if (w.chunk) {
+      w.counter_off = off;
+      off += kAlign;
+    }
   }
   w.total = off;
   return w;
 }
 
 int sweep_blocks(const rq_dims &d, const DevInfo &di, bool chunk) {
-  (void)chunk;
+  if (chunk) {  // reduce kernel: 4 rows per thread, 256 threads per block
+    int64_t n = (d.V + 1023) / 1024;
+    const int64_t cap = (int64_t)di.sms * 8;
+    if (n > cap) n = cap;
+    if (n > kMaxSweepBlocks) n = kMaxSweepBlocks;
+    return n < 1 ? 1 : (int)n;
+  }
   return l2_grid_blocks(d.V, di);
 }
 
@@ -137,12 +148,14 @@ int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, i
   cudaError_t e;
   if (w.chunk) {
     float *partial = reinterpret_cast<float *>(ws + w.partial_off);
+    unsigned *counter = argmax ? reinterpret_cast<unsigned *>(ws + w.counter_off) : nullptr;
     if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
-    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, di, s);
+    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, counter, di, s);
     if (e != cudaSuccess) return status_of(e);
     if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
-    e = launch_reduce_partials(partial, w.cp.nch, B, d.V, cap, logits, amv, ami, nblk, s);
-    if (e != cudaSuccess) return status_of(e);
+    e = launch_reduce_partials(partial, w.cp.nch, B, d.V, cap, logits, amv, ami, nblk, counter,
+                               argmax, s);
+    return status_of(e);
   } else {
     if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
     for (int b0 = 0; b0 < B; b0 += kTokenGroup) {
