@@ -44,20 +44,25 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="g2_b1", choices=["g2_b1", "g2_b32", "packed_b64"])
+    ap.add_argument("--codes", default="u16", choices=["u16", "sched"],
+                    help="uint16 code layout of the unpacked workloads: as drawn, or "
+                         "bank-scheduled once by rq_prepare_sched")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
 
-def workload_config(w):
-    fmt = "packed10 (960 B/row)" if w.packed10 else "uint16 (1536 B/row)"
+def workload_config(w, codes="u16"):
+    fmt = "packed10 (960 B/row)" if w.packed10 else (
+        "uint16 (1536 B/row)" if codes == "u16" else
+        "uint16 (1536 B/row) in the bank-scheduled order of rq_prepare_sched")
     return {
         "workload": f"{w.name}: V={w.V} D={w.D} M={w.M} L={w.L} K={w.K} B={w.B}, {fmt} codes, "
                     f"softcap {w.softcap:g}, logits + argmax, then the {w.B} picked tokens' input "
                     f"rows rebuilt (bf16)",
         "V": w.V, "D": w.D, "M": w.M, "L": w.L, "K": w.K, "B": w.B,
-        "codes": "packed10" if w.packed10 else "u16",
+        "codes": "packed10" if w.packed10 else codes,
         "l2": "inputs larger than L2: the 393 MB / 246 MB code matrix is streamed every step",
     }
 
@@ -239,12 +244,19 @@ def run_ours(args, w):
 
     data = synth.make(w, seed=1000 * rank)
     d = rq.dims(w.V, w.D, w.M, w.L, w.K)
-    fmt = rq.PACKED10 if w.packed10 else rq.U16
+    fmt = rq.PACKED10 if w.packed10 else (rq.SCHED if args.codes == "sched" else rq.U16)
     dC = torch.from_numpy(data["C"]).cuda()
     c16 = torch.from_numpy(data["codes"].reshape(w.V, -1)).cuda()
-    dcodes = rq.rq_pack10(c16, d) if w.packed10 else c16
-    if w.packed10:
+    sched_quality = None
+    if fmt == rq.PACKED10:
+        dcodes = rq.rq_pack10(c16, d)
         del c16
+    elif fmt == rq.SCHED:
+        dcodes, (st, ps) = rq.rq_prepare_sched(c16, d, stats=True)
+        sched_quality = ps / st
+        del c16
+    else:
+        dcodes = c16
     dh = torch.from_numpy(data["h"]).cuda()
     logits = torch.empty((w.B, w.V), dtype=torch.float32, device="cuda")
     am = torch.empty((w.B,), dtype=torch.int32, device="cuda")
@@ -373,8 +385,9 @@ def run_ours(args, w):
         "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
         "us_per_call": t_ms / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(workload_config(w), parallelism=f"replicas x{world}",
-                       launch="cuda graph" if graph is not None else "eager"),
+        "config": dict(workload_config(w, args.codes), parallelism=f"replicas x{world}",
+                       launch="cuda graph" if graph is not None else "eager",
+                       bank_passes_per_step=sched_quality),
         "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": profiled_traffic(kname), "algorithmic_bytes": algo_bytes,

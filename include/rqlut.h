@@ -39,6 +39,17 @@
  *            RQ_CODES_PACKED10: uint8 [V][rb], rb = ceil(10*M*L/8); code
  *                               p occupies bits [10p, 10p+10) of the row,
  *                               bit i being bit (i%8) of byte i/8
+ *            RQ_CODES_SCHED:    uint16 [M*L/32][V][32] (K <= 1024, M*L % 32
+ *                               == 0), written by rq_prepare_sched: chunk-
+ *                               major (columns 32c..32c+31 of every row form
+ *                               one contiguous [V][32] block); each aligned
+ *                               group of 16 columns holds that group's 16
+ *                               codes in a permuted order, entry = (i << 12)
+ *                               | (c << 2) with i in [0,16) the pair's
+ *                               position in the group and c its code.  The
+ *                               order only changes summation order; entries
+ *                               with c >= K add 0 to the logits
+ *                               (rq_decode_rows clamps them to K-1).
  *   lut      float [M*L][K][Bs], Bs = rq_lut_token_stride(B): token b of
  *            table (p, k) at lut[(p*K + k)*Bs + b]
  *   logits   float [B][V]
@@ -71,7 +82,8 @@ typedef struct {
 
 enum rq_code_fmt {
     RQ_CODES_U16 = 0,       /* one uint16 per code (K <= 65536)           */
-    RQ_CODES_PACKED10 = 1   /* 10-bit codes, bit stream per row (K<=1024) */
+    RQ_CODES_PACKED10 = 1,  /* 10-bit codes, bit stream per row (K<=1024) */
+    RQ_CODES_SCHED = 2      /* bank-scheduled uint16 (rq_prepare_sched)   */
 };
 
 enum rq_status {
@@ -187,6 +199,27 @@ RQ_API int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int 
  */
 RQ_API int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed,
               void *stream);
+
+/*
+ * rq_prepare_sched -- convert uint16 codes [V][M*L] into RQ_CODES_SCHED
+ * (same size; chunk-major so that each 32-pair slice streams contiguously).
+ * Not on the pages: a layout of this library.  The lookups of the B <= 2
+ * logits pass run 16 rows x 2 groups of 16 pairs per warp, one lookup per
+ * lane per step, and shared memory serves a step in as many passes as the
+ * most repeated bank (bank = code mod 32).  Random codes give ~3.5 passes;
+ * this call orders each group so that every step's 32 lookups hit as few
+ * repeated banks as a maximum bipartite matching per step allows (~1.8).
+ * Same bytes, same sums (in another order).  Run once per artifact.
+ *   codes_u16 (device) uint16 [V][M*L], values < K (larger values keep
+ *             their low 10 bits); out (device) uint16 [V][M*L], must not
+ *             overlap codes_u16; stats (device) uint64 [2] or NULL:
+ *             receives (steps scheduled, bank passes needed) summed over
+ *             all warps, for reporting the schedule's quality.
+ * Errors: RQ_ERR_INVALID_ARGUMENT (null, bad dims), RQ_ERR_UNSUPPORTED
+ *         (K > 1024 or M*L % 32 != 0), RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ */
+RQ_API int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out,
+                            uint64_t *stats, void *stream);
 
 /*
  * rq_device_error -- read (and, if `clear`, reset) the device error word

@@ -21,7 +21,7 @@ import ctypes
 import os
 
 __all__ = [
-    "RqDims", "RqError", "U16", "PACKED10", "lib", "dims",
+    "RqDims", "RqError", "U16", "PACKED10", "SCHED", "lib", "dims", "rq_prepare_sched",
     "rq_status_string", "rq_version", "rq_codes_bytes", "rq_lut_token_stride",
     "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
     "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
@@ -30,6 +30,7 @@ __all__ = [
 
 U16 = 0
 PACKED10 = 1
+SCHED = 2
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librqlut.so")
 
@@ -74,6 +75,7 @@ _SIGNATURES = {
     "rq_pack10": (_i, [_p, RqDims, _p, _p]),
     "rq_device_error": (_i, [ctypes.POINTER(ctypes.c_uint32), _i]),
     "rq_set_profile_events": (_i, [_p, _p]),
+    "rq_prepare_sched": (_i, [_p, RqDims, _p, _p, _p]),
 }
 
 
@@ -162,7 +164,7 @@ def _check(fn, status):
 
 def _codes_dtype(fmt):
     torch = _torch()
-    return torch.uint16 if fmt == U16 else torch.uint8
+    return torch.uint8 if fmt == PACKED10 else torch.uint16
 
 
 def _empty(shape, dtype, like):
@@ -266,3 +268,21 @@ def rq_set_profile_events(start=None, stop=None):
     sp = ctypes.c_void_p(start.cuda_event if start is not None else None)
     tp = ctypes.c_void_p(stop.cuda_event if stop is not None else None)
     _check("rq_set_profile_events", lib().rq_set_profile_events(sp, tp))
+
+
+def rq_prepare_sched(codes_u16, d: RqDims, out=None, stats=None, stream=None):
+    """uint16 codes [V, P] -> bank-scheduled uint16 codes [V, P] (RQ_CODES_SCHED).
+    With stats=True returns (out, (steps, bank passes)) after a sync."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty((d.V, d.M * d.L), dtype=torch.uint16, device=codes_u16.device)
+    st = None
+    if stats:
+        st = torch.zeros(2, dtype=torch.int64, device=codes_u16.device)
+    _check("rq_prepare_sched", lib().rq_prepare_sched(
+        _cuda(codes_u16, torch.uint16, "codes_u16"), d, _cuda(out, torch.uint16, "out"),
+        _ptr_or_null(st, torch.int64, "stats"), _stream(stream)))
+    if stats:
+        v = st.cpu().tolist()
+        return out, (v[0], v[1])
+    return out

@@ -17,6 +17,28 @@
 
 namespace rq {
 
+// Code of pair p of row `id` in RQ_CODES_SCHED (chunk-major [P/32][V][32]):
+// find index p % 16 in its group.
+__device__ __forceinline__ uint32_t sched_code(const uint16_t *codes, int64_t V, int64_t id,
+                                               int p) {
+  const uint16_t *g = codes + ((int64_t)(p >> 5) * V + id) * 32 + (p & 16);
+  const uint32_t want = (uint32_t)(p & 15);
+  uint32_t c = 0;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t e = g[k];
+    if ((e >> 12) == want) c = (e >> 2) & 0x3FFu;
+  }
+  return c;
+}
+
+__device__ __forceinline__ uint32_t row_code(int fmt, const uint16_t *r16, const uint8_t *r10,
+                                             const uint16_t *all16, int64_t V, int64_t id, int p) {
+  if (fmt == RQ_CODES_U16) return r16[p];
+  if (fmt == RQ_CODES_SCHED) return sched_code(all16, V, id, p);
+  return packed10_code(r10, p);
+}
+
 // Grid (N, ceil(M / 128)): one thread per (row, subspace); the L code loads,
 // then all L*ds codeword loads of a subspace are independent, so a single
 // row costs two dependent memory round trips.
@@ -46,8 +68,7 @@ __global__ void __launch_bounds__(128) decode_rows_kernel(
     for (int j = 0; j < DS; ++j) e[j] = 0.f;
     for (int l = 0; l < L; ++l) {
       const int p = m * L + l;
-      const uint32_t c =
-          fix(fmt == RQ_CODES_U16 ? (uint32_t)crow16[p] : packed10_code(crow10, p));
+      const uint32_t c = fix(row_code(fmt, crow16, crow10, static_cast<const uint16_t *>(codes), V, id, p));
       const float *cw = C + ((size_t)p * K + c) * DS;
 #pragma unroll
       for (int j = 0; j < DS; ++j) e[j] = __fadd_rn(e[j], __ldg(cw + j));
@@ -60,8 +81,7 @@ __global__ void __launch_bounds__(128) decode_rows_kernel(
       float e = 0.f;
       for (int l = 0; l < L; ++l) {
         const int p = m * L + l;
-        const uint32_t c =
-            fix(fmt == RQ_CODES_U16 ? (uint32_t)crow16[p] : packed10_code(crow10, p));
+        const uint32_t c = fix(row_code(fmt, crow16, crow10, static_cast<const uint16_t *>(codes), V, id, p));
         e = __fadd_rn(e, __ldg(C + ((size_t)p * K + c) * ds + j));
       }
       o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e, scale)));

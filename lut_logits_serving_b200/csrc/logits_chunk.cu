@@ -146,6 +146,44 @@ __device__ __forceinline__ void lookup8(uint32_t tbase, int K, uint4 w, const Co
   }
 }
 
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float x;
+  asm("ld.shared.f32 %0, [%1];" : "=f"(x) : "r"(addr));
+  return x;
+}
+
+// RQ_CODES_SCHED, one token: the 16 entries of a group (two 16-byte code
+// vectors), all 16 table loads issued before any add, summed as a tree.
+__device__ __forceinline__ float group16_sched_tb1(uint32_t gbase, uint4 w0, uint4 w1) {
+  const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  float x[16];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    x[2 * q] = lds_f32(gbase + (ws[q] & 0xFFFCu));
+    x[2 * q + 1] = lds_f32(gbase + __umulhi(ws[q] & 0xFFFC0000u, 0x10000u));
+  }
+#pragma unroll
+  for (int w = 1; w < 16; w <<= 1)
+#pragma unroll
+    for (int q = 0; q < 16; q += 2 * w) x[q] += x[q + w];
+  return x[0];
+}
+
+// RQ_CODES_SCHED: 8 entries (i << 12 | c << 2) of one 16-pair group whose
+// tables start at shared byte address `gbase`, each table 1024 * TB floats:
+// the entry times TB is the byte offset.  The mask keeps every address
+// 4-byte aligned and inside the group's 64 KB * TB.
+template <int TB>
+__device__ __forceinline__ void lookup8_sched(uint32_t gbase, uint4 w, float (&acc)[TB]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    add_entry<TB, 0>(gbase + (ws[q] & 0xFFFCu) * TB, acc);
+    // high entry: ((w & 0xFFFC0000) * 2^16) >> 32 plus the base, one IMAD.HI
+    add_entry<TB, 0>(gbase + __umulhi(ws[q] & 0xFFFC0000u, 0x10000u * TB), acc);
+  }
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -159,106 +197,164 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int TB, int KT, int NST>
+template <int TB, int KT, int NST, int FMT>
 __global__ void __launch_bounds__(1024, 1)
     logits_chunk_u16_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
   using S = ChunkShape<TB>;
+  constexpr bool SCHED = FMT == RQ_CODES_SCHED;
+  static_assert(!SCHED || S::PPT == 16, "a thread must own whole 16-pair groups");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment (TMA swizzle atoms) by pointer arithmetic, so the
   // compiler keeps the shared address space
   unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int K = KT > 0 ? KT : a.K;
+  const int KS = SCHED ? 1024 : K;           // table stride (entries) in shared memory
   float *Ts = reinterpret_cast<float *>(smem);
-  const size_t t_bytes = (size_t)align_up((int64_t)S::PC * K * TB * 4, 1024);
+  const size_t t_bytes = (size_t)align_up((int64_t)S::PC * KS * TB * 4, 1024);
   unsigned char *stages = smem + t_bytes;
   uint64_t *full = reinterpret_cast<uint64_t *>(stages + (size_t)NST * S::STAGE_BYTES);
-  unsigned *released = reinterpret_cast<unsigned *>(full + NST);
+  uint64_t *tbar = full + NST;
+  unsigned *released = reinterpret_cast<unsigned *>(tbar + 1);
   int *abort_flag = reinterpret_cast<int *>(released + NST);
 
   const int c = blockIdx.x / a.cpc;          // table chunk of this CTA
   const int sl = blockIdx.x % a.cpc;         // vocabulary slice
   const int64_t t0 = a.ntiles * sl / a.cpc;
   const int64_t t1 = a.ntiles * (sl + 1) / a.cpc;
-  const int64_t n = t1 - t0;                 // tiles of this CTA
+  const int n = (int)(t1 - t0);              // tiles of this CTA
   const int np = min(S::PC, a.P - c * S::PC);
-
   const int tid = threadIdx.x, lane = tid & 31;
+  // bulk copies need 16-byte sizes and addresses
+  const bool bulk_table = (K * TB) % 4 == 0;
+
   if (tid == 0) {
-    if (blockIdx.x == 0 && a.counter) *a.counter = 0u;
     prefetch_tmap(&tmap);
     for (int s = 0; s < NST; ++s) {
       mbar_init(smem_addr(&full[s]), 1);
       released[s] = 0u;
     }
+    mbar_init(smem_addr(tbar), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
   const uint64_t pol = l2_policy_evict_first();
-  auto issue = [&](int64_t i, int s) {   // tile t0 + i into stage s
+  const uint32_t stage0 = smem_addr(stages);
+  // Box origin of this CTA's code slice: column c*PC of the [V][P] matrix,
+  // or, for the chunk-major scheduled layout [P/32][V][32], rows c32*V + v
+  // at column (c % (32/PC)) * PC.
+  const int box_x = SCHED ? (c % (32 / S::PC)) * S::PC : c * S::PC;
+  const int64_t box_y0 = SCHED ? (int64_t)(c / (32 / S::PC)) * a.V : 0;
+  auto issue = [&](int i, int s) {           // tile t0 + i into stage s
     const uint32_t bar = smem_addr(&full[s]);
     mbar_arrive_expect_tx(bar, S::STAGE_BYTES);
-    const int y = (int)((t0 + i) * S::R);
+    const int y = (int)(box_y0 + (t0 + i) * S::R);
 #pragma unroll
     for (int q = 0; q < S::BOXES; ++q)
-      tma_load_2d(smem_addr(stages + (size_t)s * S::STAGE_BYTES + q * S::BOX_BYTES), &tmap,
-                  c * S::PC, y + q * 256, bar, pol);
+      tma_load_2d(stage0 + s * S::STAGE_BYTES + q * S::BOX_BYTES, &tmap, box_x, y + q * 256,
+                  bar, pol);
   };
+  // The code tiles do not depend on the previous kernel: start them before
+  // waiting for it (programmatic dependent launch), then fetch the tables.
   if (tid == 0)
     for (int s = 0; s < NST && s < n; ++s) issue(s, s);
+  griddep_wait();
+  if (tid == 0 && blockIdx.x == 0 && a.counter) *a.counter = 0u;
 
-  // table chunk c -> shared memory (overlaps the first code tiles in flight)
-  {
-    const float4 *src = reinterpret_cast<const float4 *>(a.lut + (size_t)c * S::PC * K * TB);
-    float4 *dst = reinterpret_cast<float4 *>(Ts);
-    const int n4 = np * K * TB / 4;
-    for (int q = tid; q < n4; q += S::THREADS) dst[q] = __ldg(src + q);
+  // table chunk c -> shared memory
+  const float *src = a.lut + (size_t)c * S::PC * K * TB;
+  if (bulk_table) {
+    if (tid == 0) {
+      const uint32_t tb = smem_addr(tbar);
+      const uint32_t per = (uint32_t)K * TB * 4;
+      if (!SCHED) {
+        mbar_arrive_expect_tx(tb, per * np);
+        bulk_g2s(smem_addr(Ts), src, per * np, tb);
+      } else {
+        mbar_arrive_expect_tx(tb, per * np);
+        for (int p = 0; p < np; ++p)
+          bulk_g2s(smem_addr(Ts) + (uint32_t)p * 1024 * TB * 4, src + (size_t)p * K * TB, per, tb);
+      }
+    }
+    if constexpr (SCHED) {
+      if (K < 1024) {                        // codes >= K read zeros
+        const int pad = (1024 - K) * TB;
+        for (int q = tid; q < np * pad; q += S::THREADS)
+          Ts[(q / pad) * 1024 * TB + K * TB + q % pad] = 0.f;
+      }
+    }
+  } else {
+    const int per = KS * TB;
+    for (int q = tid; q < np * per; q += S::THREADS) {
+      const int pp = q / per, e = q % per;
+      Ts[q] = e < K * TB ? __ldg(src + (size_t)pp * K * TB + e) : 0.f;
+    }
   }
   __syncthreads();
+  const bool table_ok = !bulk_table || mbar_wait_bounded(smem_addr(tbar), 0u);
+  if (!table_ok) *reinterpret_cast<volatile int *>(abort_flag) = 1;
 
   const int r = tid / S::TPR;                // row of the tile owned by this thread
   const int hh = tid % S::TPR;               // which PPT pairs of the row
   const int box = r >> 8, rr = r & 255;
-  const uint32_t tt = smem_addr(Ts) + (uint32_t)hh * S::PPT * K * TB * 4;
+  const uint32_t tt = smem_addr(Ts) + (uint32_t)hh * S::PPT * KS * TB * 4;
   constexpr int NQ = S::PPT / 8;             // 16-byte code vectors per thread
+  uint32_t voff[NQ];                         // this thread's code vectors in a stage
+#pragma unroll
+  for (int q = 0; q < NQ; ++q)
+    voff[q] = (uint32_t)(box * S::BOX_BYTES + rr * S::ROWB) + 16 * swz<S::ROWB>(hh * NQ + q, rr);
+  int nq = 0;                                // vectors holding real pairs
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) nq += ((hh * NQ + q) * 8 < np) ? 1 : 0;
+  float *out = a.partial + (size_t)c * a.B * a.V;
+  int64_t v = t0 * S::R + r;
 
-  for (int64_t i = 0; i < n; ++i) {
-    if (*reinterpret_cast<volatile int *>(abort_flag)) break;
-    const int s = (int)(i % NST);
-    if (!mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((i / NST) & 1))) {
+  int s = 0;
+  uint32_t phase = 0;
+  for (int i = 0; i < n && table_ok; ++i) {
+    const uint32_t fb = smem_addr(&full[s]);
+    if (!mbar_try_wait(fb, phase) && !mbar_wait_bounded(fb, phase)) {
       *reinterpret_cast<volatile int *>(abort_flag) = 1;
       break;
     }
-    const uint32_t rowp =
-        smem_addr(stages) + (uint32_t)(s * S::STAGE_BYTES + box * S::BOX_BYTES + rr * S::ROWB);
+    const uint32_t st = stage0 + s * S::STAGE_BYTES;
     float acc[TB];
 #pragma unroll
     for (int b = 0; b < TB; ++b) acc[b] = 0.f;
+    if (SCHED && TB == 1) {
+      if (nq > 0) {                          // a whole 16-pair group
+        const uint4 w0 = ld_shared_v4(st + voff[0]);
+        const uint4 w1 = ld_shared_v4(st + voff[NQ - 1]);
+        acc[0] = group16_sched_tb1(tt, w0, w1);
+      }
+    } else {
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) {
-      const int j = hh * NQ + q;
-      if (j * 8 < np) {
-        const uint4 w = ld_shared_v4(rowp + 16 * swz<S::ROWB>(j, rr));
-        lookup8<TB, KT>(tt + (uint32_t)q * 8 * K * TB * 4, K, w, a.fix, acc);
+      for (int q = 0; q < NQ; ++q) {
+        if (q < nq) {
+          const uint4 w = ld_shared_v4(st + voff[q]);
+          if (SCHED)
+            lookup8_sched<TB>(tt, w, acc);
+          else
+            lookup8<TB, KT>(tt + (uint32_t)q * 8 * K * TB * 4, K, w, a.fix, acc);
+        }
       }
     }
     if (S::TPR == 2) {
 #pragma unroll
       for (int b = 0; b < TB; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], 1);
     }
-    const int64_t v = (t0 + i) * S::R + r;
     if (hh == 0 && v < a.V) {
 #pragma unroll
       for (int b = 0; b < TB; ++b)
-        if (b < a.B) a.partial[((size_t)c * a.B + b) * a.V + v] = acc[b];
+        if (b < a.B) out[(size_t)b * a.V + v] = acc[b];
     }
+    v += S::R;
     // release the stage; the last warp re-arms it with tile i + NST
     __syncwarp();
     if (lane == 0) {
       __threadfence_block();
-      const unsigned old = atomicAdd(&released[s], 1u);
-      if (old == S::WARPS - 1) {
+      if (atomicAdd(&released[s], 1u) == S::WARPS - 1) {
         released[s] = 0u;
         if (i + NST < n && !*reinterpret_cast<volatile int *>(abort_flag)) {
           fence_proxy_async_smem();
@@ -266,15 +362,21 @@ __global__ void __launch_bounds__(1024, 1)
         }
       }
     }
+    if (++s == NST) {
+      s = 0;
+      phase ^= 1u;
+    }
   }
+  griddep_launch_dependents();
   __syncthreads();
   if (tid == 0 && *reinterpret_cast<volatile int *>(abort_flag)) {
     atomicOr(a.err, RQ_DEVERR_TIMEOUT);
     // let copies still in flight land before the CTA's shared memory goes
-    for (int s = 0; s < NST; ++s) {
-      for (int64_t i = s; i < n; i += NST) {
-        if (!mbar_try_wait(smem_addr(&full[s]), (uint32_t)((i / NST) & 1))) {
-          mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((i / NST) & 1));
+    mbar_wait_bounded(smem_addr(tbar), 0u);
+    for (int s2 = 0; s2 < NST; ++s2) {
+      for (int i = s2; i < n; i += NST) {
+        if (!mbar_try_wait(smem_addr(&full[s2]), (uint32_t)((i / NST) & 1))) {
+          mbar_wait_bounded(smem_addr(&full[s2]), (uint32_t)((i / NST) & 1));
           break;
         }
       }
@@ -307,6 +409,7 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(
     float *am_val, int *am_idx, unsigned *counter, int32_t *argmax) {
   __shared__ ArgBest scratch[8];
   __shared__ bool last;
+  griddep_wait();   // the partial sums come from the kernel before this one
   const int b = blockIdx.y;
   ArgBest best{-FLT_MAX, INT_MAX};
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -411,22 +514,23 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Variant {
-  int TB, KT, NST;
+  int TB, KT, NST, FMT;
   const void *fn;
-  size_t table_bytes_max;   // PC*K*TB*4 at the largest K served
 };
 
-#define RQ_CHUNK_VARIANT(TB, KT, NST)                                              \
-  Variant {                                                                        \
-    TB, KT, NST, reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, NST>), \
-        (size_t)ChunkShape<TB>::PC * 1024 * TB * 4                                 \
+#define RQ_CHUNK_VARIANT(TB, KT, NST, FMT)                                          \
+  Variant {                                                                         \
+    TB, KT, NST, FMT,                                                               \
+        reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, NST, FMT>)  \
   }
 
 // 128 KB table chunk + NST stages (3 x 32 KB or 5 x 16 KB) per CTA, one CTA
 // per SM.  K = 1024 has its own instances (table offsets as immediates).
 const Variant kVariants[] = {
-    RQ_CHUNK_VARIANT(1, 1024, 3), RQ_CHUNK_VARIANT(2, 1024, 3), RQ_CHUNK_VARIANT(4, 1024, 5),
-    RQ_CHUNK_VARIANT(1, 0, 3),    RQ_CHUNK_VARIANT(2, 0, 3),    RQ_CHUNK_VARIANT(4, 0, 5),
+    RQ_CHUNK_VARIANT(1, 1024, 3, RQ_CODES_U16), RQ_CHUNK_VARIANT(2, 1024, 3, RQ_CODES_U16),
+    RQ_CHUNK_VARIANT(4, 1024, 5, RQ_CODES_U16), RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_U16),
+    RQ_CHUNK_VARIANT(2, 0, 3, RQ_CODES_U16),    RQ_CHUNK_VARIANT(4, 0, 5, RQ_CODES_U16),
+    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_SCHED),  RQ_CHUNK_VARIANT(2, 0, 3, RQ_CODES_SCHED),
 };
 
 int variant_pc(const Variant &v) {
@@ -441,7 +545,8 @@ int variant_stage(const Variant &v) {
 }
 
 size_t variant_smem(const Variant &v, int K) {
-  return 1024 + (size_t)align_up((int64_t)variant_pc(v) * K * v.TB * 4, 1024) +
+  const int KS = v.FMT == RQ_CODES_SCHED ? 1024 : K;
+  return 1024 + (size_t)align_up((int64_t)variant_pc(v) * KS * v.TB * 4, 1024) +
          (size_t)v.NST * variant_stage(v) + 1024;
 }
 
@@ -450,12 +555,15 @@ size_t variant_smem(const Variant &v, int K) {
 ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di) {
   ChunkPlan cp{};
   cp.ok = false;
-  if (fmt != RQ_CODES_U16 || B < 1 || B > 4 || P % 8 != 0 || K > 1024) return cp;
+  if ((fmt != RQ_CODES_U16 && fmt != RQ_CODES_SCHED) || B < 1 || B > 4 || P % 8 != 0 ||
+      K > 1024)
+    return cp;
+  if (fmt == RQ_CODES_SCHED && P % 32 != 0) return cp;
   if (V > (int64_t)INT_MAX - 2048) return cp;
   const int TB = rq_lut_token_stride(B);
   for (int i = 0; i < (int)(sizeof(kVariants) / sizeof(kVariants[0])); ++i) {
     const Variant &v = kVariants[i];
-    if (v.TB != TB) continue;
+    if (v.TB != TB || v.FMT != fmt) continue;
     if (v.KT != 0 && v.KT != K) continue;
     const size_t smem = variant_smem(v, K);
     if (smem > (size_t)di.max_smem_optin) continue;
@@ -477,14 +585,15 @@ size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V) {
 
 cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
                                 int P, int K, int B, const float *lut, float *partial,
-                                unsigned *counter, const DevInfo &di, cudaStream_t s) {
-  (void)fmt;
+                                unsigned *counter, bool pdl, const DevInfo &di, cudaStream_t s) {
   const Variant &var = kVariants[cp.variant];
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
   const int rowb = cp.PC * 2;
-  const cuuint64_t gdim[2] = {(cuuint64_t)P, (cuuint64_t)V};
-  const cuuint64_t gstride[1] = {(cuuint64_t)P * 2};
+  // [V][P] for plain codes; the scheduled layout is chunk-major [P/32][V][32]
+  const bool cm = fmt == RQ_CODES_SCHED;
+  const cuuint64_t gdim[2] = {(cuuint64_t)(cm ? 32 : P), (cuuint64_t)(cm ? (int64_t)V * (P / 32) : V)};
+  const cuuint64_t gstride[1] = {(cuuint64_t)(cm ? 64 : P * 2)};
   const cuuint32_t box[2] = {(cuuint32_t)cp.PC, 256u};
   const cuuint32_t estride[2] = {1u, 1u};
   const CUtensorMapSwizzle swz = rowb == 64   ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -521,15 +630,16 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   a.err = di.err;
   const int64_t grid = (int64_t)cp.nch * cpc;
   void *args[] = {&tmap, &a};
-  return cudaLaunchKernel(var.fn, dim3((unsigned)grid), dim3(1024), args, cp.smem, s);
+  return launch_maybe_pdl(var.fn, dim3((unsigned)grid), dim3(1024), cp.smem, s, args, pdl);
 }
 
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
                                    float *logits, float *am_val, int *am_idx, int nblk,
-                                   unsigned *counter, int32_t *argmax, cudaStream_t s) {
-  reduce_partials_kernel<<<dim3((unsigned)nblk, (unsigned)B), 256, 0, s>>>(
-      partial, nch, B, V, cap, logits, am_val, am_idx, counter, argmax);
-  return cudaGetLastError();
+                                   unsigned *counter, int32_t *argmax, bool pdl,
+                                   cudaStream_t s) {
+  void *args[] = {&partial, &nch, &B, &V, &cap, &logits, &am_val, &am_idx, &counter, &argmax};
+  return launch_maybe_pdl(reinterpret_cast<const void *>(&reduce_partials_kernel),
+                          dim3((unsigned)nblk, (unsigned)B), dim3(256), 0, s, args, pdl);
 }
 
 cudaError_t launch_argmax_finalize(const float *am_val, const int *am_idx, int nblk, int B,

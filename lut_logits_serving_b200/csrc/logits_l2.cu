@@ -88,6 +88,27 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
           add_vec<VW>(tg + ((size_t)(2 * k + 1) * K + c1) * Bs, acc);
         }
       }
+    } else if (FMT == RQ_CODES_SCHED) {
+      // chunk-major [P/32][V][32]; groups of 16 entries (i << 12 | c << 2),
+      // any order within the group
+      const uint16_t *cbase = static_cast<const uint16_t *>(a.codes) + v * 32;
+      const int ng = a.P / 16;
+      for (int g = 0; g < ng; ++g) {
+        const float *tg = tl + (size_t)(16 * g) * K * Bs;
+        const uint4 *crow =
+            reinterpret_cast<const uint4 *>(cbase + (size_t)(g >> 1) * a.V * 32 + (g & 1) * 16);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint4 w = __ldg(crow + half);
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t e = (k & 1) ? (ws[k >> 1] >> 16) : (ws[k >> 1] & 0xFFFFu);
+            const uint32_t c = (e >> 2) & 0x3FFu;
+            if (c < (uint32_t)K) add_vec<VW>(tg + ((size_t)(e >> 12) * K + c) * Bs, acc);
+          }
+        }
+      }
     } else {
       // 64 codes = 640 bits = 5 x 16 bytes per group; rows are 16-byte aligned
       const int64_t rb = (int64_t)a.P / 64 * 80;
@@ -158,6 +179,14 @@ __global__ void __launch_bounds__(256) logits_generic_kernel(const L2Args a, int
     const uint8_t *c8 = static_cast<const uint8_t *>(a.codes) + v * rb;
     float z = 0.f;
     for (int p = 0; p < a.P; ++p) {
+      if (fmt == RQ_CODES_SCHED) {
+        const uint32_t e =
+            static_cast<const uint16_t *>(a.codes)[((size_t)(p >> 5) * a.V + v) * 32 + (p & 31)];
+        const uint32_t c = (e >> 2) & 0x3FFu;
+        const int pp = (p & ~15) + (int)(e >> 12);
+        if (c < (uint32_t)a.K) z += __ldg(tl + ((size_t)pp * a.K + c) * a.Bs);
+        continue;
+      }
       const uint32_t c = a.fix(fmt == RQ_CODES_U16 ? (uint32_t)c16[p] : packed10_code(c8, p));
       z += __ldg(tl + ((size_t)p * a.K + c) * a.Bs);
     }
@@ -217,7 +246,9 @@ cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K
   a.am_idx = am_idx;
   a.fix = make_codefix(K);
   const bool codes16 = (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
-  const bool fast_fmt = fmt == RQ_CODES_U16 ? (P % 8 == 0) : (P % 64 == 0);
+  const bool fast_fmt = fmt == RQ_CODES_U16     ? (P % 8 == 0)
+                        : fmt == RQ_CODES_SCHED ? (P % 32 == 0)
+                                                : (P % 64 == 0);
   int VW;
   if (Bs == 1) VW = 1;
   else if (Bs == 2) VW = 2;
@@ -234,12 +265,17 @@ cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K
     while (G < need) G <<= 1;
   }
   if (fmt == RQ_CODES_U16) {
-    if (VW == 1) return launch_vw<1, RQ_CODES_U16>(a, 1, nblk, s);
-    if (VW == 2) return launch_vw<2, RQ_CODES_U16>(a, 1, nblk, s);
+    if (VW == 1) return launch_fast<1, 1, RQ_CODES_U16>(a, nblk, s);
+    if (VW == 2) return launch_fast<2, 1, RQ_CODES_U16>(a, nblk, s);
     return launch_vw<4, RQ_CODES_U16>(a, G, nblk, s);
   }
-  if (VW == 1) return launch_vw<1, RQ_CODES_PACKED10>(a, 1, nblk, s);
-  if (VW == 2) return launch_vw<2, RQ_CODES_PACKED10>(a, 1, nblk, s);
+  if (fmt == RQ_CODES_SCHED) {
+    if (VW == 1) return launch_fast<1, 1, RQ_CODES_SCHED>(a, nblk, s);
+    if (VW == 2) return launch_fast<2, 1, RQ_CODES_SCHED>(a, nblk, s);
+    return launch_vw<4, RQ_CODES_SCHED>(a, G, nblk, s);
+  }
+  if (VW == 1) return launch_fast<1, 1, RQ_CODES_PACKED10>(a, nblk, s);
+  if (VW == 2) return launch_fast<2, 1, RQ_CODES_PACKED10>(a, nblk, s);
   return launch_vw<4, RQ_CODES_PACKED10>(a, G, nblk, s);
 }
 

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(256) lut_build_ds6_kernel(const float *__restr
                                                            const float *__restrict__ C, int b0,
                                                            int nb, int D, int L, int K, int Bs,
                                                            int64_t quads, float *__restrict__ lut) {
+  griddep_launch_dependents();             // the next kernel may start its prologue
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= quads) return;
   const int64_t e0 = 4 * g;                 // first codeword (p*K + k) of this thread

@@ -118,6 +118,36 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+// 2-D tiled TMA prefetch of a box into L2 only (no shared memory written),
+// normal L2 priority.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory (16-byte aligned, size a
+// multiple of 16), completing on an mbarrier.  No multicast.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Programmatic dependent launch: wait for the previous kernel of the stream
+// (a no-op when this kernel was launched without the attribute) / allow the
+// next one to start its prologue.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -157,6 +187,25 @@ __device__ __forceinline__ ArgBest arg_shfl_xor(ArgBest a, int lane_mask) {
 // Launchers implemented by the kernel translation units (host side).
 namespace rq {
 
+// cudaLaunchKernel, or with programmatic stream serialization when `pdl`:
+// the kernel may start while the previous one in the stream drains and
+// must call griddep_wait() before reading that kernel's outputs.
+inline cudaError_t launch_maybe_pdl(const void *fn, dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t s, void **args, bool pdl) {
+  if (!pdl) return cudaLaunchKernel(fn, grid, block, args, smem, s);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 struct DevInfo {
   int device;
   int sms;
@@ -176,6 +225,9 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
 cudaError_t launch_pack10(const uint16_t *codes, int64_t V, int P, uint8_t *packed,
                           cudaStream_t s);
 
+cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, uint16_t *out,
+                                 unsigned long long *stats, cudaStream_t s);
+
 // Vocabulary-tiled pass with the LUT chunk resident in shared memory.
 struct ChunkPlan {
   bool ok;      // this path applies
@@ -190,12 +242,13 @@ ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di)
 size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V);
 cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
                                 int P, int K, int B, const float *lut, float *partial,
-                                unsigned *counter, const DevInfo &di, cudaStream_t s);
+                                unsigned *counter, bool pdl, const DevInfo &di, cudaStream_t s);
 // Sums the chunk partials, softcap, logits; with `argmax` set also the
 // argmax (block partials in am_val/am_idx, finished by the last block).
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
                                    float *logits, float *am_val, int *am_idx, int nblk,
-                                   unsigned *counter, int32_t *argmax, cudaStream_t s);
+                                   unsigned *counter, int32_t *argmax, bool pdl,
+                                   cudaStream_t s);
 
 // Batched pass with the LUT read through L2 (token groups of <= 32).
 cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K,

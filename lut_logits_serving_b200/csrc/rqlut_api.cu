@@ -79,9 +79,14 @@ bool dims_ok(const rq_dims &d) {
   return true;
 }
 
+bool fmt_known(int fmt) {
+  return fmt == RQ_CODES_U16 || fmt == RQ_CODES_PACKED10 || fmt == RQ_CODES_SCHED;
+}
+
 bool fmt_ok(const rq_dims &d, int fmt) {
   if (fmt == RQ_CODES_U16) return true;
   if (fmt == RQ_CODES_PACKED10) return d.K <= 1024;
+  if (fmt == RQ_CODES_SCHED) return d.K <= 1024 && ((int64_t)d.M * d.L) % 32 == 0;
   return false;
 }
 
@@ -138,9 +143,11 @@ int sweep_blocks(const rq_dims &d, const DevInfo &di, bool chunk) {
 }
 
 // Path shared by rq_lut_logits and rq_logits_from_hidden.
+// `after_build`: the kernel just before is this library's table build (which
+// writes nothing the code stream reads), so the tiled pass may overlap it.
 int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, int B, int Bs,
                float cap, float *logits, int32_t *argmax, unsigned char *ws,
-               const WsLayout &w, const DevInfo &di, cudaStream_t s) {
+               const WsLayout &w, const DevInfo &di, cudaStream_t s, bool after_build) {
   const int P = d.M * d.L;
   float *amv = argmax ? reinterpret_cast<float *>(ws + w.amv_off) : nullptr;
   int *ami = argmax ? reinterpret_cast<int *>(ws + w.ami_off) : nullptr;
@@ -150,11 +157,13 @@ int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, i
     float *partial = reinterpret_cast<float *>(ws + w.partial_off);
     unsigned *counter = argmax ? reinterpret_cast<unsigned *>(ws + w.counter_off) : nullptr;
     if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
-    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, counter, di, s);
+    const bool prof = t_prof_start != nullptr;   // events between kernels break the overlap
+    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, counter,
+                            after_build && !prof, di, s);
     if (e != cudaSuccess) return status_of(e);
     if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
     e = launch_reduce_partials(partial, w.cp.nch, B, d.V, cap, logits, amv, ami, nblk, counter,
-                               argmax, s);
+                               argmax, !prof, s);
     return status_of(e);
   } else {
     if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
@@ -194,7 +203,7 @@ int rq_version(void) { return 100; }
 size_t rq_codes_bytes(rq_dims d, int fmt) {
   if (!dims_ok(d) || !fmt_ok(d, fmt)) return 0;
   const int64_t P = (int64_t)d.M * d.L;
-  if (fmt == RQ_CODES_U16) return (size_t)(d.V * P * 2);
+  if (fmt == RQ_CODES_U16 || fmt == RQ_CODES_SCHED) return (size_t)(d.V * P * 2);
   return (size_t)(d.V * ((10 * P + 7) / 8));
 }
 
@@ -236,7 +245,7 @@ int rq_lut_logits(const void *codes, int fmt, rq_dims d, const float *lut, int B
                   float *logits, int32_t *argmax, void *ws, size_t ws_bytes, void *stream) {
   if (!codes || !lut || B < 1 || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
   if (!logits && !argmax) return RQ_ERR_INVALID_ARGUMENT;
-  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_known(fmt)) return RQ_ERR_INVALID_ARGUMENT;
   if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
   if (!aligned(codes, 16) || !aligned(lut, 16) || (ws && !aligned(ws, 16)) ||
       (logits && !aligned(logits, 4)) || (argmax && !aligned(argmax, 4)))
@@ -246,7 +255,8 @@ int rq_lut_logits(const void *codes, int fmt, rq_dims d, const float *lut, int B
   const WsLayout w = ws_layout(d, B, fmt, argmax != nullptr, di);
   if (w.total > 0 && (!ws || ws_bytes < w.total)) return RQ_ERR_WORKSPACE_TOO_SMALL;
   return run_logits(codes, fmt, d, lut, B, rq_lut_token_stride(B), softcap, logits, argmax,
-                    static_cast<unsigned char *>(ws), w, di, static_cast<cudaStream_t>(stream));
+                    static_cast<unsigned char *>(ws), w, di, static_cast<cudaStream_t>(stream),
+                    false);
 }
 
 int rq_logits_from_hidden(const float *h, const float *C, const void *codes, int fmt, rq_dims d,
@@ -254,7 +264,7 @@ int rq_logits_from_hidden(const float *h, const float *C, const void *codes, int
                           size_t ws_bytes, void *stream) {
   if (!h || !C || !codes || B < 1 || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
   if (!logits && !argmax) return RQ_ERR_INVALID_ARGUMENT;
-  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_known(fmt)) return RQ_ERR_INVALID_ARGUMENT;
   if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
   if (!ws) return RQ_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned(h, 4) || !aligned(C, 4) || !aligned(codes, 16) || !aligned(ws, 16) ||
@@ -275,7 +285,7 @@ int rq_logits_from_hidden(const float *h, const float *C, const void *codes, int
     // B <= 4: one table for all tokens, then the vocabulary-tiled pass
     cudaError_t e = launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut, s);
     if (e != cudaSuccess) return status_of(e);
-    return run_logits(codes, fmt, d, lut, B, Bs, softcap, logits, argmax, rest, w, di, s);
+    return run_logits(codes, fmt, d, lut, B, Bs, softcap, logits, argmax, rest, w, di, s, true);
   }
   const int P = d.M * d.L;
   float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
@@ -300,7 +310,7 @@ int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt, co
   if (N < 0 || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
   if (N == 0) return RQ_OK;
   if (!ids || !codes || !C || !out) return RQ_ERR_INVALID_ARGUMENT;
-  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_known(fmt)) return RQ_ERR_INVALID_ARGUMENT;
   if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
   if (!aligned(ids, 4) || !aligned(codes, 2) || !aligned(C, 4) || !aligned(out, 2))
     return RQ_ERR_MISALIGNED;
@@ -315,6 +325,20 @@ int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed, void *strea
   if (!aligned(codes_u16, 2)) return RQ_ERR_MISALIGNED;
   return status_of(
       launch_pack10(codes_u16, d.V, d.M * d.L, packed, static_cast<cudaStream_t>(stream)));
+}
+
+int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out, uint64_t *stats,
+                     void *stream) {
+  if (!codes_u16 || !out || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_ok(d, RQ_CODES_SCHED)) return RQ_ERR_UNSUPPORTED;
+  if (!aligned(codes_u16, 2) || !aligned(out, 2) || (stats && !aligned(stats, 8)))
+    return RQ_ERR_MISALIGNED;
+  const size_t bytes = rq_codes_bytes(d, RQ_CODES_U16);
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(codes_u16), b0 = reinterpret_cast<uintptr_t>(out);
+  if (a0 < b0 + bytes && b0 < a0 + bytes) return RQ_ERR_INVALID_ARGUMENT;   // overlap
+  return status_of(launch_prepare_sched(codes_u16, d.V, d.M * d.L, out,
+                                        reinterpret_cast<unsigned long long *>(stats),
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 int rq_set_profile_events(void *start, void *stop) {

@@ -57,6 +57,7 @@ def test_code_and_lut_sizes():
     # u16 codes [V][M*L]: 393.216 MB; packed 10-bit rows of 960 bytes
     assert rq.rq_codes_bytes(G2, rq.U16) == 256000 * 768 * 2
     assert rq.rq_codes_bytes(G2, rq.PACKED10) == 256000 * 960
+    assert rq.rq_codes_bytes(G2, rq.SCHED) == 256000 * 768 * 2
     assert rq.rq_codes_bytes(TINY, rq.PACKED10) == 4096 * 80
     assert rq.rq_codes_bytes(rq.dims(10, 3, 1, 1, 1024), rq.PACKED10) == 10 * 2   # ceil(10/8)
     assert rq.rq_codes_bytes(rq.dims(10, 3, 1, 1, 2048), rq.PACKED10) == 0       # K > 1024
@@ -119,6 +120,11 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_decode_rows(null, 0, null, 0, null, G2, 48.0, null, s) == 0   # N = 0: no-op
     assert lib.rq_decode_rows(_fake(0x10002), 5, a, 0, a, G2, 48.0, a, s) == MIS
     assert lib.rq_pack10(null, G2, a, s) == INV
+    assert lib.rq_prepare_sched(null, G2, a, null, s) == INV
+    assert lib.rq_prepare_sched(a, rq.dims(10, 48, 24, 1, 64), _fake(0x900000), null, s) == UNS
+    assert lib.rq_prepare_sched(a, G2, _fake(0x10000 + 64), null, s) == INV    # overlap
+    assert lib.rq_lut_logits(a, 2, rq.dims(10, 48, 24, 1, 64), a, 1, 30.0, a, null, null, 0,
+                             s) == UNS                                        # sched, P % 32
     assert lib.rq_device_error(None, 0) == INV
 
 

@@ -58,6 +58,13 @@ def test_g2_batch1_full_sweep(g2):
     _, am2, _ = rq.rq_logits_from_hidden(dev(h), g2["dC"], g2["dc"], rq.U16, d, w.softcap,
                                          want_logits=False, want_argmax=True)
     assert int(am2.cpu()[0]) == int(am.cpu()[0])
+    # the bank-scheduled layout: same logits up to summation order
+    sched = rq.rq_prepare_sched(g2["dc"], d)
+    logits3, am3, _ = rq.rq_logits_from_hidden(dev(h), g2["dC"], sched, rq.SCHED, d, w.softcap,
+                                               want_argmax=True)
+    err3 = assert_logits_close(logits3.cpu().numpy(), ref)
+    print(f"g2_b1 sched normwise error {err3:.3g}")
+    assert check_argmax(am3.cpu().numpy(), ref) == 0
     assert rq.rq_device_error() == 0
 
 
@@ -99,11 +106,12 @@ def test_g2_packed_batch64_fused_argmax(g2):
     assert ties == 0
 
 
-@pytest.mark.parametrize("fmt", [0, 1], ids=["u16", "packed10"])
+@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["u16", "packed10", "sched"])
 def test_decode512_bit_exact(g2, fmt):
     w = synth.WORKLOADS["decode512"]
     ids = synth.zipf_ids(w.n_ids, w.V, w.zipf_s, 3)
-    codes_dev = g2["dc"] if fmt == rq.U16 else rq.rq_pack10(g2["dc"], g2["d"])
+    codes_dev = {0: lambda: g2["dc"], 1: lambda: rq.rq_pack10(g2["dc"], g2["d"]),
+                 2: lambda: rq.rq_prepare_sched(g2["dc"], g2["d"])}[fmt]()
     out = rq.rq_decode_rows(dev(ids), codes_dev, fmt, g2["dC"], g2["d"], w.decode_scale)
     got = out.view(torch.int16).cpu().numpy().view(np.uint16)
     want = oracle.decode_rows_bf16(ids, g2["codes"], g2["C"], w.decode_scale)

@@ -36,7 +36,17 @@ def gpu_codes(codes, fmt, d):
     c16 = dev(codes.reshape(codes.shape[0], -1))
     if fmt == rq.U16:
         return c16
+    if fmt == rq.SCHED:
+        return rq.rq_prepare_sched(c16, d)
     return rq.rq_pack10(c16, d)
+
+
+def fmt_applies(fmt, M, L, K):
+    if fmt == rq.PACKED10:
+        return K <= 1024
+    if fmt == rq.SCHED:
+        return K <= 1024 and (M * L) % 32 == 0
+    return True
 
 
 # ------------------------------------------------------------- lut build
@@ -74,11 +84,11 @@ CASES = [
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "V%d_D%d_M%d_L%d_K%d" % c)
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 13, 32, 33])
-@pytest.mark.parametrize("fmt", [0, 1], ids=["u16", "packed10"])
+@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["u16", "packed10", "sched"])
 def test_logits_and_argmax(case, B, fmt):
     V, D, M, L, K = case
-    if fmt == rq.PACKED10 and K > 1024:
-        pytest.skip("packed codes hold K <= 1024")
+    if not fmt_applies(fmt, M, L, K):
+        pytest.skip("format does not hold this shape")
     C, codes, h = make_case(V, D, M, L, K, B, seed=V + B)
     d = rq.dims(V, D, M, L, K)
     cap = 30.0
@@ -130,12 +140,12 @@ def test_softcap_off_gives_raw_sums():
 def test_single_codeword_ties_go_to_index_zero():
     """K = 1: every row is the same vector, all logits are bit-identical and
     the argmax is row 0 on every path."""
-    V, D, M, L, K = 3000, 48, 8, 2, 1
+    V, D, M, L, K = 3000, 96, 16, 2, 1
     for B in (1, 3, 8):
         C, codes, h = make_case(V, D, M, L, K, B)
         d = rq.dims(V, D, M, L, K)
         lut = rq.rq_lut_build(dev(h), dev(C), d)
-        for fmt in (0, 1):
+        for fmt in (0, 1, 2):
             logits, am, _ = rq.rq_lut_logits(gpu_codes(codes, fmt, d), fmt, d, lut, B, 30.0,
                                              want_argmax=True)
             lg = logits.cpu().numpy()
@@ -146,7 +156,7 @@ def test_single_codeword_ties_go_to_index_zero():
 def test_planted_maximum_is_found_at_every_position():
     """One row holds a unique maximum; the argmax must find it wherever it
     sits (first row, last row, tile and chunk boundaries)."""
-    V, D, M, L, K, B = 5000, 48, 8, 2, 16, 1
+    V, D, M, L, K, B = 5000, 96, 16, 2, 16, 1
     rng = np.random.default_rng(1)
     C = synth.codebooks(M, L, K, D // M, (0.05, 0.01), 0)
     h = synth.hidden(1, D, 1.0, 2)
@@ -159,7 +169,7 @@ def test_planted_maximum_is_found_at_every_position():
         codes = np.broadcast_to(worst, (V, M, L)).copy().astype(np.uint16)
         codes[rng.integers(0, V, 50)] = rng.integers(0, K, (50, M, L))
         codes[pos] = best
-        for fmt in (0, 1):
+        for fmt in (0, 1, 2):
             _, am, _ = rq.rq_lut_logits(gpu_codes(codes, fmt, d), fmt, d, lut, B, 30.0,
                                         want_logits=False, want_argmax=True)
             assert int(am.cpu()[0]) == pos
@@ -182,11 +192,13 @@ def test_out_of_range_codes_stay_in_bounds():
 
 # ------------------------------------------------------------ row decode
 
-@pytest.mark.parametrize("fmt", [0, 1], ids=["u16", "packed10"])
+@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["u16", "packed10", "sched"])
 @pytest.mark.parametrize("shape", [(4096, 192, 32, 2, 256), (5000, 288, 48, 2, 1024),
                                    (300, 96, 16, 3, 100), (50, 9, 3, 1, 7)])
 def test_decode_rows_bit_exact(shape, fmt):
     V, D, M, L, K = shape
+    if not fmt_applies(fmt, M, L, K):
+        pytest.skip("format does not hold this shape")
     C, codes, _ = make_case(V, D, M, L, K, 1, sigmas=(0.02, 0.005))
     ids = synth.zipf_ids(257, V, 1.1, 3)
     d = rq.dims(V, D, M, L, K)
@@ -229,3 +241,61 @@ def test_pack10_matches_oracle(P):
     d = rq.dims(V, 8 * M, M, L, 1024)
     got = rq.rq_pack10(dev(codes.reshape(V, -1)), d).cpu().numpy()
     assert np.array_equal(got, oracle.pack10(codes))
+
+
+# ------------------------------------------------------ scheduled codes
+
+@pytest.mark.parametrize("shape", [(4096, 192, 32, 2, 256), (1000, 96, 16, 2, 1024),
+                                   (77, 96, 32, 1, 64), (3000, 288, 48, 2, 1024)])
+def test_prepare_sched_is_a_permutation_within_groups(shape):
+    """Chunk-major [P/32][V][32]; every group of 16 entries of every row
+    holds exactly the group's 16 (position, code) pairs, each once, in the
+    (i << 12 | c << 2) encoding."""
+    V, D, M, L, K = shape
+    codes = synth.codes(V, M, L, K, 4)
+    d = rq.dims(V, D, M, L, K)
+    P = M * L
+    out, (steps, passes) = rq.rq_prepare_sched(dev(codes.reshape(V, -1)), d, stats=True)
+    raw = out.view(torch.int16).cpu().numpy().view(np.uint16).astype(np.int64)
+    assert raw.size == V * P
+    e = raw.reshape(P // 32, V, 32).transpose(1, 0, 2).reshape(V, P // 16, 16)
+    assert np.all(e & 3 == 0)
+    pos = e >> 12
+    code = (e >> 2) & 1023
+    order = np.argsort(pos, axis=2, kind="stable")
+    assert np.array_equal(np.take_along_axis(pos, order, 2),
+                          np.broadcast_to(np.arange(16), pos.shape))
+    assert np.array_equal(np.take_along_axis(code, order, 2), codes.reshape(V, P // 16, 16))
+    assert steps == 16 * ((V + 15) // 16) * ((P + 31) // 32)
+    assert passes >= steps
+
+
+def test_prepare_sched_quality_on_random_codes():
+    """Random codes cost ~3.5 shared-memory passes per lookup step in their
+    natural order; the schedule must bring the average below 2."""
+    V, D, M, L, K = 20000, 2304, 384, 2, 1024
+    codes = synth.codes(V, M, L, K, 1)
+    d = rq.dims(V, D, M, L, K)
+    _, (steps, passes) = rq.rq_prepare_sched(dev(codes.reshape(V, -1)), d, stats=True)
+    flat = codes.reshape(V, -1)
+    # a warp's step k: 16 rows x groups 2c and 2c+1 of chunk c, code k of each
+    natural = np.mean([np.bincount(np.concatenate([flat[r:r + 16, (2 * c) * 16 + k],
+                                                   flat[r:r + 16, (2 * c + 1) * 16 + k]]) & 31,
+                                   minlength=32).max()
+                       for r in range(0, 2000, 16) for c in range(4) for k in range(16)])
+    print(f"bank passes per step: natural order {natural:.2f}, scheduled {passes / steps:.2f}")
+    assert passes / steps < 2.0
+    assert natural > 2.5
+
+
+def test_prepare_sched_rejects_unsupported_shapes():
+    d = rq.dims(100, 48, 24, 1, 1024)          # M*L = 24: not a multiple of 32
+    c = torch.zeros((100, 24), dtype=torch.uint16, device="cuda")
+    with pytest.raises(rq.RqError):
+        rq.rq_prepare_sched(c, d)
+    d2 = rq.dims(100, 64, 32, 1, 2048)         # K > 1024
+    c2 = torch.zeros((100, 32), dtype=torch.uint16, device="cuda")
+    with pytest.raises(rq.RqError):
+        rq.rq_prepare_sched(c2, d2)
+    with pytest.raises(rq.RqError):            # in place is refused
+        rq.rq_prepare_sched(c2, rq.dims(100, 64, 32, 1, 1024), out=c2)
