@@ -229,6 +229,32 @@ RQ_API int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out,
 RQ_API int rq_device_error(uint32_t *out, int clear);
 
 /*
+ * rq_lut_logits_static -- rq_lut_logits without a caller-provided workspace,
+ * for callers that cannot allocate device memory: work being recorded into
+ * a CUDA graph (allocation is not allowed during capture), processes whose
+ * device memory belongs to another runtime's allocator, and loops that must
+ * not allocate once serving has started.  The paper has no counterpart; this
+ * is a convenience of this library.
+ *   Arguments, results and errors are those of rq_lut_logits, without ws and
+ *   ws_bytes.  The workspace comes from a fixed device array inside the
+ *   library, RQ_STATIC_SCRATCH_BYTES on every GPU that loads it, held until
+ *   the process exits; a call whose workspace (rq_logits_workspace_bytes)
+ *   would exceed it returns RQ_ERR_WORKSPACE_TOO_SMALL and launches nothing.
+ *   At the Gemma-2 shape this covers batch 1 (24.6 MB), not batch 2 (98 MB)
+ *   of the B <= 4 pass; batches > 4 need only kilobytes.
+ *   The first call on a device looks the array's address up (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.  All calls on a device share the one array: calls that
+ *   may run at the same time on the GPU (different streams without an
+ *   ordering between them) race on it and must be serialized by the caller.
+ *   Nothing in it needs to start at zero; the kernels reset what they use.
+ */
+#define RQ_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+RQ_API int rq_lut_logits_static(const void *codes, int fmt, rq_dims d, const float *lut,
+                                 int B, float softcap, float *logits, int32_t *argmax,
+                                 void *stream);
+
+/*
  * rq_set_profile_events -- optional timing hook for benchmarks.  With both
  * arguments non-NULL (cudaEvent_t handles passed as void*), each later
  * rq_lut_logits / rq_logits_from_hidden call made from this host thread

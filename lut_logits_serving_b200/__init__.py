@@ -25,7 +25,7 @@ __all__ = [
     "rq_status_string", "rq_version", "rq_codes_bytes", "rq_lut_token_stride",
     "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
     "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
-    "rq_pack10", "rq_device_error", "rq_set_profile_events",
+    "rq_pack10", "rq_device_error", "rq_set_profile_events", "rq_lut_logits_static",
 ]
 
 U16 = 0
@@ -76,6 +76,7 @@ _SIGNATURES = {
     "rq_device_error": (_i, [ctypes.POINTER(ctypes.c_uint32), _i]),
     "rq_set_profile_events": (_i, [_p, _p]),
     "rq_prepare_sched": (_i, [_p, RqDims, _p, _p, _p]),
+    "rq_lut_logits_static": (_i, [_p, _i, RqDims, _p, _i, _f, _p, _p, _p]),
 }
 
 
@@ -286,3 +287,21 @@ def rq_prepare_sched(codes_u16, d: RqDims, out=None, stats=None, stream=None):
         v = st.cpu().tolist()
         return out, (v[0], v[1])
     return out
+
+
+def rq_lut_logits_static(codes, fmt: int, d: RqDims, lut, B: int, softcap: float = 30.0,
+                         want_logits: bool = True, want_argmax: bool = False, logits=None,
+                         argmax=None, stream=None):
+    """rq_lut_logits with the library's fixed device scratch as workspace
+    (for callers that cannot allocate; see include/rqlut.h).
+    Returns (logits or None, argmax or None)."""
+    torch = _torch()
+    if want_logits and logits is None:
+        logits = _empty((B, d.V), torch.float32, lut)
+    if want_argmax and argmax is None:
+        argmax = _empty((B,), torch.int32, lut)
+    _check("rq_lut_logits_static", lib().rq_lut_logits_static(
+        _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, _cuda(lut, torch.float32, "lut"), B,
+        float(softcap), _ptr_or_null(logits, torch.float32, "logits"),
+        _ptr_or_null(argmax, torch.int32, "argmax"), _stream(stream)))
+    return logits, argmax
