@@ -20,7 +20,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import subprocess
 import sys
@@ -44,9 +43,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="g2_b1", choices=["g2_b1", "g2_b32", "packed_b64"])
-    ap.add_argument("--codes", default="u16", choices=["u16", "sched"],
-                    help="uint16 code layout of the unpacked workloads: as drawn, or "
-                         "bank-scheduled once by rq_prepare_sched")
+    ap.add_argument("--codes", default="sched", choices=["u16", "sched"],
+                    help="uint16 code layout of the unpacked workloads timed for `value`: "
+                         "bank-scheduled once by rq_prepare_sched (the serving layout), or as "
+                         "drawn; the other layout is reported under other_layouts")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -242,98 +242,127 @@ def run_ours(args, w):
         if world > 1:
             dist.barrier()
 
+    def max_over_ranks(x):
+        if world > 1:
+            t = torch.tensor([x], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+        return x
+
     data = synth.make(w, seed=1000 * rank)
     d = rq.dims(w.V, w.D, w.M, w.L, w.K)
-    fmt = rq.PACKED10 if w.packed10 else (rq.SCHED if args.codes == "sched" else rq.U16)
     dC = torch.from_numpy(data["C"]).cuda()
     c16 = torch.from_numpy(data["codes"].reshape(w.V, -1)).cuda()
-    sched_quality = None
-    if fmt == rq.PACKED10:
-        dcodes = rq.rq_pack10(c16, d)
-        del c16
-    elif fmt == rq.SCHED:
-        dcodes, (st, ps) = rq.rq_prepare_sched(c16, d, stats=True)
-        sched_quality = ps / st
-        del c16
-    else:
-        dcodes = c16
     dh = torch.from_numpy(data["h"]).cuda()
     logits = torch.empty((w.B, w.V), dtype=torch.float32, device="cuda")
     am = torch.empty((w.B,), dtype=torch.int32, device="cuda")
     rows = torch.empty((w.B, w.D), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
-                     device="cuda")
-
-    def step():
-        # logits of this step's hidden states, then the input rows of the
-        # tokens it picked (the next step's embeddings), rebuilt on demand
-        rq.rq_logits_from_hidden(dh, dC, dcodes, fmt, d, w.softcap, logits=logits, argmax=am,
-                                 ws=ws)
-        rq.rq_decode_rows(am, dcodes, fmt, dC, d, w.decode_scale, out=rows)
-
-    # decode + (build, tiled pass, reduce) or (build + pass per token group) + argmax finalize
-    if w.B <= 4:
-        launches_per_step = 1 + 1 + 1 + 1 + 1
-    else:
-        launches_per_step = 1 + 2 * ((w.B + 31) // 32) + 1
-
     stream = torch.cuda.current_stream()
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
 
-    graph = None
-    if not args.no_graph:
+    # code layouts: the artifact is prepared once, outside any timed region
+    layouts = {}
+    if w.packed10:
+        layouts["packed10"] = (rq.PACKED10, rq.rq_pack10(c16, d), None)
+        del c16
+        headline = "packed10"
+    else:
+        sched, (st, ps) = rq.rq_prepare_sched(c16, d, stats=True)
+        layouts["sched"] = (rq.SCHED, sched, ps / st)
+        layouts["u16"] = (rq.U16, c16, None)
+        headline = args.codes
+
+    def make_step(fmt, codes):
+        ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
+                         device="cuda")
+
+        def step():
+            # logits of this step's hidden states, then the input rows of the
+            # tokens it picked (the next step's embeddings), rebuilt on demand
+            rq.rq_logits_from_hidden(dh, dC, codes, fmt, d, w.softcap, logits=logits,
+                                     argmax=am, ws=ws)
+            rq.rq_decode_rows(am, codes, fmt, dC, d, w.decode_scale, out=rows)
+        return step
+
+    def graphed(step):
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        if args.no_graph:
+            return step, None
         s2 = torch.cuda.Stream()
         s2.wait_stream(stream)
         with torch.cuda.stream(s2):
             step()
         stream.wait_stream(s2)
         torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
             step()
         for _ in range(3):
-            graph.replay()
+            g.replay()
         torch.cuda.synchronize()
-    run = graph.replay if graph is not None else step
+        return g.replay, g
+
+    def time_steps(run, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    def code_pass_us(step, n):
+        """Device time of the code-streaming pass alone (profile events
+        recorded by the library around it on the launching stream)."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        stops = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for ev in starts + stops:       # torch creates the CUDA event on first record
+            ev.record(stream)
+        torch.cuda.synchronize()
+        for i in range(n):
+            rq.rq_set_profile_events(starts[i], stops[i])
+            step()
+        rq.rq_set_profile_events(None, None)
+        torch.cuda.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in zip(starts, stops)])) * 1e3
+
+    fmt, dcodes, sched_quality = layouts[headline]
+    step = make_step(fmt, dcodes)
+    run, graph = graphed(step)
 
     # ---- timed region: K steps, device time, max over ranks
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        ev0.record(stream)
-        for _ in range(args.steps):
-            run()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-    t_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([t_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_ms = float(t.item())
+        t_ms = time_steps(run, args.steps)
     sec = t_ms / 1e3
     value = world * w.V * w.B * args.steps / sec
 
-    # ---- the dominant kernel alone (code-streaming pass), live CUDA events
-    nprof = min(args.steps, 2000)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(nprof)]
-    stops = [torch.cuda.Event(enable_timing=True) for _ in range(nprof)]
-    for ev in starts + stops:       # torch creates the CUDA event on first record
-        ev.record(stream)
-    torch.cuda.synchronize()
-    for i in range(nprof):
-        rq.rq_set_profile_events(starts[i], stops[i])
-        step()
-    rq.rq_set_profile_events(None, None)
-    torch.cuda.synchronize()
-    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(starts, stops)]))
+    # ---- the dominant kernel alone, live CUDA events
+    kern_us = code_pass_us(step, min(args.steps, 2000))
     peak, peak_kind = load_peaks()
     algo_bytes = code_bytes(w)
-    achieved = algo_bytes / (kern_ms / 1e3) / 1e9
-    kname = "logits_chunk_u16_kernel" if (w.B <= 4 and not w.packed10) else "logits_l2_kernel"
+    achieved = algo_bytes / (kern_us / 1e6) / 1e9
+    kname = "logits_chunk_u16_kernel" if w.B <= 4 and not w.packed10 else "logits_l2_kernel"
+    kkey = f"{kname}/{headline}/{w.name}"
+
+    # ---- the other layout, same step (context for the headline)
+    others = {}
+    for name, (f2, c2, q2) in layouts.items():
+        if name == headline:
+            continue
+        st2 = make_step(f2, c2)
+        r2, g2 = graphed(st2)
+        n2 = min(args.steps, 3000)
+        t2 = time_steps(r2, n2)
+        k2 = code_pass_us(st2, min(n2, 1000))
+        others[name] = {"us_per_call": t2 / n2 * 1e3, "value": world * w.V * w.B * n2 / (t2 / 1e3),
+                        "code_pass_us": k2,
+                        "code_pass_frac": algo_bytes / (k2 / 1e6) / 1e9 / peak}
+        del g2
+    run, graph = graphed(step)
 
     # ---- end to end through the public API with host buffers
     h_host = torch.from_numpy(data["h"]).pin_memory()
@@ -349,19 +378,7 @@ def run_ours(args, w):
 
     for _ in range(3):
         e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(ne2e):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = time_steps(e2e_step, ne2e)
     e2e_value = world * w.V * w.B * ne2e / (e_ms / 1e3)
     h2d = data["h"].nbytes
     d2h = w.B * w.V * 4 + w.B * 4
@@ -369,6 +386,12 @@ def run_ours(args, w):
     # the argmax must agree with the logits it came from
     assert torch.equal(am.long().cpu(), logits.argmax(dim=1).cpu()), "argmax/logits mismatch"
     assert rq.rq_device_error() == 0
+
+    # decode + (build, tiled pass, reduce) or (build + pass per token group) + argmax finalize
+    if w.B <= 4 and not w.packed10:
+        launches_per_step = 1 + 1 + 1 + 1
+    else:
+        launches_per_step = 1 + 2 * ((w.B + 31) // 32) + 1
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -385,14 +408,15 @@ def run_ours(args, w):
         "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
         "us_per_call": t_ms / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(workload_config(w, args.codes), parallelism=f"replicas x{world}",
+        "config": dict(workload_config(w, headline), parallelism=f"replicas x{world}",
                        launch="cuda graph" if graph is not None else "eager",
                        bank_passes_per_step=sched_quality),
         "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": profiled_traffic(kname), "algorithmic_bytes": algo_bytes,
-                     "kernel_us": kern_ms * 1e3},
-        "step_hbm_frac": code_bytes(w) / (sec / args.steps) / 1e9 / peak,
+                     "traffic": profiled_traffic(kkey), "algorithmic_bytes": algo_bytes,
+                     "kernel_us": kern_us},
+        "step_hbm_frac": algo_bytes / (sec / args.steps) / 1e9 / peak,
+        "other_layouts": others,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ne2e},

@@ -47,6 +47,8 @@ __global__ void __launch_bounds__(128) decode_rows_kernel(
     const int32_t *__restrict__ ids, const void *__restrict__ codes, int fmt,
     const float *__restrict__ C, int64_t V, int D, int M, int L, int K, float scale,
     CodeFix fix, uint16_t *__restrict__ out, unsigned *err) {
+  griddep_launch_dependents();
+  griddep_wait();   // the ids may be the argmax the previous kernel wrote
   const int64_t n = blockIdx.x;
   const int m = blockIdx.y * blockDim.x + threadIdx.x;
   if (m >= M) return;
@@ -97,12 +99,10 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
   const dim3 grid((unsigned)N, (unsigned)((M + 127) / 128));
   const CodeFix fix = make_codefix(K);
   if (D / M == 6)
-    decode_rows_kernel<6><<<grid, 128, 0, s>>>(ids, codes, fmt, C, V, D, M, L, K, scale, fix,
-                                                 out, err);
-  else
-    decode_rows_kernel<0><<<grid, 128, 0, s>>>(ids, codes, fmt, C, V, D, M, L, K, scale, fix,
-                                                 out, err);
-  return cudaGetLastError();
+    return pdl_launch(decode_rows_kernel<6>, grid, dim3(128), 0, s, ids, codes, fmt, C, V, D, M,
+                      L, K, scale, fix, out, err);
+  return pdl_launch(decode_rows_kernel<0>, grid, dim3(128), 0, s, ids, codes, fmt, C, V, D, M, L,
+                    K, scale, fix, out, err);
 }
 
 // One thread per group of 4 codes = 5 output bytes.

@@ -35,6 +35,8 @@ struct ChunkArgs {
   const float *lut;   // [P][K][TB]
   float *partial;     // [nch][B][V]
   unsigned *counter;  // reduce-kernel block counter, zeroed here
+  unsigned long long *keys;  // reduce-kernel argmax keys [B], zeroed here
+  int early_codes;    // fetch code tiles before waiting for the previous kernel
   int64_t V;
   int64_t ntiles;     // tiles of R rows
   int P, K, B, nch, cpc;
@@ -255,12 +257,17 @@ __global__ void __launch_bounds__(1024, 1)
       tma_load_2d(stage0 + s * S::STAGE_BYTES + q * S::BOX_BYTES, &tmap, box_x, y + q * 256,
                   bar, pol);
   };
-  // The code tiles do not depend on the previous kernel: start them before
-  // waiting for it (programmatic dependent launch), then fetch the tables.
+  // When the previous kernel is the table build (which writes nothing the
+  // code stream reads) the code tiles start before waiting for it.
+  if (!a.early_codes) griddep_wait();
   if (tid == 0)
     for (int s = 0; s < NST && s < n; ++s) issue(s, s);
-  griddep_wait();
-  if (tid == 0 && blockIdx.x == 0 && a.counter) *a.counter = 0u;
+  if (a.early_codes) griddep_wait();
+  if (tid == 0 && blockIdx.x == 0) {
+    if (a.counter) *a.counter = 0u;
+    if (a.keys)
+      for (int b = 0; b < a.B; ++b) a.keys[b] = 0ull;
+  }
 
   // table chunk c -> shared memory
   const float *src = a.lut + (size_t)c * S::PC * K * TB;
@@ -401,13 +408,13 @@ __device__ __forceinline__ ArgBest block_argbest(ArgBest best, ArgBest *scratch)
 }
 
 // z = sum of the nch chunk sums in chunk order; softcap; logits; argmax.
-// Grid (nblk, B).  With `argmax` set, each block leaves its best (value,
-// index) in am_val/am_idx and the last block to finish reduces them.
-// Rows go 4 per thread (16-byte loads) when V is a multiple of 4.
+// Grid (nblk, B).  With `argmax` set, each warp folds its best (value, index)
+// into keys[b] with one 64-bit atomicMax; the last block to finish turns
+// the keys into indices and clears them.  Rows go 4 per thread (16-byte
+// loads) when V is a multiple of 4 and the logits are 16-byte aligned.
 __global__ void __launch_bounds__(256) reduce_partials_kernel(
     const float *__restrict__ partial, int nch, int B, int64_t V, float cap, float *logits,
-    float *am_val, int *am_idx, unsigned *counter, int32_t *argmax) {
-  __shared__ ArgBest scratch[8];
+    unsigned long long *keys, unsigned *counter, int32_t *argmax) {
   __shared__ bool last;
   griddep_wait();   // the partial sums come from the kernel before this one
   const int b = blockIdx.y;
@@ -445,11 +452,13 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(
       best = arg_better(best, ArgBest{y, (int)v});
     }
   }
+  griddep_launch_dependents();
   if (argmax == nullptr) return;
-  const ArgBest r = block_argbest(best, scratch);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = arg_better(best, arg_shfl_xor(best, o));
+  if ((threadIdx.x & 31) == 0 && best.i != INT_MAX) atomicMax(keys + b, arg_key(best));
+  __syncthreads();
   if (threadIdx.x == 0) {
-    am_val[(size_t)b * gridDim.x + blockIdx.x] = r.v;
-    am_idx[(size_t)b * gridDim.x + blockIdx.x] = r.i;
     __threadfence();
     const unsigned ticket = atomicAdd(counter, 1u);
     last = ticket == gridDim.x * gridDim.y - 1;
@@ -457,14 +466,9 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(
   __syncthreads();
   if (!last) return;
   __threadfence();
-  const int nblk = gridDim.x;
-  for (int bb = 0; bb < B; ++bb) {
-    ArgBest t{-FLT_MAX, INT_MAX};
-    for (int k = threadIdx.x; k < nblk; k += blockDim.x)
-      t = arg_better(t, ArgBest{__ldcg(am_val + (size_t)bb * nblk + k),
-                                __ldcg(am_idx + (size_t)bb * nblk + k)});
-    const ArgBest rb = block_argbest(t, scratch);
-    if (threadIdx.x == 0) argmax[bb] = rb.i;
+  for (int bb = threadIdx.x; bb < B; bb += blockDim.x) {
+    const unsigned long long k = atomicExch(keys + bb, 0ull);
+    argmax[bb] = arg_key_index(k);
   }
   if (threadIdx.x == 0) *counter = 0u;
 }
@@ -472,6 +476,7 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(
 __global__ void __launch_bounds__(256) argmax_finalize_kernel(const float *__restrict__ am_val,
                                                               const int *__restrict__ am_idx,
                                                               int nblk, int32_t *argmax) {
+  griddep_wait();
   const int b = blockIdx.x;
   ArgBest best{-FLT_MAX, INT_MAX};
   for (int k = threadIdx.x; k < nblk; k += blockDim.x)
@@ -585,7 +590,8 @@ size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V) {
 
 cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
                                 int P, int K, int B, const float *lut, float *partial,
-                                unsigned *counter, bool pdl, const DevInfo &di, cudaStream_t s) {
+                                unsigned *counter, unsigned long long *keys, bool early_codes,
+                                const DevInfo &di, cudaStream_t s) {
   const Variant &var = kVariants[cp.variant];
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
@@ -616,6 +622,8 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   a.lut = lut;
   a.partial = partial;
   a.counter = counter;
+  a.keys = keys;
+  a.early_codes = early_codes ? 1 : 0;
   a.V = V;
   a.ntiles = (V + cp.R - 1) / cp.R;
   a.P = P;
@@ -630,22 +638,22 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   a.err = di.err;
   const int64_t grid = (int64_t)cp.nch * cpc;
   void *args[] = {&tmap, &a};
-  return launch_maybe_pdl(var.fn, dim3((unsigned)grid), dim3(1024), cp.smem, s, args, pdl);
+  return launch_maybe_pdl(var.fn, dim3((unsigned)grid), dim3(1024), cp.smem, s, args, true);
 }
 
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
-                                   float *logits, float *am_val, int *am_idx, int nblk,
+                                   float *logits, unsigned long long *keys, int nblk,
                                    unsigned *counter, int32_t *argmax, bool pdl,
                                    cudaStream_t s) {
-  void *args[] = {&partial, &nch, &B, &V, &cap, &logits, &am_val, &am_idx, &counter, &argmax};
+  void *args[] = {&partial, &nch, &B, &V, &cap, &logits, &keys, &counter, &argmax};
   return launch_maybe_pdl(reinterpret_cast<const void *>(&reduce_partials_kernel),
                           dim3((unsigned)nblk, (unsigned)B), dim3(256), 0, s, args, pdl);
 }
 
 cudaError_t launch_argmax_finalize(const float *am_val, const int *am_idx, int nblk, int B,
                                    int32_t *argmax, cudaStream_t s) {
-  argmax_finalize_kernel<<<(unsigned)B, 256, 0, s>>>(am_val, am_idx, nblk, argmax);
-  return cudaGetLastError();
+  return pdl_launch(argmax_finalize_kernel, dim3((unsigned)B), dim3(256), 0, s, am_val, am_idx,
+                    nblk, argmax);
 }
 
 }  // namespace rq

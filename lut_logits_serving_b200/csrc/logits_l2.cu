@@ -54,6 +54,7 @@ __device__ __forceinline__ void add_vec(const float *e, float (&acc)[VW]) {
 
 template <int VW, int G, int FMT>
 __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
+  griddep_wait();
   constexpr int RPW = 32 / G;     // rows per warp
   constexpr int RPB = 8 * RPW;    // rows per CTA step
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -76,8 +77,26 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
     if (FMT == RQ_CODES_U16) {
       const uint4 *crow = reinterpret_cast<const uint4 *>(
           static_cast<const uint16_t *>(a.codes) + v * a.P);
-      const int ng = a.P / 8;
-      for (int g = 0; g < ng; ++g) {
+      // 64 codes per step, all lookups of a step independent (L2 latency)
+      const int n64 = a.P / 64;
+      for (int g = 0; g < n64; ++g) {
+        uint32_t wd[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 w = __ldg(crow + 8 * g + k);
+          wd[4 * k + 0] = w.x;
+          wd[4 * k + 1] = w.y;
+          wd[4 * k + 2] = w.z;
+          wd[4 * k + 3] = w.w;
+        }
+        const float *tg = tl + (size_t)(64 * g) * K * Bs;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const uint32_t c = a.fix((j & 1) ? (wd[j >> 1] >> 16) : (wd[j >> 1] & 0xFFFFu));
+          add_vec<VW>(tg + ((size_t)j * K + c) * Bs, acc);
+        }
+      }
+      for (int g = n64 * 8; g < a.P / 8; ++g) {
         const uint4 w = __ldg(crow + g);
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
         const float *tg = tl + (size_t)(8 * g) * K * Bs;
@@ -89,24 +108,29 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         }
       }
     } else if (FMT == RQ_CODES_SCHED) {
-      // chunk-major [P/32][V][32]; groups of 16 entries (i << 12 | c << 2),
-      // any order within the group
+      // chunk-major [P/32][V][32]; 32 entries (i << 12 | c << 2) per chunk,
+      // any order within each 16-entry group
       const uint16_t *cbase = static_cast<const uint16_t *>(a.codes) + v * 32;
-      const int ng = a.P / 16;
-      for (int g = 0; g < ng; ++g) {
-        const float *tg = tl + (size_t)(16 * g) * K * Bs;
-        const uint4 *crow =
-            reinterpret_cast<const uint4 *>(cbase + (size_t)(g >> 1) * a.V * 32 + (g & 1) * 16);
+      const int nc = a.P / 32;
+      const bool kfull = K >= 1024;       // every 10-bit code indexes a real entry
+      for (int cc = 0; cc < nc; ++cc) {
+        const uint4 *crow = reinterpret_cast<const uint4 *>(cbase + (size_t)cc * a.V * 32);
+        uint32_t wd[16];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint4 w = __ldg(crow + half);
-          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        for (int k = 0; k < 4; ++k) {
+          const uint4 w = __ldg(crow + k);
+          wd[4 * k + 0] = w.x;
+          wd[4 * k + 1] = w.y;
+          wd[4 * k + 2] = w.z;
+          wd[4 * k + 3] = w.w;
+        }
+        const float *tc = tl + (size_t)(32 * cc) * K * Bs;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t e = (k & 1) ? (ws[k >> 1] >> 16) : (ws[k >> 1] & 0xFFFFu);
-            const uint32_t c = (e >> 2) & 0x3FFu;
-            if (c < (uint32_t)K) add_vec<VW>(tg + ((size_t)(e >> 12) * K + c) * Bs, acc);
-          }
+        for (int j = 0; j < 32; ++j) {
+          const uint32_t e = (j & 1) ? (wd[j >> 1] >> 16) : (wd[j >> 1] & 0xFFFFu);
+          const uint32_t c = (e >> 2) & 0x3FFu;
+          const uint32_t pp = (uint32_t)(j & 16) + (e >> 12);   // pair within the chunk
+          if (kfull || c < (uint32_t)K) add_vec<VW>(tc + ((size_t)pp * K + c) * Bs, acc);
         }
       }
     } else {
@@ -145,6 +169,7 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
     }
   }
 
+  griddep_launch_dependents();
   if (a.am_val == nullptr) return;
   // lanes with equal q hold the same tokens: reduce across row slots
 #pragma unroll
@@ -169,6 +194,7 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
 // Any shape, any format: one thread per (row, token), scalar loads.  Used
 // when the fast kernels' alignment or size preconditions do not hold.
 __global__ void __launch_bounds__(256) logits_generic_kernel(const L2Args a, int fmt) {
+  griddep_wait();
   const int t = blockIdx.y;  // token within the group
   const int64_t rb = (10LL * a.P + 7) / 8;
   const float *tl = a.lut + a.lut_t0 + t;
@@ -212,8 +238,7 @@ __global__ void __launch_bounds__(256) logits_generic_kernel(const L2Args a, int
 
 template <int VW, int G, int FMT>
 static cudaError_t launch_fast(const L2Args &a, int nblk, cudaStream_t s) {
-  logits_l2_kernel<VW, G, FMT><<<nblk, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return pdl_launch(logits_l2_kernel<VW, G, FMT>, dim3(nblk), dim3(256), 0, s, a);
 }
 
 template <int VW, int FMT>
@@ -256,8 +281,8 @@ cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K
   const bool lut_ok = VW < 4 || ((reinterpret_cast<uintptr_t>(lut + lut_t0) & 15) == 0 &&
                                  Bs % 4 == 0);
   if (!(codes16 && fast_fmt && lut_ok) || nb > 32 || (VW < 4 && nb > VW)) {
-    logits_generic_kernel<<<dim3((unsigned)nblk, (unsigned)nb), 256, 0, s>>>(a, fmt);
-    return cudaGetLastError();
+    return pdl_launch(logits_generic_kernel, dim3((unsigned)nblk, (unsigned)nb), dim3(256), 0, s,
+                      a, fmt);
   }
   int G = 1;
   if (VW == 4) {

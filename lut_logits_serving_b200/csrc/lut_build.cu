@@ -18,6 +18,7 @@ __global__ void __launch_bounds__(256) lut_build_kernel(const float *__restrict_
                                                         int nb, int D, int M, int L, int K,
                                                         int Bs, float *__restrict__ lut) {
   extern __shared__ float hs[];  // [Bs][ds] hidden slice of subspace m
+  griddep_wait();
   const int p = blockIdx.y;
   const int m = p / L;
   const int ds = D / M;
@@ -65,24 +66,27 @@ __device__ __forceinline__ float4 ldg_v4_keep(const float *p, uint64_t pol) {
 __global__ void __launch_bounds__(256) lut_build_ds6_kernel(const float *__restrict__ h,
                                                            const float *__restrict__ C, int b0,
                                                            int nb, int D, int L, int K, int Bs,
-                                                           int64_t quads, float *__restrict__ lut) {
-  griddep_launch_dependents();             // the next kernel may start its prologue
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+                                                           int quads, float *__restrict__ lut) {
+  // One wave: let the next kernel (the code pass) start its prologue now.
+  griddep_launch_dependents();
+  griddep_wait();                          // h and the table buffer: earlier kernels
+  // P*K < 2^31 (checked by the launcher): 32-bit index math, no 64-bit divides
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= quads) return;
-  const int64_t e0 = 4 * g;                 // first codeword (p*K + k) of this thread
-  const int p = (int)(e0 / K);
+  const int e0 = 4 * g;                     // first codeword (p*K + k) of this thread
+  const int p = e0 / K;
   const int m = p / L;
   const uint64_t pol = l2_policy_evict_last();
   float c[24];
 #pragma unroll
   for (int q = 0; q < 6; ++q) {
-    const float4 v = ldg_v4_keep(C + e0 * 6 + 4 * q, pol);
+    const float4 v = ldg_v4_keep(C + (size_t)e0 * 6 + 4 * q, pol);
     c[4 * q + 0] = v.x;
     c[4 * q + 1] = v.y;
     c[4 * q + 2] = v.z;
     c[4 * q + 3] = v.w;
   }
-  float *out = lut + e0 * Bs;
+  float *out = lut + (size_t)e0 * Bs;
   for (int t = 0; t < Bs; ++t) {
     float hv[6];
 #pragma unroll
@@ -104,26 +108,71 @@ __global__ void __launch_bounds__(256) lut_build_ds6_kernel(const float *__restr
   }
 }
 
+// ds = 6, token groups of 4..64 (Bs % 4 == 0): one thread per (codeword,
+// 4 tokens); a warp writes 8 codewords x 32 tokens... as contiguous float4
+// runs, so the 100 MB table of a 32-token group streams out coalesced.
+__global__ void __launch_bounds__(256) lut_build_ds6_tok_kernel(
+    const float *__restrict__ h, const float *__restrict__ C, int b0, int nb, int D, int L, int K,
+    int Bs, int items, float *__restrict__ lut) {
+  griddep_wait();
+  // items < 2^31 (checked by the launcher): 32-bit index math
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g < items) {
+    const int q = Bs / 4;
+    const int e = g / q;                     // codeword p*K + k
+    const int t0 = (g - e * q) * 4;          // first token of this thread
+    const int m = e / K / L;
+    const float *cw = C + (size_t)e * 6;
+    const float2 c01 = __ldg(reinterpret_cast<const float2 *>(cw));
+    const float2 c23 = __ldg(reinterpret_cast<const float2 *>(cw + 2));
+    const float2 c45 = __ldg(reinterpret_cast<const float2 *>(cw + 4));
+    const float c[6] = {c01.x, c01.y, c23.x, c23.y, c45.x, c45.y};
+    float r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = t0 + i;
+      float acc = 0.f;
+      if (t < nb) {
+        const float *hm = h + (size_t)(b0 + t) * D + m * 6;
+#pragma unroll
+        for (int j = 0; j < 6; ++j) acc = fmaf(__ldg(hm + j), c[j], acc);
+      }
+      r[i] = acc;
+    }
+    *reinterpret_cast<float4 *>(lut + (size_t)e * Bs + t0) = make_float4(r[0], r[1], r[2], r[3]);
+  }
+  griddep_launch_dependents();
+}
+
 cudaError_t launch_lut_build(const float *h, const float *C, int B, int b0, int nb, int D,
                              int M, int L, int K, int Bs, float *lut, cudaStream_t s) {
   (void)B;
   const int ds = D / M;
   const int P = M * L;
-  if (ds == 6 && K % 4 == 0 && (reinterpret_cast<uintptr_t>(C) & 15) == 0 &&
+  if (ds == 6 && Bs % 4 == 0 && (reinterpret_cast<uintptr_t>(C) & 7) == 0 &&
+      (reinterpret_cast<uintptr_t>(lut) & 15) == 0) {
+    const int64_t items = (int64_t)P * K * (Bs / 4);
+    const int64_t blocks = (items + 255) / 256;
+    if (items < 0x7fffffffLL - 256)
+      return pdl_launch(lut_build_ds6_tok_kernel, dim3((unsigned)blocks), dim3(256), 0, s, h, C,
+                        b0, nb, D, L, K, Bs, (int)items, lut);
+  }
+  if (ds == 6 && Bs <= 2 && K % 4 == 0 && (reinterpret_cast<uintptr_t>(C) & 15) == 0 &&
       (reinterpret_cast<uintptr_t>(lut) & 15) == 0) {
     const int64_t quads = (int64_t)P * K / 4;
     const int64_t blocks = (quads + 255) / 256;
-    lut_build_ds6_kernel<<<(unsigned)blocks, 256, 0, s>>>(h, C, b0, nb, D, L, K, Bs, quads, lut);
-    return cudaGetLastError();
+    if (4 * quads < 0x7fffffffLL - 1024)
+      return pdl_launch(lut_build_ds6_kernel, dim3((unsigned)blocks), dim3(256), 0, s, h, C, b0,
+                        nb, D, L, K, Bs, (int)quads, lut);
   }
   dim3 grid((unsigned)((K + 255) / 256), (unsigned)P);
   size_t smem = (size_t)Bs * ds * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
   if (ds <= 8)
-    lut_build_kernel<8><<<grid, 256, smem, s>>>(h, C, b0, nb, D, M, L, K, Bs, lut);
-  else
-    lut_build_kernel<0><<<grid, 256, smem, s>>>(h, C, b0, nb, D, M, L, K, Bs, lut);
-  return cudaGetLastError();
+    return pdl_launch(lut_build_kernel<8>, grid, dim3(256), smem, s, h, C, b0, nb, D, M, L, K, Bs,
+                      lut);
+  return pdl_launch(lut_build_kernel<0>, grid, dim3(256), smem, s, h, C, b0, nb, D, M, L, K, Bs,
+                    lut);
 }
 
 }  // namespace rq

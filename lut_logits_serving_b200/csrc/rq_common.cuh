@@ -175,6 +175,19 @@ __device__ __forceinline__ ArgBest arg_better(ArgBest a, ArgBest b) {
   return a.i <= b.i ? a : b;
 }
 
+// 64-bit key whose unsigned order is the argmax order: value (NaN lowest,
+// -0 == +0) in the high word, then the lower index in the low word.  One
+// atomicMax per warp then finds the argmax in any arrival order.
+__device__ __forceinline__ unsigned long long arg_key(ArgBest a) {
+  if (a.v != a.v) return 0ull;
+  uint32_t u = a.v == 0.f ? 0u : __float_as_uint(a.v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)a.i);
+}
+__device__ __forceinline__ int arg_key_index(unsigned long long k) {
+  return k == 0ull ? 0 : (int)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+}
+
 __device__ __forceinline__ ArgBest arg_shfl_xor(ArgBest a, int lane_mask) {
   ArgBest o;
   o.v = __shfl_xor_sync(0xffffffffu, a.v, lane_mask);
@@ -186,6 +199,26 @@ __device__ __forceinline__ ArgBest arg_shfl_xor(ArgBest a, int lane_mask) {
 
 // Launchers implemented by the kernel translation units (host side).
 namespace rq {
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream drains.  Every kernel launched so
+// calls griddep_wait() before it touches memory an earlier kernel may write
+// or read, so completion still orders all kernels transitively.
+template <typename... KArgs, typename... Args>
+inline cudaError_t pdl_launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 // cudaLaunchKernel, or with programmatic stream serialization when `pdl`:
 // the kernel may start while the previous one in the stream drains and
@@ -240,13 +273,16 @@ struct ChunkPlan {
 };
 ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di);
 size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V);
+// `early_codes`: the previous kernel writes nothing the code stream reads,
+// so the code tiles may be fetched before waiting for it.
 cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
                                 int P, int K, int B, const float *lut, float *partial,
-                                unsigned *counter, bool pdl, const DevInfo &di, cudaStream_t s);
+                                unsigned *counter, unsigned long long *keys, bool early_codes,
+                                const DevInfo &di, cudaStream_t s);
 // Sums the chunk partials, softcap, logits; with `argmax` set also the
 // argmax (block partials in am_val/am_idx, finished by the last block).
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
-                                   float *logits, float *am_val, int *am_idx, int nblk,
+                                   float *logits, unsigned long long *keys, int nblk,
                                    unsigned *counter, int32_t *argmax, bool pdl,
                                    cudaStream_t s);
 

@@ -100,8 +100,8 @@ struct WsLayout {
   bool chunk;
   ChunkPlan cp;
   size_t partial_off, partial_bytes;
-  size_t amv_off, ami_off, am_bytes;
-  size_t counter_off;
+  size_t amv_off, ami_off, am_bytes;   // argmax block partials (token-group path)
+  size_t keys_off, counter_off;         // argmax keys + counter (tiled path)
   size_t total;
 };
 
@@ -116,16 +116,17 @@ WsLayout ws_layout(const rq_dims &d, int B, int fmt, bool want_argmax, const Dev
     w.partial_bytes = chunk_partial_bytes(w.cp, B, d.V);
     off += (size_t)align_up((int64_t)w.partial_bytes, kAlign);
   }
-  if (want_argmax) {
+  if (want_argmax && w.chunk) {
+    w.keys_off = off;
+    off += (size_t)align_up((int64_t)B * 8, kAlign);
+    w.counter_off = off;
+    off += kAlign;
+  } else if (want_argmax) {
     w.am_bytes = (size_t)B * kMaxSweepBlocks * 4;
     w.amv_off = off;
     off += (size_t)align_up((int64_t)w.am_bytes, kAlign);
     w.ami_off = off;
     off += (size_t)align_up((int64_t)w.am_bytes, kAlign);
-    if (w.chunk) {
-      w.counter_off = off;
-      off += kAlign;
-    }
   }
   w.total = off;
   return w;
@@ -149,23 +150,25 @@ int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, i
                float cap, float *logits, int32_t *argmax, unsigned char *ws,
                const WsLayout &w, const DevInfo &di, cudaStream_t s, bool after_build) {
   const int P = d.M * d.L;
-  float *amv = argmax ? reinterpret_cast<float *>(ws + w.amv_off) : nullptr;
-  int *ami = argmax ? reinterpret_cast<int *>(ws + w.ami_off) : nullptr;
   const int nblk = sweep_blocks(d, di, w.chunk);
   cudaError_t e;
   if (w.chunk) {
     float *partial = reinterpret_cast<float *>(ws + w.partial_off);
     unsigned *counter = argmax ? reinterpret_cast<unsigned *>(ws + w.counter_off) : nullptr;
+    unsigned long long *keys =
+        argmax ? reinterpret_cast<unsigned long long *>(ws + w.keys_off) : nullptr;
     if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
     const bool prof = t_prof_start != nullptr;   // events between kernels break the overlap
-    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, counter,
+    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, counter, keys,
                             after_build && !prof, di, s);
     if (e != cudaSuccess) return status_of(e);
     if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
-    e = launch_reduce_partials(partial, w.cp.nch, B, d.V, cap, logits, amv, ami, nblk, counter,
-                               argmax, !prof, s);
+    e = launch_reduce_partials(partial, w.cp.nch, B, d.V, cap, logits, keys, nblk, counter,
+                               argmax, true, s);
     return status_of(e);
   } else {
+    float *amv = argmax ? reinterpret_cast<float *>(ws + w.amv_off) : nullptr;
+    int *ami = argmax ? reinterpret_cast<int *>(ws + w.ami_off) : nullptr;
     if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
     for (int b0 = 0; b0 < B; b0 += kTokenGroup) {
       const int nb = B - b0 < kTokenGroup ? B - b0 : kTokenGroup;
@@ -174,10 +177,10 @@ int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, i
       if (e != cudaSuccess) return status_of(e);
     }
     if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
-  }
-  if (argmax) {
-    e = launch_argmax_finalize(amv, ami, nblk, B, argmax, s);
-    if (e != cudaSuccess) return status_of(e);
+    if (argmax) {
+      e = launch_argmax_finalize(amv, ami, nblk, B, argmax, s);
+      if (e != cudaSuccess) return status_of(e);
+    }
   }
   return RQ_OK;
 }
