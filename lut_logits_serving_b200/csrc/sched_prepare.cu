@@ -10,9 +10,12 @@
 // are reordered so that every step is, as far as possible, a matching of
 // lanes to distinct banks: step by step, a maximum bipartite matching
 // (augmenting paths, Kuhn's method) between the lanes and the banks of
-// their remaining codes; a lane left unmatched takes the remaining code
-// whose bank is least used in that step.  Any order gives the same logits
-// up to fp32 summation order; only the speed depends on it.
+// their remaining codes, grown from the banks with the most codes left (the
+// sets of banks a matching can cover form a transversal matroid, so that
+// greedy order covers the heaviest banks); a lane left unmatched takes the
+// remaining code whose bank is least used in that step, heaviest first.
+// Any order gives the same logits up to fp32 summation order; only the
+// speed depends on it.
 //
 // Entry format: (i << 12) | (c << 2), i = pair position in the group,
 // c = code (< 1024).  For a 4-byte table entry per code and a 4 KB table
@@ -29,13 +32,11 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
     const uint16_t *__restrict__ codes, int64_t V, int P, uint16_t *__restrict__ out,
     unsigned long long *stats) {
   __shared__ uint16_t s_code[kSchedThreads][32][16];   // codes of each lane
-  __shared__ uint32_t s_bmask[kSchedThreads][32];      // banks of unused codes
-  __shared__ int8_t s_match[kSchedThreads][32];        // bank -> lane
-  __shared__ int8_t s_lbank[kSchedThreads][32];        // lane -> bank
+  __shared__ uint32_t s_lmask[kSchedThreads][32];      // per bank: lanes with unused codes in it
+  __shared__ int8_t s_lbank[kSchedThreads][32];        // lane -> matched bank
   const int T = threadIdx.x;
   uint16_t(*cd)[16] = s_code[T];
-  uint32_t *bm = s_bmask[T];
-  int8_t *match = s_match[T];
+  uint32_t *bm = s_lmask[T];
   int8_t *lbank = s_lbank[T];
 
   const int nch = (P + 31) / 32;
@@ -60,52 +61,69 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
 
   unsigned long long passes = 0;
   for (int step = 0; step < 16; ++step) {
-    for (int ln = 0; ln < 32; ++ln) {
-      uint32_t m = 0;
-      if ((present >> ln) & 1)
-        for (int k = 0; k < 16; ++k)
-          if (!((used[ln] >> k) & 1)) m |= 1u << (cd[ln][k] & 31);
-      bm[ln] = m;
-      lbank[ln] = -1;
-      match[ln] = -1;
+    // per bank: lanes holding an unused code in it, and how many such codes
+    int deg[32];
+    for (int b = 0; b < 32; ++b) {
+      bm[b] = 0u;   // here: lane mask of bank b
+      deg[b] = 0;
     }
-    // maximum matching lanes -> banks by augmenting paths
-    for (int start = 0; start < 32; ++start) {
-      if (!((present >> start) & 1)) continue;
-      int stack_lane[33];
+    for (int ln = 0; ln < 32; ++ln) {
+      lbank[ln] = -1;
+      if (!((present >> ln) & 1)) continue;
+      for (int k = 0; k < 16; ++k)
+        if (!((used[ln] >> k) & 1)) {
+          const int b = cd[ln][k] & 31;
+          bm[b] |= 1u << ln;
+          deg[b] += 1;
+        }
+    }
+    // Maximum matching lanes <-> banks by augmenting paths started from the
+    // banks in decreasing order of remaining codes: the matched bank sets
+    // form a matroid, so this greedy order covers the most loaded banks.
+    uint32_t done_banks = 0u;
+    for (int it = 0; it < 32; ++it) {
+      int start = -1, best = 0;
+      for (int b = 0; b < 32; ++b)
+        if (!((done_banks >> b) & 1) && deg[b] > best) {
+          best = deg[b];
+          start = b;
+        }
+      if (start < 0) break;
+      done_banks |= 1u << start;
+      int stack_bank[33];
       uint32_t stack_cand[33];
-      int8_t stack_bank[33];
-      uint32_t seen = 0;
+      int8_t stack_lane[33];
+      uint32_t seen = 0;   // lanes visited
       int depth = 0;
-      stack_lane[0] = start;
+      stack_bank[0] = start;
       stack_cand[0] = bm[start];
-      bool done = false;
-      while (depth >= 0 && !done) {
+      bool found = false;
+      while (depth >= 0 && !found) {
         const uint32_t cand = stack_cand[depth] & ~seen;
         if (cand == 0) {
           --depth;
           continue;
         }
-        const int b = __ffs(cand) - 1;
-        stack_cand[depth] = cand & ~(1u << b);
-        seen |= 1u << b;
-        stack_bank[depth] = (int8_t)b;
-        if (match[b] < 0) {
-          for (int d = depth; d >= 0; --d) {   // flip the augmenting path
-            match[stack_bank[d]] = (int8_t)stack_lane[d];
-            lbank[stack_lane[d]] = stack_bank[d];
-          }
-          done = true;
+        const int ln = __ffs(cand) - 1;
+        stack_cand[depth] = cand & ~(1u << ln);
+        seen |= 1u << ln;
+        stack_lane[depth] = (int8_t)ln;
+        if (lbank[ln] < 0) {
+          for (int d = depth; d >= 0; --d) lbank[stack_lane[d]] = (int8_t)stack_bank[d];
+          found = true;
         } else if (depth < 32) {
           ++depth;
-          stack_lane[depth] = match[b];
-          stack_cand[depth] = bm[match[b]];
+          stack_bank[depth] = lbank[ln];
+          stack_cand[depth] = bm[lbank[ln]];
         }
       }
     }
-    // choose the items; unmatched lanes take their least crowded bank
+    // choose the codes; an unmatched lane takes its least used bank in this
+    // step, the most loaded one among equals
     int cnt[32];
-    for (int b = 0; b < 32; ++b) cnt[b] = match[b] >= 0 ? 1 : 0;
+    for (int b = 0; b < 32; ++b) cnt[b] = 0;
+    for (int ln = 0; ln < 32; ++ln)
+      if (lbank[ln] >= 0) cnt[lbank[ln]] += 1;
     int maxc = 0;
     for (int ln = 0; ln < 32; ++ln) {
       if (!((present >> ln) & 1)) continue;
@@ -114,11 +132,15 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
         for (int k = 0; k < 16 && pick < 0; ++k)
           if (!((used[ln] >> k) & 1) && (cd[ln][k] & 31) == lbank[ln]) pick = k;
       } else {
-        int best = 1 << 30;
+        int bc = 1 << 30, bd = -1;
         for (int k = 0; k < 16; ++k)
-          if (!((used[ln] >> k) & 1) && cnt[cd[ln][k] & 31] < best) {
-            best = cnt[cd[ln][k] & 31];
-            pick = k;
+          if (!((used[ln] >> k) & 1)) {
+            const int b = cd[ln][k] & 31;
+            if (cnt[b] < bc || (cnt[b] == bc && deg[b] > bd)) {
+              bc = cnt[b];
+              bd = deg[b];
+              pick = k;
+            }
           }
         cnt[cd[ln][pick] & 31] += 1;
       }
