@@ -71,6 +71,30 @@ def code_bytes(w):
     return w.V * (w.P * 10 // 8 if w.packed10 else w.P * 2)
 
 
+# --------------------------------------------------------- multi-rank math
+
+def aggregate(local_ms, world, device="cpu"):
+    """Job time of a weak-scaling replica run: the slowest rank's device time
+    (all_reduce MAX over the default process group when world > 1)."""
+    if world <= 1:
+        return float(local_ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(units_per_rank, world, job_ms):
+    """Whole-job rate: units processed by all ranks over the job time."""
+    return world * units_per_rank / (job_ms / 1e3)
+
+
+def rank_seed(rank):
+    """Each replica scores its own seeded batch and artifact."""
+    return 1000 * rank
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -243,13 +267,9 @@ def run_ours(args, w):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world > 1:
-            t = torch.tensor([x], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
-        return x
+        return aggregate(x, world, device="cuda")
 
-    data = synth.make(w, seed=1000 * rank)
+    data = synth.make(w, seed=rank_seed(rank))
     d = rq.dims(w.V, w.D, w.M, w.L, w.K)
     dC = torch.from_numpy(data["C"]).cuda()
     c16 = torch.from_numpy(data["codes"].reshape(w.V, -1)).cuda()
@@ -338,7 +358,7 @@ def run_ours(args, w):
     with ClockSampler(local) as clk:
         t_ms = time_steps(run, args.steps)
     sec = t_ms / 1e3
-    value = world * w.V * w.B * args.steps / sec
+    value = throughput(w.V * w.B * args.steps, world, t_ms)
 
     # ---- the dominant kernel alone, live CUDA events
     kern_us = code_pass_us(step, min(args.steps, 2000))
@@ -358,7 +378,7 @@ def run_ours(args, w):
         n2 = min(args.steps, 3000)
         t2 = time_steps(r2, n2)
         k2 = code_pass_us(st2, min(n2, 1000))
-        others[name] = {"us_per_call": t2 / n2 * 1e3, "value": world * w.V * w.B * n2 / (t2 / 1e3),
+        others[name] = {"us_per_call": t2 / n2 * 1e3, "value": throughput(w.V * w.B * n2, world, t2),
                         "code_pass_us": k2,
                         "code_pass_frac": algo_bytes / (k2 / 1e6) / 1e9 / peak}
         del g2
@@ -379,7 +399,7 @@ def run_ours(args, w):
     for _ in range(3):
         e2e_step()
     e_ms = time_steps(e2e_step, ne2e)
-    e2e_value = world * w.V * w.B * ne2e / (e_ms / 1e3)
+    e2e_value = throughput(w.V * w.B * ne2e, world, e_ms)
     h2d = data["h"].nbytes
     d2h = w.B * w.V * 4 + w.B * 4
 

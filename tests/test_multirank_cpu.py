@@ -1,0 +1,63 @@
+"""The N > 1 benchmark path on CPU: two gloo ranks run bench.py's
+aggregation (the job time is the slowest rank's device time, the value
+counts every rank's units) and get different replica seeds.  The GPU path
+itself needs one GPU per rank and no data-path collective (replicas)."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    from lut_logits_serving_b200 import synth
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    local_ms = [12.5, 20.0][rank]
+    job = bench.aggregate(local_ms, world)
+    value = bench.throughput(1000, world, job)
+    w = synth.WORKLOADS["tiny"]
+    d = synth.make(w, seed=bench.rank_seed(rank))
+    q.put((rank, job, value, int(d["codes"][0, 0, 0]), float(d["h"][0, 0])))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_aggregation_with_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, job0, v0, c0, h0), (r1, job1, v1, c1, h1) = res
+    assert job0 == job1 == 20.0                       # max over ranks
+    assert v0 == v1 == pytest.approx(2 * 1000 / 0.020)
+    assert (c0, h0) != (c1, h1)                       # each replica its own inputs
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.aggregate(7.0, 1) == 7.0
+    assert bench.throughput(256000, 1, 0.1) == pytest.approx(2.56e9)
