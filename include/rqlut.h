@@ -42,14 +42,16 @@
  *            RQ_CODES_SCHED:    uint16 [M*L/32][V][32] (K <= 1024, M*L % 32
  *                               == 0), written by rq_prepare_sched: chunk-
  *                               major (columns 32c..32c+31 of every row form
- *                               one contiguous [V][32] block); each aligned
- *                               group of 16 columns holds that group's 16
- *                               codes in a permuted order, entry = (i << 12)
- *                               | (c << 2) with i in [0,16) the pair's
- *                               position in the group and c its code.  The
- *                               order only changes summation order; entries
- *                               with c >= K add 0 to the logits
- *                               (rq_decode_rows clamps them to K-1).
+ *                               one contiguous [V][32] block, the row's
+ *                               "slice"); each slice holds its 32 codes in a
+ *                               permuted order, entry = (i << 10) | c with i
+ *                               in [0,32) the pair's position in the slice
+ *                               and c its code.  The order only changes the
+ *                               summation order; entries with c >= K add 0
+ *                               to the logits (rq_decode_rows clamps them to
+ *                               K-1).  Batch 1 streams it fastest; larger
+ *                               batches run it through the slower generic
+ *                               lookup order (use RQ_CODES_U16 there).
  *   lut      float [M*L][K][Bs], Bs = rq_lut_token_stride(B): token b of
  *            table (p, k) at lut[(p*K + k)*Bs + b]
  *   logits   float [B][V]
@@ -203,12 +205,12 @@ RQ_API int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed,
 /*
  * rq_prepare_sched -- convert uint16 codes [V][M*L] into RQ_CODES_SCHED
  * (same size; chunk-major so that each 32-pair slice streams contiguously).
- * Not on the pages: a layout of this library.  The lookups of the B <= 2
- * logits pass run 16 rows x 2 groups of 16 pairs per warp, one lookup per
- * lane per step, and shared memory serves a step in as many passes as the
- * most repeated bank (bank = code mod 32).  Random codes give ~3.5 passes;
- * this call orders each group so that every step's 32 lookups hit as few
- * repeated banks as a maximum bipartite matching per step allows (~1.8).
+ * Not on the pages: a layout of this library.  The lookups of the batch-1
+ * logits pass run 32 rows x one 32-pair slice per warp, one lookup per lane
+ * per step, and shared memory serves a step in as many passes as the most
+ * repeated bank (bank = code mod 32).  Random codes give ~3.5 passes; this
+ * call orders each slice so that every step's 32 lookups hit as few
+ * repeated banks as a maximum bipartite matching per step allows (~1.5).
  * Same bytes, same sums (in another order).  Run once per artifact.
  *   codes_u16 (device) uint16 [V][M*L], values < K (larger values keep
  *             their low 10 bits); out (device) uint16 [V][M*L], must not

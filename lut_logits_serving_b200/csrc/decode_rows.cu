@@ -17,17 +17,17 @@
 
 namespace rq {
 
-// Code of pair p of row `id` in RQ_CODES_SCHED (chunk-major [P/32][V][32]):
-// find index p % 16 in its group.
+// Code of pair p of row `id` in RQ_CODES_SCHED (chunk-major [P/32][V][32],
+// entries i << 10 | c): find position p % 32 in the row's chunk slice.
 __device__ __forceinline__ uint32_t sched_code(const uint16_t *codes, int64_t V, int64_t id,
                                                int p) {
-  const uint16_t *g = codes + ((int64_t)(p >> 5) * V + id) * 32 + (p & 16);
-  const uint32_t want = (uint32_t)(p & 15);
+  const uint16_t *g = codes + ((int64_t)(p >> 5) * V + id) * 32;
+  const uint32_t want = (uint32_t)(p & 31);
   uint32_t c = 0;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
+  for (int k = 0; k < 32; ++k) {
     const uint32_t e = g[k];
-    if ((e >> 12) == want) c = (e >> 2) & 0x3FFu;
+    if (((e >> 10) & 31u) == want) c = e & 0x3FFu;
   }
   return c;
 }

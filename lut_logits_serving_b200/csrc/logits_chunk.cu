@@ -44,12 +44,15 @@ struct ChunkArgs {
   unsigned *err;
 };
 
-template <int TB>
+// Plain codes: TPR threads per row, 1024 threads.  Bank-scheduled codes
+// (one token): one thread per row owns the row's whole 32-pair slice, the
+// unit the schedule was made for, 512 threads.
+template <int TB, bool SCHED = false>
 struct ChunkShape {
-  static constexpr int PC = TB == 1 ? 32 : (TB == 2 ? 16 : 8);  // pairs per chunk
-  static constexpr int PPT = TB == 4 ? 8 : 16;                  // pairs per thread
+  static constexpr int PC = SCHED ? 32 : (TB == 1 ? 32 : (TB == 2 ? 16 : 8));  // pairs/chunk
+  static constexpr int PPT = SCHED ? 32 : (TB == 4 ? 8 : 16);                  // pairs/thread
   static constexpr int TPR = PC / PPT;                          // threads per row
-  static constexpr int THREADS = 1024;
+  static constexpr int THREADS = SCHED ? 512 : 1024;
   static constexpr int WARPS = THREADS / 32;
   static constexpr int R = THREADS / TPR;                       // rows per tile
   static constexpr int ROWB = PC * 2;                           // code bytes per row slice
@@ -154,36 +157,26 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return x;
 }
 
-// RQ_CODES_SCHED, one token: the 16 entries of a group (two 16-byte code
-// vectors), all 16 table loads issued before any add, summed as a tree.
-__device__ __forceinline__ float group16_sched_tb1(uint32_t gbase, uint4 w0, uint4 w1) {
-  const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-  float x[16];
+// RQ_CODES_SCHED, one token: the 32 entries (i << 10 | c) of a row's chunk
+// slice (four 16-byte code vectors), each the word offset of its table entry
+// in the chunk's 32 x 1024 tables at shared address `tbase`.  All 32 loads
+// are issued before any add; the sum is a tree.  The 15-bit masks keep every
+// address aligned and inside the 128 KB of tables.
+__device__ __forceinline__ float chunk32_sched_tb1(uint32_t tbase, const uint4 (&w)[4]) {
+  const uint32_t ws[16] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w,
+                           w[2].x, w[2].y, w[2].z, w[2].w, w[3].x, w[3].y, w[3].z, w[3].w};
+  float x[32];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    x[2 * q] = lds_f32(gbase + (ws[q] & 0xFFFCu));
-    x[2 * q + 1] = lds_f32(gbase + __umulhi(ws[q] & 0xFFFC0000u, 0x10000u));
+  for (int q = 0; q < 16; ++q) {
+    x[2 * q] = lds_f32(tbase + ((ws[q] & 0x7FFFu) << 2));
+    // high entry: ((w & 0x7FFF0000) * 2^18) >> 32 = ((w >> 16) & 0x7FFF) * 4
+    x[2 * q + 1] = lds_f32(tbase + __umulhi(ws[q] & 0x7FFF0000u, 1u << 18));
   }
 #pragma unroll
-  for (int w = 1; w < 16; w <<= 1)
+  for (int st = 1; st < 32; st <<= 1)
 #pragma unroll
-    for (int q = 0; q < 16; q += 2 * w) x[q] += x[q + w];
+    for (int q = 0; q < 32; q += 2 * st) x[q] += x[q + st];
   return x[0];
-}
-
-// RQ_CODES_SCHED: 8 entries (i << 12 | c << 2) of one 16-pair group whose
-// tables start at shared byte address `gbase`, each table 1024 * TB floats:
-// the entry times TB is the byte offset.  The mask keeps every address
-// 4-byte aligned and inside the group's 64 KB * TB.
-template <int TB>
-__device__ __forceinline__ void lookup8_sched(uint32_t gbase, uint4 w, float (&acc)[TB]) {
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    add_entry<TB, 0>(gbase + (ws[q] & 0xFFFCu) * TB, acc);
-    // high entry: ((w & 0xFFFC0000) * 2^16) >> 32 plus the base, one IMAD.HI
-    add_entry<TB, 0>(gbase + __umulhi(ws[q] & 0xFFFC0000u, 0x10000u * TB), acc);
-  }
 }
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
@@ -200,11 +193,11 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 template <int TB, int KT, int NST, int FMT>
-__global__ void __launch_bounds__(1024, 1)
+__global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS, 1)
     logits_chunk_u16_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
-  using S = ChunkShape<TB>;
   constexpr bool SCHED = FMT == RQ_CODES_SCHED;
-  static_assert(!SCHED || S::PPT == 16, "a thread must own whole 16-pair groups");
+  using S = ChunkShape<TB, SCHED>;
+  static_assert(!SCHED || (TB == 1 && S::PPT == 32), "a thread owns a whole scheduled slice");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment (TMA swizzle atoms) by pointer arithmetic, so the
   // compiler keeps the shared address space
@@ -329,21 +322,17 @@ __global__ void __launch_bounds__(1024, 1)
     float acc[TB];
 #pragma unroll
     for (int b = 0; b < TB; ++b) acc[b] = 0.f;
-    if (SCHED && TB == 1) {
-      if (nq > 0) {                          // a whole 16-pair group
-        const uint4 w0 = ld_shared_v4(st + voff[0]);
-        const uint4 w1 = ld_shared_v4(st + voff[NQ - 1]);
-        acc[0] = group16_sched_tb1(tt, w0, w1);
-      }
+    if constexpr (SCHED) {
+      uint4 w[4];                            // the row's whole 32-pair slice
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(st + voff[q]);
+      acc[0] = chunk32_sched_tb1(tt, w);
     } else {
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         if (q < nq) {
           const uint4 w = ld_shared_v4(st + voff[q]);
-          if (SCHED)
-            lookup8_sched<TB>(tt, w, acc);
-          else
-            lookup8<TB, KT>(tt + (uint32_t)q * 8 * K * TB * 4, K, w, a.fix, acc);
+          lookup8<TB, KT>(tt + (uint32_t)q * 8 * K * TB * 4, K, w, a.fix, acc);
         }
       }
     }
@@ -520,13 +509,17 @@ EncodeTiledFn encode_fn() {
 
 struct Variant {
   int TB, KT, NST, FMT;
+  int PC, R, THREADS, STAGE_BYTES;
   const void *fn;
 };
 
-#define RQ_CHUNK_VARIANT(TB, KT, NST, FMT)                                          \
-  Variant {                                                                         \
-    TB, KT, NST, FMT,                                                               \
-        reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, NST, FMT>)  \
+#define RQ_CHUNK_VARIANT(TB, KT, NST, FMT)                                           \
+  Variant {                                                                          \
+    TB, KT, NST, FMT, ChunkShape<TB, FMT == RQ_CODES_SCHED>::PC,                     \
+        ChunkShape<TB, FMT == RQ_CODES_SCHED>::R,                                    \
+        ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS,                              \
+        ChunkShape<TB, FMT == RQ_CODES_SCHED>::STAGE_BYTES,                          \
+        reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, NST, FMT>)   \
   }
 
 // 128 KB table chunk + NST stages (3 x 32 KB or 5 x 16 KB) per CTA, one CTA
@@ -535,24 +528,13 @@ const Variant kVariants[] = {
     RQ_CHUNK_VARIANT(1, 1024, 3, RQ_CODES_U16), RQ_CHUNK_VARIANT(2, 1024, 3, RQ_CODES_U16),
     RQ_CHUNK_VARIANT(4, 1024, 5, RQ_CODES_U16), RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_U16),
     RQ_CHUNK_VARIANT(2, 0, 3, RQ_CODES_U16),    RQ_CHUNK_VARIANT(4, 0, 5, RQ_CODES_U16),
-    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_SCHED),  RQ_CHUNK_VARIANT(2, 0, 3, RQ_CODES_SCHED),
+    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_SCHED),
 };
-
-int variant_pc(const Variant &v) {
-  return v.TB == 1 ? ChunkShape<1>::PC : (v.TB == 2 ? ChunkShape<2>::PC : ChunkShape<4>::PC);
-}
-int variant_rows(const Variant &v) {
-  return v.TB == 1 ? ChunkShape<1>::R : (v.TB == 2 ? ChunkShape<2>::R : ChunkShape<4>::R);
-}
-int variant_stage(const Variant &v) {
-  return v.TB == 1 ? ChunkShape<1>::STAGE_BYTES
-                   : (v.TB == 2 ? ChunkShape<2>::STAGE_BYTES : ChunkShape<4>::STAGE_BYTES);
-}
 
 size_t variant_smem(const Variant &v, int K) {
   const int KS = v.FMT == RQ_CODES_SCHED ? 1024 : K;
-  return 1024 + (size_t)align_up((int64_t)variant_pc(v) * KS * v.TB * 4, 1024) +
-         (size_t)v.NST * variant_stage(v) + 1024;
+  return 1024 + (size_t)align_up((int64_t)v.PC * KS * v.TB * 4, 1024) +
+         (size_t)v.NST * v.STAGE_BYTES + 1024;
 }
 
 }  // namespace
@@ -574,9 +556,9 @@ ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di)
     if (smem > (size_t)di.max_smem_optin) continue;
     cp.ok = true;
     cp.TB = TB;
-    cp.PC = variant_pc(v);
+    cp.PC = v.PC;
     cp.nch = (P + cp.PC - 1) / cp.PC;
-    cp.R = variant_rows(v);
+    cp.R = v.R;
     cp.variant = i;
     cp.smem = smem;
     return cp;
@@ -638,7 +620,8 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   a.err = di.err;
   const int64_t grid = (int64_t)cp.nch * cpc;
   void *args[] = {&tmap, &a};
-  return launch_maybe_pdl(var.fn, dim3((unsigned)grid), dim3(1024), cp.smem, s, args, true);
+  return launch_maybe_pdl(var.fn, dim3((unsigned)grid), dim3(var.THREADS), cp.smem, s, args,
+                          true);
 }
 
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,

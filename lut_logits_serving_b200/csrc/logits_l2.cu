@@ -108,8 +108,8 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         }
       }
     } else if (FMT == RQ_CODES_SCHED) {
-      // chunk-major [P/32][V][32]; 32 entries (i << 12 | c << 2) per chunk,
-      // any order within each 16-entry group
+      // chunk-major [P/32][V][32]; 32 entries (i << 10 | c) per chunk slice,
+      // in any order
       const uint16_t *cbase = static_cast<const uint16_t *>(a.codes) + v * 32;
       const int nc = a.P / 32;
       const bool kfull = K >= 1024;       // every 10-bit code indexes a real entry
@@ -128,8 +128,8 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const uint32_t e = (j & 1) ? (wd[j >> 1] >> 16) : (wd[j >> 1] & 0xFFFFu);
-          const uint32_t c = (e >> 2) & 0x3FFu;
-          const uint32_t pp = (uint32_t)(j & 16) + (e >> 12);   // pair within the chunk
+          const uint32_t c = e & 0x3FFu;
+          const uint32_t pp = (e >> 10) & 31u;                 // pair within the chunk
           if (kfull || c < (uint32_t)K) add_vec<VW>(tc + ((size_t)pp * K + c) * Bs, acc);
         }
       }
@@ -208,8 +208,8 @@ __global__ void __launch_bounds__(256) logits_generic_kernel(const L2Args a, int
       if (fmt == RQ_CODES_SCHED) {
         const uint32_t e =
             static_cast<const uint16_t *>(a.codes)[((size_t)(p >> 5) * a.V + v) * 32 + (p & 31)];
-        const uint32_t c = (e >> 2) & 0x3FFu;
-        const int pp = (p & ~15) + (int)(e >> 12);
+        const uint32_t c = e & 0x3FFu;
+        const int pp = (p & ~31) + (int)((e >> 10) & 31u);
         if (c < (uint32_t)a.K) z += __ldg(tl + ((size_t)pp * a.K + c) * a.Bs);
         continue;
       }

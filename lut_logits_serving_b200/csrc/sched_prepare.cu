@@ -2,11 +2,11 @@
 //
 // Not from the pages: a layout of this library for the lookup+sum logits
 // pass ("Gemma-2 runtime compression: NF4 + LUT serving", LUT section).  In
-// the batch-1 pass a warp handles 16 rows x 2 groups of 16 pairs (one lane
-// per row and group), one table lookup per lane per step, from a shared-
+// the batch-1 pass a warp handles 32 rows x one 32-pair chunk (one lane per
+// row), one table lookup per lane per step, from a shared-
 // memory table whose bank for code c is c mod 32.  A step costs as many
 // shared-memory passes as its most repeated bank; with the codes in their
-// natural order that is ~3.5 for random codes.  Here each lane's 16 codes
+// natural order that is ~3.5 for random codes.  Here each lane's 32 codes
 // are reordered so that every step is, as far as possible, a matching of
 // lanes to distinct banks: step by step, a maximum bipartite matching
 // (augmenting paths, Kuhn's method) between the lanes and the banks of
@@ -17,30 +17,29 @@
 // Any order gives the same logits up to fp32 summation order; only the
 // speed depends on it.
 //
-// Entry format: (i << 12) | (c << 2), i = pair position in the group,
-// c = code (< 1024).  For a 4-byte table entry per code and a 4 KB table
-// per pair laid out back to back, the entry is the byte offset itself.
-// Layout: chunk-major [P/32][V][32], so the 32-pair slice that one CTA of
-// the batch-1 pass streams is contiguous in memory.
+// Entry format: (i << 10) | c, i = pair position in the 32-pair chunk,
+// c = code (< 1024): for 1024-entry tables laid out back to back it is the
+// word offset of the table entry.  Layout: chunk-major [P/32][V][32], so the
+// 32-pair slice that one CTA of the batch-1 pass streams is contiguous.
 #include "rq_common.cuh"
 
 namespace rq {
 
-constexpr int kSchedThreads = 32;   // one problem per thread, state in smem
+constexpr int kSchedThreads = 16;   // one problem per thread, state in smem
 
 __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
     const uint16_t *__restrict__ codes, int64_t V, int P, uint16_t *__restrict__ out,
     unsigned long long *stats) {
-  __shared__ uint16_t s_code[kSchedThreads][32][16];   // codes of each lane
+  __shared__ uint16_t s_code[kSchedThreads][32][32];   // codes of each lane (row)
   __shared__ uint32_t s_lmask[kSchedThreads][32];      // per bank: lanes with unused codes in it
   __shared__ int8_t s_lbank[kSchedThreads][32];        // lane -> matched bank
   const int T = threadIdx.x;
-  uint16_t(*cd)[16] = s_code[T];
+  uint16_t(*cd)[32] = s_code[T];
   uint32_t *bm = s_lmask[T];
   int8_t *lbank = s_lbank[T];
 
-  const int nch = (P + 31) / 32;
-  const int64_t nrb = (V + 15) / 16;
+  const int nch = P / 32;
+  const int64_t nrb = (V + 31) / 32;
   const int64_t prob = (int64_t)blockIdx.x * kSchedThreads + T;
   if (prob >= nrb * nch) return;
   const int64_t rb = prob / nch;
@@ -49,28 +48,27 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
   uint32_t present = 0;
   uint32_t used[32];
   for (int ln = 0; ln < 32; ++ln) {
-    const int64_t row = rb * 16 + (ln >> 1);
-    const int grp = 2 * c + (ln & 1);
+    const int64_t row = rb * 32 + ln;
     used[ln] = 0;
-    if (row < V && grp * 16 < P) {
+    if (row < V) {
       present |= 1u << ln;
-      const uint16_t *src = codes + row * P + grp * 16;
-      for (int k = 0; k < 16; ++k) cd[ln][k] = src[k] & 0x3FFu;
+      const uint16_t *src = codes + row * P + c * 32;
+      for (int k = 0; k < 32; ++k) cd[ln][k] = src[k] & 0x3FFu;
     }
   }
 
   unsigned long long passes = 0;
-  for (int step = 0; step < 16; ++step) {
+  for (int step = 0; step < 32; ++step) {
     // per bank: lanes holding an unused code in it, and how many such codes
     int deg[32];
     for (int b = 0; b < 32; ++b) {
-      bm[b] = 0u;   // here: lane mask of bank b
+      bm[b] = 0u;
       deg[b] = 0;
     }
     for (int ln = 0; ln < 32; ++ln) {
       lbank[ln] = -1;
       if (!((present >> ln) & 1)) continue;
-      for (int k = 0; k < 16; ++k)
+      for (int k = 0; k < 32; ++k)
         if (!((used[ln] >> k) & 1)) {
           const int b = cd[ln][k] & 31;
           bm[b] |= 1u << ln;
@@ -129,11 +127,11 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
       if (!((present >> ln) & 1)) continue;
       int pick = -1;
       if (lbank[ln] >= 0) {
-        for (int k = 0; k < 16 && pick < 0; ++k)
+        for (int k = 0; k < 32 && pick < 0; ++k)
           if (!((used[ln] >> k) & 1) && (cd[ln][k] & 31) == lbank[ln]) pick = k;
       } else {
         int bc = 1 << 30, bd = -1;
-        for (int k = 0; k < 16; ++k)
+        for (int k = 0; k < 32; ++k)
           if (!((used[ln] >> k) & 1)) {
             const int b = cd[ln][k] & 31;
             if (cnt[b] < bc || (cnt[b] == bc && deg[b] > bd)) {
@@ -145,23 +143,22 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
         cnt[cd[ln][pick] & 31] += 1;
       }
       used[ln] |= 1u << pick;
-      const int64_t row = rb * 16 + (ln >> 1);
+      const int64_t row = rb * 32 + ln;
       // chunk-major: chunk c of every row is one contiguous [V][32] block
-      out[((int64_t)c * V + row) * 32 + (ln & 1) * 16 + step] =
-          (uint16_t)((pick << 12) | ((uint32_t)cd[ln][pick] << 2));
+      out[((int64_t)c * V + row) * 32 + step] = (uint16_t)((pick << 10) | cd[ln][pick]);
     }
     for (int b = 0; b < 32; ++b) maxc = cnt[b] > maxc ? cnt[b] : maxc;
     passes += (unsigned long long)maxc;
   }
   if (stats) {
-    atomicAdd(stats + 0, 16ull);
+    atomicAdd(stats + 0, 32ull);
     atomicAdd(stats + 1, passes);
   }
 }
 
 cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, uint16_t *out,
                                  unsigned long long *stats, cudaStream_t s) {
-  const int64_t probs = (V + 15) / 16 * ((P + 31) / 32);
+  const int64_t probs = (V + 31) / 32 * (P / 32);
   const int64_t blocks = (probs + kSchedThreads - 1) / kSchedThreads;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   if (stats) {
