@@ -296,11 +296,10 @@ def run_ours(args, w):
                          device="cuda")
 
         def step():
-            # logits of this step's hidden states, then the input rows of the
-            # tokens it picked (the next step's embeddings), rebuilt on demand
-            rq.rq_logits_from_hidden(dh, dC, codes, fmt, d, w.softcap, logits=logits,
-                                     argmax=am, ws=ws)
-            rq.rq_decode_rows(am, codes, fmt, dC, d, w.decode_scale, out=rows)
+            # logits of this step's hidden states, the greedy picks, and the
+            # input rows of the picked tokens (the next step's embeddings)
+            rq.rq_greedy_step(dh, dC, codes, fmt, d, w.softcap, scale=w.decode_scale,
+                              logits=logits, argmax=am, rows=rows, ws=ws)
         return step
 
     def graphed(step):
@@ -407,11 +406,12 @@ def run_ours(args, w):
     assert torch.equal(am.long().cpu(), logits.argmax(dim=1).cpu()), "argmax/logits mismatch"
     assert rq.rq_device_error() == 0
 
-    # decode + (build, tiled pass, reduce) or (build + pass per token group) + argmax finalize
+    # (build, tiled pass, reduce) or (build + pass per token group), then the
+    # argmax finish that also rebuilds the picked rows
     if w.B <= 4 and not w.packed10:
-        launches_per_step = 1 + 1 + 1 + 1
+        launches_per_step = 3 + 1
     else:
-        launches_per_step = 1 + 2 * ((w.B + 31) // 32) + 1
+        launches_per_step = 2 * ((w.B + 31) // 32) + 1
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

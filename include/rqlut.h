@@ -175,6 +175,23 @@ RQ_API int rq_logits_from_hidden(const float *h, const float *C, const void *cod
                           size_t ws_bytes, void *stream);
 
 /*
+ * rq_greedy_step -- one greedy decoding step of the output head in one call:
+ * rq_logits_from_hidden with argmax, then the bf16 input rows of the picked
+ * tokens (the embeddings the next step consumes), rebuilt on demand as in
+ * rq_decode_rows (LUT serving section: output logits by lookup + sum, input
+ * rows reconstructed for the ids of the step).  The row rebuild runs inside
+ * the kernel that finishes the argmax.
+ *   logits (device) float [B][V] or NULL; argmax (device) int32 [B] and
+ *   rows (device) uint16 bf16 [B][D] are required; scale as rq_decode_rows;
+ *   ws as rq_logits_from_hidden (rq_fused_workspace_bytes(d, B, fmt, 1)).
+ * Errors: as rq_logits_from_hidden.
+ */
+RQ_API int rq_greedy_step(const float *h, const float *C, const void *codes, int fmt,
+                          rq_dims d, int B, float softcap, float *logits, int32_t *argmax,
+                          float scale, uint16_t *rows, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/*
  * rq_decode_rows -- rebuild input-embedding rows on demand (LUT serving
  * section: input token rows are reconstructed for the ids of a prompt, not
  * for the whole vocabulary).
@@ -183,8 +200,9 @@ RQ_API int rq_logits_from_hidden(const float *h, const float *C, const void *cod
  *   Gemma-2 uses scale = sqrt(D).
  *   ids    (device) int32 [N]; ids outside [0, V) give zero rows and set
  *          RQ_DEVERR_BAD_ID
- *   codes  (device) as for rq_lut_logits; C (device) float [M][L][K][ds]
- *   out    (device) uint16 [N][D] bf16 bit patterns, 4-byte aligned
+ *   codes  (device) as for rq_lut_logits (2-byte aligned; 16-byte for
+ *          RQ_CODES_SCHED); C (device) float [M][L][K][ds]
+ *   out    (device) uint16 [N][D] bf16 bit patterns, 2-byte aligned
  *   N = 0 is a no-op.
  * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
  */

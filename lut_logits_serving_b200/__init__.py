@@ -26,6 +26,7 @@ __all__ = [
     "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
     "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
     "rq_pack10", "rq_device_error", "rq_set_profile_events", "rq_lut_logits_static",
+    "rq_greedy_step",
 ]
 
 U16 = 0
@@ -77,6 +78,7 @@ _SIGNATURES = {
     "rq_set_profile_events": (_i, [_p, _p]),
     "rq_prepare_sched": (_i, [_p, RqDims, _p, _p, _p]),
     "rq_lut_logits_static": (_i, [_p, _i, RqDims, _p, _i, _f, _p, _p, _p]),
+    "rq_greedy_step": (_i, [_p, _p, _p, _i, RqDims, _i, _f, _p, _p, _f, _p, _p, _sz, _p]),
 }
 
 
@@ -305,3 +307,26 @@ def rq_lut_logits_static(codes, fmt: int, d: RqDims, lut, B: int, softcap: float
         float(softcap), _ptr_or_null(logits, torch.float32, "logits"),
         _ptr_or_null(argmax, torch.int32, "argmax"), _stream(stream)))
     return logits, argmax
+
+
+def rq_greedy_step(h, C, codes, fmt: int, d: RqDims, softcap: float = 30.0, scale: float = 1.0,
+                   want_logits: bool = True, logits=None, argmax=None, rows=None, ws=None,
+                   stream=None):
+    """Logits (optional), argmax and the bf16 input rows of the picked tokens.
+    Returns (logits or None, argmax int32 [B], rows bf16 [B, D], ws)."""
+    torch = _torch()
+    B = h.shape[0]
+    if want_logits and logits is None:
+        logits = _empty((B, d.V), torch.float32, h)
+    if argmax is None:
+        argmax = _empty((B,), torch.int32, h)
+    if rows is None:
+        rows = _empty((B, d.D), torch.bfloat16, h)
+    nbytes = rq_fused_workspace_bytes(d, B, fmt, True)
+    wp, wn, ws = _workspace(nbytes, h, ws)
+    _check("rq_greedy_step", lib().rq_greedy_step(
+        _cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C"),
+        _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, B, float(softcap),
+        _ptr_or_null(logits, torch.float32, "logits"), _cuda(argmax, torch.int32, "argmax"),
+        float(scale), _cuda(rows, None, "rows"), wp, wn, _stream(stream)))
+    return logits, argmax, rows, ws

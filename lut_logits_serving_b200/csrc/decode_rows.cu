@@ -11,84 +11,32 @@
 // Packing: the "Gemma-2-2B combined RQ+NF4" page stores the M=384, K=1024,
 // L=2 artifact at 3.59 bits/param, i.e. 10-bit codes; code p of a row sits
 // at bits [10p, 10p+10) of the row's little-endian bit string.
-#include <cuda_bf16.h>
-
 #include "rq_common.cuh"
 
 namespace rq {
-
-// Code of pair p of row `id` in RQ_CODES_SCHED (chunk-major [P/32][V][32],
-// entries i << 10 | c): find position p % 32 in the row's chunk slice.
-__device__ __forceinline__ uint32_t sched_code(const uint16_t *codes, int64_t V, int64_t id,
-                                               int p) {
-  const uint16_t *g = codes + ((int64_t)(p >> 5) * V + id) * 32;
-  const uint32_t want = (uint32_t)(p & 31);
-  uint32_t c = 0;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const uint32_t e = g[k];
-    if (((e >> 10) & 31u) == want) c = e & 0x3FFu;
-  }
-  return c;
-}
-
-__device__ __forceinline__ uint32_t row_code(int fmt, const uint16_t *r16, const uint8_t *r10,
-                                             const uint16_t *all16, int64_t V, int64_t id, int p) {
-  if (fmt == RQ_CODES_U16) return r16[p];
-  if (fmt == RQ_CODES_SCHED) return sched_code(all16, V, id, p);
-  return packed10_code(r10, p);
-}
 
 // Grid (N, ceil(M / 128)): one thread per (row, subspace); the L code loads,
 // then all L*ds codeword loads of a subspace are independent, so a single
 // row costs two dependent memory round trips.
 template <int DS>
-__global__ void __launch_bounds__(128) decode_rows_kernel(
-    const int32_t *__restrict__ ids, const void *__restrict__ codes, int fmt,
-    const float *__restrict__ C, int64_t V, int D, int M, int L, int K, float scale,
-    CodeFix fix, uint16_t *__restrict__ out, unsigned *err) {
+__global__ void __launch_bounds__(128) decode_rows_kernel(const int32_t *__restrict__ ids,
+                                                          const DecodeSpec a,
+                                                          uint16_t *__restrict__ out,
+                                                          unsigned *err) {
   griddep_launch_dependents();
   griddep_wait();   // the ids may be the argmax the previous kernel wrote
   const int64_t n = blockIdx.x;
   const int m = blockIdx.y * blockDim.x + threadIdx.x;
-  if (m >= M) return;
-  const int ds = DS > 0 ? DS : D / M;
-  const int P = M * L;
+  if (m >= a.M) return;
   const int32_t id = ids[n];
-  uint16_t *o = out + n * (int64_t)D + (int64_t)m * ds;
-  if (id < 0 || (int64_t)id >= V) {
-    for (int j = 0; j < ds; ++j) o[j] = 0;
+  uint16_t *orow = out + n * (int64_t)a.D;
+  if (id < 0 || (int64_t)id >= a.V) {
+    const int ds = a.D / a.M;
+    for (int j = 0; j < ds; ++j) orow[(int64_t)m * ds + j] = 0;
     if (m == 0) atomicOr(err, RQ_DEVERR_BAD_ID);
     return;
   }
-  const int64_t rb = (10LL * P + 7) / 8;
-  const uint16_t *crow16 = static_cast<const uint16_t *>(codes) + (int64_t)id * P;
-  const uint8_t *crow10 = static_cast<const uint8_t *>(codes) + (int64_t)id * rb;
-  if (DS > 0) {
-    float e[DS > 0 ? DS : 1];
-#pragma unroll
-    for (int j = 0; j < DS; ++j) e[j] = 0.f;
-    for (int l = 0; l < L; ++l) {
-      const int p = m * L + l;
-      const uint32_t c = fix(row_code(fmt, crow16, crow10, static_cast<const uint16_t *>(codes), V, id, p));
-      const float *cw = C + ((size_t)p * K + c) * DS;
-#pragma unroll
-      for (int j = 0; j < DS; ++j) e[j] = __fadd_rn(e[j], __ldg(cw + j));
-    }
-#pragma unroll
-    for (int j = 0; j < DS; ++j)
-      o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e[j], scale)));
-  } else {
-    for (int j = 0; j < ds; ++j) {
-      float e = 0.f;
-      for (int l = 0; l < L; ++l) {
-        const int p = m * L + l;
-        const uint32_t c = fix(row_code(fmt, crow16, crow10, static_cast<const uint16_t *>(codes), V, id, p));
-        e = __fadd_rn(e, __ldg(C + ((size_t)p * K + c) * ds + j));
-      }
-      o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e, scale)));
-    }
-  }
+  decode_subspace<DS>(a, id, m, orow);
 }
 
 cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt,
@@ -97,12 +45,19 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
   if (N <= 0) return cudaSuccess;
   if (N > 0x7fffffffLL) return cudaErrorInvalidValue;
   const dim3 grid((unsigned)N, (unsigned)((M + 127) / 128));
-  const CodeFix fix = make_codefix(K);
-  if (D / M == 6)
-    return pdl_launch(decode_rows_kernel<6>, grid, dim3(128), 0, s, ids, codes, fmt, C, V, D, M,
-                      L, K, scale, fix, out, err);
-  return pdl_launch(decode_rows_kernel<0>, grid, dim3(128), 0, s, ids, codes, fmt, C, V, D, M, L,
-                    K, scale, fix, out, err);
+  DecodeSpec a;
+  a.codes = codes;
+  a.fmt = fmt;
+  a.C = C;
+  a.V = V;
+  a.D = D;
+  a.M = M;
+  a.L = L;
+  a.K = K;
+  a.scale = scale;
+  a.fix = make_codefix(K);
+  if (D / M == 6) return pdl_launch(decode_rows_kernel<6>, grid, dim3(128), 0, s, ids, a, out, err);
+  return pdl_launch(decode_rows_kernel<0>, grid, dim3(128), 0, s, ids, a, out, err);
 }
 
 // One thread per group of 4 codes = 5 output bytes.

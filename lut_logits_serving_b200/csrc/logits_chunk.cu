@@ -34,7 +34,6 @@ namespace rq {
 struct ChunkArgs {
   const float *lut;   // [P][K][TB]
   float *partial;     // [nch][B][V]
-  unsigned *counter;  // reduce-kernel block counter, zeroed here
   unsigned long long *keys;  // reduce-kernel argmax keys [B], zeroed here
   int early_codes;    // fetch code tiles before waiting for the previous kernel
   int64_t V;
@@ -162,7 +161,9 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
 // in the chunk's 32 x 1024 tables at shared address `tbase`.  All 32 loads
 // are issued before any add; the sum is a tree.  The 15-bit masks keep every
 // address aligned and inside the 128 KB of tables.
-__device__ __forceinline__ float chunk32_sched_tb1(uint32_t tbase, const uint4 (&w)[4]) {
+template <int N>
+__device__ __forceinline__ float chunk32_sched_tb1(uint32_t tbase, const uint4 (&w)[N]) {
+  static_assert(N == 4, "a scheduled slice is four 16-byte vectors");
   const uint32_t ws[16] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w,
                            w[2].x, w[2].y, w[2].z, w[2].w, w[3].x, w[3].y, w[3].z, w[3].w};
   float x[32];
@@ -256,11 +257,8 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS
   if (tid == 0)
     for (int s = 0; s < NST && s < n; ++s) issue(s, s);
   if (a.early_codes) griddep_wait();
-  if (tid == 0 && blockIdx.x == 0) {
-    if (a.counter) *a.counter = 0u;
-    if (a.keys)
-      for (int b = 0; b < a.B; ++b) a.keys[b] = 0ull;
-  }
+  if (tid == 0 && blockIdx.x == 0 && a.keys)
+    for (int b = 0; b < a.B; ++b) a.keys[b] = 0ull;
 
   // table chunk c -> shared memory
   const float *src = a.lut + (size_t)c * S::PC * K * TB;
@@ -319,22 +317,32 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS
       break;
     }
     const uint32_t st = stage0 + s * S::STAGE_BYTES;
+    // Codes -> registers first, then give the stage back, so its refill (the
+    // tile NST ahead) is in flight while this tile's lookups run.
+    uint4 w[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+      if (q < nq) w[q] = ld_shared_v4(st + voff[q]);
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();                 // this warp's code reads are done
+      if (atomicAdd(&released[s], 1u) == S::WARPS - 1) {
+        released[s] = 0u;
+        if (i + NST < n && !*reinterpret_cast<volatile int *>(abort_flag)) {
+          fence_proxy_async_smem();
+          issue(i + NST, s);
+        }
+      }
+    }
     float acc[TB];
 #pragma unroll
     for (int b = 0; b < TB; ++b) acc[b] = 0.f;
     if constexpr (SCHED) {
-      uint4 w[4];                            // the row's whole 32-pair slice
-#pragma unroll
-      for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(st + voff[q]);
-      acc[0] = chunk32_sched_tb1(tt, w);
+      acc[0] = chunk32_sched_tb1(tt, w);     // the row's whole 32-pair slice
     } else {
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        if (q < nq) {
-          const uint4 w = ld_shared_v4(st + voff[q]);
-          lookup8<TB, KT>(tt + (uint32_t)q * 8 * K * TB * 4, K, w, a.fix, acc);
-        }
-      }
+      for (int q = 0; q < NQ; ++q)
+        if (q < nq) lookup8<TB, KT>(tt + (uint32_t)q * 8 * K * TB * 4, K, w[q], a.fix, acc);
     }
     if (S::TPR == 2) {
 #pragma unroll
@@ -346,18 +354,6 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS
         if (b < a.B) out[(size_t)b * a.V + v] = acc[b];
     }
     v += S::R;
-    // release the stage; the last warp re-arms it with tile i + NST
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence_block();
-      if (atomicAdd(&released[s], 1u) == S::WARPS - 1) {
-        released[s] = 0u;
-        if (i + NST < n && !*reinterpret_cast<volatile int *>(abort_flag)) {
-          fence_proxy_async_smem();
-          issue(i + NST, s);
-        }
-      }
-    }
     if (++s == NST) {
       s = 0;
       phase ^= 1u;
@@ -397,14 +393,13 @@ __device__ __forceinline__ ArgBest block_argbest(ArgBest best, ArgBest *scratch)
 }
 
 // z = sum of the nch chunk sums in chunk order; softcap; logits; argmax.
-// Grid (nblk, B).  With `argmax` set, each warp folds its best (value, index)
-// into keys[b] with one 64-bit atomicMax; the last block to finish turns
-// the keys into indices and clears them.  Rows go 4 per thread (16-byte
-// loads) when V is a multiple of 4 and the logits are 16-byte aligned.
+// Grid (nblk, B).  With `keys` set, each block folds its best (value, index)
+// into keys[b] with one 64-bit atomicMax (argmax_keys_kernel finishes).
+// Rows go 4 per thread (16-byte loads) when V is a multiple of 4 and the
+// logits are 16-byte aligned.
 __global__ void __launch_bounds__(256) reduce_partials_kernel(
     const float *__restrict__ partial, int nch, int B, int64_t V, float cap, float *logits,
-    unsigned long long *keys, unsigned *counter, int32_t *argmax) {
-  __shared__ bool last;
+    unsigned long long *keys) {
   griddep_wait();   // the partial sums come from the kernel before this one
   const int b = blockIdx.y;
   ArgBest best{-FLT_MAX, INT_MAX};
@@ -442,29 +437,49 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(
     }
   }
   griddep_launch_dependents();
-  if (argmax == nullptr) return;
+  if (keys == nullptr) return;
+  // block-wide best first: one atomic per block on the token's key
+  __shared__ unsigned long long wkey[8];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) best = arg_better(best, arg_shfl_xor(best, o));
-  if ((threadIdx.x & 31) == 0 && best.i != INT_MAX) atomicMax(keys + b, arg_key(best));
+  if ((threadIdx.x & 31) == 0) wkey[threadIdx.x >> 5] = best.i != INT_MAX ? arg_key(best) : 0ull;
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned ticket = atomicAdd(counter, 1u);
-    last = ticket == gridDim.x * gridDim.y - 1;
+    unsigned long long k = wkey[0];
+    for (int w = 1; w < (int)blockDim.x / 32; ++w) k = wkey[w] > k ? wkey[w] : k;
+    if (k) atomicMax(keys + b, k);
   }
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  for (int bb = threadIdx.x; bb < B; bb += blockDim.x) {
-    const unsigned long long k = atomicExch(keys + bb, 0ull);
-    argmax[bb] = arg_key_index(k);
-  }
-  if (threadIdx.x == 0) *counter = 0u;
 }
 
-__global__ void __launch_bounds__(256) argmax_finalize_kernel(const float *__restrict__ am_val,
+// keys[b] -> argmax[b] (and clears the key).  With `rows` set, the block then
+// rebuilds the picked token's bf16 input row (one thread per subspace).
+template <int DS>
+__global__ void __launch_bounds__(1024) argmax_keys_kernel(unsigned long long *keys,
+                                                          int32_t *argmax, DecodeSpec rs,
+                                                          uint16_t *rows) {
+  __shared__ int pick;
+  griddep_wait();
+  const int b = blockIdx.x;
+  if (threadIdx.x == 0) {
+    const unsigned long long k = keys[b];
+    keys[b] = 0ull;
+    pick = arg_key_index(k);
+    argmax[b] = pick;
+  }
+  griddep_launch_dependents();
+  if (rows == nullptr) return;
+  __syncthreads();
+  for (int m = threadIdx.x; m < rs.M; m += blockDim.x)
+    decode_subspace<DS>(rs, pick, m, rows + (int64_t)b * rs.D);
+}
+
+template <int DS>
+__global__ void __launch_bounds__(1024) argmax_finalize_kernel(const float *__restrict__ am_val,
                                                               const int *__restrict__ am_idx,
-                                                              int nblk, int32_t *argmax) {
+                                                              int nblk, int32_t *argmax,
+                                                              DecodeSpec rs, uint16_t *rows) {
+  __shared__ ArgBest wbest[32];
+  __shared__ int pick;
   griddep_wait();
   const int b = blockIdx.x;
   ArgBest best{-FLT_MAX, INT_MAX};
@@ -472,15 +487,20 @@ __global__ void __launch_bounds__(256) argmax_finalize_kernel(const float *__res
     best = arg_better(best, ArgBest{am_val[(size_t)b * nblk + k], am_idx[(size_t)b * nblk + k]});
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) best = arg_better(best, arg_shfl_xor(best, o));
-  __shared__ ArgBest wbest[8];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (lane == 0) wbest[warp] = best;
   __syncthreads();
   if (threadIdx.x == 0) {
     ArgBest r = wbest[0];
     for (int w = 1; w < (int)blockDim.x / 32; ++w) r = arg_better(r, wbest[w]);
-    argmax[b] = r.i;
+    pick = r.i == INT_MAX ? 0 : r.i;
+    argmax[b] = pick;
   }
+  griddep_launch_dependents();
+  if (rows == nullptr) return;
+  __syncthreads();
+  for (int m = threadIdx.x; m < rs.M; m += blockDim.x)
+    decode_subspace<DS>(rs, pick, m, rows + (int64_t)b * rs.D);
 }
 
 // ------------------------------------------------------------ host side
@@ -572,7 +592,7 @@ size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V) {
 
 cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
                                 int P, int K, int B, const float *lut, float *partial,
-                                unsigned *counter, unsigned long long *keys, bool early_codes,
+                                unsigned long long *keys, bool early_codes,
                                 const DevInfo &di, cudaStream_t s) {
   const Variant &var = kVariants[cp.variant];
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
@@ -603,7 +623,6 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   ChunkArgs a;
   a.lut = lut;
   a.partial = partial;
-  a.counter = counter;
   a.keys = keys;
   a.early_codes = early_codes ? 1 : 0;
   a.V = V;
@@ -626,17 +645,46 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
 
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
                                    float *logits, unsigned long long *keys, int nblk,
-                                   unsigned *counter, int32_t *argmax, bool pdl,
                                    cudaStream_t s) {
-  void *args[] = {&partial, &nch, &B, &V, &cap, &logits, &keys, &counter, &argmax};
-  return launch_maybe_pdl(reinterpret_cast<const void *>(&reduce_partials_kernel),
-                          dim3((unsigned)nblk, (unsigned)B), dim3(256), 0, s, args, pdl);
+  return pdl_launch(reduce_partials_kernel, dim3((unsigned)nblk, (unsigned)B), dim3(256), 0, s,
+                    partial, nch, B, V, cap, logits, keys);
+}
+
+static DecodeSpec no_rows() {
+  DecodeSpec r{};
+  r.M = 0;
+  r.D = 1;
+  return r;
+}
+
+// One thread per subspace of the row (up to 1024), so the rebuild costs two
+// dependent memory round trips.
+static unsigned rows_block(const DecodeSpec &rs, bool rows) {
+  if (!rows) return 32;
+  const int t = (rs.M + 31) / 32 * 32;
+  return (unsigned)(t > 1024 ? 1024 : t);
+}
+
+cudaError_t launch_argmax_keys(unsigned long long *keys, int B, int32_t *argmax,
+                               const DecodeSpec *rows_spec, uint16_t *rows, cudaStream_t s) {
+  const DecodeSpec rs = rows_spec ? *rows_spec : no_rows();
+  const dim3 blk(rows_block(rs, rows != nullptr));
+  if (rows && rs.D / rs.M == 6)
+    return pdl_launch(argmax_keys_kernel<6>, dim3((unsigned)B), blk, 0, s, keys, argmax, rs, rows);
+  return pdl_launch(argmax_keys_kernel<0>, dim3((unsigned)B), blk, 0, s, keys, argmax, rs, rows);
 }
 
 cudaError_t launch_argmax_finalize(const float *am_val, const int *am_idx, int nblk, int B,
-                                   int32_t *argmax, cudaStream_t s) {
-  return pdl_launch(argmax_finalize_kernel, dim3((unsigned)B), dim3(256), 0, s, am_val, am_idx,
-                    nblk, argmax);
+                                   int32_t *argmax, const DecodeSpec *rows_spec, uint16_t *rows,
+                                   cudaStream_t s) {
+  const DecodeSpec rs = rows_spec ? *rows_spec : no_rows();
+  unsigned t = rows_block(rs, rows != nullptr);
+  if (t < 256) t = 256;
+  if (rows && rs.D / rs.M == 6)
+    return pdl_launch(argmax_finalize_kernel<6>, dim3((unsigned)B), dim3(t), 0, s, am_val, am_idx,
+                      nblk, argmax, rs, rows);
+  return pdl_launch(argmax_finalize_kernel<0>, dim3((unsigned)B), dim3(t), 0, s, am_val, am_idx,
+                    nblk, argmax, rs, rows);
 }
 
 }  // namespace rq

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -51,6 +52,84 @@ __device__ __forceinline__ uint32_t packed10_code(const uint8_t *row, int p) {
   const int byte = bit >> 3;
   const uint32_t w = (uint32_t)row[byte] | ((uint32_t)row[byte + 1] << 8);
   return (w >> (bit & 7)) & 0x3FFu;
+}
+
+// Code of pair p of row `id` in RQ_CODES_SCHED (chunk-major [P/32][V][32],
+// entries i << 10 | c): find position p % 32 in the row's chunk slice.
+__device__ __forceinline__ uint32_t sched_code(const uint16_t *codes, int64_t V, int64_t id,
+                                               int p) {
+  // the slice is 64 bytes at a 64-byte aligned offset: four 16-byte loads
+  const uint4 *g = reinterpret_cast<const uint4 *>(codes + ((int64_t)(p >> 5) * V + id) * 32);
+  const uint32_t want = (uint32_t)(p & 31);
+  uint32_t c = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = __ldg(g + q);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (((w[k] >> 10) & 31u) == want) c = w[k] & 0x3FFu;
+      if (((w[k] >> 26) & 31u) == want) c = (w[k] >> 16) & 0x3FFu;
+    }
+  }
+  return c;
+}
+
+// Everything the input-row rebuild needs ("Gemma-2 runtime compression: NF4
+// + LUT serving", LUT section: input rows are reconstructed on demand).
+struct DecodeSpec {
+  const void *codes;
+  int fmt;
+  const float *C;
+  int64_t V;
+  int D, M, L, K;
+  float scale;
+  CodeFix fix;
+};
+
+// Subspace m of input row `id`:
+//   out[j] = bf16_rne( fp32( fp32(sum_l C[m][l][c_l][j]) * scale ) ),  j < ds,
+// level sum in l order with explicit round-to-nearest fp32 operations.
+template <int DS>
+__device__ __forceinline__ void decode_subspace(const DecodeSpec &a, int64_t id, int m,
+                                                uint16_t *out_row) {
+  const int ds = DS > 0 ? DS : a.D / a.M;
+  const int P = a.M * a.L;
+  const int64_t rb = (10LL * P + 7) / 8;
+  const uint16_t *all16 = static_cast<const uint16_t *>(a.codes);
+  const uint16_t *crow16 = all16 + id * P;
+  const uint8_t *crow10 = static_cast<const uint8_t *>(a.codes) + id * rb;
+  uint16_t *o = out_row + (int64_t)m * ds;
+  auto code = [&](int p) -> uint32_t {
+    uint32_t c;
+    if (a.fmt == RQ_CODES_U16) c = crow16[p];
+    else if (a.fmt == RQ_CODES_SCHED) c = sched_code(all16, a.V, id, p);
+    else c = packed10_code(crow10, p);
+    return a.fix(c);
+  };
+  if (DS > 0) {
+    float e[DS > 0 ? DS : 1];
+#pragma unroll
+    for (int j = 0; j < DS; ++j) e[j] = 0.f;
+    for (int l = 0; l < a.L; ++l) {
+      const int p = m * a.L + l;
+      const float *cw = a.C + ((size_t)p * a.K + code(p)) * DS;
+#pragma unroll
+      for (int j = 0; j < DS; ++j) e[j] = __fadd_rn(e[j], __ldg(cw + j));
+    }
+#pragma unroll
+    for (int j = 0; j < DS; ++j)
+      o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e[j], a.scale)));
+  } else {
+    for (int j = 0; j < ds; ++j) {
+      float e = 0.f;
+      for (int l = 0; l < a.L; ++l) {
+        const int p = m * a.L + l;
+        e = __fadd_rn(e, __ldg(a.C + ((size_t)p * a.K + code(p)) * ds + j));
+      }
+      o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e, a.scale)));
+    }
+  }
 }
 
 // ---------------------------------------------------------- shared memory
@@ -277,14 +356,17 @@ size_t chunk_partial_bytes(const ChunkPlan &cp, int B, int64_t V);
 // so the code tiles may be fetched before waiting for it.
 cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt, int64_t V,
                                 int P, int K, int B, const float *lut, float *partial,
-                                unsigned *counter, unsigned long long *keys, bool early_codes,
+                                unsigned long long *keys, bool early_codes,
                                 const DevInfo &di, cudaStream_t s);
-// Sums the chunk partials, softcap, logits; with `argmax` set also the
-// argmax (block partials in am_val/am_idx, finished by the last block).
+// Sums the chunk partials, softcap, logits; with `keys` set also folds each
+// block's best (value, index) into keys[b] (finished by launch_argmax_keys).
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
                                    float *logits, unsigned long long *keys, int nblk,
-                                   unsigned *counter, int32_t *argmax, bool pdl,
                                    cudaStream_t s);
+// keys -> argmax[b] (keys cleared); with `rows` set, also rebuilds the bf16
+// input row of each picked token (the next step's embeddings).
+cudaError_t launch_argmax_keys(unsigned long long *keys, int B, int32_t *argmax,
+                               const DecodeSpec *rows_spec, uint16_t *rows, cudaStream_t s);
 
 // Batched pass with the LUT read through L2 (token groups of <= 32).
 cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K,
@@ -294,6 +376,7 @@ cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K
 int l2_grid_blocks(int64_t V, const DevInfo &di);
 
 cudaError_t launch_argmax_finalize(const float *am_val, const int *am_idx, int nblk, int B,
-                                   int32_t *argmax, cudaStream_t s);
+                                   int32_t *argmax, const DecodeSpec *rows_spec, uint16_t *rows,
+                                   cudaStream_t s);
 
 }  // namespace rq

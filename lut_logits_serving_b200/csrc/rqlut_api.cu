@@ -95,13 +95,14 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 int status_of(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
 
 // Workspace layout of rq_lut_logits:
-//   [partials: nch*B*V floats (small-batch path only)][am_val][am_idx]
+//   tiled path (B <= 4):  [partials: nch*B*V floats][argmax keys: B x u64]
+//   token-group path:     [argmax block partials: values][indices]
 struct WsLayout {
   bool chunk;
   ChunkPlan cp;
   size_t partial_off, partial_bytes;
   size_t amv_off, ami_off, am_bytes;   // argmax block partials (token-group path)
-  size_t keys_off, counter_off;         // argmax keys + counter (tiled path)
+  size_t keys_off;                      // argmax keys (tiled path)
   size_t total;
 };
 
@@ -119,8 +120,6 @@ WsLayout ws_layout(const rq_dims &d, int B, int fmt, bool want_argmax, const Dev
   if (want_argmax && w.chunk) {
     w.keys_off = off;
     off += (size_t)align_up((int64_t)B * 8, kAlign);
-    w.counter_off = off;
-    off += kAlign;
   } else if (want_argmax) {
     w.am_bytes = (size_t)B * kMaxSweepBlocks * 4;
     w.amv_off = off;
@@ -143,45 +142,86 @@ int sweep_blocks(const rq_dims &d, const DevInfo &di, bool chunk) {
   return l2_grid_blocks(d.V, di);
 }
 
-// Path shared by rq_lut_logits and rq_logits_from_hidden.
+// Path shared by rq_lut_logits, rq_logits_from_hidden and rq_greedy_step.
 // `after_build`: the kernel just before is this library's table build (which
 // writes nothing the code stream reads), so the tiled pass may overlap it.
+// `rows_spec`/`rows`: also rebuild the input rows of the picked tokens.
 int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, int B, int Bs,
                float cap, float *logits, int32_t *argmax, unsigned char *ws,
-               const WsLayout &w, const DevInfo &di, cudaStream_t s, bool after_build) {
+               const WsLayout &w, const DevInfo &di, cudaStream_t s, bool after_build,
+               const DecodeSpec *rows_spec = nullptr, uint16_t *rows = nullptr) {
   const int P = d.M * d.L;
   const int nblk = sweep_blocks(d, di, w.chunk);
   cudaError_t e;
   if (w.chunk) {
     float *partial = reinterpret_cast<float *>(ws + w.partial_off);
-    unsigned *counter = argmax ? reinterpret_cast<unsigned *>(ws + w.counter_off) : nullptr;
     unsigned long long *keys =
         argmax ? reinterpret_cast<unsigned long long *>(ws + w.keys_off) : nullptr;
     if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
     const bool prof = t_prof_start != nullptr;   // events between kernels break the overlap
-    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, counter, keys,
+    e = launch_logits_chunk(w.cp, codes, fmt, d.V, P, d.K, B, lut, partial, keys,
                             after_build && !prof, di, s);
     if (e != cudaSuccess) return status_of(e);
     if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
-    e = launch_reduce_partials(partial, w.cp.nch, B, d.V, cap, logits, keys, nblk, counter,
-                               argmax, true, s);
-    return status_of(e);
-  } else {
-    float *amv = argmax ? reinterpret_cast<float *>(ws + w.amv_off) : nullptr;
-    int *ami = argmax ? reinterpret_cast<int *>(ws + w.ami_off) : nullptr;
-    if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
-    for (int b0 = 0; b0 < B; b0 += kTokenGroup) {
-      const int nb = B - b0 < kTokenGroup ? B - b0 : kTokenGroup;
-      e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, b0, b0, nb, cap, logits, amv, ami,
-                           nblk, s);
-      if (e != cudaSuccess) return status_of(e);
-    }
-    if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
-    if (argmax) {
-      e = launch_argmax_finalize(amv, ami, nblk, B, argmax, s);
-      if (e != cudaSuccess) return status_of(e);
-    }
+    e = launch_reduce_partials(partial, w.cp.nch, B, d.V, cap, logits, keys, nblk, s);
+    if (e != cudaSuccess) return status_of(e);
+    if (argmax) return status_of(launch_argmax_keys(keys, B, argmax, rows_spec, rows, s));
+    return RQ_OK;
   }
+  float *amv = argmax ? reinterpret_cast<float *>(ws + w.amv_off) : nullptr;
+  int *ami = argmax ? reinterpret_cast<int *>(ws + w.ami_off) : nullptr;
+  if ((e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
+  for (int b0 = 0; b0 < B; b0 += kTokenGroup) {
+    const int nb = B - b0 < kTokenGroup ? B - b0 : kTokenGroup;
+    e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, b0, b0, nb, cap, logits, amv, ami,
+                         nblk, s);
+    if (e != cudaSuccess) return status_of(e);
+  }
+  if ((e = prof_mark(t_prof_stop, s)) != cudaSuccess) return status_of(e);
+  if (argmax) return status_of(launch_argmax_finalize(amv, ami, nblk, B, argmax, rows_spec, rows, s));
+  return RQ_OK;
+}
+
+int fused_group(int B) { return B <= 4 ? B : (B < kTokenGroup ? B : kTokenGroup); }
+
+// rq_logits_from_hidden and rq_greedy_step: table build per token group,
+// code pass, softcap, logits/argmax, optionally the picked tokens' rows.
+int run_fused(const float *h, const float *C, const void *codes, int fmt, const rq_dims &d, int B,
+              float softcap, float *logits, int32_t *argmax, void *ws, size_t ws_bytes,
+              const DecodeSpec *rows_spec, uint16_t *rows, cudaStream_t s) {
+  DevInfo di;
+  if (dev_info(&di) != cudaSuccess) return RQ_ERR_CUDA;
+  const int G = fused_group(B);
+  const int Bs = rq_lut_token_stride(G);
+  if ((size_t)Bs * (d.D / d.M) * 4 > 48 * 1024) return RQ_ERR_UNSUPPORTED;
+  const size_t lut_bytes = (size_t)align_up((int64_t)rq_lut_bytes(d, G), kAlign);
+  const WsLayout w = ws_layout(d, B, fmt, argmax != nullptr, di);
+  if (ws_bytes < lut_bytes + w.total) return RQ_ERR_WORKSPACE_TOO_SMALL;
+  float *lut = static_cast<float *>(ws);
+  unsigned char *rest = static_cast<unsigned char *>(ws) + lut_bytes;
+  if (w.chunk) {
+    // B <= 4: one table for all tokens, then the vocabulary-tiled pass
+    cudaError_t e = launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut, s);
+    if (e != cudaSuccess) return status_of(e);
+    return run_logits(codes, fmt, d, lut, B, Bs, softcap, logits, argmax, rest, w, di, s, true,
+                      rows_spec, rows);
+  }
+  const int P = d.M * d.L;
+  float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
+  int *ami = argmax ? reinterpret_cast<int *>(rest + w.ami_off) : nullptr;
+  const int nblk = sweep_blocks(d, di, false);
+  for (int b0 = 0; b0 < B; b0 += G) {
+    const int nb = B - b0 < G ? B - b0 : G;
+    cudaError_t e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, s);
+    if (e != cudaSuccess) return status_of(e);
+    if (b0 == 0 && (e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
+    e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, 0, b0, nb, softcap, logits, amv, ami,
+                         nblk, s);
+    if (e != cudaSuccess) return status_of(e);
+  }
+  if (cudaError_t e = prof_mark(t_prof_stop, s)) return status_of(e);
+  if (argmax)
+    return status_of(launch_argmax_finalize(amv, ami, nblk, B, argmax, rows_spec, rows, s));
   return RQ_OK;
 }
 
@@ -225,8 +265,6 @@ size_t rq_logits_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax) {
   if (!dims_ok(d) || !fmt_ok(d, fmt) || B < 1) return 0;
   return ws_layout(d, B, fmt, want_argmax != 0, nominal_devinfo()).total;
 }
-
-static int fused_group(int B) { return B <= 4 ? B : (B < kTokenGroup ? B : kTokenGroup); }
 
 size_t rq_fused_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax) {
   if (!dims_ok(d) || !fmt_ok(d, fmt) || B < 1) return 0;
@@ -273,39 +311,34 @@ int rq_logits_from_hidden(const float *h, const float *C, const void *codes, int
   if (!aligned(h, 4) || !aligned(C, 4) || !aligned(codes, 16) || !aligned(ws, 16) ||
       (logits && !aligned(logits, 4)) || (argmax && !aligned(argmax, 4)))
     return RQ_ERR_MISALIGNED;
-  DevInfo di;
-  if (dev_info(&di) != cudaSuccess) return RQ_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int G = fused_group(B);
-  const int Bs = rq_lut_token_stride(G);
-  if ((size_t)Bs * (d.D / d.M) * 4 > 48 * 1024) return RQ_ERR_UNSUPPORTED;
-  const size_t lut_bytes = (size_t)align_up((int64_t)rq_lut_bytes(d, G), kAlign);
-  const WsLayout w = ws_layout(d, B, fmt, argmax != nullptr, di);
-  if (ws_bytes < lut_bytes + w.total) return RQ_ERR_WORKSPACE_TOO_SMALL;
-  float *lut = static_cast<float *>(ws);
-  unsigned char *rest = static_cast<unsigned char *>(ws) + lut_bytes;
-  if (w.chunk) {
-    // B <= 4: one table for all tokens, then the vocabulary-tiled pass
-    cudaError_t e = launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut, s);
-    if (e != cudaSuccess) return status_of(e);
-    return run_logits(codes, fmt, d, lut, B, Bs, softcap, logits, argmax, rest, w, di, s, true);
-  }
-  const int P = d.M * d.L;
-  float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
-  int *ami = argmax ? reinterpret_cast<int *>(rest + w.ami_off) : nullptr;
-  const int nblk = sweep_blocks(d, di, false);
-  for (int b0 = 0; b0 < B; b0 += G) {
-    const int nb = B - b0 < G ? B - b0 : G;
-    cudaError_t e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, s);
-    if (e != cudaSuccess) return status_of(e);
-    if (b0 == 0 && (e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
-    e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, 0, b0, nb, softcap, logits, amv, ami,
-                         nblk, s);
-    if (e != cudaSuccess) return status_of(e);
-  }
-  if (cudaError_t e = prof_mark(t_prof_stop, s)) return status_of(e);
-  if (argmax) return status_of(launch_argmax_finalize(amv, ami, nblk, B, argmax, s));
-  return RQ_OK;
+  return run_fused(h, C, codes, fmt, d, B, softcap, logits, argmax, ws, ws_bytes, nullptr,
+                   nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int rq_greedy_step(const float *h, const float *C, const void *codes, int fmt, rq_dims d, int B,
+                   float softcap, float *logits, int32_t *argmax, float scale, uint16_t *rows,
+                   void *ws, size_t ws_bytes, void *stream) {
+  if (!h || !C || !codes || !argmax || !rows || B < 1 || !dims_ok(d))
+    return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_known(fmt)) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
+  if (!ws) return RQ_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned(h, 4) || !aligned(C, 4) || !aligned(codes, 16) || !aligned(ws, 16) ||
+      (logits && !aligned(logits, 4)) || !aligned(argmax, 4) || !aligned(rows, 2))
+    return RQ_ERR_MISALIGNED;
+  DecodeSpec rs;
+  rs.codes = codes;
+  rs.fmt = fmt;
+  rs.C = C;
+  rs.V = d.V;
+  rs.D = d.D;
+  rs.M = d.M;
+  rs.L = d.L;
+  rs.K = d.K;
+  rs.scale = scale;
+  rs.fix = make_codefix(d.K);
+  return run_fused(h, C, codes, fmt, d, B, softcap, logits, argmax, ws, ws_bytes, &rs, rows,
+                   static_cast<cudaStream_t>(stream));
 }
 
 int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt, const float *C,
@@ -315,7 +348,8 @@ int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt, co
   if (!ids || !codes || !C || !out) return RQ_ERR_INVALID_ARGUMENT;
   if (!fmt_known(fmt)) return RQ_ERR_INVALID_ARGUMENT;
   if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
-  if (!aligned(ids, 4) || !aligned(codes, 2) || !aligned(C, 4) || !aligned(out, 2))
+  if (!aligned(ids, 4) || !aligned(codes, fmt == RQ_CODES_SCHED ? 16 : 2) || !aligned(C, 4) ||
+      !aligned(out, 2))
     return RQ_ERR_MISALIGNED;
   DevInfo di;
   if (dev_info(&di) != cudaSuccess) return RQ_ERR_CUDA;

@@ -65,6 +65,14 @@ def test_g2_batch1_full_sweep(g2):
     err3 = assert_logits_close(logits3.cpu().numpy(), ref)
     print(f"g2_b1 sched normwise error {err3:.3g}")
     assert check_argmax(am3.cpu().numpy(), ref) == 0
+    # the benchmark's step: logits, argmax and the picked token's input row
+    logits4, am4, rows4, _ = rq.rq_greedy_step(dev(h), g2["dC"], sched, rq.SCHED, d, w.softcap,
+                                               scale=w.decode_scale)
+    assert torch.equal(am4, am3)
+    assert_logits_close(logits4.cpu().numpy(), ref)
+    want = oracle.decode_rows_bf16(am4.cpu().numpy().astype(np.int32), g2["codes"], g2["C"],
+                                   w.decode_scale)
+    assert np.array_equal(rows4.view(torch.int16).cpu().numpy().view(np.uint16), want)
     assert rq.rq_device_error() == 0
 
 

@@ -296,3 +296,26 @@ def test_prepare_sched_rejects_unsupported_shapes():
         rq.rq_prepare_sched(c2, d2)
     with pytest.raises(rq.RqError):            # in place is refused
         rq.rq_prepare_sched(c2, rq.dims(100, 64, 32, 1, 1024), out=c2)
+
+
+# ------------------------------------------------------------ greedy step
+
+@pytest.mark.parametrize("B", [1, 3, 5, 33])
+@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["u16", "packed10", "sched"])
+def test_greedy_step_rows_are_the_picked_tokens_rows(B, fmt):
+    V, D, M, L, K = 3000, 192, 32, 2, 256
+    C, codes, h = make_case(V, D, M, L, K, B, seed=B)
+    d = rq.dims(V, D, M, L, K)
+    dc = gpu_codes(codes, fmt, d)
+    ref = oracle_logits(C, codes, h, 30.0)
+    logits, am, rows, _ = rq.rq_greedy_step(dev(h), dev(C), dc, fmt, d, 30.0, scale=8.0)
+    assert_logits_close(logits.cpu().numpy(), ref)
+    check_argmax(am.cpu().numpy(), ref)
+    ids = am.cpu().numpy().astype(np.int32)
+    want = oracle.decode_rows_bf16(ids, codes, C, 8.0)
+    assert np.array_equal(rows.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    # without logits: same picks and rows
+    _, am2, rows2, _ = rq.rq_greedy_step(dev(h), dev(C), dc, fmt, d, 30.0, scale=8.0,
+                                         want_logits=False)
+    assert torch.equal(am2, am) and torch.equal(rows2, rows)
+    assert rq.rq_device_error() == 0
