@@ -108,21 +108,29 @@ __global__ void __launch_bounds__(256) lut_build_ds6_kernel(const float *__restr
   }
 }
 
-// ds = 6, token groups of 4..64 (Bs % 4 == 0): one thread per (codeword,
-// 4 tokens); a warp writes 8 codewords x 32 tokens... as contiguous float4
-// runs, so the 100 MB table of a 32-token group streams out coalesced.
+// ds = 6, token groups (Bs % 4 == 0): grid (K*Bs/4/256, P), one pair per
+// block so the block's hidden slice h[b0..b0+Bs][m*6..m*6+6] is staged once in
+// shared memory; one thread per (codeword, 4 tokens) writes a float4, a warp
+// 8 codewords x 32 tokens... as contiguous runs.
 __global__ void __launch_bounds__(256) lut_build_ds6_tok_kernel(
     const float *__restrict__ h, const float *__restrict__ C, int b0, int nb, int D, int L, int K,
-    int Bs, int items, float *__restrict__ lut) {
+    int Bs, float *__restrict__ lut) {
+  __shared__ float hs[64][6];
   griddep_wait();
-  // items < 2^31 (checked by the launcher): 32-bit index math
-  const int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g < items) {
-    const int q = Bs / 4;
-    const int e = g / q;                     // codeword p*K + k
-    const int t0 = (g - e * q) * 4;          // first token of this thread
-    const int m = e / K / L;
-    const float *cw = C + (size_t)e * 6;
+  const int p = blockIdx.y;
+  const int m = p / L;
+  for (int i = threadIdx.x; i < Bs * 6; i += blockDim.x) {
+    const int t = i / 6, j = i % 6;
+    hs[t][j] = t < nb ? __ldg(h + (size_t)(b0 + t) * D + m * 6 + j) : 0.f;
+  }
+  __syncthreads();
+  const int q = Bs / 4;
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;   // (k, token quad) within the pair
+  if (g < K * q) {
+    const int k = g / q;
+    const int t0 = (g - k * q) * 4;
+    const size_t e = (size_t)p * K + k;
+    const float *cw = C + e * 6;
     const float2 c01 = __ldg(reinterpret_cast<const float2 *>(cw));
     const float2 c23 = __ldg(reinterpret_cast<const float2 *>(cw + 2));
     const float2 c45 = __ldg(reinterpret_cast<const float2 *>(cw + 4));
@@ -130,16 +138,12 @@ __global__ void __launch_bounds__(256) lut_build_ds6_tok_kernel(
     float r[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int t = t0 + i;
       float acc = 0.f;
-      if (t < nb) {
-        const float *hm = h + (size_t)(b0 + t) * D + m * 6;
 #pragma unroll
-        for (int j = 0; j < 6; ++j) acc = fmaf(__ldg(hm + j), c[j], acc);
-      }
+      for (int j = 0; j < 6; ++j) acc = fmaf(hs[t0 + i][j], c[j], acc);
       r[i] = acc;
     }
-    *reinterpret_cast<float4 *>(lut + (size_t)e * Bs + t0) = make_float4(r[0], r[1], r[2], r[3]);
+    *reinterpret_cast<float4 *>(lut + e * Bs + t0) = make_float4(r[0], r[1], r[2], r[3]);
   }
   griddep_launch_dependents();
 }
@@ -149,13 +153,13 @@ cudaError_t launch_lut_build(const float *h, const float *C, int B, int b0, int 
   (void)B;
   const int ds = D / M;
   const int P = M * L;
-  if (ds == 6 && Bs % 4 == 0 && (reinterpret_cast<uintptr_t>(C) & 7) == 0 &&
+  if (ds == 6 && Bs % 4 == 0 && Bs <= 64 && (reinterpret_cast<uintptr_t>(C) & 7) == 0 &&
       (reinterpret_cast<uintptr_t>(lut) & 15) == 0) {
-    const int64_t items = (int64_t)P * K * (Bs / 4);
-    const int64_t blocks = (items + 255) / 256;
-    if (items < 0x7fffffffLL - 256)
-      return pdl_launch(lut_build_ds6_tok_kernel, dim3((unsigned)blocks), dim3(256), 0, s, h, C,
-                        b0, nb, D, L, K, Bs, (int)items, lut);
+    const int64_t items = (int64_t)K * (Bs / 4);     // per pair
+    const int64_t bx = (items + 255) / 256;
+    if (items < 0x7fffffffLL - 256 && P <= 65535)
+      return pdl_launch(lut_build_ds6_tok_kernel, dim3((unsigned)bx, (unsigned)P), dim3(256), 0, s,
+                        h, C, b0, nb, D, L, K, Bs, lut);
   }
   if (ds == 6 && Bs <= 2 && K % 4 == 0 && (reinterpret_cast<uintptr_t>(C) & 15) == 0 &&
       (reinterpret_cast<uintptr_t>(lut) & 15) == 0) {
