@@ -42,7 +42,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="g2_b1", choices=["g2_b1", "g2_b32", "packed_b64"])
+    ap.add_argument("--workload", default="g2_b1",
+                    choices=["g2_b1", "g2_b32", "packed_b64", "mlp_gate_b1", "mlp_down_b1"])
     ap.add_argument("--codes", default="sched", choices=["u16", "sched"],
                     help="uint16 code layout of the unpacked workloads timed for `value`: "
                          "bank-scheduled once by rq_prepare_sched (the serving layout), or as "
@@ -54,16 +55,20 @@ def parse():
 
 
 def workload_config(w, codes="u16"):
-    fmt = "packed10 (960 B/row)" if w.packed10 else (
-        "uint16 (1536 B/row)" if codes == "u16" else
-        "uint16 (1536 B/row) in the bank-scheduled order of rq_prepare_sched")
+    rb = w.P * 10 // 8 if w.packed10 else w.P * 2
+    fmt = f"packed10 ({rb} B/row)" if w.packed10 else (
+        f"uint16 ({rb} B/row)" if codes == "u16" else
+        f"uint16 ({rb} B/row) in the bank-scheduled order of rq_prepare_sched")
+    what = (f"softcap {w.softcap:g}, logits + argmax, then the {w.B} picked tokens' input rows "
+            f"rebuilt (bf16)") if w.argmax else "y = W x, no softcap (RQ-coded MLP weight)"
     return {
         "workload": f"{w.name}: V={w.V} D={w.D} M={w.M} L={w.L} K={w.K} B={w.B}, {fmt} codes, "
-                    f"softcap {w.softcap:g}, logits + argmax, then the {w.B} picked tokens' input "
-                    f"rows rebuilt (bf16)",
+                    f"{what}",
         "V": w.V, "D": w.D, "M": w.M, "L": w.L, "K": w.K, "B": w.B,
         "codes": "packed10" if w.packed10 else codes,
-        "l2": "inputs larger than L2: the 393 MB / 246 MB code matrix is streamed every step",
+        "l2": ("inputs larger than L2: the code matrix is streamed from HBM every step"
+               if (w.V * (w.P * 10 // 8 if w.packed10 else w.P * 2)) > 2 * 126 * 2**20 else
+               "inputs smaller than L2: a 256 MB buffer is written between timed steps"),
     }
 
 
@@ -295,6 +300,12 @@ def run_ours(args, w):
         ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
                          device="cuda")
 
+        if not w.argmax:
+            def step():
+                # an RQ-coded weight matrix applied without reconstruction
+                rq.rq_logits_from_hidden(dh, dC, codes, fmt, d, w.softcap, logits=logits, ws=ws)
+            return step
+
         def step():
             # logits of this step's hidden states, the greedy picks, and the
             # input rows of the picked tokens (the next step's embeddings)
@@ -322,17 +333,36 @@ def run_ours(args, w):
         torch.cuda.synchronize()
         return g.replay, g
 
+    # Inputs smaller than twice the 126 MB L2 would stay cached between steps:
+    # then every step is timed by its own event pair and a 256 MB buffer is
+    # written between steps, outside the pairs.
+    flush = None
+    if code_bytes(w) + data["C"].nbytes < 2 * 126 * 2**20:
+        flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
+
     def time_steps(run, n):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(n):
-            run()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        if flush is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                run()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+        else:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(n)]
+            for a0, a1 in evs:
+                flush.fill_(1)
+                a0.record(stream)
+                run()
+                a1.record(stream)
+            torch.cuda.synchronize()
+            ms = sum(a0.elapsed_time(a1) for a0, a1 in evs)
         barrier()
-        return max_over_ranks(e0.elapsed_time(e1))
+        return max_over_ranks(ms)
 
     def code_pass_us(step, n):
         """Device time of the code-streaming pass alone (profile events
@@ -343,6 +373,8 @@ def run_ours(args, w):
             ev.record(stream)
         torch.cuda.synchronize()
         for i in range(n):
+            if flush is not None:
+                flush.fill_(1)
             rq.rq_set_profile_events(starts[i], stops[i])
             step()
         rq.rq_set_profile_events(None, None)
@@ -393,28 +425,30 @@ def run_ours(args, w):
         dh.copy_(h_host, non_blocking=True)
         step()
         out_host.copy_(logits, non_blocking=True)
-        am_host.copy_(am, non_blocking=True)
+        if w.argmax:
+            am_host.copy_(am, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
     e_ms = time_steps(e2e_step, ne2e)
     e2e_value = throughput(w.V * w.B * ne2e, world, e_ms)
     h2d = data["h"].nbytes
-    d2h = w.B * w.V * 4 + w.B * 4
+    d2h = w.B * w.V * 4 + (w.B * 4 if w.argmax else 0)
 
     # the argmax must agree with the logits it came from
-    assert torch.equal(am.long().cpu(), logits.argmax(dim=1).cpu()), "argmax/logits mismatch"
+    if w.argmax:
+        assert torch.equal(am.long().cpu(), logits.argmax(dim=1).cpu()), "argmax/logits mismatch"
     assert rq.rq_device_error() == 0
 
     # (build, tiled pass, reduce) or (build + pass per token group), then the
     # argmax finish that also rebuilds the picked rows
     if w.B <= 4 and not w.packed10:
-        launches_per_step = 3 + 1
+        launches_per_step = 3 + (1 if w.argmax else 0)
     else:
-        launches_per_step = 2 * ((w.B + 31) // 32) + 1
+        launches_per_step = 2 * ((w.B + 31) // 32) + (1 if w.argmax else 0)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.argmax:
         cpu = cpu_baseline(w, data, args.cpu_seconds)
 
     if world > 1:

@@ -61,6 +61,15 @@ WORKLOADS = {
     "packed_b64": Workload("packed_b64", V=256000, D=2304, M=384, L=2, K=1024, B=64,
                            sigmas=(0.02, 0.005), hidden_scale=0.83, packed10=True,
                            argmax=True, n_ids=64, decode_scale=math.sqrt(2304.0)),
+    # RQ-compressed MLP weights of a Gemma-2-2B layer, applied without
+    # reconstruction (the follow-up the MLP-RQ page names): y = W x with
+    # W [out x in], ds = 2, L = 2 and K chosen per matrix for ~10 bits/param
+    # including the per-subspace codebooks (L*log2(K)/ds + L*K*32/out):
+    # gate/up 8 + 1.8 = 9.8, down 7 + 3.6 = 10.6.
+    "mlp_gate_b1": Workload("mlp_gate_b1", V=9216, D=2304, M=1152, L=2, K=256, B=1,
+                            sigmas=(0.02, 0.005), hidden_scale=1.0, softcap=0.0),
+    "mlp_down_b1": Workload("mlp_down_b1", V=2304, D=9216, M=4608, L=2, K=128, B=1,
+                            sigmas=(0.02, 0.005), hidden_scale=1.0, softcap=0.0),
 }
 
 

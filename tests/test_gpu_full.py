@@ -124,3 +124,22 @@ def test_decode512_bit_exact(g2, fmt):
     got = out.view(torch.int16).cpu().numpy().view(np.uint16)
     want = oracle.decode_rows_bf16(ids, g2["codes"], g2["C"], w.decode_scale)
     assert np.array_equal(got, want)
+
+
+# ------------------------------------------------- RQ MLP matvec (no softcap)
+
+@pytest.mark.parametrize("name", ["mlp_gate_b1", "mlp_down_b1"])
+@pytest.mark.parametrize("fmt", [0, 2], ids=["u16", "sched"])
+def test_rq_mlp_matvec(name, fmt):
+    """y = W x for an RQ-coded MLP weight W [out x in] (ds = 2, about 10 bits/param with the codebooks):
+    the same lookup + sum with V = out features and the softcap off."""
+    w = synth.WORKLOADS[name]
+    d = rq.dims(w.V, w.D, w.M, w.L, w.K)
+    data = synth.make(w)
+    C, codes, h = data["C"], data["codes"], data["h"]
+    c16 = dev(codes.reshape(w.V, -1))
+    dc = c16 if fmt == rq.U16 else rq.rq_prepare_sched(c16, d)
+    y, _, _ = rq.rq_logits_from_hidden(dev(h), dev(C), dc, fmt, d, 0.0)
+    ref = oracle.logits_direct(codes, C, h)        # the plain definition: W x
+    err = assert_logits_close(y.cpu().numpy(), ref)
+    print(f"{name} normwise error {err:.3g}")

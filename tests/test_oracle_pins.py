@@ -323,3 +323,15 @@ def test_zipf_ids_shape_and_repeats():
     assert ids.dtype == np.int32 and ids.shape == (512,)
     assert ids.min() >= 0 and ids.max() < 256000
     assert np.unique(ids).size < 512        # heavy head: repeats occur
+
+
+def test_mlp_workloads_hit_about_ten_bits_per_param():
+    """The MLP-RQ page targets ~10 bits/param per matrix, codebooks included
+    (its first fixed-K attempt cost 16.72 for down_proj); the synthetic MLP
+    shapes are chosen that way."""
+    for name, lo, hi in (("mlp_gate_b1", 9.0, 11.0), ("mlp_down_b1", 9.0, 11.0)):
+        w = synth.WORKLOADS[name]
+        code_bits = w.V * w.M * w.L * math.log2(w.K)
+        book_bits = w.M * w.L * w.K * w.ds * 32
+        bpp = (code_bits + book_bits) / (w.V * w.D)
+        assert lo < bpp < hi, (name, bpp)
