@@ -7,7 +7,7 @@ here.
 
 Seeds: one ``numpy.random.default_rng`` stream per tensor, derived from a
 base seed: codebooks = seed, codes = seed + 1, hidden states = seed + 2,
-token ids = seed + 3.
+token ids = seed + 3, rows to encode = seed + 4.
 """
 from __future__ import annotations
 
@@ -34,6 +34,7 @@ class Workload:
     n_ids: int = 0              # input rows rebuilt per call
     zipf_s: float = 1.1
     decode_scale: float = 0.0   # embedding scale applied to rebuilt rows
+    encode: bool = False        # the call encodes V rows instead of scoring them
 
     @property
     def ds(self) -> int:
@@ -70,6 +71,11 @@ WORKLOADS = {
                             sigmas=(0.02, 0.005), hidden_scale=1.0, softcap=0.0),
     "mlp_down_b1": Workload("mlp_down_b1", V=2304, D=9216, M=4608, L=2, K=128, B=1,
                             sigmas=(0.02, 0.005), hidden_scale=1.0, softcap=0.0),
+    # Producing the codes: all 256000 embedding rows encoded against the
+    # artifact's codebooks (rows ~ N(0, sqrt(0.02^2 + 0.005^2)), the spread of
+    # a row the two levels describe).
+    "encode_g2": Workload("encode_g2", V=256000, D=2304, M=384, L=2, K=1024, B=0,
+                          sigmas=(0.02, 0.005), hidden_scale=0.0, encode=True),
 }
 
 
@@ -109,6 +115,22 @@ def zipf_ids(N: int, V: int, s: float = 1.1, seed: int = 3) -> np.ndarray:
     return perm[r].astype(np.int32)
 
 
+def rows(N: int, D: int, sigma: float, seed: int = 4, chunk: int = 16384) -> np.ndarray:
+    """float32 [N, D] ~ N(0, sigma), drawn in row chunks of one stream."""
+    rng = np.random.default_rng(seed)
+    out = np.empty((N, D), np.float32)
+    for r0 in range(0, N, chunk):
+        r1 = min(N, r0 + chunk)
+        out[r0:r1] = rng.standard_normal((r1 - r0, D), dtype=np.float32)
+        out[r0:r1] *= np.float32(sigma)
+    return out
+
+
+def row_sigma(w: Workload) -> float:
+    """Spread of a row whose levels have std sigmas[l]."""
+    return float(math.sqrt(sum(s * s for s in w.sigmas)))
+
+
 def make(w: Workload, seed: int = 0, V: int | None = None):
     """All inputs of a workload: dict with C, codes, h, ids (V may be cut for
     a smaller sample of the same distributions)."""
@@ -121,4 +143,7 @@ def make(w: Workload, seed: int = 0, V: int | None = None):
         out["h"] = hidden(w.B, w.D, w.hidden_scale, seed + 2)
     if w.n_ids > 0:
         out["ids"] = zipf_ids(w.n_ids, V, w.zipf_s, seed + 3)
+    if w.encode:
+        del out["codes"]
+        out["X"] = rows(V, w.D, row_sigma(w), seed + 4)
     return out

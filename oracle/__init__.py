@@ -20,6 +20,9 @@ RQ shape paragraph):
 * ``argmax``: lowest index of the maximum
 * ``decode_rows_bf16``: bf16_rne(fp32(fp32(sum_l C[m,l,c_l,j]) * scale))
 * ``pack10`` / ``unpack10``: 10-bit codes, little-endian bit stream per row
+* ``encode``: greedy residual nearest-codeword codes of rows X (per subspace,
+  level by level, fp32 squared distances accumulated with fma in dimension
+  order, lowest index on ties, fp32 residual update)
 """
 from __future__ import annotations
 
@@ -73,6 +76,7 @@ def _load():
         "rqo_packed10_row_bytes": (_i64, [_i]),
         "rqo_pack10": (None, [_p, _i64, _i, _p]),
         "rqo_unpack10": (None, [_p, _i64, _i, _p]),
+        "rqo_encode_f32": (None, [_p, _i64, _p, _i, _i, _i, _i, _p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -226,6 +230,19 @@ def unpack10(packed: np.ndarray, P: int) -> np.ndarray:
     assert packed.shape[1] == packed10_row_bytes(P)
     out = np.empty((V, P), np.uint16)
     lib.rqo_unpack10(_ptr(packed), V, P, _ptr(out))
+    return out
+
+
+def encode(X: np.ndarray, C: np.ndarray) -> np.ndarray:
+    """codes uint16 [N, M, L] of rows X [N, D] against codebooks C [M, L, K, ds]."""
+    lib = _load()
+    X = _c(np.atleast_2d(X), np.float32)
+    C = _c(C, np.float32)
+    M, L, K, ds = _dims(C)
+    N, D = X.shape
+    assert D == M * ds and ds <= 64 and K <= 65536
+    out = np.empty((N, M, L), np.uint16)
+    lib.rqo_encode_f32(_ptr(X), N, _ptr(C), D, M, L, K, _ptr(out))
     return out
 
 

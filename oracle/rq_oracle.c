@@ -40,6 +40,18 @@
  *   packed uint8  [V][ceil(10*M*L/8)] (10-bit codes, little-endian bit
  *                                      stream per row, code j in bits
  *                                      [10j, 10j+10))
+ *   X      float  [N][D]              (rows to encode)
+ *
+ * Encoder.  The pages call the embedding compression residual product
+ * quantization and give no assignment rule ("Gemma-2-2B combined RQ+NF4",
+ * RQ paragraph).  The plain reading, used here: per subspace, level 0 takes
+ * the nearest codeword of the subspace's level-0 codebook, and each later
+ * level the nearest codeword to what the earlier levels left over (the
+ * residual).  "Nearest" is a decision taken in fp32: the squared distance
+ * is accumulated over j = 0..ds-1 in order as acc = fma(t, t, acc) with
+ * t = r[j] - c[j] rounded to fp32 (fmaf is exactly rounded, so the result
+ * is fixed by IEEE 754), ties go to the lowest codeword index, and the
+ * residual is updated as r[j] = r[j] - c[j] in fp32.
  */
 #include <math.h>
 #include <stdint.h>
@@ -276,5 +288,41 @@ void rqo_unpack10(const uint8_t *packed, int64_t V, int P, uint16_t *codes)
                 c |= ((byte >> (bit % 8)) & 1u) << t;
             }
             codes[(size_t)v * P + j] = (uint16_t)c;
+        }
+}
+
+/* ----------------------------------------------------------------- encoder */
+
+/* codes[n][m][l] = greedy residual nearest-codeword assignment of row n
+ * (definition in the file header). */
+void rqo_encode_f32(const float *X, int64_t N, const float *C, int D, int M,
+                    int L, int K, uint16_t *codes)
+{
+    int ds = D / M;
+    float r[64];
+    for (int64_t n = 0; n < N; ++n)
+        for (int m = 0; m < M; ++m) {
+            for (int j = 0; j < ds; ++j)
+                r[j] = X[n * D + (int64_t)m * ds + j];
+            for (int l = 0; l < L; ++l) {
+                const float *book = C + ((size_t)m * L + l) * K * ds;
+                int best = 0;
+                float bestd = INFINITY;
+                for (int k = 0; k < K; ++k) {
+                    const float *cw = book + (size_t)k * ds;
+                    float acc = 0.0f;
+                    for (int j = 0; j < ds; ++j) {
+                        float t = r[j] - cw[j];
+                        acc = fmaf(t, t, acc);
+                    }
+                    if (acc < bestd) {
+                        bestd = acc;
+                        best = k;
+                    }
+                }
+                codes[(n * M + m) * L + l] = (uint16_t)best;
+                for (int j = 0; j < ds; ++j)
+                    r[j] = r[j] - book[(size_t)best * ds + j];
+            }
         }
 }

@@ -1,6 +1,7 @@
 """Planted mistakes: each mutation below is a plausible slip in the oracle
 (transposed operand, dropped term, wrong sign, wrong index split, wrong
-rounding, wrong bit order, wrong tie-break, wrong softcap).  A mutated copy
+rounding, wrong bit order, wrong tie-break, wrong softcap, encoder
+residual / codebook / sign slips).  A mutated copy
 of the oracle source is compiled on the CPU and the pin checks must catch
 every one of them.  The oracle itself is never modified."""
 import os
@@ -27,6 +28,12 @@ MUTATIONS = {
     "argmax_last_tie": ("if (y[i] > y[best])", "if (y[i] >= y[best])"),
     "softcap_inverted": ("cap * tanh(y[i] / cap)", "cap * tanh(y[i] * cap)"),
     "decode_scale_before_sum": ("float s = e * scale;", "float s = e * scale * scale;"),
+    "encode_no_residual": ("r[j] = r[j] - book[(size_t)best * ds + j];",
+                           "r[j] = r[j] - 0.0f * book[(size_t)best * ds + j];"),
+    "encode_last_tie": ("if (acc < bestd) {", "if (acc <= bestd) {"),
+    "encode_level0_book": ("C + ((size_t)m * L + l) * K * ds;", "C + ((size_t)m * L) * K * ds;"),
+    "encode_plus_sign": ("float t = r[j] - cw[j];", "float t = r[j] + cw[j];"),
+    "encode_subspace_offset": ("X[n * D + (int64_t)m * ds + j]", "X[n * D + (int64_t)m + j]"),
 }
 
 
@@ -41,6 +48,9 @@ def _checks(golden_dir):
         pins.check_softcap,
         pins.check_argmax,
         lambda: pins.check_pages_fp32_identity(nrows=40),
+        pins.check_encode_brute_force,
+        pins.check_encode_vq,
+        pins.check_encode_planted,
     ]
 
 
@@ -67,7 +77,7 @@ def test_mutation_is_caught(name, golden_dir, monkeypatch, tmp_path):
                 "rqo_logits_lut_f32", "rqo_logits_direct_f64", "rqo_logits_direct_f32",
                 "rqo_softcap_f64", "rqo_argmax_f32", "rqo_argmax_f64",
                 "rqo_f32_to_bf16_rne", "rqo_decode_rows_bf16", "rqo_packed10_row_bytes",
-                "rqo_pack10", "rqo_unpack10"):
+                "rqo_pack10", "rqo_unpack10", "rqo_encode_f32"):
         src, dst = getattr(real, sym), getattr(lib, sym)
         dst.restype, dst.argtypes = src.restype, src.argtypes
     monkeypatch.setattr(oracle, "_lib", lib)

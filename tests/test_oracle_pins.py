@@ -229,6 +229,87 @@ def check_pages_fp32_identity(nrows=400):
     return rel
 
 
+# ------------------------------------------------------------------ encoder
+# The encoder oracle takes its nearest-codeword decisions in fp32 (squared
+# distance accumulated with fma over the subspace's dims, lowest index on
+# ties).  The pins below reach the same decisions another way: fp64 brute
+# force and a library nearest-centroid routine agree with it wherever the
+# fp64 margin between the two nearest codewords exceeds the fp32 rounding of
+# a ds-term sum of squares (< (ds + 2) * 2^-24 relative), and planted rows
+# whose answer is known exactly.
+
+def _nearest_f64(R, book):
+    d = ((R.astype(np.float64)[:, None, :] - book.astype(np.float64)[None]) ** 2).sum(-1)
+    order = np.argsort(d, axis=1, kind="stable")
+    n = np.arange(R.shape[0])
+    return order[:, 0], d[n, order[:, 1]] - d[n, order[:, 0]], d[n, order[:, 0]]
+
+
+def check_encode_brute_force():
+    rng = np.random.default_rng(21)
+    N, M, L, K, ds = 300, 8, 3, 64, 5
+    C = np.stack([rng.normal(0, 0.5 ** l, (M, K, ds)) for l in range(L)], axis=1)
+    C = C.astype(np.float32)
+    X = rng.normal(0, 1, (N, M * ds)).astype(np.float32)
+    codes = oracle.encode(X, C)
+    unsure = 0
+    for m in range(M):
+        R = X[:, m * ds:(m + 1) * ds].copy()
+        for l in range(L):
+            want, gap, dmin = _nearest_f64(R, C[m, l])
+            sure = gap > 1e-5 * dmin
+            got = codes[:, m, l].astype(np.int64)
+            assert np.array_equal(got[sure], want[sure]), (m, l)
+            unsure += int((~sure).sum())
+            # the residual the next level sees: an fp32 subtraction
+            R = (R - C[m, l][got]).astype(np.float32)
+    assert unsure < 0.01 * N * M * L
+
+
+def check_encode_vq():
+    from scipy.cluster.vq import vq
+    rng = np.random.default_rng(22)
+    N, M, K, ds = 500, 6, 128, 4
+    C = rng.normal(0, 1, (M, 1, K, ds)).astype(np.float32)
+    X = rng.normal(0, 1, (N, M * ds)).astype(np.float32)
+    codes = oracle.encode(X, C)
+    for m in range(M):
+        R = X[:, m * ds:(m + 1) * ds]
+        want, _ = vq(R.astype(np.float64), C[m, 0].astype(np.float64), check_finite=False)
+        _, gap, dmin = _nearest_f64(R, C[m, 0])
+        sure = gap > 1e-5 * dmin
+        assert np.array_equal(codes[sure, m, 0], want[sure])
+
+
+def check_encode_planted():
+    rng = np.random.default_rng(23)
+    M, K, ds, N = 5, 64, 6, 200
+    # L = 1, rows made of codewords: every distance but the planted one is > 0
+    C1 = rng.normal(0, 1, (M, 1, K, ds)).astype(np.float32)
+    a = rng.integers(0, K, (N, M))
+    X1 = np.concatenate([C1[m, 0][a[:, m]] for m in range(M)], axis=1)
+    assert np.array_equal(oracle.encode(X1, C1)[:, :, 0], a)
+    # L = 2 with a small second level: level 0 finds a, and only the residual
+    # (not the row) leads level 1 to b
+    C2 = np.stack([rng.normal(0, 1, (M, K, ds)), rng.normal(0, 1e-3, (M, K, ds))], axis=1)
+    C2 = C2.astype(np.float32)
+    b = rng.integers(0, K, (N, M))
+    X2 = np.concatenate([(C2[m, 0][a[:, m]] + C2[m, 1][b[:, m]]).astype(np.float32)
+                         for m in range(M)], axis=1)
+    got = oracle.encode(X2, C2)
+    assert np.array_equal(got[:, :, 0], a)
+    assert np.array_equal(got[:, :, 1], b)
+    # ties: a duplicated codeword goes to its lower index; a constant
+    # codebook gives code 0 everywhere
+    C3 = C2.copy()
+    C3[:, 0, 41] = C3[:, 0, 17]
+    C3[:, 1] = 0.25
+    X3 = np.concatenate([np.repeat(C3[m, 0][41][None], 3, 0) for m in range(M)], axis=1)
+    got3 = oracle.encode(X3, C3)
+    assert np.all(got3[:, :, 0] == 17)
+    assert np.all(got3[:, :, 1] == 0)
+
+
 def check_sizes():
     """Artifact sizes printed on the pages pin the layout we read:
     u16 codes [V][M][L] + fp32 codebooks [M][L][K][ds]."""
@@ -335,3 +416,15 @@ def test_mlp_workloads_hit_about_ten_bits_per_param():
         book_bits = w.M * w.L * w.K * w.ds * 32
         bpp = (code_bits + book_bits) / (w.V * w.D)
         assert lo < bpp < hi, (name, bpp)
+
+
+def test_encode_brute_force():
+    check_encode_brute_force()
+
+
+def test_encode_vq():
+    check_encode_vq()
+
+
+def test_encode_planted():
+    check_encode_planted()
