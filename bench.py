@@ -34,6 +34,11 @@ from lut_logits_serving_b200 import synth  # noqa: E402
 
 METRIC = "LUT logits vocab-rows/s & µs/call at V=256000 (1 B200), % of HBM roofline"
 UNIT = "vocab-rows/s"
+ENC_METRIC = "RQ encode rows/s (greedy residual nearest codeword, fp32), % of FP32-pipe roofline"
+ENC_UNIT = "rows/s"
+# FP32 pipe: 148 SMs x 128 lanes per clock (B200); the clock is the sampled
+# maximum (clocks.max.sm), 1965 MHz when no sample exists.
+SMS, FP32_LANES, NOMINAL_SM_MHZ = 148, 128, 1965.0
 
 
 def parse():
@@ -43,7 +48,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="g2_b1",
-                    choices=["g2_b1", "g2_b32", "packed_b64", "mlp_gate_b1", "mlp_down_b1"])
+                    choices=["g2_b1", "g2_b32", "packed_b64", "mlp_gate_b1", "mlp_down_b1",
+                             "encode_g2"])
     ap.add_argument("--codes", default="sched", choices=["u16", "sched"],
                     help="uint16 code layout of the unpacked workloads timed for `value`: "
                          "bank-scheduled once by rq_prepare_sched (the serving layout), or as "
@@ -183,10 +189,53 @@ def cpu_baseline(w, data, seconds):
                       f"softcap, argmax, row decode), single-threaded C, {el:.1f} s"}
 
 
+def encode_terms(w, rows):
+    """Distance terms (one fp32 subtract + one fma each) of encoding `rows`."""
+    return rows * w.M * w.L * w.K * w.ds
+
+
+def run_reference_encode(args, w):
+    import oracle
+    data = synth.make(w, V=4096)
+    X, C = data["X"], data["C"]
+    t0 = time.perf_counter()
+    oracle.encode(X[:4], C)
+    per_row = (time.perf_counter() - t0) / 4
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    nrows = int(max(1, min(X.shape[0], budget / max(per_row, 1e-9))))
+    for _ in range(args.warmup):
+        oracle.encode(X[:nrows], C)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.encode(X[:nrows], C)
+    el = time.perf_counter() - t0
+    value = nrows * args.steps / el
+    line = {
+        "impl": "reference", "metric": ENC_METRIC, "value": value, "unit": ENC_UNIT,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": encode_config(w),
+        "cpu_baseline": {"value": value, "unit": ENC_UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{nrows} of {w.V} rows per step"},
+        "e2e": {"value": value, "unit": ENC_UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def encode_config(w):
+    return {"workload": f"{w.name}: encode V={w.V} rows of D={w.D} fp32 against M={w.M} x "
+                        f"L={w.L} codebooks of K={w.K} ({w.ds}-dim) codewords -> uint16 codes",
+            "V": w.V, "D": w.D, "M": w.M, "L": w.L, "K": w.K,
+            "l2": "inputs larger than L2: the 2.36 GB of rows are read every step"}
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    if w.encode:
+        return run_reference_encode(args, w)
     data = synth.make(w)
     step = oracle_step_fn(w, data)
     # size each step's row sample so that warmup + steps end within ~2 minutes
@@ -480,11 +529,116 @@ def run_ours(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_encode(args, w):
+    """Encode all V rows per step (rows resident on the device)."""
+    import torch
+    import torch.distributed as dist
+
+    import lut_logits_serving_b200 as rq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    data = synth.make(w, seed=rank_seed(rank))
+    d = rq.dims(w.V, w.D, w.M, w.L, w.K)
+    X = torch.from_numpy(data["X"]).cuda()
+    C = torch.from_numpy(data["C"]).cuda()
+    codes = torch.empty((w.V, w.P), dtype=torch.uint16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rq.rq_encode(X, C, d, out=codes)
+
+    def timed(fn, n):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return aggregate(e0.elapsed_time(e1), world, device="cuda")
+
+    for _ in range(args.warmup):
+        step()
+    with ClockSampler(local) as clk:
+        t_ms = timed(step, args.steps)
+    value = throughput(w.V * args.steps, world, t_ms)
+    clocks = clk.summary()
+    kern_s = t_ms / args.steps / 1e3                  # one launch per step
+    ops = 2 * encode_terms(w, w.V)
+    mhz = clocks["sm_max_mhz"] or NOMINAL_SM_MHZ
+    peak = SMS * FP32_LANES * mhz * 1e6 / 1e12
+    achieved = ops / kern_s / 1e12
+    assert rq.rq_device_error() == 0
+
+    # end to end: rows from pinned host memory, codes back to the host
+    Xh = torch.from_numpy(data["X"]).pin_memory()
+    ch = torch.empty((w.V, w.P), dtype=torch.uint16).pin_memory()
+
+    def e2e_step():
+        X.copy_(Xh, non_blocking=True)
+        step()
+        ch.copy_(codes, non_blocking=True)
+
+    e2e_step()
+    ne2e = 3
+    e_ms = timed(e2e_step, ne2e)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        n, t0, sample = 0, time.perf_counter(), 64
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            oracle.encode(data["X"][:sample], data["C"])
+            n += sample
+        el = time.perf_counter() - t0
+        cpu = {"value": n / el, "unit": ENC_UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{n} rows ({sample} per call) encoded by the C oracle, "
+                         f"single-threaded, {el:.1f} s"}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": ENC_METRIC, "value": value, "unit": ENC_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": dict(encode_config(w), parallelism=f"replicas x{world}",
+                                            launch="eager"),
+        "roofline": {"bound": "alu", "kernel": "encode_kernel<6,2>", "achieved": achieved,
+                     "peak": peak, "peak_kind": f"derived: {SMS} SMs x {FP32_LANES} FP32 lanes "
+                                                f"x {mhz:g} MHz",
+                     "unit": "T fp32 lane-ops/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_ops": ops, "kernel_us": kern_s * 1e6},
+        "cpu_baseline": cpu,
+        "e2e": {"value": throughput(w.V * ne2e, world, e_ms), "unit": ENC_UNIT,
+                "h2d_bytes_per_step": data["X"].nbytes, "d2h_bytes_per_step": w.V * w.P * 2,
+                "ms_per_step": e_ms / ne2e},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+    elif w.encode:
+        run_encode(args, w)
     else:
         run_ours(args, w)
 

@@ -221,6 +221,31 @@ RQ_API int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed,
               void *stream);
 
 /*
+ * rq_encode -- produce the codes: greedy residual nearest-codeword
+ * assignment of V rows ("Gemma-2-2B combined RQ+NF4" names the compression
+ * residual product quantization, M subspaces x L levels of K codewords,
+ * without stating the assignment; this is its plain reading).  Per row x
+ * and subspace m, with r = x[m*ds, (m+1)*ds):
+ *   for l = 0..L-1: code[v][m*L + l] = argmin_k sum_j (r_j - C[m][l][k][j])^2
+ *                   r_j -= C[m][l][code][j]
+ * The argmin is an fp32 decision: t_j = fp32(r_j - c_j), the sum
+ * accumulated j = 0..ds-1 as fma(t_j, t_j, acc), the lowest k wins ties
+ * (a NaN distance never wins: an all-NaN subspace gets code 0), and the
+ * residual update is an fp32 subtraction.  The codes are therefore
+ * reproducible bit for bit.  Training the codebooks is not part of it.
+ *   X     (device) float [V][D], 4-byte aligned (the rows; d.V of them)
+ *   C     (device) float [M][L][K][ds]
+ *   codes (device) uint16 [V][M*L] (RQ_CODES_U16), 2-byte aligned; must
+ *         not overlap X or C
+ *   V = 0 is a no-op.  Supported: ds = D/M <= 32 (ds 2, 4, 6, 8 have
+ *   specialised kernels), K <= 65536.
+ * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_UNSUPPORTED (ds > 32),
+ *         RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ */
+RQ_API int rq_encode(const float *X, rq_dims d, const float *C, uint16_t *codes,
+                     void *stream);
+
+/*
  * rq_prepare_sched -- convert uint16 codes [V][M*L] into RQ_CODES_SCHED
  * (same size; chunk-major so that each 32-pair slice streams contiguously).
  * Not on the pages: a layout of this library.  The lookups of the batch-1

@@ -26,7 +26,7 @@ __all__ = [
     "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
     "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
     "rq_pack10", "rq_device_error", "rq_set_profile_events", "rq_lut_logits_static",
-    "rq_greedy_step",
+    "rq_greedy_step", "rq_encode",
 ]
 
 U16 = 0
@@ -74,6 +74,7 @@ _SIGNATURES = {
     "rq_logits_from_hidden": (_i, [_p, _p, _p, _i, RqDims, _i, _f, _p, _p, _p, _sz, _p]),
     "rq_decode_rows": (_i, [_p, _i64, _p, _i, _p, RqDims, _f, _p, _p]),
     "rq_pack10": (_i, [_p, RqDims, _p, _p]),
+    "rq_encode": (_i, [_p, RqDims, _p, _p, _p]),
     "rq_device_error": (_i, [ctypes.POINTER(ctypes.c_uint32), _i]),
     "rq_set_profile_events": (_i, [_p, _p]),
     "rq_prepare_sched": (_i, [_p, RqDims, _p, _p, _p]),
@@ -257,6 +258,18 @@ def rq_pack10(codes_u16, d: RqDims, out=None, stream=None):
         out = _empty((d.V, rq_codes_bytes(d, PACKED10) // d.V), torch.uint8, codes_u16)
     _check("rq_pack10", lib().rq_pack10(_cuda(codes_u16, torch.uint16, "codes_u16"), d,
                                         _cuda(out, torch.uint8, "packed"), _stream(stream)))
+    return out
+
+
+def rq_encode(X, C, d: RqDims, out=None, stream=None):
+    """Rows float32 [V, D] -> uint16 codes [V, M*L]: greedy residual
+    nearest-codeword assignment against C [M, L, K, ds]."""
+    torch = _torch()
+    if out is None:
+        out = _empty((d.V, d.M * d.L), torch.uint16, X)
+    _check("rq_encode", lib().rq_encode(_cuda(X, torch.float32, "X"), d,
+                                        _cuda(C, torch.float32, "C"),
+                                        _cuda(out, torch.uint16, "codes"), _stream(stream)))
     return out
 
 

@@ -337,6 +337,8 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
 cudaError_t launch_pack10(const uint16_t *codes, int64_t V, int P, uint8_t *packed,
                           cudaStream_t s);
 
+cudaError_t launch_encode(const float *X, int64_t N, const float *C, int D, int M, int L, int K,
+                          uint16_t *codes, cudaStream_t s);
 cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, uint16_t *out,
                                  unsigned long long *stats, cudaStream_t s);
 

@@ -378,6 +378,25 @@ int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out, uint64
                                         static_cast<cudaStream_t>(stream)));
 }
 
+int rq_encode(const float *X, rq_dims d, const float *C, uint16_t *codes, void *stream) {
+  rq_dims d1 = d;
+  if (d1.V == 0) d1.V = 1;
+  if (!dims_ok(d1)) return RQ_ERR_INVALID_ARGUMENT;
+  if (d.V == 0) return RQ_OK;
+  if (!X || !C || !codes) return RQ_ERR_INVALID_ARGUMENT;
+  if (d.D / d.M > 32) return RQ_ERR_UNSUPPORTED;
+  if (!aligned(X, 4) || !aligned(C, 4) || !aligned(codes, 2)) return RQ_ERR_MISALIGNED;
+  const uintptr_t c0 = reinterpret_cast<uintptr_t>(codes);
+  const size_t cb = rq_codes_bytes(d, RQ_CODES_U16);
+  const uintptr_t x0 = reinterpret_cast<uintptr_t>(X), k0 = reinterpret_cast<uintptr_t>(C);
+  const size_t xb = (size_t)d.V * d.D * sizeof(float);
+  const size_t kb = (size_t)d.M * d.L * d.K * (d.D / d.M) * sizeof(float);
+  if ((c0 < x0 + xb && x0 < c0 + cb) || (c0 < k0 + kb && k0 < c0 + cb))
+    return RQ_ERR_INVALID_ARGUMENT;   // overlap
+  return status_of(launch_encode(X, d.V, C, d.D, d.M, d.L, d.K, codes,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
 int rq_set_profile_events(void *start, void *stop) {
   if ((start == nullptr) != (stop == nullptr)) return RQ_ERR_INVALID_ARGUMENT;
   t_prof_start = static_cast<cudaEvent_t>(start);

@@ -126,6 +126,11 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_lut_logits(a, 2, rq.dims(10, 48, 24, 1, 64), a, 1, 30.0, a, null, null, 0,
                              s) == UNS                                        # sched, P % 32
     assert lib.rq_device_error(None, 0) == INV
+    assert lib.rq_encode(null, G2, a, a, s) == INV
+    assert lib.rq_encode(null, rq.dims(0, 2304, 384, 2, 1024), null, null, s) == 0   # V = 0
+    assert lib.rq_encode(a, rq.dims(10, 66, 2, 2, 16), a, _fake(0x900000), s) == UNS   # ds 33
+    assert lib.rq_encode(_fake(0x10002), G2, a, _fake(0x90000000), s) == MIS
+    assert lib.rq_encode(a, G2, _fake(0x90000000), _fake(0x10000 + 4096), s) == INV   # overlap
 
 
 def test_python_binding_rejects_cpu_tensors():
