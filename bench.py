@@ -617,7 +617,7 @@ def run_encode(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": dict(encode_config(w), parallelism=f"replicas x{world}",
                                             launch="eager"),
-        "roofline": {"bound": "alu", "kernel": "encode_kernel<6,2>", "achieved": achieved,
+        "roofline": {"bound": "alu", "kernel": "encode_pair_kernel<6,4>", "achieved": achieved,
                      "peak": peak, "peak_kind": f"derived: {SMS} SMs x {FP32_LANES} FP32 lanes "
                                                 f"x {mhz:g} MHz",
                      "unit": "T fp32 lane-ops/s", "frac": achieved / peak, "traffic": None,
