@@ -20,6 +20,12 @@ RQ shape paragraph):
 * ``argmax``: lowest index of the maximum
 * ``decode_rows_bf16``: bf16_rne(fp32(fp32(sum_l C[m,l,c_l,j]) * scale))
 * ``pack10`` / ``unpack10``: 10-bit codes, little-endian bit stream per row
+* ``topk``: the k largest values, descending, lower index first on ties
+* ``philox4x64_10`` / ``uniform``: the counter-based generator of the
+  sampler, u = (word0 >> 11) * 2^-53 for counter (step, row, 0, 0), key
+  (seed, 0)
+* ``sample_position``: inverse CDF of the temperature softmax over the
+  sorted top-k (fp64): first i with running sum > u * total
 * ``encode``: greedy residual nearest-codeword codes of rows X (per subspace,
   level by level, fp32 squared distances accumulated with fma in dimension
   order, lowest index on ties, fp32 residual update)
@@ -77,6 +83,10 @@ def _load():
         "rqo_pack10": (None, [_p, _i64, _i, _p]),
         "rqo_unpack10": (None, [_p, _i64, _i, _p]),
         "rqo_encode_f32": (None, [_p, _i64, _p, _i, _i, _i, _i, _p]),
+        "rqo_philox4x64_10": (None, [_p, _p, _p]),
+        "rqo_uniform": (_d, [ctypes.c_uint64, ctypes.c_uint64, _i64]),
+        "rqo_topk_f32": (None, [_p, _i64, _i, _p, _p, _p]),
+        "rqo_sample_position": (_i, [_p, _i, _d, _d]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -244,6 +254,49 @@ def encode(X: np.ndarray, C: np.ndarray) -> np.ndarray:
     out = np.empty((N, M, L), np.uint16)
     lib.rqo_encode_f32(_ptr(X), N, _ptr(C), D, M, L, K, _ptr(out))
     return out
+
+
+def philox4x64_10(ctr, key) -> np.ndarray:
+    lib = _load()
+    c = _c(np.asarray(ctr, dtype=np.uint64), np.uint64)
+    k = _c(np.asarray(key, dtype=np.uint64), np.uint64)
+    out = np.empty(4, np.uint64)
+    lib.rqo_philox4x64_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def uniform(seed: int, step: int, row: int) -> float:
+    return float(_load().rqo_uniform(seed, step, row))
+
+
+def topk(y: np.ndarray, k: int):
+    """(values float32 [B, k], indices int32 [B, k]) of y [B, n] float32."""
+    lib = _load()
+    y2 = np.atleast_2d(_c(y, np.float32))
+    B, n = y2.shape
+    val = np.empty((B, k), np.float32)
+    idx = np.empty((B, k), np.int32)
+    taken = np.empty(n, np.uint8)
+    for b in range(B):
+        row = np.ascontiguousarray(y2[b])
+        vb = np.empty(k, np.float32)
+        ib = np.empty(k, np.int32)
+        lib.rqo_topk_f32(_ptr(row), n, k, _ptr(vb), _ptr(ib), _ptr(taken))
+        val[b], idx[b] = vb, ib
+    return val, idx
+
+
+def sample_position(val: np.ndarray, temperature: float, u: float) -> int:
+    v = _c(val, np.float32)
+    return int(_load().rqo_sample_position(_ptr(v), v.size, float(temperature), float(u)))
+
+
+def sample(y: np.ndarray, k: int, temperature: float, seed: int, step: int):
+    """Top-k values/indices and the sampled token of every row of y [B, n]."""
+    val, idx = topk(y, k)
+    tok = np.array([idx[b, sample_position(val[b], temperature, uniform(seed, step, b))]
+                    for b in range(val.shape[0])], np.int32)
+    return val, idx, tok
 
 
 def reference_logits(codes: np.ndarray, C: np.ndarray, h: np.ndarray, cap: float,

@@ -42,6 +42,17 @@
  *                                      [10j, 10j+10))
  *   X      float  [N][D]              (rows to encode)
  *
+ * Top-k and sampling.  The pages cap generation length and state no sampler
+ * ("Gemma-2-2B combined RQ+NF4", closing note on generation).  Plain reading for
+ * generation beyond greedy: the k largest softcapped logits (descending,
+ * the lower index first among equal values), then a draw from the
+ * temperature softmax restricted to them by inverse CDF: weights
+ * w_i = exp((y_i - y_max) / T) in sorted order, S_i their running sums, and
+ * the token is the first i with S_i > u * S_k.  The uniform u in [0, 1) is
+ * the top 53 bits of word 0 of Philox4x64-10 (Salmon et al., SC'11) with
+ * counter (step, token row, 0, 0) and key (seed, 0), times 2^-53.  The
+ * sampling arithmetic here is fp64.
+ *
  * Encoder.  The pages call the embedding compression residual product
  * quantization and give no assignment rule ("Gemma-2-2B combined RQ+NF4",
  * RQ paragraph).  The plain reading, used here: per subspace, level 0 takes
@@ -325,4 +336,73 @@ void rqo_encode_f32(const float *X, int64_t N, const float *C, int D, int M,
                     r[j] = r[j] - book[(size_t)best * ds + j];
             }
         }
+}
+
+/* ------------------------------------------------------ top-k and sampling */
+
+/* Philox4x64 with 10 rounds: the multipliers and Weyl key increments of the
+ * published generator. */
+void rqo_philox4x64_10(const uint64_t *ctr, const uint64_t *key, uint64_t *out)
+{
+    uint64_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint64_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        unsigned __int128 p0 = (unsigned __int128)c0 * 0xD2E7470EE14C6C93ull;
+        unsigned __int128 p1 = (unsigned __int128)c2 * 0xCA5A826395121157ull;
+        uint64_t hi0 = (uint64_t)(p0 >> 64), lo0 = (uint64_t)p0;
+        uint64_t hi1 = (uint64_t)(p1 >> 64), lo1 = (uint64_t)p1;
+        uint64_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = lo1;
+        c2 = n2;
+        c3 = lo0;
+        k0 += 0x9E3779B97F4A7C15ull;
+        k1 += 0xBB67AE8584CAA73Bull;
+    }
+    out[0] = c0;
+    out[1] = c1;
+    out[2] = c2;
+    out[3] = c3;
+}
+
+double rqo_uniform(uint64_t seed, uint64_t step, int64_t row)
+{
+    uint64_t ctr[4] = {step, (uint64_t)row, 0, 0}, key[2] = {seed, 0}, out[4];
+    rqo_philox4x64_10(ctr, key, out);
+    return (double)(out[0] >> 11) * (1.0 / 9007199254740992.0);
+}
+
+/* The k largest of y[0..n): repeated scans for the largest value not yet
+ * taken, the lower index winning among equal values. */
+void rqo_topk_f32(const float *y, int64_t n, int k, float *val, int32_t *idx,
+                  unsigned char *taken)
+{
+    memset(taken, 0, (size_t)n);
+    for (int i = 0; i < k; ++i) {
+        int64_t best = -1;
+        for (int64_t v = 0; v < n; ++v)
+            if (!taken[v] && (best < 0 || y[v] > y[best]))
+                best = v;
+        taken[best] = 1;
+        val[i] = y[best];
+        idx[i] = (int32_t)best;
+    }
+}
+
+/* Position (0..k-1) in the sorted top-k of the token drawn with uniform u;
+ * temperature <= 0 or k == 1 is greedy (position 0). */
+int rqo_sample_position(const float *val, int k, double temperature, double u)
+{
+    if (k <= 1 || temperature <= 0.0)
+        return 0;
+    double S = 0.0;
+    for (int i = 0; i < k; ++i)
+        S += exp(((double)val[i] - (double)val[0]) / temperature);
+    double t = u * S, cum = 0.0;
+    for (int i = 0; i < k; ++i) {
+        cum += exp(((double)val[i] - (double)val[0]) / temperature);
+        if (cum > t)
+            return i;
+    }
+    return k - 1;
 }

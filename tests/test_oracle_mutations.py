@@ -34,6 +34,12 @@ MUTATIONS = {
     "encode_level0_book": ("C + ((size_t)m * L + l) * K * ds;", "C + ((size_t)m * L) * K * ds;"),
     "encode_plus_sign": ("float t = r[j] - cw[j];", "float t = r[j] + cw[j];"),
     "encode_subspace_offset": ("X[n * D + (int64_t)m * ds + j]", "X[n * D + (int64_t)m + j]"),
+    "philox_lanes_swapped": ("c1 = lo1;", "c1 = lo0;"),
+    "philox_key_schedule": ("k1 += 0xBB67AE8584CAA73Bull;", "k1 += 0x9E3779B97F4A7C15ull;"),
+    "uniform_52_bits": ("(out[0] >> 11)", "(out[0] >> 12)"),
+    "topk_last_tie": ("(best < 0 || y[v] > y[best])", "(best < 0 || y[v] >= y[best])"),
+    "sample_ge": ("if (cum > t)", "if (cum >= t)"),
+    "sample_no_temperature": ("(double)val[0]) / temperature);\n        if", "(double)val[0]));\n        if"),
 }
 
 
@@ -51,6 +57,9 @@ def _checks(golden_dir):
         pins.check_encode_brute_force,
         pins.check_encode_vq,
         pins.check_encode_planted,
+        pins.check_philox_numpy,
+        pins.check_topk,
+        pins.check_sampling,
     ]
 
 
@@ -77,7 +86,8 @@ def test_mutation_is_caught(name, golden_dir, monkeypatch, tmp_path):
                 "rqo_logits_lut_f32", "rqo_logits_direct_f64", "rqo_logits_direct_f32",
                 "rqo_softcap_f64", "rqo_argmax_f32", "rqo_argmax_f64",
                 "rqo_f32_to_bf16_rne", "rqo_decode_rows_bf16", "rqo_packed10_row_bytes",
-                "rqo_pack10", "rqo_unpack10", "rqo_encode_f32"):
+                "rqo_pack10", "rqo_unpack10", "rqo_encode_f32",
+                "rqo_philox4x64_10", "rqo_uniform", "rqo_topk_f32", "rqo_sample_position"):
         src, dst = getattr(real, sym), getattr(lib, sym)
         dst.restype, dst.argtypes = src.restype, src.argtypes
     monkeypatch.setattr(oracle, "_lib", lib)

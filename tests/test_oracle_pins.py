@@ -310,6 +310,68 @@ def check_encode_planted():
     assert np.all(got3[:, :, 1] == 0)
 
 
+# ------------------------------------------------------- top-k and sampling
+
+def _philox_numpy(ctr, key):
+    """The same block from numpy's Philox (4x64, 10 rounds), which steps its
+    256-bit counter by one before producing each block."""
+    c = sum(int(x) << (64 * i) for i, x in enumerate(ctr)) - 1
+    words = [(c >> (64 * i)) & (2 ** 64 - 1) for i in range(4)]
+    return np.random.Philox(counter=np.array(words, np.uint64),
+                            key=np.array(key, np.uint64)).random_raw(4)
+
+
+def check_philox_numpy():
+    for ctr, key in (([1, 0, 0, 0], [0, 0]), ([7, 3, 0, 0], [12345, 0]),
+                     ([0, 5, 0, 0], [2 ** 64 - 1, 0]),
+                     ([2 ** 63 + 11, 2 ** 64 - 2, 9, 2 ** 40], [0xDEADBEEF, 0x1234])):
+        assert np.array_equal(oracle.philox4x64_10(ctr, key), _philox_numpy(ctr, key)), ctr
+    # the uniform: numpy's double from the same 64-bit word
+    for seed, step, row in ((1234, 0, 0), (1234, 17, 3), (2 ** 60 + 1, 2 ** 33, 63)):
+        c = step + (row << 64) - 1
+        words = [(c >> (64 * i)) & (2 ** 64 - 1) for i in range(4)]
+        g = np.random.Generator(np.random.Philox(counter=np.array(words, np.uint64),
+                                                 key=np.array([seed, 0], np.uint64)))
+        assert oracle.uniform(seed, step, row) == g.random()
+
+
+def check_topk():
+    rng = np.random.default_rng(31)
+    # coarse values: many exact ties, which go to the lower index
+    y = (rng.integers(-40, 40, (3, 5000)) / 8.0).astype(np.float32)
+    y[1, 4000:] = 100.0           # a tied block at the top
+    for k in (1, 7, 64, 300):
+        val, idx = oracle.topk(y, k)
+        for b in range(y.shape[0]):
+            order = np.lexsort((np.arange(y.shape[1]), -y[b].astype(np.float64)))[:k]
+            assert np.array_equal(idx[b], order)
+            assert np.array_equal(val[b], y[b, order])
+
+
+def check_sampling():
+    # equal logits: weights all exactly 1, running sums 1..k, so u = (j + f)/k
+    # (0 <= f < 1) draws position j
+    k = 10
+    val = np.full(k, 2.5, np.float32)
+    for j in range(k):
+        for f in (0.0, 0.25, 0.999):
+            assert oracle.sample_position(val, 0.7, (j + f) / k) == j
+    # greedy cases
+    v = np.array([3.0, 2.0, 1.0], np.float32)
+    assert oracle.sample_position(v, 0.0, 0.99) == 0
+    assert oracle.sample_position(v[:1], 1.0, 0.99) == 0
+    # frequencies over many counters follow the temperature softmax
+    from scipy.special import softmax
+    from scipy.stats import chisquare
+    v = np.array([1.0, 0.6, 0.5, -0.2, -1.5], np.float32)
+    T = 0.8
+    n = 20000
+    pos = [oracle.sample_position(v, T, oracle.uniform(99, s, 0)) for s in range(n)]
+    obs = np.bincount(pos, minlength=v.size)
+    exp_ = softmax(v.astype(np.float64) / T) * n
+    assert chisquare(obs, exp_).pvalue > 1e-6
+
+
 def check_sizes():
     """Artifact sizes printed on the pages pin the layout we read:
     u16 codes [V][M][L] + fp32 codebooks [M][L][K][ds]."""
@@ -428,3 +490,15 @@ def test_encode_vq():
 
 def test_encode_planted():
     check_encode_planted()
+
+
+def test_philox_numpy():
+    check_philox_numpy()
+
+
+def test_topk():
+    check_topk()
+
+
+def test_sampling():
+    check_sampling()
