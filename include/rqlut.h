@@ -221,6 +221,34 @@ RQ_API int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed,
               void *stream);
 
 /*
+ * rq_topk_sample -- top-k of softcapped logits and a temperature draw among
+ * them (generation beyond greedy argmax; the pages state no sampler, see the
+ * "Gemma-2-2B combined RQ+NF4" note on generation, so this is the plain
+ * reading).  Per token row b of logits [B][V]:
+ *   topk_val[b][i], topk_idx[b][i], i < k: the k largest logits, descending,
+ *     the lower vocabulary index first among equal values (-0 equals +0;
+ *     NaN logits are not supported);
+ *   token[b]: with T > 0 and k > 1, w_i = exp((y_i - y_0) / T) in fp64 over
+ *     the sorted top-k, and token = topk_idx[b][i] for the first i whose
+ *     running sum of w exceeds u * sum(w), where u = (word0 >> 11) * 2^-53,
+ *     word0 the first output word of Philox4x64-10 (Salmon et al., SC'11) for
+ *     counter (step, b, 0, 0) and key (seed, 0); T <= 0 or k = 1: the top
+ *     index (greedy).
+ *   logits   (device) float [B][V], 4-byte aligned (e.g. rq_lut_logits')
+ *   topk_val (device) float [B][k] or NULL; topk_idx (device) int32 [B][k]
+ *            or NULL; token (device) int32 [B] or NULL
+ *   ws       (device) workspace of rq_topk_workspace_bytes(V, B, k) bytes,
+ *            256-byte aligned; contents need no initialisation
+ * Supported: 1 <= k <= min(V, 1024), 1 <= B <= 65535.
+ * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_UNSUPPORTED (k > 1024),
+ *         RQ_ERR_WORKSPACE_TOO_SMALL, RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ */
+RQ_API size_t rq_topk_workspace_bytes(int64_t V, int B, int k);
+RQ_API int rq_topk_sample(const float *logits, int64_t V, int B, int k, float temperature,
+                          uint64_t seed, uint64_t step, float *topk_val, int32_t *topk_idx,
+                          int32_t *token, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * rq_encode -- produce the codes: greedy residual nearest-codeword
  * assignment of V rows ("Gemma-2-2B combined RQ+NF4" names the compression
  * residual product quantization, M subspaces x L levels of K codewords,

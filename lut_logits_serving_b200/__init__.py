@@ -26,7 +26,7 @@ __all__ = [
     "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
     "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
     "rq_pack10", "rq_device_error", "rq_set_profile_events", "rq_lut_logits_static",
-    "rq_greedy_step", "rq_encode",
+    "rq_greedy_step", "rq_encode", "rq_topk_workspace_bytes", "rq_topk_sample",
 ]
 
 U16 = 0
@@ -75,6 +75,9 @@ _SIGNATURES = {
     "rq_decode_rows": (_i, [_p, _i64, _p, _i, _p, RqDims, _f, _p, _p]),
     "rq_pack10": (_i, [_p, RqDims, _p, _p]),
     "rq_encode": (_i, [_p, RqDims, _p, _p, _p]),
+    "rq_topk_workspace_bytes": (_sz, [_i64, _i, _i]),
+    "rq_topk_sample": (_i, [_p, _i64, _i, _i, _f, ctypes.c_uint64, ctypes.c_uint64, _p, _p, _p,
+                            _p, _sz, _p]),
     "rq_device_error": (_i, [ctypes.POINTER(ctypes.c_uint32), _i]),
     "rq_set_profile_events": (_i, [_p, _p]),
     "rq_prepare_sched": (_i, [_p, RqDims, _p, _p, _p]),
@@ -271,6 +274,35 @@ def rq_encode(X, C, d: RqDims, out=None, stream=None):
                                         _cuda(C, torch.float32, "C"),
                                         _cuda(out, torch.uint16, "codes"), _stream(stream)))
     return out
+
+
+def rq_topk_workspace_bytes(V: int, B: int, k: int) -> int:
+    return int(lib().rq_topk_workspace_bytes(V, B, k))
+
+
+def rq_topk_sample(logits, k: int, temperature: float = 1.0, seed: int = 0, step: int = 0,
+                   topk_val=None, topk_idx=None, token=None, want_topk: bool = True,
+                   ws=None, stream=None):
+    """logits float32 [B, V] (device) -> (topk_val [B, k], topk_idx [B, k], token [B]);
+    the top-k outputs are None with want_topk=False."""
+    torch = _torch()
+    B, V = logits.shape
+    if want_topk:
+        if topk_val is None:
+            topk_val = _empty((B, k), torch.float32, logits)
+        if topk_idx is None:
+            topk_idx = _empty((B, k), torch.int32, logits)
+    if token is None:
+        token = _empty((B,), torch.int32, logits)
+    nbytes = rq_topk_workspace_bytes(V, B, k)
+    wsp, wsn, ws = _workspace(max(nbytes, 1), logits, ws)
+    _check("rq_topk_sample", lib().rq_topk_sample(
+        _cuda(logits, torch.float32, "logits"), V, B, k, float(temperature),
+        ctypes.c_uint64(seed), ctypes.c_uint64(step),
+        _ptr_or_null(topk_val, torch.float32, "topk_val"),
+        _ptr_or_null(topk_idx, torch.int32, "topk_idx"),
+        _cuda(token, torch.int32, "token"), wsp, wsn, _stream(stream)))
+    return topk_val, topk_idx, token
 
 
 def rq_device_error(clear: bool = True) -> int:

@@ -337,6 +337,10 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
 cudaError_t launch_pack10(const uint16_t *codes, int64_t V, int P, uint8_t *packed,
                           cudaStream_t s);
 
+size_t topk_workspace_bytes(int64_t V, int B, int k);
+cudaError_t launch_topk_sample(const float *logits, int64_t V, int B, int k, double temperature,
+                               unsigned long long seed, unsigned long long step, float *val,
+                               int32_t *idx, int32_t *token, void *ws, cudaStream_t s);
 cudaError_t launch_encode(const float *X, int64_t N, const float *C, int D, int M, int L, int K,
                           uint16_t *codes, cudaStream_t s);
 cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, uint16_t *out,

@@ -397,6 +397,29 @@ int rq_encode(const float *X, rq_dims d, const float *C, uint16_t *codes, void *
                                  static_cast<cudaStream_t>(stream)));
 }
 
+size_t rq_topk_workspace_bytes(int64_t V, int B, int k) {
+  if (V < 1 || V > (int64_t)0x7fffffff - 1024 || B < 1 || B > 65535 || k < 1 || k > 1024 ||
+      k > V)
+    return 0;
+  return topk_workspace_bytes(V, B, k);
+}
+
+int rq_topk_sample(const float *logits, int64_t V, int B, int k, float temperature,
+                   uint64_t seed, uint64_t step, float *topk_val, int32_t *topk_idx,
+                   int32_t *token, void *ws, size_t ws_bytes, void *stream) {
+  if (!logits || !ws || V < 1 || V > (int64_t)0x7fffffff - 1024 || B < 1 || B > 65535 ||
+      k < 1 || k > V)
+    return RQ_ERR_INVALID_ARGUMENT;
+  if (k > 1024) return RQ_ERR_UNSUPPORTED;
+  if (!aligned(logits, 4) || !aligned(ws, 256) || (topk_val && !aligned(topk_val, 4)) ||
+      (topk_idx && !aligned(topk_idx, 4)) || (token && !aligned(token, 4)))
+    return RQ_ERR_MISALIGNED;
+  if (ws_bytes < rq_topk_workspace_bytes(V, B, k)) return RQ_ERR_WORKSPACE_TOO_SMALL;
+  return status_of(launch_topk_sample(logits, V, B, k, (double)temperature, seed, step,
+                                      topk_val, topk_idx, token, ws,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 int rq_set_profile_events(void *start, void *stop) {
   if ((start == nullptr) != (stop == nullptr)) return RQ_ERR_INVALID_ARGUMENT;
   t_prof_start = static_cast<cudaEvent_t>(start);

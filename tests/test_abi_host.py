@@ -127,6 +127,15 @@ def test_argument_errors_return_before_any_launch():
                              s) == UNS                                        # sched, P % 32
     assert lib.rq_device_error(None, 0) == INV
     assert lib.rq_encode(null, G2, a, a, s) == INV
+    big = 1 << 40
+    assert lib.rq_topk_sample(a, 256000, 1, 0, 1.0, 0, 0, null, null, a, a, big, s) == INV
+    assert lib.rq_topk_sample(a, 256000, 1, 1025, 1.0, 0, 0, null, null, a, a, big, s) == UNS
+    assert lib.rq_topk_sample(a, 100, 1, 101, 1.0, 0, 0, null, null, a, a, big, s) == INV
+    assert lib.rq_topk_sample(a, 256000, 1, 50, 1.0, 0, 0, null, null, a, a, 16, s) == WS
+    assert lib.rq_topk_sample(a, 256000, 1, 50, 1.0, 0, 0, null, null, a, _fake(0x10010), big,
+                              s) == MIS
+    assert rq.rq_topk_workspace_bytes(256000, 1, 50) > 0
+    assert rq.rq_topk_workspace_bytes(256000, 1, 1025) == 0
     assert lib.rq_encode(null, rq.dims(0, 2304, 384, 2, 1024), null, null, s) == 0   # V = 0
     assert lib.rq_encode(a, rq.dims(10, 66, 2, 2, 16), a, _fake(0x900000), s) == UNS   # ds 33
     assert lib.rq_encode(_fake(0x10002), G2, a, _fake(0x90000000), s) == MIS
