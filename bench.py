@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="g2_b1",
                     choices=["g2_b1", "g2_b32", "packed_b64", "mlp_gate_b1", "mlp_down_b1",
-                             "encode_g2"])
+                             "encode_g2", "g2_b1_topk50"])
     ap.add_argument("--codes", default="sched", choices=["u16", "sched"],
                     help="uint16 code layout of the unpacked workloads timed for `value`: "
                          "bank-scheduled once by rq_prepare_sched (the serving layout), or as "
@@ -65,8 +65,14 @@ def workload_config(w, codes="u16"):
     fmt = f"packed10 ({rb} B/row)" if w.packed10 else (
         f"uint16 ({rb} B/row)" if codes == "u16" else
         f"uint16 ({rb} B/row) in the bank-scheduled order of rq_prepare_sched")
-    what = (f"softcap {w.softcap:g}, logits + argmax, then the {w.B} picked tokens' input rows "
-            f"rebuilt (bf16)") if w.argmax else "y = W x, no softcap (RQ-coded MLP weight)"
+    if w.argmax:
+        what = (f"softcap {w.softcap:g}, logits + argmax, then the {w.B} picked tokens' input "
+                f"rows rebuilt (bf16)")
+    elif w.topk:
+        what = (f"softcap {w.softcap:g}, logits, top-{w.topk} + draw at temperature "
+                f"{w.temperature:g}, then the drawn tokens' input rows rebuilt (bf16)")
+    else:
+        what = "y = W x, no softcap (RQ-coded MLP weight)"
     return {
         "workload": f"{w.name}: V={w.V} D={w.D} M={w.M} L={w.L} K={w.K} B={w.B}, {fmt} codes, "
                     f"{what}",
@@ -168,9 +174,12 @@ def oracle_step_fn(w, data):
         T = oracle.lut_build(data["h"], data["C"], "f64")
         z = oracle.logits_lut(data["codes"], T, rows)
         y = oracle.softcap(z, w.softcap)
-        am = oracle.argmax(y.astype(np.float32))
+        if w.topk:
+            _, _, pick = oracle.sample(y.astype(np.float32), w.topk, w.temperature, 1234, 0)
+        else:
+            pick = oracle.argmax(y.astype(np.float32))
         oracle.decode_rows_bf16(data["ids"], data["codes"], data["C"], w.decode_scale)
-        return am
+        return pick
     return step
 
 
@@ -184,9 +193,10 @@ def cpu_baseline(w, data, seconds):
         el = time.perf_counter() - t0
         if el >= seconds:
             break
+    pick = f"top-{w.topk} draw" if w.topk else "argmax"
     return {"value": w.V * w.B * n / el, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} full steps of {w.name} (all {w.V} rows x {w.B} tokens, fp64 tables, "
-                      f"softcap, argmax, row decode), single-threaded C, {el:.1f} s"}
+                      f"softcap, {pick}, row decode), single-threaded C, {el:.1f} s"}
 
 
 def encode_terms(w, rows):
@@ -299,6 +309,12 @@ def profiled_traffic(kernel):
     return e.get("dram_bytes_per_launch")
 
 
+def topk_launches(V, k):
+    """Kernels of one rq_topk_sample call: the histogram pass and the gather
+    pass whose last CTA per token sorts and draws (plus a memset)."""
+    return 2
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -331,6 +347,9 @@ def run_ours(args, w):
     logits = torch.empty((w.B, w.V), dtype=torch.float32, device="cuda")
     am = torch.empty((w.B,), dtype=torch.int32, device="cuda")
     rows = torch.empty((w.B, w.D), dtype=torch.bfloat16, device="cuda")
+    tok = torch.empty((w.B,), dtype=torch.int32, device="cuda")
+    tws = (torch.empty(rq.rq_topk_workspace_bytes(w.V, w.B, w.topk), dtype=torch.uint8,
+                       device="cuda") if w.topk else None)
     stream = torch.cuda.current_stream()
 
     # code layouts: the artifact is prepared once, outside any timed region
@@ -348,6 +367,15 @@ def run_ours(args, w):
     def make_step(fmt, codes):
         ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
                          device="cuda")
+
+        if w.topk:
+            def step():
+                # logits, the top-k draw, and the drawn tokens' input rows
+                rq.rq_logits_from_hidden(dh, dC, codes, fmt, d, w.softcap, logits=logits, ws=ws)
+                rq.rq_topk_sample(logits, w.topk, w.temperature, seed=1234, step=0, token=tok,
+                                  want_topk=False, ws=tws)
+                rq.rq_decode_rows(tok, codes, fmt, dC, d, w.decode_scale, out=rows)
+            return step
 
         if not w.argmax:
             def step():
@@ -470,19 +498,21 @@ def run_ours(args, w):
     am_host = torch.empty((w.B,), dtype=torch.int32).pin_memory()
     ne2e = min(args.steps, 2000)
 
+    picked = am if w.argmax else (tok if w.topk else None)
+
     def e2e_step():
         dh.copy_(h_host, non_blocking=True)
         step()
         out_host.copy_(logits, non_blocking=True)
-        if w.argmax:
-            am_host.copy_(am, non_blocking=True)
+        if picked is not None:
+            am_host.copy_(picked, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
     e_ms = time_steps(e2e_step, ne2e)
     e2e_value = throughput(w.V * w.B * ne2e, world, e_ms)
     h2d = data["h"].nbytes
-    d2h = w.B * w.V * 4 + (w.B * 4 if w.argmax else 0)
+    d2h = w.B * w.V * 4 + (w.B * 4 if picked is not None else 0)
 
     # the argmax must agree with the logits it came from
     if w.argmax:
@@ -495,9 +525,24 @@ def run_ours(args, w):
         launches_per_step = 3 + (1 if w.argmax else 0)
     else:
         launches_per_step = 2 * ((w.B + 31) // 32) + (1 if w.argmax else 0)
+    topk_us = None
+    if w.topk:
+        launches_per_step += topk_launches(w.V, w.topk) + 1     # top-k + draw, row decode
+        # the epilogue alone, on the step's own logits
+        for _ in range(10):
+            rq.rq_topk_sample(logits, w.topk, w.temperature, 1234, 0, token=tok, want_topk=False,
+                              ws=tws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(200):
+            rq.rq_topk_sample(logits, w.topk, w.temperature, 1234, 0, token=tok, want_topk=False,
+                              ws=tws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        topk_us = e0.elapsed_time(e1) / 200 * 1e3
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.argmax:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and (w.argmax or w.topk):
         cpu = cpu_baseline(w, data, args.cpu_seconds)
 
     if world > 1:
@@ -520,6 +565,7 @@ def run_ours(args, w):
                      "kernel_us": kern_us},
         "step_hbm_frac": algo_bytes / (sec / args.steps) / 1e9 / peak,
         "other_layouts": others,
+        "topk_sample_us": topk_us,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ne2e},

@@ -12,19 +12,23 @@
 //     "Parallel random numbers: as easy as 1, 2, 3", SC'11) for counter
 //     (step, row, 0, 0) and key (seed, 0), times 2^-53.
 //
-// Design for sm_100a.  The logits of a token (1 MB at V = 256000) are read
-// once.  Each value becomes a 64-bit key: the order-preserving transform of
-// its fp32 bits (high word) and the complement of its index (low word), so
-// that one unsigned compare orders by value, then by lower index.
-//   stage 1 -- one CTA per 2048-logit slice and token sorts its keys with a
-//              bitonic network in shared memory and keeps the first KP
-//              (k rounded up to a power of two);
-//   stage 2 -- a CTA loads G such lists and merges them pairwise in shared
-//              memory: the elementwise max of list A and reversed list B is
-//              a bitonic sequence holding the top KP of both, and log2(KP)
-//              half-cleaner passes sort it.  Launches repeat until one list
-//              per token is left; that last launch also writes the outputs
-//              and makes the draw (one warp: lane-chunked sums, a warp scan).
+// Design for sm_100a: a radix select, then a sort of the few survivors.
+// Each logit's fp32 bits map to an order-preserving 32-bit word (ord), and
+// the 64-bit key (ord, complement of the index) orders by value, then lower
+// index, under one unsigned compare.
+//   pass 1 -- a grid of CTAs histograms the top 12 bits of ord of every
+//             logit (shared-memory counts, then one global add per occupied
+//             bin);
+//   pass 2 -- the same CTAs find the threshold bin t (the highest bin whose
+//             suffix count reaches k) and append the keys of bin >= t to a
+//             candidate list (about k to 3k keys for logit-like values).  The
+//             last CTA of each token (a completion counter) sorts the
+//             candidates with a bitonic network in shared memory, writes the
+//             top k and makes the draw (one warp: lane-chunked fp64 sums and a
+//             warp scan).  When bin t holds more keys than the list (heavy
+//             ties), the last CTA instead refines the threshold exactly over
+//             the row (two more 10-bit histograms) and takes the keys above it
+//             plus the tied ones in index order.
 #include <cfloat>
 #include <climits>
 
@@ -32,15 +36,35 @@
 
 namespace rq {
 
-constexpr int kTopkSlice = 2048;         // logits per stage-1 CTA
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkMergeSmem = 96 * 1024;
+constexpr int kTopkThreads = 512;
+constexpr int kTopkBins = 4096;            // top 12 bits of ord
+constexpr int kTopkCap = 8192;             // candidate keys per token
+constexpr int kTopkMaxK = 1024;
 
-__device__ __forceinline__ unsigned long long topk_key(float v, int64_t idx) {
+struct TopkWs {
+  unsigned *hist;              // [B][kTopkBins]       zeroed per call
+  unsigned *cnt;               // [B] candidates        zeroed per call
+  unsigned *done;              // [B] finished CTAs     zeroed per call
+  unsigned long long *cand;    // [B][kTopkCap]
+};
+
+struct TopkOut {
+  int k;
+  double temperature;
+  unsigned long long seed, step;
+  float *val;      // [B][k] or null
+  int32_t *idx;    // [B][k] or null
+  int32_t *token;  // [B] or null
+};
+
+__device__ __forceinline__ unsigned topk_ord(float v) {
   unsigned b = __float_as_uint(v);
   if (b == 0x80000000u) b = 0u;          // -0 orders as +0
-  b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-  return ((unsigned long long)b << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)idx);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned long long topk_key(unsigned ord, int64_t idx) {
+  return ((unsigned long long)ord << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)idx);
 }
 
 __device__ __forceinline__ float topk_value(unsigned long long key) {
@@ -73,27 +97,88 @@ __device__ double philox_uniform(unsigned long long seed, unsigned long long ste
   return (double)(c0 >> 11) * (1.0 / 9007199254740992.0);
 }
 
-// Stage 1: grid (nblk, B).  Keys of slice blockIdx.x sorted descending;
-// the first KP go to lists[b][blk][0..KP).  Keys past V are 0 (below every
-// real key: the smallest real key has a nonzero high word).
-__global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(const float *__restrict__ y,
-                                                                 int64_t V, int KP,
-                                                                 unsigned long long *lists) {
-  __shared__ unsigned long long sk[kTopkSlice];
+// This CTA's range of row elements: nb CTAs split V evenly.
+__device__ __forceinline__ void topk_range(int64_t V, int64_t &v0, int64_t &v1) {
+  v0 = V * blockIdx.x / gridDim.x;
+  v1 = V * (blockIdx.x + 1) / gridDim.x;
+}
+
+// Pass 1: grid (nb, B).
+__global__ void __launch_bounds__(kTopkThreads) topk_hist_kernel(const float *__restrict__ y,
+                                                                int64_t V, TopkWs w) {
+  __shared__ unsigned h[kTopkBins];
+  for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) h[i] = 0u;
   griddep_wait();
+  __syncthreads();
   const int b = blockIdx.y;
-  const int64_t v0 = (int64_t)blockIdx.x * kTopkSlice;
+  int64_t v0, v1;
+  topk_range(V, v0, v1);
   const float *row = y + (int64_t)b * V;
-  for (int i = threadIdx.x; i < kTopkSlice; i += kTopkThreads) {
-    const int64_t v = v0 + i;
-    sk[i] = v < V ? topk_key(__ldg(row + v), v) : 0ull;
+  for (int64_t v = v0 + threadIdx.x; v < v1; v += kTopkThreads)
+    atomicAdd(&h[topk_ord(__ldg(row + v)) >> 20], 1u);
+  __syncthreads();
+  griddep_launch_dependents();
+  unsigned *H = w.hist + (int64_t)b * kTopkBins;
+  for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads)
+    if (h[i]) atomicAdd(&H[i], h[i]);
+}
+
+// Block-wide: of the counts c[0..n) (n = 8 * kTopkThreads at most, given as
+// 8 per thread in `mine`), the highest index t whose suffix sum reaches
+// `need`, that suffix sum (ge) and the sum above t (gt).  Every thread gets
+// the result.  need >= 1 and the total reaches it.
+struct SuffixPick {
+  int t;
+  unsigned ge, gt;
+};
+
+template <int PER>
+__device__ SuffixPick suffix_pick(const unsigned (&mine)[PER], unsigned need, unsigned *scr) {
+  // thread i owns entries [i*PER, (i+1)*PER); suffix order is thread order reversed
+  unsigned s = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) s += mine[j];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // exclusive suffix sum over threads: sum of threads with a higher index
+  unsigned incl = s;   // inclusive suffix within the warp (lanes >= this one)
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const unsigned t = __shfl_down_sync(0xffffffffu, incl, d);
+    if (lane + d < 32) incl += t;
   }
-  for (int size = 2; size <= kTopkSlice; size <<= 1)
+  if (lane == 0) scr[warp] = incl;       // warp total
+  __syncthreads();
+  unsigned above_warp = 0;
+  for (int w2 = warp + 1; w2 < kTopkThreads / 32; ++w2) above_warp += scr[w2];
+  const unsigned above = above_warp + incl - s;   // entries after this thread's
+  __syncthreads();
+  // the thread whose range holds t: above < need <= above + s
+  if (above < need && need <= above + s) {
+    unsigned acc = above;
+    for (int j = PER - 1; j >= 0; --j) {
+      if (acc + mine[j] >= need) {
+        scr[0] = (unsigned)(threadIdx.x * PER + j);
+        scr[1] = acc + mine[j];
+        scr[2] = acc;
+        break;
+      }
+      acc += mine[j];
+    }
+  }
+  __syncthreads();
+  SuffixPick r{(int)scr[0], scr[1], scr[2]};
+  __syncthreads();
+  return r;
+}
+
+// Bitonic sort of n (a power of two) keys in shared memory, descending.
+__device__ void sort_desc(unsigned long long *sk, int n) {
+  for (int size = 2; size <= n; size <<= 1)
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       __syncthreads();
-      for (int t = threadIdx.x; t < kTopkSlice / 2; t += kTopkThreads) {
+      for (int t = threadIdx.x; t < n / 2; t += kTopkThreads) {
         const int i = 2 * t - (t & (stride - 1)), j = i + stride;
-        const bool desc = (i & size) == 0;  // the last merge (size = slice) is descending
+        const bool desc = (i & size) == 0;
         const unsigned long long a = sk[i], c = sk[j];
         if (desc ? a < c : a > c) {
           sk[i] = c;
@@ -102,82 +187,26 @@ __global__ void __launch_bounds__(kTopkThreads) topk_slice_kernel(const float *_
       }
     }
   __syncthreads();
-  griddep_launch_dependents();
-  unsigned long long *out = lists + ((int64_t)b * gridDim.x + blockIdx.x) * KP;
-  for (int i = threadIdx.x; i < KP; i += kTopkThreads) out[i] = sk[i];
 }
 
-struct TopkOut {
-  int k;
-  double temperature;
-  unsigned long long seed, step;
-  float *val;      // [B][k] or null
-  int32_t *idx;    // [B][k] or null
-  int32_t *token;  // [B] or null
-};
-
-// Stage 2: grid (ceil(nl / G), B).  G lists of KP keys (sorted descending)
-// merged into one; with `fin` (one CTA per token left) the outputs and the
-// draw are made here.
-__global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(
-    const unsigned long long *__restrict__ in, int nl, int KP, int G,
-    unsigned long long *out, int fin, TopkOut o) {
-  extern __shared__ unsigned long long sm[];   // [G][KP]
-  griddep_wait();
-  const int b = blockIdx.y;
-  const int l0 = blockIdx.x * G;
-  for (int i = threadIdx.x; i < G * KP; i += kTopkThreads) {
-    const int l = i / KP;
-    sm[i] = l0 + l < nl ? in[((int64_t)b * nl + l0 + l) * KP + (i - l * KP)] : 0ull;
-  }
-  for (int w = 1; w < G; w <<= 1) {
-    const int npairs = G / (2 * w);
-    __syncthreads();
-    // A[i] = max(A[i], B[KP-1-i]): the top KP of A and B, as a bitonic sequence
-    for (int t = threadIdx.x; t < npairs * KP; t += kTopkThreads) {
-      const int p = t / KP, i = t - p * KP;
-      unsigned long long *A = sm + (int64_t)(2 * w * p) * KP;
-      const unsigned long long *Bl = A + (int64_t)w * KP;
-      const unsigned long long x = A[i], z = Bl[KP - 1 - i];
-      A[i] = x > z ? x : z;
-    }
-    for (int stride = KP >> 1; stride > 0; stride >>= 1) {
-      __syncthreads();
-      for (int t = threadIdx.x; t < npairs * (KP / 2); t += kTopkThreads) {
-        const int p = t / (KP / 2), r = t - p * (KP / 2);
-        unsigned long long *A = sm + (int64_t)(2 * w * p) * KP;
-        const int i = 2 * r - (r & (stride - 1)), j = i + stride;
-        const unsigned long long x = A[i], z = A[j];
-        if (x < z) {
-          A[i] = z;
-          A[j] = x;
-        }
-      }
-    }
-  }
-  __syncthreads();
-  griddep_launch_dependents();
-  if (!fin) {
-    unsigned long long *dst = out + ((int64_t)b * gridDim.x + blockIdx.x) * KP;
-    for (int i = threadIdx.x; i < KP; i += kTopkThreads) dst[i] = sm[i];
-    return;
-  }
+// Outputs of token b from its top keys sk[0..k), sorted descending.
+__device__ void topk_finish(const unsigned long long *sk, int b, const TopkOut &o) {
   const int k = o.k;
   for (int i = threadIdx.x; i < k; i += kTopkThreads) {
-    if (o.val) o.val[(int64_t)b * k + i] = topk_value(sm[i]);
-    if (o.idx) o.idx[(int64_t)b * k + i] = topk_index(sm[i]);
+    if (o.val) o.val[(int64_t)b * k + i] = topk_value(sk[i]);
+    if (o.idx) o.idx[(int64_t)b * k + i] = topk_index(sk[i]);
   }
   if (o.token == nullptr || threadIdx.x >= 32) return;
   const int lane = threadIdx.x;
   if (k == 1 || !(o.temperature > 0.0)) {
-    if (lane == 0) o.token[b] = topk_index(sm[0]);
+    if (lane == 0) o.token[b] = topk_index(sk[0]);
     return;
   }
-  const double y0 = (double)topk_value(sm[0]);
+  const double y0 = (double)topk_value(sk[0]);
   const int per = (k + 31) / 32;
   const int lo = lane * per, hi = min(k, lo + per);
   double s = 0.0;
-  for (int i = lo; i < hi; ++i) s += exp(((double)topk_value(sm[i]) - y0) / o.temperature);
+  for (int i = lo; i < hi; ++i) s += exp(((double)topk_value(sk[i]) - y0) / o.temperature);
   double incl = s;                        // inclusive scan of the lane sums
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -190,7 +219,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(
   const double target = philox_uniform(o.seed, o.step, (unsigned long long)b) * total;
   int pick = INT_MAX;
   for (int i = lo; i < hi; ++i) {
-    cum += exp(((double)topk_value(sm[i]) - y0) / o.temperature);
+    cum += exp(((double)topk_value(sk[i]) - y0) / o.temperature);
     if (cum > target) {
       pick = i;
       break;
@@ -198,72 +227,157 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(
   }
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) pick = min(pick, __shfl_xor_sync(0xffffffffu, pick, d));
-  if (lane == 0) o.token[b] = topk_index(sm[pick == INT_MAX ? k - 1 : pick]);
+  if (lane == 0) o.token[b] = topk_index(sk[pick == INT_MAX ? k - 1 : pick]);
 }
 
-int topk_pow2(int k) {
-  int p = 1;
-  while (p < k) p <<= 1;
-  return p;
+// Heavy ties: the exact k-th key over the whole row by one CTA.  `bin` is
+// the threshold bin of the top 12 bits and `gt` the count above it.
+__device__ void topk_exact_row(const float *__restrict__ row, int64_t V, unsigned bin,
+                               unsigned gt, unsigned long long *sk, unsigned *scr,
+                               unsigned *h, int b, const TopkOut &o) {
+  const unsigned k = (unsigned)o.k;
+  // refine ord below the top 12 bits: bits 19..10, then 9..0
+  unsigned prefix = bin, shift = 20, above = gt;
+  for (int level = 0; level < 2; ++level) {
+    const unsigned sub = 10, nsub = 1u << sub;
+    for (unsigned i = threadIdx.x; i < nsub; i += kTopkThreads) h[i] = 0u;
+    __syncthreads();
+    for (int64_t v = threadIdx.x; v < V; v += kTopkThreads) {
+      const unsigned ord = topk_ord(__ldg(row + v));
+      if ((ord >> shift) == prefix) atomicAdd(&h[(ord >> (shift - sub)) & (nsub - 1)], 1u);
+    }
+    __syncthreads();
+    unsigned mine[2] = {h[2 * threadIdx.x], h[2 * threadIdx.x + 1]};
+    const SuffixPick p = suffix_pick<2>(mine, k - above, scr);
+    prefix = (prefix << sub) | (unsigned)p.t;
+    above += p.gt;
+    shift -= sub;
+  }
+  // prefix is now the full ord of the k-th largest value; `above` values
+  // exceed it and k - above of its copies are taken in index order
+  const unsigned tau = prefix;
+  const unsigned need_eq = k - above;
+  if (threadIdx.x == 0) {
+    scr[0] = 0u;    // keys placed
+    scr[1] = 0u;    // ties taken so far
+  }
+  __syncthreads();
+  for (int64_t base = 0; base < V; base += kTopkThreads) {
+    const int64_t v = base + threadIdx.x;
+    const unsigned ord = v < V ? topk_ord(__ldg(row + v)) : 0u;
+    const bool gtv = v < V && ord > tau, eqv = v < V && ord == tau;
+    if (gtv) sk[atomicAdd(&scr[0], 1u)] = topk_key(ord, v);
+    // ties in index order: rank among this tile's ties, offset by earlier tiles
+    const unsigned ball = __ballot_sync(0xffffffffu, eqv);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) h[warp] = __popc(ball);
+    __syncthreads();
+    unsigned before = scr[1];
+    for (int w2 = 0; w2 < warp; ++w2) before += h[w2];
+    before += __popc(ball & ((1u << lane) - 1u));
+    if (eqv && before < need_eq) sk[atomicAdd(&scr[0], 1u)] = topk_key(ord, v);
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int w2 = 0; w2 < kTopkThreads / 32; ++w2) scr[1] += h[w2];
+    __syncthreads();
+  }
+  int n = 1;
+  while (n < (int)k) n <<= 1;
+  for (int i = (int)k + threadIdx.x; i < n; i += kTopkThreads) sk[i] = 0ull;
+  sort_desc(sk, n);
+  topk_finish(sk, b, o);
 }
 
-static int topk_max_group(int KP) {
-  int g = 1;
-  while (2 * g * KP * (int)sizeof(unsigned long long) <= kTopkMergeSmem) g <<= 1;
-  return g;
+// Pass 2: grid (nb, B); dynamic shared memory kTopkCap keys.
+__global__ void __launch_bounds__(kTopkThreads) topk_gather_kernel(const float *__restrict__ y,
+                                                                  int64_t V, TopkWs w,
+                                                                  TopkOut o) {
+  extern __shared__ unsigned long long sk[];   // [kTopkCap]
+  __shared__ unsigned scr[kTopkThreads / 32 + 4];
+  __shared__ unsigned h[1024];
+  __shared__ int last;
+  griddep_wait();
+  const int b = blockIdx.y;
+  const unsigned *H = w.hist + (int64_t)b * kTopkBins;
+  constexpr int PER = kTopkBins / kTopkThreads;
+  unsigned mine[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) mine[j] = H[threadIdx.x * PER + j];
+  const SuffixPick p = suffix_pick<PER>(mine, (unsigned)o.k, scr);
+  const bool fits = p.ge <= (unsigned)kTopkCap;
+  const float *row = y + (int64_t)b * V;
+  if (fits) {
+    int64_t v0, v1;
+    topk_range(V, v0, v1);
+    unsigned long long *cand = w.cand + (int64_t)b * kTopkCap;
+    for (int64_t v = v0 + threadIdx.x; v < v1; v += kTopkThreads) {
+      const unsigned ord = topk_ord(__ldg(row + v));
+      if ((int)(ord >> 20) >= p.t) cand[atomicAdd(&w.cnt[b], 1u)] = topk_key(ord, v);
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&w.done[b], 1u) == gridDim.x - 1;
+  __syncthreads();
+  griddep_launch_dependents();
+  if (!last) return;
+  __threadfence();
+  if (fits) {
+    const unsigned long long *cand = w.cand + (int64_t)b * kTopkCap;
+    int n = 1;
+    while (n < (int)p.ge) n <<= 1;
+    for (int i = threadIdx.x; i < n; i += kTopkThreads)
+      sk[i] = i < (int)p.ge ? __ldcg(cand + i) : 0ull;
+    sort_desc(sk, n);
+    topk_finish(sk, b, o);
+  } else {
+    topk_exact_row(row, V, (unsigned)p.t, p.gt, sk, scr, h, b, o);
+  }
 }
 
 size_t topk_workspace_bytes(int64_t V, int B, int k) {
-  const int KP = topk_pow2(k);
-  const int64_t nblk = (V + kTopkSlice - 1) / kTopkSlice;
-  const int G = topk_max_group(KP);
-  const int64_t n2 = (nblk + G - 1) / G;
-  const size_t a = (size_t)B * nblk * KP * sizeof(unsigned long long);
-  const size_t b = (size_t)B * (n2 > 1 ? n2 : 1) * KP * sizeof(unsigned long long);
-  return align_up((int64_t)a, 256) + align_up((int64_t)b, 256);
+  (void)V;
+  (void)k;
+  const size_t counters = (size_t)B * (kTopkBins + 2) * sizeof(unsigned);
+  return align_up((int64_t)counters, 256) + (size_t)B * kTopkCap * sizeof(unsigned long long);
+}
+
+static int topk_blocks(int64_t V, int B, int sms) {
+  int64_t nb = (2 * (int64_t)sms + B - 1) / B;           // about two CTAs per SM in all
+  const int64_t most = (V + 1023) / 1024;               // at least ~1024 logits per CTA
+  if (nb > most) nb = most;
+  return (int)(nb < 1 ? 1 : nb);
 }
 
 cudaError_t launch_topk_sample(const float *logits, int64_t V, int B, int k, double temperature,
                                unsigned long long seed, unsigned long long step, float *val,
                                int32_t *idx, int32_t *token, void *ws, cudaStream_t s) {
-  const int KP = topk_pow2(k);
-  const int64_t nblk = (V + kTopkSlice - 1) / kTopkSlice;
-  if (nblk > 0x7fffffffLL || B > 65535) return cudaErrorInvalidValue;
-  const int G = topk_max_group(KP);
-  unsigned long long *bufA = static_cast<unsigned long long *>(ws);
-  unsigned long long *bufB = reinterpret_cast<unsigned long long *>(
+  if (B > 65535 || k < 1 || k > kTopkMaxK) return cudaErrorInvalidValue;
+  TopkWs w;
+  w.hist = static_cast<unsigned *>(ws);
+  w.cnt = w.hist + (size_t)B * kTopkBins;
+  w.done = w.cnt + B;
+  w.cand = reinterpret_cast<unsigned long long *>(
       static_cast<unsigned char *>(ws) +
-      align_up((int64_t)B * nblk * KP * (int64_t)sizeof(unsigned long long), 256));
-  static bool attr[128] = {};
-  int dev = 0;
+      align_up((int64_t)B * (kTopkBins + 2) * (int64_t)sizeof(unsigned), 256));
+  int dev = 0, sms = 148;
   cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool attr[128] = {};
+  const size_t smem = (size_t)kTopkCap * sizeof(unsigned long long);
   if (dev < 128 && !attr[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(topk_merge_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kTopkMergeSmem);
+    cudaError_t e = cudaFuncSetAttribute(topk_gather_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr[dev] = true;
   }
-  cudaError_t e = pdl_launch(topk_slice_kernel, dim3((unsigned)nblk, (unsigned)B),
-                             dim3(kTopkThreads), 0, s, logits, V, KP, bufA);
+  cudaError_t e = cudaMemsetAsync(w.hist, 0, (size_t)B * (kTopkBins + 2) * sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)topk_blocks(V, B, sms), (unsigned)B);
+  e = pdl_launch(topk_hist_kernel, grid, dim3(kTopkThreads), 0, s, logits, V, w);
   if (e != cudaSuccess) return e;
   TopkOut o{k, temperature, seed, step, val, idx, token};
-  int nl = (int)nblk;
-  const unsigned long long *in = bufA;
-  unsigned long long *out = bufB;
-  while (true) {
-    int g = 1;
-    while (g < nl && g < G) g <<= 1;
-    const int nout = (nl + g - 1) / g;
-    const int fin = nout == 1;
-    e = pdl_launch(topk_merge_kernel, dim3((unsigned)nout, (unsigned)B), dim3(kTopkThreads),
-                   (size_t)g * KP * sizeof(unsigned long long), s, in, nl, KP, g, out, fin, o);
-    if (e != cudaSuccess || fin) return e;
-    nl = nout;
-    unsigned long long *t = const_cast<unsigned long long *>(in);
-    in = out;
-    out = t;
-  }
+  return pdl_launch(topk_gather_kernel, grid, dim3(kTopkThreads), smem, s, logits, V, w, o);
 }
 
 }  // namespace rq

@@ -35,6 +35,8 @@ class Workload:
     zipf_s: float = 1.1
     decode_scale: float = 0.0   # embedding scale applied to rebuilt rows
     encode: bool = False        # the call encodes V rows instead of scoring them
+    topk: int = 0               # > 0: draw the next token from the top-k
+    temperature: float = 1.0    # of that draw
 
     @property
     def ds(self) -> int:
@@ -59,6 +61,12 @@ WORKLOADS = {
     "decode512": Workload("decode512", V=256000, D=2304, M=384, L=2, K=1024, B=0,
                           sigmas=(0.02, 0.005), hidden_scale=0.83,
                           n_ids=512, decode_scale=math.sqrt(2304.0)),
+    # Generation beyond greedy: the top-50 of the softcapped logits, a draw
+    # at temperature 0.8, and the drawn token's input row.
+    "g2_b1_topk50": Workload("g2_b1_topk50", V=256000, D=2304, M=384, L=2, K=1024, B=1,
+                             sigmas=(0.02, 0.005), hidden_scale=40.0 / math.sqrt(2304.0),
+                             topk=50, temperature=0.8, n_ids=1,
+                             decode_scale=math.sqrt(2304.0)),
     "packed_b64": Workload("packed_b64", V=256000, D=2304, M=384, L=2, K=1024, B=64,
                            sigmas=(0.02, 0.005), hidden_scale=0.83, packed10=True,
                            argmax=True, n_ids=64, decode_scale=math.sqrt(2304.0)),

@@ -4,9 +4,11 @@ indices must match exactly (descending, lower index first among equal
 values), and the drawn token must be the oracle's (both draw in fp64 from the
 same Philox4x64-10 uniform; a disagreement is only possible when u * total
 falls within rounding of a running-sum boundary, which the test reports).
-Cases span several 2048-logit slices with a ragged tail, k from 1 to 1024
-(and k = V), heavy ties and signed zeros, several merge launches, and the
-logits of the full Gemma-2 shaped path."""
+Cases span ragged row splits, k from 1 to 1024 (and k = V), ties and
+signed zeros, rows whose threshold bin overflows the candidate list (the
+exact in-CTA refinement: all-equal rows, values that differ only in low
+mantissa bits, a huge tie at the top), and the logits of the full Gemma-2
+shaped path."""
 import numpy as np
 import pytest
 
@@ -57,11 +59,11 @@ CASES = [
     (1, 5000, 1, False),
     (3, 5000, 7, True),
     (2, 4096, 64, False),
-    (4, 70000, 300, True),     # 35 slices, KP 512: two merge launches
-    (1, 2049, 1024, False),    # a one-logit tail slice
+    (4, 70000, 300, True),
+    (1, 2049, 1024, False),
     (2, 1024, 1024, False),    # k = V
     (5, 100, 13, True),
-    (2, 300000, 1000, False),  # 147 slices, KP 1024: three merge launches
+    (2, 300000, 1000, False),
 ]
 
 
@@ -85,6 +87,26 @@ def test_greedy_and_signed_zero():
     z[0, 2500] = 1.0
     _, gi, _ = rq.rq_topk_sample(dev(z), 5, 1.0, 1, 0)
     assert gi.cpu().numpy().tolist() == [[2500, 0, 1, 2, 3]]
+
+
+def _heavy_ties(kind, V, seed):
+    rng = np.random.default_rng(seed)
+    if kind == "all_equal":
+        return np.full((2, V), 1.75, np.float32)
+    if kind == "low_bits":    # one 12-bit bin: only mantissa bits below it differ
+        y = 1.0 + (rng.integers(0, 977, (2, V)) * 2.0 ** -20)
+        return y.astype(np.float32)
+    y = rng.normal(0, 1, (2, V)).astype(np.float32)    # a huge tie at the top
+    y[:, rng.choice(V, 20000, replace=False)] = 9.5
+    return y
+
+
+@pytest.mark.parametrize("kind", ["all_equal", "low_bits", "top_tie"])
+@pytest.mark.parametrize("k", [1, 50, 1024])
+def test_threshold_bin_overflow(kind, k):
+    y = _heavy_ties(kind, 30000, 17)
+    for step in (0, 3):
+        _check(y, k, 1.1, seed=8, step=step)
 
 
 def test_many_steps_same_draws():
