@@ -44,9 +44,10 @@
  *                               major (columns 32c..32c+31 of every row form
  *                               one contiguous [V][32] block, the row's
  *                               "slice"); each slice holds its 32 codes in a
- *                               permuted order, entry = (i << 10) | c with i
- *                               in [0,32) the pair's position in the slice
- *                               and c its code.  The order only changes the
+ *                               permuted order, entry = (i << s) | c with i
+ *                               in [0,32) the pair's position in the slice,
+ *                               c its code and 2^s the smallest power of two
+ *                               >= K, at least 32 (s = 10 at K = 1024).  The order only changes the
  *                               summation order; entries with c >= K add 0
  *                               to the logits (rq_decode_rows clamps them to
  *                               K-1).  Batch 1 streams it fastest; larger
@@ -221,6 +222,15 @@ RQ_API int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed,
               void *stream);
 
 /*
+ * rq_last_cuda_error -- the CUDA runtime error code behind the last
+ * RQ_ERR_CUDA returned to the calling host thread (0 if none); clear != 0
+ * resets it.  rq_cuda_error_name gives the runtime's name for a code (a
+ * static string).  Diagnostics of this library, no counterpart in the pages.
+ */
+RQ_API int rq_last_cuda_error(int clear);
+RQ_API const char *rq_cuda_error_name(int err);
+
+/*
  * rq_topk_sample -- top-k of softcapped logits and a temperature draw among
  * them (generation beyond greedy argmax; the pages state no sampler, see the
  * "Gemma-2-2B combined RQ+NF4" note on generation, so this is the plain
@@ -284,7 +294,7 @@ RQ_API int rq_encode(const float *X, rq_dims d, const float *C, uint16_t *codes,
  * repeated banks as a maximum bipartite matching per step allows (~1.5).
  * Same bytes, same sums (in another order).  Run once per artifact.
  *   codes_u16 (device) uint16 [V][M*L], values < K (larger values keep
- *             their low 10 bits); out (device) uint16 [V][M*L], must not
+ *             their low s bits); out (device) uint16 [V][M*L], must not
  *             overlap codes_u16; stats (device) uint64 [2] or NULL:
  *             receives (steps scheduled, bank passes needed) summed over
  *             all warps, for reporting the schedule's quality.

@@ -27,6 +27,7 @@ __all__ = [
     "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
     "rq_pack10", "rq_device_error", "rq_set_profile_events", "rq_lut_logits_static",
     "rq_greedy_step", "rq_encode", "rq_topk_workspace_bytes", "rq_topk_sample",
+    "rq_last_cuda_error", "rq_cuda_error_name",
 ]
 
 U16 = 0
@@ -51,7 +52,11 @@ def dims(V, D, M, L, K) -> RqDims:
 class RqError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
-        super().__init__(f"{fn} failed: {rq_status_string(status)} ({status})")
+        msg = f"{fn} failed: {rq_status_string(status)} ({status})"
+        if status == 4:   # RQ_ERR_CUDA: name the runtime error behind it
+            err = rq_last_cuda_error(clear=True)
+            msg += f" [{rq_cuda_error_name(err)}]"
+        super().__init__(msg)
 
 
 _lib = None
@@ -76,6 +81,8 @@ _SIGNATURES = {
     "rq_pack10": (_i, [_p, RqDims, _p, _p]),
     "rq_encode": (_i, [_p, RqDims, _p, _p, _p]),
     "rq_topk_workspace_bytes": (_sz, [_i64, _i, _i]),
+    "rq_last_cuda_error": (_i, [_i]),
+    "rq_cuda_error_name": (ctypes.c_char_p, [_i]),
     "rq_topk_sample": (_i, [_p, _i64, _i, _i, _f, ctypes.c_uint64, ctypes.c_uint64, _p, _p, _p,
                             _p, _sz, _p]),
     "rq_device_error": (_i, [ctypes.POINTER(ctypes.c_uint32), _i]),
@@ -274,6 +281,14 @@ def rq_encode(X, C, d: RqDims, out=None, stream=None):
                                         _cuda(C, torch.float32, "C"),
                                         _cuda(out, torch.uint16, "codes"), _stream(stream)))
     return out
+
+
+def rq_last_cuda_error(clear: bool = False) -> int:
+    return int(lib().rq_last_cuda_error(int(bool(clear))))
+
+
+def rq_cuda_error_name(err: int) -> str:
+    return lib().rq_cuda_error_name(int(err)).decode()
 
 
 def rq_topk_workspace_bytes(V: int, B: int, k: int) -> int:

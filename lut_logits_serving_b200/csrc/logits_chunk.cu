@@ -156,22 +156,24 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return x;
 }
 
-// RQ_CODES_SCHED, one token: the 32 entries (i << 10 | c) of a row's chunk
+// RQ_CODES_SCHED, one token: the 32 entries (i << KSH | c) of a row's chunk
 // slice (four 16-byte code vectors), each the word offset of its table entry
-// in the chunk's 32 x 1024 tables at shared address `tbase`.  All 32 loads
-// are issued before any add; the sum is a tree.  The 15-bit masks keep every
-// address aligned and inside the 128 KB of tables.
-template <int N>
+// in the chunk's 32 tables of stride 2^KSH at shared address `tbase`.  All
+// 32 loads are issued before any add; the sum is a tree.  The (5 + KSH)-bit
+// masks keep every address aligned and inside the 32 * 2^KSH * 4 bytes of
+// tables.
+template <int KSH, int N>
 __device__ __forceinline__ float chunk32_sched_tb1(uint32_t tbase, const uint4 (&w)[N]) {
   static_assert(N == 4, "a scheduled slice is four 16-byte vectors");
+  constexpr uint32_t EM = (1u << (5 + KSH)) - 1u;
   const uint32_t ws[16] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w,
                            w[2].x, w[2].y, w[2].z, w[2].w, w[3].x, w[3].y, w[3].z, w[3].w};
   float x[32];
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
-    x[2 * q] = lds_f32(tbase + ((ws[q] & 0x7FFFu) << 2));
-    // high entry: ((w & 0x7FFF0000) * 2^18) >> 32 = ((w >> 16) & 0x7FFF) * 4
-    x[2 * q + 1] = lds_f32(tbase + __umulhi(ws[q] & 0x7FFF0000u, 1u << 18));
+    x[2 * q] = lds_f32(tbase + ((ws[q] & EM) << 2));
+    // high entry: ((w & EM << 16) * 2^18) >> 32 = ((w >> 16) & EM) * 4
+    x[2 * q + 1] = lds_f32(tbase + __umulhi(ws[q] & (EM << 16), 1u << 18));
   }
 #pragma unroll
   for (int st = 1; st < 32; st <<= 1)
@@ -193,8 +195,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int TB, int KT, int NST, int FMT>
-__global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS, 1)
+// KSH: the table stride 2^KSH of RQ_CODES_SCHED entries (unused otherwise);
+// MINB: CTAs per SM the register budget is made for.
+template <int TB, int KT, int NST, int FMT, int KSH, int MINB>
+__global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS, MINB)
     logits_chunk_u16_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
   constexpr bool SCHED = FMT == RQ_CODES_SCHED;
   using S = ChunkShape<TB, SCHED>;
@@ -204,7 +208,7 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS
   // compiler keeps the shared address space
   unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int K = KT > 0 ? KT : a.K;
-  const int KS = SCHED ? 1024 : K;           // table stride (entries) in shared memory
+  const int KS = SCHED ? (1 << KSH) : K;     // table stride (entries) in shared memory
   float *Ts = reinterpret_cast<float *>(smem);
   const size_t t_bytes = (size_t)align_up((int64_t)S::PC * KS * TB * 4, 1024);
   unsigned char *stages = smem + t_bytes;
@@ -272,14 +276,14 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS
       } else {
         mbar_arrive_expect_tx(tb, per * np);
         for (int p = 0; p < np; ++p)
-          bulk_g2s(smem_addr(Ts) + (uint32_t)p * 1024 * TB * 4, src + (size_t)p * K * TB, per, tb);
+          bulk_g2s(smem_addr(Ts) + (uint32_t)p * KS * TB * 4, src + (size_t)p * K * TB, per, tb);
       }
     }
     if constexpr (SCHED) {
-      if (K < 1024) {                        // codes >= K read zeros
-        const int pad = (1024 - K) * TB;
+      if (K < KS) {                          // codes >= K read zeros
+        const int pad = (KS - K) * TB;
         for (int q = tid; q < np * pad; q += S::THREADS)
-          Ts[(q / pad) * 1024 * TB + K * TB + q % pad] = 0.f;
+          Ts[(q / pad) * KS * TB + K * TB + q % pad] = 0.f;
       }
     }
   } else {
@@ -338,7 +342,7 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS
 #pragma unroll
     for (int b = 0; b < TB; ++b) acc[b] = 0.f;
     if constexpr (SCHED) {
-      acc[0] = chunk32_sched_tb1(tt, w);     // the row's whole 32-pair slice
+      acc[0] = chunk32_sched_tb1<KSH>(tt, w);   // the row's whole 32-pair slice
     } else {
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
@@ -528,31 +532,42 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Variant {
-  int TB, KT, NST, FMT;
+  int TB, KT, NST, FMT, KSH;
   int PC, R, THREADS, STAGE_BYTES;
   const void *fn;
 };
 
-#define RQ_CHUNK_VARIANT(TB, KT, NST, FMT)                                           \
-  Variant {                                                                          \
-    TB, KT, NST, FMT, ChunkShape<TB, FMT == RQ_CODES_SCHED>::PC,                     \
-        ChunkShape<TB, FMT == RQ_CODES_SCHED>::R,                                    \
-        ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS,                              \
-        ChunkShape<TB, FMT == RQ_CODES_SCHED>::STAGE_BYTES,                          \
-        reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, NST, FMT>)   \
+#define RQ_CHUNK_VARIANT(TB, KT, NST, FMT, KSH, MINB)                                      \
+  Variant {                                                                                \
+    TB, KT, NST, FMT, KSH, ChunkShape<TB, FMT == RQ_CODES_SCHED>::PC,                      \
+        ChunkShape<TB, FMT == RQ_CODES_SCHED>::R,                                          \
+        ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS,                                    \
+        ChunkShape<TB, FMT == RQ_CODES_SCHED>::STAGE_BYTES,                                \
+        reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, NST, FMT, KSH, MINB>) \
   }
 
-// 128 KB table chunk + NST stages (3 x 32 KB or 5 x 16 KB) per CTA, one CTA
-// per SM.  K = 1024 has its own instances (table offsets as immediates).
+// Plain codes: 128 KB table chunk + NST stages (3 x 32 KB or 5 x 16 KB) per
+// CTA, one CTA per SM; K = 1024 has its own instances (table offsets as
+// immediates).  Scheduled codes: one instance per table stride 2^KSH; up to
+// 256 entries a chunk's tables (<= 32 KB) and two 32 KB stages leave room
+// for two CTAs per SM.
 const Variant kVariants[] = {
-    RQ_CHUNK_VARIANT(1, 1024, 3, RQ_CODES_U16), RQ_CHUNK_VARIANT(2, 1024, 3, RQ_CODES_U16),
-    RQ_CHUNK_VARIANT(4, 1024, 5, RQ_CODES_U16), RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_U16),
-    RQ_CHUNK_VARIANT(2, 0, 3, RQ_CODES_U16),    RQ_CHUNK_VARIANT(4, 0, 5, RQ_CODES_U16),
-    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_SCHED),
+    RQ_CHUNK_VARIANT(1, 1024, 3, RQ_CODES_U16, 0, 1),
+    RQ_CHUNK_VARIANT(2, 1024, 3, RQ_CODES_U16, 0, 1),
+    RQ_CHUNK_VARIANT(4, 1024, 5, RQ_CODES_U16, 0, 1),
+    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_U16, 0, 1),
+    RQ_CHUNK_VARIANT(2, 0, 3, RQ_CODES_U16, 0, 1),
+    RQ_CHUNK_VARIANT(4, 0, 5, RQ_CODES_U16, 0, 1),
+    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_SCHED, 10, 1),
+    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_SCHED, 9, 1),
+    RQ_CHUNK_VARIANT(1, 0, 2, RQ_CODES_SCHED, 8, 2),
+    RQ_CHUNK_VARIANT(1, 0, 2, RQ_CODES_SCHED, 7, 2),
+    RQ_CHUNK_VARIANT(1, 0, 2, RQ_CODES_SCHED, 6, 2),
+    RQ_CHUNK_VARIANT(1, 0, 2, RQ_CODES_SCHED, 5, 2),
 };
 
 size_t variant_smem(const Variant &v, int K) {
-  const int KS = v.FMT == RQ_CODES_SCHED ? 1024 : K;
+  const int KS = v.FMT == RQ_CODES_SCHED ? (1 << v.KSH) : K;
   return 1024 + (size_t)align_up((int64_t)v.PC * KS * v.TB * 4, 1024) +
          (size_t)v.NST * v.STAGE_BYTES + 1024;
 }
@@ -572,6 +587,7 @@ ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di)
     const Variant &v = kVariants[i];
     if (v.TB != TB || v.FMT != fmt) continue;
     if (v.KT != 0 && v.KT != K) continue;
+    if (fmt == RQ_CODES_SCHED && v.KSH != sched_shift(K)) continue;
     const size_t smem = variant_smem(v, K);
     if (smem > (size_t)di.max_smem_optin) continue;
     cp.ok = true;
@@ -612,12 +628,18 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
-  static bool attr_set[128][sizeof(kVariants) / sizeof(kVariants[0])] = {};
-  if (di.device < 128 && !attr_set[di.device][cp.variant]) {
+  // the shared-memory limit set so far per (device, instance): raised when a
+  // larger K needs more (plain-code tables scale with K)
+  constexpr int NV = sizeof(kVariants) / sizeof(kVariants[0]);
+  static size_t smem_set[128][NV] = {};
+  static int occ_cache[128][NV] = {};
+  static size_t occ_smem[128][NV] = {};
+  if (di.device >= 128) return cudaErrorInvalidDevice;
+  if (cp.smem > smem_set[di.device][cp.variant]) {
     cudaError_t e = cudaFuncSetAttribute(var.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cp.smem);
     if (e != cudaSuccess) return e;
-    attr_set[di.device][cp.variant] = true;
+    smem_set[di.device][cp.variant] = cp.smem;
   }
 
   ChunkArgs a;
@@ -631,7 +653,17 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   a.K = K;
   a.B = B;
   a.nch = cp.nch;
-  int64_t cpc = di.sms / cp.nch;
+  // CTAs per SM this instance reaches (shared memory and registers)
+  int occ = occ_cache[di.device][cp.variant];
+  if (occ == 0 || occ_smem[di.device][cp.variant] != cp.smem) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, var.fn, var.THREADS, cp.smem) !=
+            cudaSuccess ||
+        occ < 1)
+      occ = 1;
+    occ_cache[di.device][cp.variant] = occ;
+    occ_smem[di.device][cp.variant] = cp.smem;
+  }
+  int64_t cpc = (int64_t)di.sms * occ / cp.nch;
   if (cpc < 1) cpc = 1;
   if (cpc > a.ntiles) cpc = a.ntiles;
   a.cpc = (int)cpc;

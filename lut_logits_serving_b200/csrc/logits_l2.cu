@@ -33,6 +33,7 @@ struct L2Args {
   float *am_val;      // [Btot][nblk] or null
   int *am_idx;
   CodeFix fix;
+  int ssh;            // RQ_CODES_SCHED entry shift (table stride 2^ssh)
 };
 
 template <int VW>
@@ -108,11 +109,12 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         }
       }
     } else if (FMT == RQ_CODES_SCHED) {
-      // chunk-major [P/32][V][32]; 32 entries (i << 10 | c) per chunk slice,
-      // in any order
+      // chunk-major [P/32][V][32]; 32 entries (i << ssh | c) per chunk
+      // slice, in any order
       const uint16_t *cbase = static_cast<const uint16_t *>(a.codes) + v * 32;
       const int nc = a.P / 32;
-      const bool kfull = K >= 1024;       // every 10-bit code indexes a real entry
+      const uint32_t cmask = (1u << a.ssh) - 1u;
+      const bool kfull = K > (int)cmask;  // every masked code indexes a real entry
       for (int cc = 0; cc < nc; ++cc) {
         const uint4 *crow = reinterpret_cast<const uint4 *>(cbase + (size_t)cc * a.V * 32);
         uint32_t wd[16];
@@ -128,8 +130,8 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const uint32_t e = (j & 1) ? (wd[j >> 1] >> 16) : (wd[j >> 1] & 0xFFFFu);
-          const uint32_t c = e & 0x3FFu;
-          const uint32_t pp = (e >> 10) & 31u;                 // pair within the chunk
+          const uint32_t c = e & cmask;
+          const uint32_t pp = (e >> a.ssh) & 31u;              // pair within the chunk
           if (kfull || c < (uint32_t)K) add_vec<VW>(tc + ((size_t)pp * K + c) * Bs, acc);
         }
       }
@@ -208,8 +210,8 @@ __global__ void __launch_bounds__(256) logits_generic_kernel(const L2Args a, int
       if (fmt == RQ_CODES_SCHED) {
         const uint32_t e =
             static_cast<const uint16_t *>(a.codes)[((size_t)(p >> 5) * a.V + v) * 32 + (p & 31)];
-        const uint32_t c = e & 0x3FFu;
-        const int pp = (p & ~31) + (int)((e >> 10) & 31u);
+        const uint32_t c = e & ((1u << a.ssh) - 1u);
+        const int pp = (p & ~31) + (int)((e >> a.ssh) & 31u);
         if (c < (uint32_t)a.K) z += __ldg(tl + ((size_t)pp * a.K + c) * a.Bs);
         continue;
       }
@@ -270,6 +272,7 @@ cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K
   a.am_val = am_val;
   a.am_idx = am_idx;
   a.fix = make_codefix(K);
+  a.ssh = sched_shift(K);
   const bool codes16 = (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
   const bool fast_fmt = fmt == RQ_CODES_U16     ? (P % 8 == 0)
                         : fmt == RQ_CODES_SCHED ? (P % 32 == 0)

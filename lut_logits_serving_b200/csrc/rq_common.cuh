@@ -54,13 +54,24 @@ __device__ __forceinline__ uint32_t packed10_code(const uint8_t *row, int p) {
   return (w >> (bit & 7)) & 0x3FFu;
 }
 
-// Code of pair p of row `id` in RQ_CODES_SCHED (chunk-major [P/32][V][32],
-// entries i << 10 | c): find position p % 32 in the row's chunk slice.
+// RQ_CODES_SCHED entry = (i << s) | c: i the pair's position in its 32-pair
+// slice, c the code, and 2^s the table stride -- the smallest power of two
+// >= K, at least 32, so that the shared-memory bank of the entry's table
+// word (entry mod 32) is the code's own bank (c mod 32).
+__host__ __device__ __forceinline__ int sched_shift(int K) {
+  int s = 5;
+  while ((1 << s) < K) ++s;
+  return s;
+}
+
+// Code of pair p of row `id` in RQ_CODES_SCHED (chunk-major [P/32][V][32]):
+// find position p % 32 in the row's chunk slice.
 __device__ __forceinline__ uint32_t sched_code(const uint16_t *codes, int64_t V, int64_t id,
-                                               int p) {
+                                               int p, int sh) {
   // the slice is 64 bytes at a 64-byte aligned offset: four 16-byte loads
   const uint4 *g = reinterpret_cast<const uint4 *>(codes + ((int64_t)(p >> 5) * V + id) * 32);
   const uint32_t want = (uint32_t)(p & 31);
+  const uint32_t cmask = (1u << sh) - 1u;
   uint32_t c = 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -68,8 +79,9 @@ __device__ __forceinline__ uint32_t sched_code(const uint16_t *codes, int64_t V,
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      if (((w[k] >> 10) & 31u) == want) c = w[k] & 0x3FFu;
-      if (((w[k] >> 26) & 31u) == want) c = (w[k] >> 16) & 0x3FFu;
+      const uint32_t lo = w[k] & 0xFFFFu, hi = w[k] >> 16;
+      if (((lo >> sh) & 31u) == want) c = lo & cmask;
+      if (((hi >> sh) & 31u) == want) c = hi & cmask;
     }
   }
   return c;
@@ -103,7 +115,7 @@ __device__ __forceinline__ void decode_subspace(const DecodeSpec &a, int64_t id,
   auto code = [&](int p) -> uint32_t {
     uint32_t c;
     if (a.fmt == RQ_CODES_U16) c = crow16[p];
-    else if (a.fmt == RQ_CODES_SCHED) c = sched_code(all16, a.V, id, p);
+    else if (a.fmt == RQ_CODES_SCHED) c = sched_code(all16, a.V, id, p, sched_shift(a.K));
     else c = packed10_code(crow10, p);
     return a.fix(c);
   };
@@ -343,7 +355,7 @@ cudaError_t launch_topk_sample(const float *logits, int64_t V, int B, int k, dou
                                int32_t *idx, int32_t *token, void *ws, cudaStream_t s);
 cudaError_t launch_encode(const float *X, int64_t N, const float *C, int D, int M, int L, int K,
                           uint16_t *codes, cudaStream_t s);
-cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, uint16_t *out,
+cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, int K, uint16_t *out,
                                  unsigned long long *stats, cudaStream_t s);
 
 // Vocabulary-tiled pass with the LUT chunk resident in shared memory.

@@ -92,7 +92,14 @@ bool fmt_ok(const rq_dims &d, int fmt) {
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-int status_of(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+// The last CUDA error a call of this host thread met (rq_last_cuda_error).
+thread_local int t_last_cuda_error = 0;
+
+int status_of(cudaError_t e) {
+  if (e == cudaSuccess) return RQ_OK;
+  t_last_cuda_error = (int)e;
+  return RQ_ERR_CUDA;
+}
 
 // Workspace layout of rq_lut_logits:
 //   tiled path (B <= 4):  [partials: nch*B*V floats][argmax keys: B x u64]
@@ -373,7 +380,7 @@ int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out, uint64
   const size_t bytes = rq_codes_bytes(d, RQ_CODES_U16);
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(codes_u16), b0 = reinterpret_cast<uintptr_t>(out);
   if (a0 < b0 + bytes && b0 < a0 + bytes) return RQ_ERR_INVALID_ARGUMENT;   // overlap
-  return status_of(launch_prepare_sched(codes_u16, d.V, d.M * d.L, out,
+  return status_of(launch_prepare_sched(codes_u16, d.V, d.M * d.L, d.K, out,
                                         reinterpret_cast<unsigned long long *>(stats),
                                         static_cast<cudaStream_t>(stream)));
 }
@@ -419,6 +426,14 @@ int rq_topk_sample(const float *logits, int64_t V, int B, int k, float temperatu
                                       topk_val, topk_idx, token, ws,
                                       static_cast<cudaStream_t>(stream)));
 }
+
+int rq_last_cuda_error(int clear) {
+  const int e = t_last_cuda_error;
+  if (clear) t_last_cuda_error = 0;
+  return e;
+}
+
+const char *rq_cuda_error_name(int err) { return cudaGetErrorName(static_cast<cudaError_t>(err)); }
 
 int rq_set_profile_events(void *start, void *stop) {
   if ((start == nullptr) != (stop == nullptr)) return RQ_ERR_INVALID_ARGUMENT;

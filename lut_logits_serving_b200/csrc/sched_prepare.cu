@@ -17,10 +17,12 @@
 // Any order gives the same logits up to fp32 summation order; only the
 // speed depends on it.
 //
-// Entry format: (i << 10) | c, i = pair position in the 32-pair chunk,
-// c = code (< 1024): for 1024-entry tables laid out back to back it is the
-// word offset of the table entry.  Layout: chunk-major [P/32][V][32], so the
-// 32-pair slice that one CTA of the batch-1 pass streams is contiguous.
+// Entry format: (i << s) | c, i = pair position in the 32-pair chunk,
+// c = code, 2^s = the table stride (the smallest power of two >= K, at least
+// 32): for tables of that stride laid out back to back it is the word offset
+// of the table entry, and its bank (entry mod 32) is the code's.  Layout:
+// chunk-major [P/32][V][32], so the 32-pair slice that one CTA of the
+// batch-1 pass streams is contiguous.
 #include "rq_common.cuh"
 
 namespace rq {
@@ -28,7 +30,7 @@ namespace rq {
 constexpr int kSchedThreads = 16;   // one problem per thread, state in smem
 
 __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
-    const uint16_t *__restrict__ codes, int64_t V, int P, uint16_t *__restrict__ out,
+    const uint16_t *__restrict__ codes, int64_t V, int P, int sh, uint16_t *__restrict__ out,
     unsigned long long *stats) {
   __shared__ uint16_t s_code[kSchedThreads][32][32];   // codes of each lane (row)
   __shared__ uint32_t s_lmask[kSchedThreads][32];      // per bank: lanes with unused codes in it
@@ -53,7 +55,7 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
     if (row < V) {
       present |= 1u << ln;
       const uint16_t *src = codes + row * P + c * 32;
-      for (int k = 0; k < 32; ++k) cd[ln][k] = src[k] & 0x3FFu;
+      for (int k = 0; k < 32; ++k) cd[ln][k] = src[k] & ((1u << sh) - 1u);
     }
   }
 
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
       used[ln] |= 1u << pick;
       const int64_t row = rb * 32 + ln;
       // chunk-major: chunk c of every row is one contiguous [V][32] block
-      out[((int64_t)c * V + row) * 32 + step] = (uint16_t)((pick << 10) | cd[ln][pick]);
+      out[((int64_t)c * V + row) * 32 + step] = (uint16_t)((pick << sh) | cd[ln][pick]);
     }
     for (int b = 0; b < 32; ++b) maxc = cnt[b] > maxc ? cnt[b] : maxc;
     passes += (unsigned long long)maxc;
@@ -156,7 +158,7 @@ __global__ void __launch_bounds__(kSchedThreads) prepare_sched_kernel(
   }
 }
 
-cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, uint16_t *out,
+cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, int K, uint16_t *out,
                                  unsigned long long *stats, cudaStream_t s) {
   const int64_t probs = (V + 31) / 32 * (P / 32);
   const int64_t blocks = (probs + kSchedThreads - 1) / kSchedThreads;
@@ -165,7 +167,8 @@ cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, uint16
     cudaError_t e = cudaMemsetAsync(stats, 0, 2 * sizeof(unsigned long long), s);
     if (e != cudaSuccess) return e;
   }
-  prepare_sched_kernel<<<(unsigned)blocks, kSchedThreads, 0, s>>>(codes, V, P, out, stats);
+  prepare_sched_kernel<<<(unsigned)blocks, kSchedThreads, 0, s>>>(codes, V, P, sched_shift(K),
+                                                                 out, stats);
   return cudaGetLastError();
 }
 

@@ -79,6 +79,9 @@ CASES = [
     (2000, 96, 16, 3, 100),    # L = 3, non-power-of-two K (clamped codes path)
     (1500, 64, 64, 1, 32),     # ds = 1, L = 1
     (700, 9, 3, 1, 7),         # P = 3: generic fallback
+    (1200, 128, 64, 1, 100),   # scheduled table stride 128 (two CTAs per SM)
+    (900, 96, 16, 2, 300),     # scheduled table stride 512
+    (600, 64, 32, 2, 37),      # scheduled table stride 64
 ]
 
 
@@ -245,12 +248,24 @@ def test_pack10_matches_oracle(P):
 
 # ------------------------------------------------------ scheduled codes
 
+def _sched_shift(K):
+    """The entry shift the header defines: table stride 2^s, the smallest
+    power of two >= K and at least 32."""
+    s = 5
+    while (1 << s) < K:
+        s += 1
+    return s
+
+
 @pytest.mark.parametrize("shape", [(4096, 192, 32, 2, 256), (1000, 96, 16, 2, 1024),
-                                   (77, 96, 32, 1, 64), (3000, 288, 48, 2, 1024)])
+                                   (77, 96, 32, 1, 64), (3000, 288, 48, 2, 1024),
+                                   (500, 64, 32, 2, 16), (700, 64, 32, 1, 37),
+                                   (900, 128, 64, 1, 100), (333, 64, 32, 2, 300)])
 def test_prepare_sched_is_a_permutation_within_groups(shape):
     """Chunk-major [P/32][V][32]; every row's 32-entry slice holds exactly
-    the slice's 32 (position, code) pairs, each once, as i << 10 | c."""
+    the slice's 32 (position, code) pairs, each once, as i << s | c."""
     V, D, M, L, K = shape
+    sh = _sched_shift(K)
     codes = synth.codes(V, M, L, K, 4)
     d = rq.dims(V, D, M, L, K)
     P = M * L
@@ -258,9 +273,9 @@ def test_prepare_sched_is_a_permutation_within_groups(shape):
     raw = out.view(torch.int16).cpu().numpy().view(np.uint16).astype(np.int64)
     assert raw.size == V * P
     e = raw.reshape(P // 32, V, 32).transpose(1, 0, 2)     # [V, P/32, 32]
-    assert np.all(e >> 15 == 0)
-    pos = e >> 10
-    code = e & 1023
+    assert np.all(e >> (sh + 5) == 0)
+    pos = e >> sh
+    code = e & ((1 << sh) - 1)
     order = np.argsort(pos, axis=2, kind="stable")
     assert np.array_equal(np.take_along_axis(pos, order, 2),
                           np.broadcast_to(np.arange(32), pos.shape))
