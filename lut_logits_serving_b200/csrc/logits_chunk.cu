@@ -531,6 +531,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+}  // namespace
+
+bool encode_tmap_2d_u16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                        uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swz) {
+  if (encode_fn() == nullptr) return false;
+  const cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  const cuuint64_t gstride[1] = {(cuuint64_t)stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estride[2] = {1u, 1u};
+  return encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), gdim,
+                     gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
 struct Variant {
   int TB, KT, NST, FMT, KSH;
   int PC, R, THREADS, STAGE_BYTES;

@@ -62,7 +62,10 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
   const int q = lane % G;
   const int rw = lane / G;
   const int tok = q * VW;         // first token of this lane, within the group
-  const float *tl = a.lut + a.lut_t0 + tok;
+  // G is a power of two, so lanes can lie past the group's last token (and
+  // past the table's token stride Bs): they read token 0's entries instead,
+  // and their sums are never stored
+  const float *tl = a.lut + a.lut_t0 + (tok < a.nb ? tok : 0);
   const int K = a.K, Bs = a.Bs;
 
   ArgBest best[VW];

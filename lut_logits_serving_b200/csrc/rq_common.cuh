@@ -386,6 +386,22 @@ cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t
 cudaError_t launch_argmax_keys(unsigned long long *keys, int B, int32_t *argmax,
                                const DecodeSpec *rows_spec, uint16_t *rows, cudaStream_t s);
 
+// 2-D uint16 tensor map (driver entry point looked up once); false on failure.
+bool encode_tmap_2d_u16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                        uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swz);
+
+// Token groups (<= 32) by decoding rows into shared memory and fp32 FMAs
+// with the hidden states (ds = 6, L = 2, uint16 codes, K <= 1024).  Argmax
+// partials go to columns [0, grid) of [B][nblk]; the rest are set to -inf.
+bool decode_fma_applies(int fmt, int64_t V, int D, int M, int L, int K, int B, const float *C,
+                        const void *codes, const DevInfo &di);
+int decode_fma_blocks(int64_t V, const DevInfo &di);
+cudaError_t launch_logits_decode_fma(const float *h, const float *C, const void *codes,
+                                     int64_t V, int D, int M, int K, int t0, int nb, float cap,
+                                     float *logits, float *am_val, int *am_idx, int nblk,
+                                     const DevInfo &di, cudaStream_t s);
+
 // Batched pass with the LUT read through L2 (token groups of <= 32).
 cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K,
                              const float *lut, int Bs, int lut_t0, int out_t0, int nb,

@@ -191,6 +191,7 @@ int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, i
 
 int fused_group(int B) { return B <= 4 ? B : (B < kTokenGroup ? B : kTokenGroup); }
 
+
 // rq_logits_from_hidden and rq_greedy_step: table build per token group,
 // code pass, softcap, logits/argmax, optionally the picked tokens' rows.
 int run_fused(const float *h, const float *C, const void *codes, int fmt, const rq_dims &d, int B,
@@ -216,16 +217,31 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   const int P = d.M * d.L;
   float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
   int *ami = argmax ? reinterpret_cast<int *>(rest + w.ami_off) : nullptr;
+  // Full 32-token groups decode rows into shared memory and multiply them
+  // with the hidden states (measured faster there); other groups read their
+  // tables through L2.  Both write argmax partials into the same [B][nblk].
   const int nblk = sweep_blocks(d, di, false);
-  for (int b0 = 0; b0 < B; b0 += G) {
+  const bool dfma = decode_fma_applies(fmt, d.V, d.D, d.M, d.L, d.K, B, C, codes, di) &&
+                    decode_fma_blocks(d.V, di) <= nblk;
+  cudaError_t e = cudaSuccess;
+  bool marked = false;   // the profile start goes before the first logits kernel
+  for (int b0 = 0; b0 < B && e == cudaSuccess; b0 += G) {
     const int nb = B - b0 < G ? B - b0 : G;
-    cudaError_t e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, s);
-    if (e != cudaSuccess) return status_of(e);
-    if (b0 == 0 && (e = prof_mark(t_prof_start, s)) != cudaSuccess) return status_of(e);
-    e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, 0, b0, nb, softcap, logits, amv, ami,
-                         nblk, s);
-    if (e != cudaSuccess) return status_of(e);
+    if (dfma && nb == kTokenGroup) {
+      if (!marked && (e = prof_mark(t_prof_start, s)) != cudaSuccess) break;
+      marked = true;
+      e = launch_logits_decode_fma(h, C, codes, d.V, d.D, d.M, d.K, b0, nb, softcap, logits, amv,
+                                   ami, nblk, di, s);
+      continue;
+    }
+    e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, s);
+    if (e == cudaSuccess && !marked) e = prof_mark(t_prof_start, s);
+    marked = true;
+    if (e == cudaSuccess)
+      e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, 0, b0, nb, softcap, logits, amv, ami,
+                           nblk, s);
   }
+  if (e != cudaSuccess) return status_of(e);
   if (cudaError_t e = prof_mark(t_prof_stop, s)) return status_of(e);
   if (argmax)
     return status_of(launch_argmax_finalize(amv, ami, nblk, B, argmax, rows_spec, rows, s));

@@ -107,7 +107,7 @@ def test_logits_and_argmax(case, B, fmt):
     # the fused call gives the same numbers
     logits2, am2, _ = rq.rq_logits_from_hidden(dh, dC, dc, fmt, d, cap, want_argmax=True)
     assert_logits_close(logits2.cpu().numpy(), ref)
-    assert np.array_equal(am2.cpu().numpy(), am.cpu().numpy())
+    check_argmax(am2.cpu().numpy(), ref)      # (B >= 8 may sum in the decode order)
     # argmax alone (logits not written) agrees
     _, am3, _ = rq.rq_lut_logits(dc, fmt, d, lut, B, cap, want_logits=False, want_argmax=True)
     assert np.array_equal(am3.cpu().numpy(), am.cpu().numpy())
@@ -334,3 +334,60 @@ def test_greedy_step_rows_are_the_picked_tokens_rows(B, fmt):
                                          want_logits=False)
     assert torch.equal(am2, am) and torch.equal(rows2, rows)
     assert rq.rq_device_error() == 0
+
+
+# --------------------------------------- batched rows decoded in shared memory
+
+@pytest.mark.parametrize("V,M,K,B", [
+    (1, 8, 64, 8),            # a single row
+    (255, 8, 1024, 9),        # fewer rows than one CTA's share
+    (148 * 1024 + 7, 16, 300, 32),   # every CTA two tiles, K not a power of two
+    (5000, 40, 7, 33),        # 5 code groups, a one-token second group (table path)
+    (3001, 16, 1024, 64),     # two full token groups
+    (2500, 8, 256, 48),       # a full group (decoded) and a 16-token group (tables)
+])
+def test_fused_decode_fma_path(V, M, K, B):
+    """Full 32-token groups with uint16 codes, ds = 6, L = 2, M % 8 == 0: the
+    fused call decodes rows into shared memory and multiplies them with the
+    hidden states (other groups use the tables); logits and argmax must meet
+    the same bounds, with both kinds of group in one call."""
+    D, L = 6 * M, 2
+    C, codes, h = make_case(V, D, M, L, K, B, seed=V + B)
+    d = rq.dims(V, D, M, L, K)
+    ref = oracle_logits(C, codes, h, 30.0)
+    logits, am, _ = rq.rq_logits_from_hidden(dev(h), dev(C), dev(codes.reshape(V, -1)), rq.U16, d,
+                                             30.0, want_argmax=True)
+    assert_logits_close(logits.cpu().numpy(), ref)
+    check_argmax(am.cpu().numpy(), ref)
+    assert rq.rq_device_error() == 0
+
+
+def test_fused_decode_fma_clamps_out_of_range_codes():
+    """Codes >= K read codeword K-1 (non-power-of-two K), as in the other paths."""
+    V, M, K, B = 2000, 8, 100, 32
+    C, codes, h = make_case(V, 6 * M, M, 2, K, B, seed=3)
+    bad = codes.copy()
+    bad[::7, :, 1] = 1000
+    d = rq.dims(V, 6 * M, M, 2, K)
+    ref = oracle_logits(C, np.minimum(bad, K - 1), h, 30.0)
+    logits, _, _ = rq.rq_logits_from_hidden(dev(h), dev(C), dev(bad.reshape(V, -1)), rq.U16, d,
+                                            30.0)
+    assert_logits_close(logits.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("B", [9, 12, 20, 24, 28, 31])
+def test_l2_pass_with_an_exactly_sized_table(B):
+    """Token counts whose lane groups are not a power of two: the table is
+    allocated to exactly [P][K][Bs] (no workspace after it), so every read
+    must stay inside it."""
+    V, D, M, L, K = 3000, 192, 32, 2, 256
+    C, codes, h = make_case(V, D, M, L, K, B, seed=B)
+    d = rq.dims(V, D, M, L, K)
+    Bs = rq.rq_lut_token_stride(B)
+    lut = torch.empty((M * L, K, Bs), dtype=torch.float32, device="cuda")
+    rq.rq_lut_build(dev(h), dev(C), d, lut=lut)
+    logits, am, _ = rq.rq_lut_logits(dev(codes.reshape(V, -1)), rq.U16, d, lut, B, 30.0,
+                                     want_argmax=True)
+    ref = oracle_logits(C, codes, h, 30.0)
+    assert_logits_close(logits.cpu().numpy(), ref)
+    check_argmax(am.cpu().numpy(), ref)
