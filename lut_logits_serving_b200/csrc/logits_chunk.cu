@@ -455,6 +455,61 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(
   }
 }
 
+// The same sum for few rows and many chunks (small V, e.g. an RQ-coded MLP
+// matrix with 72-288 chunks): a block covers 64 rows (16 float4 lanes), and
+// its 16 lane groups sum every 16th chunk; the 16 partial sums are then added
+// in lane-group order (a fixed order: deterministic).  Requires V % 4 == 0
+// and 16-byte aligned logits.  Grid (ceil(V/64), B), 256 threads.
+__global__ void __launch_bounds__(256) reduce_partials_split_kernel(
+    const float *__restrict__ partial, int nch, int B, int64_t V, float cap, float *logits,
+    unsigned long long *keys) {
+  __shared__ float4 part[16][16];
+  griddep_wait();
+  const int b = blockIdx.y;
+  const int rl = threadIdx.x & 15, cs = threadIdx.x >> 4;
+  const int64_t V4 = V / 4;
+  const int64_t v4 = (int64_t)blockIdx.x * 16 + rl;
+  float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (v4 < V4) {
+    const float4 *src = reinterpret_cast<const float4 *>(partial + (size_t)b * V) + v4;
+    const size_t cstride = (size_t)B * V4;
+    for (int c = cs; c < nch; c += 16) {
+      const float4 t = __ldcs(src + c * cstride);
+      z.x += t.x;
+      z.y += t.y;
+      z.z += t.z;
+      z.w += t.w;
+    }
+  }
+  part[cs][rl] = z;
+  __syncthreads();
+  griddep_launch_dependents();
+  if (cs != 0) return;                       // lanes 0..15 of warp 0 finish
+  float4 y = part[0][rl];
+  for (int c = 1; c < 16; ++c) {
+    const float4 t = part[c][rl];
+    y.x += t.x;
+    y.y += t.y;
+    y.z += t.z;
+    y.w += t.w;
+  }
+  ArgBest best{-FLT_MAX, INT_MAX};
+  if (v4 < V4) {
+    y = make_float4(softcap_f(y.x, cap), softcap_f(y.y, cap), softcap_f(y.z, cap),
+                    softcap_f(y.w, cap));
+    if (logits) reinterpret_cast<float4 *>(logits + (size_t)b * V)[v4] = y;
+    const int v = (int)(4 * v4);
+    best = arg_better(best, ArgBest{y.x, v});
+    best = arg_better(best, ArgBest{y.y, v + 1});
+    best = arg_better(best, ArgBest{y.z, v + 2});
+    best = arg_better(best, ArgBest{y.w, v + 3});
+  }
+  if (keys == nullptr) return;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) best = arg_better(best, arg_shfl_xor(best, o, 0x0000ffffu));
+  if (rl == 0 && best.i != INT_MAX) atomicMax(keys + b, arg_key(best));
+}
+
 // keys[b] -> argmax[b] (and clears the key).  With `rows` set, the block then
 // rebuilds the picked token's bf16 input row (one thread per subspace).
 template <int DS>
@@ -696,6 +751,15 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
 cudaError_t launch_reduce_partials(const float *partial, int nch, int B, int64_t V, float cap,
                                    float *logits, unsigned long long *keys, int nblk,
                                    cudaStream_t s) {
+  // few rows per chunk: split the chunks over the block (fewer than ~one
+  // 1024-row block per SM otherwise)
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (V < 1024LL * sms && nch >= 32 && (V & 3) == 0 &&
+      (reinterpret_cast<uintptr_t>(logits) & 15) == 0)
+    return pdl_launch(reduce_partials_split_kernel, dim3((unsigned)((V + 63) / 64), (unsigned)B),
+                      dim3(256), 0, s, partial, nch, B, V, cap, logits, keys);
   return pdl_launch(reduce_partials_kernel, dim3((unsigned)nblk, (unsigned)B), dim3(256), 0, s,
                     partial, nch, B, V, cap, logits, keys);
 }

@@ -51,6 +51,32 @@ __global__ void __launch_bounds__(256) lut_build_kernel(const float *__restrict_
   }
 }
 
+// Small tables, B <= 2 (e.g. the RQ-coded MLP matrices: ds = 2, K = 128 or
+// 256): one thread per table row (p, k) over the flattened P*K rows, so every
+// block is full whatever K is.
+template <int DS>
+__global__ void __launch_bounds__(256) lut_build_flat_kernel(const float *__restrict__ h,
+                                                            const float *__restrict__ C, int b0,
+                                                            int nb, int D, int L, int K, int Bs,
+                                                            int rows, float *__restrict__ lut) {
+  griddep_wait();
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // p*K + k (< 2^31, checked)
+  if (e >= rows) return;
+  const int p = e / K, m = p / L;
+  float c[DS];
+#pragma unroll
+  for (int j = 0; j < DS; ++j) c[j] = __ldg(C + (size_t)e * DS + j);
+  for (int t = 0; t < Bs; ++t) {
+    float acc = 0.f;
+    if (t < nb) {
+      const float *hm = h + (size_t)(b0 + t) * D + (size_t)m * DS;
+#pragma unroll
+      for (int j = 0; j < DS; ++j) acc = fmaf(__ldg(hm + j), c[j], acc);
+    }
+    lut[(size_t)e * Bs + t] = acc;
+  }
+}
+
 // ds = 6 (the Gemma-2 shape: D = 2304, M = 384): one thread per 4
 // consecutive codewords of a table = 96 contiguous bytes of C read as six
 // 16-byte loads with an L2 evict-last hint (the 18.9 MB codebook is reused
@@ -168,6 +194,18 @@ cudaError_t launch_lut_build(const float *h, const float *C, int B, int b0, int 
     if (4 * quads < 0x7fffffffLL - 1024)
       return pdl_launch(lut_build_ds6_kernel, dim3((unsigned)blocks), dim3(256), 0, s, h, C, b0,
                         nb, D, L, K, Bs, (int)quads, lut);
+  }
+  const int64_t rows = (int64_t)P * K;
+  if (Bs <= 2 && rows < 0x7fffffffLL - 256) {
+    const dim3 g((unsigned)((rows + 255) / 256));
+    switch (ds) {
+      case 1: return pdl_launch(lut_build_flat_kernel<1>, g, dim3(256), 0, s, h, C, b0, nb, D, L, K, Bs, (int)rows, lut);
+      case 2: return pdl_launch(lut_build_flat_kernel<2>, g, dim3(256), 0, s, h, C, b0, nb, D, L, K, Bs, (int)rows, lut);
+      case 3: return pdl_launch(lut_build_flat_kernel<3>, g, dim3(256), 0, s, h, C, b0, nb, D, L, K, Bs, (int)rows, lut);
+      case 4: return pdl_launch(lut_build_flat_kernel<4>, g, dim3(256), 0, s, h, C, b0, nb, D, L, K, Bs, (int)rows, lut);
+      case 8: return pdl_launch(lut_build_flat_kernel<8>, g, dim3(256), 0, s, h, C, b0, nb, D, L, K, Bs, (int)rows, lut);
+      default: break;
+    }
   }
   dim3 grid((unsigned)((K + 255) / 256), (unsigned)P);
   size_t smem = (size_t)Bs * ds * sizeof(float);

@@ -279,10 +279,11 @@ __device__ __forceinline__ int arg_key_index(unsigned long long k) {
   return k == 0ull ? 0 : (int)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
 }
 
-__device__ __forceinline__ ArgBest arg_shfl_xor(ArgBest a, int lane_mask) {
+__device__ __forceinline__ ArgBest arg_shfl_xor(ArgBest a, int lane_mask,
+                                                unsigned members = 0xffffffffu) {
   ArgBest o;
-  o.v = __shfl_xor_sync(0xffffffffu, a.v, lane_mask);
-  o.i = __shfl_xor_sync(0xffffffffu, a.i, lane_mask);
+  o.v = __shfl_xor_sync(members, a.v, lane_mask);
+  o.i = __shfl_xor_sync(members, a.i, lane_mask);
   return o;
 }
 
