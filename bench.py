@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--workload", default="g2_b1",
                     choices=["g2_b1", "g2_b32", "packed_b64", "mlp_gate_b1", "mlp_down_b1",
                              "encode_g2", "g2_b1_topk50"])
-    ap.add_argument("--codes", default="sched", choices=["u16", "sched"],
+    ap.add_argument("--codes", default="sched", choices=["u16", "sched", "u8"],
                     help="uint16 code layout of the unpacked workloads timed for `value`: "
                          "bank-scheduled once by rq_prepare_sched (the serving layout), or as "
                          "drawn; the other layout is reported under other_layouts")
@@ -61,9 +61,10 @@ def parse():
 
 
 def workload_config(w, codes="u16"):
-    rb = w.P * 10 // 8 if w.packed10 else w.P * 2
+    rb = code_bytes(w, codes) // w.V
     fmt = f"packed10 ({rb} B/row)" if w.packed10 else (
         f"uint16 ({rb} B/row)" if codes == "u16" else
+        f"uint8 ({rb} B/row, K <= 256)" if codes == "u8" else
         f"uint16 ({rb} B/row) in the bank-scheduled order of rq_prepare_sched")
     if w.argmax:
         what = (f"softcap {w.softcap:g}, logits + argmax, then the {w.B} picked tokens' input "
@@ -84,8 +85,10 @@ def workload_config(w, codes="u16"):
     }
 
 
-def code_bytes(w):
-    return w.V * (w.P * 10 // 8 if w.packed10 else w.P * 2)
+def code_bytes(w, codes="u16"):
+    if w.packed10:
+        return w.V * (w.P * 10 // 8)
+    return w.V * w.P * (1 if codes == "u8" else 2)
 
 
 # --------------------------------------------------------- multi-rank math
@@ -366,7 +369,9 @@ def run_ours(args, w):
         sched, (st, ps) = rq.rq_prepare_sched(c16, d, stats=True)
         layouts["sched"] = (rq.SCHED, sched, ps / st)
         layouts["u16"] = (rq.U16, c16, None)
-        headline = args.codes
+        if w.K <= 256:                 # one byte per code
+            layouts["u8"] = (rq.U8, rq.rq_pack8(c16, d), None)
+        headline = args.codes if args.codes in layouts else "sched"
 
     def make_step(fmt, codes, out=None):
         ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
@@ -478,7 +483,7 @@ def run_ours(args, w):
     # ---- the dominant kernel alone, live CUDA events
     kern_us = code_pass_us(step, min(args.steps, 2000))
     peak, peak_kind = load_peaks()
-    algo_bytes = code_bytes(w)
+    algo_bytes = code_bytes(w, headline)
     achieved = algo_bytes / (kern_us / 1e6) / 1e9
     kname = "logits_chunk_u16_kernel" if w.B <= 4 and not w.packed10 else "logits_l2_kernel"
     kkey = f"{kname}/{headline}/{w.name}"
@@ -495,7 +500,7 @@ def run_ours(args, w):
         k2 = code_pass_us(st2, min(n2, 1000))
         others[name] = {"us_per_call": t2 / n2 * 1e3, "value": throughput(w.V * w.B * n2, world, t2),
                         "code_pass_us": k2,
-                        "code_pass_frac": algo_bytes / (k2 / 1e6) / 1e9 / peak}
+                        "code_pass_frac": code_bytes(w, name) / (k2 / 1e6) / 1e9 / peak}
         del g2
     run, graph = graphed(step)
 

@@ -39,6 +39,10 @@
  *            RQ_CODES_PACKED10: uint8 [V][rb], rb = ceil(10*M*L/8); code
  *                               p occupies bits [10p, 10p+10) of the row,
  *                               bit i being bit (i%8) of byte i/8
+ *            RQ_CODES_U8:       uint8 [V][M*L], K <= 256: the byte form
+ *                               of small codebooks (the per-matrix K of
+ *                               the MLP-RQ page, 8 bits per code), half the
+ *                               bytes of RQ_CODES_U16; written by rq_pack8
  *            RQ_CODES_SCHED:    uint16 [M*L/32][V][32] (K <= 1024, M*L % 32
  *                               == 0), written by rq_prepare_sched: chunk-
  *                               major (columns 32c..32c+31 of every row form
@@ -86,7 +90,8 @@ typedef struct {
 enum rq_code_fmt {
     RQ_CODES_U16 = 0,       /* one uint16 per code (K <= 65536)           */
     RQ_CODES_PACKED10 = 1,  /* 10-bit codes, bit stream per row (K<=1024) */
-    RQ_CODES_SCHED = 2      /* bank-scheduled uint16 (rq_prepare_sched)   */
+    RQ_CODES_SCHED = 2,     /* bank-scheduled uint16 (rq_prepare_sched)   */
+    RQ_CODES_U8 = 3         /* one byte per code (K <= 256, rq_pack8)     */
 };
 
 enum rq_status {
@@ -282,6 +287,15 @@ RQ_API int rq_topk_sample(const float *logits, int64_t V, int B, int k, float te
  */
 RQ_API int rq_encode(const float *X, rq_dims d, const float *C, uint16_t *codes,
                      void *stream);
+
+/*
+ * rq_pack8 -- convert uint16 codes [V][M*L] into RQ_CODES_U8 (one byte per
+ * code; K <= 256).  Codes >= 256 keep their low 8 bits.  packed (device)
+ * uint8 [V][M*L].
+ * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_UNSUPPORTED (K > 256),
+ *         RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ */
+RQ_API int rq_pack8(const uint16_t *codes_u16, rq_dims d, uint8_t *packed, void *stream);
 
 /*
  * rq_prepare_sched -- convert uint16 codes [V][M*L] into RQ_CODES_SCHED

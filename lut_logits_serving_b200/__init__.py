@@ -21,7 +21,7 @@ import ctypes
 import os
 
 __all__ = [
-    "RqDims", "RqError", "U16", "PACKED10", "SCHED", "lib", "dims", "rq_prepare_sched",
+    "RqDims", "RqError", "U16", "PACKED10", "SCHED", "U8", "lib", "rq_pack8", "dims", "rq_prepare_sched",
     "rq_status_string", "rq_version", "rq_codes_bytes", "rq_lut_token_stride",
     "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
     "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
@@ -33,6 +33,7 @@ __all__ = [
 U16 = 0
 PACKED10 = 1
 SCHED = 2
+U8 = 3
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librqlut.so")
 
@@ -79,6 +80,7 @@ _SIGNATURES = {
     "rq_logits_from_hidden": (_i, [_p, _p, _p, _i, RqDims, _i, _f, _p, _p, _p, _sz, _p]),
     "rq_decode_rows": (_i, [_p, _i64, _p, _i, _p, RqDims, _f, _p, _p]),
     "rq_pack10": (_i, [_p, RqDims, _p, _p]),
+    "rq_pack8": (_i, [_p, RqDims, _p, _p]),
     "rq_encode": (_i, [_p, RqDims, _p, _p, _p]),
     "rq_topk_workspace_bytes": (_sz, [_i64, _i, _i]),
     "rq_last_cuda_error": (_i, [_i]),
@@ -178,7 +180,7 @@ def _check(fn, status):
 
 def _codes_dtype(fmt):
     torch = _torch()
-    return torch.uint8 if fmt == PACKED10 else torch.uint16
+    return torch.uint8 if fmt in (PACKED10, U8) else torch.uint16
 
 
 def _empty(shape, dtype, like):
@@ -318,6 +320,16 @@ def rq_topk_sample(logits, k: int, temperature: float = 1.0, seed: int = 0, step
         _ptr_or_null(topk_idx, torch.int32, "topk_idx"),
         _cuda(token, torch.int32, "token"), wsp, wsn, _stream(stream)))
     return topk_val, topk_idx, token
+
+
+def rq_pack8(codes_u16, d: RqDims, out=None, stream=None):
+    """uint16 [V, P] (or [V, M, L]) -> uint8 [V, P] (RQ_CODES_U8, K <= 256)."""
+    torch = _torch()
+    if out is None:
+        out = _empty((d.V, d.M * d.L), torch.uint8, codes_u16)
+    _check("rq_pack8", lib().rq_pack8(_cuda(codes_u16, torch.uint16, "codes_u16"), d,
+                                      _cuda(out, torch.uint8, "packed"), _stream(stream)))
+    return out
 
 
 def rq_device_error(clear: bool = True) -> int:

@@ -92,3 +92,23 @@ cudaError_t launch_pack10(const uint16_t *codes, int64_t V, int P, uint8_t *pack
 }
 
 }  // namespace rq
+
+namespace rq {
+
+// uint16 codes -> one byte each (grid-stride, 16 codes per thread step).
+__global__ void pack8_kernel(const uint16_t *__restrict__ codes, int64_t n,
+                             uint8_t *__restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = (uint8_t)codes[i];
+}
+
+cudaError_t launch_pack8(const uint16_t *codes, int64_t n, uint8_t *packed, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 65536) blocks = 65536;
+  pack8_kernel<<<(unsigned)blocks, 256, 0, s>>>(codes, n, packed);
+  return cudaGetLastError();
+}
+
+}  // namespace rq

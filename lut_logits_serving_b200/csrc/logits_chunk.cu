@@ -43,21 +43,25 @@ struct ChunkArgs {
   unsigned *err;
 };
 
-// Plain codes: TPR threads per row, 1024 threads.  Bank-scheduled codes
+// Plain uint16 codes: TPR threads per row, 1024 threads.  Bank-scheduled codes
 // (one token): one thread per row owns the row's whole 32-pair slice, the
-// unit the schedule was made for, 512 threads.
-template <int TB, bool SCHED = false>
+// unit the schedule was made for, 512 threads.  Byte codes: one thread per
+// row and 32-pair slice (32 bytes), 512 threads.
+template <int TB, int FMT>
 struct ChunkShape {
-  static constexpr int PC = SCHED ? 32 : (TB == 1 ? 32 : (TB == 2 ? 16 : 8));  // pairs/chunk
-  static constexpr int PPT = SCHED ? 32 : (TB == 4 ? 8 : 16);                  // pairs/thread
+  static constexpr bool WHOLE = FMT == RQ_CODES_SCHED || FMT == RQ_CODES_U8;
+  static constexpr int PC = WHOLE ? 32 : (TB == 1 ? 32 : (TB == 2 ? 16 : 8));  // pairs/chunk
+  static constexpr int PPT = WHOLE ? 32 : (TB == 4 ? 8 : 16);                  // pairs/thread
   static constexpr int TPR = PC / PPT;                          // threads per row
-  static constexpr int THREADS = SCHED ? 512 : 1024;
+  static constexpr int THREADS = WHOLE ? 512 : 1024;
   static constexpr int WARPS = THREADS / 32;
   static constexpr int R = THREADS / TPR;                       // rows per tile
-  static constexpr int ROWB = PC * 2;                           // code bytes per row slice
+  static constexpr int CB = FMT == RQ_CODES_U8 ? 1 : 2;         // bytes per code
+  static constexpr int ROWB = PC * CB;                          // code bytes per row slice
   static constexpr int BOXES = R / 256;
   static constexpr int BOX_BYTES = 256 * ROWB;
   static constexpr int STAGE_BYTES = R * ROWB;
+  static constexpr int CPV = 16 / CB;                           // codes per 16-byte vector
 };
 
 // 16-byte chunk j of row r (row index inside a 1024-byte-aligned TMA box) as
@@ -150,6 +154,22 @@ __device__ __forceinline__ void lookup8(uint32_t tbase, int K, uint4 w, const Co
   }
 }
 
+// RQ_CODES_U8: 16 consecutive pairs (one 16-byte vector of byte codes) of
+// one row; `tbase` is the shared byte address of the first of those tables.
+template <int TB, int KT>
+__device__ __forceinline__ void lookup16_u8(uint32_t tbase, int K, uint4 w, const CodeFix &f,
+                                            float (&acc)[TB]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  const uint32_t pb = (uint32_t)(KT > 0 ? KT : K) * TB * 4;   // bytes per table
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t c = fix_code<KT>((ws[q] >> (8 * b)) & 0xFFu, f);
+      add_entry_rt<TB>(tbase + (uint32_t)(4 * q + b) * pb + c * (TB * 4), acc);
+    }
+}
+
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float x;
   asm("ld.shared.f32 %0, [%1];" : "=f"(x) : "r"(addr));
@@ -198,10 +218,11 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // KSH: the table stride 2^KSH of RQ_CODES_SCHED entries (unused otherwise);
 // MINB: CTAs per SM the register budget is made for.
 template <int TB, int KT, int NST, int FMT, int KSH, int MINB>
-__global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS, MINB)
+__global__ void __launch_bounds__(ChunkShape<TB, FMT>::THREADS, MINB)
     logits_chunk_u16_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
   constexpr bool SCHED = FMT == RQ_CODES_SCHED;
-  using S = ChunkShape<TB, SCHED>;
+  constexpr bool U8 = FMT == RQ_CODES_U8;
+  using S = ChunkShape<TB, FMT>;
   static_assert(!SCHED || (TB == 1 && S::PPT == 32), "a thread owns a whole scheduled slice");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment (TMA swizzle atoms) by pointer arithmetic, so the
@@ -301,14 +322,14 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS
   const int hh = tid % S::TPR;               // which PPT pairs of the row
   const int box = r >> 8, rr = r & 255;
   const uint32_t tt = smem_addr(Ts) + (uint32_t)hh * S::PPT * KS * TB * 4;
-  constexpr int NQ = S::PPT / 8;             // 16-byte code vectors per thread
+  constexpr int NQ = S::PPT / S::CPV;        // 16-byte code vectors per thread
   uint32_t voff[NQ];                         // this thread's code vectors in a stage
 #pragma unroll
   for (int q = 0; q < NQ; ++q)
     voff[q] = (uint32_t)(box * S::BOX_BYTES + rr * S::ROWB) + 16 * swz<S::ROWB>(hh * NQ + q, rr);
   int nq = 0;                                // vectors holding real pairs
 #pragma unroll
-  for (int q = 0; q < NQ; ++q) nq += ((hh * NQ + q) * 8 < np) ? 1 : 0;
+  for (int q = 0; q < NQ; ++q) nq += ((hh * NQ + q) * S::CPV < np) ? 1 : 0;
   float *out = a.partial + (size_t)c * a.B * a.V;
   int64_t v = t0 * S::R + r;
 
@@ -343,6 +364,10 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS
     for (int b = 0; b < TB; ++b) acc[b] = 0.f;
     if constexpr (SCHED) {
       acc[0] = chunk32_sched_tb1<KSH>(tt, w);   // the row's whole 32-pair slice
+    } else if constexpr (U8) {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+        if (q < nq) lookup16_u8<TB, KT>(tt + (uint32_t)q * 16 * K * TB * 4, K, w[q], a.fix, acc);
     } else {
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
@@ -612,16 +637,14 @@ struct Variant {
 
 #define RQ_CHUNK_VARIANT(TB, KT, NST, FMT, KSH, MINB)                                      \
   Variant {                                                                                \
-    TB, KT, NST, FMT, KSH, ChunkShape<TB, FMT == RQ_CODES_SCHED>::PC,                      \
-        ChunkShape<TB, FMT == RQ_CODES_SCHED>::R,                                          \
-        ChunkShape<TB, FMT == RQ_CODES_SCHED>::THREADS,                                    \
-        ChunkShape<TB, FMT == RQ_CODES_SCHED>::STAGE_BYTES,                                \
+    TB, KT, NST, FMT, KSH, ChunkShape<TB, FMT>::PC, ChunkShape<TB, FMT>::R,                \
+        ChunkShape<TB, FMT>::THREADS, ChunkShape<TB, FMT>::STAGE_BYTES,                    \
         reinterpret_cast<const void *>(&logits_chunk_u16_kernel<TB, KT, NST, FMT, KSH, MINB>) \
   }
 
-// Plain codes: 128 KB table chunk + NST stages (3 x 32 KB or 5 x 16 KB) per
-// CTA, one CTA per SM; K = 1024 has its own instances (table offsets as
-// immediates).  Scheduled codes: one instance per table stride 2^KSH; up to
+// Plain uint16 codes: 128 KB table chunk + NST stages (3 x 32 KB or 5 x 16
+// KB) per CTA, one CTA per SM; K = 1024 has its own instances (table offsets
+// as immediates).  Scheduled codes: one instance per table stride 2^KSH; up to
 // 256 entries a chunk's tables (<= 32 KB) and two 32 KB stages leave room
 // for two CTAs per SM.
 const Variant kVariants[] = {
@@ -637,6 +660,11 @@ const Variant kVariants[] = {
     RQ_CHUNK_VARIANT(1, 0, 2, RQ_CODES_SCHED, 7, 2),
     RQ_CHUNK_VARIANT(1, 0, 2, RQ_CODES_SCHED, 6, 2),
     RQ_CHUNK_VARIANT(1, 0, 2, RQ_CODES_SCHED, 5, 2),
+    // byte codes (K <= 256): tables of at most 32 KB per token, 16 KB stages
+    RQ_CHUNK_VARIANT(1, 256, 3, RQ_CODES_U8, 0, 2),
+    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_U8, 0, 2),
+    RQ_CHUNK_VARIANT(2, 0, 3, RQ_CODES_U8, 0, 1),
+    RQ_CHUNK_VARIANT(4, 0, 3, RQ_CODES_U8, 0, 1),
 };
 
 size_t variant_smem(const Variant &v, int K) {
@@ -650,9 +678,10 @@ size_t variant_smem(const Variant &v, int K) {
 ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di) {
   ChunkPlan cp{};
   cp.ok = false;
-  if ((fmt != RQ_CODES_U16 && fmt != RQ_CODES_SCHED) || B < 1 || B > 4 || P % 8 != 0 ||
-      K > 1024)
+  if ((fmt != RQ_CODES_U16 && fmt != RQ_CODES_SCHED && fmt != RQ_CODES_U8) || B < 1 || B > 4 ||
+      P % 8 != 0 || K > 1024)
     return cp;
+  if (fmt == RQ_CODES_U8 && (K > 256 || P % 16 != 0)) return cp;   // 16-byte row pitch
   if (fmt == RQ_CODES_SCHED && P % 32 != 0) return cp;
   if (V > (int64_t)INT_MAX - 2048) return cp;
   const int TB = rq_lut_token_stride(B);
@@ -686,17 +715,20 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   const Variant &var = kVariants[cp.variant];
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
-  const int rowb = cp.PC * 2;
+  const int cb = fmt == RQ_CODES_U8 ? 1 : 2;   // bytes per code
+  const int rowb = cp.PC * cb;
   // [V][P] for plain codes; the scheduled layout is chunk-major [P/32][V][32]
   const bool cm = fmt == RQ_CODES_SCHED;
   const cuuint64_t gdim[2] = {(cuuint64_t)(cm ? 32 : P), (cuuint64_t)(cm ? (int64_t)V * (P / 32) : V)};
-  const cuuint64_t gstride[1] = {(cuuint64_t)(cm ? 64 : P * 2)};
+  const cuuint64_t gstride[1] = {(cuuint64_t)(cm ? 64 : P * cb)};
   const cuuint32_t box[2] = {(cuuint32_t)cp.PC, 256u};
   const cuuint32_t estride[2] = {1u, 1u};
   const CUtensorMapSwizzle swz = rowb == 64   ? CU_TENSOR_MAP_SWIZZLE_64B
                                  : rowb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
                                               : CU_TENSOR_MAP_SWIZZLE_NONE;
-  CUresult r = encode_fn()(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(codes),
+  CUresult r = encode_fn()(&tmap,
+                           cb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                           2, const_cast<void *>(codes),
                            gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;

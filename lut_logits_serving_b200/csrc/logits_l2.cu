@@ -111,6 +111,31 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
           add_vec<VW>(tg + ((size_t)(2 * k + 1) * K + c1) * Bs, acc);
         }
       }
+    } else if (FMT == RQ_CODES_U8) {
+      // 16 byte codes per 16-byte vector; rows are 16-byte aligned (P % 16 == 0)
+      const uint4 *crow = reinterpret_cast<const uint4 *>(
+          static_cast<const uint8_t *>(a.codes) + v * a.P);
+      const int n16 = a.P / 16;
+      for (int g = 0; g < n16; g += 4) {
+        uint32_t wd[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 w = g + k < n16 ? __ldg(crow + g + k) : make_uint4(0, 0, 0, 0);
+          wd[4 * k + 0] = w.x;
+          wd[4 * k + 1] = w.y;
+          wd[4 * k + 2] = w.z;
+          wd[4 * k + 3] = w.w;
+        }
+        const float *tg = tl + (size_t)(16 * g) * K * Bs;
+        const int nj = (n16 - g < 4 ? n16 - g : 4) * 16;   // codes of this step
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          if (j < nj) {
+            const uint32_t c = a.fix((wd[j >> 2] >> (8 * (j & 3))) & 0xFFu);
+            add_vec<VW>(tg + ((size_t)j * K + c) * Bs, acc);
+          }
+        }
+      }
     } else if (FMT == RQ_CODES_SCHED) {
       // chunk-major [P/32][V][32]; 32 entries (i << ssh | c) per chunk
       // slice, in any order
@@ -218,7 +243,10 @@ __global__ void __launch_bounds__(256) logits_generic_kernel(const L2Args a, int
         if (c < (uint32_t)a.K) z += __ldg(tl + ((size_t)pp * a.K + c) * a.Bs);
         continue;
       }
-      const uint32_t c = a.fix(fmt == RQ_CODES_U16 ? (uint32_t)c16[p] : packed10_code(c8, p));
+      const uint32_t c = a.fix(fmt == RQ_CODES_U16  ? (uint32_t)c16[p]
+                               : fmt == RQ_CODES_U8 ? (uint32_t)static_cast<const uint8_t *>(
+                                                          a.codes)[v * a.P + p]
+                                                    : packed10_code(c8, p));
       z += __ldg(tl + ((size_t)p * a.K + c) * a.Bs);
     }
     const float y = softcap_f(z, a.cap);
@@ -279,6 +307,7 @@ cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K
   const bool codes16 = (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
   const bool fast_fmt = fmt == RQ_CODES_U16     ? (P % 8 == 0)
                         : fmt == RQ_CODES_SCHED ? (P % 32 == 0)
+                        : fmt == RQ_CODES_U8    ? (P % 16 == 0)
                                                 : (P % 64 == 0);
   int VW;
   if (Bs == 1) VW = 1;
@@ -304,6 +333,11 @@ cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K
     if (VW == 1) return launch_fast<1, 1, RQ_CODES_SCHED>(a, nblk, s);
     if (VW == 2) return launch_fast<2, 1, RQ_CODES_SCHED>(a, nblk, s);
     return launch_vw<4, RQ_CODES_SCHED>(a, G, nblk, s);
+  }
+  if (fmt == RQ_CODES_U8) {
+    if (VW == 1) return launch_fast<1, 1, RQ_CODES_U8>(a, nblk, s);
+    if (VW == 2) return launch_fast<2, 1, RQ_CODES_U8>(a, nblk, s);
+    return launch_vw<4, RQ_CODES_U8>(a, G, nblk, s);
   }
   if (VW == 1) return launch_fast<1, 1, RQ_CODES_PACKED10>(a, nblk, s);
   if (VW == 2) return launch_fast<2, 1, RQ_CODES_PACKED10>(a, nblk, s);

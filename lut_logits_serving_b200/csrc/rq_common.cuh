@@ -116,6 +116,7 @@ __device__ __forceinline__ void decode_subspace(const DecodeSpec &a, int64_t id,
     uint32_t c;
     if (a.fmt == RQ_CODES_U16) c = crow16[p];
     else if (a.fmt == RQ_CODES_SCHED) c = sched_code(all16, a.V, id, p, sched_shift(a.K));
+    else if (a.fmt == RQ_CODES_U8) c = static_cast<const uint8_t *>(a.codes)[id * P + p];
     else c = packed10_code(crow10, p);
     return a.fix(c);
   };
@@ -349,6 +350,7 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
 
 cudaError_t launch_pack10(const uint16_t *codes, int64_t V, int P, uint8_t *packed,
                           cudaStream_t s);
+cudaError_t launch_pack8(const uint16_t *codes, int64_t n, uint8_t *packed, cudaStream_t s);
 
 size_t topk_workspace_bytes(int64_t V, int B, int k);
 cudaError_t launch_topk_sample(const float *logits, int64_t V, int B, int k, double temperature,

@@ -80,13 +80,15 @@ bool dims_ok(const rq_dims &d) {
 }
 
 bool fmt_known(int fmt) {
-  return fmt == RQ_CODES_U16 || fmt == RQ_CODES_PACKED10 || fmt == RQ_CODES_SCHED;
+  return fmt == RQ_CODES_U16 || fmt == RQ_CODES_PACKED10 || fmt == RQ_CODES_SCHED ||
+         fmt == RQ_CODES_U8;
 }
 
 bool fmt_ok(const rq_dims &d, int fmt) {
   if (fmt == RQ_CODES_U16) return true;
   if (fmt == RQ_CODES_PACKED10) return d.K <= 1024;
   if (fmt == RQ_CODES_SCHED) return d.K <= 1024 && ((int64_t)d.M * d.L) % 32 == 0;
+  if (fmt == RQ_CODES_U8) return d.K <= 256;
   return false;
 }
 
@@ -270,6 +272,7 @@ size_t rq_codes_bytes(rq_dims d, int fmt) {
   if (!dims_ok(d) || !fmt_ok(d, fmt)) return 0;
   const int64_t P = (int64_t)d.M * d.L;
   if (fmt == RQ_CODES_U16 || fmt == RQ_CODES_SCHED) return (size_t)(d.V * P * 2);
+  if (fmt == RQ_CODES_U8) return (size_t)(d.V * P);
   return (size_t)(d.V * ((10 * P + 7) / 8));
 }
 
@@ -371,7 +374,8 @@ int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt, co
   if (!ids || !codes || !C || !out) return RQ_ERR_INVALID_ARGUMENT;
   if (!fmt_known(fmt)) return RQ_ERR_INVALID_ARGUMENT;
   if (!fmt_ok(d, fmt)) return RQ_ERR_UNSUPPORTED;
-  if (!aligned(ids, 4) || !aligned(codes, fmt == RQ_CODES_SCHED ? 16 : 2) || !aligned(C, 4) ||
+  if (!aligned(ids, 4) ||
+      !aligned(codes, fmt == RQ_CODES_SCHED ? 16 : (fmt == RQ_CODES_U8 ? 1 : 2)) || !aligned(C, 4) ||
       !aligned(out, 2))
     return RQ_ERR_MISALIGNED;
   DevInfo di;
@@ -385,6 +389,14 @@ int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed, void *strea
   if (!aligned(codes_u16, 2)) return RQ_ERR_MISALIGNED;
   return status_of(
       launch_pack10(codes_u16, d.V, d.M * d.L, packed, static_cast<cudaStream_t>(stream)));
+}
+
+int rq_pack8(const uint16_t *codes_u16, rq_dims d, uint8_t *packed, void *stream) {
+  if (!codes_u16 || !packed || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_ok(d, RQ_CODES_U8)) return RQ_ERR_UNSUPPORTED;
+  if (!aligned(codes_u16, 2)) return RQ_ERR_MISALIGNED;
+  return status_of(launch_pack8(codes_u16, d.V * d.M * d.L, packed,
+                                static_cast<cudaStream_t>(stream)));
 }
 
 int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out, uint64_t *stats,

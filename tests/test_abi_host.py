@@ -59,6 +59,8 @@ def test_code_and_lut_sizes():
     assert rq.rq_codes_bytes(G2, rq.PACKED10) == 256000 * 960
     assert rq.rq_codes_bytes(G2, rq.SCHED) == 256000 * 768 * 2
     assert rq.rq_codes_bytes(TINY, rq.PACKED10) == 4096 * 80
+    assert rq.rq_codes_bytes(TINY, rq.U8) == 4096 * 64                        # K = 256: bytes
+    assert rq.rq_codes_bytes(G2, rq.U8) == 0                                 # K = 1024: none
     assert rq.rq_codes_bytes(rq.dims(10, 3, 1, 1, 1024), rq.PACKED10) == 10 * 2   # ceil(10/8)
     assert rq.rq_codes_bytes(rq.dims(10, 3, 1, 1, 2048), rq.PACKED10) == 0       # K > 1024
     for B, Bs in ((1, 1), (2, 2), (3, 4), (4, 4), (5, 8), (32, 32), (33, 36), (64, 64)):
@@ -120,6 +122,7 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_decode_rows(null, 0, null, 0, null, G2, 48.0, null, s) == 0   # N = 0: no-op
     assert lib.rq_decode_rows(_fake(0x10002), 5, a, 0, a, G2, 48.0, a, s) == MIS
     assert lib.rq_pack10(null, G2, a, s) == INV
+    assert lib.rq_pack8(a, G2, a, s) == UNS                                   # K > 256
     assert lib.rq_prepare_sched(null, G2, a, null, s) == INV
     assert lib.rq_prepare_sched(a, rq.dims(10, 48, 24, 1, 64), _fake(0x900000), null, s) == UNS
     assert lib.rq_prepare_sched(a, G2, _fake(0x10000 + 64), null, s) == INV    # overlap

@@ -129,7 +129,7 @@ def test_decode512_bit_exact(g2, fmt):
 # ------------------------------------------------- RQ MLP matvec (no softcap)
 
 @pytest.mark.parametrize("name", ["mlp_gate_b1", "mlp_down_b1"])
-@pytest.mark.parametrize("fmt", [0, 2], ids=["u16", "sched"])
+@pytest.mark.parametrize("fmt", [0, 2, 3], ids=["u16", "sched", "u8"])
 def test_rq_mlp_matvec(name, fmt):
     """y = W x for an RQ-coded MLP weight W [out x in] (ds = 2, about 10 bits/param with the codebooks):
     the same lookup + sum with V = out features and the softcap off."""
@@ -138,7 +138,8 @@ def test_rq_mlp_matvec(name, fmt):
     data = synth.make(w)
     C, codes, h = data["C"], data["codes"], data["h"]
     c16 = dev(codes.reshape(w.V, -1))
-    dc = c16 if fmt == rq.U16 else rq.rq_prepare_sched(c16, d)
+    dc = {rq.U16: lambda: c16, rq.SCHED: lambda: rq.rq_prepare_sched(c16, d),
+          rq.U8: lambda: rq.rq_pack8(c16, d)}[fmt]()
     y, _, _ = rq.rq_logits_from_hidden(dev(h), dev(C), dc, fmt, d, 0.0)
     ref = oracle.logits_direct(codes, C, h)        # the plain definition: W x
     err = assert_logits_close(y.cpu().numpy(), ref)

@@ -38,6 +38,8 @@ def gpu_codes(codes, fmt, d):
         return c16
     if fmt == rq.SCHED:
         return rq.rq_prepare_sched(c16, d)
+    if fmt == rq.U8:
+        return rq.rq_pack8(c16, d)
     return rq.rq_pack10(c16, d)
 
 
@@ -46,6 +48,8 @@ def fmt_applies(fmt, M, L, K):
         return K <= 1024
     if fmt == rq.SCHED:
         return K <= 1024 and (M * L) % 32 == 0
+    if fmt == rq.U8:
+        return K <= 256
     return True
 
 
@@ -87,7 +91,7 @@ CASES = [
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "V%d_D%d_M%d_L%d_K%d" % c)
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 13, 32, 33])
-@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["u16", "packed10", "sched"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3], ids=["u16", "packed10", "sched", "u8"])
 def test_logits_and_argmax(case, B, fmt):
     V, D, M, L, K = case
     if not fmt_applies(fmt, M, L, K):
@@ -195,7 +199,7 @@ def test_out_of_range_codes_stay_in_bounds():
 
 # ------------------------------------------------------------ row decode
 
-@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["u16", "packed10", "sched"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3], ids=["u16", "packed10", "sched", "u8"])
 @pytest.mark.parametrize("shape", [(4096, 192, 32, 2, 256), (5000, 288, 48, 2, 1024),
                                    (300, 96, 16, 3, 100), (50, 9, 3, 1, 7)])
 def test_decode_rows_bit_exact(shape, fmt):
@@ -316,7 +320,7 @@ def test_prepare_sched_rejects_unsupported_shapes():
 # ------------------------------------------------------------ greedy step
 
 @pytest.mark.parametrize("B", [1, 3, 5, 33])
-@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["u16", "packed10", "sched"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3], ids=["u16", "packed10", "sched", "u8"])
 def test_greedy_step_rows_are_the_picked_tokens_rows(B, fmt):
     V, D, M, L, K = 3000, 192, 32, 2, 256
     C, codes, h = make_case(V, D, M, L, K, B, seed=B)
@@ -391,3 +395,19 @@ def test_l2_pass_with_an_exactly_sized_table(B):
     ref = oracle_logits(C, codes, h, 30.0)
     assert_logits_close(logits.cpu().numpy(), ref)
     check_argmax(am.cpu().numpy(), ref)
+
+
+def test_pack8_round_trip_and_decode():
+    """RQ_CODES_U8 holds each code in one byte; rows rebuilt from it are the
+    oracle's, bit for bit."""
+    V, D, M, L, K = 3000, 96, 16, 2, 200
+    C, codes, _ = make_case(V, D, M, L, K, 1, seed=9)
+    d = rq.dims(V, D, M, L, K)
+    u8 = rq.rq_pack8(dev(codes.reshape(V, -1)), d)
+    assert np.array_equal(u8.cpu().numpy(), codes.reshape(V, -1).astype(np.uint8))
+    ids = synth.zipf_ids(300, V, 1.1, 4)
+    out = rq.rq_decode_rows(dev(ids), u8, rq.U8, dev(C), d, 5.0)
+    want = oracle.decode_rows_bf16(ids, codes, C, 5.0)
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    with pytest.raises(rq.RqError):             # K > 256 has no byte form
+        rq.rq_pack8(dev(codes.reshape(V, -1)), rq.dims(V, D, M, L, 300))
