@@ -596,7 +596,12 @@ def run_ours(args, w):
     if w.B <= 4 and not w.packed10:
         launches_per_step = 3 + (1 if w.argmax else 0)
     else:
-        launches_per_step = 2 * ((w.B + 31) // 32) + (1 if w.argmax else 0)
+        # per 32-token group: rows decoded + multiplied (one kernel: full groups
+        # of uint16 codes at ds = 6, L = 2) or table build + L2 pass (two)
+        decoded = (headline == "u16" and w.ds == 6 and w.L == 2 and w.K <= 1024 and w.M % 8 == 0)
+        groups = [min(32, w.B - b0) for b0 in range(0, w.B, 32)]
+        launches_per_step = sum(1 if decoded and g == 32 else 2 for g in groups)
+        launches_per_step += 1 if w.argmax else 0
     topk_us = None
     if w.topk:
         launches_per_step += topk_launches(w.V, w.topk) + 1     # top-k + draw, row decode
