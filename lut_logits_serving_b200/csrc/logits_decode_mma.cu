@@ -1,0 +1,539 @@
+// logits_decode_mma.cu -- logits of a token group by decoding vocabulary rows
+// straight into tensor memory and multiplying them with the hidden states on
+// the tcgen05 tensor cores.
+//
+// "Gemma-2 runtime compression: NF4 + LUT serving", LUT section: the lookup
+// + sum equals the decode-then-matmul the pages check it against,
+//   z[b][v] = sum_m sum_j h[b][m*ds + j] * (C[m][0][c0][j] + C[m][1][c1][j]);
+// Gemma-2's softcap follows.  For a batch this is a dense contraction of the
+// decoded rows with the hidden states, which is what the tensor cores do.
+//
+// fp32 accuracy from tf32 operands: every operand x is split into x_hi = x
+// rounded to nearest (even) at the tf32 boundary (low 13 mantissa bits zero,
+// so a tf32 MMA reads it exactly) and x_lo = x - x_hi (exact in fp32, at most
+// half a tf32 ulp of x), and
+//   E . h = E_hi h_hi + E_hi h_lo + E_lo h_hi + (E_lo h_lo, dropped),
+// three MMAs whose error is about 2^-22 of |E||h| per product.  The tensor
+// core's fp32 accumulation does not round to nearest and its error grows with
+// the length of an accumulation chain, so a chain covers 16 subspaces; each
+// finished chain is added into fp32 registers (round to nearest) by the
+// threads that own its rows.  Measured against fp64 this keeps the logits
+// near 1e-6 of their scale; one chain over all 384 subspaces was ~3e-5.
+//
+// Design for sm_100a (ds = 6, L = 2, uint16 codes, K <= 1024, 32 tokens).
+// One CTA per SM walks an even share of the vocabulary in passes of up to
+// 1024 rows = 8 M = 128 tiles; per pass it runs every subspace once, so each
+// codebook is fetched once per 1024 rows.  Warp-specialised, mbarrier-driven:
+//   * 16 decoder warps (4 warpgroups).  Thread (warpgroup g, warp q, lane)
+//     owns row 32 q + lane of tiles g and g + 4.  Per subspace it gathers the
+//     row's two codewords from the shared-memory codebook, adds them, splits
+//     the sum into hi and lo and stores both (6 dims + 2 zero pads each) into
+//     its own TMEM lane with one tcgen05.st -- the MMA's A operand lives in
+//     tensor memory, so decoded rows never touch shared memory.  Its fp32
+//     sums are in registers for tile g and in shared memory (thread-private
+//     columns) for tile g + 4: 17 warps leave 96 registers a thread;
+//   * one control warp: one lane issues the TMA code tiles ({8 codes, 256
+//     rows}, 3 stages of 4 subspaces), one bulk copy per subspace of the
+//     codebook pair (48 KB at K = 1024, double-buffered) plus the pre-split
+//     hidden operand (2 KB, 4-slot ring), and the 3 x 8 MMAs (M = 128,
+//     N = 32, K = 8; A from TMEM, B from shared memory) per subspace;
+//   * TMEM: accumulators 8 tiles x 32 columns, and two A slots per tile of
+//     16 columns (hi, lo), 512 columns in all.  Decoding subspace s + 1 fills
+//     the other A slot while the MMAs of s run.
+// Every wait is bounded; a timed-out wait raises a CTA-wide abort flag, the
+// control lane waits (bounded) for its copies and MMAs in flight, and the CTA
+// frees its TMEM and ends.
+#include <cfloat>
+#include <climits>
+
+#include "rq_common.cuh"
+
+namespace rq {
+
+namespace {
+
+constexpr int kDmTokens = 32;
+constexpr int kDmDecWarps = 16;
+constexpr int kDmThreads = (kDmDecWarps + 1) * 32;   // + the control warp
+constexpr int kDmTiles = 8;                          // M = 128 tiles per pass
+constexpr int kDmRows = kDmTiles * 128;              // rows per pass
+constexpr int kDmGroup = 4;                          // subspaces per code stage (16 B per row)
+constexpr int kDmStageBytes = kDmRows * kDmGroup * 4;   // 16 KB
+constexpr int kDmStages = 3;
+constexpr int kDmChain = 16;                         // subspaces per accumulation chain
+constexpr int kDmHFloats = 512;                      // one subspace's hidden operand: hi, lo
+constexpr int kDmHSlots = 4;
+constexpr uint32_t kDmTmemCols = 512;
+constexpr uint32_t kDmAcol = 256;                    // first A-slot column
+
+// mbarriers
+constexpr int kBarCodes = 0;                         // 3: code stages (TMA)
+constexpr int kBarBook = 3;                          // 2: codebook + hidden operand (bulk)
+constexpr int kBarFull = 5;                          // 2: A slot written (16 decoder warps)
+constexpr int kBarMma = 7;                           // 2: MMAs of a subspace done (commit)
+constexpr int kBarChain = 9;                         // 1: MMAs of a chain done (commit)
+constexpr int kBarFlush = 10;                        // 1: chain read into registers (16 warps)
+constexpr int kBars = 11;
+
+struct DmArgs {
+  const float *C;      // [M][2][K][6]
+  const float *hop;    // [M][512]: hi then lo hidden operand per subspace
+  int64_t V;
+  int M, K;
+  int t0, nb;          // tokens t0 .. t0 + nb - 1
+  float cap;
+  float *logits;       // [Btot][V] or null
+  float *am_val;       // [Btot][nblk] or null (columns past the grid get -inf)
+  int *am_idx;
+  int nblk;
+  CodeFix fix;
+  unsigned *err;
+};
+
+// Canonical K-major, no-swizzle operand of 32-bit elements: 8-row groups of
+// two 128-byte core matrices (K halves 0..3, 4..7); float offset of (row, k).
+__host__ __device__ __forceinline__ int opnd_idx(int row, int k) {
+  return (row >> 3) * 64 + (k >> 2) * 32 + (row & 7) * 4 + (k & 3);
+}
+
+// Shared-memory matrix descriptor (sm_100): start, leading-dimension byte
+// offset (between the K halves: 128 B), stride byte offset (between 8-row
+// groups: 256 B), all in 16-byte units; version 1; no swizzle.
+__device__ __forceinline__ unsigned long long opnd_desc(uint32_t saddr) {
+  return (unsigned long long)((saddr >> 4) & 0x3FFFu) | ((unsigned long long)(128 >> 4) << 16) |
+         ((unsigned long long)(256 >> 4) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor: D fp32, A and B tf32, both K-major, M = 128, N = 32.
+__device__ __forceinline__ uint32_t mma_idesc() {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(kDmTokens >> 3) << 17) |
+         ((uint32_t)(128 >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] . B[smem]^T
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d, uint32_t a, unsigned long long b,
+                                            uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(accum), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// one TMEM row segment: hi[0..5], 0, 0, lo[0..5], 0, 0
+__device__ __forceinline__ void tmem_st_hilo(uint32_t taddr, const float (&hi)[6],
+                                             const float (&lo)[6]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %7, %8, %9, %10, "
+      "%11, %12, %13, %7, %7};" ::"r"(taddr),
+      "r"(__float_as_uint(hi[0])), "r"(__float_as_uint(hi[1])), "r"(__float_as_uint(hi[2])),
+      "r"(__float_as_uint(hi[3])), "r"(__float_as_uint(hi[4])), "r"(__float_as_uint(hi[5])),
+      "r"(0u), "r"(__float_as_uint(lo[0])), "r"(__float_as_uint(lo[1])),
+      "r"(__float_as_uint(lo[2])), "r"(__float_as_uint(lo[3])), "r"(__float_as_uint(lo[4])),
+      "r"(__float_as_uint(lo[5])));
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// x rounded to nearest (ties to even) with the low 13 mantissa bits cleared
+// (finite inputs of logit magnitude; no overflow handling is needed here)
+__device__ __forceinline__ float tf32_hi(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return __uint_as_float((u + 0xFFFu + ((u >> 13) & 1u)) & 0xFFFFE000u);
+}
+
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+}  // namespace
+
+// Hidden operand of one token group, per subspace m: h_hi then h_lo, each
+// [32 tokens][K = 8] in the canonical K-major layout (dims 6, 7 and tokens
+// past the group are zero).
+__global__ void __launch_bounds__(256) split_hidden_kernel(const float *__restrict__ h, int D,
+                                                           int t0, int nb,
+                                                           float *__restrict__ hop) {
+  griddep_wait();
+  const int m = blockIdx.x, tok = threadIdx.x >> 3, k = threadIdx.x & 7;
+  const float x = (k < 6 && tok < nb) ? h[(int64_t)(t0 + tok) * D + m * 6 + k] : 0.f;
+  const float xh = tf32_hi(x);
+  float *o = hop + (size_t)m * kDmHFloats;
+  o[opnd_idx(tok, k)] = xh;
+  o[256 + opnd_idx(tok, k)] = __fsub_rn(x, xh);
+  griddep_launch_dependents();
+}
+
+__global__ void __launch_bounds__(kDmThreads, 1)
+    logits_decode_mma_kernel(const __grid_constant__ CUtensorMap tmap, const DmArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const int cbf = 2 * a.K * 6;                                     // floats per codebook pair
+  const uint32_t cbb = (uint32_t)cbf * 4u;
+  const size_t cbs = (size_t)align_up(cbf, 256);                   // floats per book buffer
+  unsigned char *st = smem;                                        // code stages
+  float *cb = reinterpret_cast<float *>(st + kDmStages * kDmStageBytes);
+  float *hs = cb + 2 * cbs;                                        // hidden operand slots
+  float *sacc = hs + kDmHSlots * kDmHFloats;                       // [32 tokens][512 threads]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sacc + kDmTokens * kDmDecWarps * 32);
+  ArgBest *wbest = reinterpret_cast<ArgBest *>(bar + kBars);      // [16 warps][32]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(wbest + kDmDecWarps * kDmTokens);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    prefetch_tmap(&tmap);
+    for (int i = 0; i < kBars; ++i)
+      mbar_init(smem_addr(&bar[i]), (i == kBarFull || i == kBarFull + 1 || i == kBarFlush)
+                                        ? (uint32_t)kDmDecWarps
+                                        : 1u);
+    fence_mbar_init();
+    *abort_flag = 0;
+  }
+  if (warp == kDmDecWarps) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kDmTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+
+  const int M = a.M, G = a.M / kDmGroup, NC = (a.M + kDmChain - 1) / kDmChain;
+  const int64_t r0 = a.V * blockIdx.x / gridDim.x, r1 = a.V * (blockIdx.x + 1) / gridDim.x;
+  const int npass = (int)((r1 - r0 + kDmRows - 1) / kDmRows);
+  const int S = npass * M;                   // steps: (pass, subspace)
+  const int NG = npass * G;                  // code groups
+  auto pass_row0 = [&](int p) { return r0 + (r1 - r0) * p / npass; };
+  auto bar_at = [&](int i) { return smem_addr(&bar[i]); };
+
+  if (warp == kDmDecWarps) {
+    // ------------------------------------------------------------ control
+    if (lane == 0 && S > 0) {
+      const uint64_t pol_codes = l2_policy_evict_first();
+      const uint32_t idesc = mma_idesc();
+      int last_codes[kDmStages] = {-1, -1, -1}, last_book[2] = {-1, -1}, last_mma[2] = {-1, -1};
+      bool to = false;
+      auto wait = [&](int i, uint32_t parity) {
+        if (!to && !mbar_try_wait(bar_at(i), parity) && !mbar_wait_bounded(bar_at(i), parity)) {
+          to = true;
+          *abort_flag = 1;
+        }
+      };
+      auto issue_codes = [&](int g) {
+        const int sidx = g % kDmStages, p = g / G, gi = g % G;
+        const uint32_t b = bar_at(kBarCodes + sidx);
+        const int64_t pr0 = pass_row0(p);
+        mbar_arrive_expect_tx(b, kDmStageBytes);
+        const uint32_t dst = smem_addr(st + sidx * kDmStageBytes);
+#pragma unroll
+        for (int q = 0; q < kDmRows / 256; ++q)
+          tma_load_2d(dst + q * (kDmStageBytes / 4), &tmap, gi * 2 * kDmGroup, (int)(pr0 + q * 256),
+                      b, pol_codes);
+        last_codes[sidx] = g;
+      };
+      auto issue_book = [&](int s) {
+        const int m = s % M;
+        const uint32_t b = bar_at(kBarBook + (s & 1));
+        mbar_arrive_expect_tx(b, cbb + kDmHFloats * 4);
+        bulk_g2s(smem_addr(cb + (size_t)(s & 1) * cbs), a.C + (size_t)m * cbf, cbb, b);
+        bulk_g2s(smem_addr(hs + (s & 3) * kDmHFloats), a.hop + (size_t)m * kDmHFloats,
+                 kDmHFloats * 4, b);
+        last_book[s & 1] = s;
+      };
+      for (int g = 0; g < NG && g < kDmStages; ++g) issue_codes(g);
+      for (int s = 0; s < S && s < 2; ++s) issue_book(s);
+      for (int s = 0; s < S; ++s) {
+        if (*abort_flag) break;
+        const int p = s / M, m = s % M;
+        const int64_t rows = pass_row0(p + 1) - pass_row0(p);
+        const int nt = (int)((rows + 127) / 128);
+        wait(kBarFull + (s & 1), (uint32_t)(s >> 1) & 1u);   // A slot of s written
+        wait(kBarBook + (s & 1), (uint32_t)(s >> 1) & 1u);   // hidden operand of s landed
+        if (s + 2 < S) {
+          // the book buffer of s is read out; the hidden slot of s + 2 was last
+          // read by the MMAs of s - 2
+          if (s >= 2) wait(kBarMma + (s & 1), (uint32_t)((s - 2) >> 1) & 1u);
+          if (to) break;
+          issue_book(s + 2);
+        }
+        if (m % kDmGroup == kDmGroup - 1) {
+          const int g = p * G + m / kDmGroup;                  // its stage is read out
+          if (g + kDmStages < NG) issue_codes(g + kDmStages);
+        }
+        const int c = p * NC + m / kDmChain;
+        const bool first = m % kDmChain == 0;
+        if (first && c > 0) wait(kBarFlush, (uint32_t)(c - 1) & 1u);   // previous chain read out
+        if (to) break;
+        tc_fence_after();
+        const uint32_t hb = smem_addr(hs + (s & 3) * kDmHFloats);
+        const unsigned long long bh = opnd_desc(hb), bl = opnd_desc(hb + 1024);
+        const uint32_t aslot = tmem + kDmAcol + (uint32_t)(s & 1) * 128u;
+        for (int t = 0; t < nt; ++t) {
+          const uint32_t d = tmem + (uint32_t)(t * kDmTokens);
+          const uint32_t ah = aslot + (uint32_t)(t * 16), al = ah + 8u;
+          mma_tf32_ts(d, ah, bh, idesc, first ? 0u : 1u);
+          mma_tf32_ts(d, ah, bl, idesc, 1u);
+          mma_tf32_ts(d, al, bh, idesc, 1u);
+        }
+        mma_commit(bar_at(kBarMma + (s & 1)));
+        last_mma[s & 1] = s;
+        if (m % kDmChain == kDmChain - 1 || m == M - 1) mma_commit(bar_at(kBarChain));
+      }
+      if (*abort_flag) {
+        // let the copies and MMAs in flight land before the CTA's resources go
+        for (int i = 0; i < kDmStages; ++i)
+          if (last_codes[i] >= 0)
+            mbar_wait_bounded(bar_at(kBarCodes + i), (uint32_t)(last_codes[i] / kDmStages) & 1u);
+        for (int i = 0; i < 2; ++i) {
+          if (last_book[i] >= 0)
+            mbar_wait_bounded(bar_at(kBarBook + i), (uint32_t)(last_book[i] >> 1) & 1u);
+          if (last_mma[i] >= 0)
+            mbar_wait_bounded(bar_at(kBarMma + i), (uint32_t)(last_mma[i] >> 1) & 1u);
+        }
+        atomicOr(a.err, RQ_DEVERR_TIMEOUT);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ decoders
+    const int wg = warp >> 2, q = warp & 3;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    ArgBest mine{-FLT_MAX, INT_MAX};          // lane tok: this warp's best row for token tok
+    bool to = false;
+    auto wait = [&](int i, uint32_t parity) {
+      bool ok = to || mbar_try_wait(bar_at(i), parity) || mbar_wait_bounded(bar_at(i), parity);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok && !to) {
+        to = true;
+        *abort_flag = 1;
+      }
+    };
+    float *my = sacc + tid;                   // this thread's column of the tile g + 4 sums
+    auto flush = [&](int c, float (&acc)[kDmTokens], int nt) {
+      wait(kBarChain, (uint32_t)c & 1u);
+      if (to) return;
+      tc_fence_after();
+      if (wg < nt) {
+        const uint32_t base = tmem + lane_base + (uint32_t)(wg * kDmTokens);
+#pragma unroll
+        for (int c0 = 0; c0 < kDmTokens; c0 += 16) {
+          uint32_t raw[16];
+          tmem_ld16(base + (uint32_t)c0, raw);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc[c0 + j] = __fadd_rn(acc[c0 + j], __uint_as_float(raw[j]));
+        }
+      }
+      if (wg + 4 < nt) {
+        const uint32_t base = tmem + lane_base + (uint32_t)((wg + 4) * kDmTokens);
+#pragma unroll
+        for (int c0 = 0; c0 < kDmTokens; c0 += 16) {
+          uint32_t raw[16];
+          tmem_ld16(base + (uint32_t)c0, raw);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            my[(c0 + j) * 512] = __fadd_rn(my[(c0 + j) * 512], __uint_as_float(raw[j]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_at(kBarFlush));
+    };
+
+    for (int p = 0; p < npass && !to; ++p) {
+      const int64_t pr0 = pass_row0(p), rows = pass_row0(p + 1) - pr0;
+      const int nt = (int)((rows + 127) / 128);
+      float acc[kDmTokens];
+#pragma unroll
+      for (int t = 0; t < kDmTokens; ++t) {
+        acc[t] = 0.f;
+        my[t * 512] = 0.f;
+      }
+      uint4 cw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+      for (int m = 0; m < M; ++m) {
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+          to = true;
+          break;
+        }
+        const int s = p * M + m, i4 = m % kDmGroup;
+        if (i4 == 0) {
+          const int g = p * G + m / kDmGroup, sidx = g % kDmStages;
+          wait(kBarCodes + sidx, (uint32_t)(g / kDmStages) & 1u);
+          if (to) break;
+          const uint32_t stage = smem_addr(st + sidx * kDmStageBytes);
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+            cw[i] = lds_u4(stage + (uint32_t)((wg + 4 * i) * 128 + q * 32 + lane) * 16u);
+        }
+        wait(kBarBook + (s & 1), (uint32_t)(s >> 1) & 1u);
+        if (s >= 2) wait(kBarMma + (s & 1), (uint32_t)((s - 2) >> 1) & 1u);   // A slot free
+        if (to) break;
+        tc_fence_after();
+        const float *book = cb + (size_t)(s & 1) * cbs;
+        const uint32_t aslot = tmem + lane_base + kDmAcol + (uint32_t)(s & 1) * 128u;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (wg + 4 * i < nt) {
+            const uint32_t w = i4 == 0 ? cw[i].x : i4 == 1 ? cw[i].y : i4 == 2 ? cw[i].z : cw[i].w;
+            const float2 *p0 = reinterpret_cast<const float2 *>(book + a.fix(w & 0xFFFFu) * 6);
+            const float2 *p1 =
+                reinterpret_cast<const float2 *>(book + (a.K + a.fix(w >> 16)) * 6);
+            float hi[6], lo[6];
+#pragma unroll
+            for (int j2 = 0; j2 < 3; ++j2) {
+              const float2 x = p0[j2], y = p1[j2];
+              const float e0 = __fadd_rn(x.x, y.x), e1 = __fadd_rn(x.y, y.y);
+              hi[2 * j2] = tf32_hi(e0);
+              hi[2 * j2 + 1] = tf32_hi(e1);
+              lo[2 * j2] = __fsub_rn(e0, hi[2 * j2]);
+              lo[2 * j2 + 1] = __fsub_rn(e1, hi[2 * j2 + 1]);
+            }
+            tmem_st_hilo(aslot + (uint32_t)((wg + 4 * i) * 16), hi, lo);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_at(kBarFull + (s & 1)));
+        // the chain before this one has had its last MMAs issued: read it out
+        if (m % kDmChain == 0 && m > 0) flush(p * NC + m / kDmChain - 1, acc, nt);
+      }
+      if (to) break;
+      flush(p * NC + NC - 1, acc, nt);
+      if (to) break;
+
+      // epilogue: softcap, logits, per-token best row of this warp
+#pragma unroll
+      for (int tok = 0; tok < kDmTokens; ++tok) {
+        ArgBest best{-FLT_MAX, INT_MAX};
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = (wg + 4 * i) * 128 + q * 32 + lane;
+          if (r < rows && tok < a.nb) {
+            const int64_t v = pr0 + r;
+            const float y = softcap_f(i == 0 ? acc[tok] : my[tok * 512], a.cap);
+            if (a.logits) a.logits[(int64_t)(a.t0 + tok) * a.V + v] = y;
+            best = arg_better(best, ArgBest{y, (int)v});
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) best = arg_better(best, arg_shfl_xor(best, o));
+        if (lane == tok) mine = arg_better(mine, best);
+      }
+    }
+    wbest[warp * kDmTokens + lane] = mine;
+  }
+
+  griddep_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  if (a.am_val && tid < a.nb && tid < kDmTokens) {
+    ArgBest bb{-FLT_MAX, INT_MAX};
+    for (int w2 = 0; w2 < kDmDecWarps; ++w2) bb = arg_better(bb, wbest[w2 * kDmTokens + tid]);
+    const int64_t rowi = (int64_t)(a.t0 + tid) * a.nblk;
+    a.am_val[rowi + blockIdx.x] = bb.v;
+    a.am_idx[rowi + blockIdx.x] = bb.i;
+    for (int c = gridDim.x + blockIdx.x; c < a.nblk; c += gridDim.x) {
+      a.am_val[rowi + c] = -FLT_MAX;
+      a.am_idx[rowi + c] = INT_MAX;
+    }
+  }
+  if (warp == kDmDecWarps) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kDmTmemCols));
+  }
+}
+
+size_t decode_mma_smem(int K, int N) {
+  (void)N;
+  const size_t cbs = (size_t)align_up(2 * K * 6, 256) * 4;
+  return 1024 + (size_t)kDmStages * kDmStageBytes + 2 * cbs + kDmHSlots * kDmHFloats * 4 +
+         (size_t)kDmTokens * kDmDecWarps * 32 * 4 + kBars * 8 + (size_t)kDmDecWarps * kDmTokens * sizeof(ArgBest) + 16;
+}
+
+size_t decode_mma_hop_bytes(int M) { return (size_t)M * kDmHFloats * 4; }
+
+cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void *codes,
+                                     int64_t V, int D, int M, int K, int t0, int nb, int N,
+                                     float cap, float *hop, float *logits, float *am_val,
+                                     int *am_idx, int nblk, const DevInfo &di, cudaStream_t s) {
+  if (N != kDmTokens || nb < 1 || nb > kDmTokens || M % kDmGroup != 0) return cudaErrorInvalidValue;
+  CUtensorMap tmap;
+  const int P = 2 * M;
+  if (!encode_tmap_2d_u16(&tmap, codes, (uint64_t)P, (uint64_t)V, (uint64_t)P * 2,
+                          2 * kDmGroup, 256, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  {
+    void *args[] = {&h, &D, &t0, &nb, &hop};
+    cudaError_t e = launch_maybe_pdl(reinterpret_cast<const void *>(&split_hidden_kernel),
+                                     dim3((unsigned)M), dim3(256), 0, s, args, true);
+    if (e != cudaSuccess) return e;
+  }
+  const size_t smem = decode_mma_smem(K, N);
+  static size_t smem_set[128] = {};
+  if (di.device >= 128) return cudaErrorInvalidDevice;
+  const void *fn = reinterpret_cast<const void *>(&logits_decode_mma_kernel);
+  if (smem > smem_set[di.device]) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    smem_set[di.device] = smem;
+  }
+  DmArgs a;
+  a.C = C;
+  a.hop = hop;
+  a.V = V;
+  a.M = M;
+  a.K = K;
+  a.t0 = t0;
+  a.nb = nb;
+  a.cap = cap;
+  a.logits = logits;
+  a.am_val = am_val;
+  a.am_idx = am_idx;
+  a.nblk = nblk;
+  a.fix = make_codefix(K);
+  a.err = di.err;
+  void *args[] = {&tmap, &a};
+  return launch_maybe_pdl(fn, dim3((unsigned)decode_fma_blocks(V, di)), dim3(kDmThreads), smem, s,
+                          args, true);
+}
+
+}  // namespace rq

@@ -405,6 +405,16 @@ cudaError_t launch_logits_decode_fma(const float *h, const float *C, const void 
                                      float *logits, float *am_val, int *am_idx, int nblk,
                                      const DevInfo &di, cudaStream_t s);
 
+// The same on the tcgen05 tensor cores (tf32 MMAs with a hi/lo split for
+// fp32 accuracy); N = 32 tokens per group, M % 4 == 0.  hop: device scratch of
+// decode_mma_hop_bytes(M) for the group's split hidden operand.
+cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void *codes,
+                                     int64_t V, int D, int M, int K, int t0, int nb, int N,
+                                     float cap, float *hop, float *logits, float *am_val,
+                                     int *am_idx, int nblk, const DevInfo &di, cudaStream_t s);
+size_t decode_mma_smem(int K, int N);
+size_t decode_mma_hop_bytes(int M);
+
 // Batched pass with the LUT read through L2 (token groups of <= 32).
 cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K,
                              const float *lut, int Bs, int lut_t0, int out_t0, int nb,

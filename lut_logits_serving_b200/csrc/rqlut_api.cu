@@ -232,8 +232,15 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
     if (dfma && nb == kTokenGroup) {
       if (!marked && (e = prof_mark(t_prof_start, s)) != cudaSuccess) break;
       marked = true;
-      e = launch_logits_decode_fma(h, C, codes, d.V, d.D, d.M, d.K, b0, nb, softcap, logits, amv,
-                                   ami, nblk, di, s);
+      // the tensor-core path keeps the group's split hidden operand in the
+      // (here unused) table region
+      if (decode_mma_smem(d.K, kTokenGroup) <= (size_t)di.max_smem_optin &&
+          decode_mma_hop_bytes(d.M) <= lut_bytes)
+        e = launch_logits_decode_mma(h, C, codes, d.V, d.D, d.M, d.K, b0, nb, kTokenGroup, softcap,
+                                     lut, logits, amv, ami, nblk, di, s);
+      else
+        e = launch_logits_decode_fma(h, C, codes, d.V, d.D, d.M, d.K, b0, nb, softcap, logits,
+                                     amv, ami, nblk, di, s);
       continue;
     }
     e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, s);
