@@ -181,6 +181,34 @@ RQ_API int rq_logits_from_hidden(const float *h, const float *C, const void *cod
                           size_t ws_bytes, void *stream);
 
 /*
+ * Kernel choice for the full 32-token groups of rq_logits_from_hidden_path
+ * (groups of fewer tokens always read their tables through L2).  The decode
+ * paths rebuild each vocabulary row once per group (the decode-then-matmul
+ * the LUT section checks the lookup against) and contract it with the
+ * group's hidden states; they need RQ_CODES_U16, L = 2, D = 6 M, M % 8 == 0,
+ * K <= 1024 and 16-byte aligned C and codes.
+ *   RQ_PATH_AUTO        -- RQ_PATH_DECODE_FP32 where it applies, else tables
+ *   RQ_PATH_TABLES      -- per-group tables read through L2 (lookup + sum)
+ *   RQ_PATH_DECODE_FP32 -- rows decoded into shared memory, fp32 FMAs
+ *   RQ_PATH_DECODE_TC   -- rows decoded into shared memory, tcgen05 tf32
+ *                          MMAs on a hi/lo split with fp32 chain sums; also
+ *                          needs K >= 8 (its hidden operand is staged in the
+ *                          workspace's table region)
+ */
+enum { RQ_PATH_AUTO = 0, RQ_PATH_TABLES = 1, RQ_PATH_DECODE_FP32 = 2, RQ_PATH_DECODE_TC = 3 };
+
+/*
+ * rq_logits_from_hidden_path -- rq_logits_from_hidden with an explicit
+ * kernel choice for full token groups.  Same arguments, workspace and
+ * errors; an unknown `path` is RQ_ERR_INVALID_ARGUMENT, a decode path the
+ * shape, format or alignment cannot take is RQ_ERR_UNSUPPORTED.
+ */
+RQ_API int rq_logits_from_hidden_path(const float *h, const float *C, const void *codes,
+                                      int fmt, rq_dims d, int B, float softcap,
+                                      float *logits, int32_t *argmax, void *ws,
+                                      size_t ws_bytes, int path, void *stream);
+
+/*
  * rq_greedy_step -- one greedy decoding step of the output head in one call:
  * rq_logits_from_hidden with argmax, then the bf16 input rows of the picked
  * tokens (the embeddings the next step consumes), rebuilt on demand as in

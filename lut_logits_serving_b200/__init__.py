@@ -24,16 +24,23 @@ __all__ = [
     "RqDims", "RqError", "U16", "PACKED10", "SCHED", "U8", "lib", "rq_pack8", "dims", "rq_prepare_sched",
     "rq_status_string", "rq_version", "rq_codes_bytes", "rq_lut_token_stride",
     "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
-    "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_decode_rows",
+    "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_logits_from_hidden_path",
+    "rq_decode_rows",
     "rq_pack10", "rq_device_error", "rq_set_profile_events", "rq_lut_logits_static",
     "rq_greedy_step", "rq_encode", "rq_topk_workspace_bytes", "rq_topk_sample",
-    "rq_last_cuda_error", "rq_cuda_error_name",
+    "rq_last_cuda_error", "rq_cuda_error_name", "PATH_AUTO", "PATH_TABLES", "PATH_DECODE_FP32",
+    "PATH_DECODE_TC",
 ]
 
 U16 = 0
 PACKED10 = 1
 SCHED = 2
 U8 = 3
+# kernel of full 32-token groups in rq_logits_from_hidden (rqlut.h RQ_PATH_*)
+PATH_AUTO = 0
+PATH_TABLES = 1
+PATH_DECODE_FP32 = 2
+PATH_DECODE_TC = 3
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librqlut.so")
 
@@ -78,6 +85,8 @@ _SIGNATURES = {
     "rq_lut_build": (_i, [_p, _p, RqDims, _i, _p, _p]),
     "rq_lut_logits": (_i, [_p, _i, RqDims, _p, _i, _f, _p, _p, _p, _sz, _p]),
     "rq_logits_from_hidden": (_i, [_p, _p, _p, _i, RqDims, _i, _f, _p, _p, _p, _sz, _p]),
+    "rq_logits_from_hidden_path": (_i, [_p, _p, _p, _i, RqDims, _i, _f, _p, _p, _p, _sz, _i,
+                                        _p]),
     "rq_decode_rows": (_i, [_p, _i64, _p, _i, _p, RqDims, _f, _p, _p]),
     "rq_pack10": (_i, [_p, RqDims, _p, _p]),
     "rq_pack8": (_i, [_p, RqDims, _p, _p]),
@@ -230,8 +239,10 @@ def rq_lut_logits(codes, fmt: int, d: RqDims, lut, B: int, softcap: float = 30.0
 
 def rq_logits_from_hidden(h, C, codes, fmt: int, d: RqDims, softcap: float = 30.0,
                           want_logits: bool = True, want_argmax: bool = False, logits=None,
-                          argmax=None, ws=None, stream=None):
-    """Returns (logits float32 [B, V] or None, argmax int32 [B] or None, ws)."""
+                          argmax=None, ws=None, stream=None, path: int = None):
+    """Returns (logits float32 [B, V] or None, argmax int32 [B] or None, ws).
+    ``path`` (one of PATH_*) picks the kernel of full 32-token groups; None
+    is the library's default (rq_logits_from_hidden)."""
     torch = _torch()
     B = h.shape[0]
     if want_logits and logits is None:
@@ -240,12 +251,22 @@ def rq_logits_from_hidden(h, C, codes, fmt: int, d: RqDims, softcap: float = 30.
         argmax = _empty((B,), torch.int32, h)
     nbytes = rq_fused_workspace_bytes(d, B, fmt, argmax is not None)
     wp, wn, ws = _workspace(nbytes, h, ws)
-    _check("rq_logits_from_hidden", lib().rq_logits_from_hidden(
-        _cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C"),
-        _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, B, float(softcap),
-        _ptr_or_null(logits, torch.float32, "logits"),
-        _ptr_or_null(argmax, torch.int32, "argmax"), wp, wn, _stream(stream)))
+    args = (_cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C"),
+            _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, B, float(softcap),
+            _ptr_or_null(logits, torch.float32, "logits"),
+            _ptr_or_null(argmax, torch.int32, "argmax"), wp, wn)
+    if path is None:
+        _check("rq_logits_from_hidden", lib().rq_logits_from_hidden(*args, _stream(stream)))
+    else:
+        _check("rq_logits_from_hidden_path",
+               lib().rq_logits_from_hidden_path(*args, int(path), _stream(stream)))
     return logits, argmax, ws
+
+
+def rq_logits_from_hidden_path(h, C, codes, fmt: int, d: RqDims, path: int,
+                               softcap: float = 30.0, **kw):
+    """rq_logits_from_hidden with an explicit kernel for full token groups."""
+    return rq_logits_from_hidden(h, C, codes, fmt, d, softcap, path=path, **kw)
 
 
 def rq_decode_rows(ids, codes, fmt: int, C, d: RqDims, scale: float, out=None, stream=None):

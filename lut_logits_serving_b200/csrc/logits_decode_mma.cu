@@ -1,6 +1,6 @@
 // logits_decode_mma.cu -- logits of a token group by decoding vocabulary rows
-// straight into tensor memory and multiplying them with the hidden states on
-// the tcgen05 tensor cores.
+// into shared memory and multiplying them with the hidden states on the
+// tcgen05 tensor cores.
 //
 // "Gemma-2 runtime compression: NF4 + LUT serving", LUT section: the lookup
 // + sum equals the decode-then-matmul the pages check it against,
@@ -13,33 +13,30 @@
 // so a tf32 MMA reads it exactly) and x_lo = x - x_hi (exact in fp32, at most
 // half a tf32 ulp of x), and
 //   E . h = E_hi h_hi + E_hi h_lo + E_lo h_hi + (E_lo h_lo, dropped),
-// three MMAs whose error is about 2^-22 of |E||h| per product.  The tensor
-// core's fp32 accumulation does not round to nearest and its error grows with
-// the length of an accumulation chain, so a chain covers 16 subspaces; each
-// finished chain is added into fp32 registers (round to nearest) by the
-// threads that own its rows.  Measured against fp64 this keeps the logits
-// near 1e-6 of their scale; one chain over all 384 subspaces was ~3e-5.
+// with error about 2^-22 of |E||h| per product.  Two MMAs per tile and
+// subspace: E_hi against the 64 columns [h_hi | h_lo] (an N = 64 MMA costs
+// what an N = 32 one does), and E_lo against h_hi into the first 32.  The
+// tensor core's fp32 accumulation does not round to nearest and its error
+// grows with the length of an accumulation chain, so a chain covers 16
+// subspaces in one of two TMEM accumulator sets; the threads that own a
+// finished chain's rows add it into fp32 registers (round to nearest) while
+// the next chain runs in the other set.  Measured against fp64 this keeps the
+// logits near 1e-6 of their scale; one chain over all 384 subspaces was ~3e-5.
 //
 // Design for sm_100a (ds = 6, L = 2, uint16 codes, K <= 1024, 32 tokens).
 // One CTA per SM walks an even share of the vocabulary in passes of up to
-// 1024 rows = 8 M = 128 tiles; per pass it runs every subspace once, so each
-// codebook is fetched once per 1024 rows.  Warp-specialised, mbarrier-driven:
+// 512 rows = 4 M = 128 tiles, running every subspace once per pass.
+// Warp-specialised and mbarrier-driven, nothing waits on a CTA barrier:
 //   * 16 decoder warps (4 warpgroups).  Thread (warpgroup g, warp q, lane)
-//     owns row 32 q + lane of tiles g and g + 4.  Per subspace it gathers the
-//     row's two codewords from the shared-memory codebook, adds them, splits
-//     the sum into hi and lo and stores both (6 dims + 2 zero pads each) into
-//     its own TMEM lane with one tcgen05.st -- the MMA's A operand lives in
-//     tensor memory, so decoded rows never touch shared memory.  Its fp32
-//     sums are in registers for tile g and in shared memory (thread-private
-//     columns) for tile g + 4: 17 warps leave 96 registers a thread;
+//     owns row 32 q + lane of tile g.  Per subspace it gathers the row's two
+//     codewords from the shared-memory codebook, adds them, splits the sum
+//     into hi and lo and stores both as one K = 8 row (6 dims, 2 zero pads)
+//     of the canonical K-major operand layout into a double-buffered A slot;
 //   * one control warp: one lane issues the TMA code tiles ({8 codes, 256
 //     rows}, 3 stages of 4 subspaces), one bulk copy per subspace of the
 //     codebook pair (48 KB at K = 1024, double-buffered) plus the pre-split
-//     hidden operand (2 KB, 4-slot ring), and the 3 x 8 MMAs (M = 128,
-//     N = 32, K = 8; A from TMEM, B from shared memory) per subspace;
-//   * TMEM: accumulators 8 tiles x 32 columns, and two A slots per tile of
-//     16 columns (hi, lo), 512 columns in all.  Decoding subspace s + 1 fills
-//     the other A slot while the MMAs of s run.
+//     hidden operand (2 KB, 4-slot ring), and the 2 x 4 MMAs per subspace;
+//   * TMEM: two accumulator sets of 4 tiles x 64 columns, 512 columns.
 // Every wait is bounded; a timed-out wait raises a CTA-wide abort flag, the
 // control lane waits (bounded) for its copies and MMAs in flight, and the CTA
 // frees its TMEM and ends.
@@ -55,29 +52,30 @@ namespace {
 constexpr int kDmTokens = 32;
 constexpr int kDmDecWarps = 16;
 constexpr int kDmThreads = (kDmDecWarps + 1) * 32;   // + the control warp
-constexpr int kDmTiles = 8;                          // M = 128 tiles per pass
+constexpr int kDmTiles = 4;                          // M = 128 tiles per pass
 constexpr int kDmRows = kDmTiles * 128;              // rows per pass
 constexpr int kDmGroup = 4;                          // subspaces per code stage (16 B per row)
-constexpr int kDmStageBytes = kDmRows * kDmGroup * 4;   // 16 KB
+constexpr int kDmStageBytes = kDmRows * kDmGroup * 4;   // 8 KB
 constexpr int kDmStages = 3;
+constexpr int kDmASlots = 2;                         // A slots: decoding runs 2 subspaces ahead
 constexpr int kDmChain = 16;                         // subspaces per accumulation chain
-constexpr int kDmHFloats = 512;                      // one subspace's hidden operand: hi, lo
+constexpr int kDmTileBytes = 128 * 32;               // one M = 128, K = 8 tf32 operand
+constexpr int kDmSlotBytes = 2 * kDmTiles * kDmTileBytes;   // A slot: [E_hi tiles][E_lo tiles]
+constexpr int kDmHFloats = 512;                      // hidden operand: 64 rows x K = 8
 constexpr int kDmHSlots = 4;
-constexpr uint32_t kDmTmemCols = 512;
-constexpr uint32_t kDmAcol = 256;                    // first A-slot column
+constexpr uint32_t kDmTmemCols = 512;                // 2 sets x 4 tiles x 64 columns
 
 // mbarriers
-constexpr int kBarCodes = 0;                         // 3: code stages (TMA)
-constexpr int kBarBook = 3;                          // 2: codebook + hidden operand (bulk)
-constexpr int kBarFull = 5;                          // 2: A slot written (16 decoder warps)
-constexpr int kBarMma = 7;                           // 2: MMAs of a subspace done (commit)
-constexpr int kBarChain = 9;                         // 1: MMAs of a chain done (commit)
-constexpr int kBarFlush = 10;                        // 1: chain read into registers (16 warps)
-constexpr int kBars = 11;
+constexpr int kBarCodes = 0;                           // code stage g % 3 landed (TMA)
+constexpr int kBarBook = kBarCodes + kDmStages;        // 2: codebook + hidden operand (bulk)
+constexpr int kBarFull = kBarBook + 2;                 // A slot s % 2 written (16 decoder warps)
+constexpr int kBarMma = kBarFull + kDmASlots;          // MMAs of subspace s done, on s % 2 (commit)
+constexpr int kBarFlush = kBarMma + kDmASlots;         // 2: chain c read out, on c & 1 (16 warps)
+constexpr int kBars = kBarFlush + 2;
 
 struct DmArgs {
   const float *C;      // [M][2][K][6]
-  const float *hop;    // [M][512]: hi then lo hidden operand per subspace
+  const float *hop;    // [M][512]: per subspace rows 0..31 h_hi, 32..63 h_lo
   int64_t V;
   int M, K;
   int t0, nb;          // tokens t0 .. t0 + nb - 1
@@ -104,19 +102,19 @@ __device__ __forceinline__ unsigned long long opnd_desc(uint32_t saddr) {
          ((unsigned long long)(256 >> 4) << 32) | (1ull << 46);
 }
 
-// Instruction descriptor: D fp32, A and B tf32, both K-major, M = 128, N = 32.
-__device__ __forceinline__ uint32_t mma_idesc() {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(kDmTokens >> 3) << 17) |
+// Instruction descriptor: D fp32, A and B tf32, both K-major, M = 128, N.
+__device__ __forceinline__ uint32_t mma_idesc(int n) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(128 >> 4) << 24);
 }
 
-// D[tmem] (+)= A[tmem] . B[smem]^T
-__device__ __forceinline__ void mma_tf32_ts(uint32_t d, uint32_t a, unsigned long long b,
-                                            uint32_t idesc, uint32_t accum) {
+// D[tmem] (+)= A[smem] . B[smem]^T
+__device__ __forceinline__ void mma_tf32(uint32_t d, unsigned long long a, unsigned long long b,
+                                         uint32_t idesc, uint32_t accum) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d),
-      "r"(a), "l"(b), "r"(idesc), "r"(accum), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -137,6 +135,10 @@ __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 
+__device__ __forceinline__ void proxy_fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -145,24 +147,10 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// one TMEM row segment: hi[0..5], 0, 0, lo[0..5], 0, 0
-__device__ __forceinline__ void tmem_st_hilo(uint32_t taddr, const float (&hi)[6],
-                                             const float (&lo)[6]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %7, %8, %9, %10, "
-      "%11, %12, %13, %7, %7};" ::"r"(taddr),
-      "r"(__float_as_uint(hi[0])), "r"(__float_as_uint(hi[1])), "r"(__float_as_uint(hi[2])),
-      "r"(__float_as_uint(hi[3])), "r"(__float_as_uint(hi[4])), "r"(__float_as_uint(hi[5])),
-      "r"(0u), "r"(__float_as_uint(lo[0])), "r"(__float_as_uint(lo[1])),
-      "r"(__float_as_uint(lo[2])), "r"(__float_as_uint(lo[3])), "r"(__float_as_uint(lo[4])),
-      "r"(__float_as_uint(lo[5])));
-}
-
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // x rounded to nearest (ties to even) with the low 13 mantissa bits cleared
@@ -182,9 +170,9 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
 
 }  // namespace
 
-// Hidden operand of one token group, per subspace m: h_hi then h_lo, each
-// [32 tokens][K = 8] in the canonical K-major layout (dims 6, 7 and tokens
-// past the group are zero).
+// Hidden operand of one token group, per subspace m: 64 rows of K = 8 in the
+// canonical K-major layout, rows 0..31 the tokens' hi parts and rows 32..63
+// their lo parts (dims 6, 7 and tokens past the group are zero).
 __global__ void __launch_bounds__(256) split_hidden_kernel(const float *__restrict__ h, int D,
                                                            int t0, int nb,
                                                            float *__restrict__ hop) {
@@ -194,7 +182,7 @@ __global__ void __launch_bounds__(256) split_hidden_kernel(const float *__restri
   const float xh = tf32_hi(x);
   float *o = hop + (size_t)m * kDmHFloats;
   o[opnd_idx(tok, k)] = xh;
-  o[256 + opnd_idx(tok, k)] = __fsub_rn(x, xh);
+  o[opnd_idx(32 + tok, k)] = __fsub_rn(x, xh);
   griddep_launch_dependents();
 }
 
@@ -205,11 +193,11 @@ __global__ void __launch_bounds__(kDmThreads, 1)
   const int cbf = 2 * a.K * 6;                                     // floats per codebook pair
   const uint32_t cbb = (uint32_t)cbf * 4u;
   const size_t cbs = (size_t)align_up(cbf, 256);                   // floats per book buffer
-  unsigned char *st = smem;                                        // code stages
+  unsigned char *aop = smem;                                       // A slots
+  unsigned char *st = aop + kDmASlots * kDmSlotBytes;              // code stages
   float *cb = reinterpret_cast<float *>(st + kDmStages * kDmStageBytes);
   float *hs = cb + 2 * cbs;                                        // hidden operand slots
-  float *sacc = hs + kDmHSlots * kDmHFloats;                       // [32 tokens][512 threads]
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sacc + kDmTokens * kDmDecWarps * 32);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(hs + kDmHSlots * kDmHFloats);
   ArgBest *wbest = reinterpret_cast<ArgBest *>(bar + kBars);      // [16 warps][32]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(wbest + kDmDecWarps * kDmTokens);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -218,18 +206,23 @@ __global__ void __launch_bounds__(kDmThreads, 1)
   if (tid == 0) {
     prefetch_tmap(&tmap);
     for (int i = 0; i < kBars; ++i)
-      mbar_init(smem_addr(&bar[i]), (i == kBarFull || i == kBarFull + 1 || i == kBarFlush)
-                                        ? (uint32_t)kDmDecWarps
-                                        : 1u);
+      mbar_init(smem_addr(&bar[i]),
+                ((i >= kBarFull && i < kBarFull + kDmASlots) || i == kBarFlush || i == kBarFlush + 1)
+                    ? (uint32_t)kDmDecWarps
+                    : 1u);
     fence_mbar_init();
     *abort_flag = 0;
   }
+  // the K pads (dims 6, 7) of the A slots stay zero
+  for (int i = tid; i < kDmASlots * kDmSlotBytes / 16; i += kDmThreads)
+    reinterpret_cast<uint4 *>(aop)[i] = make_uint4(0, 0, 0, 0);
   if (warp == kDmDecWarps) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kDmTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  proxy_fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -238,18 +231,19 @@ __global__ void __launch_bounds__(kDmThreads, 1)
 
   const int M = a.M, G = a.M / kDmGroup, NC = (a.M + kDmChain - 1) / kDmChain;
   const int64_t r0 = a.V * blockIdx.x / gridDim.x, r1 = a.V * (blockIdx.x + 1) / gridDim.x;
-  const int npass = (int)((r1 - r0 + kDmRows - 1) / kDmRows);
+  const int npass = (int)((r1 - r0 + kDmRows - 1) / kDmRows);   // full passes, then the rest
   const int S = npass * M;                   // steps: (pass, subspace)
   const int NG = npass * G;                  // code groups
-  auto pass_row0 = [&](int p) { return r0 + (r1 - r0) * p / npass; };
   auto bar_at = [&](int i) { return smem_addr(&bar[i]); };
 
   if (warp == kDmDecWarps) {
     // ------------------------------------------------------------ control
     if (lane == 0 && S > 0) {
       const uint64_t pol_codes = l2_policy_evict_first();
-      const uint32_t idesc = mma_idesc();
-      int last_codes[kDmStages] = {-1, -1, -1}, last_book[2] = {-1, -1}, last_mma[2] = {-1, -1};
+      const uint32_t id64 = mma_idesc(2 * kDmTokens), id32 = mma_idesc(kDmTokens);
+      int last_codes[kDmStages], last_book[2] = {-1, -1}, last_mma[kDmASlots];
+      for (int i = 0; i < kDmStages; ++i) last_codes[i] = -1;
+      for (int i = 0; i < kDmASlots; ++i) last_mma[i] = -1;
       bool to = false;
       auto wait = [&](int i, uint32_t parity) {
         if (!to && !mbar_try_wait(bar_at(i), parity) && !mbar_wait_bounded(bar_at(i), parity)) {
@@ -260,17 +254,15 @@ __global__ void __launch_bounds__(kDmThreads, 1)
       auto issue_codes = [&](int g) {
         const int sidx = g % kDmStages, p = g / G, gi = g % G;
         const uint32_t b = bar_at(kBarCodes + sidx);
-        const int64_t pr0 = pass_row0(p);
         mbar_arrive_expect_tx(b, kDmStageBytes);
         const uint32_t dst = smem_addr(st + sidx * kDmStageBytes);
 #pragma unroll
         for (int q = 0; q < kDmRows / 256; ++q)
-          tma_load_2d(dst + q * (kDmStageBytes / 4), &tmap, gi * 2 * kDmGroup, (int)(pr0 + q * 256),
-                      b, pol_codes);
+          tma_load_2d(dst + q * 4096, &tmap, gi * 2 * kDmGroup,
+                      (int)(r0 + (int64_t)p * kDmRows + q * 256), b, pol_codes);
         last_codes[sidx] = g;
       };
-      auto issue_book = [&](int s) {
-        const int m = s % M;
+      auto issue_book = [&](int s, int m) {
         const uint32_t b = bar_at(kBarBook + (s & 1));
         mbar_arrive_expect_tx(b, cbb + kDmHFloats * 4);
         bulk_g2s(smem_addr(cb + (size_t)(s & 1) * cbs), a.C + (size_t)m * cbf, cbb, b);
@@ -279,20 +271,23 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         last_book[s & 1] = s;
       };
       for (int g = 0; g < NG && g < kDmStages; ++g) issue_codes(g);
-      for (int s = 0; s < S && s < 2; ++s) issue_book(s);
+      for (int s = 0; s < S && s < 2; ++s) issue_book(s, s % M);
+      int p = 0, m = 0, nt = 0;
       for (int s = 0; s < S; ++s) {
+        if (m == 0) {
+          const int64_t rows = (r1 - r0) - (int64_t)p * kDmRows;
+          nt = (int)(((rows < kDmRows ? rows : kDmRows) + 127) / 128);
+        }
         if (*abort_flag) break;
-        const int p = s / M, m = s % M;
-        const int64_t rows = pass_row0(p + 1) - pass_row0(p);
-        const int nt = (int)((rows + 127) / 128);
-        wait(kBarFull + (s & 1), (uint32_t)(s >> 1) & 1u);   // A slot of s written
+        wait(kBarFull + s % kDmASlots, (uint32_t)(s / kDmASlots) & 1u);   // A slot of s written
         wait(kBarBook + (s & 1), (uint32_t)(s >> 1) & 1u);   // hidden operand of s landed
         if (s + 2 < S) {
-          // the book buffer of s is read out; the hidden slot of s + 2 was last
-          // read by the MMAs of s - 2
-          if (s >= 2) wait(kBarMma + (s & 1), (uint32_t)((s - 2) >> 1) & 1u);
+          // the book buffer of s is read out (its decode is done); the hidden
+          // slot of s + 2 was last read by the MMAs of s - 2 (waited for
+          // before the commit of s, which lands on the same barrier)
+          if (s >= 2) wait(kBarMma + (s - 2) % kDmASlots, (uint32_t)((s - 2) / kDmASlots) & 1u);
           if (to) break;
-          issue_book(s + 2);
+          issue_book(s + 2, m + 2 < M ? m + 2 : m + 2 - M);
         }
         if (m % kDmGroup == kDmGroup - 1) {
           const int g = p * G + m / kDmGroup;                  // its stage is read out
@@ -300,42 +295,48 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         }
         const int c = p * NC + m / kDmChain;
         const bool first = m % kDmChain == 0;
-        if (first && c > 0) wait(kBarFlush, (uint32_t)(c - 1) & 1u);   // previous chain read out
+        // chain c - 2 (same set) is read out; one barrier per set, as the
+        // decoders may finish reading chain c - 1 before this wait
+        if (first && c >= 2) wait(kBarFlush + (c & 1), (uint32_t)((c - 2) >> 1) & 1u);
         if (to) break;
         tc_fence_after();
         const uint32_t hb = smem_addr(hs + (s & 3) * kDmHFloats);
-        const unsigned long long bh = opnd_desc(hb), bl = opnd_desc(hb + 1024);
-        const uint32_t aslot = tmem + kDmAcol + (uint32_t)(s & 1) * 128u;
+        const unsigned long long bd = opnd_desc(hb);
+        const uint32_t slot = smem_addr(aop + (s % kDmASlots) * kDmSlotBytes);
+        const uint32_t set = tmem + (uint32_t)(c & 1) * (kDmTiles * 2 * kDmTokens);
         for (int t = 0; t < nt; ++t) {
-          const uint32_t d = tmem + (uint32_t)(t * kDmTokens);
-          const uint32_t ah = aslot + (uint32_t)(t * 16), al = ah + 8u;
-          mma_tf32_ts(d, ah, bh, idesc, first ? 0u : 1u);
-          mma_tf32_ts(d, ah, bl, idesc, 1u);
-          mma_tf32_ts(d, al, bh, idesc, 1u);
+          const uint32_t d = set + (uint32_t)(t * 2 * kDmTokens);
+          mma_tf32(d, opnd_desc(slot + t * kDmTileBytes), bd, id64, first ? 0u : 1u);
+          mma_tf32(d, opnd_desc(slot + (kDmTiles + t) * kDmTileBytes), bd, id32, 1u);
         }
-        mma_commit(bar_at(kBarMma + (s & 1)));
-        last_mma[s & 1] = s;
-        if (m % kDmChain == kDmChain - 1 || m == M - 1) mma_commit(bar_at(kBarChain));
+        mma_commit(bar_at(kBarMma + s % kDmASlots));
+        last_mma[s % kDmASlots] = s;
+        if (++m == M) {
+          m = 0;
+          ++p;
+        }
       }
       if (*abort_flag) {
         // let the copies and MMAs in flight land before the CTA's resources go
         for (int i = 0; i < kDmStages; ++i)
           if (last_codes[i] >= 0)
             mbar_wait_bounded(bar_at(kBarCodes + i), (uint32_t)(last_codes[i] / kDmStages) & 1u);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 2; ++i)
           if (last_book[i] >= 0)
             mbar_wait_bounded(bar_at(kBarBook + i), (uint32_t)(last_book[i] >> 1) & 1u);
+        for (int i = 0; i < kDmASlots; ++i)
           if (last_mma[i] >= 0)
-            mbar_wait_bounded(bar_at(kBarMma + i), (uint32_t)(last_mma[i] >> 1) & 1u);
-        }
+            mbar_wait_bounded(bar_at(kBarMma + i), (uint32_t)(last_mma[i] / kDmASlots) & 1u);
         atomicOr(a.err, RQ_DEVERR_TIMEOUT);
       }
     }
   } else {
     // ------------------------------------------------------------ decoders
     const int wg = warp >> 2, q = warp & 3;
+    const int r = wg * 128 + q * 32 + lane;   // this thread's row of a pass
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     ArgBest mine{-FLT_MAX, INT_MAX};          // lane tok: this warp's best row for token tok
+    float acc[kDmTokens];
     bool to = false;
     auto wait = [&](int i, uint32_t parity) {
       bool ok = to || mbar_try_wait(bar_at(i), parity) || mbar_wait_bounded(bar_at(i), parity);
@@ -345,47 +346,37 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         *abort_flag = 1;
       }
     };
-    float *my = sacc + tid;                   // this thread's column of the tile g + 4 sums
-    auto flush = [&](int c, float (&acc)[kDmTokens], int nt) {
-      wait(kBarChain, (uint32_t)c & 1u);
-      if (to) return;
-      tc_fence_after();
+    // add chain c (its MMAs are done) into the register sums; tiles past the
+    // pass's rows are skipped warp-uniformly but every warp arrives
+    auto flush = [&](int c, int nt) {
       if (wg < nt) {
-        const uint32_t base = tmem + lane_base + (uint32_t)(wg * kDmTokens);
+        tc_fence_after();
+        const uint32_t base = tmem + lane_base +
+                              (uint32_t)((c & 1) * (kDmTiles * 2 * kDmTokens) + wg * 2 * kDmTokens);
+        uint32_t x[16], y[16];
 #pragma unroll
         for (int c0 = 0; c0 < kDmTokens; c0 += 16) {
-          uint32_t raw[16];
-          tmem_ld16(base + (uint32_t)c0, raw);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) acc[c0 + j] = __fadd_rn(acc[c0 + j], __uint_as_float(raw[j]));
-        }
-      }
-      if (wg + 4 < nt) {
-        const uint32_t base = tmem + lane_base + (uint32_t)((wg + 4) * kDmTokens);
-#pragma unroll
-        for (int c0 = 0; c0 < kDmTokens; c0 += 16) {
-          uint32_t raw[16];
-          tmem_ld16(base + (uint32_t)c0, raw);
+          tmem_ld16(base + (uint32_t)c0, x);
+          tmem_ld16(base + (uint32_t)(kDmTokens + c0), y);
+          tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            my[(c0 + j) * 512] = __fadd_rn(my[(c0 + j) * 512], __uint_as_float(raw[j]));
+            acc[c0 + j] = __fadd_rn(acc[c0 + j],
+                                    __fadd_rn(__uint_as_float(x[j]), __uint_as_float(y[j])));
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_at(kBarFlush));
+      if (lane == 0) mbar_arrive(bar_at(kBarFlush + (c & 1)));
     };
 
     for (int p = 0; p < npass && !to; ++p) {
-      const int64_t pr0 = pass_row0(p), rows = pass_row0(p + 1) - pr0;
+      const int64_t pr0 = r0 + (int64_t)p * kDmRows;
+      const int64_t rows = (r1 - pr0) < kDmRows ? (r1 - pr0) : kDmRows;
       const int nt = (int)((rows + 127) / 128);
-      float acc[kDmTokens];
 #pragma unroll
-      for (int t = 0; t < kDmTokens; ++t) {
-        acc[t] = 0.f;
-        my[t * 512] = 0.f;
-      }
-      uint4 cw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+      for (int t = 0; t < kDmTokens; ++t) acc[t] = 0.f;
+      uint4 cw = make_uint4(0, 0, 0, 0);
       for (int m = 0; m < M; ++m) {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) {
           to = true;
@@ -396,61 +387,61 @@ __global__ void __launch_bounds__(kDmThreads, 1)
           const int g = p * G + m / kDmGroup, sidx = g % kDmStages;
           wait(kBarCodes + sidx, (uint32_t)(g / kDmStages) & 1u);
           if (to) break;
-          const uint32_t stage = smem_addr(st + sidx * kDmStageBytes);
-#pragma unroll
-          for (int i = 0; i < 2; ++i)
-            cw[i] = lds_u4(stage + (uint32_t)((wg + 4 * i) * 128 + q * 32 + lane) * 16u);
+          cw = lds_u4(smem_addr(st + sidx * kDmStageBytes) + (uint32_t)r * 16u);
         }
         wait(kBarBook + (s & 1), (uint32_t)(s >> 1) & 1u);
-        if (s >= 2) wait(kBarMma + (s & 1), (uint32_t)((s - 2) >> 1) & 1u);   // A slot free
+        if (s >= kDmASlots)                                     // A slot free
+          wait(kBarMma + s % kDmASlots, (uint32_t)((s - kDmASlots) / kDmASlots) & 1u);
         if (to) break;
-        tc_fence_after();
-        const float *book = cb + (size_t)(s & 1) * cbs;
-        const uint32_t aslot = tmem + lane_base + kDmAcol + (uint32_t)(s & 1) * 128u;
+        // the MMAs of s - 3, the last of the previous chain, are done: read it out
+        if (m % kDmChain == kDmASlots - 1 && m > kDmChain) flush(p * NC + m / kDmChain - 1, nt);
+        if (wg < nt) {
+          const float *book = cb + (size_t)(s & 1) * cbs;
+          const uint32_t w = i4 == 0 ? cw.x : i4 == 1 ? cw.y : i4 == 2 ? cw.z : cw.w;
+          const float2 *p0 = reinterpret_cast<const float2 *>(book + a.fix(w & 0xFFFFu) * 6);
+          const float2 *p1 = reinterpret_cast<const float2 *>(book + (a.K + a.fix(w >> 16)) * 6);
+          float hi[6], lo[6];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if (wg + 4 * i < nt) {
-            const uint32_t w = i4 == 0 ? cw[i].x : i4 == 1 ? cw[i].y : i4 == 2 ? cw[i].z : cw[i].w;
-            const float2 *p0 = reinterpret_cast<const float2 *>(book + a.fix(w & 0xFFFFu) * 6);
-            const float2 *p1 =
-                reinterpret_cast<const float2 *>(book + (a.K + a.fix(w >> 16)) * 6);
-            float hi[6], lo[6];
-#pragma unroll
-            for (int j2 = 0; j2 < 3; ++j2) {
-              const float2 x = p0[j2], y = p1[j2];
-              const float e0 = __fadd_rn(x.x, y.x), e1 = __fadd_rn(x.y, y.y);
-              hi[2 * j2] = tf32_hi(e0);
-              hi[2 * j2 + 1] = tf32_hi(e1);
-              lo[2 * j2] = __fsub_rn(e0, hi[2 * j2]);
-              lo[2 * j2 + 1] = __fsub_rn(e1, hi[2 * j2 + 1]);
-            }
-            tmem_st_hilo(aslot + (uint32_t)((wg + 4 * i) * 16), hi, lo);
+          for (int j2 = 0; j2 < 3; ++j2) {
+            const float2 x = p0[j2], y = p1[j2];
+            const float e0 = __fadd_rn(x.x, y.x), e1 = __fadd_rn(x.y, y.y);
+            hi[2 * j2] = tf32_hi(e0);
+            hi[2 * j2 + 1] = tf32_hi(e1);
+            lo[2 * j2] = __fsub_rn(e0, hi[2 * j2]);
+            lo[2 * j2 + 1] = __fsub_rn(e1, hi[2 * j2 + 1]);
           }
+          const int rr = q * 32 + lane;
+          unsigned char *eh = aop + (s % kDmASlots) * kDmSlotBytes + wg * kDmTileBytes;
+          unsigned char *el = eh + kDmTiles * kDmTileBytes;
+          float *fh = reinterpret_cast<float *>(eh), *fl = reinterpret_cast<float *>(el);
+          *reinterpret_cast<float4 *>(fh + opnd_idx(rr, 0)) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<float2 *>(fh + opnd_idx(rr, 4)) = make_float2(hi[4], hi[5]);
+          *reinterpret_cast<float4 *>(fl + opnd_idx(rr, 0)) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<float2 *>(fl + opnd_idx(rr, 4)) = make_float2(lo[4], lo[5]);
         }
-        tmem_wait_st();
-        tc_fence_before();
+        proxy_fence_async_smem();                 // generic stores -> tensor-core reads
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_at(kBarFull + (s & 1)));
-        // the chain before this one has had its last MMAs issued: read it out
-        if (m % kDmChain == 0 && m > 0) flush(p * NC + m / kDmChain - 1, acc, nt);
+        if (lane == 0) mbar_arrive(bar_at(kBarFull + s % kDmASlots));
       }
       if (to) break;
-      flush(p * NC + NC - 1, acc, nt);
-      if (to) break;
+      // the chains not read inside the loop, once the pass's last MMAs are done
+      {
+        const int sl = p * M + M - 1;
+        wait(kBarMma + sl % kDmASlots, (uint32_t)(sl / kDmASlots) & 1u);
+        if (to) break;
+        if (NC >= 2 && (NC - 1) * kDmChain + kDmASlots - 1 > M - 1) flush(p * NC + NC - 2, nt);
+        flush(p * NC + NC - 1, nt);
+      }
 
       // epilogue: softcap, logits, per-token best row of this warp
 #pragma unroll
       for (int tok = 0; tok < kDmTokens; ++tok) {
         ArgBest best{-FLT_MAX, INT_MAX};
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int r = (wg + 4 * i) * 128 + q * 32 + lane;
-          if (r < rows && tok < a.nb) {
-            const int64_t v = pr0 + r;
-            const float y = softcap_f(i == 0 ? acc[tok] : my[tok * 512], a.cap);
-            if (a.logits) a.logits[(int64_t)(a.t0 + tok) * a.V + v] = y;
-            best = arg_better(best, ArgBest{y, (int)v});
-          }
+        if (r < rows && tok < a.nb) {
+          const int64_t v = pr0 + r;
+          const float y = softcap_f(acc[tok], a.cap);
+          if (a.logits) a.logits[(int64_t)(a.t0 + tok) * a.V + v] = y;
+          best = ArgBest{y, (int)v};
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) best = arg_better(best, arg_shfl_xor(best, o));
@@ -485,8 +476,9 @@ __global__ void __launch_bounds__(kDmThreads, 1)
 size_t decode_mma_smem(int K, int N) {
   (void)N;
   const size_t cbs = (size_t)align_up(2 * K * 6, 256) * 4;
-  return 1024 + (size_t)kDmStages * kDmStageBytes + 2 * cbs + kDmHSlots * kDmHFloats * 4 +
-         (size_t)kDmTokens * kDmDecWarps * 32 * 4 + kBars * 8 + (size_t)kDmDecWarps * kDmTokens * sizeof(ArgBest) + 16;
+  return 1024 + (size_t)kDmASlots * kDmSlotBytes + (size_t)kDmStages * kDmStageBytes + 2 * cbs +
+         kDmHSlots * kDmHFloats * 4 + kBars * 8 + (size_t)kDmDecWarps * kDmTokens * sizeof(ArgBest) +
+         16;
 }
 
 size_t decode_mma_hop_bytes(int M) { return (size_t)M * kDmHFloats * 4; }

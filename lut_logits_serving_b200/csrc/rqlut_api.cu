@@ -198,7 +198,8 @@ int fused_group(int B) { return B <= 4 ? B : (B < kTokenGroup ? B : kTokenGroup)
 // code pass, softcap, logits/argmax, optionally the picked tokens' rows.
 int run_fused(const float *h, const float *C, const void *codes, int fmt, const rq_dims &d, int B,
               float softcap, float *logits, int32_t *argmax, void *ws, size_t ws_bytes,
-              const DecodeSpec *rows_spec, uint16_t *rows, cudaStream_t s) {
+              const DecodeSpec *rows_spec, uint16_t *rows, cudaStream_t s,
+              int path = RQ_PATH_AUTO) {
   DevInfo di;
   if (dev_info(&di) != cudaSuccess) return RQ_ERR_CUDA;
   const int G = fused_group(B);
@@ -219,23 +220,28 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   const int P = d.M * d.L;
   float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
   int *ami = argmax ? reinterpret_cast<int *>(rest + w.ami_off) : nullptr;
-  // Full 32-token groups decode rows into shared memory and multiply them
-  // with the hidden states (measured faster there); other groups read their
-  // tables through L2.  Both write argmax partials into the same [B][nblk].
+  // Full 32-token groups decode their rows and multiply them with the hidden
+  // states (the FP32 kernel by default: measured faster there than the
+  // tables and than the tensor-core kernel); other groups read their tables
+  // through L2.  All write argmax partials into the same [B][nblk].
   const int nblk = sweep_blocks(d, di, false);
   const bool dfma = decode_fma_applies(fmt, d.V, d.D, d.M, d.L, d.K, B, C, codes, di) &&
                     decode_fma_blocks(d.V, di) <= nblk;
+  const bool dtc = dfma && decode_mma_smem(d.K, kTokenGroup) <= (size_t)di.max_smem_optin &&
+                   decode_mma_hop_bytes(d.M) <= lut_bytes;
+  if ((path == RQ_PATH_DECODE_FP32 && !dfma) || (path == RQ_PATH_DECODE_TC && !dtc))
+    return RQ_ERR_UNSUPPORTED;
+  const bool decode = path != RQ_PATH_TABLES && dfma;
   cudaError_t e = cudaSuccess;
   bool marked = false;   // the profile start goes before the first logits kernel
   for (int b0 = 0; b0 < B && e == cudaSuccess; b0 += G) {
     const int nb = B - b0 < G ? B - b0 : G;
-    if (dfma && nb == kTokenGroup) {
+    if (decode && nb == kTokenGroup) {
       if (!marked && (e = prof_mark(t_prof_start, s)) != cudaSuccess) break;
       marked = true;
-      // the tensor-core path keeps the group's split hidden operand in the
+      // the tensor-core kernel keeps the group's split hidden operand in the
       // (here unused) table region
-      if (decode_mma_smem(d.K, kTokenGroup) <= (size_t)di.max_smem_optin &&
-          decode_mma_hop_bytes(d.M) <= lut_bytes)
+      if (path == RQ_PATH_DECODE_TC)
         e = launch_logits_decode_mma(h, C, codes, d.V, d.D, d.M, d.K, b0, nb, kTokenGroup, softcap,
                                      lut, logits, amv, ami, nblk, di, s);
       else
@@ -336,6 +342,14 @@ int rq_lut_logits(const void *codes, int fmt, rq_dims d, const float *lut, int B
 int rq_logits_from_hidden(const float *h, const float *C, const void *codes, int fmt, rq_dims d,
                           int B, float softcap, float *logits, int32_t *argmax, void *ws,
                           size_t ws_bytes, void *stream) {
+  return rq_logits_from_hidden_path(h, C, codes, fmt, d, B, softcap, logits, argmax, ws, ws_bytes,
+                                    RQ_PATH_AUTO, stream);
+}
+
+int rq_logits_from_hidden_path(const float *h, const float *C, const void *codes, int fmt,
+                               rq_dims d, int B, float softcap, float *logits, int32_t *argmax,
+                               void *ws, size_t ws_bytes, int path, void *stream) {
+  if (path < RQ_PATH_AUTO || path > RQ_PATH_DECODE_TC) return RQ_ERR_INVALID_ARGUMENT;
   if (!h || !C || !codes || B < 1 || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
   if (!logits && !argmax) return RQ_ERR_INVALID_ARGUMENT;
   if (!fmt_known(fmt)) return RQ_ERR_INVALID_ARGUMENT;
@@ -345,7 +359,7 @@ int rq_logits_from_hidden(const float *h, const float *C, const void *codes, int
       (logits && !aligned(logits, 4)) || (argmax && !aligned(argmax, 4)))
     return RQ_ERR_MISALIGNED;
   return run_fused(h, C, codes, fmt, d, B, softcap, logits, argmax, ws, ws_bytes, nullptr,
-                   nullptr, static_cast<cudaStream_t>(stream));
+                   nullptr, static_cast<cudaStream_t>(stream), path);
 }
 
 int rq_greedy_step(const float *h, const float *C, const void *codes, int fmt, rq_dims d, int B,

@@ -117,6 +117,8 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_lut_logits(odd, 0, G2, a, 1, 30.0, a, null, null, 0, s) == MIS
     assert lib.rq_lut_logits(a, 0, G2, odd, 1, 30.0, a, null, null, 0, s) == MIS
     assert lib.rq_logits_from_hidden(a, a, a, 0, G2, 1, 30.0, a, null, null, 0, s) == WS
+    assert lib.rq_logits_from_hidden_path(a, a, a, 0, G2, 1, 30.0, a, null, null, 0, 7, s) == INV
+    assert lib.rq_logits_from_hidden_path(a, a, a, 0, G2, 1, 30.0, a, null, null, 0, 3, s) == WS
     assert lib.rq_decode_rows(null, 5, a, 0, a, G2, 48.0, a, s) == INV
     assert lib.rq_decode_rows(a, -1, a, 0, a, G2, 48.0, a, s) == INV
     assert lib.rq_decode_rows(null, 0, null, 0, null, G2, 48.0, null, s) == 0   # N = 0: no-op

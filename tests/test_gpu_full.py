@@ -76,12 +76,15 @@ def test_g2_batch1_full_sweep(g2):
     assert rq.rq_device_error() == 0
 
 
-def _batched(g2, w, fmt, seed_rows):
+def _batched(g2, w, fmt, seed_rows, path=None):
     d = g2["d"]
     h = synth.hidden(w.B, w.D, w.hidden_scale, 2)
     codes_dev = g2["dc"] if fmt == rq.U16 else rq.rq_pack10(g2["dc"], d)
+    # NaN-filled output: a kernel that writes nothing cannot pass on stale memory
+    out = torch.full((w.B, w.V), float("nan"), device="cuda")
     logits, am, _ = rq.rq_logits_from_hidden(dev(h), g2["dC"], codes_dev, fmt, d, w.softcap,
-                                             want_argmax=True)
+                                             want_argmax=True, logits=out, path=path)
+    assert rq.rq_device_error() == 0
     got = logits.cpu().numpy()
     amv = am.cpu().numpy()
     T = oracle.lut_build(h, g2["C"], "f64")
@@ -97,11 +100,13 @@ def _batched(g2, w, fmt, seed_rows):
     return err, ties
 
 
-def test_g2_batch32_one_code_pass(g2):
+@pytest.mark.parametrize("path", [None, rq.PATH_TABLES, rq.PATH_DECODE_TC])
+def test_g2_batch32_one_code_pass(g2, path):
     w = synth.WORKLOADS["g2_b32"]
-    err, ties = _batched(g2, w, rq.U16, 7)
-    print(f"g2_b32 normwise error {err:.3g}, ties {ties}")
+    err, ties = _batched(g2, w, rq.U16, 7, path)
+    print(f"g2_b32 path {path} normwise error {err:.3g}, ties {ties}")
     assert ties == 0
+    assert rq.rq_device_error() == 0
 
 
 def test_g2_packed_batch64_fused_argmax(g2):

@@ -350,23 +350,48 @@ def test_greedy_step_rows_are_the_picked_tokens_rows(B, fmt):
     (3001, 16, 1024, 64),     # two full token groups
     (2500, 8, 256, 48),       # a full group (decoded) and a 16-token group (tables)
 ])
-def test_fused_decode_fma_path(V, M, K, B):
+@pytest.mark.parametrize("path", [None, rq.PATH_TABLES, rq.PATH_DECODE_FP32, rq.PATH_DECODE_TC])
+def test_fused_decode_paths(V, M, K, B, path):
     """Full 32-token groups with uint16 codes, ds = 6, L = 2, M % 8 == 0: the
-    fused call decodes rows into shared memory and multiplies them with the
-    hidden states (other groups use the tables); logits and argmax must meet
-    the same bounds, with both kinds of group in one call."""
+    fused call decodes rows (FP32 FMAs or tcgen05 MMAs) or reads tables, as
+    asked; groups of fewer tokens use the tables.  Logits and argmax meet the
+    same bounds on every path, with both kinds of group in one call."""
     D, L = 6 * M, 2
     C, codes, h = make_case(V, D, M, L, K, B, seed=V + B)
     d = rq.dims(V, D, M, L, K)
     ref = oracle_logits(C, codes, h, 30.0)
-    logits, am, _ = rq.rq_logits_from_hidden(dev(h), dev(C), dev(codes.reshape(V, -1)), rq.U16, d,
-                                             30.0, want_argmax=True)
+    args = (dev(h), dev(C), dev(codes.reshape(V, -1)), rq.U16, d, 30.0)
+    if path == rq.PATH_DECODE_TC and K < 8:
+        # the tensor-core kernel stages its hidden operand in the table region
+        with pytest.raises(rq.RqError, match="UNSUPPORTED"):
+            rq.rq_logits_from_hidden(*args, want_argmax=True, path=path)
+        return
+    out = torch.full((B, V), float("nan"), device="cuda")   # stale memory cannot pass
+    logits, am, _ = rq.rq_logits_from_hidden(*args, want_argmax=True, logits=out, path=path)
+    assert rq.rq_device_error() == 0
     assert_logits_close(logits.cpu().numpy(), ref)
     check_argmax(am.cpu().numpy(), ref)
-    assert rq.rq_device_error() == 0
 
 
-def test_fused_decode_fma_clamps_out_of_range_codes():
+def test_decode_paths_need_their_format():
+    """A decode path the format cannot take is refused, not silently replaced."""
+    V, M, K, B = 512, 8, 256, 32
+    C, codes, h = make_case(V, 6 * M, M, 2, K, B)
+    d = rq.dims(V, 6 * M, M, 2, K)
+    packed = rq.rq_pack10(dev(codes.reshape(V, -1)), d)
+    for path in (rq.PATH_DECODE_FP32, rq.PATH_DECODE_TC):
+        with pytest.raises(rq.RqError, match="UNSUPPORTED"):
+            rq.rq_logits_from_hidden(dev(h), dev(C), packed, rq.PACKED10, d, 30.0, path=path)
+    # the default and the tables serve it
+    ref = oracle_logits(C, codes, h, 30.0)
+    for path in (None, rq.PATH_TABLES):
+        logits, _, _ = rq.rq_logits_from_hidden(dev(h), dev(C), packed, rq.PACKED10, d, 30.0,
+                                                path=path)
+        assert_logits_close(logits.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("path", [rq.PATH_DECODE_FP32, rq.PATH_DECODE_TC])
+def test_fused_decode_clamps_out_of_range_codes(path):
     """Codes >= K read codeword K-1 (non-power-of-two K), as in the other paths."""
     V, M, K, B = 2000, 8, 100, 32
     C, codes, h = make_case(V, 6 * M, M, 2, K, B, seed=3)
@@ -375,7 +400,7 @@ def test_fused_decode_fma_clamps_out_of_range_codes():
     d = rq.dims(V, 6 * M, M, 2, K)
     ref = oracle_logits(C, np.minimum(bad, K - 1), h, 30.0)
     logits, _, _ = rq.rq_logits_from_hidden(dev(h), dev(C), dev(bad.reshape(V, -1)), rq.U16, d,
-                                            30.0)
+                                            30.0, path=path)
     assert_logits_close(logits.cpu().numpy(), ref)
 
 
