@@ -485,7 +485,12 @@ def run_ours(args, w):
     peak, peak_kind = load_peaks()
     algo_bytes = code_bytes(w, headline)
     achieved = algo_bytes / (kern_us / 1e6) / 1e9
-    kname = "logits_chunk_u16_kernel" if w.B <= 4 and not w.packed10 else "logits_l2_kernel"
+    # full 32-token groups of uint16 codes at ds = 6, L = 2 decode their rows
+    decodable = (w.ds == 6 and w.L == 2 and w.K <= 1024 and w.M % 8 == 0 and w.B >= 32
+                 and not w.packed10)
+    decoded = headline == "u16" and decodable
+    kname = ("logits_chunk_u16_kernel" if w.B <= 4 and not w.packed10 else
+             "logits_decode_fma_kernel" if decoded else "logits_l2_kernel")
     kkey = f"{kname}/{headline}/{w.name}"
 
     # ---- the other layout, same step (context for the headline)
@@ -502,6 +507,24 @@ def run_ours(args, w):
                         "code_pass_us": k2,
                         "code_pass_frac": code_bytes(w, name) / (k2 / 1e6) / 1e9 / peak}
         del g2
+
+    # ---- the kernel choices of full token groups (uint16 codes): logits and
+    # argmax of one rq_logits_from_hidden_path call per step
+    paths = {}
+    if decodable and "u16" in layouts:
+        pws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, rq.U16, True), dtype=torch.uint8,
+                          device="cuda")
+        for name, pth in (("tables", rq.PATH_TABLES), ("decode_fp32", rq.PATH_DECODE_FP32),
+                          ("decode_tc", rq.PATH_DECODE_TC)):
+            def pstep(pth=pth):
+                rq.rq_logits_from_hidden(dh0, dC, layouts["u16"][1], rq.U16, d, w.softcap,
+                                         logits=logits0, argmax=am0, ws=pws, path=pth)
+            rp, gp = graphed(pstep)
+            n3 = min(args.steps, 200)
+            t3 = time_steps(rp, n3)
+            paths[name] = {"us_per_call": t3 / n3 * 1e3,
+                           "code_pass_us": code_pass_us(pstep, min(n3, 50))}
+            del gp
     run, graph = graphed(step)
 
     # ---- end to end through the public API with host buffers: every step
@@ -598,7 +621,6 @@ def run_ours(args, w):
     else:
         # per 32-token group: rows decoded + multiplied (one kernel: full groups
         # of uint16 codes at ds = 6, L = 2) or table build + L2 pass (two)
-        decoded = (headline == "u16" and w.ds == 6 and w.L == 2 and w.K <= 1024 and w.M % 8 == 0)
         groups = [min(32, w.B - b0) for b0 in range(0, w.B, 32)]
         launches_per_step = sum(1 if decoded and g == 32 else 2 for g in groups)
         launches_per_step += 1 if w.argmax else 0
@@ -642,6 +664,7 @@ def run_ours(args, w):
                      "kernel_us": kern_us},
         "step_hbm_frac": algo_bytes / (sec / args.steps) / 1e9 / peak,
         "other_layouts": others,
+        "full_group_paths": paths or None,
         "topk_sample_us": topk_us,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
