@@ -490,7 +490,7 @@ def run_ours(args, w):
                  and not w.packed10)
     decoded = headline == "u16" and decodable
     kname = ("logits_chunk_u16_kernel" if w.B <= 4 and not w.packed10 else
-             "logits_decode_fma_kernel" if decoded else "logits_l2_kernel")
+             "logits_decode_mma_kernel" if decoded else "logits_l2_kernel")
     kkey = f"{kname}/{headline}/{w.name}"
 
     # ---- the other layout, same step (context for the headline)
@@ -619,10 +619,11 @@ def run_ours(args, w):
     if w.B <= 4 and not w.packed10:
         launches_per_step = 3 + (1 if w.argmax else 0)
     else:
-        # per 32-token group: rows decoded + multiplied (one kernel: full groups
-        # of uint16 codes at ds = 6, L = 2) or table build + L2 pass (two)
+        # per 32-token group: hidden split + rows decoded and multiplied on the
+        # tensor cores (full groups of uint16 codes at ds = 6, L = 2) or table
+        # build + L2 pass: two kernels either way
         groups = [min(32, w.B - b0) for b0 in range(0, w.B, 32)]
-        launches_per_step = sum(1 if decoded and g == 32 else 2 for g in groups)
+        launches_per_step = 2 * len(groups)
         launches_per_step += 1 if w.argmax else 0
     topk_us = None
     if w.topk:

@@ -187,7 +187,8 @@ RQ_API int rq_logits_from_hidden(const float *h, const float *C, const void *cod
  * the LUT section checks the lookup against) and contract it with the
  * group's hidden states; they need RQ_CODES_U16, L = 2, D = 6 M, M % 8 == 0,
  * K <= 1024 and 16-byte aligned C and codes.
- *   RQ_PATH_AUTO        -- RQ_PATH_DECODE_FP32 where it applies, else tables
+ *   RQ_PATH_AUTO        -- RQ_PATH_DECODE_TC where it applies, else
+ *                          RQ_PATH_DECODE_FP32 where that applies, else tables
  *   RQ_PATH_TABLES      -- per-group tables read through L2 (lookup + sum)
  *   RQ_PATH_DECODE_FP32 -- rows decoded into shared memory, fp32 FMAs
  *   RQ_PATH_DECODE_TC   -- rows decoded into shared memory, tcgen05 tf32

@@ -51,7 +51,7 @@ namespace {
 
 constexpr int kDmTokens = 32;
 constexpr int kDmDecWarps = 16;
-constexpr int kDmThreads = (kDmDecWarps + 1) * 32;   // + the control warp
+constexpr int kDmThreads = (kDmDecWarps + 2) * 32;   // + the MMA warp and the copy warp
 constexpr int kDmTiles = 4;                          // M = 128 tiles per pass
 constexpr int kDmRows = kDmTiles * 128;              // rows per pass
 constexpr int kDmGroup = 4;                          // subspaces per code stage (16 B per row)
@@ -59,19 +59,19 @@ constexpr int kDmStageBytes = kDmRows * kDmGroup * 4;   // 8 KB
 constexpr int kDmStages = 3;
 constexpr int kDmASlots = 2;                         // A slots: decoding runs 2 subspaces ahead
 constexpr int kDmChain = 16;                         // subspaces per accumulation chain
-constexpr int kDmTileBytes = 128 * 32;               // one M = 128, K = 8 tf32 operand
-constexpr int kDmSlotBytes = 2 * kDmTiles * kDmTileBytes;   // A slot: [E_hi tiles][E_lo tiles]
 constexpr int kDmHFloats = 512;                      // hidden operand: 64 rows x K = 8
 constexpr int kDmHSlots = 4;
-constexpr uint32_t kDmTmemCols = 512;                // 2 sets x 4 tiles x 64 columns
+constexpr uint32_t kDmTmemCols = 512;
+constexpr uint32_t kDmAcol = kDmTiles * 2 * kDmTokens;   // A slots after the 4 x 64 accumulator columns
+constexpr uint32_t kDmAslot = kDmTiles * 16;             // per slot: 4 tiles x (hi 8, lo 8) columns
 
 // mbarriers
 constexpr int kBarCodes = 0;                           // code stage g % 3 landed (TMA)
-constexpr int kBarBook = kBarCodes + kDmStages;        // 2: codebook + hidden operand (bulk)
+constexpr int kBarBook = kBarCodes + kDmStages;        // 2: codebook pair + hidden operand (bulk)
 constexpr int kBarFull = kBarBook + 2;                 // A slot s % 2 written (16 decoder warps)
 constexpr int kBarMma = kBarFull + kDmASlots;          // MMAs of subspace s done, on s % 2 (commit)
-constexpr int kBarFlush = kBarMma + kDmASlots;         // 2: chain c read out, on c & 1 (16 warps)
-constexpr int kBars = kBarFlush + 2;
+constexpr int kBarFlush = kBarMma + kDmASlots;         // a chain read out (16 warps)
+constexpr int kBars = kBarFlush + 1;
 
 struct DmArgs {
   const float *C;      // [M][2][K][6]
@@ -108,13 +108,13 @@ __device__ __forceinline__ uint32_t mma_idesc(int n) {
          ((uint32_t)(128 >> 4) << 24);
 }
 
-// D[tmem] (+)= A[smem] . B[smem]^T
-__device__ __forceinline__ void mma_tf32(uint32_t d, unsigned long long a, unsigned long long b,
-                                         uint32_t idesc, uint32_t accum) {
+// D[tmem] (+)= A[tmem] . B[smem]^T
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d, uint32_t a, unsigned long long b,
+                                            uint32_t idesc, uint32_t accum) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(accum));
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -151,6 +151,23 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// one row of an A slot in tensor memory: hi[0..5], 0, 0, lo[0..5], 0, 0
+__device__ __forceinline__ void tmem_st_hilo(uint32_t taddr, const float (&hi)[6],
+                                             const float (&lo)[6]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %7, %8, %9, %10, "
+      "%11, %12, %13, %7, %7};" ::"r"(taddr),
+      "r"(__float_as_uint(hi[0])), "r"(__float_as_uint(hi[1])), "r"(__float_as_uint(hi[2])),
+      "r"(__float_as_uint(hi[3])), "r"(__float_as_uint(hi[4])), "r"(__float_as_uint(hi[5])),
+      "r"(0u), "r"(__float_as_uint(lo[0])), "r"(__float_as_uint(lo[1])),
+      "r"(__float_as_uint(lo[2])), "r"(__float_as_uint(lo[3])), "r"(__float_as_uint(lo[4])),
+      "r"(__float_as_uint(lo[5])));
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // x rounded to nearest (ties to even) with the low 13 mantissa bits cleared
@@ -193,8 +210,7 @@ __global__ void __launch_bounds__(kDmThreads, 1)
   const int cbf = 2 * a.K * 6;                                     // floats per codebook pair
   const uint32_t cbb = (uint32_t)cbf * 4u;
   const size_t cbs = (size_t)align_up(cbf, 256);                   // floats per book buffer
-  unsigned char *aop = smem;                                       // A slots
-  unsigned char *st = aop + kDmASlots * kDmSlotBytes;              // code stages
+  unsigned char *st = smem;                                        // code stages
   float *cb = reinterpret_cast<float *>(st + kDmStages * kDmStageBytes);
   float *hs = cb + 2 * cbs;                                        // hidden operand slots
   uint64_t *bar = reinterpret_cast<uint64_t *>(hs + kDmHSlots * kDmHFloats);
@@ -207,22 +223,18 @@ __global__ void __launch_bounds__(kDmThreads, 1)
     prefetch_tmap(&tmap);
     for (int i = 0; i < kBars; ++i)
       mbar_init(smem_addr(&bar[i]),
-                ((i >= kBarFull && i < kBarFull + kDmASlots) || i == kBarFlush || i == kBarFlush + 1)
+                ((i >= kBarFull && i < kBarFull + kDmASlots) || i == kBarFlush)
                     ? (uint32_t)kDmDecWarps
                     : 1u);
     fence_mbar_init();
     *abort_flag = 0;
   }
-  // the K pads (dims 6, 7) of the A slots stay zero
-  for (int i = tid; i < kDmASlots * kDmSlotBytes / 16; i += kDmThreads)
-    reinterpret_cast<uint4 *>(aop)[i] = make_uint4(0, 0, 0, 0);
   if (warp == kDmDecWarps) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kDmTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  proxy_fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -236,14 +248,15 @@ __global__ void __launch_bounds__(kDmThreads, 1)
   const int NG = npass * G;                  // code groups
   auto bar_at = [&](int i) { return smem_addr(&bar[i]); };
 
-  if (warp == kDmDecWarps) {
-    // ------------------------------------------------------------ control
+  if (warp == kDmDecWarps + 1) {
+    // ------------------------------------------------------------ producer
+    // code tiles, codebooks and hidden operands; a buffer is refilled once
+    // the A slot of the step that read it is full (its decode is done, and
+    // the decoders had waited for the MMAs of two steps before)
     if (lane == 0 && S > 0) {
       const uint64_t pol_codes = l2_policy_evict_first();
-      const uint32_t id64 = mma_idesc(2 * kDmTokens), id32 = mma_idesc(kDmTokens);
-      int last_codes[kDmStages], last_book[2] = {-1, -1}, last_mma[kDmASlots];
+      int last_codes[kDmStages], last_book[2] = {-1, -1};
       for (int i = 0; i < kDmStages; ++i) last_codes[i] = -1;
-      for (int i = 0; i < kDmASlots; ++i) last_mma[i] = -1;
       bool to = false;
       auto wait = [&](int i, uint32_t parity) {
         if (!to && !mbar_try_wait(bar_at(i), parity) && !mbar_wait_bounded(bar_at(i), parity)) {
@@ -262,6 +275,8 @@ __global__ void __launch_bounds__(kDmThreads, 1)
                       (int)(r0 + (int64_t)p * kDmRows + q * 256), b, pol_codes);
         last_codes[sidx] = g;
       };
+      // the decoders wait for both before decoding s, so a full A slot of s
+      // also tells the MMA warp that the hidden operand of s has landed
       auto issue_book = [&](int s, int m) {
         const uint32_t b = bar_at(kBarBook + (s & 1));
         mbar_arrive_expect_tx(b, cbb + kDmHFloats * 4);
@@ -272,6 +287,46 @@ __global__ void __launch_bounds__(kDmThreads, 1)
       };
       for (int g = 0; g < NG && g < kDmStages; ++g) issue_codes(g);
       for (int s = 0; s < S && s < 2; ++s) issue_book(s, s % M);
+      int p = 0, m = 0;
+      for (int s = 0; s < S; ++s) {
+        if (*abort_flag) break;
+        wait(kBarFull + s % kDmASlots, (uint32_t)(s / kDmASlots) & 1u);   // decode of s done
+        if (to) break;
+        if (s + 2 < S) issue_book(s + 2, m + 2 < M ? m + 2 : m + 2 - M);
+        if (m % kDmGroup == kDmGroup - 1) {
+          const int g = p * G + m / kDmGroup;                  // its stage is read out
+          if (g + kDmStages < NG) issue_codes(g + kDmStages);
+        }
+        if (++m == M) {
+          m = 0;
+          ++p;
+        }
+      }
+      if (*abort_flag) {
+        // let the copies in flight land before the CTA's shared memory goes
+        for (int i = 0; i < kDmStages; ++i)
+          if (last_codes[i] >= 0)
+            mbar_wait_bounded(bar_at(kBarCodes + i), (uint32_t)(last_codes[i] / kDmStages) & 1u);
+        for (int i = 0; i < 2; ++i)
+          if (last_book[i] >= 0)
+            mbar_wait_bounded(bar_at(kBarBook + i), (uint32_t)(last_book[i] >> 1) & 1u);
+        atomicOr(a.err, RQ_DEVERR_TIMEOUT);
+      }
+    }
+  } else if (warp == kDmDecWarps) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0 && S > 0) {
+      const uint32_t id64 = mma_idesc(2 * kDmTokens), id32 = mma_idesc(kDmTokens);
+      int issued = 0;                          // steps whose MMAs are committed
+      bool to = false;
+      auto wait = [&](int i, uint32_t parity) {
+        if (!to && !mbar_try_wait(bar_at(i), parity) && !mbar_wait_bounded(bar_at(i), parity)) {
+          to = true;
+          *abort_flag = 1;
+        }
+      };
+      // descriptor of hidden slot i: the start field counts 16-byte units
+      const unsigned long long bd0 = opnd_desc(smem_addr(hs));
       int p = 0, m = 0, nt = 0;
       for (int s = 0; s < S; ++s) {
         if (m == 0) {
@@ -279,54 +334,38 @@ __global__ void __launch_bounds__(kDmThreads, 1)
           nt = (int)(((rows < kDmRows ? rows : kDmRows) + 127) / 128);
         }
         if (*abort_flag) break;
-        wait(kBarFull + s % kDmASlots, (uint32_t)(s / kDmASlots) & 1u);   // A slot of s written
-        wait(kBarBook + (s & 1), (uint32_t)(s >> 1) & 1u);   // hidden operand of s landed
-        if (s + 2 < S) {
-          // the book buffer of s is read out (its decode is done); the hidden
-          // slot of s + 2 was last read by the MMAs of s - 2 (waited for
-          // before the commit of s, which lands on the same barrier)
-          if (s >= 2) wait(kBarMma + (s - 2) % kDmASlots, (uint32_t)((s - 2) / kDmASlots) & 1u);
-          if (to) break;
-          issue_book(s + 2, m + 2 < M ? m + 2 : m + 2 - M);
-        }
-        if (m % kDmGroup == kDmGroup - 1) {
-          const int g = p * G + m / kDmGroup;                  // its stage is read out
-          if (g + kDmStages < NG) issue_codes(g + kDmStages);
-        }
+        // A slot of s written (and, as the decoders waited for it, the hidden
+        // operand of s landed)
+        wait(kBarFull + s % kDmASlots, (uint32_t)(s / kDmASlots) & 1u);
         const int c = p * NC + m / kDmChain;
         const bool first = m % kDmChain == 0;
-        // chain c - 2 (same set) is read out; one barrier per set, as the
-        // decoders may finish reading chain c - 1 before this wait
-        if (first && c >= 2) wait(kBarFlush + (c & 1), (uint32_t)((c - 2) >> 1) & 1u);
+        // one accumulator set: the previous chain is read out before this one
+        // starts over it
+        if (first && c >= 1) wait(kBarFlush, (uint32_t)(c - 1) & 1u);
         if (to) break;
         tc_fence_after();
-        const uint32_t hb = smem_addr(hs + (s & 3) * kDmHFloats);
-        const unsigned long long bd = opnd_desc(hb);
-        const uint32_t slot = smem_addr(aop + (s % kDmASlots) * kDmSlotBytes);
-        const uint32_t set = tmem + (uint32_t)(c & 1) * (kDmTiles * 2 * kDmTokens);
-        for (int t = 0; t < nt; ++t) {
-          const uint32_t d = set + (uint32_t)(t * 2 * kDmTokens);
-          mma_tf32(d, opnd_desc(slot + t * kDmTileBytes), bd, id64, first ? 0u : 1u);
-          mma_tf32(d, opnd_desc(slot + (kDmTiles + t) * kDmTileBytes), bd, id32, 1u);
+        const uint32_t slot = tmem + kDmAcol + (uint32_t)(s % kDmASlots) * kDmAslot;
+        const unsigned long long b = bd0 + (unsigned long long)((s & 3) * (kDmHFloats * 4 / 16));
+#pragma unroll
+        for (int t = 0; t < kDmTiles; ++t) {
+          if (t < nt) {
+            const uint32_t d = tmem + (uint32_t)(t * 2 * kDmTokens);
+            const uint32_t ah = slot + (uint32_t)(t * 16);
+            mma_tf32_ts(d, ah, b, id64, first ? 0u : 1u);
+            mma_tf32_ts(d, ah + 8u, b, id32, 1u);
+          }
         }
         mma_commit(bar_at(kBarMma + s % kDmASlots));
-        last_mma[s % kDmASlots] = s;
+        issued = s + 1;
         if (++m == M) {
           m = 0;
           ++p;
         }
       }
       if (*abort_flag) {
-        // let the copies and MMAs in flight land before the CTA's resources go
-        for (int i = 0; i < kDmStages; ++i)
-          if (last_codes[i] >= 0)
-            mbar_wait_bounded(bar_at(kBarCodes + i), (uint32_t)(last_codes[i] / kDmStages) & 1u);
-        for (int i = 0; i < 2; ++i)
-          if (last_book[i] >= 0)
-            mbar_wait_bounded(bar_at(kBarBook + i), (uint32_t)(last_book[i] >> 1) & 1u);
-        for (int i = 0; i < kDmASlots; ++i)
-          if (last_mma[i] >= 0)
-            mbar_wait_bounded(bar_at(kBarMma + i), (uint32_t)(last_mma[i] / kDmASlots) & 1u);
+        // let the MMAs in flight finish before the CTA's tensor memory goes
+        for (int s = issued - kDmASlots; s < issued; ++s)
+          if (s >= 0) mbar_wait_bounded(bar_at(kBarMma + s % kDmASlots), (uint32_t)(s / kDmASlots) & 1u);
         atomicOr(a.err, RQ_DEVERR_TIMEOUT);
       }
     }
@@ -351,8 +390,7 @@ __global__ void __launch_bounds__(kDmThreads, 1)
     auto flush = [&](int c, int nt) {
       if (wg < nt) {
         tc_fence_after();
-        const uint32_t base = tmem + lane_base +
-                              (uint32_t)((c & 1) * (kDmTiles * 2 * kDmTokens) + wg * 2 * kDmTokens);
+        const uint32_t base = tmem + lane_base + (uint32_t)(wg * 2 * kDmTokens);
         uint32_t x[16], y[16];
 #pragma unroll
         for (int c0 = 0; c0 < kDmTokens; c0 += 16) {
@@ -367,7 +405,7 @@ __global__ void __launch_bounds__(kDmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_at(kBarFlush + (c & 1)));
+      if (lane == 0) mbar_arrive(bar_at(kBarFlush));
     };
 
     for (int p = 0; p < npass && !to; ++p) {
@@ -393,8 +431,10 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         if (s >= kDmASlots)                                     // A slot free
           wait(kBarMma + s % kDmASlots, (uint32_t)((s - kDmASlots) / kDmASlots) & 1u);
         if (to) break;
-        // the MMAs of s - 3, the last of the previous chain, are done: read it out
-        if (m % kDmChain == kDmASlots - 1 && m > kDmChain) flush(p * NC + m / kDmChain - 1, nt);
+        // the MMAs of s - 2, the last of the previous chain, are done (waited
+        // for above): read it out before the next chain starts over it
+        if (m % kDmChain == 1 && m > kDmChain) flush(p * NC + m / kDmChain - 1, nt);
+        tc_fence_after();
         if (wg < nt) {
           const float *book = cb + (size_t)(s & 1) * cbs;
           const uint32_t w = i4 == 0 ? cw.x : i4 == 1 ? cw.y : i4 == 2 ? cw.z : cw.w;
@@ -410,16 +450,12 @@ __global__ void __launch_bounds__(kDmThreads, 1)
             lo[2 * j2] = __fsub_rn(e0, hi[2 * j2]);
             lo[2 * j2 + 1] = __fsub_rn(e1, hi[2 * j2 + 1]);
           }
-          const int rr = q * 32 + lane;
-          unsigned char *eh = aop + (s % kDmASlots) * kDmSlotBytes + wg * kDmTileBytes;
-          unsigned char *el = eh + kDmTiles * kDmTileBytes;
-          float *fh = reinterpret_cast<float *>(eh), *fl = reinterpret_cast<float *>(el);
-          *reinterpret_cast<float4 *>(fh + opnd_idx(rr, 0)) = make_float4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<float2 *>(fh + opnd_idx(rr, 4)) = make_float2(hi[4], hi[5]);
-          *reinterpret_cast<float4 *>(fl + opnd_idx(rr, 0)) = make_float4(lo[0], lo[1], lo[2], lo[3]);
-          *reinterpret_cast<float2 *>(fl + opnd_idx(rr, 4)) = make_float2(lo[4], lo[5]);
+          tmem_st_hilo(tmem + lane_base + kDmAcol + (uint32_t)(s % kDmASlots) * kDmAslot +
+                           (uint32_t)(wg * 16),
+                       hi, lo);
+          tmem_wait_st();
         }
-        proxy_fence_async_smem();                 // generic stores -> tensor-core reads
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_at(kBarFull + s % kDmASlots));
       }
@@ -429,7 +465,7 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         const int sl = p * M + M - 1;
         wait(kBarMma + sl % kDmASlots, (uint32_t)(sl / kDmASlots) & 1u);
         if (to) break;
-        if (NC >= 2 && (NC - 1) * kDmChain + kDmASlots - 1 > M - 1) flush(p * NC + NC - 2, nt);
+        if (NC >= 2 && (NC - 1) * kDmChain + 1 > M - 1) flush(p * NC + NC - 2, nt);
         flush(p * NC + NC - 1, nt);
       }
 
@@ -476,7 +512,7 @@ __global__ void __launch_bounds__(kDmThreads, 1)
 size_t decode_mma_smem(int K, int N) {
   (void)N;
   const size_t cbs = (size_t)align_up(2 * K * 6, 256) * 4;
-  return 1024 + (size_t)kDmASlots * kDmSlotBytes + (size_t)kDmStages * kDmStageBytes + 2 * cbs +
+  return 1024 + (size_t)kDmStages * kDmStageBytes + 2 * cbs +
          kDmHSlots * kDmHFloats * 4 + kBars * 8 + (size_t)kDmDecWarps * kDmTokens * sizeof(ArgBest) +
          16;
 }

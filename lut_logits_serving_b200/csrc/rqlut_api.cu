@@ -221,9 +221,9 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
   int *ami = argmax ? reinterpret_cast<int *>(rest + w.ami_off) : nullptr;
   // Full 32-token groups decode their rows and multiply them with the hidden
-  // states (the FP32 kernel by default: measured faster there than the
-  // tables and than the tensor-core kernel); other groups read their tables
-  // through L2.  All write argmax partials into the same [B][nblk].
+  // states (on the tensor cores by default, measured fastest there, else the
+  // FP32 kernel); other groups read their tables through L2.  All write
+  // argmax partials into the same [B][nblk].
   const int nblk = sweep_blocks(d, di, false);
   const bool dfma = decode_fma_applies(fmt, d.V, d.D, d.M, d.L, d.K, B, C, codes, di) &&
                     decode_fma_blocks(d.V, di) <= nblk;
@@ -241,7 +241,7 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
       marked = true;
       // the tensor-core kernel keeps the group's split hidden operand in the
       // (here unused) table region
-      if (path == RQ_PATH_DECODE_TC)
+      if (path == RQ_PATH_DECODE_TC || (path == RQ_PATH_AUTO && dtc))
         e = launch_logits_decode_mma(h, C, codes, d.V, d.D, d.M, d.K, b0, nb, kTokenGroup, softcap,
                                      lut, logits, amv, ami, nblk, di, s);
       else

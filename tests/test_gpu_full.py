@@ -100,7 +100,7 @@ def _batched(g2, w, fmt, seed_rows, path=None):
     return err, ties
 
 
-@pytest.mark.parametrize("path", [None, rq.PATH_TABLES, rq.PATH_DECODE_TC])
+@pytest.mark.parametrize("path", [None, rq.PATH_TABLES, rq.PATH_DECODE_FP32, rq.PATH_DECODE_TC])
 def test_g2_batch32_one_code_pass(g2, path):
     w = synth.WORKLOADS["g2_b32"]
     err, ties = _batched(g2, w, rq.U16, 7, path)
