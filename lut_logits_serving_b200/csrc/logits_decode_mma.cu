@@ -1,5 +1,5 @@
 // logits_decode_mma.cu -- logits of a token group by decoding vocabulary rows
-// into shared memory and multiplying them with the hidden states on the
+// into tensor memory and multiplying them with the hidden states on the
 // tcgen05 tensor cores.
 //
 // "Gemma-2 runtime compression: NF4 + LUT serving", LUT section: the lookup
@@ -18,10 +18,10 @@
 // what an N = 32 one does), and E_lo against h_hi into the first 32.  The
 // tensor core's fp32 accumulation does not round to nearest and its error
 // grows with the length of an accumulation chain, so a chain covers 16
-// subspaces in one of two TMEM accumulator sets; the threads that own a
-// finished chain's rows add it into fp32 registers (round to nearest) while
-// the next chain runs in the other set.  Measured against fp64 this keeps the
-// logits near 1e-6 of their scale; one chain over all 384 subspaces was ~3e-5.
+// subspaces; the threads that own a finished chain's rows add it into fp32
+// registers (round to nearest) before the next chain starts over it.
+// Measured against fp64 this keeps the logits near 1e-6 of their scale; one
+// chain over all 384 subspaces was ~3e-5.
 //
 // Design for sm_100a (ds = 6, L = 2, uint16 codes, K <= 1024, 32 tokens).
 // One CTA per SM walks an even share of the vocabulary in passes of up to
@@ -30,16 +30,20 @@
 //   * 16 decoder warps (4 warpgroups).  Thread (warpgroup g, warp q, lane)
 //     owns row 32 q + lane of tile g.  Per subspace it gathers the row's two
 //     codewords from the shared-memory codebook, adds them, splits the sum
-//     into hi and lo and stores both as one K = 8 row (6 dims, 2 zero pads)
-//     of the canonical K-major operand layout into a double-buffered A slot;
-//   * one control warp: one lane issues the TMA code tiles ({8 codes, 256
-//     rows}, 3 stages of 4 subspaces), one bulk copy per subspace of the
-//     codebook pair (48 KB at K = 1024, double-buffered) plus the pre-split
-//     hidden operand (2 KB, 4-slot ring), and the 2 x 4 MMAs per subspace;
-//   * TMEM: two accumulator sets of 4 tiles x 64 columns, 512 columns.
+//     into hi and lo and stores both (6 dims + 2 zero pads each) into its own
+//     TMEM lane of a double-buffered A slot with one tcgen05.st: the MMA reads
+//     its A operand from tensor memory;
+//   * one copy warp: TMA code tiles ({8 codes, 256 rows}, 3 stages of 4
+//     subspaces), and per subspace one bulk copy of the codebook pair (48 KB
+//     at K = 1024, double-buffered) plus the pre-split hidden operand (2 KB,
+//     4-slot ring) on the same barrier, which the decoders wait for;
+//   * one MMA warp: per subspace it waits for the A slot alone and issues the
+//     2 x 4 MMAs (M = 128, K = 8; A in TMEM, B in shared memory).  Issuing
+//     small MMAs costs ~100 cycles each, so nothing else sits on this warp.
+//   * TMEM: 4 tiles x 64 accumulator columns, then 2 A slots x 4 tiles x 16.
 // Every wait is bounded; a timed-out wait raises a CTA-wide abort flag, the
-// control lane waits (bounded) for its copies and MMAs in flight, and the CTA
-// frees its TMEM and ends.
+// copy and MMA warps wait (bounded) for their copies and MMAs in flight, and
+// the CTA frees its TMEM and ends.
 #include <cfloat>
 #include <climits>
 
@@ -133,10 +137,6 @@ __device__ __forceinline__ void tc_fence_after() {
 
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void proxy_fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
