@@ -290,9 +290,12 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel="logits_chunk"):
+    """Hash of the sources a kernel is built from (its .cu file and the common
+    header), to tell whether committed ncu counters still describe it."""
+    src = "logits_decode_mma.cu" if kernel.startswith("logits_decode_mma") else "logits_chunk.cu"
     h = hashlib.sha256()
-    for name in ("logits_chunk.cu", "rq_common.cuh"):
+    for name in (src, "rq_common.cuh"):
         with open(os.path.join(ROOT, "lut_logits_serving_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -307,7 +310,7 @@ def profiled_traffic(kernel):
     with open(p) as f:
         j = json.load(f)
     e = j.get(kernel)
-    if not e or e.get("source_sha") != kernel_source_hash():
+    if not e or e.get("source_sha") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
