@@ -8,7 +8,9 @@ names:
 
 * ``rq_lut_build``  -- per-token tables T[p][k][b] = <h_b[m], C[m][l][k]>
 * ``rq_lut_logits`` -- z[b][v] = sum_p T[p][code[v][p]][b], softcap, argmax
-* ``rq_logits_from_hidden`` -- both, large batches in L2-sized token groups
+* ``rq_logits_from_hidden`` -- both, large batches in token groups of 32;
+  a full group's rows are decoded and multiplied on the tensor cores
+  (``rq_logits_from_hidden_path`` picks tables, FP32 or tensor cores)
 * ``rq_decode_rows`` -- bf16 input rows rebuilt on demand
 * ``rq_pack10`` -- uint16 codes -> 10-bit packed rows
 
