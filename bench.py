@@ -50,10 +50,12 @@ def parse():
     ap.add_argument("--workload", default="g2_b1",
                     choices=["g2_b1", "g2_b32", "packed_b64", "mlp_gate_b1", "mlp_down_b1",
                              "encode_g2", "g2_b1_topk50"])
-    ap.add_argument("--codes", default="sched", choices=["u16", "sched", "u8"],
-                    help="uint16 code layout of the unpacked workloads timed for `value`: "
-                         "bank-scheduled once by rq_prepare_sched (the serving layout), or as "
-                         "drawn; the other layout is reported under other_layouts")
+    ap.add_argument("--codes", default=None, choices=["u16", "sched", "u8"],
+                    help="code layout of the unpacked workloads timed for `value`: "
+                         "bank-scheduled once by rq_prepare_sched (the default at B <= 4), as "
+                         "drawn (the default for batches, whose full token groups decode rows "
+                         "on the tensor cores), or one byte per code; the other layouts are "
+                         "reported under other_layouts")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -374,7 +376,8 @@ def run_ours(args, w):
         layouts["u16"] = (rq.U16, c16, None)
         if w.K <= 256:                 # one byte per code
             layouts["u8"] = (rq.U8, rq.rq_pack8(c16, d), None)
-        headline = args.codes if args.codes in layouts else "sched"
+        default = "sched" if w.B <= 4 else "u16"
+        headline = args.codes if args.codes in layouts else default
 
     def make_step(fmt, codes, out=None):
         ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
@@ -488,10 +491,11 @@ def run_ours(args, w):
     peak, peak_kind = load_peaks()
     algo_bytes = code_bytes(w, headline)
     achieved = algo_bytes / (kern_us / 1e6) / 1e9
-    # full 32-token groups of uint16 codes at ds = 6, L = 2 decode their rows
-    decodable = (w.ds == 6 and w.L == 2 and w.K <= 1024 and w.M % 8 == 0 and w.B >= 32
-                 and not w.packed10)
-    decoded = headline == "u16" and decodable
+    # full token groups (64, then 32) of uint16 or 10-bit packed codes at
+    # ds = 6, L = 2 decode their rows on the tensor cores
+    decodable = (w.ds == 6 and w.L == 2 and 16 <= w.K <= 1024 and w.B >= 32 and
+                 w.M % (32 if w.packed10 else 8) == 0)
+    decoded = headline in ("u16", "packed10") and decodable
     kname = ("logits_chunk_u16_kernel" if w.B <= 4 and not w.packed10 else
              "logits_decode_mma_kernel" if decoded else "logits_l2_kernel")
     kkey = f"{kname}/{headline}/{w.name}"
@@ -514,13 +518,16 @@ def run_ours(args, w):
     # ---- the kernel choices of full token groups (uint16 codes): logits and
     # argmax of one rq_logits_from_hidden_path call per step
     paths = {}
-    if decodable and "u16" in layouts:
-        pws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, rq.U16, True), dtype=torch.uint8,
+    if decodable and headline in ("u16", "packed10"):
+        pf, pc = layouts[headline][0], layouts[headline][1]
+        pws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, pf, True), dtype=torch.uint8,
                           device="cuda")
-        for name, pth in (("tables", rq.PATH_TABLES), ("decode_fp32", rq.PATH_DECODE_FP32),
-                          ("decode_tc", rq.PATH_DECODE_TC)):
+        choices = [("tables", rq.PATH_TABLES), ("decode_tc", rq.PATH_DECODE_TC)]
+        if headline == "u16":
+            choices.insert(1, ("decode_fp32", rq.PATH_DECODE_FP32))
+        for name, pth in choices:
             def pstep(pth=pth):
-                rq.rq_logits_from_hidden(dh0, dC, layouts["u16"][1], rq.U16, d, w.softcap,
+                rq.rq_logits_from_hidden(dh0, dC, pc, pf, d, w.softcap,
                                          logits=logits0, argmax=am0, ws=pws, path=pth)
             rp, gp = graphed(pstep)
             n3 = min(args.steps, 200)
@@ -622,10 +629,15 @@ def run_ours(args, w):
     if w.B <= 4 and not w.packed10:
         launches_per_step = 3 + (1 if w.argmax else 0)
     else:
-        # per 32-token group: hidden split + rows decoded and multiplied on the
-        # tensor cores (full groups of uint16 codes at ds = 6, L = 2) or table
-        # build + L2 pass: two kernels either way
-        groups = [min(32, w.B - b0) for b0 in range(0, w.B, 32)]
+        # per token group: hidden split + rows decoded and multiplied on the
+        # tensor cores (full groups of 64, then 32) or table build + L2 pass
+        # (groups of up to 32): two kernels either way
+        groups, b0 = [], 0
+        while b0 < w.B:
+            g = 64 if decoded and w.B - b0 >= 64 else 32 if decoded and w.B - b0 >= 32 else \
+                min(32, w.B - b0)
+            groups.append(g)
+            b0 += g
         launches_per_step = 2 * len(groups)
         launches_per_step += 1 if w.argmax else 0
     topk_us = None

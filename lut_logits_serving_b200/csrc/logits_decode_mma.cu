@@ -53,33 +53,40 @@ namespace rq {
 
 namespace {
 
-constexpr int kDmTokens = 32;
-constexpr int kDmDecWarps = 16;
-constexpr int kDmThreads = (kDmDecWarps + 2) * 32;   // + the MMA warp and the copy warp
-constexpr int kDmTiles = 4;                          // M = 128 tiles per pass
-constexpr int kDmRows = kDmTiles * 128;              // rows per pass
-constexpr int kDmGroup = 4;                          // subspaces per code stage (16 B per row)
-constexpr int kDmStageBytes = kDmRows * kDmGroup * 4;   // 8 KB
-constexpr int kDmStages = 3;
+// Shape of one instance: NT tokens per group, FMT the code format.
+//   NT = 32: 16 decoder warps, 4 tiles (512 rows) per pass, 32 register sums;
+//   NT = 64: 12 decoder warps, 3 tiles (384 rows), 64 register sums (14 warps
+//            leave 128 registers a thread, where 18 leave 96).
+//   uint16 codes: stages of 4 subspaces, 16 bytes per row (TMA {8 codes,
+//   128 rows}); 10-bit packed codes: stages of 32 subspaces, 80 bytes per
+//   row (TMA boxes of {40 16-bit units, 128 rows} over the 960-byte rows).
+template <int NT, int FMT>
+struct DmShape {
+  static constexpr int DEC_WARPS = NT == 32 ? 16 : 12;
+  static constexpr int THREADS = (DEC_WARPS + 2) * 32;   // + the MMA warp and the copy warp
+  static constexpr int TILES = DEC_WARPS / 4;              // M = 128 tiles per pass
+  static constexpr int ROWS = TILES * 128;                 // rows per pass
+  static constexpr bool PACKED = FMT == RQ_CODES_PACKED10;
+  static constexpr int GROUP = PACKED ? 32 : 4;            // subspaces per code stage
+  static constexpr int ROW_BYTES = PACKED ? 80 : 16;       // code bytes per row and stage
+  static constexpr int STAGE_BYTES = ROWS * ROW_BYTES;
+  static constexpr int STAGES = PACKED ? 2 : 3;
+  static constexpr int BOX_INNER = ROW_BYTES / 2;          // TMA box inner extent (16-bit units)
+  static constexpr int HFLOATS = 2 * NT * 8;               // hidden operand: [h_hi | h_lo] x K = 8
+  static constexpr uint32_t ACC = 2 * NT;                  // accumulator columns per tile
+  static constexpr uint32_t ACOL = TILES * ACC;            // first A-slot column
+  static constexpr uint32_t ASLOT = TILES * 16;            // per slot: tiles x (hi 8, lo 8)
+  static_assert(ACOL + 2 * ASLOT <= 512, "tensor memory");
+};
+
 constexpr int kDmASlots = 2;                         // A slots: decoding runs 2 subspaces ahead
 constexpr int kDmChain = 16;                         // subspaces per accumulation chain
-constexpr int kDmHFloats = 512;                      // hidden operand: 64 rows x K = 8
 constexpr int kDmHSlots = 4;
 constexpr uint32_t kDmTmemCols = 512;
-constexpr uint32_t kDmAcol = kDmTiles * 2 * kDmTokens;   // A slots after the 4 x 64 accumulator columns
-constexpr uint32_t kDmAslot = kDmTiles * 16;             // per slot: 4 tiles x (hi 8, lo 8) columns
-
-// mbarriers
-constexpr int kBarCodes = 0;                           // code stage g % 3 landed (TMA)
-constexpr int kBarBook = kBarCodes + kDmStages;        // 2: codebook pair + hidden operand (bulk)
-constexpr int kBarFull = kBarBook + 2;                 // A slot s % 2 written (16 decoder warps)
-constexpr int kBarMma = kBarFull + kDmASlots;          // MMAs of subspace s done, on s % 2 (commit)
-constexpr int kBarFlush = kBarMma + kDmASlots;         // a chain read out (16 warps)
-constexpr int kBars = kBarFlush + 1;
 
 struct DmArgs {
   const float *C;      // [M][2][K][6]
-  const float *hop;    // [M][512]: per subspace rows 0..31 h_hi, 32..63 h_lo
+  const float *hop;    // [M][2 NT][8]: per subspace rows 0..NT-1 h_hi, NT..2NT-1 h_lo
   int64_t V;
   int M, K;
   int t0, nb;          // tokens t0 .. t0 + nb - 1
@@ -185,37 +192,55 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 }  // namespace
 
-// Hidden operand of one token group, per subspace m: 64 rows of K = 8 in the
-// canonical K-major layout, rows 0..31 the tokens' hi parts and rows 32..63
+// Hidden operand of one token group, per subspace m: 2 NT rows of K = 8 in the
+// canonical K-major layout, rows 0..NT-1 the tokens' hi parts and NT..2NT-1
 // their lo parts (dims 6, 7 and tokens past the group are zero).
-__global__ void __launch_bounds__(256) split_hidden_kernel(const float *__restrict__ h, int D,
-                                                           int t0, int nb,
-                                                           float *__restrict__ hop) {
+template <int NT>
+__global__ void __launch_bounds__(NT * 8) split_hidden_kernel(const float *__restrict__ h, int D,
+                                                              int t0, int nb,
+                                                              float *__restrict__ hop) {
   griddep_wait();
   const int m = blockIdx.x, tok = threadIdx.x >> 3, k = threadIdx.x & 7;
   const float x = (k < 6 && tok < nb) ? h[(int64_t)(t0 + tok) * D + m * 6 + k] : 0.f;
   const float xh = tf32_hi(x);
-  float *o = hop + (size_t)m * kDmHFloats;
+  float *o = hop + (size_t)m * (2 * NT * 8);
   o[opnd_idx(tok, k)] = xh;
-  o[opnd_idx(32 + tok, k)] = __fsub_rn(x, xh);
+  o[opnd_idx(NT + tok, k)] = __fsub_rn(x, xh);
   griddep_launch_dependents();
 }
 
-__global__ void __launch_bounds__(kDmThreads, 1)
+template <int NT, int FMT>
+__global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
     logits_decode_mma_kernel(const __grid_constant__ CUtensorMap tmap, const DmArgs a) {
+  using S_ = DmShape<NT, FMT>;
+  constexpr int DW = S_::DEC_WARPS;
+  // mbarriers
+  constexpr int kBarCodes = 0;                         // code stage g % STAGES landed (TMA)
+  constexpr int kBarBook = kBarCodes + S_::STAGES;     // 2: codebook pair + hidden operand (bulk)
+  constexpr int kBarFull = kBarBook + 2;               // A slot s % 2 written (decoder warps)
+  constexpr int kBarMma = kBarFull + kDmASlots;        // MMAs of subspace s done, on s % 2 (commit)
+  constexpr int kBarFlush = kBarMma + kDmASlots;       // a chain read out (decoder warps)
+  constexpr int kBars = kBarFlush + 1;
+
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int cbf = 2 * a.K * 6;                                     // floats per codebook pair
   const uint32_t cbb = (uint32_t)cbf * 4u;
   const size_t cbs = (size_t)align_up(cbf, 256);                   // floats per book buffer
   unsigned char *st = smem;                                        // code stages
-  float *cb = reinterpret_cast<float *>(st + kDmStages * kDmStageBytes);
+  float *cb = reinterpret_cast<float *>(st + S_::STAGES * S_::STAGE_BYTES);
   float *hs = cb + 2 * cbs;                                        // hidden operand slots
-  uint64_t *bar = reinterpret_cast<uint64_t *>(hs + kDmHSlots * kDmHFloats);
-  ArgBest *wbest = reinterpret_cast<ArgBest *>(bar + kBars);      // [16 warps][32]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(wbest + kDmDecWarps * kDmTokens);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(hs + kDmHSlots * S_::HFLOATS);
+  ArgBest *wbest = reinterpret_cast<ArgBest *>(bar + kBars);      // [decoder warps][NT]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(wbest + DW * NT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -223,13 +248,12 @@ __global__ void __launch_bounds__(kDmThreads, 1)
     prefetch_tmap(&tmap);
     for (int i = 0; i < kBars; ++i)
       mbar_init(smem_addr(&bar[i]),
-                ((i >= kBarFull && i < kBarFull + kDmASlots) || i == kBarFlush)
-                    ? (uint32_t)kDmDecWarps
-                    : 1u);
+                ((i >= kBarFull && i < kBarFull + kDmASlots) || i == kBarFlush) ? (uint32_t)DW
+                                                                                : 1u);
     fence_mbar_init();
     *abort_flag = 0;
   }
-  if (warp == kDmDecWarps) {
+  if (warp == DW) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kDmTmemCols));
@@ -241,22 +265,22 @@ __global__ void __launch_bounds__(kDmThreads, 1)
   const uint32_t tmem = *tmem_slot;
   griddep_wait();
 
-  const int M = a.M, G = a.M / kDmGroup, NC = (a.M + kDmChain - 1) / kDmChain;
+  const int M = a.M, G = a.M / S_::GROUP, NC = (a.M + kDmChain - 1) / kDmChain;
   const int64_t r0 = a.V * blockIdx.x / gridDim.x, r1 = a.V * (blockIdx.x + 1) / gridDim.x;
-  const int npass = (int)((r1 - r0 + kDmRows - 1) / kDmRows);   // full passes, then the rest
+  const int npass = (int)((r1 - r0 + S_::ROWS - 1) / S_::ROWS);   // full passes, then the rest
   const int S = npass * M;                   // steps: (pass, subspace)
   const int NG = npass * G;                  // code groups
   auto bar_at = [&](int i) { return smem_addr(&bar[i]); };
 
-  if (warp == kDmDecWarps + 1) {
-    // ------------------------------------------------------------ producer
+  if (warp == DW + 1) {
+    // ------------------------------------------------------------ copies
     // code tiles, codebooks and hidden operands; a buffer is refilled once
     // the A slot of the step that read it is full (its decode is done, and
     // the decoders had waited for the MMAs of two steps before)
     if (lane == 0 && S > 0) {
       const uint64_t pol_codes = l2_policy_evict_first();
-      int last_codes[kDmStages], last_book[2] = {-1, -1};
-      for (int i = 0; i < kDmStages; ++i) last_codes[i] = -1;
+      int last_codes[S_::STAGES], last_book[2] = {-1, -1};
+      for (int i = 0; i < S_::STAGES; ++i) last_codes[i] = -1;
       bool to = false;
       auto wait = [&](int i, uint32_t parity) {
         if (!to && !mbar_try_wait(bar_at(i), parity) && !mbar_wait_bounded(bar_at(i), parity)) {
@@ -265,27 +289,27 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         }
       };
       auto issue_codes = [&](int g) {
-        const int sidx = g % kDmStages, p = g / G, gi = g % G;
+        const int sidx = g % S_::STAGES, p = g / G, gi = g % G;
         const uint32_t b = bar_at(kBarCodes + sidx);
-        mbar_arrive_expect_tx(b, kDmStageBytes);
-        const uint32_t dst = smem_addr(st + sidx * kDmStageBytes);
+        mbar_arrive_expect_tx(b, S_::STAGE_BYTES);
+        const uint32_t dst = smem_addr(st + sidx * S_::STAGE_BYTES);
 #pragma unroll
-        for (int q = 0; q < kDmRows / 256; ++q)
-          tma_load_2d(dst + q * 4096, &tmap, gi * 2 * kDmGroup,
-                      (int)(r0 + (int64_t)p * kDmRows + q * 256), b, pol_codes);
+        for (int q = 0; q < S_::ROWS / 128; ++q)
+          tma_load_2d(dst + q * (128 * S_::ROW_BYTES), &tmap, gi * S_::BOX_INNER,
+                      (int)(r0 + (int64_t)p * S_::ROWS + q * 128), b, pol_codes);
         last_codes[sidx] = g;
       };
       // the decoders wait for both before decoding s, so a full A slot of s
       // also tells the MMA warp that the hidden operand of s has landed
       auto issue_book = [&](int s, int m) {
         const uint32_t b = bar_at(kBarBook + (s & 1));
-        mbar_arrive_expect_tx(b, cbb + kDmHFloats * 4);
+        mbar_arrive_expect_tx(b, cbb + S_::HFLOATS * 4);
         bulk_g2s(smem_addr(cb + (size_t)(s & 1) * cbs), a.C + (size_t)m * cbf, cbb, b);
-        bulk_g2s(smem_addr(hs + (s & 3) * kDmHFloats), a.hop + (size_t)m * kDmHFloats,
-                 kDmHFloats * 4, b);
+        bulk_g2s(smem_addr(hs + (s & 3) * S_::HFLOATS), a.hop + (size_t)m * S_::HFLOATS,
+                 S_::HFLOATS * 4, b);
         last_book[s & 1] = s;
       };
-      for (int g = 0; g < NG && g < kDmStages; ++g) issue_codes(g);
+      for (int g = 0; g < NG && g < S_::STAGES; ++g) issue_codes(g);
       for (int s = 0; s < S && s < 2; ++s) issue_book(s, s % M);
       int p = 0, m = 0;
       for (int s = 0; s < S; ++s) {
@@ -293,9 +317,9 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         wait(kBarFull + s % kDmASlots, (uint32_t)(s / kDmASlots) & 1u);   // decode of s done
         if (to) break;
         if (s + 2 < S) issue_book(s + 2, m + 2 < M ? m + 2 : m + 2 - M);
-        if (m % kDmGroup == kDmGroup - 1) {
-          const int g = p * G + m / kDmGroup;                  // its stage is read out
-          if (g + kDmStages < NG) issue_codes(g + kDmStages);
+        if (m % S_::GROUP == S_::GROUP - 1) {
+          const int g = p * G + m / S_::GROUP;                 // its stage is read out
+          if (g + S_::STAGES < NG) issue_codes(g + S_::STAGES);
         }
         if (++m == M) {
           m = 0;
@@ -304,19 +328,19 @@ __global__ void __launch_bounds__(kDmThreads, 1)
       }
       if (*abort_flag) {
         // let the copies in flight land before the CTA's shared memory goes
-        for (int i = 0; i < kDmStages; ++i)
+        for (int i = 0; i < S_::STAGES; ++i)
           if (last_codes[i] >= 0)
-            mbar_wait_bounded(bar_at(kBarCodes + i), (uint32_t)(last_codes[i] / kDmStages) & 1u);
+            mbar_wait_bounded(bar_at(kBarCodes + i), (uint32_t)(last_codes[i] / S_::STAGES) & 1u);
         for (int i = 0; i < 2; ++i)
           if (last_book[i] >= 0)
             mbar_wait_bounded(bar_at(kBarBook + i), (uint32_t)(last_book[i] >> 1) & 1u);
         atomicOr(a.err, RQ_DEVERR_TIMEOUT);
       }
     }
-  } else if (warp == kDmDecWarps) {
+  } else if (warp == DW) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0 && S > 0) {
-      const uint32_t id64 = mma_idesc(2 * kDmTokens), id32 = mma_idesc(kDmTokens);
+      const uint32_t idw = mma_idesc(2 * NT), idn = mma_idesc(NT);
       int issued = 0;                          // steps whose MMAs are committed
       bool to = false;
       auto wait = [&](int i, uint32_t parity) {
@@ -330,8 +354,8 @@ __global__ void __launch_bounds__(kDmThreads, 1)
       int p = 0, m = 0, nt = 0;
       for (int s = 0; s < S; ++s) {
         if (m == 0) {
-          const int64_t rows = (r1 - r0) - (int64_t)p * kDmRows;
-          nt = (int)(((rows < kDmRows ? rows : kDmRows) + 127) / 128);
+          const int64_t rows = (r1 - r0) - (int64_t)p * S_::ROWS;
+          nt = (int)(((rows < S_::ROWS ? rows : S_::ROWS) + 127) / 128);
         }
         if (*abort_flag) break;
         // A slot of s written (and, as the decoders waited for it, the hidden
@@ -344,15 +368,16 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         if (first && c >= 1) wait(kBarFlush, (uint32_t)(c - 1) & 1u);
         if (to) break;
         tc_fence_after();
-        const uint32_t slot = tmem + kDmAcol + (uint32_t)(s % kDmASlots) * kDmAslot;
-        const unsigned long long b = bd0 + (unsigned long long)((s & 3) * (kDmHFloats * 4 / 16));
+        const uint32_t slot = tmem + S_::ACOL + (uint32_t)(s % kDmASlots) * S_::ASLOT;
+        const unsigned long long b =
+            bd0 + (unsigned long long)((s & 3) * (S_::HFLOATS * 4 / 16));
 #pragma unroll
-        for (int t = 0; t < kDmTiles; ++t) {
+        for (int t = 0; t < S_::TILES; ++t) {
           if (t < nt) {
-            const uint32_t d = tmem + (uint32_t)(t * 2 * kDmTokens);
+            const uint32_t d = tmem + (uint32_t)t * S_::ACC;
             const uint32_t ah = slot + (uint32_t)(t * 16);
-            mma_tf32_ts(d, ah, b, id64, first ? 0u : 1u);
-            mma_tf32_ts(d, ah + 8u, b, id32, 1u);
+            mma_tf32_ts(d, ah, b, idw, first ? 0u : 1u);   // E_hi . [h_hi | h_lo]
+            mma_tf32_ts(d, ah + 8u, b, idn, 1u);           // E_lo . h_hi
           }
         }
         mma_commit(bar_at(kBarMma + s % kDmASlots));
@@ -365,7 +390,8 @@ __global__ void __launch_bounds__(kDmThreads, 1)
       if (*abort_flag) {
         // let the MMAs in flight finish before the CTA's tensor memory goes
         for (int s = issued - kDmASlots; s < issued; ++s)
-          if (s >= 0) mbar_wait_bounded(bar_at(kBarMma + s % kDmASlots), (uint32_t)(s / kDmASlots) & 1u);
+          if (s >= 0)
+            mbar_wait_bounded(bar_at(kBarMma + s % kDmASlots), (uint32_t)(s / kDmASlots) & 1u);
         atomicOr(a.err, RQ_DEVERR_TIMEOUT);
       }
     }
@@ -374,8 +400,10 @@ __global__ void __launch_bounds__(kDmThreads, 1)
     const int wg = warp >> 2, q = warp & 3;
     const int r = wg * 128 + q * 32 + lane;   // this thread's row of a pass
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    ArgBest mine{-FLT_MAX, INT_MAX};          // lane tok: this warp's best row for token tok
-    float acc[kDmTokens];
+    ArgBest mine[NT / 32];                    // lane l: this warp's best row for token 32 i + l
+#pragma unroll
+    for (int i = 0; i < NT / 32; ++i) mine[i] = ArgBest{-FLT_MAX, INT_MAX};
+    float acc[NT];
     bool to = false;
     auto wait = [&](int i, uint32_t parity) {
       bool ok = to || mbar_try_wait(bar_at(i), parity) || mbar_wait_bounded(bar_at(i), parity);
@@ -387,15 +415,15 @@ __global__ void __launch_bounds__(kDmThreads, 1)
     };
     // add chain c (its MMAs are done) into the register sums; tiles past the
     // pass's rows are skipped warp-uniformly but every warp arrives
-    auto flush = [&](int c, int nt) {
+    auto flush = [&](int nt) {
       if (wg < nt) {
         tc_fence_after();
-        const uint32_t base = tmem + lane_base + (uint32_t)(wg * 2 * kDmTokens);
+        const uint32_t base = tmem + lane_base + (uint32_t)wg * S_::ACC;
         uint32_t x[16], y[16];
 #pragma unroll
-        for (int c0 = 0; c0 < kDmTokens; c0 += 16) {
+        for (int c0 = 0; c0 < NT; c0 += 16) {
           tmem_ld16(base + (uint32_t)c0, x);
-          tmem_ld16(base + (uint32_t)(kDmTokens + c0), y);
+          tmem_ld16(base + (uint32_t)(NT + c0), y);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -409,23 +437,25 @@ __global__ void __launch_bounds__(kDmThreads, 1)
     };
 
     for (int p = 0; p < npass && !to; ++p) {
-      const int64_t pr0 = r0 + (int64_t)p * kDmRows;
-      const int64_t rows = (r1 - pr0) < kDmRows ? (r1 - pr0) : kDmRows;
+      const int64_t pr0 = r0 + (int64_t)p * S_::ROWS;
+      const int64_t rows = (r1 - pr0) < S_::ROWS ? (r1 - pr0) : S_::ROWS;
       const int nt = (int)((rows + 127) / 128);
 #pragma unroll
-      for (int t = 0; t < kDmTokens; ++t) acc[t] = 0.f;
+      for (int t = 0; t < NT; ++t) acc[t] = 0.f;
       uint4 cw = make_uint4(0, 0, 0, 0);
+      uint32_t stage = 0;
       for (int m = 0; m < M; ++m) {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) {
           to = true;
           break;
         }
-        const int s = p * M + m, i4 = m % kDmGroup;
-        if (i4 == 0) {
-          const int g = p * G + m / kDmGroup, sidx = g % kDmStages;
-          wait(kBarCodes + sidx, (uint32_t)(g / kDmStages) & 1u);
+        const int s = p * M + m, ig = m % S_::GROUP;
+        if (ig == 0) {
+          const int g = p * G + m / S_::GROUP, sidx = g % S_::STAGES;
+          wait(kBarCodes + sidx, (uint32_t)(g / S_::STAGES) & 1u);
           if (to) break;
-          cw = lds_u4(smem_addr(st + sidx * kDmStageBytes) + (uint32_t)r * 16u);
+          stage = smem_addr(st + sidx * S_::STAGE_BYTES) + (uint32_t)r * S_::ROW_BYTES;
+          if (!S_::PACKED) cw = lds_u4(stage);
         }
         wait(kBarBook + (s & 1), (uint32_t)(s >> 1) & 1u);
         if (s >= kDmASlots)                                     // A slot free
@@ -433,13 +463,27 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         if (to) break;
         // the MMAs of s - 2, the last of the previous chain, are done (waited
         // for above): read it out before the next chain starts over it
-        if (m % kDmChain == 1 && m > kDmChain) flush(p * NC + m / kDmChain - 1, nt);
+        if (m % kDmChain == 1 && m > kDmChain) flush(nt);
         tc_fence_after();
         if (wg < nt) {
+          uint32_t c0, c1;
+          if (S_::PACKED) {
+            // codes 2m and 2m + 1 of the row: bits [20 ig, 20 ig + 20) of its
+            // 80-byte slice, LSB first (a field spans at most two words)
+            const int bit = 20 * ig, wi = bit >> 5, sh = bit & 31;
+            const uint32_t w0 = lds_u32(stage + 4u * wi);
+            const uint32_t w1 = lds_u32(stage + 4u * (wi + 1 < 20 ? wi + 1 : wi));
+            const uint32_t v = sh == 0 ? w0 : __funnelshift_r(w0, w1, sh);
+            c0 = a.fix(v & 1023u);
+            c1 = a.fix((v >> 10) & 1023u);
+          } else {
+            const uint32_t w = ig == 0 ? cw.x : ig == 1 ? cw.y : ig == 2 ? cw.z : cw.w;
+            c0 = a.fix(w & 0xFFFFu);
+            c1 = a.fix(w >> 16);
+          }
           const float *book = cb + (size_t)(s & 1) * cbs;
-          const uint32_t w = i4 == 0 ? cw.x : i4 == 1 ? cw.y : i4 == 2 ? cw.z : cw.w;
-          const float2 *p0 = reinterpret_cast<const float2 *>(book + a.fix(w & 0xFFFFu) * 6);
-          const float2 *p1 = reinterpret_cast<const float2 *>(book + (a.K + a.fix(w >> 16)) * 6);
+          const float2 *p0 = reinterpret_cast<const float2 *>(book + c0 * 6);
+          const float2 *p1 = reinterpret_cast<const float2 *>(book + (a.K + c1) * 6);
           float hi[6], lo[6];
 #pragma unroll
           for (int j2 = 0; j2 < 3; ++j2) {
@@ -450,7 +494,7 @@ __global__ void __launch_bounds__(kDmThreads, 1)
             lo[2 * j2] = __fsub_rn(e0, hi[2 * j2]);
             lo[2 * j2 + 1] = __fsub_rn(e1, hi[2 * j2 + 1]);
           }
-          tmem_st_hilo(tmem + lane_base + kDmAcol + (uint32_t)(s % kDmASlots) * kDmAslot +
+          tmem_st_hilo(tmem + lane_base + S_::ACOL + (uint32_t)(s % kDmASlots) * S_::ASLOT +
                            (uint32_t)(wg * 16),
                        hi, lo);
           tmem_wait_st();
@@ -465,13 +509,13 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         const int sl = p * M + M - 1;
         wait(kBarMma + sl % kDmASlots, (uint32_t)(sl / kDmASlots) & 1u);
         if (to) break;
-        if (NC >= 2 && (NC - 1) * kDmChain + 1 > M - 1) flush(p * NC + NC - 2, nt);
-        flush(p * NC + NC - 1, nt);
+        if (NC >= 2 && (NC - 1) * kDmChain + 1 > M - 1) flush(nt);
+        flush(nt);
       }
 
       // epilogue: softcap, logits, per-token best row of this warp
 #pragma unroll
-      for (int tok = 0; tok < kDmTokens; ++tok) {
+      for (int tok = 0; tok < NT; ++tok) {
         ArgBest best{-FLT_MAX, INT_MAX};
         if (r < rows && tok < a.nb) {
           const int64_t v = pr0 + r;
@@ -481,18 +525,19 @@ __global__ void __launch_bounds__(kDmThreads, 1)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) best = arg_better(best, arg_shfl_xor(best, o));
-        if (lane == tok) mine = arg_better(mine, best);
+        if (lane == (tok & 31)) mine[tok >> 5] = arg_better(mine[tok >> 5], best);
       }
     }
-    wbest[warp * kDmTokens + lane] = mine;
+#pragma unroll
+    for (int i = 0; i < NT / 32; ++i) wbest[warp * NT + 32 * i + lane] = mine[i];
   }
 
   griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
-  if (a.am_val && tid < a.nb && tid < kDmTokens) {
+  if (a.am_val && tid < a.nb && tid < NT) {
     ArgBest bb{-FLT_MAX, INT_MAX};
-    for (int w2 = 0; w2 < kDmDecWarps; ++w2) bb = arg_better(bb, wbest[w2 * kDmTokens + tid]);
+    for (int w2 = 0; w2 < DW; ++w2) bb = arg_better(bb, wbest[w2 * NT + tid]);
     const int64_t rowi = (int64_t)(a.t0 + tid) * a.nblk;
     a.am_val[rowi + blockIdx.x] = bb.v;
     a.am_idx[rowi + blockIdx.x] = bb.i;
@@ -501,7 +546,7 @@ __global__ void __launch_bounds__(kDmThreads, 1)
       a.am_idx[rowi + c] = INT_MAX;
     }
   }
-  if (warp == kDmDecWarps) {
+  if (warp == DW) {
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -509,36 +554,41 @@ __global__ void __launch_bounds__(kDmThreads, 1)
   }
 }
 
-size_t decode_mma_smem(int K, int N) {
-  (void)N;
+namespace {
+
+template <int NT, int FMT>
+size_t dm_smem(int K) {
+  using S_ = DmShape<NT, FMT>;
   const size_t cbs = (size_t)align_up(2 * K * 6, 256) * 4;
-  return 1024 + (size_t)kDmStages * kDmStageBytes + 2 * cbs +
-         kDmHSlots * kDmHFloats * 4 + kBars * 8 + (size_t)kDmDecWarps * kDmTokens * sizeof(ArgBest) +
+  return 1024 + (size_t)S_::STAGES * S_::STAGE_BYTES + 2 * cbs + kDmHSlots * S_::HFLOATS * 4 +
+         (S_::STAGES + 2 + 2 * kDmASlots + 1) * 8 + (size_t)S_::DEC_WARPS * NT * sizeof(ArgBest) +
          16;
 }
 
-size_t decode_mma_hop_bytes(int M) { return (size_t)M * kDmHFloats * 4; }
-
-cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void *codes,
-                                     int64_t V, int D, int M, int K, int t0, int nb, int N,
-                                     float cap, float *hop, float *logits, float *am_val,
-                                     int *am_idx, int nblk, const DevInfo &di, cudaStream_t s) {
-  if (N != kDmTokens || nb < 1 || nb > kDmTokens || M % kDmGroup != 0) return cudaErrorInvalidValue;
+template <int NT, int FMT>
+cudaError_t launch_dm(const float *h, const float *C, const void *codes, int64_t V, int D, int M,
+                      int K, int t0, int nb, float cap, float *hop, float *logits, float *am_val,
+                      int *am_idx, int nblk, const DevInfo &di, cudaStream_t s) {
+  using S_ = DmShape<NT, FMT>;
+  if (nb < 1 || nb > NT || M % S_::GROUP != 0) return cudaErrorInvalidValue;
   CUtensorMap tmap;
   const int P = 2 * M;
-  if (!encode_tmap_2d_u16(&tmap, codes, (uint64_t)P, (uint64_t)V, (uint64_t)P * 2,
-                          2 * kDmGroup, 256, CU_TENSOR_MAP_SWIZZLE_NONE))
+  // packed rows (P * 10 / 8 bytes, a multiple of 16 as M % 32 == 0) are
+  // copied as 16-bit units: the copy moves bytes whatever the element type
+  const uint64_t row_bytes = S_::PACKED ? (uint64_t)P * 10 / 8 : (uint64_t)P * 2;
+  if (!encode_tmap_2d_u16(&tmap, codes, row_bytes / 2, (uint64_t)V, row_bytes, S_::BOX_INNER, 128,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   {
     void *args[] = {&h, &D, &t0, &nb, &hop};
-    cudaError_t e = launch_maybe_pdl(reinterpret_cast<const void *>(&split_hidden_kernel),
-                                     dim3((unsigned)M), dim3(256), 0, s, args, true);
+    cudaError_t e = launch_maybe_pdl(reinterpret_cast<const void *>(&split_hidden_kernel<NT>),
+                                     dim3((unsigned)M), dim3(NT * 8), 0, s, args, true);
     if (e != cudaSuccess) return e;
   }
-  const size_t smem = decode_mma_smem(K, N);
+  const size_t smem = dm_smem<NT, FMT>(K);
   static size_t smem_set[128] = {};
   if (di.device >= 128) return cudaErrorInvalidDevice;
-  const void *fn = reinterpret_cast<const void *>(&logits_decode_mma_kernel);
+  const void *fn = reinterpret_cast<const void *>(&logits_decode_mma_kernel<NT, FMT>);
   if (smem > smem_set[di.device]) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -560,8 +610,45 @@ cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void 
   a.fix = make_codefix(K);
   a.err = di.err;
   void *args[] = {&tmap, &a};
-  return launch_maybe_pdl(fn, dim3((unsigned)decode_fma_blocks(V, di)), dim3(kDmThreads), smem, s,
+  return launch_maybe_pdl(fn, dim3((unsigned)decode_fma_blocks(V, di)), dim3(S_::THREADS), smem, s,
                           args, true);
+}
+
+}  // namespace
+
+size_t decode_mma_smem(int K, int N, int fmt) {
+  const bool packed = fmt == RQ_CODES_PACKED10;
+  if (N == 32) return packed ? dm_smem<32, RQ_CODES_PACKED10>(K) : dm_smem<32, RQ_CODES_U16>(K);
+  return packed ? dm_smem<64, RQ_CODES_PACKED10>(K) : dm_smem<64, RQ_CODES_U16>(K);
+}
+
+size_t decode_mma_hop_bytes(int M, int N) { return (size_t)M * 2 * N * 8 * 4; }
+
+bool decode_mma_applies(int fmt, int64_t V, int D, int M, int L, int K, const float *C,
+                        const void *codes) {
+  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return false;
+  if (L != 2 || D != 6 * M || K > 1024 || K < 1) return false;
+  if (M % (fmt == RQ_CODES_PACKED10 ? 32 : 8) != 0) return false;
+  if (V < 1 || V > (int64_t)INT_MAX - 2048) return false;
+  return (reinterpret_cast<uintptr_t>(C) & 15) == 0 && (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
+}
+
+cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void *codes, int fmt,
+                                     int64_t V, int D, int M, int K, int t0, int nb, int N,
+                                     float cap, float *hop, float *logits, float *am_val,
+                                     int *am_idx, int nblk, const DevInfo &di, cudaStream_t s) {
+  const bool packed = fmt == RQ_CODES_PACKED10;
+  if (N == 32)
+    return packed ? launch_dm<32, RQ_CODES_PACKED10>(h, C, codes, V, D, M, K, t0, nb, cap, hop,
+                                                      logits, am_val, am_idx, nblk, di, s)
+                  : launch_dm<32, RQ_CODES_U16>(h, C, codes, V, D, M, K, t0, nb, cap, hop, logits,
+                                                am_val, am_idx, nblk, di, s);
+  if (N == 64)
+    return packed ? launch_dm<64, RQ_CODES_PACKED10>(h, C, codes, V, D, M, K, t0, nb, cap, hop,
+                                                      logits, am_val, am_idx, nblk, di, s)
+                  : launch_dm<64, RQ_CODES_U16>(h, C, codes, V, D, M, K, t0, nb, cap, hop, logits,
+                                                am_val, am_idx, nblk, di, s);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace rq

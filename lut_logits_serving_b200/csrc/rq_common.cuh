@@ -406,14 +406,17 @@ cudaError_t launch_logits_decode_fma(const float *h, const float *C, const void 
                                      const DevInfo &di, cudaStream_t s);
 
 // The same on the tcgen05 tensor cores (tf32 MMAs with a hi/lo split for
-// fp32 accuracy); N = 32 tokens per group, M % 4 == 0.  hop: device scratch of
-// decode_mma_hop_bytes(M) for the group's split hidden operand.
-cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void *codes,
+// fp32 accuracy): token groups of N = 32 or 64, uint16 or 10-bit packed
+// codes (decode_mma_applies).  hop: device scratch of decode_mma_hop_bytes(M,
+// N) for the group's split hidden operand.
+bool decode_mma_applies(int fmt, int64_t V, int D, int M, int L, int K, const float *C,
+                        const void *codes);
+cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void *codes, int fmt,
                                      int64_t V, int D, int M, int K, int t0, int nb, int N,
                                      float cap, float *hop, float *logits, float *am_val,
                                      int *am_idx, int nblk, const DevInfo &di, cudaStream_t s);
-size_t decode_mma_smem(int K, int N);
-size_t decode_mma_hop_bytes(int M);
+size_t decode_mma_smem(int K, int N, int fmt);
+size_t decode_mma_hop_bytes(int M, int N);
 
 // Batched pass with the LUT read through L2 (token groups of <= 32).
 cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K,

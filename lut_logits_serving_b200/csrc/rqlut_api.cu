@@ -220,41 +220,50 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   const int P = d.M * d.L;
   float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
   int *ami = argmax ? reinterpret_cast<int *>(rest + w.ami_off) : nullptr;
-  // Full 32-token groups decode their rows and multiply them with the hidden
-  // states (on the tensor cores by default, measured fastest there, else the
-  // FP32 kernel); other groups read their tables through L2.  All write
-  // argmax partials into the same [B][nblk].
+  // Full token groups decode their rows and multiply them with the hidden
+  // states: on the tensor cores by default (groups of 64, then 32; measured
+  // fastest), else the FP32 kernel (groups of 32); other groups read their
+  // tables through L2.  All write argmax partials into the same [B][nblk].
   const int nblk = sweep_blocks(d, di, false);
-  const bool dfma = decode_fma_applies(fmt, d.V, d.D, d.M, d.L, d.K, B, C, codes, di) &&
-                    decode_fma_blocks(d.V, di) <= nblk;
-  const bool dtc = dfma && decode_mma_smem(d.K, kTokenGroup) <= (size_t)di.max_smem_optin &&
-                   decode_mma_hop_bytes(d.M) <= lut_bytes;
-  if ((path == RQ_PATH_DECODE_FP32 && !dfma) || (path == RQ_PATH_DECODE_TC && !dtc))
+  const bool grid_ok = decode_fma_blocks(d.V, di) <= nblk;
+  const bool dfma = grid_ok && decode_fma_applies(fmt, d.V, d.D, d.M, d.L, d.K, B, C, codes, di);
+  const bool tc_fmt = grid_ok && decode_mma_applies(fmt, d.V, d.D, d.M, d.L, d.K, C, codes);
+  // the tensor-core kernel keeps the group's split hidden operand in the
+  // (here unused) table region
+  auto tc_fits = [&](int n) {
+    return tc_fmt && decode_mma_smem(d.K, n, fmt) <= (size_t)di.max_smem_optin &&
+           decode_mma_hop_bytes(d.M, n) <= lut_bytes;
+  };
+  const bool tc32 = tc_fits(32), tc64 = tc_fits(64);
+  if ((path == RQ_PATH_DECODE_FP32 && !dfma) || (path == RQ_PATH_DECODE_TC && !tc32))
     return RQ_ERR_UNSUPPORTED;
-  const bool decode = path != RQ_PATH_TABLES && dfma;
+  const bool use_tc = (path == RQ_PATH_DECODE_TC || path == RQ_PATH_AUTO) && tc32;
+  const bool use_fma = !use_tc && (path == RQ_PATH_DECODE_FP32 || path == RQ_PATH_AUTO) && dfma;
   cudaError_t e = cudaSuccess;
   bool marked = false;   // the profile start goes before the first logits kernel
-  for (int b0 = 0; b0 < B && e == cudaSuccess; b0 += G) {
-    const int nb = B - b0 < G ? B - b0 : G;
-    if (decode && nb == kTokenGroup) {
+  for (int b0 = 0; b0 < B && e == cudaSuccess;) {
+    const int rem = B - b0;
+    const int nd = use_tc && tc64 && rem >= 64 ? 64 : (use_tc || use_fma) && rem >= 32 ? 32 : 0;
+    if (nd > 0) {
       if (!marked && (e = prof_mark(t_prof_start, s)) != cudaSuccess) break;
       marked = true;
-      // the tensor-core kernel keeps the group's split hidden operand in the
-      // (here unused) table region
-      if (path == RQ_PATH_DECODE_TC || (path == RQ_PATH_AUTO && dtc))
-        e = launch_logits_decode_mma(h, C, codes, d.V, d.D, d.M, d.K, b0, nb, kTokenGroup, softcap,
+      if (use_tc)
+        e = launch_logits_decode_mma(h, C, codes, fmt, d.V, d.D, d.M, d.K, b0, nd, nd, softcap,
                                      lut, logits, amv, ami, nblk, di, s);
       else
-        e = launch_logits_decode_fma(h, C, codes, d.V, d.D, d.M, d.K, b0, nb, softcap, logits,
+        e = launch_logits_decode_fma(h, C, codes, d.V, d.D, d.M, d.K, b0, nd, softcap, logits,
                                      amv, ami, nblk, di, s);
+      b0 += nd;
       continue;
     }
+    const int nb = rem < G ? rem : G;
     e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, s);
     if (e == cudaSuccess && !marked) e = prof_mark(t_prof_start, s);
     marked = true;
     if (e == cudaSuccess)
       e = launch_logits_l2(codes, fmt, d.V, P, d.K, lut, Bs, 0, b0, nb, softcap, logits, amv, ami,
                            nblk, s);
+    b0 += nb;
   }
   if (e != cudaSuccess) return status_of(e);
   if (cudaError_t e = prof_mark(t_prof_stop, s)) return status_of(e);

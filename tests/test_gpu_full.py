@@ -109,13 +109,14 @@ def test_g2_batch32_one_code_pass(g2, path):
     assert rq.rq_device_error() == 0
 
 
-def test_g2_packed_batch64_fused_argmax(g2):
+@pytest.mark.parametrize("path", [None, rq.PATH_TABLES])
+def test_g2_packed_batch64_fused_argmax(g2, path):
     w = synth.WORKLOADS["packed_b64"]
     packed = rq.rq_pack10(g2["dc"], g2["d"]).cpu().numpy()
     rows = _sample_rows(w.V, 2000, 11)
     assert np.array_equal(packed[rows], oracle.pack10(g2["codes"][rows]))
-    err, ties = _batched(g2, w, rq.PACKED10, 9)
-    print(f"packed_b64 normwise error {err:.3g}, ties {ties}")
+    err, ties = _batched(g2, w, rq.PACKED10, 9, path)
+    print(f"packed_b64 path {path} normwise error {err:.3g}, ties {ties}")
     assert ties == 0
 
 

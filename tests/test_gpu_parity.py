@@ -349,6 +349,9 @@ def test_greedy_step_rows_are_the_picked_tokens_rows(B, fmt):
     (5000, 40, 7, 33),        # 5 code groups, a one-token second group (table path)
     (3001, 16, 1024, 64),     # two full token groups
     (2500, 8, 256, 48),       # a full group (decoded) and a 16-token group (tables)
+    (7001, 16, 1024, 64),     # one 64-token group on the tensor cores
+    (3333, 8, 512, 100),      # groups of 64 and 32 and a 4-token rest
+    (999, 24, 13, 64),        # K < 16: the tensor cores take two 32-token groups
 ])
 @pytest.mark.parametrize("path", [None, rq.PATH_TABLES, rq.PATH_DECODE_FP32, rq.PATH_DECODE_TC])
 def test_fused_decode_paths(V, M, K, B, path):
@@ -371,6 +374,31 @@ def test_fused_decode_paths(V, M, K, B, path):
     assert rq.rq_device_error() == 0
     assert_logits_close(logits.cpu().numpy(), ref)
     check_argmax(am.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("V,M,K,B", [
+    (4096, 32, 256, 32),      # the tiny workload's shape, one 32-token group
+    (5003, 32, 1024, 64),     # one 64-token group, ragged rows
+    (2222, 64, 100, 70),      # groups of 64 + a 6-token rest (tables), K not a power of two
+])
+def test_packed_codes_on_the_tensor_cores(V, M, K, B):
+    """10-bit packed codes (M % 32 == 0) are unpacked by the tensor-core kernel's
+    decoders: logits and argmax as for uint16 codes, codes >= K clamped."""
+    D = 6 * M
+    C, codes, h = make_case(V, D, M, 2, K, B, seed=V + 7)
+    d = rq.dims(V, D, M, 2, K)
+    ref = oracle_logits(C, codes, h, 30.0)
+    packed = rq.rq_pack10(dev(codes.reshape(V, -1)), d)
+    out = torch.full((B, V), float("nan"), device="cuda")
+    logits, am, _ = rq.rq_logits_from_hidden(dev(h), dev(C), packed, rq.PACKED10, d, 30.0,
+                                             want_argmax=True, logits=out,
+                                             path=rq.PATH_DECODE_TC)
+    assert rq.rq_device_error() == 0
+    assert_logits_close(logits.cpu().numpy(), ref)
+    check_argmax(am.cpu().numpy(), ref)
+    # the default takes the same kernel and gives the same numbers
+    logits2, _, _ = rq.rq_logits_from_hidden(dev(h), dev(C), packed, rq.PACKED10, d, 30.0)
+    assert torch.equal(logits2, logits)
 
 
 def test_decode_paths_need_their_format():
