@@ -181,20 +181,22 @@ RQ_API int rq_logits_from_hidden(const float *h, const float *C, const void *cod
                           size_t ws_bytes, void *stream);
 
 /*
- * Kernel choice for the full token groups of rq_logits_from_hidden_path
- * (groups of fewer tokens always read their tables through L2).  The decode
+ * Kernel choice for the token groups of rq_logits_from_hidden_path (batches
+ * of up to 4 tokens always take the shared-memory table pass).  The decode
  * paths rebuild each vocabulary row once per group (the decode-then-matmul
  * the LUT section checks the lookup against) and contract it with the
  * group's hidden states; they need L = 2, D = 6 M, K <= 1024 and 16-byte
  * aligned C and codes.
- *   RQ_PATH_AUTO        -- RQ_PATH_DECODE_TC where it applies, else
+ *   RQ_PATH_AUTO        -- RQ_PATH_DECODE_TC where it applies (for a group
+ *                          of fewer than 32 tokens from 17 tokens on), else
  *                          RQ_PATH_DECODE_FP32 where that applies, else tables
  *   RQ_PATH_TABLES      -- per-group tables read through L2 (lookup + sum)
  *   RQ_PATH_DECODE_FP32 -- groups of 32; rows decoded into shared memory,
  *                          fp32 FMAs; RQ_CODES_U16 with M % 8 == 0
- *   RQ_PATH_DECODE_TC   -- groups of 64, then 32; rows decoded into tensor
- *                          memory, tcgen05 tf32 MMAs on a hi/lo split with
- *                          fp32 chain sums; RQ_CODES_U16 with M % 8 == 0 or
+ *   RQ_PATH_DECODE_TC   -- groups of 64, then 32, then the rest; rows
+ *                          decoded into tensor memory, tcgen05 tf32 MMAs on
+ *                          a hi/lo split with fp32 chain sums;
+ *                          RQ_CODES_U16 with M % 8 == 0 or
  *                          RQ_CODES_PACKED10 with M % 32 == 0; K >= 8 (16 for
  *                          groups of 64: the hidden operand is staged in the
  *                          workspace's table region)

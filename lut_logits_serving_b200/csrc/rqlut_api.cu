@@ -193,6 +193,12 @@ int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, i
 
 int fused_group(int B) { return B <= 4 ? B : (B < kTokenGroup ? B : kTokenGroup); }
 
+// Smallest partial token group (fewer than 32 tokens) that the fused calls
+// send to the tensor cores: with RQ_PATH_DECODE_TC every group does (down to
+// one token); by default from the size where the tables measured slower.
+constexpr int kTcPartialMin = 17;
+int tc_partial_min(int path) { return path == RQ_PATH_DECODE_TC ? 1 : kTcPartialMin; }
+
 
 // rq_logits_from_hidden and rq_greedy_step: table build per token group,
 // code pass, softcap, logits/argmax, optionally the picked tokens' rows.
@@ -243,13 +249,20 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   bool marked = false;   // the profile start goes before the first logits kernel
   for (int b0 = 0; b0 < B && e == cudaSuccess;) {
     const int rem = B - b0;
-    const int nd = use_tc && tc64 && rem >= 64 ? 64 : (use_tc || use_fma) && rem >= 32 ? 32 : 0;
+    // a group of fewer than 32 tokens also takes the tensor cores from
+    // kTcPartialMin tokens on: their time hardly depends on the group's fill,
+    // the tables' grows with it
+    const int nd = use_tc && tc64 && rem >= 64                 ? 64
+                   : (use_tc || use_fma) && rem >= 32          ? 32
+                   : use_tc && rem >= tc_partial_min(path)     ? rem
+                                                               : 0;
     if (nd > 0) {
       if (!marked && (e = prof_mark(t_prof_start, s)) != cudaSuccess) break;
       marked = true;
       if (use_tc)
-        e = launch_logits_decode_mma(h, C, codes, fmt, d.V, d.D, d.M, d.K, b0, nd, nd, softcap,
-                                     lut, logits, amv, ami, nblk, di, s);
+        e = launch_logits_decode_mma(h, C, codes, fmt, d.V, d.D, d.M, d.K, b0, nd,
+                                     nd > 32 ? 64 : 32, softcap, lut, logits, amv, ami, nblk, di,
+                                     s);
       else
         e = launch_logits_decode_fma(h, C, codes, d.V, d.D, d.M, d.K, b0, nd, softcap, logits,
                                      amv, ami, nblk, di, s);
