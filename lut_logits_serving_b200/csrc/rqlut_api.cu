@@ -226,10 +226,11 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   const int P = d.M * d.L;
   float *amv = argmax ? reinterpret_cast<float *>(rest + w.amv_off) : nullptr;
   int *ami = argmax ? reinterpret_cast<int *>(rest + w.ami_off) : nullptr;
-  // Full token groups decode their rows and multiply them with the hidden
-  // states: on the tensor cores by default (groups of 64, then 32; measured
-  // fastest), else the FP32 kernel (groups of 32); other groups read their
-  // tables through L2.  All write argmax partials into the same [B][nblk].
+  // Token groups decode their rows and multiply them with the hidden states:
+  // on the tensor cores by default (groups of 64, then 32, then a rest of 17
+  // or more tokens; measured fastest), else the FP32 kernel (groups of 32);
+  // other groups read their tables through L2.  All write argmax partials
+  // into the same [B][nblk].
   const int nblk = sweep_blocks(d, di, false);
   const bool grid_ok = decode_fma_blocks(d.V, di) <= nblk;
   const bool dfma = grid_ok && decode_fma_applies(fmt, d.V, d.D, d.M, d.L, d.K, B, C, codes, di);
