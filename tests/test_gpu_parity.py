@@ -406,6 +406,26 @@ def test_packed_codes_on_the_tensor_cores(V, M, K, B):
     assert_logits_close(logits2.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("B", [32, 64])
+def test_tensor_core_decode_argmax_only_and_softcap_off(B):
+    """Without a logits buffer the tensor-core kernel still leaves the argmax
+    partials; with the softcap off it returns the raw sums."""
+    V, M, K = 3001, 16, 256
+    C, codes, h = make_case(V, 6 * M, M, 2, K, B, seed=11, hscale=20.0)   # logits well past 30
+    d = rq.dims(V, 6 * M, M, 2, K)
+    args = (dev(h), dev(C), dev(codes.reshape(V, -1)), rq.U16, d)
+    ref = oracle_logits(C, codes, h, 30.0)
+    _, am, _ = rq.rq_logits_from_hidden(*args, 30.0, want_logits=False, want_argmax=True,
+                                        path=rq.PATH_DECODE_TC)
+    check_argmax(am.cpu().numpy(), ref)
+    raw = oracle_logits(C, codes, h, 0.0)
+    assert np.abs(raw).max() > 30.0
+    logits, am0, _ = rq.rq_logits_from_hidden(*args, 0.0, want_argmax=True, path=rq.PATH_DECODE_TC)
+    assert_logits_close(logits.cpu().numpy(), raw)
+    check_argmax(am0.cpu().numpy(), raw)
+    assert rq.rq_device_error() == 0
+
+
 def test_decode_paths_need_their_format():
     """A decode path the format cannot take is refused, not silently replaced."""
     V, M, K, B = 512, 8, 256, 32
