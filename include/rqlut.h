@@ -353,6 +353,30 @@ RQ_API int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out,
                             uint64_t *stats, void *stream);
 
 /*
+ * Greedy pick over a vocabulary split across ranks ("Gemma-2 runtime
+ * compression: NF4 + LUT serving", LUT section: argmax of the softcapped
+ * logits of every vocabulary row; rows are independent, so rank g may hold
+ * only the code rows [row0_g, row0_g + V_g) and run the calls above on them).
+ *
+ * rq_argmax_candidates -- per token b of the shard's results: val[b] =
+ *   logits[b][argmax[b]] and gidx[b] = row0 + argmax[b] (the global row).
+ *   logits [B][V] fp32 and argmax [B] int32 as written for the shard; val
+ *   [B] fp32, gidx [B] int32 out.  row0 + V must fit in int32.  Device
+ *   pointers, 4-byte aligned; stream-ordered.
+ * rq_argmax_merge -- argmax[b] = the best of the n candidates val[k][b],
+ *   gidx[k][b] (rank-major [n][B], as an all-gather of the ranks' candidate
+ *   arrays lays them out): larger value first, lower index on equal values,
+ *   NaN never above a number -- the order of the single-GPU argmax, so the
+ *   merged pick equals the unsharded one.  argmax [B] int32 out.
+ * Errors: RQ_ERR_INVALID_ARGUMENT (null pointer, B < 1, n < 1, V < 1,
+ * row0 < 0 or an int32 overflow), RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ */
+RQ_API int rq_argmax_candidates(const float *logits, const int32_t *argmax, int B, int64_t V,
+                                int64_t row0, float *val, int32_t *gidx, void *stream);
+RQ_API int rq_argmax_merge(const float *val, const int32_t *gidx, int n, int B, int32_t *argmax,
+                           void *stream);
+
+/*
  * rq_device_error -- read (and, if `clear`, reset) the device error word
  * of the current device.  Synchronous: call after synchronizing the streams
  * that ran the kernels of interest.  *out receives RQ_DEVERR_* bits.

@@ -31,7 +31,7 @@ __all__ = [
     "rq_pack10", "rq_device_error", "rq_set_profile_events", "rq_lut_logits_static",
     "rq_greedy_step", "rq_encode", "rq_topk_workspace_bytes", "rq_topk_sample",
     "rq_last_cuda_error", "rq_cuda_error_name", "PATH_AUTO", "PATH_TABLES", "PATH_DECODE_FP32",
-    "PATH_DECODE_TC",
+    "PATH_DECODE_TC", "rq_argmax_candidates", "rq_argmax_merge", "shard_rows", "rq_sharded_logits",
 ]
 
 U16 = 0
@@ -103,6 +103,8 @@ _SIGNATURES = {
     "rq_prepare_sched": (_i, [_p, RqDims, _p, _p, _p]),
     "rq_lut_logits_static": (_i, [_p, _i, RqDims, _p, _i, _f, _p, _p, _p]),
     "rq_greedy_step": (_i, [_p, _p, _p, _i, RqDims, _i, _f, _p, _p, _f, _p, _p, _sz, _p]),
+    "rq_argmax_candidates": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p]),
+    "rq_argmax_merge": (_i, [_p, _p, _i, _i, _p, _p]),
 }
 
 
@@ -269,6 +271,69 @@ def rq_logits_from_hidden_path(h, C, codes, fmt: int, d: RqDims, path: int,
                                softcap: float = 30.0, **kw):
     """rq_logits_from_hidden with an explicit kernel for full token groups."""
     return rq_logits_from_hidden(h, C, codes, fmt, d, softcap, path=path, **kw)
+
+
+def rq_argmax_candidates(logits, argmax, row0: int, val=None, gidx=None, stream=None):
+    """A vocabulary shard's winner per token: (value float32 [B], global row
+    int32 [B]) from its logits [B, V_shard] and argmax [B]."""
+    torch = _torch()
+    B, V = logits.shape
+    if val is None:
+        val = _empty((B,), torch.float32, logits)
+    if gidx is None:
+        gidx = _empty((B,), torch.int32, logits)
+    _check("rq_argmax_candidates", lib().rq_argmax_candidates(
+        _cuda(logits, torch.float32, "logits"), _cuda(argmax, torch.int32, "argmax"), B, V,
+        int(row0), _cuda(val, torch.float32, "val"), _cuda(gidx, torch.int32, "gidx"),
+        _stream(stream)))
+    return val, gidx
+
+
+def rq_argmax_merge(val, gidx, out=None, stream=None):
+    """Global argmax int32 [B] from n shards' candidates val, gidx [n, B]."""
+    torch = _torch()
+    if val.dim() != 2 or tuple(gidx.shape) != tuple(val.shape):
+        raise ValueError("val, gidx: [n, B] expected")
+    n, B = val.shape
+    if out is None:
+        out = _empty((B,), torch.int32, val)
+    _check("rq_argmax_merge", lib().rq_argmax_merge(
+        _cuda(val, torch.float32, "val"), _cuda(gidx, torch.int32, "gidx"), n, B,
+        _cuda(out, torch.int32, "argmax"), _stream(stream)))
+    return out
+
+
+def shard_rows(V: int, rank: int, world: int):
+    """Rows [row0, row1) of vocabulary shard `rank` of `world` (even split)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank, world")
+    return V * rank // world, V * (rank + 1) // world
+
+
+def rq_sharded_logits(h, C, codes_shard, fmt: int, d_shard: RqDims, row0: int,
+                      softcap: float = 30.0, group=None, ws=None, stream=None):
+    """Logits of this rank's vocabulary rows and the global greedy pick: the
+    fused call on the shard, its per-token winner, one all-gather of the
+    winners over the process group (NCCL), and the merge.  Returns (logits
+    [B, V_shard], argmax int32 [B] of global rows, ws)."""
+    torch = _torch()
+    logits, am, ws = rq_logits_from_hidden(h, C, codes_shard, fmt, d_shard, softcap,
+                                           want_argmax=True, ws=ws, stream=stream)
+    val, gidx = rq_argmax_candidates(logits, am, row0, stream=stream)
+    world = 1
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        world = dist.get_world_size(group)
+    if world > 1:
+        # flat [world * B] buffers, rank-major (the layout every backend takes)
+        vals = _empty((world * val.numel(),), torch.float32, val)
+        idxs = _empty((world * gidx.numel(),), torch.int32, gidx)
+        dist.all_gather_into_tensor(vals, val, group=group)
+        dist.all_gather_into_tensor(idxs, gidx, group=group)
+        vals, idxs = vals.view(world, -1), idxs.view(world, -1)
+    else:
+        vals, idxs = val.view(1, -1), gidx.view(1, -1)
+    return logits, rq_argmax_merge(vals, idxs, stream=stream), ws
 
 
 def rq_decode_rows(ids, codes, fmt: int, C, d: RqDims, scale: float, out=None, stream=None):

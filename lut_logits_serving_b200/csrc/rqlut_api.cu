@@ -288,6 +288,14 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
 
 }  // namespace
 
+namespace rq {
+// Greedy pick over a vocabulary split across ranks (shard_argmax.cu).
+cudaError_t launch_argmax_candidates(const float *logits, const int32_t *argmax, int B, int64_t V,
+                                     int64_t row0, float *val, int32_t *gidx, cudaStream_t s);
+cudaError_t launch_argmax_merge(const float *val, const int32_t *gidx, int n, int B,
+                                int32_t *argmax, cudaStream_t s);
+}  // namespace rq
+
 extern "C" {
 
 const char *rq_status_string(int status) {
@@ -512,6 +520,24 @@ int rq_set_profile_events(void *start, void *stop) {
   t_prof_start = static_cast<cudaEvent_t>(start);
   t_prof_stop = static_cast<cudaEvent_t>(stop);
   return RQ_OK;
+}
+
+int rq_argmax_candidates(const float *logits, const int32_t *argmax, int B, int64_t V,
+                         int64_t row0, float *val, int32_t *gidx, void *stream) {
+  if (!logits || !argmax || !val || !gidx || B < 1 || V < 1 || row0 < 0 ||
+      row0 + V > (int64_t)INT_MAX)
+    return RQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(logits, 4) || !aligned(argmax, 4) || !aligned(val, 4) || !aligned(gidx, 4))
+    return RQ_ERR_MISALIGNED;
+  return status_of(launch_argmax_candidates(logits, argmax, B, V, row0, val, gidx,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int rq_argmax_merge(const float *val, const int32_t *gidx, int n, int B, int32_t *argmax,
+                    void *stream) {
+  if (!val || !gidx || !argmax || n < 1 || B < 1) return RQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(val, 4) || !aligned(gidx, 4) || !aligned(argmax, 4)) return RQ_ERR_MISALIGNED;
+  return status_of(launch_argmax_merge(val, gidx, n, B, argmax, static_cast<cudaStream_t>(stream)));
 }
 
 int rq_device_error(uint32_t *out, int clear) {

@@ -118,6 +118,13 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_lut_logits(a, 0, G2, odd, 1, 30.0, a, null, null, 0, s) == MIS
     assert lib.rq_logits_from_hidden(a, a, a, 0, G2, 1, 30.0, a, null, null, 0, s) == WS
     assert lib.rq_logits_from_hidden_path(a, a, a, 0, G2, 1, 30.0, a, null, null, 0, 7, s) == INV
+    assert lib.rq_argmax_candidates(null, a, 1, 10, 0, a, a, s) == INV
+    assert lib.rq_argmax_candidates(a, a, 1, 10, 2**31 - 5, a, a, s) == INV   # int32 rows
+    assert lib.rq_argmax_candidates(a, a, 0, 10, 0, a, a, s) == INV
+    assert lib.rq_argmax_candidates(_fake(0x10002), a, 1, 10, 0, a, a, s) == MIS
+    assert lib.rq_argmax_merge(a, a, 0, 1, a, s) == INV
+    assert lib.rq_argmax_merge(a, null, 2, 1, a, s) == INV
+    assert lib.rq_argmax_merge(a, a, 2, 1, _fake(0x10002), s) == MIS
     assert lib.rq_logits_from_hidden_path(a, a, a, 0, G2, 1, 30.0, a, null, null, 0, 3, s) == WS
     assert lib.rq_decode_rows(null, 5, a, 0, a, G2, 48.0, a, s) == INV
     assert lib.rq_decode_rows(a, -1, a, 0, a, G2, 48.0, a, s) == INV

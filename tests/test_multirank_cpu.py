@@ -61,3 +61,50 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.aggregate(7.0, 1) == 7.0
     assert bench.throughput(256000, 1, 0.1) == pytest.approx(2.56e9)
+
+
+def _shard_worker(rank, world, port, q):
+    """The exchange of the vocabulary-sharded pick: shard_rows covers the rows
+    once, and all_gather_into_tensor lays the ranks' per-token winners out
+    rank-major, [world][B], as rq_argmax_merge reads them."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import lut_logits_serving_b200 as rq
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    V, B = 1001, 5
+    r0, r1 = rq.shard_rows(V, rank, world)
+    val = torch.arange(B, dtype=torch.float32) + 100 * rank
+    gidx = torch.full((B,), r0, dtype=torch.int32)
+    vals = torch.empty((world * B,), dtype=torch.float32)   # flat, as rq_sharded_logits
+    idxs = torch.empty((world * B,), dtype=torch.int32)
+    dist.all_gather_into_tensor(vals, val)
+    dist.all_gather_into_tensor(idxs, gidx)
+    q.put((rank, r0, r1, vals.view(world, B).tolist(), idxs.view(world, B).tolist()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_sharded_pick_exchange_layout_with_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 3
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    bounds = [(r0, r1) for _, r0, r1, _, _ in res]
+    assert bounds[0][0] == 0 and bounds[-1][1] == 1001
+    assert all(bounds[i][1] == bounds[i + 1][0] for i in range(world - 1))
+    for _, _, _, vals, idxs in res:
+        assert vals == [[b + 100.0 * k for b in range(5)] for k in range(world)]
+        assert idxs == [[bounds[k][0]] * 5 for k in range(world)]
