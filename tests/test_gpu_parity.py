@@ -354,6 +354,7 @@ def test_greedy_step_rows_are_the_picked_tokens_rows(B, fmt):
     (999, 24, 13, 64),        # K < 16: the tensor cores take two 32-token groups
     (4099, 16, 256, 20),      # one partial group: the tensor cores by default (>= 17 tokens)
     (3000, 8, 1024, 57),      # 32 + a 25-token partial group on the tensor cores
+    (4100, 40, 64, 32),       # M = 40: accumulation chains of 16, 16 and 8 subspaces
 ])
 @pytest.mark.parametrize("path", [None, rq.PATH_TABLES, rq.PATH_DECODE_FP32, rq.PATH_DECODE_TC])
 def test_fused_decode_paths(V, M, K, B, path):
