@@ -87,6 +87,18 @@ def workload_config(w, codes="u16"):
     }
 
 
+def headline_layout(w, codes=None, available=("sched", "u16", "u8")):
+    """Code layout timed for `value` (both arms name it in `config`): 10-bit
+    packed workloads are packed; otherwise --codes if given, else the
+    bank-scheduled layout at B <= 4 and the drawn uint16 layout for batches
+    (whose full token groups decode rows on the tensor cores)."""
+    if w.packed10:
+        return "packed10"
+    if codes in available:
+        return codes
+    return "sched" if w.B <= 4 else "u16"
+
+
 def code_bytes(w, codes="u16"):
     if w.packed10:
         return w.V * (w.P * 10 // 8)
@@ -273,7 +285,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic", "config": workload_config(w, headline_layout(w, args.codes)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"{nrows} of {w.V} rows per step, {w.B} token(s)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -376,8 +388,7 @@ def run_ours(args, w):
         layouts["u16"] = (rq.U16, c16, None)
         if w.K <= 256:                 # one byte per code
             layouts["u8"] = (rq.U8, rq.rq_pack8(c16, d), None)
-        default = "sched" if w.B <= 4 else "u16"
-        headline = args.codes if args.codes in layouts else default
+        headline = headline_layout(w, args.codes, tuple(layouts))
 
     def make_step(fmt, codes, out=None):
         ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
