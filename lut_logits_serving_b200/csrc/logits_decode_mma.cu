@@ -23,9 +23,10 @@
 // Measured against fp64 this keeps the logits near 1e-6 of their scale; one
 // chain over all 384 subspaces was ~3e-5.
 //
-// Design for sm_100a (ds = 6, L = 2, uint16 codes, K <= 1024, 32 tokens).
-// One CTA per SM walks an even share of the vocabulary in passes of up to
-// 512 rows = 4 M = 128 tiles, running every subspace once per pass.
+// Design for sm_100a (ds = 6, L = 2, K <= 1024), described below for groups
+// of 32 tokens and uint16 codes; DmShape gives the 64-token and 10-bit packed
+// instances.  One CTA per SM walks an even share of the vocabulary in passes
+// of up to 512 rows = 4 M = 128 tiles, running every subspace once per pass.
 // Warp-specialised and mbarrier-driven, nothing waits on a CTA barrier:
 //   * 16 decoder warps (4 warpgroups).  Thread (warpgroup g, warp q, lane)
 //     owns row 32 q + lane of tile g.  Per subspace it gathers the row's two
@@ -33,7 +34,7 @@
 //     into hi and lo and stores both (6 dims + 2 zero pads each) into its own
 //     TMEM lane of a double-buffered A slot with one tcgen05.st: the MMA reads
 //     its A operand from tensor memory;
-//   * one copy warp: TMA code tiles ({8 codes, 256 rows}, 3 stages of 4
+//   * one copy warp: TMA code tiles ({8 codes, 128 rows}, 3 stages of 4
 //     subspaces), and per subspace one bulk copy of the codebook pair (48 KB
 //     at K = 1024, double-buffered) plus the pre-split hidden operand (2 KB,
 //     4-slot ring) on the same barrier, which the decoders wait for;
