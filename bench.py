@@ -35,6 +35,8 @@ from lut_logits_serving_b200 import synth  # noqa: E402
 METRIC = "LUT logits vocab-rows/s & µs/call at V=256000 (1 B200), % of HBM roofline"
 UNIT = "vocab-rows/s"
 ENC_METRIC = "RQ encode rows/s (greedy residual nearest codeword, fp32), % of FP32-pipe roofline"
+DEC_METRIC = "input rows rebuilt/s (bf16, Zipf ids, L2 flushed between calls), % of HBM roofline"
+DEC_UNIT = "rows/s"
 ENC_UNIT = "rows/s"
 # FP32 pipe: 148 SMs x 128 lanes per clock (B200); the clock is the sampled
 # maximum (clocks.max.sm), 1965 MHz when no sample exists.
@@ -49,7 +51,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="g2_b1",
                     choices=["g2_b1", "g2_b32", "packed_b64", "mlp_gate_b1", "mlp_down_b1",
-                             "encode_g2", "g2_b1_topk50"])
+                             "encode_g2", "g2_b1_topk50", "decode512"])
     ap.add_argument("--codes", default=None, choices=["u16", "sched", "u8"],
                     help="code layout of the unpacked workloads timed for `value`: "
                          "bank-scheduled once by rq_prepare_sched (the default at B <= 4), as "
@@ -250,6 +252,44 @@ def run_reference_encode(args, w):
     print(json.dumps(line), flush=True)
 
 
+def decode_config(w):
+    return {"workload": f"{w.name}: {w.n_ids} ids drawn Zipf(s={w.zipf_s:g}) over V={w.V} rows "
+                        f"(repeats kept), each rebuilt from M={w.M} x L={w.L} uint16 codes and "
+                        f"K={w.K} codebooks, x {w.decode_scale:g}, bf16 rows of D={w.D}",
+            "V": w.V, "D": w.D, "M": w.M, "L": w.L, "K": w.K, "ids": w.n_ids,
+            "l2": "inputs smaller than L2: a 256 MB buffer is written between timed calls"}
+
+
+def decode_bytes(w):
+    """Bytes a call touches: each id's code row, its L codewords per subspace
+    and its bf16 output row (repeated ids counted again)."""
+    return w.n_ids * (w.P * 2 + w.P * w.ds * 4 + w.D * 2)
+
+
+def run_reference_decode(args, w):
+    import oracle
+    data = synth.make(w)
+    ids, codes, C = data["ids"], data["codes"], data["C"]
+    for _ in range(args.warmup):
+        oracle.decode_rows_bf16(ids, codes, C, w.decode_scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.decode_rows_bf16(ids, codes, C, w.decode_scale)
+    el = time.perf_counter() - t0
+    value = w.n_ids * args.steps / el
+    line = {
+        "impl": "reference", "metric": DEC_METRIC, "value": value, "unit": DEC_UNIT,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": decode_config(w),
+        "cpu_baseline": {"value": value, "unit": DEC_UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"all {w.n_ids} ids per step"},
+        "e2e": {"value": value, "unit": DEC_UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def encode_config(w):
     return {"workload": f"{w.name}: encode V={w.V} rows of D={w.D} fp32 against M={w.M} x "
                         f"L={w.L} codebooks of K={w.K} ({w.ds}-dim) codewords -> uint16 codes",
@@ -263,6 +303,8 @@ def run_reference(args, w):
         return
     if w.encode:
         return run_reference_encode(args, w)
+    if w.B == 0:
+        return run_reference_decode(args, w)
     data = synth.make(w)
     step = oracle_step_fn(w, data)
     # size each step's row sample so that warmup + steps end within ~2 minutes
@@ -805,6 +847,146 @@ def run_encode(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args, w):
+    """Rebuild the bf16 input rows of a step's ids (decode512): each call
+    timed alone by its own events, with the L2 written over in between."""
+    import torch
+    import torch.distributed as dist
+
+    import lut_logits_serving_b200 as rq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    data = synth.make(w, seed=rank_seed(rank))
+    d = rq.dims(w.V, w.D, w.M, w.L, w.K)
+    ids = torch.from_numpy(data["ids"]).cuda()
+    codes = torch.from_numpy(data["codes"].reshape(w.V, -1)).cuda()
+    C = torch.from_numpy(data["C"]).cuda()
+    rows = torch.empty((w.n_ids, w.D), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        rq.rq_decode_rows(ids, codes, rq.U16, C, d, w.decode_scale, out=rows)
+
+    def timed(fn, n, cold):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n if cold else 1)]
+        if cold:
+            for a0, a1 in evs:
+                flush.fill_(1)
+                a0.record(stream)
+                fn()
+                a1.record(stream)
+        else:
+            evs[0][0].record(stream)
+            for _ in range(n):
+                fn()
+            evs[0][1].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return aggregate(sum(a0.elapsed_time(a1) for a0, a1 in evs), world, device="cuda")
+
+    def graphed(calls):
+        """`calls` back-to-back decode calls as one CUDA graph (a call is a
+        few microseconds, shorter than a Python launch)."""
+        s2 = torch.cuda.Stream()
+        s2.wait_stream(stream)
+        with torch.cuda.stream(s2):
+            step()
+        stream.wait_stream(s2)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(calls):
+                step()
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    burst = 20
+    g1, gb = (None, None) if args.no_graph else (graphed(1), graphed(burst))
+    with ClockSampler(local) as clk:
+        t_ms = timed(step if g1 is None else g1.replay, args.steps, True)
+    if gb is None:
+        warm_ms = timed(step, args.steps, False)
+    else:
+        reps = max(1, args.steps // burst)
+        warm_ms = timed(gb.replay, reps, False) * args.steps / (reps * burst)
+    value = throughput(w.n_ids * args.steps, world, t_ms)
+    want = None
+    if rank == 0:
+        import oracle
+        want = oracle.decode_rows_bf16(data["ids"], data["codes"], data["C"], w.decode_scale)
+        assert np.array_equal(rows.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    assert rq.rq_device_error() == 0
+    peak, peak_kind = load_peaks()
+    kern_s = t_ms / args.steps / 1e3
+    nbytes = decode_bytes(w)
+    achieved = nbytes / kern_s / 1e9
+
+    # end to end: ids in from pinned host memory, rows back to the host
+    idh = torch.from_numpy(data["ids"]).pin_memory()
+    rh = torch.empty((w.n_ids, w.D), dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        ids.copy_(idh, non_blocking=True)
+        step() if g1 is None else g1.replay()
+        rh.copy_(rows, non_blocking=True)
+
+    e2e_step()
+    e_ms = timed(e2e_step, args.steps, True)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        n, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < min(args.cpu_seconds, 5.0):
+            oracle.decode_rows_bf16(data["ids"], data["codes"], data["C"], w.decode_scale)
+            n += w.n_ids
+        el = time.perf_counter() - t0
+        cpu = {"value": n / el, "unit": DEC_UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{n // w.n_ids} calls of {w.n_ids} ids, single-threaded C, {el:.1f} s"}
+    launch = "eager" if g1 is None else "cuda graph"
+    del g1, gb
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": DEC_METRIC, "value": value, "unit": DEC_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+        "us_per_call": t_ms / args.steps * 1e3, "us_per_call_warm": warm_ms / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": dict(decode_config(w), parallelism=f"replicas x{world}",
+                                            launch=launch),
+        "roofline": {"bound": "hbm", "kernel": "decode_rows_pair_kernel", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "algorithmic_bytes": nbytes, "kernel_us": kern_s * 1e6},
+        "cpu_baseline": cpu,
+        "e2e": {"value": throughput(w.n_ids * args.steps, world, e_ms), "unit": DEC_UNIT,
+                "h2d_bytes_per_step": w.n_ids * 4, "d2h_bytes_per_step": w.n_ids * w.D * 2,
+                "ms_per_step": e_ms / args.steps},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
@@ -812,6 +994,8 @@ def main():
         run_reference(args, w)
     elif w.encode:
         run_encode(args, w)
+    elif w.B == 0:
+        run_decode(args, w)
     else:
         run_ours(args, w)
 

@@ -39,6 +39,49 @@ __global__ void __launch_bounds__(128) decode_rows_kernel(const int32_t *__restr
   decode_subspace<DS>(a, id, m, orow);
 }
 
+// ds = 6 rows, three threads per (row, subspace): thread q of subspace m
+// rebuilds elements 2q and 2q+1.  A warp then spans about eleven subspaces, so
+// each float2 codeword load touches about eleven lines instead of one per
+// lane, and the bf16 pairs leave as coalesced 4-byte stores.  The element
+// arithmetic is that of decode_subspace: level sum from 0 in l order, then
+// the scale, then bf16 round to nearest even.
+constexpr int kPairSub = 128;   // subspaces per block
+
+__global__ void __launch_bounds__(3 * kPairSub) decode_rows_pair_kernel(
+    const int32_t *__restrict__ ids, const DecodeSpec a, uint32_t *__restrict__ out,
+    unsigned *err) {
+  griddep_launch_dependents();
+  griddep_wait();   // the ids may be the argmax the previous kernel wrote
+  const int64_t n = blockIdx.x;
+  const int t = blockIdx.y * (3 * kPairSub) + threadIdx.x;
+  const int m = t / 3, q = t - 3 * m;
+  if (m >= a.M) return;
+  const int32_t id = ids[n];
+  uint32_t *o = out + n * (int64_t)(3 * a.M) + t;
+  if (id < 0 || (int64_t)id >= a.V) {
+    *o = 0u;
+    if (t == 0) atomicOr(err, RQ_DEVERR_BAD_ID);
+    return;
+  }
+  const int P = a.M * a.L;
+  const uint16_t *all16 = static_cast<const uint16_t *>(a.codes);
+  float e0 = 0.f, e1 = 0.f;
+  for (int l = 0; l < a.L; ++l) {
+    const int p = m * a.L + l;
+    uint32_t c;
+    if (a.fmt == RQ_CODES_U16) c = all16[(int64_t)id * P + p];
+    else if (a.fmt == RQ_CODES_SCHED) c = sched_code(all16, a.V, id, p, sched_shift(a.K));
+    else if (a.fmt == RQ_CODES_U8) c = static_cast<const uint8_t *>(a.codes)[(int64_t)id * P + p];
+    else c = packed10_code(static_cast<const uint8_t *>(a.codes) + (int64_t)id * ((10LL * P + 7) / 8), p);
+    const float2 w = __ldg(reinterpret_cast<const float2 *>(a.C + ((size_t)p * a.K + a.fix(c)) * 6) + q);
+    e0 = __fadd_rn(e0, w.x);
+    e1 = __fadd_rn(e1, w.y);
+  }
+  const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e0, a.scale)));
+  const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e1, a.scale)));
+  *o = lo | (hi << 16);
+}
+
 cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt,
                                const float *C, int64_t V, int D, int M, int L, int K,
                                float scale, uint16_t *out, unsigned *err, cudaStream_t s) {
@@ -56,6 +99,10 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
   a.K = K;
   a.scale = scale;
   a.fix = make_codefix(K);
+  if (D == 6 * M && ((uintptr_t)out & 3) == 0 && ((uintptr_t)C & 7) == 0)
+    return pdl_launch(decode_rows_pair_kernel,
+                      dim3((unsigned)N, (unsigned)((M + kPairSub - 1) / kPairSub)),
+                      dim3(3 * kPairSub), 0, s, ids, a, reinterpret_cast<uint32_t *>(out), err);
   if (D / M == 6) return pdl_launch(decode_rows_kernel<6>, grid, dim3(128), 0, s, ids, a, out, err);
   return pdl_launch(decode_rows_kernel<0>, grid, dim3(128), 0, s, ids, a, out, err);
 }

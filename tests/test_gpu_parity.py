@@ -216,6 +216,27 @@ def test_decode_rows_bit_exact(shape, fmt):
     assert np.array_equal(got, want)
 
 
+@pytest.mark.parametrize("shift_out,shift_C", [(0, 0), (1, 0), (0, 1)],
+                         ids=["aligned", "odd_out", "odd_C"])
+def test_decode_rows_ragged_subspace_blocks_and_odd_pointers(shift_out, shift_C):
+    """M = 200 spans two blocks of the pair kernel with a ragged second one;
+    an output 2 bytes off a 4-byte boundary, or codebooks 4 bytes off an
+    8-byte one, take the one-thread-per-subspace kernel, bit for bit alike."""
+    V, D, M, L, K = 3000, 1200, 200, 2, 512
+    C, codes, _ = make_case(V, D, M, L, K, 1, sigmas=(0.02, 0.005))
+    ids = synth.zipf_ids(129, V, 1.1, 5)
+    d = rq.dims(V, D, M, L, K)
+    cbuf = torch.empty(C.size + 1, dtype=torch.float32, device="cuda")
+    dC = cbuf[shift_C:shift_C + C.size].view(C.shape)
+    dC.copy_(dev(C))
+    obuf = torch.full((len(ids) * D + 1,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = obuf[shift_out:shift_out + len(ids) * D].view(len(ids), D)
+    rq.rq_decode_rows(dev(ids), dev(codes.reshape(V, -1)), rq.U16, dC, d, 7.0, out=out)
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, oracle.decode_rows_bf16(ids, codes, C, 7.0))
+    assert rq.rq_device_error() == 0
+
+
 def test_decode_rows_bad_ids_give_zero_rows_and_a_device_error():
     V, D, M, L, K = 100, 48, 8, 2, 16
     C, codes, _ = make_case(V, D, M, L, K, 1)
