@@ -349,7 +349,8 @@ def load_peaks():
 def kernel_source_hash(kernel="logits_chunk"):
     """Hash of the sources a kernel is built from (its .cu file and the common
     header), to tell whether committed ncu counters still describe it."""
-    src = "logits_decode_mma.cu" if kernel.startswith("logits_decode_mma") else "logits_chunk.cu"
+    src = ("logits_decode_mma.cu" if kernel.startswith("logits_decode_mma") else
+           "decode_rows.cu" if kernel.startswith("decode_rows") else "logits_chunk.cu")
     h = hashlib.sha256()
     for name in (src, "rq_common.cuh"):
         with open(os.path.join(ROOT, "lut_logits_serving_b200", "csrc", name), "rb") as f:
@@ -976,7 +977,8 @@ def run_decode(args, w):
                                             launch=launch),
         "roofline": {"bound": "hbm", "kernel": "decode_rows_pair_kernel", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "algorithmic_bytes": nbytes, "kernel_us": kern_s * 1e6},
+                     "traffic": profiled_traffic("decode_rows_pair_kernel/u16/decode512"),
+                     "algorithmic_bytes": nbytes, "kernel_us": kern_s * 1e6},
         "cpu_baseline": cpu,
         "e2e": {"value": throughput(w.n_ids * args.steps, world, e_ms), "unit": DEC_UNIT,
                 "h2d_bytes_per_step": w.n_ids * 4, "d2h_bytes_per_step": w.n_ids * w.D * 2,
