@@ -42,44 +42,97 @@ __global__ void __launch_bounds__(128) decode_rows_kernel(const int32_t *__restr
 // ds = 6 rows, three threads per (row, subspace): thread q of subspace m
 // rebuilds elements 2q and 2q+1.  A warp then spans about eleven subspaces, so
 // each float2 codeword load touches about eleven lines instead of one per
-// lane, and the bf16 pairs leave as coalesced 4-byte stores.  The element
-// arithmetic is that of decode_subspace: level sum from 0 in l order, then
-// the scale, then bf16 round to nearest even.
+// lane, and the bf16 pairs leave as coalesced 4-byte stores.  Each thread
+// takes R consecutive rows and issues their loads together: the launch picks
+// R = 1 or 2 when that grid is resident in one wave, else 4, so the
+// id -> code -> codeword round trips are paid once per wave of R rows.  The
+// element arithmetic is that of decode_subspace: level sum from 0 in l order,
+// then the scale, then bf16 round to nearest even.
 constexpr int kPairSub = 128;   // subspaces per block
 
+template <int R>
 __global__ void __launch_bounds__(3 * kPairSub) decode_rows_pair_kernel(
-    const int32_t *__restrict__ ids, const DecodeSpec a, uint32_t *__restrict__ out,
+    const int32_t *__restrict__ ids, int64_t N, const DecodeSpec a, uint32_t *__restrict__ out,
     unsigned *err) {
   griddep_launch_dependents();
   griddep_wait();   // the ids may be the argmax the previous kernel wrote
-  const int64_t n = blockIdx.x;
+  const int64_t n0 = (int64_t)blockIdx.x * R;
   const int t = blockIdx.y * (3 * kPairSub) + threadIdx.x;
   const int m = t / 3, q = t - 3 * m;
   if (m >= a.M) return;
-  const int32_t id = ids[n];
-  uint32_t *o = out + n * (int64_t)(3 * a.M) + t;
-  if (id < 0 || (int64_t)id >= a.V) {
-    *o = 0u;
-    if (t == 0) atomicOr(err, RQ_DEVERR_BAD_ID);
-    return;
-  }
   const int P = a.M * a.L;
+  const int64_t rb10 = (10LL * P + 7) / 8;
   const uint16_t *all16 = static_cast<const uint16_t *>(a.codes);
-  float e0 = 0.f, e1 = 0.f;
+  const uint8_t *all8 = static_cast<const uint8_t *>(a.codes);
+  int32_t id[R];
+  uint32_t ok = 0u;   // bit r: row n0 + r exists and its id is in [0, V)
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const bool in = n0 + r < N;
+    const int32_t v = in ? ids[n0 + r] : 0;
+    const bool good = in && v >= 0 && (int64_t)v < a.V;
+    ok |= (uint32_t)good << r;
+    id[r] = good ? v : 0;
+    if (in && !good && t == 0) atomicOr(err, RQ_DEVERR_BAD_ID);
+  }
+  float e0[R], e1[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) e0[r] = e1[r] = 0.f;
   for (int l = 0; l < a.L; ++l) {
     const int p = m * a.L + l;
-    uint32_t c;
-    if (a.fmt == RQ_CODES_U16) c = all16[(int64_t)id * P + p];
-    else if (a.fmt == RQ_CODES_SCHED) c = sched_code(all16, a.V, id, p, sched_shift(a.K));
-    else if (a.fmt == RQ_CODES_U8) c = static_cast<const uint8_t *>(a.codes)[(int64_t)id * P + p];
-    else c = packed10_code(static_cast<const uint8_t *>(a.codes) + (int64_t)id * ((10LL * P + 7) / 8), p);
-    const float2 w = __ldg(reinterpret_cast<const float2 *>(a.C + ((size_t)p * a.K + a.fix(c)) * 6) + q);
-    e0 = __fadd_rn(e0, w.x);
-    e1 = __fadd_rn(e1, w.y);
+    uint32_t c[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      c[r] = 0u;
+      if (ok >> r & 1u) {
+        const int64_t v = id[r];
+        if (a.fmt == RQ_CODES_U16) c[r] = all16[v * P + p];
+        else if (a.fmt == RQ_CODES_SCHED) c[r] = sched_code(all16, a.V, v, p, sched_shift(a.K));
+        else if (a.fmt == RQ_CODES_U8) c[r] = all8[v * P + p];
+        else c[r] = packed10_code(all8 + v * rb10, p);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (ok >> r & 1u) {
+        const float2 w =
+            __ldg(reinterpret_cast<const float2 *>(a.C + ((size_t)p * a.K + a.fix(c[r])) * 6) + q);
+        e0[r] = __fadd_rn(e0[r], w.x);
+        e1[r] = __fadd_rn(e1[r], w.y);
+      }
+    }
   }
-  const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e0, a.scale)));
-  const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e1, a.scale)));
-  *o = lo | (hi << 16);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (n0 + r >= N) break;
+    uint32_t v = 0u;
+    if (ok >> r & 1u) {
+      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e0[r], a.scale)));
+      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e1[r], a.scale)));
+      v = lo | (hi << 16);
+    }
+    out[(n0 + r) * (int64_t)(3 * a.M) + t] = v;
+  }
+}
+
+template <int R>
+cudaError_t launch_pair(const int32_t *ids, int64_t N, const DecodeSpec &a, uint16_t *out,
+                        unsigned *err, cudaStream_t s) {
+  const int64_t gx = (N + R - 1) / R;
+  if (gx > 0x7fffffffLL) return cudaErrorInvalidValue;
+  return pdl_launch(decode_rows_pair_kernel<R>,
+                    dim3((unsigned)gx, (unsigned)((a.M + kPairSub - 1) / kPairSub)),
+                    dim3(3 * kPairSub), 0, s, ids, N, a, reinterpret_cast<uint32_t *>(out), err);
+}
+
+// Whether the grid of R rows per thread is resident in one wave.
+template <int R>
+bool pair_fits(int64_t N, int M, int sms) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_rows_pair_kernel<R>,
+                                                    3 * kPairSub, 0) != cudaSuccess)
+    return false;
+  return (N + R - 1) / R * ((M + kPairSub - 1) / kPairSub) <= (int64_t)per_sm * sms;
 }
 
 cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt,
@@ -99,10 +152,15 @@ cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes,
   a.K = K;
   a.scale = scale;
   a.fix = make_codefix(K);
-  if (D == 6 * M && ((uintptr_t)out & 3) == 0 && ((uintptr_t)C & 7) == 0)
-    return pdl_launch(decode_rows_pair_kernel,
-                      dim3((unsigned)N, (unsigned)((M + kPairSub - 1) / kPairSub)),
-                      dim3(3 * kPairSub), 0, s, ids, a, reinterpret_cast<uint32_t *>(out), err);
+  if (D == 6 * M && ((uintptr_t)out & 3) == 0 && ((uintptr_t)C & 7) == 0) {
+    DevInfo di;
+    const int sms = dev_info(&di) == cudaSuccess ? di.sms : 148;
+    (void)cudaGetLastError();
+    if (pair_fits<1>(N, M, sms)) return launch_pair<1>(ids, N, a, out, err, s);
+    if (pair_fits<2>(N, M, sms)) return launch_pair<2>(ids, N, a, out, err, s);
+    (void)cudaGetLastError();
+    return launch_pair<4>(ids, N, a, out, err, s);
+  }
   if (D / M == 6) return pdl_launch(decode_rows_kernel<6>, grid, dim3(128), 0, s, ids, a, out, err);
   return pdl_launch(decode_rows_kernel<0>, grid, dim3(128), 0, s, ids, a, out, err);
 }

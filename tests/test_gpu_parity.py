@@ -237,6 +237,27 @@ def test_decode_rows_ragged_subspace_blocks_and_odd_pointers(shift_out, shift_C)
     assert rq.rq_device_error() == 0
 
 
+@pytest.mark.parametrize("N", [389, 1003])
+def test_decode_rows_several_rows_per_thread(N):
+    """At D = 2304, M = 384, 389 ids take two rows per thread and 1003 ids four
+    (the grid of one row per thread would not be resident in one wave), with a
+    ragged last block and bad ids inside a thread's group of rows."""
+    V, D, M, L, K = 700, 2304, 384, 2, 1024
+    C, codes, _ = make_case(V, D, M, L, K, 1, sigmas=(0.02, 0.005))
+    ids = synth.zipf_ids(N, V, 1.1, 11)
+    bad = [5, N // 2, N - 1]
+    ids[bad] = [-3, V, V + 1000]
+    d = rq.dims(V, D, M, L, K)
+    rq.rq_device_error(clear=True)
+    out = torch.full((N, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    rq.rq_decode_rows(dev(ids), dev(codes.reshape(V, -1)), rq.U16, dev(C), d, 48.0, out=out)
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    good = np.setdiff1d(np.arange(N), bad)
+    assert np.all(got[bad] == 0)
+    assert np.array_equal(got[good], oracle.decode_rows_bf16(ids[good], codes, C, 48.0))
+    assert rq.rq_device_error(clear=True) == 2
+
+
 def test_decode_rows_bad_ids_give_zero_rows_and_a_device_error():
     V, D, M, L, K = 100, 48, 8, 2, 16
     C, codes, _ = make_case(V, D, M, L, K, 1)
