@@ -241,10 +241,15 @@ RQ_API int rq_greedy_step(const float *h, const float *C, const void *codes, int
  *   ids    (device) int32 [N]; ids outside [0, V) give zero rows and set
  *          RQ_DEVERR_BAD_ID
  *   codes  (device) as for rq_lut_logits (2-byte aligned; 16-byte for
- *          RQ_CODES_SCHED); C (device) float [M][L][K][ds]
+ *          RQ_CODES_SCHED); C (device) float [M][L][K][ds], 4-byte aligned
  *   out    (device) uint16 [N][D] bf16 bit patterns, 2-byte aligned
- *   N = 0 is a no-op.
- * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ *   N = 0 is a no-op.  With ds = 6, out 4-byte aligned and C 8-byte
+ *   aligned, three threads share a (row, subspace) and each thread takes up
+ *   to four rows; otherwise one thread per (row, subspace).  The results are
+ *   the same bits either way.
+ * Errors: RQ_ERR_INVALID_ARGUMENT (null pointer, N < 0, bad dims or format),
+ * RQ_ERR_UNSUPPORTED (the format cannot hold the shape), RQ_ERR_MISALIGNED,
+ * RQ_ERR_CUDA.
  */
 RQ_API int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt,
                    const float *C, rq_dims d, float scale, uint16_t *out,

@@ -130,6 +130,11 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_decode_rows(a, -1, a, 0, a, G2, 48.0, a, s) == INV
     assert lib.rq_decode_rows(null, 0, null, 0, null, G2, 48.0, null, s) == 0   # N = 0: no-op
     assert lib.rq_decode_rows(_fake(0x10002), 5, a, 0, a, G2, 48.0, a, s) == MIS
+    assert lib.rq_decode_rows(a, 5, a, 9, a, G2, 48.0, a, s) == INV            # unknown format
+    assert lib.rq_decode_rows(a, 5, a, 3, a, G2, 48.0, a, s) == UNS            # u8 codes, K > 256
+    assert lib.rq_decode_rows(a, 5, a, 0, _fake(0x10002), G2, 48.0, a, s) == MIS  # C 4-B
+    assert lib.rq_decode_rows(a, 5, a, 0, a, G2, 48.0, _fake(0x10001), s) == MIS  # out 2-B
+    assert lib.rq_decode_rows(a, 5, _fake(0x10008), 2, a, G2, 48.0, a, s) == MIS  # sched 16-B
     assert lib.rq_pack10(null, G2, a, s) == INV
     assert lib.rq_pack8(a, G2, a, s) == UNS                                   # K > 256
     assert lib.rq_prepare_sched(null, G2, a, null, s) == INV
