@@ -142,7 +142,10 @@ RQ_API size_t rq_fused_workspace_bytes(rq_dims d, int B, int fmt, int want_argma
  *   lut (device) float, rq_lut_bytes(d, B) bytes, 16-byte aligned; padding
  *       tokens b in [B, Bs) are written as 0.
  * Errors: RQ_ERR_INVALID_ARGUMENT (null, B < 1, bad dims),
- *         RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ *         RQ_ERR_MISALIGNED, RQ_ERR_UNSUPPORTED (one subspace's slice of
+ *         all Bs padded tokens, Bs * ds floats, above 48 KB of shared
+ *         memory; token groups go through rq_logits_from_hidden),
+ *         RQ_ERR_CUDA.
  */
 RQ_API int rq_lut_build(const float *h, const float *C, rq_dims d, int B, float *lut,
                  void *stream);
@@ -259,8 +262,9 @@ RQ_API int rq_decode_rows(const int32_t *ids, int64_t N, const void *codes, int 
  * rq_pack10 -- convert uint16 codes [V][M*L] (values < 1024) into the
  * PACKED10 layout above (the 10-bit storage implied by the 3.59 bits/param
  * figure of the combined RQ+NF4 page).  Codes >= 1024 keep their low 10
- * bits.  packed (device) uint8 [V][rb], rb = ceil(10*M*L/8).
- * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_CUDA.
+ * bits.  codes_u16 (device) 2-byte aligned; packed (device) uint8 [V][rb],
+ * rb = ceil(10*M*L/8).
+ * Errors: RQ_ERR_INVALID_ARGUMENT, RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
  */
 RQ_API int rq_pack10(const uint16_t *codes_u16, rq_dims d, uint8_t *packed,
               void *stream);
@@ -385,6 +389,7 @@ RQ_API int rq_argmax_merge(const float *val, const int32_t *gidx, int n, int B, 
  * rq_device_error -- read (and, if `clear`, reset) the device error word
  * of the current device.  Synchronous: call after synchronizing the streams
  * that ran the kernels of interest.  *out receives RQ_DEVERR_* bits.
+ * Errors: RQ_ERR_INVALID_ARGUMENT (out NULL), RQ_ERR_CUDA.
  */
 RQ_API int rq_device_error(uint32_t *out, int clear);
 

@@ -110,6 +110,7 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_lut_build(a, a, G2, 0, a, s) == INV
     assert lib.rq_lut_build(a, a, rq.dims(10, 7, 2, 1, 4), 1, a, s) == INV   # D % M != 0
     assert lib.rq_lut_build(a, a, G2, 1, odd, s) == MIS                     # lut 16-B
+    assert lib.rq_lut_build(a, a, G2, 4096, a, s) == UNS                    # 4096 x 6 floats > 48 KB
     assert lib.rq_lut_logits(a, 0, G2, a, 1, 30.0, null, null, null, 0, s) == INV
     assert lib.rq_lut_logits(a, 7, G2, a, 1, 30.0, a, null, null, 0, s) == INV
     assert lib.rq_lut_logits(a, 1, rq.dims(10, 8, 4, 2, 2048), a, 1, 30.0, a, null, null, 0,
@@ -136,6 +137,8 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_decode_rows(a, 5, a, 0, a, G2, 48.0, _fake(0x10001), s) == MIS  # out 2-B
     assert lib.rq_decode_rows(a, 5, _fake(0x10008), 2, a, G2, 48.0, a, s) == MIS  # sched 16-B
     assert lib.rq_pack10(null, G2, a, s) == INV
+    assert lib.rq_pack10(_fake(0x10001), G2, a, s) == MIS
+    assert lib.rq_device_error(null, 0) == INV
     assert lib.rq_pack8(a, G2, a, s) == UNS                                   # K > 256
     assert lib.rq_prepare_sched(null, G2, a, null, s) == INV
     assert lib.rq_prepare_sched(a, rq.dims(10, 48, 24, 1, 64), _fake(0x900000), null, s) == UNS
