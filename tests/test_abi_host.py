@@ -138,7 +138,7 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rq_decode_rows(a, 5, _fake(0x10008), 2, a, G2, 48.0, a, s) == MIS  # sched 16-B
     assert lib.rq_pack10(null, G2, a, s) == INV
     assert lib.rq_pack10(_fake(0x10001), G2, a, s) == MIS
-    assert lib.rq_device_error(null, 0) == INV
+    assert lib.rq_device_error(ctypes.POINTER(ctypes.c_uint32)(), 0) == INV   # out NULL
     assert lib.rq_pack8(a, G2, a, s) == UNS                                   # K > 256
     assert lib.rq_prepare_sched(null, G2, a, null, s) == INV
     assert lib.rq_prepare_sched(a, rq.dims(10, 48, 24, 1, 64), _fake(0x900000), null, s) == UNS
