@@ -19,6 +19,7 @@ There is no CPU fallback: if the library or a GPU is missing, calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -169,21 +170,46 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _cuda(t, dtype, name):
+def _cuda(t, dtype, name, nbytes=None):
+    """Device pointer of `t` after checking its type, layout and, with
+    `nbytes`, that it holds at least that many bytes: the C calls take bare
+    pointers, so a short buffer would otherwise be read or written past its
+    end."""
     torch = _torch()
     if not isinstance(t, torch.Tensor):
         raise ValueError(f"{name}: expected a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name}: must be a CUDA tensor (no CPU fallback)")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name}: must be contiguous")
+    if nbytes is not None and t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name}: {t.numel() * t.element_size()} bytes, "
+                         f"the call needs {nbytes}")
+    if not _on_device(t):
+        raise ValueError(f"{name}: must be a CUDA tensor (no CPU fallback)")
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _ptr_or_null(t, dtype, name):
-    return ctypes.c_void_p(None) if t is None else _cuda(t, dtype, name)
+def _on_device(t):
+    return t.is_cuda
+
+
+def _ptr_or_null(t, dtype, name, nbytes=None):
+    return ctypes.c_void_p(None) if t is None else _cuda(t, dtype, name, nbytes)
+
+
+def _book_bytes(d):
+    """Bytes of the codebooks C [M, L, K, ds] (fp32)."""
+    return d.M * d.L * d.K * (d.D // d.M if d.M > 0 else 0) * 4
+
+
+def _tokens(h, d, name="h"):
+    """B of hidden states h [B, D] (or [D] for one token)."""
+    if h.dim() == 1 and h.shape[0] == d.D:
+        return 1
+    if h.dim() != 2 or h.shape[1] != d.D:
+        raise ValueError(f"{name}: shape {tuple(h.shape)}, expected [B, {d.D}]")
+    return h.shape[0]
 
 
 def _check(fn, status):
@@ -213,13 +239,13 @@ def _workspace(nbytes, like, ws):
 def rq_lut_build(h, C, d: RqDims, lut=None, stream=None):
     """h float32 [B, D], C float32 [M, L, K, ds] -> lut float32 [P, K, Bs]."""
     torch = _torch()
-    B = h.shape[0] if h.dim() == 2 else 1
+    B = _tokens(h, d)
     Bs = rq_lut_token_stride(B)
     if lut is None:
         lut = _empty((d.M * d.L, d.K, Bs), torch.float32, h)
     _check("rq_lut_build", lib().rq_lut_build(
-        _cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C"), d, B,
-        _cuda(lut, torch.float32, "lut"), _stream(stream)))
+        _cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C", _book_bytes(d)), d, B,
+        _cuda(lut, torch.float32, "lut", rq_lut_bytes(d, B)), _stream(stream)))
     return lut
 
 
@@ -235,9 +261,10 @@ def rq_lut_logits(codes, fmt: int, d: RqDims, lut, B: int, softcap: float = 30.0
     nbytes = rq_logits_workspace_bytes(d, B, fmt, argmax is not None)
     wp, wn, ws = _workspace(nbytes, lut, ws)
     _check("rq_lut_logits", lib().rq_lut_logits(
-        _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, _cuda(lut, torch.float32, "lut"), B,
-        float(softcap), _ptr_or_null(logits, torch.float32, "logits"),
-        _ptr_or_null(argmax, torch.int32, "argmax"), wp, wn, _stream(stream)))
+        _cuda(codes, _codes_dtype(fmt), "codes", rq_codes_bytes(d, fmt)), fmt, d,
+        _cuda(lut, torch.float32, "lut", rq_lut_bytes(d, B)), B,
+        float(softcap), _ptr_or_null(logits, torch.float32, "logits", B * d.V * 4),
+        _ptr_or_null(argmax, torch.int32, "argmax", B * 4), wp, wn, _stream(stream)))
     return logits, argmax, ws
 
 
@@ -248,17 +275,17 @@ def rq_logits_from_hidden(h, C, codes, fmt: int, d: RqDims, softcap: float = 30.
     ``path`` (one of PATH_*) picks the kernel of full 32-token groups; None
     is the library's default (rq_logits_from_hidden)."""
     torch = _torch()
-    B = h.shape[0]
+    B = _tokens(h, d)
     if want_logits and logits is None:
         logits = _empty((B, d.V), torch.float32, h)
     if want_argmax and argmax is None:
         argmax = _empty((B,), torch.int32, h)
     nbytes = rq_fused_workspace_bytes(d, B, fmt, argmax is not None)
     wp, wn, ws = _workspace(nbytes, h, ws)
-    args = (_cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C"),
-            _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, B, float(softcap),
-            _ptr_or_null(logits, torch.float32, "logits"),
-            _ptr_or_null(argmax, torch.int32, "argmax"), wp, wn)
+    args = (_cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C", _book_bytes(d)),
+            _cuda(codes, _codes_dtype(fmt), "codes", rq_codes_bytes(d, fmt)), fmt, d, B,
+            float(softcap), _ptr_or_null(logits, torch.float32, "logits", B * d.V * 4),
+            _ptr_or_null(argmax, torch.int32, "argmax", B * 4), wp, wn)
     if path is None:
         _check("rq_logits_from_hidden", lib().rq_logits_from_hidden(*args, _stream(stream)))
     else:
@@ -277,15 +304,17 @@ def rq_argmax_candidates(logits, argmax, row0: int, val=None, gidx=None, stream=
     """A vocabulary shard's winner per token: (value float32 [B], global row
     int32 [B]) from its logits [B, V_shard] and argmax [B]."""
     torch = _torch()
+    if logits.dim() != 2:
+        raise ValueError("logits: [B, V_shard] expected")
     B, V = logits.shape
     if val is None:
         val = _empty((B,), torch.float32, logits)
     if gidx is None:
         gidx = _empty((B,), torch.int32, logits)
     _check("rq_argmax_candidates", lib().rq_argmax_candidates(
-        _cuda(logits, torch.float32, "logits"), _cuda(argmax, torch.int32, "argmax"), B, V,
-        int(row0), _cuda(val, torch.float32, "val"), _cuda(gidx, torch.int32, "gidx"),
-        _stream(stream)))
+        _cuda(logits, torch.float32, "logits"), _cuda(argmax, torch.int32, "argmax", B * 4),
+        B, V, int(row0), _cuda(val, torch.float32, "val", B * 4),
+        _cuda(gidx, torch.int32, "gidx", B * 4), _stream(stream)))
     return val, gidx
 
 
@@ -299,7 +328,7 @@ def rq_argmax_merge(val, gidx, out=None, stream=None):
         out = _empty((B,), torch.int32, val)
     _check("rq_argmax_merge", lib().rq_argmax_merge(
         _cuda(val, torch.float32, "val"), _cuda(gidx, torch.int32, "gidx"), n, B,
-        _cuda(out, torch.int32, "argmax"), _stream(stream)))
+        _cuda(out, torch.int32, "argmax", B * 4), _stream(stream)))
     return out
 
 
@@ -325,11 +354,13 @@ def rq_sharded_logits(h, C, codes_shard, fmt: int, d_shard: RqDims, row0: int,
     if dist.is_available() and dist.is_initialized():
         world = dist.get_world_size(group)
     if world > 1:
-        # flat [world * B] buffers, rank-major (the layout every backend takes)
+        # flat [world * B] buffers, rank-major (the layout every backend takes);
+        # the collectives are ordered after the candidates on the call's stream
         vals = _empty((world * val.numel(),), torch.float32, val)
         idxs = _empty((world * gidx.numel(),), torch.int32, gidx)
-        dist.all_gather_into_tensor(vals, val, group=group)
-        dist.all_gather_into_tensor(idxs, gidx, group=group)
+        with torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext():
+            dist.all_gather_into_tensor(vals, val, group=group)
+            dist.all_gather_into_tensor(idxs, gidx, group=group)
         vals, idxs = vals.view(world, -1), idxs.view(world, -1)
     else:
         vals, idxs = val.view(1, -1), gidx.view(1, -1)
@@ -345,9 +376,10 @@ def rq_decode_rows(ids, codes, fmt: int, C, d: RqDims, scale: float, out=None, s
     if out.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
         raise ValueError("out: bf16 rows expected")
     _check("rq_decode_rows", lib().rq_decode_rows(
-        _cuda(ids, torch.int32, "ids"), N, _cuda(codes, _codes_dtype(fmt), "codes"), fmt,
-        _cuda(C, torch.float32, "C"), d, float(scale), _cuda(out, None, "out"),
-        _stream(stream)))
+        _cuda(ids, torch.int32, "ids"), N,
+        _cuda(codes, _codes_dtype(fmt), "codes", rq_codes_bytes(d, fmt)), fmt,
+        _cuda(C, torch.float32, "C", _book_bytes(d)), d, float(scale),
+        _cuda(out, None, "out", N * d.D * 2), _stream(stream)))
     return out
 
 
@@ -356,8 +388,9 @@ def rq_pack10(codes_u16, d: RqDims, out=None, stream=None):
     torch = _torch()
     if out is None:
         out = _empty((d.V, rq_codes_bytes(d, PACKED10) // d.V), torch.uint8, codes_u16)
-    _check("rq_pack10", lib().rq_pack10(_cuda(codes_u16, torch.uint16, "codes_u16"), d,
-                                        _cuda(out, torch.uint8, "packed"), _stream(stream)))
+    _check("rq_pack10", lib().rq_pack10(
+        _cuda(codes_u16, torch.uint16, "codes_u16", rq_codes_bytes(d, U16)), d,
+        _cuda(out, torch.uint8, "packed", rq_codes_bytes(d, PACKED10)), _stream(stream)))
     return out
 
 
@@ -367,9 +400,10 @@ def rq_encode(X, C, d: RqDims, out=None, stream=None):
     torch = _torch()
     if out is None:
         out = _empty((d.V, d.M * d.L), torch.uint16, X)
-    _check("rq_encode", lib().rq_encode(_cuda(X, torch.float32, "X"), d,
-                                        _cuda(C, torch.float32, "C"),
-                                        _cuda(out, torch.uint16, "codes"), _stream(stream)))
+    _check("rq_encode", lib().rq_encode(
+        _cuda(X, torch.float32, "X", d.V * d.D * 4), d,
+        _cuda(C, torch.float32, "C", _book_bytes(d)),
+        _cuda(out, torch.uint16, "codes", rq_codes_bytes(d, U16)), _stream(stream)))
     return out
 
 
@@ -391,6 +425,8 @@ def rq_topk_sample(logits, k: int, temperature: float = 1.0, seed: int = 0, step
     """logits float32 [B, V] (device) -> (topk_val [B, k], topk_idx [B, k], token [B]);
     the top-k outputs are None with want_topk=False."""
     torch = _torch()
+    if logits.dim() != 2:
+        raise ValueError("logits: [B, V] expected")
     B, V = logits.shape
     if want_topk:
         if topk_val is None:
@@ -404,9 +440,9 @@ def rq_topk_sample(logits, k: int, temperature: float = 1.0, seed: int = 0, step
     _check("rq_topk_sample", lib().rq_topk_sample(
         _cuda(logits, torch.float32, "logits"), V, B, k, float(temperature),
         ctypes.c_uint64(seed), ctypes.c_uint64(step),
-        _ptr_or_null(topk_val, torch.float32, "topk_val"),
-        _ptr_or_null(topk_idx, torch.int32, "topk_idx"),
-        _cuda(token, torch.int32, "token"), wsp, wsn, _stream(stream)))
+        _ptr_or_null(topk_val, torch.float32, "topk_val", B * k * 4),
+        _ptr_or_null(topk_idx, torch.int32, "topk_idx", B * k * 4),
+        _cuda(token, torch.int32, "token", B * 4), wsp, wsn, _stream(stream)))
     return topk_val, topk_idx, token
 
 
@@ -415,8 +451,9 @@ def rq_pack8(codes_u16, d: RqDims, out=None, stream=None):
     torch = _torch()
     if out is None:
         out = _empty((d.V, d.M * d.L), torch.uint8, codes_u16)
-    _check("rq_pack8", lib().rq_pack8(_cuda(codes_u16, torch.uint16, "codes_u16"), d,
-                                      _cuda(out, torch.uint8, "packed"), _stream(stream)))
+    _check("rq_pack8", lib().rq_pack8(
+        _cuda(codes_u16, torch.uint16, "codes_u16", rq_codes_bytes(d, U16)), d,
+        _cuda(out, torch.uint8, "packed", rq_codes_bytes(d, U8)), _stream(stream)))
     return out
 
 
@@ -443,8 +480,9 @@ def rq_prepare_sched(codes_u16, d: RqDims, out=None, stats=None, stream=None):
     if stats:
         st = torch.zeros(2, dtype=torch.int64, device=codes_u16.device)
     _check("rq_prepare_sched", lib().rq_prepare_sched(
-        _cuda(codes_u16, torch.uint16, "codes_u16"), d, _cuda(out, torch.uint16, "out"),
-        _ptr_or_null(st, torch.int64, "stats"), _stream(stream)))
+        _cuda(codes_u16, torch.uint16, "codes_u16", rq_codes_bytes(d, U16)), d,
+        _cuda(out, torch.uint16, "out", rq_codes_bytes(d, SCHED)),
+        _ptr_or_null(st, torch.int64, "stats", 16), _stream(stream)))
     if stats:
         v = st.cpu().tolist()
         return out, (v[0], v[1])
@@ -463,9 +501,10 @@ def rq_lut_logits_static(codes, fmt: int, d: RqDims, lut, B: int, softcap: float
     if want_argmax and argmax is None:
         argmax = _empty((B,), torch.int32, lut)
     _check("rq_lut_logits_static", lib().rq_lut_logits_static(
-        _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, _cuda(lut, torch.float32, "lut"), B,
-        float(softcap), _ptr_or_null(logits, torch.float32, "logits"),
-        _ptr_or_null(argmax, torch.int32, "argmax"), _stream(stream)))
+        _cuda(codes, _codes_dtype(fmt), "codes", rq_codes_bytes(d, fmt)), fmt, d,
+        _cuda(lut, torch.float32, "lut", rq_lut_bytes(d, B)), B,
+        float(softcap), _ptr_or_null(logits, torch.float32, "logits", B * d.V * 4),
+        _ptr_or_null(argmax, torch.int32, "argmax", B * 4), _stream(stream)))
     return logits, argmax
 
 
@@ -475,7 +514,7 @@ def rq_greedy_step(h, C, codes, fmt: int, d: RqDims, softcap: float = 30.0, scal
     """Logits (optional), argmax and the bf16 input rows of the picked tokens.
     Returns (logits or None, argmax int32 [B], rows bf16 [B, D], ws)."""
     torch = _torch()
-    B = h.shape[0]
+    B = _tokens(h, d)
     if want_logits and logits is None:
         logits = _empty((B, d.V), torch.float32, h)
     if argmax is None:
@@ -485,8 +524,9 @@ def rq_greedy_step(h, C, codes, fmt: int, d: RqDims, softcap: float = 30.0, scal
     nbytes = rq_fused_workspace_bytes(d, B, fmt, True)
     wp, wn, ws = _workspace(nbytes, h, ws)
     _check("rq_greedy_step", lib().rq_greedy_step(
-        _cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C"),
-        _cuda(codes, _codes_dtype(fmt), "codes"), fmt, d, B, float(softcap),
-        _ptr_or_null(logits, torch.float32, "logits"), _cuda(argmax, torch.int32, "argmax"),
-        float(scale), _cuda(rows, None, "rows"), wp, wn, _stream(stream)))
+        _cuda(h, torch.float32, "h"), _cuda(C, torch.float32, "C", _book_bytes(d)),
+        _cuda(codes, _codes_dtype(fmt), "codes", rq_codes_bytes(d, fmt)), fmt, d, B,
+        float(softcap), _ptr_or_null(logits, torch.float32, "logits", B * d.V * 4),
+        _cuda(argmax, torch.int32, "argmax", B * 4), float(scale),
+        _cuda(rows, None, "rows", B * d.D * 2), wp, wn, _stream(stream)))
     return logits, argmax, rows, ws

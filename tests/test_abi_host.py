@@ -168,3 +168,77 @@ def test_python_binding_rejects_cpu_tensors():
     C = torch.zeros(32, 2, 256, 6)
     with pytest.raises(ValueError):
         rq.rq_lut_build(h, C, TINY, lut=torch.zeros(64, 256, 1))
+
+
+def test_python_binding_checks_buffer_sizes_before_the_call(monkeypatch):
+    """A short buffer is refused by name before any pointer reaches the C
+    call (the C ABI takes bare pointers and could not tell).  CPU tensors
+    stand in for device ones here: the device check is switched off and the
+    library's launching calls are replaced by one that only reports being
+    reached, so no pointer is ever passed on."""
+    import torch
+    real = rq.lib()
+
+    class NoLaunch:
+        def __getattr__(self, name):
+            if name.endswith("_bytes") or name in ("rq_lut_token_stride", "rq_status_string"):
+                return getattr(real, name)
+
+            def reached(*a):
+                raise RuntimeError(f"{name} reached")
+            return reached
+
+    monkeypatch.setattr(rq, "lib", lambda: NoLaunch())
+    monkeypatch.setattr(rq, "_on_device", lambda t: True)
+    monkeypatch.setattr(rq, "_stream", lambda s: ctypes.c_void_p(None))
+
+    d = TINY                                  # V 4096, D 192, M 32, L 2, K 256
+    V, D, P = d.V, d.D, d.M * d.L
+    h = torch.zeros(2, D)
+    C = torch.zeros(d.M, d.L, d.K, D // d.M)
+    codes = torch.zeros((V, P), dtype=torch.uint16)
+    lut = torch.zeros(P, d.K, 2)
+
+    def refused(fn, *a, match, **kw):
+        with pytest.raises(ValueError, match=match):
+            fn(*a, **kw)
+
+    def reaches(fn, *a, **kw):
+        with pytest.raises(RuntimeError, match="reached"):
+            fn(*a, **kw)
+
+    refused(rq.rq_lut_build, h, C[:-1], d, match="C: .* bytes")
+    refused(rq.rq_lut_build, h, C, d, lut=torch.zeros(P, d.K, 1), match="lut: .* bytes")
+    refused(rq.rq_lut_build, torch.zeros(2, D + 1), C, d, match=r"h: shape")
+    reaches(rq.rq_lut_build, h, C, d, lut=lut)
+    refused(rq.rq_lut_logits, codes[:-1], rq.U16, d, lut, 2, match="codes: .* bytes")
+    refused(rq.rq_lut_logits, codes, rq.U16, d, lut, 2, logits=torch.zeros(2, V - 1),
+            match="logits: .* bytes")
+    reaches(rq.rq_lut_logits, codes, rq.U16, d, lut, 2, want_argmax=True)
+    refused(rq.rq_logits_from_hidden, h, C, codes, rq.U16, d, logits=torch.zeros(1, V),
+            match="logits: .* bytes")
+    refused(rq.rq_logits_from_hidden, h, C, codes, rq.U16, d, want_argmax=True,
+            logits=torch.zeros(2, V), argmax=torch.zeros(1, dtype=torch.int32),
+            match="argmax: .* bytes")
+    reaches(rq.rq_logits_from_hidden, h, C, codes, rq.U16, d, want_argmax=True)
+    ids = torch.zeros(5, dtype=torch.int32)
+    refused(rq.rq_decode_rows, ids, codes, rq.U16, C, d, 1.0,
+            out=torch.zeros((4, D), dtype=torch.bfloat16), match="out: .* bytes")
+    reaches(rq.rq_decode_rows, ids, codes, rq.U16, C, d, 1.0)
+    refused(rq.rq_pack10, codes, d, out=torch.zeros((V, 79), dtype=torch.uint8),
+            match="packed: .* bytes")             # a row needs ceil(10 * 64 / 8) = 80 bytes
+    reaches(rq.rq_pack10, codes, d)
+    refused(rq.rq_greedy_step, h, C, codes, rq.U16, d,
+            rows=torch.zeros((1, D), dtype=torch.bfloat16), match="rows: .* bytes")
+    reaches(rq.rq_greedy_step, h, C, codes, rq.U16, d)
+    refused(rq.rq_topk_sample, torch.zeros(2, 100), 8, token=torch.zeros(1, dtype=torch.int32),
+            match="token: .* bytes")
+    reaches(rq.rq_topk_sample, torch.zeros(2, 100), 8)
+    refused(rq.rq_argmax_merge, torch.zeros(3, 4), torch.zeros((3, 4), dtype=torch.int32),
+            out=torch.zeros(3, dtype=torch.int32), match="argmax: .* bytes")
+    refused(rq.rq_argmax_candidates, torch.zeros(3, 50), torch.zeros(2, dtype=torch.int32), 0,
+            match="argmax: .* bytes")
+    refused(rq.rq_encode, torch.zeros(V - 1, D), C, d, match="X: .* bytes")
+    reaches(rq.rq_encode, torch.zeros(V, D), C, d)
+    refused(rq.rq_prepare_sched, codes, d, out=codes[:-1], match="out: .* bytes")
+    reaches(rq.rq_prepare_sched, codes, d)

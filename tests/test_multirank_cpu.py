@@ -108,3 +108,67 @@ def test_sharded_pick_exchange_layout_with_gloo():
     for _, _, _, vals, idxs in res:
         assert vals == [[b + 100.0 * k for b in range(5)] for k in range(world)]
         assert idxs == [[bounds[k][0]] * 5 for k in range(world)]
+
+
+def _sharded_call_worker(rank, world, port, q):
+    """rq_sharded_logits itself over gloo, its three device calls replaced by
+    CPU stand-ins that read a fixed full logits matrix: what is checked is the
+    glue -- process-group size, the flat all-gathers, the [world][B] layout
+    handed to the merge -- against the argmax of the full matrix."""
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import lut_logits_serving_b200 as rq
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    V, B = 1003, 4
+    full = torch.from_numpy(np.random.default_rng(7).standard_normal((B, V)).astype(np.float32))
+    r0, r1 = rq.shard_rows(V, rank, world)
+
+    def logits_from_hidden(h, C, codes, fmt, d, softcap, want_argmax, ws, stream):
+        part = full[:, r0:r1].contiguous()
+        return part, part.argmax(dim=1).to(torch.int32), ws
+
+    def candidates(logits, am, row0, stream=None):
+        b = torch.arange(logits.shape[0])
+        return logits[b, am.long()], am + row0
+
+    def merge(vals, idxs, stream=None):
+        n, nb = vals.shape
+        out = torch.empty(nb, dtype=torch.int32)
+        for b in range(nb):
+            best = max(range(n), key=lambda k: (float(vals[k, b]), -int(idxs[k, b])))
+            out[b] = idxs[best, b]
+        return out
+
+    rq.rq_logits_from_hidden = logits_from_hidden
+    rq.rq_argmax_candidates = candidates
+    rq.rq_argmax_merge = merge
+    d = rq.dims(r1 - r0, 12, 2, 2, 4)
+    logits, pick, _ = rq.rq_sharded_logits(None, None, None, rq.U16, d, r0)
+    q.put((rank, logits.shape[1] == r1 - r0, pick.tolist(),
+           full.argmax(dim=1).tolist()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_sharded_logits_glue_with_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 3
+    procs = [ctx.Process(target=_sharded_call_worker, args=(r, world, port, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, own_rows, pick, want in res:
+        assert own_rows and pick == want
