@@ -242,3 +242,49 @@ def test_python_binding_checks_buffer_sizes_before_the_call(monkeypatch):
     reaches(rq.rq_encode, torch.zeros(V, D), C, d)
     refused(rq.rq_prepare_sched, codes, d, out=codes[:-1], match="out: .* bytes")
     reaches(rq.rq_prepare_sched, codes, d)
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "rqlut.h"
+
+int main(void) {
+    rq_dims g2 = {256000, 2304, 384, 2, 1024};
+    if (rq_version() <= 0) return 10;
+    if (rq_codes_bytes(g2, RQ_CODES_U16) != (size_t)256000 * 768 * 2) return 11;
+    if (rq_codes_bytes(g2, RQ_CODES_PACKED10) != (size_t)256000 * 960) return 12;
+    if (rq_codes_bytes(g2, RQ_CODES_U8) != 0) return 13;              /* K > 256 */
+    if (rq_lut_bytes(g2, 1) != (size_t)768 * 1024 * 4) return 14;
+    if (rq_lut_build(NULL, NULL, g2, 1, NULL, NULL) != RQ_ERR_INVALID_ARGUMENT) return 15;
+    if (rq_decode_rows(NULL, 0, NULL, RQ_CODES_U16, NULL, g2, 48.0f, NULL, NULL) != RQ_OK)
+        return 16;                                                     /* N = 0: no-op */
+    if (strlen(rq_status_string(RQ_ERR_MISALIGNED)) == 0) return 17;
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_header_serves_a_plain_c_client(tmp_path):
+    """include/rqlut.h compiles as C99 and C++11 with warnings as errors, and a
+    C program linked against the library runs its host-side queries and
+    argument checks (no device work, no torch, no Python)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    inc = os.path.join(ROOT, "include")
+    libdir = os.path.dirname(rq.LIB_PATH)
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", f"-I{inc}", str(src),
+                    f"-L{libdir}", "-l:librqlut.so", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stderr)
+    cpp = tmp_path / "client.cpp"
+    cpp.write_text('#include "rqlut.h"\nint main() { return rq_version() > 0 ? 0 : 1; }\n')
+    subprocess.run(["g++", "-std=c++11", "-Wall", "-Wextra", "-Werror", "-fsyntax-only",
+                    f"-I{inc}", str(cpp)], check=True, capture_output=True, text=True)
