@@ -288,3 +288,33 @@ def test_header_serves_a_plain_c_client(tmp_path):
     cpp.write_text('#include "rqlut.h"\nint main() { return rq_version() > 0 ? 0 : 1; }\n')
     subprocess.run(["g++", "-std=c++11", "-Wall", "-Wextra", "-Werror", "-fsyntax-only",
                     f"-I{inc}", str(cpp)], check=True, capture_output=True, text=True)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without the built library the binding raises; nothing falls back to
+    the oracle or to PyTorch."""
+    import subprocess
+    import sys
+    code = ("import lut_logits_serving_b200 as rq\n"
+            f"rq.LIB_PATH = {str(tmp_path / 'librqlut.so')!r}\n"
+            "try:\n"
+            "    rq.rq_version()\n"
+            "except RuntimeError as e:\n"
+            "    print('raised:', 'no CPU fallback' in str(e))\n"
+            "else:\n"
+            "    print('returned')\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         cwd=ROOT, timeout=120)
+    assert out.stdout.strip() == "raised: True", (out.stdout, out.stderr[-500:])
+
+
+def test_product_code_does_not_reach_the_oracle():
+    """Only tests, smoke() and the bench's CPU legs may load the oracle: the
+    package's sources never import it."""
+    pkg = os.path.join(ROOT, "lut_logits_serving_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "rq_oracle" not in text and "librq_oracle" not in text, f
