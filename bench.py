@@ -50,8 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="g2_b1",
-                    choices=["g2_b1", "g2_b32", "packed_b64", "mlp_gate_b1", "mlp_down_b1",
-                             "encode_g2", "g2_b1_topk50", "decode512"])
+                    choices=["g2_b1", "g2_b16", "g2_b32", "packed_b64", "mlp_gate_b1",
+                             "mlp_down_b1", "encode_g2", "g2_b1_topk50", "decode512"])
     ap.add_argument("--codes", default=None, choices=["u16", "sched", "u8"],
                     help="code layout of the unpacked workloads timed for `value`: "
                          "bank-scheduled once by rq_prepare_sched (the default at B <= 4), as "
@@ -60,6 +60,12 @@ def parse():
                          "reported under other_layouts")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sustain-seconds", type=float, default=1.0,
+                    help="after the timed steps, replay the same step for this long so the "
+                         "clock record has samples under load (0: skip)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the workload alone (by default the batch-1 run also measures "
+                         "g2_b32, packed_b64, decode512 and batch 1 on packed codes)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -126,6 +132,11 @@ def throughput(units_per_rank, world, job_ms):
     return world * units_per_rank / (job_ms / 1e3)
 
 
+def parallelism():
+    """The config key both arms print: one replica per rank."""
+    return f"replicas x{int(os.environ.get('WORLD_SIZE', '1'))}"
+
+
 def rank_seed(rank):
     """Each replica scores its own seeded batch and artifact."""
     return 1000 * rank
@@ -134,7 +145,11 @@ def rank_seed(rank):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi samples during the timed region (median SM clock, reasons)."""
+    """nvidia-smi samples (every 100 ms) of the SM clock and the throttle
+    reasons.  A reader thread stamps each sample with the host time it
+    arrived; `window()` / `close_window()` bracket the region of interest and
+    `summary()` keeps the samples inside it (all samples when no window was
+    opened)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -142,8 +157,14 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.lines = []            # (host time, line)
+        self.t_open = self.t_close = None
+        self._thread = None
+        self._first = None
 
     def __enter__(self):
+        import threading
+        self._first = threading.Event()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -151,21 +172,50 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+
+        def read():
+            for line in self.proc.stdout:
+                self.lines.append((time.monotonic(), line))
+                self._first.set()
+        self._thread = threading.Thread(target=read, daemon=True)
+        self._thread.start()
         return self
 
+    def wait_first(self, timeout=5.0):
+        """Block until the sampler has produced its first line (it takes
+        nvidia-smi a moment to start), so the timed region is covered."""
+        if self.proc is not None:
+            self._first.wait(timeout)
+
+    def window(self):
+        self.t_open = time.monotonic()
+
+    def close_window(self):
+        self.t_close = time.monotonic()
+
     def __exit__(self, *exc):
-        self.out = ""
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self.proc.wait()
+            if self._thread is not None:
+                self._thread.join(timeout=5)
+
+    @property
+    def out(self):
+        return "".join(l for _, l in self.lines)
 
     def summary(self):
         rows = []
-        for line in (self.out or "").splitlines():
+        lo = self.t_open if self.t_open is not None else -1e300
+        hi = self.t_close if self.t_close is not None else 1e300
+        for t, line in self.lines:
+            if not (lo <= t <= hi):
+                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -180,6 +230,20 @@ class ClockSampler:
         return {"sm_mhz": float(np.median([r[0] for r in rows])),
                 "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
                 "samples": len(rows)}
+
+
+def cpu_info():
+    """Host cores and CPU model of the box the oracle is timed on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -202,20 +266,27 @@ def oracle_step_fn(w, data):
     return step
 
 
-def cpu_baseline(w, data, seconds):
-    """Time the oracle as it stands on full-vocabulary steps until `seconds`."""
-    step = oracle_step_fn(w, data)
-    n, t0 = 0, time.perf_counter()
-    while True:
-        step()
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
+def cpu_baseline(w, data, seconds, threads=0):
+    """Time the oracle as it stands on full-vocabulary steps until `seconds`
+    (threads < 1: all host cores, else that many)."""
+    import oracle
+    used = oracle.set_threads(threads)
+    try:
+        step = oracle_step_fn(w, data)
+        n, t0 = 0, time.perf_counter()
+        while True:
+            step()
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    finally:
+        oracle.set_threads(0)
     pick = f"top-{w.topk} draw" if w.topk else "argmax"
-    return {"value": w.V * w.B * n / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} full steps of {w.name} (all {w.V} rows x {w.B} tokens, fp64 tables, "
-                      f"softcap, {pick}, row decode), single-threaded C, {el:.1f} s"}
+    return dict({"value": w.V * w.B * n / el, "unit": UNIT, "cores": used, "kind": "oracle",
+                 "sample": f"{n} full steps of {w.name} (all {w.V} rows x {w.B} tokens, fp64 "
+                           f"tables, softcap, {pick}, row decode), C with {used} OpenMP "
+                           f"thread(s) over vocabulary rows, {el:.1f} s"}, **cpu_info())
 
 
 def encode_terms(w, rows):
@@ -225,6 +296,7 @@ def encode_terms(w, rows):
 
 def run_reference_encode(args, w):
     import oracle
+    threads = oracle.set_threads(0)
     data = synth.make(w, V=4096)
     X, C = data["X"], data["C"]
     t0 = time.perf_counter()
@@ -243,9 +315,11 @@ def run_reference_encode(args, w):
         "impl": "reference", "metric": ENC_METRIC, "value": value, "unit": ENC_UNIT,
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": encode_config(w),
-        "cpu_baseline": {"value": value, "unit": ENC_UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{nrows} of {w.V} rows per step"},
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(encode_config(w), parallelism=parallelism()),
+        "cpu_baseline": dict({"value": value, "unit": ENC_UNIT, "cores": threads, "kind": "oracle",
+                              "sample": f"{nrows} of {w.V} rows per step, {threads} OpenMP "
+                                        f"thread(s) over rows"}, **cpu_info()),
         "e2e": {"value": value, "unit": ENC_UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -268,6 +342,7 @@ def decode_bytes(w):
 
 def run_reference_decode(args, w):
     import oracle
+    threads = oracle.set_threads(0)
     data = synth.make(w)
     ids, codes, C = data["ids"], data["codes"], data["C"]
     # each step rebuilds the first n ids, n sized so that warmup + steps end
@@ -289,9 +364,11 @@ def run_reference_decode(args, w):
         "impl": "reference", "metric": DEC_METRIC, "value": value, "unit": DEC_UNIT,
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": decode_config(w),
-        "cpu_baseline": {"value": value, "unit": DEC_UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"the first {n} of the {w.n_ids} ids per step"},
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(decode_config(w), parallelism=parallelism()),
+        "cpu_baseline": dict({"value": value, "unit": DEC_UNIT, "cores": threads, "kind": "oracle",
+                              "sample": f"the first {n} of the {w.n_ids} ids per step, "
+                                        f"{threads} OpenMP thread(s) over ids"}, **cpu_info()),
         "e2e": {"value": value, "unit": DEC_UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -313,6 +390,8 @@ def run_reference(args, w):
         return run_reference_encode(args, w)
     if w.B == 0:
         return run_reference_decode(args, w)
+    import oracle
+    threads = oracle.set_threads(0)
     data = synth.make(w)
     step = oracle_step_fn(w, data)
     # size each step's row sample so that warmup + steps end within ~2 minutes
@@ -335,9 +414,12 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w, headline_layout(w, args.codes)),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{nrows} of {w.V} rows per step, {w.B} token(s)"},
+        "data": "synthetic",
+        "config": dict(workload_config(w, headline_layout(w, args.codes)),
+                       parallelism=parallelism()),
+        "cpu_baseline": dict({"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                              "sample": f"{nrows} of {w.V} rows per step, {w.B} token(s), "
+                                        f"{threads} OpenMP thread(s) over rows"}, **cpu_info()),
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -354,11 +436,32 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
+def tf32_peak():
+    """Dense tf32 tensor peak (TFLOP/s): the measured bf16 burst figure times
+    the nominal tf32/bf16 ratio (1.1 / 2.25 PFLOP/s dense)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]) * 1.1 / 2.25, "measured bf16 x 1.1/2.25"
+    return 1590.0 * 1.1 / 2.25, "fallback bf16 x 1.1/2.25"
+
+
+# Shared memory delivers 128 bytes per clock per SM (32 banks x 4 bytes).
+SMEM_BYTES_PER_CLK = 128
+
+
+def smem_peak(mhz):
+    """Aggregate shared-memory bandwidth (GB/s) at an SM clock."""
+    return SMS * SMEM_BYTES_PER_CLK * (mhz or NOMINAL_SM_MHZ) * 1e6 / 1e9
+
+
 def kernel_source_hash(kernel="logits_chunk"):
     """Hash of the sources a kernel is built from (its .cu file and the common
     header), to tell whether committed ncu counters still describe it."""
     src = ("logits_decode_mma.cu" if kernel.startswith("logits_decode_mma") else
-           "decode_rows.cu" if kernel.startswith("decode_rows") else "logits_chunk.cu")
+           "decode_rows.cu" if kernel.startswith("decode_rows") else
+           "lut_build.cu" if kernel.startswith("lut_build") else
+           "logits_l2.cu" if kernel.startswith("logits_l2") else "logits_chunk.cu")
     h = hashlib.sha256()
     for name in (src, "rq_common.cuh"):
         with open(os.path.join(ROOT, "lut_logits_serving_b200", "csrc", name), "rb") as f:
@@ -386,60 +489,197 @@ def topk_launches(V, k):
     return 2
 
 
-def run_ours(args, w):
-    import torch
-    import torch.distributed as dist
+def decodable(w):
+    """Full token groups (64, then 32) of uint16 or 10-bit packed codes at
+    ds = 6, L = 2 decode their rows on the tensor cores."""
+    return (w.ds == 6 and w.L == 2 and 16 <= w.K <= 1024 and w.B >= 32 and
+            w.M % (32 if w.packed10 else 8) == 0)
 
+
+def token_groups(w, decoded):
+    groups, b0 = [], 0
+    while b0 < w.B:
+        g = 64 if decoded and w.B - b0 >= 64 else 32 if decoded and w.B - b0 >= 32 else \
+            min(32, w.B - b0)
+        groups.append(g)
+        b0 += g
+    return groups
+
+
+def launches_per_step(w, decoded):
+    """Kernels of one step: (table build, tiled pass, reduce) at B <= 4, else
+    two kernels per token group (hidden split + tensor-core decode, or table
+    build + L2 pass); then the argmax finish that also rebuilds the picked
+    rows, or the top-k draw and the row decode."""
+    if w.B <= 4 and not w.packed10:
+        n = 3 + (1 if w.argmax else 0)
+    else:
+        n = 2 * len(token_groups(w, decoded)) + (1 if w.argmax else 0)
+    if w.topk:
+        n += topk_launches(w.V, w.topk) + 1
+    return n
+
+
+class Rig:
+    """Our arm's process state: ranks, the launching stream, and the timing
+    helpers (CUDA events on that stream, barrier + max over ranks)."""
+
+    def __init__(self, args):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist, self.args = torch, dist, args
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world != args.gpus:
+            raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={self.world}")
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import datetime
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+        self.stream = torch.cuda.current_stream()
+        self.graphs = []
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_over_ranks(self, x):
+        return aggregate(x, self.world, device="cuda")
+
+    def close(self):
+        self.graphs.clear()
+        if self.world > 1:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+    def graphed(self, step):
+        """Warm `step` up, then capture it as a CUDA graph (unless --no-graph)."""
+        torch = self.torch
+        for _ in range(max(3, self.args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        if self.args.no_graph:
+            return step
+        s2 = torch.cuda.Stream()
+        s2.wait_stream(self.stream)
+        with torch.cuda.stream(s2):
+            step()
+        self.stream.wait_stream(s2)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        self.graphs.append(g)
+        return g.replay
+
+    def time_steps(self, run, n, flush=None):
+        """Device time (ms) of n steps, max over ranks.  With `flush` each step
+        is timed alone and the buffer is written between steps."""
+        torch = self.torch
+        self.barrier()
+        torch.cuda.synchronize()
+        if flush is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            for _ in range(n):
+                run()
+            e1.record(self.stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+        else:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(n)]
+            for a0, a1 in evs:
+                flush.fill_(1)
+                a0.record(self.stream)
+                run()
+                a1.record(self.stream)
+            torch.cuda.synchronize()
+            ms = sum(a0.elapsed_time(a1) for a0, a1 in evs)
+        self.barrier()
+        return self.max_over_ranks(ms)
+
+    def code_pass_us(self, step, n, flush=None):
+        """Mean device time (us) of the code-streaming pass alone: profile
+        events the library records around it on the launching stream."""
+        torch = self.torch
+        import lut_logits_serving_b200 as rq
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        stops = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for ev in starts + stops:       # torch creates the CUDA event on first record
+            ev.record(self.stream)
+        torch.cuda.synchronize()
+        for i in range(n):
+            if flush is not None:
+                flush.fill_(1)
+            rq.rq_set_profile_events(starts[i], stops[i])
+            step()
+        rq.rq_set_profile_events(None, None)
+        torch.cuda.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in zip(starts, stops)])) * 1e3
+
+
+class Artifact:
+    """The resident RQ artifact on the device: codebooks and the code matrix
+    in each layout a step may read (prepared once, outside timed regions)."""
+
+    def __init__(self, w, data, need=("sched", "u16", "u8", "packed10")):
+        import torch
+        import lut_logits_serving_b200 as rq
+        self.d = rq.dims(w.V, w.D, w.M, w.L, w.K)
+        self.C = torch.from_numpy(data["C"]).cuda()
+        c16 = torch.from_numpy(data["codes"].reshape(w.V, -1)).cuda()
+        self.layouts = {}
+        self.sched_passes = None
+        if "packed10" in need and w.K <= 1024:
+            self.layouts["packed10"] = (rq.PACKED10, rq.rq_pack10(c16, self.d))
+        if "sched" in need and w.K <= 1024 and w.P % 32 == 0:
+            sched, (st, ps) = rq.rq_prepare_sched(c16, self.d, stats=True)
+            self.layouts["sched"] = (rq.SCHED, sched)
+            self.sched_passes = ps / st
+        if "u8" in need and w.K <= 256:
+            self.layouts["u8"] = (rq.U8, rq.rq_pack8(c16, self.d))
+        if "u16" in need:
+            self.layouts["u16"] = (rq.U16, c16)
+
+    def bytes(self, layout):
+        t = self.layouts[layout][1]
+        return t.numel() * t.element_size() + self.C.numel() * 4
+
+
+def kernel_of(w, layout):
+    decoded = layout in ("u16", "packed10") and decodable(w)
+    if w.B <= 4 and not w.packed10 and layout != "packed10":
+        return "logits_chunk_u16_kernel", decoded
+    return ("logits_decode_mma_kernel" if decoded else "logits_l2_kernel"), decoded
+
+
+def measure_logits(rig, w, art, layout, h_np, full=False, clk=None):
+    """Time one workload's step on the resident artifact: K steps as CUDA-graph
+    replays, the code pass alone, end to end from host buffers, and the
+    device memory the step adds.  With `full`, also the other code layouts and
+    the kernel choices of full token groups; with `clk`, the timed steps and
+    a sustained run of at least a second after them are the clock window."""
+    torch, args = rig.torch, rig.args
     import lut_logits_serving_b200 as rq
+    d, dC = art.d, art.C
+    fmt, dcodes = art.layouts[layout]
+    stream = rig.stream
+    dh0 = torch.from_numpy(h_np).cuda()
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        return aggregate(x, world, device="cuda")
-
-    data = synth.make(w, seed=rank_seed(rank))
-    d = rq.dims(w.V, w.D, w.M, w.L, w.K)
-    dC = torch.from_numpy(data["C"]).cuda()
-    c16 = torch.from_numpy(data["codes"].reshape(w.V, -1)).cuda()
-    dh0 = torch.from_numpy(data["h"]).cuda()
-    dh = dh0
     def outputs():
         return (torch.empty((w.B, w.V), dtype=torch.float32, device="cuda"),
                 torch.empty((w.B,), dtype=torch.int32, device="cuda"),
                 torch.empty((w.B, w.D), dtype=torch.bfloat16, device="cuda"),
                 torch.empty((w.B,), dtype=torch.int32, device="cuda"))
     logits0, am0, rows0, tok0 = outputs()
-    logits, am, tok = logits0, am0, tok0
     tws = (torch.empty(rq.rq_topk_workspace_bytes(w.V, w.B, w.topk), dtype=torch.uint8,
                        device="cuda") if w.topk else None)
-    stream = torch.cuda.current_stream()
-
-    # code layouts: the artifact is prepared once, outside any timed region
-    layouts = {}
-    if w.packed10:
-        layouts["packed10"] = (rq.PACKED10, rq.rq_pack10(c16, d), None)
-        del c16
-        headline = "packed10"
-    else:
-        sched, (st, ps) = rq.rq_prepare_sched(c16, d, stats=True)
-        layouts["sched"] = (rq.SCHED, sched, ps / st)
-        layouts["u16"] = (rq.U16, c16, None)
-        if w.K <= 256:                 # one byte per code
-            layouts["u8"] = (rq.U8, rq.rq_pack8(c16, d), None)
-        headline = headline_layout(w, args.codes, tuple(layouts))
 
     def make_step(fmt, codes, out=None):
         ws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
@@ -455,149 +695,130 @@ def run_ours(args, w):
                 rq.rq_topk_sample(logits, w.topk, w.temperature, seed=1234, step=0, token=tok,
                                   want_topk=False, ws=tws)
                 rq.rq_decode_rows(tok, codes, fmt, dC, d, w.decode_scale, out=rows)
-            return step
-
-        if not w.argmax:
+        elif not w.argmax:
             def step():
                 # an RQ-coded weight matrix applied without reconstruction
                 rq.rq_logits_from_hidden(dh, dC, codes, fmt, d, w.softcap, logits=logits, ws=ws)
-            return step
-
-        def step():
-            # logits of this step's hidden states, the greedy picks, and the
-            # input rows of the picked tokens (the next step's embeddings)
-            rq.rq_greedy_step(dh, dC, codes, fmt, d, w.softcap, scale=w.decode_scale,
-                              logits=logits, argmax=am, rows=rows, ws=ws)
+        else:
+            def step():
+                # logits of this step's hidden states, the greedy picks, and the
+                # input rows of the picked tokens (the next step's embeddings)
+                rq.rq_greedy_step(dh, dC, codes, fmt, d, w.softcap, scale=w.decode_scale,
+                                  logits=logits, argmax=am, rows=rows, ws=ws)
+        step.ws_bytes = ws.numel()
         return step
-
-    def graphed(step):
-        for _ in range(max(3, args.warmup)):
-            step()
-        torch.cuda.synchronize()
-        if args.no_graph:
-            return step, None
-        s2 = torch.cuda.Stream()
-        s2.wait_stream(stream)
-        with torch.cuda.stream(s2):
-            step()
-        stream.wait_stream(s2)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step()
-        for _ in range(3):
-            g.replay()
-        torch.cuda.synchronize()
-        return g.replay, g
 
     # Inputs smaller than twice the 126 MB L2 would stay cached between steps:
     # then every step is timed by its own event pair and a 256 MB buffer is
     # written between steps, outside the pairs.
     flush = None
-    if code_bytes(w) + data["C"].nbytes < 2 * 126 * 2**20:
+    if code_bytes(w, layout) + dC.numel() * 4 < 2 * 126 * 2**20:
         flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
 
-    def time_steps(run, n):
-        barrier()
-        torch.cuda.synchronize()
-        if flush is None:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(n):
-                run()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1)
-        else:
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(n)]
-            for a0, a1 in evs:
-                flush.fill_(1)
-                a0.record(stream)
-                run()
-                a1.record(stream)
-            torch.cuda.synchronize()
-            ms = sum(a0.elapsed_time(a1) for a0, a1 in evs)
-        barrier()
-        return max_over_ranks(ms)
-
-    def code_pass_us(step, n):
-        """Device time of the code-streaming pass alone (profile events
-        recorded by the library around it on the launching stream)."""
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        stops = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        for ev in starts + stops:       # torch creates the CUDA event on first record
-            ev.record(stream)
-        torch.cuda.synchronize()
-        for i in range(n):
-            if flush is not None:
-                flush.fill_(1)
-            rq.rq_set_profile_events(starts[i], stops[i])
-            step()
-        rq.rq_set_profile_events(None, None)
-        torch.cuda.synchronize()
-        return float(np.mean([a.elapsed_time(b) for a, b in zip(starts, stops)])) * 1e3
-
-    fmt, dcodes, sched_quality = layouts[headline]
     step = make_step(fmt, dcodes)
-    run, graph = graphed(step)
+    run = rig.graphed(step)
 
     # ---- timed region: K steps, device time, max over ranks
-    with ClockSampler(local) as clk:
-        t_ms = time_steps(run, args.steps)
-    sec = t_ms / 1e3
-    value = throughput(w.V * w.B * args.steps, world, t_ms)
+    if clk is not None:
+        clk.wait_first()
+        clk.window()
+    t_ms = rig.time_steps(run, args.steps, flush)
+    sustained = None
+    if clk is not None:
+        # the same step replayed for at least a second, so that the clock
+        # record has samples under this load
+        per = max(t_ms / args.steps, 1e-3)
+        n_sus = int(min(200000, 1000.0 * args.sustain_seconds / per))
+        if n_sus > 0:
+            s_ms = rig.time_steps(run, n_sus, flush)
+            sustained = {"steps": n_sus, "seconds": s_ms / 1e3,
+                         "us_per_step": s_ms / n_sus * 1e3}
+        else:
+            sustained = {"steps": 0, "seconds": 0.0, "us_per_step": None}
+        clk.close_window()
+    res = {"us_per_call": t_ms / args.steps * 1e3,
+           "value": throughput(w.V * w.B * args.steps, rig.world, t_ms),
+           "unit": UNIT, "steps": args.steps, "codes": layout, "t_ms": t_ms,
+           "sustained": sustained}
 
     # ---- the dominant kernel alone, live CUDA events
-    kern_us = code_pass_us(step, min(args.steps, 2000))
+    kern_us = rig.code_pass_us(step, min(args.steps, 2000), flush)
     peak, peak_kind = load_peaks()
-    algo_bytes = code_bytes(w, headline)
+    algo_bytes = code_bytes(w, layout)
     achieved = algo_bytes / (kern_us / 1e6) / 1e9
-    # full token groups (64, then 32) of uint16 or 10-bit packed codes at
-    # ds = 6, L = 2 decode their rows on the tensor cores
-    decodable = (w.ds == 6 and w.L == 2 and 16 <= w.K <= 1024 and w.B >= 32 and
-                 w.M % (32 if w.packed10 else 8) == 0)
-    decoded = headline in ("u16", "packed10") and decodable
-    kname = ("logits_chunk_u16_kernel" if w.B <= 4 and not w.packed10 else
-             "logits_decode_mma_kernel" if decoded else "logits_l2_kernel")
-    kkey = f"{kname}/{headline}/{w.name}"
+    kname, decoded = kernel_of(w, layout)
+    kkey = f"{kname}/{layout}/{w.name}"
+    res["roofline"] = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
+                       "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                       "traffic": profiled_traffic(kkey), "algorithmic_bytes": algo_bytes,
+                       "kernel_us": kern_us}
+    res["step_hbm_frac"] = algo_bytes / (t_ms / args.steps / 1e3) / 1e9 / peak
+    if decoded:
+        # the decode-then-multiply kernels: their binding pipes, on
+        # algorithmic work (2 B V D flops; two L-level codeword gathers of ds
+        # fp32 per row and subspace, per group)
+        groups = token_groups(w, True)
+        flops = 2.0 * w.B * w.V * w.D
+        tpk, tpk_kind = tf32_peak()
+        smem_bytes = len(groups) * w.V * w.M * w.L * w.ds * 4
+        mhz = (clk.summary().get("sm_mhz") if clk is not None else None) or NOMINAL_SM_MHZ
+        res["pipes"] = {
+            "tensor": {"achieved": flops / (kern_us / 1e6) / 1e12, "peak": tpk,
+                       "peak_kind": tpk_kind, "unit": "TFLOP/s",
+                       "frac": flops / (kern_us / 1e6) / 1e12 / tpk},
+            "smem": {"achieved": smem_bytes / (kern_us / 1e6) / 1e9,
+                     "peak": smem_peak(mhz), "unit": "GB/s",
+                     "peak_kind": f"derived: {SMS} SMs x {SMEM_BYTES_PER_CLK} B x {mhz:g} MHz",
+                     "frac": smem_bytes / (kern_us / 1e6) / 1e9 / smem_peak(mhz),
+                     "algorithmic_bytes": smem_bytes}}
 
-    # ---- the other layout, same step (context for the headline)
-    others = {}
-    for name, (f2, c2, q2) in layouts.items():
-        if name == headline:
-            continue
-        st2 = make_step(f2, c2)
-        r2, g2 = graphed(st2)
-        n2 = min(args.steps, 3000)
-        t2 = time_steps(r2, n2)
-        k2 = code_pass_us(st2, min(n2, 1000))
-        others[name] = {"us_per_call": t2 / n2 * 1e3, "value": throughput(w.V * w.B * n2, world, t2),
-                        "code_pass_us": k2,
-                        "code_pass_frac": code_bytes(w, name) / (k2 / 1e6) / 1e9 / peak}
-        del g2
+    # ---- device memory: the resident artifact, the caller's workspace, and
+    # what a step adds on top (the library allocates nothing itself)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    step()
+    torch.cuda.synchronize()
+    res["memory"] = {"resident_bytes": art.bytes(layout), "workspace_bytes": step.ws_bytes,
+                     "peak_delta_bytes": torch.cuda.max_memory_allocated() - base,
+                     "outputs_bytes": w.B * w.V * 4 + w.B * 4 + w.B * w.D * 2,
+                     "how": "torch.cuda.max_memory_allocated around one eager step"}
 
-    # ---- the kernel choices of full token groups (uint16 codes): logits and
-    # argmax of one rq_logits_from_hidden_path call per step
-    paths = {}
-    if decodable and headline in ("u16", "packed10"):
-        pf, pc = layouts[headline][0], layouts[headline][1]
-        pws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, pf, True), dtype=torch.uint8,
-                          device="cuda")
-        choices = [("tables", rq.PATH_TABLES), ("decode_tc", rq.PATH_DECODE_TC)]
-        if headline == "u16":
-            choices.insert(1, ("decode_fp32", rq.PATH_DECODE_FP32))
-        for name, pth in choices:
-            def pstep(pth=pth):
-                rq.rq_logits_from_hidden(dh0, dC, pc, pf, d, w.softcap,
-                                         logits=logits0, argmax=am0, ws=pws, path=pth)
-            rp, gp = graphed(pstep)
-            n3 = min(args.steps, 200)
-            t3 = time_steps(rp, n3)
-            paths[name] = {"us_per_call": t3 / n3 * 1e3,
-                           "code_pass_us": code_pass_us(pstep, min(n3, 50))}
-            del gp
-    run, graph = graphed(step)
+    if full:
+        # ---- the other layouts, same step (context for the headline)
+        others = {}
+        for name, (f2, c2) in art.layouts.items():
+            if name == layout or (name == "packed10") != w.packed10:
+                continue
+            st2 = make_step(f2, c2)
+            r2 = rig.graphed(st2)
+            n2 = min(args.steps, 3000)
+            t2 = rig.time_steps(r2, n2, flush)
+            k2 = rig.code_pass_us(st2, min(n2, 1000), flush)
+            others[name] = {"us_per_call": t2 / n2 * 1e3,
+                            "value": throughput(w.V * w.B * n2, rig.world, t2),
+                            "code_pass_us": k2,
+                            "code_pass_frac": code_bytes(w, name) / (k2 / 1e6) / 1e9 / peak}
+        res["other_layouts"] = others
+        # ---- the kernel choices of full token groups: logits and argmax of
+        # one rq_logits_from_hidden_path call per step
+        paths = {}
+        if decoded:
+            pws = torch.empty(rq.rq_fused_workspace_bytes(d, w.B, fmt, True), dtype=torch.uint8,
+                              device="cuda")
+            choices = [("tables", rq.PATH_TABLES), ("decode_tc", rq.PATH_DECODE_TC)]
+            if layout == "u16":
+                choices.insert(1, ("decode_fp32", rq.PATH_DECODE_FP32))
+            for name, pth in choices:
+                def pstep(pth=pth):
+                    rq.rq_logits_from_hidden(dh0, dC, dcodes, fmt, d, w.softcap,
+                                             logits=logits0, argmax=am0, ws=pws, path=pth)
+                rp = rig.graphed(pstep)
+                n3 = min(args.steps, 200)
+                t3 = rig.time_steps(rp, n3)
+                paths[name] = {"us_per_call": t3 / n3 * 1e3,
+                               "code_pass_us": rig.code_pass_us(pstep, min(n3, 50))}
+        res["full_group_paths"] = paths or None
 
     # ---- end to end through the public API with host buffers: every step
     # copies its hidden states in from pinned host memory and reads its logits
@@ -605,13 +826,11 @@ def run_ours(args, w):
     # steps' compute, as a serving loop does: two input/output sets, the input
     # of step i+2 and the readback of step i run on copy streams while step i+1
     # computes.  The L2-flushed workloads serialise each step and time it alone.
-    h_host = torch.from_numpy(data["h"]).pin_memory()
+    h_host = torch.from_numpy(h_np).pin_memory()
     ne2e = min(args.steps, 2000)
-    outs = [(dh0, logits0, am0, rows0, tok0),
-            (torch.empty_like(dh0),) + outputs()]
+    outs = [(dh0, logits0, am0, rows0, tok0), (torch.empty_like(dh0),) + outputs()]
     # the compute of each set replays as a CUDA graph, as in the device timing
-    graph_b = graphed(make_step(fmt, dcodes, outs[1]))
-    steps2 = [run, graph_b[0]]
+    steps2 = [run, rig.graphed(make_step(fmt, dcodes, outs[1]))]
     hosts = [(torch.empty((w.B, w.V), dtype=torch.float32).pin_memory(),
               torch.empty((w.B,), dtype=torch.int32).pin_memory()) for _ in range(2)]
     d2h_stream, h2d_stream = torch.cuda.Stream(), torch.cuda.Stream()
@@ -660,95 +879,241 @@ def run_ours(args, w):
     if flush is None:
         e2e_run(4)
         torch.cuda.synchronize()
-        barrier()
+        rig.barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         e2e_run(ne2e)
         e1.record(stream)
         torch.cuda.synchronize()
-        barrier()
-        e_ms = max_over_ranks(e0.elapsed_time(e1))
+        rig.barrier()
+        e_ms = rig.max_over_ranks(e0.elapsed_time(e1))
     else:
         for i in range(3):
             e2e_step(i)
-        e_ms = time_steps(e2e_step, ne2e)
-    e2e_value = throughput(w.V * w.B * ne2e, world, e_ms)
-    h2d = data["h"].nbytes
+        e_ms = rig.time_steps(e2e_step, ne2e)
     picked = picked_of(outs[0])
-    d2h = w.B * w.V * 4 + (w.B * 4 if picked is not None else 0)
+    res["e2e"] = {"value": throughput(w.V * w.B * ne2e, rig.world, e_ms), "unit": UNIT,
+                  "h2d_bytes_per_step": h_np.nbytes,
+                  "d2h_bytes_per_step": w.B * w.V * 4 + (w.B * 4 if picked is not None else 0),
+                  "ms_per_step": e_ms / ne2e}
     # the last step's host copy equals its device result
     last = (ne2e - 1) % 2 if flush is None else 0
     assert torch.equal(hosts[last][0], outs[last][1].cpu()), "logits readback mismatch"
-
     # the argmax must agree with the logits it came from
     if w.argmax:
-        assert torch.equal(am.long().cpu(), logits.argmax(dim=1).cpu()), "argmax/logits mismatch"
+        assert torch.equal(am0.long().cpu(), logits0.argmax(dim=1).cpu()), \
+            "argmax/logits mismatch"
     assert rq.rq_device_error() == 0
 
-    # (build, tiled pass, reduce) or (build + pass per token group), then the
-    # argmax finish that also rebuilds the picked rows
-    if w.B <= 4 and not w.packed10:
-        launches_per_step = 3 + (1 if w.argmax else 0)
-    else:
-        # per token group: hidden split + rows decoded and multiplied on the
-        # tensor cores (full groups of 64, then 32) or table build + L2 pass
-        # (groups of up to 32): two kernels either way
-        groups, b0 = [], 0
-        while b0 < w.B:
-            g = 64 if decoded and w.B - b0 >= 64 else 32 if decoded and w.B - b0 >= 32 else \
-                min(32, w.B - b0)
-            groups.append(g)
-            b0 += g
-        launches_per_step = 2 * len(groups)
-        launches_per_step += 1 if w.argmax else 0
-    topk_us = None
+    res["launches_per_step"] = launches_per_step(w, decoded)
     if w.topk:
-        launches_per_step += topk_launches(w.V, w.topk) + 1     # top-k + draw, row decode
         # the epilogue alone, on the step's own logits
         for _ in range(10):
-            rq.rq_topk_sample(logits, w.topk, w.temperature, 1234, 0, token=tok, want_topk=False,
-                              ws=tws)
+            rq.rq_topk_sample(logits0, w.topk, w.temperature, 1234, 0, token=tok0,
+                              want_topk=False, ws=tws)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(200):
-            rq.rq_topk_sample(logits, w.topk, w.temperature, 1234, 0, token=tok, want_topk=False,
-                              ws=tws)
+            rq.rq_topk_sample(logits0, w.topk, w.temperature, 1234, 0, token=tok0,
+                              want_topk=False, ws=tws)
         e1.record(stream)
         torch.cuda.synchronize()
-        topk_us = e0.elapsed_time(e1) / 200 * 1e3
+        res["topk_sample_us"] = e0.elapsed_time(e1) / 200 * 1e3
+    rig.graphs.clear()
+    return res
+
+
+def measure_decode(rig, w, art, ids_np, clk=None):
+    """Rebuild the bf16 input rows of a step's ids (decode512): each call
+    timed alone by its own events, with the L2 written over in between; a
+    burst of calls for the warm figure; end to end with the ids copied in and
+    the rows read back."""
+    torch, args = rig.torch, rig.args
+    import lut_logits_serving_b200 as rq
+    d, C = art.d, art.C
+    codes = art.layouts["u16"][1]
+    stream = rig.stream
+    ids = torch.from_numpy(ids_np).cuda()
+    rows = torch.empty((len(ids_np), w.D), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        rq.rq_decode_rows(ids, codes, rq.U16, C, d, w.decode_scale, out=rows)
+
+    def timed(fn, n, cold):
+        rig.barrier()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n if cold else 1)]
+        if cold:
+            for a0, a1 in evs:
+                flush.fill_(1)
+                a0.record(stream)
+                fn()
+                a1.record(stream)
+        else:
+            evs[0][0].record(stream)
+            for _ in range(n):
+                fn()
+            evs[0][1].record(stream)
+        torch.cuda.synchronize()
+        rig.barrier()
+        return rig.max_over_ranks(sum(a0.elapsed_time(a1) for a0, a1 in evs))
+
+    def graphed(calls):
+        """`calls` back-to-back decode calls as one CUDA graph (a call is a
+        few microseconds, shorter than a Python launch)."""
+        s2 = torch.cuda.Stream()
+        s2.wait_stream(stream)
+        with torch.cuda.stream(s2):
+            step()
+        stream.wait_stream(s2)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(calls):
+                step()
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    burst = 20
+    g1, gb = (None, None) if args.no_graph else (graphed(1), graphed(burst))
+    if clk is not None:
+        clk.wait_first()
+        clk.window()
+    t_ms = timed(step if g1 is None else g1.replay, args.steps, True)
+    if clk is not None:
+        clk.close_window()
+    if gb is None:
+        warm_ms = timed(step, args.steps, False)
+    else:
+        reps = max(1, args.steps // burst)
+        warm_ms = timed(gb.replay, reps, False) * args.steps / (reps * burst)
+    n_ids = len(ids_np)
+    want = None
+    if rig.rank == 0:
+        import oracle
+        want = oracle.decode_rows_bf16(ids_np, art.codes_np, art.C_np, w.decode_scale)
+        assert np.array_equal(rows.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    assert rq.rq_device_error() == 0
+    peak, peak_kind = load_peaks()
+    kern_s = t_ms / args.steps / 1e3
+    nbytes = decode_bytes(w)
+    achieved = nbytes / kern_s / 1e9
+
+    # end to end: ids in from pinned host memory, rows back to the host
+    idh = torch.from_numpy(ids_np).pin_memory()
+    rh = torch.empty((n_ids, w.D), dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        ids.copy_(idh, non_blocking=True)
+        step() if g1 is None else g1.replay()
+        rh.copy_(rows, non_blocking=True)
+
+    e2e_step()
+    e_ms = timed(e2e_step, args.steps, True)
+    del g1, gb
+    return {
+        "metric": DEC_METRIC, "unit": DEC_UNIT, "steps": args.steps,
+        "value": throughput(n_ids * args.steps, rig.world, t_ms),
+        "us_per_call": t_ms / args.steps * 1e3, "us_per_call_warm": warm_ms / args.steps * 1e3,
+        "ms_per_step": t_ms / args.steps,
+        "launch": "eager" if args.no_graph else "cuda graph",
+        "roofline": {"bound": "hbm", "kernel": "decode_rows_pair_kernel", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": profiled_traffic("decode_rows_pair_kernel/u16/decode512"),
+                     "algorithmic_bytes": nbytes, "kernel_us": kern_s * 1e6},
+        "e2e": {"value": throughput(n_ids * args.steps, rig.world, e_ms), "unit": DEC_UNIT,
+                "h2d_bytes_per_step": n_ids * 4, "d2h_bytes_per_step": n_ids * w.D * 2,
+                "ms_per_step": e_ms / args.steps},
+        "memory": {"resident_bytes": art.bytes("u16"), "workspace_bytes": 0,
+                   "outputs_bytes": n_ids * w.D * 2},
+    }
+
+
+# The default run measures the headline (decode batch 1) and, on the same
+# resident artifact, the batched, packed and row-decode configurations.
+EXTRA_WORKLOADS = ("g2_b32", "packed_b64", "decode512")
+
+
+def run_ours(args, w):
+    rig = Rig(args)
+    torch = rig.torch
+    data = synth.make(w, seed=rank_seed(rig.rank))
+    extras = (not args.no_extras and w.name == "g2_b1" and not args.codes)
+    need = ("sched", "u16", "u8", "packed10") if (extras or w.packed10) else \
+        ("sched", "u16", "u8")
+    art = Artifact(w, data, need)
+    art.codes_np, art.C_np = data["codes"], data["C"]
+    headline = headline_layout(w, args.codes, tuple(k for k in art.layouts if k != "packed10"))
+
+    with ClockSampler(rig.local) as clk:
+        res = measure_logits(rig, w, art, headline, data["h"], full=True, clk=clk)
+    clocks = clk.summary()
+    res["sustained"]["clocks"] = clocks
+    if clocks.get("sm_mhz") and res["sustained"]["us_per_step"]:
+        res["sustained"]["us_x_mhz"] = res["sustained"]["us_per_step"] * clocks["sm_mhz"]
+
+    others = {}
+    if extras:
+        # the packed 10-bit layout at batch 1 (the pages' 3.59 bits/param form)
+        p1 = measure_logits(rig, w, art, "packed10", data["h"])
+        p1.pop("t_ms", None)
+        others["g2_b1_packed10"] = dict(p1, config=workload_config(w, "packed10"))
+        for name in EXTRA_WORKLOADS:
+            w2 = synth.WORKLOADS[name]
+            seed = rank_seed(rig.rank)
+            with ClockSampler(rig.local) as c2:
+                if w2.B == 0:
+                    ids = synth.zipf_ids(w2.n_ids, w2.V, w2.zipf_s, seed + 3)
+                    r2 = measure_decode(rig, w2, art, ids, clk=c2)
+                    r2["config"] = decode_config(w2)
+                else:
+                    h2 = synth.hidden(w2.B, w2.D, w2.hidden_scale, seed + 2)
+                    lay = headline_layout(w2, None, tuple(art.layouts))
+                    r2 = measure_logits(rig, w2, art, lay, h2)
+                    r2["config"] = workload_config(w2, lay)
+                    r2.pop("t_ms", None)
+            r2["clocks"] = c2.summary()
+            others[name] = r2
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and (w.argmax or w.topk):
-        cpu = cpu_baseline(w, data, args.cpu_seconds)
-
-    if world > 1:
-        dist.barrier()
-        del graph, graph_b
-        dist.destroy_process_group()
-    if rank != 0:
+    if rig.rank == 0 and rig.world == 1 and not args.no_cpu_baseline and (w.argmax or w.topk):
+        cpu = cpu_baseline(w, data, args.cpu_seconds, threads=0)
+        cpu["single_thread"] = cpu_baseline(w, data, args.cpu_seconds / 2, threads=1)
+    rig.close()
+    if rig.rank != 0:
         return
+    t_ms = res["t_ms"]
+    roof = dict(res["roofline"])
+    if art.sched_passes is not None and headline == "sched":
+        roof["bank_passes_per_step"] = art.sched_passes
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
-        "us_per_call": t_ms / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": rig.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+        "us_per_call": res["us_per_call"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(workload_config(w, headline), parallelism=f"replicas x{world}",
-                       launch="cuda graph" if graph is not None else "eager",
-                       bank_passes_per_step=sched_quality),
-        "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": profiled_traffic(kkey), "algorithmic_bytes": algo_bytes,
-                     "kernel_us": kern_us},
-        "step_hbm_frac": algo_bytes / (sec / args.steps) / 1e9 / peak,
-        "other_layouts": others,
-        "full_group_paths": paths or None,
-        "topk_sample_us": topk_us,
+        "config": dict(workload_config(w, headline), parallelism=parallelism()),
+        "launch": "eager" if args.no_graph else "cuda graph",
+        "roofline": roof,
+        "step_hbm_frac": res["step_hbm_frac"],
+        "pipes": res.get("pipes"),
+        "memory": res["memory"],
+        "other_layouts": res.get("other_layouts"),
+        "full_group_paths": res.get("full_group_paths"),
+        "topk_sample_us": res.get("topk_sample_us"),
+        "other_workloads": others or None,
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ne2e},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "e2e": res["e2e"],
+        "gpu_launches": res["launches_per_step"] * args.steps,
+        "clocks": dict(clocks, window=f"the {args.steps} timed steps and "
+                                      f"{res['sustained']['steps']} more replays of the same "
+                                      f"step right after them"),
+        "sustained": res["sustained"],
     }
     print(json.dumps(line), flush=True)
 
@@ -823,14 +1188,15 @@ def run_encode(args, w):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        n, t0, sample = 0, time.perf_counter(), 64
+        threads = oracle.set_threads(0)
+        n, t0, sample = 0, time.perf_counter(), 64 * threads
         while time.perf_counter() - t0 < args.cpu_seconds:
             oracle.encode(data["X"][:sample], data["C"])
             n += sample
         el = time.perf_counter() - t0
-        cpu = {"value": n / el, "unit": ENC_UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{n} rows ({sample} per call) encoded by the C oracle, "
-                         f"single-threaded, {el:.1f} s"}
+        cpu = dict({"value": n / el, "unit": ENC_UNIT, "cores": threads, "kind": "oracle",
+                    "sample": f"{n} rows ({sample} per call) encoded by the C oracle, "
+                              f"{threads} OpenMP thread(s) over rows, {el:.1f} s"}, **cpu_info())
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -839,8 +1205,8 @@ def run_encode(args, w):
         "metric": ENC_METRIC, "value": value, "unit": ENC_UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic", "config": dict(encode_config(w), parallelism=f"replicas x{world}",
-                                            launch="eager"),
+        "data": "synthetic", "config": dict(encode_config(w), parallelism=parallelism()),
+        "launch": "eager",
         "roofline": {"bound": "alu", "kernel": "encode_pair_kernel<6,4>", "achieved": achieved,
                      "peak": peak, "peak_kind": f"derived: {SMS} SMs x {FP32_LANES} FP32 lanes "
                                                 f"x {mhz:g} MHz",
@@ -857,141 +1223,36 @@ def run_encode(args, w):
 
 
 def run_decode(args, w):
-    """Rebuild the bf16 input rows of a step's ids (decode512): each call
-    timed alone by its own events, with the L2 written over in between."""
-    import torch
-    import torch.distributed as dist
-
-    import lut_logits_serving_b200 as rq
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    data = synth.make(w, seed=rank_seed(rank))
-    d = rq.dims(w.V, w.D, w.M, w.L, w.K)
-    ids = torch.from_numpy(data["ids"]).cuda()
-    codes = torch.from_numpy(data["codes"].reshape(w.V, -1)).cuda()
-    C = torch.from_numpy(data["C"]).cuda()
-    rows = torch.empty((w.n_ids, w.D), dtype=torch.bfloat16, device="cuda")
-    stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
-
-    def step():
-        rq.rq_decode_rows(ids, codes, rq.U16, C, d, w.decode_scale, out=rows)
-
-    def timed(fn, n, cold):
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(n if cold else 1)]
-        if cold:
-            for a0, a1 in evs:
-                flush.fill_(1)
-                a0.record(stream)
-                fn()
-                a1.record(stream)
-        else:
-            evs[0][0].record(stream)
-            for _ in range(n):
-                fn()
-            evs[0][1].record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        return aggregate(sum(a0.elapsed_time(a1) for a0, a1 in evs), world, device="cuda")
-
-    def graphed(calls):
-        """`calls` back-to-back decode calls as one CUDA graph (a call is a
-        few microseconds, shorter than a Python launch)."""
-        s2 = torch.cuda.Stream()
-        s2.wait_stream(stream)
-        with torch.cuda.stream(s2):
-            step()
-        stream.wait_stream(s2)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for _ in range(calls):
-                step()
-        g.replay()
-        torch.cuda.synchronize()
-        return g
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    burst = 20
-    g1, gb = (None, None) if args.no_graph else (graphed(1), graphed(burst))
-    with ClockSampler(local) as clk:
-        t_ms = timed(step if g1 is None else g1.replay, args.steps, True)
-    if gb is None:
-        warm_ms = timed(step, args.steps, False)
-    else:
-        reps = max(1, args.steps // burst)
-        warm_ms = timed(gb.replay, reps, False) * args.steps / (reps * burst)
-    value = throughput(w.n_ids * args.steps, world, t_ms)
-    want = None
-    if rank == 0:
-        import oracle
-        want = oracle.decode_rows_bf16(data["ids"], data["codes"], data["C"], w.decode_scale)
-        assert np.array_equal(rows.view(torch.int16).cpu().numpy().view(np.uint16), want)
-    assert rq.rq_device_error() == 0
-    peak, peak_kind = load_peaks()
-    kern_s = t_ms / args.steps / 1e3
-    nbytes = decode_bytes(w)
-    achieved = nbytes / kern_s / 1e9
-
-    # end to end: ids in from pinned host memory, rows back to the host
-    idh = torch.from_numpy(data["ids"]).pin_memory()
-    rh = torch.empty((w.n_ids, w.D), dtype=torch.bfloat16).pin_memory()
-
-    def e2e_step():
-        ids.copy_(idh, non_blocking=True)
-        step() if g1 is None else g1.replay()
-        rh.copy_(rows, non_blocking=True)
-
-    e2e_step()
-    e_ms = timed(e2e_step, args.steps, True)
-
+    """The row-decode workload alone (decode512)."""
+    rig = Rig(args)
+    data = synth.make(w, seed=rank_seed(rig.rank))
+    art = Artifact(w, data, ("u16",))
+    art.codes_np, art.C_np = data["codes"], data["C"]
+    with ClockSampler(rig.local) as clk:
+        res = measure_decode(rig, w, art, data["ids"], clk=clk)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rig.rank == 0 and rig.world == 1 and not args.no_cpu_baseline:
         import oracle
+        threads = oracle.set_threads(0)
         n, t0 = 0, time.perf_counter()
         while time.perf_counter() - t0 < min(args.cpu_seconds, 5.0):
             oracle.decode_rows_bf16(data["ids"], data["codes"], data["C"], w.decode_scale)
             n += w.n_ids
         el = time.perf_counter() - t0
-        cpu = {"value": n / el, "unit": DEC_UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{n // w.n_ids} calls of {w.n_ids} ids, single-threaded C, {el:.1f} s"}
-    launch = "eager" if g1 is None else "cuda graph"
-    del g1, gb
-    if world > 1:
-        dist.destroy_process_group()
-    if rank != 0:
+        cpu = dict({"value": n / el, "unit": DEC_UNIT, "cores": threads, "kind": "oracle",
+                    "sample": f"{n // w.n_ids} calls of {w.n_ids} ids, C with {threads} OpenMP "
+                              f"thread(s) over ids, {el:.1f} s"}, **cpu_info())
+    rig.close()
+    if rig.rank != 0:
         return
     line = {
-        "metric": DEC_METRIC, "value": value, "unit": DEC_UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
-        "us_per_call": t_ms / args.steps * 1e3, "us_per_call_warm": warm_ms / args.steps * 1e3,
+        "metric": DEC_METRIC, "value": res["value"], "unit": DEC_UNIT, "n_gpus": rig.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "us_per_call": res["us_per_call"], "us_per_call_warm": res["us_per_call_warm"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic", "config": dict(decode_config(w), parallelism=f"replicas x{world}",
-                                            launch=launch),
-        "roofline": {"bound": "hbm", "kernel": "decode_rows_pair_kernel", "achieved": achieved,
-                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": profiled_traffic("decode_rows_pair_kernel/u16/decode512"),
-                     "algorithmic_bytes": nbytes, "kernel_us": kern_s * 1e6},
-        "cpu_baseline": cpu,
-        "e2e": {"value": throughput(w.n_ids * args.steps, world, e_ms), "unit": DEC_UNIT,
-                "h2d_bytes_per_step": w.n_ids * 4, "d2h_bytes_per_step": w.n_ids * w.D * 2,
-                "ms_per_step": e_ms / args.steps},
-        "gpu_launches": args.steps,
+        "data": "synthetic", "config": dict(decode_config(w), parallelism=parallelism()),
+        "launch": res["launch"], "roofline": res["roofline"], "memory": res["memory"],
+        "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": args.steps,
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)

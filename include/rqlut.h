@@ -395,11 +395,11 @@ RQ_API int rq_device_error(uint32_t *out, int clear);
 
 /*
  * rq_lut_logits_static -- rq_lut_logits without a caller-provided workspace,
- * for callers that cannot allocate device memory: work being recorded into
- * a CUDA graph (allocation is not allowed during capture), processes whose
- * device memory belongs to another runtime's allocator, and loops that must
- * not allocate once serving has started.  The paper has no counterpart; this
- * is a convenience of this library.
+ * for callers that cannot allocate device memory: processes whose device
+ * memory belongs to another runtime's allocator, which this library cannot
+ * draw from, and serving loops that must not allocate once they have
+ * started.  The paper has no counterpart; this is a convenience of this
+ * library.
  *   Arguments, results and errors are those of rq_lut_logits, without ws and
  *   ws_bytes.  The workspace comes from a fixed device array inside the
  *   library, RQ_STATIC_SCRATCH_BYTES on every GPU that loads it, held until
@@ -413,6 +413,9 @@ RQ_API int rq_device_error(uint32_t *out, int clear);
  *   may run at the same time on the GPU (different streams without an
  *   ordering between them) race on it and must be serialized by the caller.
  *   Nothing in it needs to start at zero; the kernels reset what they use.
+ *   The looked-up address is cached per device index for the life of the
+ *   process: do not use the library across a cudaDeviceReset (the same holds
+ *   for the device error word behind rq_device_error).
  */
 #define RQ_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
 RQ_API int rq_lut_logits_static(const void *codes, int fmt, rq_dims d, const float *lut,

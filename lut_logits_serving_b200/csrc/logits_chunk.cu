@@ -596,18 +596,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// looked up once (a function-local static: initialised by one thread)
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -733,18 +732,11 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
-  // the shared-memory limit set so far per (device, instance): raised when a
-  // larger K needs more (plain-code tables scale with K)
-  constexpr int NV = sizeof(kVariants) / sizeof(kVariants[0]);
-  static size_t smem_set[128][NV] = {};
-  static int occ_cache[128][NV] = {};
-  static size_t occ_smem[128][NV] = {};
-  if (di.device >= 128) return cudaErrorInvalidDevice;
-  if (cp.smem > smem_set[di.device][cp.variant]) {
-    cudaError_t e = cudaFuncSetAttribute(var.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)cp.smem);
+  // the shared-memory limit is raised when a larger K needs more (plain-code
+  // tables scale with K)
+  {
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(var.fn), di.device, cp.smem);
     if (e != cudaSuccess) return e;
-    smem_set[di.device][cp.variant] = cp.smem;
   }
 
   ChunkArgs a;
@@ -759,15 +751,8 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   a.B = B;
   a.nch = cp.nch;
   // CTAs per SM this instance reaches (shared memory and registers)
-  int occ = occ_cache[di.device][cp.variant];
-  if (occ == 0 || occ_smem[di.device][cp.variant] != cp.smem) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, var.fn, var.THREADS, cp.smem) !=
-            cudaSuccess ||
-        occ < 1)
-      occ = 1;
-    occ_cache[di.device][cp.variant] = occ;
-    occ_smem[di.device][cp.variant] = cp.smem;
-  }
+  const int occ =
+      occupancy_cached(reinterpret_cast<const void *>(var.fn), di.device, var.THREADS, cp.smem);
   int64_t cpc = (int64_t)di.sms * occ / cp.nch;
   if (cpc < 1) cpc = 1;
   if (cpc > a.ntiles) cpc = a.ntiles;

@@ -368,13 +368,10 @@ cudaError_t launch_logits_decode_fma(const float *h, const float *C, const void 
                           kDfStageCodes, 256, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
   const size_t smem = decode_fma_smem(K);
-  static size_t smem_set[128] = {};
-  if (di.device >= 128) return cudaErrorInvalidDevice;
-  if (smem > smem_set[di.device]) {
-    cudaError_t e = cudaFuncSetAttribute(logits_decode_fma_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(&logits_decode_fma_kernel),
+                                      di.device, smem);
     if (e != cudaSuccess) return e;
-    smem_set[di.device] = smem;
   }
   DfArgs a;
   a.h = h;

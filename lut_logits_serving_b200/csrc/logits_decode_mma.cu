@@ -587,13 +587,10 @@ cudaError_t launch_dm(const float *h, const float *C, const void *codes, int64_t
     if (e != cudaSuccess) return e;
   }
   const size_t smem = dm_smem<NT, FMT>(K);
-  static size_t smem_set[128] = {};
-  if (di.device >= 128) return cudaErrorInvalidDevice;
   const void *fn = reinterpret_cast<const void *>(&logits_decode_mma_kernel<NT, FMT>);
-  if (smem > smem_set[di.device]) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e = ensure_smem_limit(fn, di.device, smem);
     if (e != cudaSuccess) return e;
-    smem_set[di.device] = smem;
   }
   DmArgs a;
   a.C = C;

@@ -341,6 +341,16 @@ struct DevInfo {
 
 cudaError_t dev_info(DevInfo *out);
 
+// Raises the dynamic shared-memory limit of kernel `fn` on `device` (the
+// current device) to at least `smem` bytes.  The limit set so far is kept per
+// (kernel, device) under a lock, so concurrent host threads may launch.
+cudaError_t ensure_smem_limit(const void *fn, int device, size_t smem);
+
+// CTAs of `fn` resident per SM with `threads` threads and `smem` bytes of
+// dynamic shared memory (at least 1), computed once per (kernel, device,
+// smem) under a lock.
+int occupancy_cached(const void *fn, int device, int threads, size_t smem);
+
 cudaError_t launch_lut_build(const float *h, const float *C, int B, int b0, int nb, int D,
                              int M, int L, int K, int Bs, float *lut, cudaStream_t s);
 

@@ -1,6 +1,9 @@
 // rqlut_api.cu -- the C ABI of librqlut (see include/rqlut.h): argument
 // validation, workspace layout, path selection and launches.
+#include <map>
 #include <mutex>
+#include <tuple>
+#include <utility>
 
 #include "rq_common.cuh"
 
@@ -41,6 +44,34 @@ cudaError_t dev_info(DevInfo *out) {
   }
   *out = d;
   return cudaSuccess;
+}
+
+namespace {
+std::mutex g_attr_mu;
+std::map<std::pair<const void *, int>, size_t> g_smem_limit;
+std::map<std::tuple<const void *, int, int, size_t>, int> g_occupancy;
+}  // namespace
+
+cudaError_t ensure_smem_limit(const void *fn, int device, size_t smem) {
+  std::lock_guard<std::mutex> g(g_attr_mu);
+  size_t &have = g_smem_limit[std::make_pair(fn, device)];
+  if (smem <= have) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) have = smem;
+  return e;
+}
+
+int occupancy_cached(const void *fn, int device, int threads, size_t smem) {
+  std::lock_guard<std::mutex> g(g_attr_mu);
+  int &occ = g_occupancy[std::make_tuple(fn, device, threads, smem)];
+  if (occ == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    occ = n;
+  }
+  return occ;
 }
 
 // Device-independent sizing: the B200 limits (148 SMs, 227 KB opt-in shared

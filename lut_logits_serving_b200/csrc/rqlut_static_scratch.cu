@@ -2,12 +2,11 @@
 // callers that cannot allocate device memory themselves.
 //
 // rq_lut_logits needs a device workspace (per-chunk partial sums, argmax
-// partials, a reduction counter).  Some callers have no way to provide one:
-// code recorded into a CUDA graph while capture is active (no allocation
-// allowed then), hosts whose device memory is owned by another runtime's
-// pool, or embedded/real-time loops that must never allocate after start-up.
-// This entry point takes the workspace from a fixed array in the library's
-// own device memory instead.
+// keys).  Some callers have no way to provide one: hosts whose device memory
+// is owned by another runtime's pool, which this library cannot draw from,
+// or embedded and real-time serving loops that must never allocate once
+// they have started.  This entry point takes the workspace from a fixed
+// array in the library's own device memory instead.
 #include <mutex>
 
 #include "rq_common.cuh"
@@ -43,17 +42,17 @@ int static_scratch(void **out) {
 extern "C" int rq_lut_logits_static(const void *codes, int fmt, rq_dims d, const float *lut,
                                     int B, float softcap, float *logits, int32_t *argmax,
                                     void *stream) {
-  // The same workspace rq_lut_logits would ask for; refuse what does not fit.
+  // Refuse early, launching nothing, what cannot fit on a B200; the call
+  // below checks the scratch size again against the plan of the device it
+  // runs on, which may differ.
   const size_t need = rq_logits_workspace_bytes(d, B, fmt, argmax != nullptr ? 1 : 0);
   if (need > (size_t)RQ_STATIC_SCRATCH_BYTES) return RQ_ERR_WORKSPACE_TOO_SMALL;
   void *ws = nullptr;
-  if (need > 0) {
-    const int st = static_scratch(&ws);
-    if (st != RQ_OK) return st;
-  }
-  // Nothing in the scratch has to start at zero: the partial sums and argmax
-  // partials are written before they are read, and the reduction counter is
-  // reset by the code-pass kernel at the start of every call.
+  const int st = static_scratch(&ws);
+  if (st != RQ_OK) return st;
+  // Nothing in the scratch has to start at zero: the partial sums are
+  // written before they are read, and the code pass zeroes the argmax keys
+  // at the start of every call, before the reduce folds values into them.
   return rq_lut_logits(codes, fmt, d, lut, B, softcap, logits, argmax, ws,
-                       need > 0 ? (size_t)RQ_STATIC_SCRATCH_BYTES : 0, stream);
+                       (size_t)RQ_STATIC_SCRATCH_BYTES, stream);
 }

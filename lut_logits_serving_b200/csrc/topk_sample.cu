@@ -363,13 +363,11 @@ cudaError_t launch_topk_sample(const float *logits, int64_t V, int B, int k, dou
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr[128] = {};
   const size_t smem = (size_t)kTopkCap * sizeof(unsigned long long);
-  if (dev < 128 && !attr[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(topk_gather_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e =
+        ensure_smem_limit(reinterpret_cast<const void *>(&topk_gather_kernel), dev, smem);
     if (e != cudaSuccess) return e;
-    attr[dev] = true;
   }
   cudaError_t e = cudaMemsetAsync(w.hist, 0, (size_t)B * (kTopkBins + 2) * sizeof(unsigned), s);
   if (e != cudaSuccess) return e;

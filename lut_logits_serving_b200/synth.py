@@ -55,6 +55,10 @@ WORKLOADS = {
     "g2_b1": Workload("g2_b1", V=256000, D=2304, M=384, L=2, K=1024, B=1,
                       sigmas=(0.02, 0.005), hidden_scale=40.0 / math.sqrt(2304.0),
                       argmax=True, n_ids=1, decode_scale=math.sqrt(2304.0)),
+    # a batch in the range the L2-served tables take (5 to 16 tokens)
+    "g2_b16": Workload("g2_b16", V=256000, D=2304, M=384, L=2, K=1024, B=16,
+                       sigmas=(0.02, 0.005), hidden_scale=0.83,
+                       argmax=True, n_ids=16, decode_scale=math.sqrt(2304.0)),
     "g2_b32": Workload("g2_b32", V=256000, D=2304, M=384, L=2, K=1024, B=32,
                        sigmas=(0.02, 0.005), hidden_scale=0.83,
                        argmax=True, n_ids=32, decode_scale=math.sqrt(2304.0)),

@@ -46,9 +46,10 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (plain C99, no FMA contraction)."""
+    """Compile the oracle with gcc (plain C99, no FMA contraction; OpenMP
+    splits the row loops across host threads without changing any result)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math",
+        cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
                "-fPIC", "-shared", "-o", _LIB + ".tmp", _SRC, "-lm"]
         subprocess.check_call(cmd)
         os.replace(_LIB + ".tmp", _LIB)
@@ -87,6 +88,8 @@ def _load():
         "rqo_uniform": (_d, [ctypes.c_uint64, ctypes.c_uint64, _i64]),
         "rqo_topk_f32": (None, [_p, _i64, _i, _p, _p, _p]),
         "rqo_sample_position": (_i, [_p, _i, _d, _d]),
+        "rqo_set_threads": (None, [_i]),
+        "rqo_max_threads": (_i, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -94,6 +97,14 @@ def _load():
         fn.argtypes = args
     _lib = lib
     return lib
+
+
+def set_threads(n: int) -> int:
+    """Host threads of the row loops (n < 1: all); returns the count now in
+    use.  Results are the same for every count."""
+    lib = _load()
+    lib.rqo_set_threads(int(n))
+    return int(lib.rqo_max_threads())
 
 
 def _c(a: np.ndarray, dtype) -> np.ndarray:

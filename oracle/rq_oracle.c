@@ -31,6 +31,12 @@
  * sums run in the order written (j, then m-major / l-minor, then i), and the
  * file is compiled with -ffp-contract=off so no multiply-add is fused.
  *
+ * Threads.  Built with OpenMP, the loops over vocabulary rows (and over
+ * the rows to decode or encode, and the table entries) are split across
+ * host threads.  Each output element is still computed by one thread in the
+ * order written above, so the results do not depend on the thread count;
+ * rqo_set_threads(1) gives the single-threaded timing.
+ *
  * Layouts (plain row-major C arrays):
  *   h      float  [B][D]
  *   C      float  [M][L][K][ds]
@@ -68,6 +74,30 @@
 #include <stdint.h>
 #include <stddef.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ threads */
+
+/* Host threads the parallel loops use (n < 1: all the runtime offers). */
+void rqo_set_threads(int n)
+{
+#ifdef _OPENMP
+    omp_set_num_threads(n > 0 ? n : omp_get_num_procs());
+#else
+    (void)n;
+#endif
+}
+
+int rqo_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* ---------------------------------------------------------------- LUT build */
 
@@ -75,6 +105,7 @@ void rqo_lut_build_f64(const float *h, int B, const float *C, int D, int M,
                        int L, int K, double *T)
 {
     int ds = D / M;
+    #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
         for (int m = 0; m < M; ++m)
             for (int l = 0; l < L; ++l)
@@ -92,6 +123,7 @@ void rqo_lut_build_f32(const float *h, int B, const float *C, int D, int M,
                        int L, int K, float *T)
 {
     int ds = D / M;
+    #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
         for (int m = 0; m < M; ++m)
             for (int l = 0; l < L; ++l)
@@ -114,6 +146,7 @@ void rqo_logits_lut_f64(const uint16_t *codes, int64_t V, int M, int L, int K,
                         int64_t nrows, double *z)
 {
     (void)V;
+    #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
         for (int64_t r = 0; r < nrows; ++r) {
             const uint16_t *cr = codes + (size_t)rows[r] * M * L;
@@ -132,6 +165,7 @@ void rqo_logits_lut_f32(const uint16_t *codes, int64_t V, int M, int L, int K,
                         int64_t nrows, float *z)
 {
     (void)V;
+    #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
         for (int64_t r = 0; r < nrows; ++r) {
             const uint16_t *cr = codes + (size_t)rows[r] * M * L;
@@ -153,6 +187,7 @@ void rqo_logits_direct_f64(const uint16_t *codes, int64_t V, const float *C,
 {
     (void)V;
     int ds = D / M;
+    #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
         for (int64_t r = 0; r < nrows; ++r) {
             const uint16_t *cr = codes + (size_t)rows[r] * M * L;
@@ -176,6 +211,7 @@ void rqo_logits_direct_f32(const uint16_t *codes, int64_t V, const float *C,
 {
     (void)V;
     int ds = D / M;
+    #pragma omp parallel for collapse(2) schedule(static)
     for (int b = 0; b < B; ++b)
         for (int64_t r = 0; r < nrows; ++r) {
             const uint16_t *cr = codes + (size_t)rows[r] * M * L;
@@ -250,6 +286,7 @@ void rqo_decode_rows_bf16(const int32_t *ids, int64_t N, const uint16_t *codes,
 {
     (void)V;
     int ds = D / M;
+    #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
         const uint16_t *cr = codes + (size_t)ids[n] * M * L;
         for (int m = 0; m < M; ++m)
@@ -310,9 +347,10 @@ void rqo_encode_f32(const float *X, int64_t N, const float *C, int D, int M,
                     int L, int K, uint16_t *codes)
 {
     int ds = D / M;
-    float r[64];
+    #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n)
         for (int m = 0; m < M; ++m) {
+            float r[64];
             for (int j = 0; j < ds; ++j)
                 r[j] = X[n * D + (int64_t)m * ds + j];
             for (int l = 0; l < L; ++l) {

@@ -19,7 +19,9 @@ def test_reference_arm_prints_one_json_line():
     assert j["impl"] == "reference"
     assert j["unit"] == "vocab-rows/s" and j["higher_is_better"] is True
     assert j["value"] > 0 and j["steps"] == 2 and j["warmup"] == 1
-    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] == 1
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
+    assert j["cpu_baseline"]["nproc"] == os.cpu_count() and j["cpu_baseline"]["cpu_model"]
+    assert j["config"]["parallelism"] == "replicas x1"
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
     assert j["config"]["V"] == 256000
 
@@ -39,6 +41,7 @@ def test_reference_arm_on_the_row_decode_workload():
     j = json.loads(lines[0])
     assert j["impl"] == "reference" and j["metric"] == bench.DEC_METRIC
     assert j["unit"] == "rows/s" and j["value"] > 0
-    assert j["config"] == bench.decode_config(synth.WORKLOADS["decode512"])
+    assert j["config"] == dict(bench.decode_config(synth.WORKLOADS["decode512"]),
+                               parallelism="replicas x1")
     assert j["config"]["ids"] == 512
     assert j["cpu_baseline"]["value"] == j["value"] and j["e2e"]["value"] == j["value"]

@@ -3,10 +3,10 @@ K=1024), in the launch configuration the benchmark times.
 
 * decode batch 1, uint16 codes: all 256000 logits and the argmax against
   the oracle (the oracle does the full row sweep in about a second);
-* batch 32, uint16 codes, one code pass for all tokens: 4096 sampled rows for
-  every token, the full sweep and the argmax for four tokens;
+* batch 32, uint16 codes, one code pass for all tokens: all 32 x 256000
+  logits and every token's argmax, on every kernel choice;
 * batch 64, 10-bit packed codes, fused build + unpack + sum + softcap +
-  argmax: sampled rows for every token, full argmax for four tokens;
+  argmax: all 64 x 256000 logits and every token's argmax;
 * 512 Zipf-drawn input rows rebuilt in bf16: all of them, bit for bit.
 """
 import numpy as np
@@ -76,9 +76,31 @@ def test_g2_batch1_full_sweep(g2):
     assert rq.rq_device_error() == 0
 
 
-def _batched(g2, w, fmt, seed_rows, path=None):
+_REF = {}
+
+
+def _full_ref(g2, w):
+    """The oracle's fp64 logits of every token and row (computed once per
+    workload; the oracle's row loop runs on all host cores)."""
+    if w.name not in _REF:
+        h = synth.hidden(w.B, w.D, w.hidden_scale, 2)
+        T = oracle.lut_build(h, g2["C"], "f64")
+        _REF[w.name] = (h, oracle.softcap(oracle.logits_lut(g2["codes"], T), w.softcap))
+    return _REF[w.name]
+
+
+def elementwise_rel(got, ref, floor=1e-2):
+    """Largest elementwise relative error over the logits whose magnitude is
+    at least `floor` of their token's largest (reported, not gated: below that
+    the ratio measures cancellation, not the kernel)."""
+    ref = np.asarray(ref, np.float64)
+    big = np.abs(ref) >= floor * np.max(np.abs(ref), axis=1, keepdims=True)
+    return float(np.max(np.abs(got.astype(np.float64)[big] - ref[big]) / np.abs(ref[big])))
+
+
+def _batched(g2, w, fmt, path=None):
     d = g2["d"]
-    h = synth.hidden(w.B, w.D, w.hidden_scale, 2)
+    h, ref = _full_ref(g2, w)
     codes_dev = g2["dc"] if fmt == rq.U16 else rq.rq_pack10(g2["dc"], d)
     # NaN-filled output: a kernel that writes nothing cannot pass on stale memory
     out = torch.full((w.B, w.V), float("nan"), device="cuda")
@@ -87,24 +109,19 @@ def _batched(g2, w, fmt, seed_rows, path=None):
     assert rq.rq_device_error() == 0
     got = logits.cpu().numpy()
     amv = am.cpu().numpy()
-    T = oracle.lut_build(h, g2["C"], "f64")
-    rows = _sample_rows(w.V, 4096, seed_rows)
-    ref = oracle.softcap(oracle.logits_lut(g2["codes"], T, rows), w.softcap)
-    err = assert_logits_close(got[:, rows], ref)
-    full_tokens = [0, 1, w.B // 2, w.B - 1]
-    ref_full = oracle.softcap(oracle.logits_lut(g2["codes"], T[full_tokens]), w.softcap)
-    assert_logits_close(got[full_tokens], ref_full)
-    ties = check_argmax(amv[full_tokens], ref_full)
-    # every token's argmax is the argmax of the GPU's own logits
+    err = assert_logits_close(got, ref)          # every token, every row
+    ties = check_argmax(amv, ref)                 # every token
+    # every token's argmax is also the argmax of the GPU's own logits
     assert np.array_equal(amv, np.argmax(got, axis=1))
-    return err, ties
+    return err, elementwise_rel(got, ref), ties
 
 
 @pytest.mark.parametrize("path", [None, rq.PATH_TABLES, rq.PATH_DECODE_FP32, rq.PATH_DECODE_TC])
 def test_g2_batch32_one_code_pass(g2, path):
     w = synth.WORKLOADS["g2_b32"]
-    err, ties = _batched(g2, w, rq.U16, 7, path)
-    print(f"g2_b32 path {path} normwise error {err:.3g}, ties {ties}")
+    err, rel, ties = _batched(g2, w, rq.U16, path)
+    print(f"g2_b32 path {path} normwise error {err:.3g}, elementwise relative error "
+          f"(|ref| >= 1e-2 max) {rel:.3g}, ties {ties}")
     assert ties == 0
     assert rq.rq_device_error() == 0
 
@@ -115,8 +132,9 @@ def test_g2_packed_batch64_fused_argmax(g2, path):
     packed = rq.rq_pack10(g2["dc"], g2["d"]).cpu().numpy()
     rows = _sample_rows(w.V, 2000, 11)
     assert np.array_equal(packed[rows], oracle.pack10(g2["codes"][rows]))
-    err, ties = _batched(g2, w, rq.PACKED10, 9, path)
-    print(f"packed_b64 path {path} normwise error {err:.3g}, ties {ties}")
+    err, rel, ties = _batched(g2, w, rq.PACKED10, path)
+    print(f"packed_b64 path {path} normwise error {err:.3g}, elementwise relative error "
+          f"(|ref| >= 1e-2 max) {rel:.3g}, ties {ties}")
     assert ties == 0
 
 

@@ -502,3 +502,27 @@ def test_topk():
 
 def test_sampling():
     check_sampling()
+
+
+def test_thread_count_changes_no_result():
+    """The oracle's row loops run on host threads (OpenMP); every output is
+    computed by one thread in the written order, so one thread and all of
+    them give the same bits."""
+    w = synth.WORKLOADS["tiny"]
+    data = synth.make(w)
+    h = synth.hidden(3, w.D, w.hidden_scale, 2)
+    X = synth.rows(50, w.D, synth.row_sigma(w), 4)
+    ids = synth.zipf_ids(40, w.V, 1.1, 3)
+    outs = []
+    for n in (1, 0):
+        oracle.set_threads(n)
+        T = oracle.lut_build(h, data["C"], "f64")
+        T32 = oracle.lut_build(h, data["C"], "f32")
+        outs.append((T, T32, oracle.logits_lut(data["codes"], T),
+                     oracle.logits_lut(data["codes"], T32),
+                     oracle.logits_direct(data["codes"], data["C"], h, precision="f64"),
+                     oracle.decode_rows_bf16(ids, data["codes"], data["C"], 8.0),
+                     oracle.encode(X, data["C"])))
+    oracle.set_threads(0)
+    for a, b in zip(*outs):
+        assert a.dtype == b.dtype and np.array_equal(a, b)

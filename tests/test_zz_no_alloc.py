@@ -1,6 +1,6 @@
 """rq_lut_logits_static: the logits call that allocates nothing, for callers
-that cannot allocate device memory (capture in progress, memory owned by
-another allocator, loops that must not allocate).  It must give what
+that cannot allocate device memory (memory owned by another runtime's
+allocator, serving loops that must not allocate once started).  It must give what
 rq_lut_logits gives with a workspace the caller allocated, on consecutive
 calls that reuse its fixed scratch, and refuse a call whose workspace would
 not fit.  This file is collected last on purpose."""
