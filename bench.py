@@ -108,7 +108,7 @@ def headline_layout(w, codes=None, available=("sched", "u16", "u8")):
 
 
 def code_bytes(w, codes="u16"):
-    if w.packed10:
+    if w.packed10 or codes == "packed10":
         return w.V * (w.P * 10 // 8)
     return w.V * w.P * (1 if codes == "u8" else 2)
 

@@ -120,3 +120,9 @@ def test_workload_choices_cover_the_workloads():
         parse_argv(["--workload", "nope"])
     a = parse_argv([])
     assert (a.gpus, a.workload, a.impl) == (1, "g2_b1", "ours") and a.warmup >= 3
+
+
+def test_packed_code_bytes_on_a_uint16_workload():
+    """A batch-1 workload timed on 10-bit packed codes divides by the packed
+    matrix (960 B per row), not by the uint16 one."""
+    assert bench.code_bytes(synth.WORKLOADS["g2_b1"], "packed10") == 256000 * 960
