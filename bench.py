@@ -830,7 +830,10 @@ def measure_logits(rig, w, art, layout, h_np, full=False, clk=None):
     ne2e = min(args.steps, 2000)
     outs = [(dh0, logits0, am0, rows0, tok0), (torch.empty_like(dh0),) + outputs()]
     # the compute of each set replays as a CUDA graph, as in the device timing
-    steps2 = [run, rig.graphed(make_step(fmt, dcodes, outs[1]))]
+    # (the step object, and so its workspace, lives as long as its graph: a
+    # later capture empties torch's cache and would free a dropped workspace)
+    step_b = make_step(fmt, dcodes, outs[1])
+    steps2 = [run, rig.graphed(step_b)]
     hosts = [(torch.empty((w.B, w.V), dtype=torch.float32).pin_memory(),
               torch.empty((w.B,), dtype=torch.int32).pin_memory()) for _ in range(2)]
     d2h_stream, h2d_stream = torch.cuda.Stream(), torch.cuda.Stream()

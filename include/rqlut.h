@@ -129,7 +129,8 @@ RQ_API size_t rq_lut_bytes(rq_dims d, int B);
 RQ_API size_t rq_logits_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax);
 
 /* Device workspace of rq_logits_from_hidden (includes the lookup table of
- * one token group). */
+ * one token group or, where the shape can take the tensor-core decode, that
+ * kernel's scratch -- split hidden states and codebooks -- if larger). */
 RQ_API size_t rq_fused_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax);
 
 /*

@@ -27,7 +27,7 @@ def sources():
 
 
 def headers():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + \
+    return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))) + \
         [os.path.join(os.path.dirname(HERE), "include", "rqlut.h")]
 
 

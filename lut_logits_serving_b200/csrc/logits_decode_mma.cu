@@ -808,15 +808,22 @@ size_t decode_mma_smem(int K, int N, int fmt) {
   return packed ? dm_smem<64, RQ_CODES_PACKED10>(K) : dm_smem<64, RQ_CODES_U16>(K);
 }
 
-size_t decode_mma_hop_bytes(int M, int N) { return (size_t)kDmHopHead + (size_t)M * 2 * N * 32; }
+size_t decode_mma_hop_bytes(int M, int N, int K) {
+  (void)K;
+  return (size_t)kDmHopHead + (size_t)M * 2 * N * 32;
+}
 
-bool decode_mma_applies(int fmt, int64_t V, int D, int M, int L, int K, const float *C,
-                        const void *codes) {
+bool decode_mma_shape_ok(int fmt, int64_t V, int D, int M, int L, int K) {
   if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return false;
   if (L != 2 || D != 6 * M || K > 1024 || K < 1) return false;
   if (M % (fmt == RQ_CODES_PACKED10 ? 32 : 8) != 0) return false;
-  if (V < 1 || V > (int64_t)INT_MAX - 2048) return false;
-  return (reinterpret_cast<uintptr_t>(C) & 15) == 0 && (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
+  return V >= 1 && V <= (int64_t)INT_MAX - 2048;
+}
+
+bool decode_mma_applies(int fmt, int64_t V, int D, int M, int L, int K, const float *C,
+                        const void *codes) {
+  return decode_mma_shape_ok(fmt, V, D, M, L, K) && (reinterpret_cast<uintptr_t>(C) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
 }
 
 cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void *codes, int fmt,

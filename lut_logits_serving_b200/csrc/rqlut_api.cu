@@ -224,6 +224,19 @@ int run_logits(const void *codes, int fmt, const rq_dims &d, const float *lut, i
 
 int fused_group(int B) { return B <= 4 ? B : (B < kTokenGroup ? B : kTokenGroup); }
 
+// First region of the fused calls' workspace: the token group's tables, or,
+// for a group decoded on the tensor cores, that kernel's scratch (scales,
+// split hidden operand, split codebooks) -- whichever is larger, for every
+// shape the tensor-core kernel can take.
+size_t table_region_bytes(const rq_dims &d, int B, int fmt) {
+  size_t n = (size_t)align_up((int64_t)rq_lut_bytes(d, fused_group(B)), kAlign);
+  if (B > 4 && decode_mma_shape_ok(fmt, d.V, d.D, d.M, d.L, d.K)) {
+    const size_t tc = (size_t)align_up((int64_t)decode_mma_hop_bytes(d.M, 64, d.K), kAlign);
+    if (tc > n) n = tc;
+  }
+  return n;
+}
+
 // Smallest partial token group (fewer than 32 tokens) that the fused calls
 // send to the tensor cores: with RQ_PATH_DECODE_TC every group does (down to
 // one token); by default from the size where the tables measured slower.
@@ -242,7 +255,7 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   const int G = fused_group(B);
   const int Bs = rq_lut_token_stride(G);
   if ((size_t)Bs * (d.D / d.M) * 4 > 48 * 1024) return RQ_ERR_UNSUPPORTED;
-  const size_t lut_bytes = (size_t)align_up((int64_t)rq_lut_bytes(d, G), kAlign);
+  const size_t lut_bytes = table_region_bytes(d, B, fmt);
   const WsLayout w = ws_layout(d, B, fmt, argmax != nullptr, di);
   if (ws_bytes < lut_bytes + w.total) return RQ_ERR_WORKSPACE_TOO_SMALL;
   float *lut = static_cast<float *>(ws);
@@ -266,11 +279,11 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   const bool grid_ok = decode_fma_blocks(d.V, di) <= nblk;
   const bool dfma = grid_ok && decode_fma_applies(fmt, d.V, d.D, d.M, d.L, d.K, B, C, codes, di);
   const bool tc_fmt = grid_ok && decode_mma_applies(fmt, d.V, d.D, d.M, d.L, d.K, C, codes);
-  // the tensor-core kernel keeps the group's split hidden operand in the
-  // (here unused) table region
+  // the tensor-core kernel keeps its scratch (scales, split hidden operand,
+  // split codebooks) in the (here unused) table region
   auto tc_fits = [&](int n) {
     return tc_fmt && decode_mma_smem(d.K, n, fmt) <= (size_t)di.max_smem_optin &&
-           decode_mma_hop_bytes(d.M, n) <= lut_bytes;
+           decode_mma_hop_bytes(d.M, n, d.K) <= lut_bytes;
   };
   const bool tc32 = tc_fits(32), tc64 = tc_fits(64);
   if ((path == RQ_PATH_DECODE_FP32 && !dfma) || (path == RQ_PATH_DECODE_TC && !tc32))
@@ -369,8 +382,7 @@ size_t rq_logits_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax) {
 
 size_t rq_fused_workspace_bytes(rq_dims d, int B, int fmt, int want_argmax) {
   if (!dims_ok(d) || !fmt_ok(d, fmt) || B < 1) return 0;
-  const int G = fused_group(B);
-  const size_t lut = (size_t)align_up((int64_t)rq_lut_bytes(d, G), kAlign);
+  const size_t lut = table_region_bytes(d, B, fmt);
   return lut + ws_layout(d, B, fmt, want_argmax != 0, nominal_devinfo()).total;
 }
 

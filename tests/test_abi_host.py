@@ -82,6 +82,13 @@ def test_workspace_sizes():
     f64 = rq.rq_fused_workspace_bytes(G2, 64, rq.PACKED10, True)
     assert f64 >= rq.rq_lut_bytes(G2, 32)
     assert f64 < rq.rq_lut_bytes(G2, 64)
+    # a small shape the tensor-core decode can take: its scratch (split hidden
+    # states and codebooks) is larger than an 8-token table, and the fused
+    # workspace covers it; a shape it cannot take keeps the table size
+    small = rq.dims(1000, 48, 8, 2, 64)
+    assert rq.rq_fused_workspace_bytes(small, 8, rq.U16, False) > rq.rq_lut_bytes(small, 8)
+    odd = rq.dims(1000, 40, 8, 2, 64)                  # ds = 5
+    assert rq.rq_fused_workspace_bytes(odd, 8, rq.U16, False) == rq.rq_lut_bytes(odd, 8)
     # never O(V*M*L) (the pages' naive gather index would be 1.57 GB)
     for B in (1, 2, 3, 4, 5, 32, 64):
         assert rq.rq_logits_workspace_bytes(G2, B, rq.U16, True) < 256000 * 768 * 8
