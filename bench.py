@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="g2_b1",
-                    choices=["g2_b1", "g2_b16", "g2_b32", "packed_b64", "mlp_gate_b1",
+                    choices=["g2_b1", "g2_b1_packed10", "g2_b16", "g2_b32", "packed_b64", "mlp_gate_b1",
                              "mlp_down_b1", "encode_g2", "g2_b1_topk50", "decode512"])
     ap.add_argument("--codes", default=None, choices=["u16", "sched", "u8"],
                     help="code layout of the unpacked workloads timed for `value`: "
@@ -511,7 +511,7 @@ def launches_per_step(w, decoded):
     two kernels per token group (hidden split + tensor-core decode, or table
     build + L2 pass); then the argmax finish that also rebuilds the picked
     rows, or the top-k draw and the row decode."""
-    if w.B <= 4 and not w.packed10:
+    if w.B <= 4 and (not w.packed10 or w.B == 1):
         n = 3 + (1 if w.argmax else 0)
     else:
         n = 2 * len(token_groups(w, decoded)) + (1 if w.argmax else 0)
@@ -654,7 +654,8 @@ class Artifact:
 
 def kernel_of(w, layout):
     decoded = layout in ("u16", "packed10") and decodable(w)
-    if w.B <= 4 and not w.packed10 and layout != "packed10":
+    packed = w.packed10 or layout == "packed10"
+    if w.B <= 4 and (not packed or w.B == 1):
         return "logits_chunk_u16_kernel", decoded
     return ("logits_decode_mma_kernel" if decoded else "logits_l2_kernel"), decoded
 

@@ -198,12 +198,12 @@ RQ_API int rq_logits_from_hidden(const float *h, const float *C, const void *cod
  *   RQ_PATH_DECODE_FP32 -- groups of 32; rows decoded into shared memory,
  *                          fp32 FMAs; RQ_CODES_U16 with M % 8 == 0
  *   RQ_PATH_DECODE_TC   -- groups of 64, then 32, then the rest; rows
- *                          decoded into tensor memory, tcgen05 tf32 MMAs on
- *                          a hi/lo split with fp32 chain sums;
- *                          RQ_CODES_U16 with M % 8 == 0 or
- *                          RQ_CODES_PACKED10 with M % 32 == 0; K >= 8 (16 for
- *                          groups of 64: the hidden operand is staged in the
- *                          workspace's table region)
+ *                          decoded into tensor memory, tcgen05 fp16 MMAs on
+ *                          hi/lo splits of the rows and hidden states (with
+ *                          power-of-two scales), fp32 sums of short MMA
+ *                          chains; RQ_CODES_U16 with M % 8 == 0 or
+ *                          RQ_CODES_PACKED10 with M % 32 == 0 (its scratch
+ *                          lives in the workspace's table region)
  */
 enum { RQ_PATH_AUTO = 0, RQ_PATH_TABLES = 1, RQ_PATH_DECODE_FP32 = 2, RQ_PATH_DECODE_TC = 3 };
 

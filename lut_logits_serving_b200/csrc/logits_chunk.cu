@@ -26,6 +26,7 @@
 //     writes the logits and reduces the argmax (its last block finishes it).
 #include <cfloat>
 #include <climits>
+#include <utility>
 
 #include "rq_common.cuh"
 
@@ -46,10 +47,14 @@ struct ChunkArgs {
 // Plain uint16 codes: TPR threads per row, 1024 threads.  Bank-scheduled codes
 // (one token): one thread per row owns the row's whole 32-pair slice, the
 // unit the schedule was made for, 512 threads.  Byte codes: one thread per
-// row and 32-pair slice (32 bytes), 512 threads.
+// row and 32-pair slice (32 bytes), 512 threads.  10-bit codes (one token,
+// M*L % 64 == 0): one thread per row and 32-pair slice, whose 40 bytes start
+// at byte 40c of the row -- 8 bytes off a 16-byte boundary for odd c -- so
+// the TMA box is the 48-byte, 16-byte-aligned window around it.
 template <int TB, int FMT>
 struct ChunkShape {
-  static constexpr bool WHOLE = FMT == RQ_CODES_SCHED || FMT == RQ_CODES_U8;
+  static constexpr bool PK10 = FMT == RQ_CODES_PACKED10;
+  static constexpr bool WHOLE = FMT == RQ_CODES_SCHED || FMT == RQ_CODES_U8 || PK10;
   static constexpr int PC = WHOLE ? 32 : (TB == 1 ? 32 : (TB == 2 ? 16 : 8));  // pairs/chunk
   static constexpr int PPT = WHOLE ? 32 : (TB == 4 ? 8 : 16);                  // pairs/thread
   static constexpr int TPR = PC / PPT;                          // threads per row
@@ -57,11 +62,12 @@ struct ChunkShape {
   static constexpr int WARPS = THREADS / 32;
   static constexpr int R = THREADS / TPR;                       // rows per tile
   static constexpr int CB = FMT == RQ_CODES_U8 ? 1 : 2;         // bytes per code
-  static constexpr int ROWB = PC * CB;                          // code bytes per row slice
+  static constexpr int ROWB = PK10 ? 48 : PC * CB;              // code bytes per row slice
   static constexpr int BOXES = R / 256;
   static constexpr int BOX_BYTES = 256 * ROWB;
   static constexpr int STAGE_BYTES = R * ROWB;
   static constexpr int CPV = 16 / CB;                           // codes per 16-byte vector
+  static constexpr int NQ = PK10 ? 3 : PPT / CPV;               // 16-byte vectors per thread
 };
 
 // 16-byte chunk j of row r (row index inside a 1024-byte-aligned TMA box) as
@@ -202,6 +208,51 @@ __device__ __forceinline__ float chunk32_sched_tb1(uint32_t tbase, const uint4 (
   return x[0];
 }
 
+template <int OFF>
+__device__ __forceinline__ float lds_f32_imm(uint32_t addr) {
+  float x;
+  asm("ld.shared.f32 %0, [%1+%2];" : "=f"(x) : "r"(addr), "n"(OFF));
+  return x;
+}
+
+// Code j of a 32-code, 10-bit slice held LSB-first in x[0..9] (x[10] = 0).
+template <int J>
+__device__ __forceinline__ uint32_t pk10_code(const uint32_t (&x)[11]) {
+  return __funnelshift_r(x[(10 * J) >> 5], x[((10 * J) >> 5) + 1], (10 * J) & 31) & 0x3FFu;
+}
+
+template <int KT, int... J>
+__device__ __forceinline__ void pk10_loads(uint32_t tbase, int K, const uint32_t (&x)[11],
+                                           const CodeFix &f, float (&y)[32],
+                                           std::integer_sequence<int, J...>) {
+  if (KT > 0)   // table offsets as immediates
+    ((y[J] = lds_f32_imm<J * KT * 4>(tbase + 4u * fix_code<KT>(pk10_code<J>(x), f))), ...);
+  else
+    ((y[J] = lds_f32(tbase + (uint32_t)J * K * 4 + 4u * fix_code<KT>(pk10_code<J>(x), f))), ...);
+}
+
+// RQ_CODES_PACKED10, one token: the row's 32 codes of this chunk are bits
+// [10j, 10j + 10) of its 40-byte slice, which begins 8 bytes into the
+// 48-byte window w when `skip8`, else at its start.  All 32 table loads are
+// issued before any add; the sum is a tree.
+template <int KT>
+__device__ __forceinline__ float chunk32_packed_tb1(uint32_t tbase, int K, const uint4 (&w)[3],
+                                                    bool skip8, const CodeFix &f) {
+  const uint32_t a[12] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y,
+                          w[1].z, w[1].w, w[2].x, w[2].y, w[2].z, w[2].w};
+  uint32_t x[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) x[i] = skip8 ? a[i + 2] : a[i];
+  x[10] = 0u;
+  float y[32];
+  pk10_loads<KT>(tbase, K, x, f, y, std::make_integer_sequence<int, 32>{});
+#pragma unroll
+  for (int st = 1; st < 32; st <<= 1)
+#pragma unroll
+    for (int q = 0; q < 32; q += 2 * st) y[q] += y[q + st];
+  return y[0];
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -222,7 +273,9 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT>::THREADS, MINB)
     logits_chunk_u16_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
   constexpr bool SCHED = FMT == RQ_CODES_SCHED;
   constexpr bool U8 = FMT == RQ_CODES_U8;
+  constexpr bool PK10 = FMT == RQ_CODES_PACKED10;
   using S = ChunkShape<TB, FMT>;
+  static_assert(!PK10 || (TB == 1 && S::PPT == 32), "a thread owns a whole 10-bit slice");
   static_assert(!SCHED || (TB == 1 && S::PPT == 32), "a thread owns a whole scheduled slice");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment (TMA swizzle atoms) by pointer arithmetic, so the
@@ -264,8 +317,10 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT>::THREADS, MINB)
   const uint32_t stage0 = smem_addr(stages);
   // Box origin of this CTA's code slice: column c*PC of the [V][P] matrix,
   // or, for the chunk-major scheduled layout [P/32][V][32], rows c32*V + v
-  // at column (c % (32/PC)) * PC.
-  const int box_x = SCHED ? (c % (32 / S::PC)) * S::PC : c * S::PC;
+  // at column (c % (32/PC)) * PC, or, for 10-bit codes, byte 40c of the row
+  // rounded down to 16 bytes.
+  const int box_x = SCHED ? (c % (32 / S::PC)) * S::PC : PK10 ? (40 * c) & ~15 : c * S::PC;
+  const bool skip8 = PK10 && ((40 * c) & 15) != 0;
   const int64_t box_y0 = SCHED ? (int64_t)(c / (32 / S::PC)) * a.V : 0;
   auto issue = [&](int i, int s) {           // tile t0 + i into stage s
     const uint32_t bar = smem_addr(&full[s]);
@@ -322,14 +377,14 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT>::THREADS, MINB)
   const int hh = tid % S::TPR;               // which PPT pairs of the row
   const int box = r >> 8, rr = r & 255;
   const uint32_t tt = smem_addr(Ts) + (uint32_t)hh * S::PPT * KS * TB * 4;
-  constexpr int NQ = S::PPT / S::CPV;        // 16-byte code vectors per thread
+  constexpr int NQ = S::NQ;                  // 16-byte code vectors per thread
   uint32_t voff[NQ];                         // this thread's code vectors in a stage
 #pragma unroll
   for (int q = 0; q < NQ; ++q)
     voff[q] = (uint32_t)(box * S::BOX_BYTES + rr * S::ROWB) + 16 * swz<S::ROWB>(hh * NQ + q, rr);
   int nq = 0;                                // vectors holding real pairs
 #pragma unroll
-  for (int q = 0; q < NQ; ++q) nq += ((hh * NQ + q) * S::CPV < np) ? 1 : 0;
+  for (int q = 0; q < NQ; ++q) nq += (PK10 || (hh * NQ + q) * S::CPV < np) ? 1 : 0;
   float *out = a.partial + (size_t)c * a.B * a.V;
   int64_t v = t0 * S::R + r;
 
@@ -364,6 +419,8 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT>::THREADS, MINB)
     for (int b = 0; b < TB; ++b) acc[b] = 0.f;
     if constexpr (SCHED) {
       acc[0] = chunk32_sched_tb1<KSH>(tt, w);   // the row's whole 32-pair slice
+    } else if constexpr (PK10) {
+      acc[0] = chunk32_packed_tb1<KT>(tt, K, w, skip8, a.fix);
     } else if constexpr (U8) {
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
@@ -664,6 +721,9 @@ const Variant kVariants[] = {
     RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_U8, 0, 2),
     RQ_CHUNK_VARIANT(2, 0, 3, RQ_CODES_U8, 0, 1),
     RQ_CHUNK_VARIANT(4, 0, 3, RQ_CODES_U8, 0, 1),
+    // 10-bit codes, one token: 128 KB of tables (K = 1024), three 24 KB stages
+    RQ_CHUNK_VARIANT(1, 1024, 3, RQ_CODES_PACKED10, 0, 1),
+    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_PACKED10, 0, 1),
 };
 
 size_t variant_smem(const Variant &v, int K) {
@@ -677,9 +737,12 @@ size_t variant_smem(const Variant &v, int K) {
 ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di) {
   ChunkPlan cp{};
   cp.ok = false;
-  if ((fmt != RQ_CODES_U16 && fmt != RQ_CODES_SCHED && fmt != RQ_CODES_U8) || B < 1 || B > 4 ||
-      P % 8 != 0 || K > 1024)
+  if ((fmt != RQ_CODES_U16 && fmt != RQ_CODES_SCHED && fmt != RQ_CODES_U8 &&
+       fmt != RQ_CODES_PACKED10) ||
+      B < 1 || B > 4 || P % 8 != 0 || K > 1024)
     return cp;
+  // 10-bit codes: one token, whole 64-code groups (80-byte, 16-byte-aligned rows)
+  if (fmt == RQ_CODES_PACKED10 && (B != 1 || P % 64 != 0)) return cp;
   if (fmt == RQ_CODES_U8 && (K > 256 || P % 16 != 0)) return cp;   // 16-byte row pitch
   if (fmt == RQ_CODES_SCHED && P % 32 != 0) return cp;
   if (V > (int64_t)INT_MAX - 2048) return cp;
@@ -714,13 +777,17 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   const Variant &var = kVariants[cp.variant];
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
-  const int cb = fmt == RQ_CODES_U8 ? 1 : 2;   // bytes per code
-  const int rowb = cp.PC * cb;
-  // [V][P] for plain codes; the scheduled layout is chunk-major [P/32][V][32]
+  const bool pk = fmt == RQ_CODES_PACKED10;
+  const int cb = fmt == RQ_CODES_U8 || pk ? 1 : 2;   // bytes per element of the map
+  const int rowb = pk ? 48 : cp.PC * cb;
+  // [V][P] for plain codes; the scheduled layout is chunk-major [P/32][V][32];
+  // 10-bit codes are bytes [V][P/64*80], read in 48-byte windows
   const bool cm = fmt == RQ_CODES_SCHED;
-  const cuuint64_t gdim[2] = {(cuuint64_t)(cm ? 32 : P), (cuuint64_t)(cm ? (int64_t)V * (P / 32) : V)};
-  const cuuint64_t gstride[1] = {(cuuint64_t)(cm ? 64 : P * cb)};
-  const cuuint32_t box[2] = {(cuuint32_t)cp.PC, 256u};
+  const int64_t pk_row = (int64_t)P / 64 * 80;
+  const cuuint64_t gdim[2] = {(cuuint64_t)(cm ? 32 : pk ? pk_row : P),
+                              (cuuint64_t)(cm ? (int64_t)V * (P / 32) : V)};
+  const cuuint64_t gstride[1] = {(cuuint64_t)(cm ? 64 : pk ? pk_row : P * cb)};
+  const cuuint32_t box[2] = {(cuuint32_t)(pk ? 48 : cp.PC), 256u};
   const cuuint32_t estride[2] = {1u, 1u};
   const CUtensorMapSwizzle swz = rowb == 64   ? CU_TENSOR_MAP_SWIZZLE_64B
                                  : rowb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B

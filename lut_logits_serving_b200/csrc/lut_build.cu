@@ -92,9 +92,13 @@ __device__ __forceinline__ float4 ldg_v4_keep(const float *p, uint64_t pol) {
 __global__ void __launch_bounds__(256) lut_build_ds6_kernel(const float *__restrict__ h,
                                                            const float *__restrict__ C, int b0,
                                                            int nb, int D, int L, int K, int Bs,
-                                                           int quads, float *__restrict__ lut) {
-  // One wave: let the next kernel (the code pass) start its prologue now.
-  griddep_launch_dependents();
+                                                           int quads, int early,
+                                                           float *__restrict__ lut) {
+  // One wave.  `early`: let the next kernel start now; the shared-memory
+  // chunk pass loads its first codes before it waits on this one.  A pass
+  // that reads its tables through L2 is not started early: measured on a
+  // B200 at V = 256000, P = 768, K = 1024, one token, it then ran 3x longer.
+  if (early) griddep_launch_dependents();
   griddep_wait();                          // h and the table buffer: earlier kernels
   // P*K < 2^31 (checked by the launcher): 32-bit index math, no 64-bit divides
   const int g = blockIdx.x * blockDim.x + threadIdx.x;
@@ -175,7 +179,8 @@ __global__ void __launch_bounds__(256) lut_build_ds6_tok_kernel(
 }
 
 cudaError_t launch_lut_build(const float *h, const float *C, int B, int b0, int nb, int D,
-                             int M, int L, int K, int Bs, float *lut, cudaStream_t s) {
+                             int M, int L, int K, int Bs, float *lut, bool early_dependents,
+                             cudaStream_t s) {
   (void)B;
   const int ds = D / M;
   const int P = M * L;
@@ -193,7 +198,7 @@ cudaError_t launch_lut_build(const float *h, const float *C, int B, int b0, int 
     const int64_t blocks = (quads + 255) / 256;
     if (4 * quads < 0x7fffffffLL - 1024)
       return pdl_launch(lut_build_ds6_kernel, dim3((unsigned)blocks), dim3(256), 0, s, h, C, b0,
-                        nb, D, L, K, Bs, (int)quads, lut);
+                        nb, D, L, K, Bs, (int)quads, early_dependents ? 1 : 0, lut);
   }
   const int64_t rows = (int64_t)P * K;
   if (Bs <= 2 && rows < 0x7fffffffLL - 256) {

@@ -74,8 +74,12 @@ cudaError_t ensure_smem_limit(const void *fn, int device, size_t smem);
 // smem) under a lock.
 int occupancy_cached(const void *fn, int device, int threads, size_t smem);
 
+// early_dependents: the kernel launched next on `s` (with the programmatic
+// dependency attribute) may start while the build runs; pass true only when
+// that kernel is the shared-memory chunk pass.
 cudaError_t launch_lut_build(const float *h, const float *C, int B, int b0, int nb, int D,
-                             int M, int L, int K, int Bs, float *lut, cudaStream_t s);
+                             int M, int L, int K, int Bs, float *lut, bool early_dependents,
+                             cudaStream_t s);
 
 cudaError_t launch_decode_rows(const int32_t *ids, int64_t N, const void *codes, int fmt,
                                const float *C, int64_t V, int D, int M, int L, int K,

@@ -262,7 +262,7 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
   unsigned char *rest = static_cast<unsigned char *>(ws) + lut_bytes;
   if (w.chunk) {
     // B <= 4: one table for all tokens, then the vocabulary-tiled pass
-    cudaError_t e = launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut, s);
+    cudaError_t e = launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut, true, s);
     if (e != cudaSuccess) return status_of(e);
     return run_logits(codes, fmt, d, lut, B, Bs, softcap, logits, argmax, rest, w, di, s, true,
                       rows_spec, rows);
@@ -315,7 +315,7 @@ int run_fused(const float *h, const float *C, const void *codes, int fmt, const 
       continue;
     }
     const int nb = rem < G ? rem : G;
-    e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, s);
+    e = launch_lut_build(h, C, B, b0, nb, d.D, d.M, d.L, d.K, Bs, lut, false, s);
     if (e == cudaSuccess && !marked) e = prof_mark(t_prof_start, s);
     marked = true;
     if (e == cudaSuccess)
@@ -391,7 +391,7 @@ int rq_lut_build(const float *h, const float *C, rq_dims d, int B, float *lut, v
   if (!aligned(h, 4) || !aligned(C, 4) || !aligned(lut, 16)) return RQ_ERR_MISALIGNED;
   const int Bs = rq_lut_token_stride(B);
   if ((size_t)Bs * (d.D / d.M) * 4 > 48 * 1024) return RQ_ERR_UNSUPPORTED;
-  return status_of(launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut,
+  return status_of(launch_lut_build(h, C, B, 0, B, d.D, d.M, d.L, d.K, Bs, lut, false,
                                     static_cast<cudaStream_t>(stream)));
 }
 

@@ -55,6 +55,11 @@ WORKLOADS = {
     "g2_b1": Workload("g2_b1", V=256000, D=2304, M=384, L=2, K=1024, B=1,
                       sigmas=(0.02, 0.005), hidden_scale=40.0 / math.sqrt(2304.0),
                       argmax=True, n_ids=1, decode_scale=math.sqrt(2304.0)),
+    # batch 1 on the 10-bit packed artifact (960 bytes per row)
+    "g2_b1_packed10": Workload("g2_b1_packed10", V=256000, D=2304, M=384, L=2, K=1024, B=1,
+                               sigmas=(0.02, 0.005), hidden_scale=40.0 / math.sqrt(2304.0),
+                               packed10=True, argmax=True, n_ids=1,
+                               decode_scale=math.sqrt(2304.0)),
     # a batch in the range the L2-served tables take (5 to 16 tokens)
     "g2_b16": Workload("g2_b16", V=256000, D=2304, M=384, L=2, K=1024, B=16,
                        sigmas=(0.02, 0.005), hidden_scale=0.83,

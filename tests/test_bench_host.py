@@ -112,7 +112,8 @@ def parse_argv(argv):
 
 
 def test_workload_choices_cover_the_workloads():
-    for name in ("g2_b1", "g2_b32", "packed_b64", "decode512", "encode_g2", "g2_b1_topk50",
+    for name in ("g2_b1", "g2_b1_packed10", "g2_b32", "packed_b64", "decode512", "encode_g2",
+                 "g2_b1_topk50",
                  "mlp_gate_b1", "mlp_down_b1"):
         assert name in synth.WORKLOADS
         assert parse_argv(["--workload", name]).workload == name

@@ -1,8 +1,9 @@
 """GPU parity at the full Gemma-2 shapes (V=256000, D=2304, M=384, L=2,
 K=1024), in the launch configuration the benchmark times.
 
-* decode batch 1, uint16 codes: all 256000 logits and the argmax against
-  the oracle (the oracle does the full row sweep in about a second);
+* decode batch 1, uint16, bank-scheduled and 10-bit packed codes: all
+  256000 logits and the argmax against the oracle (the oracle does the full
+  row sweep in about a second);
 * batch 32, uint16 codes, one code pass for all tokens: all 32 x 256000
   logits and every token's argmax, on every kernel choice;
 * batch 64, 10-bit packed codes, fused build + unpack + sum + softcap +
@@ -73,6 +74,16 @@ def test_g2_batch1_full_sweep(g2):
     want = oracle.decode_rows_bf16(am4.cpu().numpy().astype(np.int32), g2["codes"], g2["C"],
                                    w.decode_scale)
     assert np.array_equal(rows4.view(torch.int16).cpu().numpy().view(np.uint16), want)
+    # 10-bit packed codes: the same pass over 48-byte windows of the packed rows
+    packed = rq.rq_pack10(g2["dc"], d)
+    out5 = torch.full((1, w.V), float("nan"), device="cuda")
+    logits5, am5, rows5, _ = rq.rq_greedy_step(dev(h), g2["dC"], packed, rq.PACKED10, d,
+                                               w.softcap, scale=w.decode_scale, logits=out5)
+    err5 = assert_logits_close(logits5.cpu().numpy(), ref)
+    print(f"g2_b1 packed10 normwise error {err5:.3g}")
+    assert check_argmax(am5.cpu().numpy(), ref) == 0
+    assert torch.equal(am5, am3)
+    assert torch.equal(rows5, rows4)
     assert rq.rq_device_error() == 0
 
 

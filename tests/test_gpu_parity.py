@@ -86,6 +86,7 @@ CASES = [
     (1200, 128, 64, 1, 100),   # scheduled table stride 128 (two CTAs per SM)
     (900, 96, 16, 2, 300),     # scheduled table stride 512
     (600, 64, 32, 2, 37),      # scheduled table stride 64
+    (2600, 384, 64, 2, 1024),  # K = 1024, P = 128: 10-bit slices at both window offsets
 ]
 
 
