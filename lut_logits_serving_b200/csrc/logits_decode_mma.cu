@@ -27,7 +27,7 @@
 //
 // Design for sm_100a (ds = 6, L = 2, K <= 1024); DmShape gives the instances.
 // One CTA per SM walks an even share of the vocabulary in passes of up to
-// TILES x 128 rows (1024 for 32-token groups of uint16 codes), running every
+// TILES x 128 rows (1024 for 32-token groups), running every
 // subspace once per pass, so a subspace's codebook pair (48 KB at K = 1024)
 // is copied into shared memory once per pass.  Warp-specialised and
 // mbarrier-driven; no CTA barrier inside the loop:
@@ -37,7 +37,10 @@
 //     sums into fp16 hi and lo and stores each row's A operand (8 TMEM
 //     columns) into its TMEM lane of a double-buffered A slot;
 //   * one copy warp: TMA code tiles (uint16: {8 codes, 128 rows} boxes, stages
-//     of 4 subspaces; 10-bit packed rows: {80 bytes, 128 rows}, stages of 32),
+//     of 4 subspaces; 10-bit packed rows: stages of 16 subspaces, whose 40
+//     bytes start at byte 40j of the row -- 8 bytes off a 16-byte boundary for
+//     odd j -- so each box is the 48-byte, 16-byte-aligned window around them,
+//     {48 bytes, 128 rows}),
 //     and per subspace one bulk copy of the codebook pair into a ring of
 //     NBOOK buffers plus the pre-split hidden operand (B1, B2) into a ring of
 //     6 slots, on one transaction barrier;
@@ -65,16 +68,16 @@ namespace {
 template <int NT, int FMT>
 struct DmShape {
   static constexpr bool PACKED = FMT == RQ_CODES_PACKED10;
-  static constexpr int TILES = (NT == 32 && !PACKED) ? 8 : 4;   // M = 128 tiles per pass
+  static constexpr int TILES = NT == 32 ? 8 : 4;                // M = 128 tiles per pass
   static constexpr int RPT = TILES / 4;                         // rows per decoder thread
   static constexpr int DEC_WARPS = 16;                          // 4 lane quarters x 4
   static constexpr int THREADS = (DEC_WARPS + 2) * 32;          // + copy warp + MMA warp
   static constexpr int ROWS = TILES * 128;                      // rows per pass
-  static constexpr int GROUP = PACKED ? 32 : 4;                 // subspaces per code stage
-  static constexpr int ROW_BYTES = PACKED ? 80 : 16;            // code bytes per row and stage
+  static constexpr int GROUP = PACKED ? 16 : 4;                 // subspaces per code stage
+  static constexpr int ROW_BYTES = PACKED ? 48 : 16;            // code bytes per row and stage
   static constexpr int STAGE_BYTES = ROWS * ROW_BYTES;
   static constexpr int STAGES = 2;
-  static constexpr int NBOOK = PACKED ? 2 : 3;                  // codebook buffers
+  static constexpr int NBOOK = (PACKED && NT == 32) ? 2 : 3;    // codebook buffers (shared memory)
   static constexpr int BOX_INNER = ROW_BYTES / 2;               // TMA box inner extent (16-bit units)
   static constexpr int HBYTES = 2 * NT * 32;                    // B1 and B2: NT rows x 16 fp16 each
   static constexpr uint32_t ACOL = TILES * NT;                  // first A-slot column
@@ -420,7 +423,8 @@ __global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
         const uint32_t dst = smem_addr(st + sidx * S_::STAGE_BYTES);
 #pragma unroll
         for (int q = 0; q < S_::TILES; ++q)
-          tma_load_2d(dst + q * (128 * S_::ROW_BYTES), &tmap, gi * S_::BOX_INNER,
+          tma_load_2d(dst + q * (128 * S_::ROW_BYTES), &tmap,
+                      S_::PACKED ? ((40 * gi) & ~15) / 2 : gi * S_::BOX_INNER,
                       (int)(r0 + (int64_t)p * S_::ROWS + q * 128), b, pol_codes);
         last_codes[sidx] = g;
       };
@@ -630,11 +634,14 @@ __global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
             uint32_t c0, c1;
             if (S_::PACKED) {
               // codes 2m and 2m + 1 of the row: bits [20 ig, 20 ig + 20) of its
-              // 80-byte slice, LSB first (a field spans at most two words)
+              // group's 40 bytes, which start 8 bytes into the 48-byte window
+              // for odd groups; LSB first (a field spans at most two words)
               const uint32_t rowa = stage + (uint32_t)r * S_::ROW_BYTES;
-              const int bit = 20 * ig, wi = bit >> 5, sh = bit & 31;
+              const int bit = 20 * ig + (((40 * (m / S_::GROUP)) & 8) << 3);
+              const int wi = bit >> 5, sh = bit & 31;
               const uint32_t w0 = lds_u32(rowa + 4u * wi);
-              const uint32_t w1 = lds_u32(rowa + 4u * (wi + 1 < 20 ? wi + 1 : wi));
+              const uint32_t w1 =
+                  lds_u32(rowa + 4u * (wi + 1 < S_::ROW_BYTES / 4 ? wi + 1 : wi));
               const uint32_t v = sh == 0 ? w0 : __funnelshift_r(w0, w1, sh);
               c0 = a.fix(v & 1023u);
               c1 = a.fix((v >> 10) & 1023u);
@@ -756,7 +763,9 @@ cudaError_t launch_dm(const float *h, const float *C, const void *codes, int64_t
   CUtensorMap tmap;
   const int P = 2 * M;
   // packed rows (P * 10 / 8 bytes, a multiple of 16 as M % 32 == 0) are
-  // copied as 16-bit units: the copy moves bytes whatever the element type
+  // copied as 16-bit units: the copy moves bytes whatever the element type;
+  // the last window of a row ends at the row's end (its group starts 8 bytes
+  // past a 16-byte boundary)
   const uint64_t row_bytes = S_::PACKED ? (uint64_t)P * 10 / 8 : (uint64_t)P * 2;
   if (!encode_tmap_2d_u16(&tmap, codes, row_bytes / 2, (uint64_t)V, row_bytes, S_::BOX_INNER, 128,
                           CU_TENSOR_MAP_SWIZZLE_NONE))
