@@ -20,6 +20,15 @@
  *     caller owns every buffer.  The library never allocates device memory.
  *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *     stream.  Every call only enqueues work and never synchronizes.
+ *   - Kernels are launched with programmatic dependent launch: each waits
+ *     for the kernels before it in the stream before it reads their outputs
+ *     (h, tables, partial sums).  The code matrix and the codebooks are
+ *     treated as a resident artifact: a code pass may start fetching code
+ *     tiles as soon as the kernel ahead of it in the stream has signalled
+ *     that its dependents may launch, so codes must not be written by a
+ *     kernel that lets its dependents start early.  The library's own layout
+ *     calls (rq_pack10, rq_pack8, rq_prepare_sched) launch without that
+ *     signal: what follows them starts after they end.
  *   - Return value: rq_status (0 = RQ_OK).  Argument errors are detected on
  *     the host before anything is launched.  RQ_ERR_CUDA reports a launch
  *     error (cudaGetLastError); kernel faults surface at the caller's next

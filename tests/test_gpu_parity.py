@@ -423,6 +423,7 @@ def test_fused_decode_paths(V, M, K, B, path):
     (4096, 32, 256, 32),      # the tiny workload's shape, one 32-token group
     (5003, 32, 1024, 64),     # one 64-token group, ragged rows
     (2222, 64, 100, 70),      # groups of 64 + a 6-token rest (tables), K not a power of two
+    (160000, 32, 256, 40),    # full 1024-row passes of a 32-token group, then an 8-token group
 ])
 def test_packed_codes_on_the_tensor_cores(V, M, K, B):
     """10-bit packed codes (M % 32 == 0) are unpacked by the tensor-core kernel's
