@@ -490,8 +490,8 @@ def topk_launches(V, k):
 
 
 def decodable(w):
-    """Full token groups (64, then 32) of uint16 or 10-bit packed codes at
-    ds = 6, L = 2 decode their rows on the tensor cores."""
+    """Full token groups (64, then 32) of uint16, bank-scheduled or 10-bit
+    packed codes at ds = 6, L = 2 decode their rows on the tensor cores."""
     return (w.ds == 6 and w.L == 2 and 16 <= w.K <= 1024 and w.B >= 32 and
             w.M % (32 if w.packed10 else 8) == 0)
 
@@ -653,7 +653,7 @@ class Artifact:
 
 
 def kernel_of(w, layout):
-    decoded = layout in ("u16", "packed10") and decodable(w)
+    decoded = layout in ("u16", "packed10", "sched") and decodable(w)
     packed = w.packed10 or layout == "packed10"
     if w.B <= 4 and (not packed or w.B == 1):
         return "logits_chunk_u16_kernel", decoded

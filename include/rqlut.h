@@ -63,9 +63,12 @@
  *                               >= K, at least 32 (s = 10 at K = 1024).  The order only changes the
  *                               summation order; entries with c >= K add 0
  *                               to the logits (rq_decode_rows clamps them to
- *                               K-1).  Batch 1 streams it fastest; larger
- *                               batches run it through the slower generic
- *                               lookup order (use RQ_CODES_U16 there).
+ *                               K-1).  Batch 1 streams it fastest; full
+ *                               token groups of larger batches decode it on
+ *                               the tensor cores (M % 16 == 0; 1.15-1.3x the
+ *                               time of RQ_CODES_U16 there, one stage of
+ *                               codes in flight instead of two), other groups
+ *                               read it in the generic lookup order.
  *   lut      float [M*L][K][Bs], Bs = rq_lut_token_stride(B): token b of
  *            table (p, k) at lut[(p*K + k)*Bs + b]
  *   logits   float [B][V]
@@ -210,7 +213,9 @@ RQ_API int rq_logits_from_hidden(const float *h, const float *C, const void *cod
  *                          decoded into tensor memory, tcgen05 fp16 MMAs on
  *                          hi/lo splits of the rows and hidden states (with
  *                          power-of-two scales), fp32 sums of short MMA
- *                          chains; RQ_CODES_U16 with M % 8 == 0 or
+ *                          chains; RQ_CODES_U16 with M % 8 == 0,
+ *                          RQ_CODES_SCHED with M % 16 == 0 (codes >= K
+ *                          clamped to K-1, as rq_decode_rows does) or
  *                          RQ_CODES_PACKED10 with M % 32 == 0 (its scratch
  *                          lives in the workspace's table region)
  */

@@ -40,7 +40,9 @@
 //     of 4 subspaces; 10-bit packed rows: stages of 16 subspaces, whose 40
 //     bytes start at byte 40j of the row -- 8 bytes off a 16-byte boundary for
 //     odd j -- so each box is the 48-byte, 16-byte-aligned window around them,
-//     {48 bytes, 128 rows}),
+//     {48 bytes, 128 rows}; bank-scheduled codes: one stage of 16 subspaces,
+//     the rows' whole 64-byte slices {32 entries, 128 rows}, which the decoders
+//     put back in pair order in place when the stage lands),
 //     and per subspace one bulk copy of the codebook pair into a ring of
 //     NBOOK buffers plus the pre-split hidden operand (B1, B2) into a ring of
 //     6 slots, on one transaction barrier;
@@ -68,15 +70,17 @@ namespace {
 template <int NT, int FMT>
 struct DmShape {
   static constexpr bool PACKED = FMT == RQ_CODES_PACKED10;
+  static constexpr bool SCHED = FMT == RQ_CODES_SCHED;
   static constexpr int TILES = NT == 32 ? 8 : 4;                // M = 128 tiles per pass
   static constexpr int RPT = TILES / 4;                         // rows per decoder thread
   static constexpr int DEC_WARPS = 16;                          // 4 lane quarters x 4
   static constexpr int THREADS = (DEC_WARPS + 2) * 32;          // + copy warp + MMA warp
   static constexpr int ROWS = TILES * 128;                      // rows per pass
-  static constexpr int GROUP = PACKED ? 16 : 4;                 // subspaces per code stage
-  static constexpr int ROW_BYTES = PACKED ? 48 : 16;            // code bytes per row and stage
+  static constexpr int GROUP = PACKED || SCHED ? 16 : 4;        // subspaces per code stage
+  static constexpr int ROW_BYTES = PACKED ? 48 : SCHED ? 64 : 16;   // code bytes per row and stage
   static constexpr int STAGE_BYTES = ROWS * ROW_BYTES;
-  static constexpr int STAGES = 2;
+  // a scheduled stage (64 KB at 1024 rows) leaves room for one only
+  static constexpr int STAGES = SCHED ? 1 : 2;
   static constexpr int NBOOK = (PACKED && NT == 32) ? 2 : 3;    // codebook buffers (shared memory)
   static constexpr int BOX_INNER = ROW_BYTES / 2;               // TMA box inner extent (16-bit units)
   static constexpr int HBYTES = 2 * NT * 32;                    // B1 and B2: NT rows x 16 fp16 each
@@ -219,6 +223,19 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
+}
+
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void sts_u16(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"((unsigned short)v) : "memory");
 }
 
 __device__ __forceinline__ float2 lds_f2(uint32_t addr) {
@@ -396,6 +413,7 @@ __global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
   const float sE = *esc;
 
   const int M = a.M, G = a.M / S_::GROUP, NC = (a.M + kDmChain - 1) / kDmChain;
+  const int ssh = sched_shift(a.K);          // bank-scheduled entries: (i << ssh) | c
   const int64_t r0 = a.V * blockIdx.x / gridDim.x, r1 = a.V * (blockIdx.x + 1) / gridDim.x;
   const int npass = (int)((r1 - r0 + S_::ROWS - 1) / S_::ROWS);
   const int S = npass * M;                   // steps: (pass, subspace)
@@ -424,8 +442,12 @@ __global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
 #pragma unroll
         for (int q = 0; q < S_::TILES; ++q)
           tma_load_2d(dst + q * (128 * S_::ROW_BYTES), &tmap,
-                      S_::PACKED ? ((40 * gi) & ~15) / 2 : gi * S_::BOX_INNER,
-                      (int)(r0 + (int64_t)p * S_::ROWS + q * 128), b, pol_codes);
+                      S_::PACKED  ? ((40 * gi) & ~15) / 2
+                      : S_::SCHED ? 0
+                                  : gi * S_::BOX_INNER,
+                      (int)((S_::SCHED ? (int64_t)gi * a.V : 0) + r0 + (int64_t)p * S_::ROWS +
+                            q * 128),
+                      b, pol_codes);
         last_codes[sidx] = g;
       };
       auto issue_book = [&](int s) {
@@ -612,6 +634,32 @@ __global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
           wait(kBarCodes + gcode % ST, (uint32_t)(gcode / ST) & 1u);
           if (to) break;
           stage = smem_addr(st + (gcode % ST) * S_::STAGE_BYTES);
+          if (S_::SCHED) {
+            // each entry (i << ssh) | c of a row's slice back to position i:
+            // the row's 32 codes in pair order, in place (a thread's own rows)
+            const uint32_t cmask = (1u << ssh) - 1u;
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+              const int ti = g * RPT + i;
+              if (ti < nt) {
+                const uint32_t rowa = stage + (uint32_t)(ti * 128 + q * 32 + lane) * 64u;
+                uint32_t e[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const uint4 v = lds_u4(rowa + 16u * k);
+                  e[4 * k] = v.x;
+                  e[4 * k + 1] = v.y;
+                  e[4 * k + 2] = v.z;
+                  e[4 * k + 3] = v.w;
+                }
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                  const uint32_t en = (k & 1) ? e[k >> 1] >> 16 : e[k >> 1] & 0xFFFFu;
+                  sts_u16(rowa + 2u * ((en >> ssh) & 31u), en & cmask);
+                }
+              }
+            }
+          }
         }
         wait(kBarBook + s % NB, (uint32_t)(s / NB) & 1u);
         if (s >= kDmASlots)                                     // A slot free
@@ -645,6 +693,10 @@ __global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
               const uint32_t v = sh == 0 ? w0 : __funnelshift_r(w0, w1, sh);
               c0 = a.fix(v & 1023u);
               c1 = a.fix((v >> 10) & 1023u);
+            } else if (S_::SCHED) {
+              const uint32_t w = lds_u32(stage + (uint32_t)r * 64u + 4u * ig);
+              c0 = a.fix(w & 0xFFFFu);
+              c1 = a.fix(w >> 16);
             } else {
               const uint32_t w = lds_u32(stage + (uint32_t)r * S_::ROW_BYTES + 4u * ig);
               c0 = a.fix(w & 0xFFFFu);
@@ -767,9 +819,13 @@ cudaError_t launch_dm(const float *h, const float *C, const void *codes, int64_t
   // the last window of a row ends at the row's end (its group starts 8 bytes
   // past a 16-byte boundary)
   const uint64_t row_bytes = S_::PACKED ? (uint64_t)P * 10 / 8 : (uint64_t)P * 2;
-  if (!encode_tmap_2d_u16(&tmap, codes, row_bytes / 2, (uint64_t)V, row_bytes, S_::BOX_INNER, 128,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
+  // the bank-scheduled layout is chunk-major [P/32][V][32]: rows of 64 bytes
+  const bool ok_map =
+      S_::SCHED ? encode_tmap_2d_u16(&tmap, codes, 32, (uint64_t)V * (P / 32), 64, 32, 128,
+                                     CU_TENSOR_MAP_SWIZZLE_NONE)
+                : encode_tmap_2d_u16(&tmap, codes, row_bytes / 2, (uint64_t)V, row_bytes,
+                                     S_::BOX_INNER, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok_map) return cudaErrorInvalidValue;
   {
     void *args[] = {&h, &D, &t0, &nb, &C, &M, &K, &hop};
     cudaError_t e = launch_maybe_pdl(reinterpret_cast<const void *>(&dm_scale_kernel<NT>),
@@ -812,9 +868,11 @@ cudaError_t launch_dm(const float *h, const float *C, const void *codes, int64_t
 }  // namespace
 
 size_t decode_mma_smem(int K, int N, int fmt) {
-  const bool packed = fmt == RQ_CODES_PACKED10;
-  if (N == 32) return packed ? dm_smem<32, RQ_CODES_PACKED10>(K) : dm_smem<32, RQ_CODES_U16>(K);
-  return packed ? dm_smem<64, RQ_CODES_PACKED10>(K) : dm_smem<64, RQ_CODES_U16>(K);
+  if (fmt == RQ_CODES_PACKED10)
+    return N == 32 ? dm_smem<32, RQ_CODES_PACKED10>(K) : dm_smem<64, RQ_CODES_PACKED10>(K);
+  if (fmt == RQ_CODES_SCHED)
+    return N == 32 ? dm_smem<32, RQ_CODES_SCHED>(K) : dm_smem<64, RQ_CODES_SCHED>(K);
+  return N == 32 ? dm_smem<32, RQ_CODES_U16>(K) : dm_smem<64, RQ_CODES_U16>(K);
 }
 
 size_t decode_mma_hop_bytes(int M, int N, int K) {
@@ -823,9 +881,10 @@ size_t decode_mma_hop_bytes(int M, int N, int K) {
 }
 
 bool decode_mma_shape_ok(int fmt, int64_t V, int D, int M, int L, int K) {
-  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10) return false;
+  if (fmt != RQ_CODES_U16 && fmt != RQ_CODES_PACKED10 && fmt != RQ_CODES_SCHED) return false;
   if (L != 2 || D != 6 * M || K > 1024 || K < 1) return false;
-  if (M % (fmt == RQ_CODES_PACKED10 ? 32 : 8) != 0) return false;
+  if (M % (fmt == RQ_CODES_PACKED10 ? 32 : fmt == RQ_CODES_SCHED ? 16 : 8) != 0) return false;
+  if (fmt == RQ_CODES_SCHED && V * (M / 16) > (int64_t)INT_MAX - 2048) return false;
   return V >= 1 && V <= (int64_t)INT_MAX - 2048;
 }
 
@@ -839,18 +898,16 @@ cudaError_t launch_logits_decode_mma(const float *h, const float *C, const void 
                                      int64_t V, int D, int M, int K, int t0, int nb, int N,
                                      float cap, float *hop, float *logits, float *am_val,
                                      int *am_idx, int nblk, const DevInfo &di, cudaStream_t s) {
-  const bool packed = fmt == RQ_CODES_PACKED10;
-  if (N == 32)
-    return packed ? launch_dm<32, RQ_CODES_PACKED10>(h, C, codes, V, D, M, K, t0, nb, cap, hop,
-                                                      logits, am_val, am_idx, nblk, di, s)
-                  : launch_dm<32, RQ_CODES_U16>(h, C, codes, V, D, M, K, t0, nb, cap, hop, logits,
-                                                am_val, am_idx, nblk, di, s);
-  if (N == 64)
-    return packed ? launch_dm<64, RQ_CODES_PACKED10>(h, C, codes, V, D, M, K, t0, nb, cap, hop,
-                                                      logits, am_val, am_idx, nblk, di, s)
-                  : launch_dm<64, RQ_CODES_U16>(h, C, codes, V, D, M, K, t0, nb, cap, hop, logits,
-                                                am_val, am_idx, nblk, di, s);
-  return cudaErrorInvalidValue;
+#define RQ_DM_LAUNCH(NT_, FMT_)                                                                  \
+  launch_dm<NT_, FMT_>(h, C, codes, V, D, M, K, t0, nb, cap, hop, logits, am_val, am_idx, nblk,  \
+                       di, s)
+  if (N != 32 && N != 64) return cudaErrorInvalidValue;
+  if (fmt == RQ_CODES_PACKED10)
+    return N == 32 ? RQ_DM_LAUNCH(32, RQ_CODES_PACKED10) : RQ_DM_LAUNCH(64, RQ_CODES_PACKED10);
+  if (fmt == RQ_CODES_SCHED)
+    return N == 32 ? RQ_DM_LAUNCH(32, RQ_CODES_SCHED) : RQ_DM_LAUNCH(64, RQ_CODES_SCHED);
+  return N == 32 ? RQ_DM_LAUNCH(32, RQ_CODES_U16) : RQ_DM_LAUNCH(64, RQ_CODES_U16);
+#undef RQ_DM_LAUNCH
 }
 
 }  // namespace rq

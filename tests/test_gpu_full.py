@@ -5,7 +5,8 @@ K=1024), in the launch configuration the benchmark times.
   256000 logits and the argmax against the oracle (the oracle does the full
   row sweep in about a second);
 * batch 32, uint16 codes, one code pass for all tokens: all 32 x 256000
-  logits and every token's argmax, on every kernel choice;
+  logits and every token's argmax, on every kernel choice, and on the
+  bank-scheduled layout;
 * batch 64, 10-bit packed codes, fused build + unpack + sum + softcap +
   argmax: all 64 x 256000 logits and every token's argmax;
 * 512 Zipf-drawn input rows rebuilt in bf16: all of them, bit for bit.
@@ -112,7 +113,9 @@ def elementwise_rel(got, ref, floor=1e-2):
 def _batched(g2, w, fmt, path=None):
     d = g2["d"]
     h, ref = _full_ref(g2, w)
-    codes_dev = g2["dc"] if fmt == rq.U16 else rq.rq_pack10(g2["dc"], d)
+    codes_dev = (g2["dc"] if fmt == rq.U16 else
+                 rq.rq_prepare_sched(g2["dc"], d) if fmt == rq.SCHED else
+                 rq.rq_pack10(g2["dc"], d))
     # NaN-filled output: a kernel that writes nothing cannot pass on stale memory
     out = torch.full((w.B, w.V), float("nan"), device="cuda")
     logits, am, _ = rq.rq_logits_from_hidden(dev(h), g2["dC"], codes_dev, fmt, d, w.softcap,
@@ -132,6 +135,17 @@ def test_g2_batch32_one_code_pass(g2, path):
     w = synth.WORKLOADS["g2_b32"]
     err, rel, ties = _batched(g2, w, rq.U16, path)
     print(f"g2_b32 path {path} normwise error {err:.3g}, elementwise relative error "
+          f"(|ref| >= 1e-2 max) {rel:.3g}, ties {ties}")
+    assert ties == 0
+    assert rq.rq_device_error() == 0
+
+
+def test_g2_batch32_scheduled_codes(g2):
+    """The batch-1 layout also serves a 32-token group: the tensor-core decode
+    puts its slices back in pair order."""
+    w = synth.WORKLOADS["g2_b32"]
+    err, rel, ties = _batched(g2, w, rq.SCHED)
+    print(f"g2_b32 scheduled codes normwise error {err:.3g}, elementwise relative error "
           f"(|ref| >= 1e-2 max) {rel:.3g}, ties {ties}")
     assert ties == 0
     assert rq.rq_device_error() == 0

@@ -448,6 +448,39 @@ def test_packed_codes_on_the_tensor_cores(V, M, K, B):
     assert_logits_close(logits2.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("V,M,K,B", [
+    (4096, 32, 256, 32),      # two 16-subspace slices, one 32-token group
+    (5003, 16, 1024, 64),     # one slice, one 64-token group, ragged rows
+    (2222, 48, 100, 70),      # three slices, K not a power of two (7-bit table stride)
+    (160000, 32, 256, 40),    # full 1024-row passes of a 32-token group, then 8 tokens
+])
+def test_scheduled_codes_on_the_tensor_cores(V, M, K, B):
+    """Bank-scheduled codes (M % 16 == 0) are put back in pair order by the
+    tensor-core kernel's decoders as each stage lands: the logits are those of
+    the same codes as drawn, bit for bit, and match the oracle."""
+    D = 6 * M
+    C, codes, h = make_case(V, D, M, 2, K, B, seed=V + 11)
+    d = rq.dims(V, D, M, 2, K)
+    ref = oracle_logits(C, codes, h, 30.0)
+    c16 = dev(codes.reshape(V, -1))
+    sched = rq.rq_prepare_sched(c16, d)
+    out = torch.full((B, V), float("nan"), device="cuda")
+    logits, am, _ = rq.rq_logits_from_hidden(dev(h), dev(C), sched, rq.SCHED, d, 30.0,
+                                             want_argmax=True, logits=out,
+                                             path=rq.PATH_DECODE_TC)
+    assert rq.rq_device_error() == 0
+    assert_logits_close(logits.cpu().numpy(), ref)
+    check_argmax(am.cpu().numpy(), ref)
+    plain, am_u, _ = rq.rq_logits_from_hidden(dev(h), dev(C), c16, rq.U16, d, 30.0,
+                                              want_argmax=True, path=rq.PATH_DECODE_TC)
+    assert torch.equal(logits, plain)
+    assert torch.equal(am, am_u)
+    # the default takes the tensor cores for the full groups of this layout too
+    logits2, _, _ = rq.rq_logits_from_hidden(dev(h), dev(C), sched, rq.SCHED, d, 30.0)
+    full = B - B % 32 if B % 32 < 17 else B
+    assert torch.equal(logits2[:full], logits[:full])
+
+
 @pytest.mark.parametrize("B", [32, 64])
 def test_tensor_core_decode_argmax_only_and_softcap_off(B):
     """Without a logits buffer the tensor-core kernel still leaves the argmax
