@@ -1079,7 +1079,9 @@ def run_ours(args, w):
                 else:
                     h2 = synth.hidden(w2.B, w2.D, w2.hidden_scale, seed + 2)
                     lay = headline_layout(w2, None, tuple(art.layouts))
-                    r2 = measure_logits(rig, w2, art, lay, h2)
+                    # the 32-token batch also on the other layouts (the batch-1
+                    # layout through the tensor cores) and every group kernel
+                    r2 = measure_logits(rig, w2, art, lay, h2, full=name == "g2_b32")
                     r2["config"] = workload_config(w2, lay)
                     r2.pop("t_ms", None)
             r2["clocks"] = c2.summary()
