@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--workload", default="g2_b1",
                     choices=["g2_b1", "g2_b1_packed10", "g2_b16", "g2_b32", "packed_b64", "mlp_gate_b1",
                              "mlp_down_b1", "encode_g2", "g2_b1_topk50", "decode512"])
-    ap.add_argument("--codes", default=None, choices=["u16", "sched", "u8"],
+    ap.add_argument("--codes", default=None, choices=["u16", "sched", "u8", "rot10"],
                     help="code layout of the unpacked workloads timed for `value`: "
                          "bank-scheduled once by rq_prepare_sched (the default at B <= 4), as "
                          "drawn (the default for batches, whose full token groups decode rows "
@@ -72,10 +72,11 @@ def parse():
 
 def workload_config(w, codes="u16"):
     rb = code_bytes(w, codes) // w.V
-    fmt = f"packed10 ({rb} B/row)" if w.packed10 else (
-        f"uint16 ({rb} B/row)" if codes == "u16" else
-        f"uint8 ({rb} B/row, K <= 256)" if codes == "u8" else
-        f"uint16 ({rb} B/row) in the bank-scheduled order of rq_prepare_sched")
+    fmt = (f"packed10 ({rb} B/row)" if w.packed10 or codes == "packed10" else
+           f"10-bit ({rb} B/row) in the rotated slices of rq_prepare_rot10" if codes == "rot10" else
+           f"uint16 ({rb} B/row)" if codes == "u16" else
+           f"uint8 ({rb} B/row, K <= 256)" if codes == "u8" else
+           f"uint16 ({rb} B/row) in the bank-scheduled order of rq_prepare_sched")
     if w.argmax:
         what = (f"softcap {w.softcap:g}, logits + argmax, then the {w.B} picked tokens' input "
                 f"rows rebuilt (bf16)")
@@ -90,7 +91,7 @@ def workload_config(w, codes="u16"):
         "V": w.V, "D": w.D, "M": w.M, "L": w.L, "K": w.K, "B": w.B,
         "codes": "packed10" if w.packed10 else codes,
         "l2": ("inputs larger than L2: the code matrix is streamed from HBM every step"
-               if (w.V * (w.P * 10 // 8 if w.packed10 else w.P * 2)) > 2 * 126 * 2**20 else
+               if code_bytes(w, codes) > 2 * 126 * 2**20 else
                "inputs smaller than L2: a 256 MB buffer is written between timed steps"),
     }
 
@@ -110,6 +111,8 @@ def headline_layout(w, codes=None, available=("sched", "u16", "u8")):
 def code_bytes(w, codes="u16"):
     if w.packed10 or codes == "packed10":
         return w.V * (w.P * 10 // 8)
+    if codes == "rot10":                      # packed rows + one rotation byte per slice
+        return w.V * (w.P * 10 // 8 + w.P // 32)
     return w.V * w.P * (1 if codes == "u8" else 2)
 
 
@@ -628,7 +631,7 @@ class Artifact:
     """The resident RQ artifact on the device: codebooks and the code matrix
     in each layout a step may read (prepared once, outside timed regions)."""
 
-    def __init__(self, w, data, need=("sched", "u16", "u8", "packed10")):
+    def __init__(self, w, data, need=("sched", "u16", "u8", "packed10", "rot10")):
         import torch
         import lut_logits_serving_b200 as rq
         self.d = rq.dims(w.V, w.D, w.M, w.L, w.K)
@@ -642,6 +645,11 @@ class Artifact:
             sched, (st, ps) = rq.rq_prepare_sched(c16, self.d, stats=True)
             self.layouts["sched"] = (rq.SCHED, sched)
             self.sched_passes = ps / st
+        self.rot_passes = None
+        if "rot10" in need and w.K <= 1024 and w.P % 64 == 0:
+            rot, (st, ps) = rq.rq_prepare_rot10(c16, self.d, stats=True)
+            self.layouts["rot10"] = (rq.ROT10, rot)
+            self.rot_passes = ps / st
         if "u8" in need and w.K <= 256:
             self.layouts["u8"] = (rq.U8, rq.rq_pack8(c16, self.d))
         if "u16" in need:
@@ -654,7 +662,7 @@ class Artifact:
 
 def kernel_of(w, layout):
     decoded = layout in ("u16", "packed10", "sched") and decodable(w)
-    packed = w.packed10 or layout == "packed10"
+    packed = w.packed10 or layout in ("packed10", "rot10")
     if w.B <= 4 and (not packed or w.B == 1):
         return "logits_chunk_u16_kernel", decoded
     return ("logits_decode_mma_kernel" if decoded else "logits_l2_kernel"), decoded
@@ -790,6 +798,8 @@ def measure_logits(rig, w, art, layout, h_np, full=False, clk=None):
         others = {}
         for name, (f2, c2) in art.layouts.items():
             if name == layout or (name == "packed10") != w.packed10:
+                continue
+            if name == "rot10" and w.B > 1:   # the batch-1 layout of 10-bit codes
                 continue
             st2 = make_step(f2, c2)
             r2 = rig.graphed(st2)
@@ -1049,8 +1059,9 @@ def run_ours(args, w):
     torch = rig.torch
     data = synth.make(w, seed=rank_seed(rig.rank))
     extras = (not args.no_extras and w.name == "g2_b1" and not args.codes)
-    need = ("sched", "u16", "u8", "packed10") if (extras or w.packed10) else \
-        ("sched", "u16", "u8")
+    need = ("sched", "u16", "u8", "packed10", "rot10") if extras else \
+        ("sched", "u16", "u8", "packed10") if w.packed10 else ("sched", "u16", "u8") + \
+        (("rot10",) if args.codes == "rot10" else ())
     art = Artifact(w, data, need)
     art.codes_np, art.C_np = data["codes"], data["C"]
     headline = headline_layout(w, args.codes, tuple(k for k in art.layouts if k != "packed10"))
@@ -1068,6 +1079,12 @@ def run_ours(args, w):
         p1 = measure_logits(rig, w, art, "packed10", data["h"])
         p1.pop("t_ms", None)
         others["g2_b1_packed10"] = dict(p1, config=workload_config(w, "packed10"))
+        if "rot10" in art.layouts:
+            # the same 10-bit codes in rotated slices (rq_prepare_rot10)
+            r1 = measure_logits(rig, w, art, "rot10", data["h"])
+            r1.pop("t_ms", None)
+            r1["roofline"]["bank_passes_per_step"] = art.rot_passes
+            others["g2_b1_rot10"] = dict(r1, config=workload_config(w, "rot10"))
         for name in EXTRA_WORKLOADS:
             w2 = synth.WORKLOADS[name]
             seed = rank_seed(rig.rank)

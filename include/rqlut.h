@@ -103,7 +103,8 @@ enum rq_code_fmt {
     RQ_CODES_U16 = 0,       /* one uint16 per code (K <= 65536)           */
     RQ_CODES_PACKED10 = 1,  /* 10-bit codes, bit stream per row (K<=1024) */
     RQ_CODES_SCHED = 2,     /* bank-scheduled uint16 (rq_prepare_sched)   */
-    RQ_CODES_U8 = 3         /* one byte per code (K <= 256, rq_pack8)     */
+    RQ_CODES_U8 = 3,        /* one byte per code (K <= 256, rq_pack8)     */
+    RQ_CODES_PACKED10_ROT = 4 /* 10-bit codes, rotated slices (rq_prepare_rot10) */
 };
 
 enum rq_status {
@@ -374,6 +375,32 @@ RQ_API int rq_pack8(const uint16_t *codes_u16, rq_dims d, uint8_t *packed, void 
  *         (K > 1024 or M*L % 32 != 0), RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
  */
 RQ_API int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out,
+                            uint64_t *stats, void *stream);
+
+/*
+ * rq_prepare_rot10 -- convert uint16 codes [V][M*L] into
+ * RQ_CODES_PACKED10_ROT: the 10-bit packed rows with each 32-code slice
+ * rotated, plus one rotation byte per (row, slice).  Not on the pages: a
+ * layout of this library for the batch-1 pass on 10-bit codes, which has no
+ * room for RQ_CODES_SCHED's per-code positions; a rotation of each slice
+ * (5 bits per 32 codes) lets the 32 rows of a warp's step spread over the
+ * shared-memory banks (bank = (pair * K + code) mod 32): ~2.6 passes per step
+ * for random codes instead of ~3.5.  Same sums in another order.  Run once
+ * per artifact.
+ *   Layout: bytes [V][rb], rb = 10*M*L/8, then uint8 [M*L/32][V];
+ *   rq_codes_bytes(d, RQ_CODES_PACKED10_ROT) = V*rb + V*M*L/32.  Bits
+ *   [10j, 10j+10) of slice s (bits [320s, 320s+320) of the row, LSB first as
+ *   in RQ_CODES_PACKED10) hold the code of pair 32s + ((j + r) mod 32), with
+ *   r = the low 5 bits of rotation byte [s][v].
+ *   codes_u16 (device) uint16 [V][M*L], values < K (values >= 1024 keep
+ *             their low 10 bits); out (device) uint8, rq_codes_bytes(d,
+ *             RQ_CODES_PACKED10_ROT) bytes, 16-byte aligned, not
+ *             overlapping codes_u16; stats (device) uint64 [2] or NULL:
+ *             (steps, bank passes needed) summed over all warps.
+ * Errors: RQ_ERR_INVALID_ARGUMENT (null, bad dims), RQ_ERR_UNSUPPORTED
+ *         (K > 1024 or M*L % 64 != 0), RQ_ERR_MISALIGNED, RQ_ERR_CUDA.
+ */
+RQ_API int rq_prepare_rot10(const uint16_t *codes_u16, rq_dims d, uint8_t *out,
                             uint64_t *stats, void *stream);
 
 /*

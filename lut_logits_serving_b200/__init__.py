@@ -13,6 +13,8 @@ names:
   (``rq_logits_from_hidden_path`` picks tables, FP32 or tensor cores)
 * ``rq_decode_rows`` -- bf16 input rows rebuilt on demand
 * ``rq_pack10`` -- uint16 codes -> 10-bit packed rows
+* ``rq_prepare_sched``, ``rq_prepare_rot10`` -- the batch-1 layouts of
+  uint16 and 10-bit codes (bank-scheduled, rotated slices)
 
 (method: "Gemma-2 runtime compression: NF4 + LUT serving", LUT section.)
 There is no CPU fallback: if the library or a GPU is missing, calls raise.
@@ -24,7 +26,8 @@ import ctypes
 import os
 
 __all__ = [
-    "RqDims", "RqError", "U16", "PACKED10", "SCHED", "U8", "lib", "rq_pack8", "dims", "rq_prepare_sched",
+    "RqDims", "RqError", "U16", "PACKED10", "SCHED", "U8", "ROT10", "lib", "rq_pack8", "dims",
+    "rq_prepare_sched", "rq_prepare_rot10",
     "rq_status_string", "rq_version", "rq_codes_bytes", "rq_lut_token_stride",
     "rq_lut_bytes", "rq_logits_workspace_bytes", "rq_fused_workspace_bytes",
     "rq_lut_build", "rq_lut_logits", "rq_logits_from_hidden", "rq_logits_from_hidden_path",
@@ -39,6 +42,7 @@ U16 = 0
 PACKED10 = 1
 SCHED = 2
 U8 = 3
+ROT10 = 4        # RQ_CODES_PACKED10_ROT
 # kernel of full 32-token groups in rq_logits_from_hidden (rqlut.h RQ_PATH_*)
 PATH_AUTO = 0
 PATH_TABLES = 1
@@ -102,6 +106,7 @@ _SIGNATURES = {
     "rq_device_error": (_i, [ctypes.POINTER(ctypes.c_uint32), _i]),
     "rq_set_profile_events": (_i, [_p, _p]),
     "rq_prepare_sched": (_i, [_p, RqDims, _p, _p, _p]),
+    "rq_prepare_rot10": (_i, [_p, RqDims, _p, _p, _p]),
     "rq_lut_logits_static": (_i, [_p, _i, RqDims, _p, _i, _f, _p, _p, _p]),
     "rq_greedy_step": (_i, [_p, _p, _p, _i, RqDims, _i, _f, _p, _p, _f, _p, _p, _sz, _p]),
     "rq_argmax_candidates": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p]),
@@ -219,7 +224,7 @@ def _check(fn, status):
 
 def _codes_dtype(fmt):
     torch = _torch()
-    return torch.uint8 if fmt in (PACKED10, U8) else torch.uint16
+    return torch.uint8 if fmt in (PACKED10, U8, ROT10) else torch.uint16
 
 
 def _empty(shape, dtype, like):
@@ -483,6 +488,27 @@ def rq_prepare_sched(codes_u16, d: RqDims, out=None, stats=None, stream=None):
         _cuda(codes_u16, torch.uint16, "codes_u16", rq_codes_bytes(d, U16)), d,
         _cuda(out, torch.uint16, "out", rq_codes_bytes(d, SCHED)),
         _ptr_or_null(st, torch.int64, "stats", 16), _stream(stream)))
+    if stats:
+        v = st.cpu().tolist()
+        return out, (v[0], v[1])
+    return out
+
+
+def rq_prepare_rot10(codes_u16, d: RqDims, out=None, stats=None, stream=None):
+    """uint16 codes [V, P] -> RQ_CODES_PACKED10_ROT bytes (rotated 10-bit slices,
+    then the rotations).  With stats=True returns (out, (steps, bank passes))
+    after a sync."""
+    torch = _torch()
+    nbytes = rq_codes_bytes(d, ROT10)
+    if out is None:
+        out = torch.empty((nbytes,), dtype=torch.uint8, device=codes_u16.device)
+    st = None
+    if stats:
+        st = torch.zeros(2, dtype=torch.int64, device=codes_u16.device)
+    _check("rq_prepare_rot10", lib().rq_prepare_rot10(
+        _cuda(codes_u16, torch.uint16, "codes_u16", rq_codes_bytes(d, U16)), d,
+        _cuda(out, torch.uint8, "out", nbytes), _ptr_or_null(st, torch.int64, "stats", 16),
+        _stream(stream)))
     if stats:
         v = st.cpu().tolist()
         return out, (v[0], v[1])

@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(3 * kPairSub) decode_rows_pair_kernel(
         if (a.fmt == RQ_CODES_U16) c[r] = all16[v * P + p];
         else if (a.fmt == RQ_CODES_SCHED) c[r] = sched_code(all16, a.V, v, p, sched_shift(a.K));
         else if (a.fmt == RQ_CODES_U8) c[r] = all8[v * P + p];
+        else if (a.fmt == RQ_CODES_PACKED10_ROT) c[r] = rot10_code(all8, a.V, P, v, p);
         else c[r] = packed10_code(all8 + v * rb10, p);
       }
     }

@@ -42,6 +42,7 @@ struct ChunkArgs {
   int P, K, B, nch, cpc;
   CodeFix fix;
   unsigned *err;
+  const uint8_t *rot;  // RQ_CODES_PACKED10_ROT: rotations [P/32][V]
 };
 
 // Plain uint16 codes: TPR threads per row, 1024 threads.  Bank-scheduled codes
@@ -53,7 +54,7 @@ struct ChunkArgs {
 // the TMA box is the 48-byte, 16-byte-aligned window around it.
 template <int TB, int FMT>
 struct ChunkShape {
-  static constexpr bool PK10 = FMT == RQ_CODES_PACKED10;
+  static constexpr bool PK10 = FMT == RQ_CODES_PACKED10 || FMT == RQ_CODES_PACKED10_ROT;
   static constexpr bool WHOLE = FMT == RQ_CODES_SCHED || FMT == RQ_CODES_U8 || PK10;
   static constexpr int PC = WHOLE ? 32 : (TB == 1 ? 32 : (TB == 2 ? 16 : 8));  // pairs/chunk
   static constexpr int PPT = WHOLE ? 32 : (TB == 4 ? 8 : 16);                  // pairs/thread
@@ -231,13 +232,23 @@ __device__ __forceinline__ void pk10_loads(uint32_t tbase, int K, const uint32_t
     ((y[J] = lds_f32(tbase + (uint32_t)J * K * 4 + 4u * fix_code<KT>(pk10_code<J>(x), f))), ...);
 }
 
+// Rotated slices: slot J holds pair (J + rot) mod 32 of the chunk.
+template <int KT, int... J>
+__device__ __forceinline__ void pk10r_loads(uint32_t tbase, int K, const uint32_t (&x)[11],
+                                            const CodeFix &f, int rot, float (&y)[32],
+                                            std::integer_sequence<int, J...>) {
+  const uint32_t pb = (uint32_t)(KT > 0 ? KT : K) * 4u;
+  ((y[J] = lds_f32(tbase + (uint32_t)((J + rot) & 31) * pb + 4u * fix_code<KT>(pk10_code<J>(x), f))),
+   ...);
+}
+
 // RQ_CODES_PACKED10, one token: the row's 32 codes of this chunk are bits
 // [10j, 10j + 10) of its 40-byte slice, which begins 8 bytes into the
 // 48-byte window w when `skip8`, else at its start.  All 32 table loads are
 // issued before any add; the sum is a tree.
-template <int KT>
+template <int KT, bool ROT>
 __device__ __forceinline__ float chunk32_packed_tb1(uint32_t tbase, int K, const uint4 (&w)[3],
-                                                    bool skip8, const CodeFix &f) {
+                                                    bool skip8, const CodeFix &f, int rot) {
   const uint32_t a[12] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y,
                           w[1].z, w[1].w, w[2].x, w[2].y, w[2].z, w[2].w};
   uint32_t x[11];
@@ -245,7 +256,10 @@ __device__ __forceinline__ float chunk32_packed_tb1(uint32_t tbase, int K, const
   for (int i = 0; i < 10; ++i) x[i] = skip8 ? a[i + 2] : a[i];
   x[10] = 0u;
   float y[32];
-  pk10_loads<KT>(tbase, K, x, f, y, std::make_integer_sequence<int, 32>{});
+  if (ROT)
+    pk10r_loads<KT>(tbase, K, x, f, rot, y, std::make_integer_sequence<int, 32>{});
+  else
+    pk10_loads<KT>(tbase, K, x, f, y, std::make_integer_sequence<int, 32>{});
 #pragma unroll
   for (int st = 1; st < 32; st <<= 1)
 #pragma unroll
@@ -273,7 +287,8 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT>::THREADS, MINB)
     logits_chunk_u16_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
   constexpr bool SCHED = FMT == RQ_CODES_SCHED;
   constexpr bool U8 = FMT == RQ_CODES_U8;
-  constexpr bool PK10 = FMT == RQ_CODES_PACKED10;
+  constexpr bool PK10 = FMT == RQ_CODES_PACKED10 || FMT == RQ_CODES_PACKED10_ROT;
+  constexpr bool ROT = FMT == RQ_CODES_PACKED10_ROT;
   using S = ChunkShape<TB, FMT>;
   static_assert(!PK10 || (TB == 1 && S::PPT == 32), "a thread owns a whole 10-bit slice");
   static_assert(!SCHED || (TB == 1 && S::PPT == 32), "a thread owns a whole scheduled slice");
@@ -390,7 +405,13 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT>::THREADS, MINB)
 
   int s = 0;
   uint32_t phase = 0;
+  int rot_next = ROT && n > 0 && v < a.V ? __ldg(a.rot + (int64_t)c * a.V + v) & 31 : 0;
   for (int i = 0; i < n && table_ok; ++i) {
+    // this row's rotation of the chunk's slice (rotated 10-bit codes), loaded
+    // one tile ahead so that its latency hides behind a tile's lookups
+    const int rot = rot_next;
+    if (ROT)
+      rot_next = i + 1 < n && v + S::R < a.V ? __ldg(a.rot + (int64_t)c * a.V + v + S::R) & 31 : 0;
     const uint32_t fb = smem_addr(&full[s]);
     if (!mbar_try_wait(fb, phase) && !mbar_wait_bounded(fb, phase)) {
       *reinterpret_cast<volatile int *>(abort_flag) = 1;
@@ -420,7 +441,7 @@ __global__ void __launch_bounds__(ChunkShape<TB, FMT>::THREADS, MINB)
     if constexpr (SCHED) {
       acc[0] = chunk32_sched_tb1<KSH>(tt, w);   // the row's whole 32-pair slice
     } else if constexpr (PK10) {
-      acc[0] = chunk32_packed_tb1<KT>(tt, K, w, skip8, a.fix);
+      acc[0] = chunk32_packed_tb1<KT, ROT>(tt, K, w, skip8, a.fix, rot);
     } else if constexpr (U8) {
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
@@ -724,6 +745,8 @@ const Variant kVariants[] = {
     // 10-bit codes, one token: 128 KB of tables (K = 1024), three 24 KB stages
     RQ_CHUNK_VARIANT(1, 1024, 3, RQ_CODES_PACKED10, 0, 1),
     RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_PACKED10, 0, 1),
+    RQ_CHUNK_VARIANT(1, 1024, 3, RQ_CODES_PACKED10_ROT, 0, 1),
+    RQ_CHUNK_VARIANT(1, 0, 3, RQ_CODES_PACKED10_ROT, 0, 1),
 };
 
 size_t variant_smem(const Variant &v, int K) {
@@ -737,12 +760,12 @@ size_t variant_smem(const Variant &v, int K) {
 ChunkPlan plan_chunk(int64_t V, int P, int K, int B, int fmt, const DevInfo &di) {
   ChunkPlan cp{};
   cp.ok = false;
-  if ((fmt != RQ_CODES_U16 && fmt != RQ_CODES_SCHED && fmt != RQ_CODES_U8 &&
-       fmt != RQ_CODES_PACKED10) ||
-      B < 1 || B > 4 || P % 8 != 0 || K > 1024)
+  const bool pk10 = fmt == RQ_CODES_PACKED10 || fmt == RQ_CODES_PACKED10_ROT;
+  if ((fmt != RQ_CODES_U16 && fmt != RQ_CODES_SCHED && fmt != RQ_CODES_U8 && !pk10) || B < 1 ||
+      B > 4 || P % 8 != 0 || K > 1024)
     return cp;
   // 10-bit codes: one token, whole 64-code groups (80-byte, 16-byte-aligned rows)
-  if (fmt == RQ_CODES_PACKED10 && (B != 1 || P % 64 != 0)) return cp;
+  if (pk10 && (B != 1 || P % 64 != 0)) return cp;
   if (fmt == RQ_CODES_U8 && (K > 256 || P % 16 != 0)) return cp;   // 16-byte row pitch
   if (fmt == RQ_CODES_SCHED && P % 32 != 0) return cp;
   if (V > (int64_t)INT_MAX - 2048) return cp;
@@ -777,7 +800,7 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   const Variant &var = kVariants[cp.variant];
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
-  const bool pk = fmt == RQ_CODES_PACKED10;
+  const bool pk = fmt == RQ_CODES_PACKED10 || fmt == RQ_CODES_PACKED10_ROT;
   const int cb = fmt == RQ_CODES_U8 || pk ? 1 : 2;   // bytes per element of the map
   const int rowb = pk ? 48 : cp.PC * cb;
   // [V][P] for plain codes; the scheduled layout is chunk-major [P/32][V][32];
@@ -826,6 +849,9 @@ cudaError_t launch_logits_chunk(const ChunkPlan &cp, const void *codes, int fmt,
   a.cpc = (int)cpc;
   a.fix = make_codefix(K);
   a.err = di.err;
+  a.rot = fmt == RQ_CODES_PACKED10_ROT
+              ? static_cast<const uint8_t *>(codes) + V * ((int64_t)P / 64 * 80)
+              : nullptr;
   const int64_t grid = (int64_t)cp.nch * cpc;
   void *args[] = {&tmap, &a};
   return launch_maybe_pdl(var.fn, dim3((unsigned)grid), dim3(var.THREADS), cp.smem, s, args,

@@ -169,7 +169,14 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
       const uint4 *crow = reinterpret_cast<const uint4 *>(
           static_cast<const uint8_t *>(a.codes) + v * rb);
       const int ng = a.P / 64;
+      // rotated slices: the rotation bytes [P/32][V] after the V packed rows
+      const uint8_t *rotp = static_cast<const uint8_t *>(a.codes) + a.V * rb + v;
       for (int g = 0; g < ng; ++g) {
+        int r0 = 0, r1 = 0;
+        if (FMT == RQ_CODES_PACKED10_ROT) {
+          r0 = __ldg(rotp + (int64_t)(2 * g) * a.V) & 31;
+          r1 = __ldg(rotp + (int64_t)(2 * g + 1) * a.V) & 31;
+        }
         uint32_t w[21];
 #pragma unroll
         for (int k = 0; k < 5; ++k) {
@@ -185,7 +192,11 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         for (int j = 0; j < 64; ++j) {
           const int bit = 10 * j;
           const uint32_t c = a.fix(__funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & 0x3FFu);
-          add_vec<VW>(tg + ((size_t)j * K + c) * Bs, acc);
+          // slot j of a rotated slice holds pair (j + r) mod 32 of that slice
+          const int pj = FMT == RQ_CODES_PACKED10_ROT
+                             ? ((j & 32) | (((j & 31) + ((j & 32) ? r1 : r0)) & 31))
+                             : j;
+          add_vec<VW>(tg + ((size_t)pj * K + c) * Bs, acc);
         }
       }
     }
@@ -243,10 +254,12 @@ __global__ void __launch_bounds__(256) logits_generic_kernel(const L2Args a, int
         if (c < (uint32_t)a.K) z += __ldg(tl + ((size_t)pp * a.K + c) * a.Bs);
         continue;
       }
-      const uint32_t c = a.fix(fmt == RQ_CODES_U16  ? (uint32_t)c16[p]
-                               : fmt == RQ_CODES_U8 ? (uint32_t)static_cast<const uint8_t *>(
-                                                          a.codes)[v * a.P + p]
-                                                    : packed10_code(c8, p));
+      const uint32_t c = a.fix(
+          fmt == RQ_CODES_U16 ? (uint32_t)c16[p]
+          : fmt == RQ_CODES_U8 ? (uint32_t)static_cast<const uint8_t *>(a.codes)[v * a.P + p]
+          : fmt == RQ_CODES_PACKED10_ROT
+              ? rot10_code(static_cast<const uint8_t *>(a.codes), a.V, a.P, v, p)
+              : packed10_code(c8, p));
       z += __ldg(tl + ((size_t)p * a.K + c) * a.Bs);
     }
     const float y = softcap_f(z, a.cap);
@@ -338,6 +351,11 @@ cudaError_t launch_logits_l2(const void *codes, int fmt, int64_t V, int P, int K
     if (VW == 1) return launch_fast<1, 1, RQ_CODES_U8>(a, nblk, s);
     if (VW == 2) return launch_fast<2, 1, RQ_CODES_U8>(a, nblk, s);
     return launch_vw<4, RQ_CODES_U8>(a, G, nblk, s);
+  }
+  if (fmt == RQ_CODES_PACKED10_ROT) {
+    if (VW == 1) return launch_fast<1, 1, RQ_CODES_PACKED10_ROT>(a, nblk, s);
+    if (VW == 2) return launch_fast<2, 1, RQ_CODES_PACKED10_ROT>(a, nblk, s);
+    return launch_vw<4, RQ_CODES_PACKED10_ROT>(a, G, nblk, s);
   }
   if (VW == 1) return launch_fast<1, 1, RQ_CODES_PACKED10>(a, nblk, s);
   if (VW == 2) return launch_fast<2, 1, RQ_CODES_PACKED10>(a, nblk, s);

@@ -54,6 +54,16 @@ __device__ __forceinline__ uint32_t packed10_code(const uint8_t *row, int p) {
   return (w >> (bit & 7)) & 0x3FFu;
 }
 
+// Code p of row v of RQ_CODES_PACKED10_ROT (all: the layout's first byte, P
+// a multiple of 64): slot ((p mod 32) - r) mod 32 of the row's slice p / 32,
+// r the slice's rotation byte [p / 32][v] after the V packed rows.
+__device__ __forceinline__ uint32_t rot10_code(const uint8_t *all, int64_t V, int P, int64_t v,
+                                               int p) {
+  const int64_t rb = (int64_t)P / 8 * 10;
+  const int r = all[V * rb + (int64_t)(p >> 5) * V + v] & 31;
+  return packed10_code(all + v * rb, (p & ~31) | (((p & 31) - r) & 31));
+}
+
 // RQ_CODES_SCHED entry = (i << s) | c: i the pair's position in its 32-pair
 // slice, c the code, and 2^s the table stride -- the smallest power of two
 // >= K, at least 32, so that the shared-memory bank of the entry's table
@@ -117,6 +127,8 @@ __device__ __forceinline__ void decode_subspace(const DecodeSpec &a, int64_t id,
     if (a.fmt == RQ_CODES_U16) c = crow16[p];
     else if (a.fmt == RQ_CODES_SCHED) c = sched_code(all16, a.V, id, p, sched_shift(a.K));
     else if (a.fmt == RQ_CODES_U8) c = static_cast<const uint8_t *>(a.codes)[id * P + p];
+    else if (a.fmt == RQ_CODES_PACKED10_ROT)
+      c = rot10_code(static_cast<const uint8_t *>(a.codes), a.V, P, id, p);
     else c = packed10_code(crow10, p);
     return a.fix(c);
   };

@@ -97,6 +97,8 @@ cudaError_t launch_encode(const float *X, int64_t N, const float *C, int D, int 
                           uint16_t *codes, cudaStream_t s);
 cudaError_t launch_prepare_sched(const uint16_t *codes, int64_t V, int P, int K, uint16_t *out,
                                  unsigned long long *stats, cudaStream_t s);
+cudaError_t launch_prepare_rot10(const uint16_t *codes, int64_t V, int P, int K, uint8_t *out,
+                                 unsigned long long *stats, cudaStream_t s);
 
 // Vocabulary-tiled pass with the LUT chunk resident in shared memory.
 struct ChunkPlan {

@@ -112,7 +112,7 @@ bool dims_ok(const rq_dims &d) {
 
 bool fmt_known(int fmt) {
   return fmt == RQ_CODES_U16 || fmt == RQ_CODES_PACKED10 || fmt == RQ_CODES_SCHED ||
-         fmt == RQ_CODES_U8;
+         fmt == RQ_CODES_U8 || fmt == RQ_CODES_PACKED10_ROT;
 }
 
 bool fmt_ok(const rq_dims &d, int fmt) {
@@ -120,6 +120,7 @@ bool fmt_ok(const rq_dims &d, int fmt) {
   if (fmt == RQ_CODES_PACKED10) return d.K <= 1024;
   if (fmt == RQ_CODES_SCHED) return d.K <= 1024 && ((int64_t)d.M * d.L) % 32 == 0;
   if (fmt == RQ_CODES_U8) return d.K <= 256;
+  if (fmt == RQ_CODES_PACKED10_ROT) return d.K <= 1024 && ((int64_t)d.M * d.L) % 64 == 0;
   return false;
 }
 
@@ -361,6 +362,7 @@ size_t rq_codes_bytes(rq_dims d, int fmt) {
   const int64_t P = (int64_t)d.M * d.L;
   if (fmt == RQ_CODES_U16 || fmt == RQ_CODES_SCHED) return (size_t)(d.V * P * 2);
   if (fmt == RQ_CODES_U8) return (size_t)(d.V * P);
+  if (fmt == RQ_CODES_PACKED10_ROT) return (size_t)(d.V * (10 * P / 8) + d.V * (P / 32));
   return (size_t)(d.V * ((10 * P + 7) / 8));
 }
 
@@ -504,6 +506,21 @@ int rq_prepare_sched(const uint16_t *codes_u16, rq_dims d, uint16_t *out, uint64
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(codes_u16), b0 = reinterpret_cast<uintptr_t>(out);
   if (a0 < b0 + bytes && b0 < a0 + bytes) return RQ_ERR_INVALID_ARGUMENT;   // overlap
   return status_of(launch_prepare_sched(codes_u16, d.V, d.M * d.L, d.K, out,
+                                        reinterpret_cast<unsigned long long *>(stats),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int rq_prepare_rot10(const uint16_t *codes_u16, rq_dims d, uint8_t *out, uint64_t *stats,
+                     void *stream) {
+  if (!codes_u16 || !out || !dims_ok(d)) return RQ_ERR_INVALID_ARGUMENT;
+  if (!fmt_ok(d, RQ_CODES_PACKED10_ROT)) return RQ_ERR_UNSUPPORTED;
+  if (!aligned(codes_u16, 2) || !aligned(out, 16) || (stats && !aligned(stats, 8)))
+    return RQ_ERR_MISALIGNED;
+  const size_t in_bytes = rq_codes_bytes(d, RQ_CODES_U16);
+  const size_t out_bytes = rq_codes_bytes(d, RQ_CODES_PACKED10_ROT);
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(codes_u16), b0 = reinterpret_cast<uintptr_t>(out);
+  if (a0 < b0 + out_bytes && b0 < a0 + in_bytes) return RQ_ERR_INVALID_ARGUMENT;   // overlap
+  return status_of(launch_prepare_rot10(codes_u16, d.V, d.M * d.L, d.K, out,
                                         reinterpret_cast<unsigned long long *>(stats),
                                         static_cast<cudaStream_t>(stream)));
 }

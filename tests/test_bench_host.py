@@ -127,3 +127,8 @@ def test_packed_code_bytes_on_a_uint16_workload():
     """A batch-1 workload timed on 10-bit packed codes divides by the packed
     matrix (960 B per row), not by the uint16 one."""
     assert bench.code_bytes(synth.WORKLOADS["g2_b1"], "packed10") == 256000 * 960
+    # the rotated slices add one byte per 32 codes
+    assert bench.code_bytes(synth.WORKLOADS["g2_b1"], "rot10") == 256000 * (960 + 24)
+    c = bench.workload_config(synth.WORKLOADS["g2_b1"], "packed10")
+    assert c["codes"] == "packed10" and "packed10 (960 B/row)" in c["workload"]
+    assert "rotated" in bench.workload_config(synth.WORKLOADS["g2_b1"], "rot10")["workload"]

@@ -85,6 +85,16 @@ def test_g2_batch1_full_sweep(g2):
     assert check_argmax(am5.cpu().numpy(), ref) == 0
     assert torch.equal(am5, am3)
     assert torch.equal(rows5, rows4)
+    # the rotated 10-bit layout: the same sums in another order
+    rot, (steps, passes) = rq.rq_prepare_rot10(g2["dc"], d, stats=True)
+    print(f"g2_b1 rotated slices: {passes / steps:.3f} bank passes per step")
+    logits6, am6, rows6, _ = rq.rq_greedy_step(dev(h), g2["dC"], rot, rq.ROT10, d, w.softcap,
+                                               scale=w.decode_scale)
+    err6 = assert_logits_close(logits6.cpu().numpy(), ref)
+    print(f"g2_b1 rot10 normwise error {err6:.3g}")
+    assert check_argmax(am6.cpu().numpy(), ref) == 0
+    assert torch.equal(am6, am3)
+    assert torch.equal(rows6, rows4)
     assert rq.rq_device_error() == 0
 
 
@@ -163,12 +173,13 @@ def test_g2_packed_batch64_fused_argmax(g2, path):
     assert ties == 0
 
 
-@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["u16", "packed10", "sched"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 4], ids=["u16", "packed10", "sched", "rot10"])
 def test_decode512_bit_exact(g2, fmt):
     w = synth.WORKLOADS["decode512"]
     ids = synth.zipf_ids(w.n_ids, w.V, w.zipf_s, 3)
     codes_dev = {0: lambda: g2["dc"], 1: lambda: rq.rq_pack10(g2["dc"], g2["d"]),
-                 2: lambda: rq.rq_prepare_sched(g2["dc"], g2["d"])}[fmt]()
+                 2: lambda: rq.rq_prepare_sched(g2["dc"], g2["d"]),
+                 4: lambda: rq.rq_prepare_rot10(g2["dc"], g2["d"])}[fmt]()
     out = rq.rq_decode_rows(dev(ids), codes_dev, fmt, g2["dC"], g2["d"], w.decode_scale)
     got = out.view(torch.int16).cpu().numpy().view(np.uint16)
     want = oracle.decode_rows_bf16(ids, g2["codes"], g2["C"], w.decode_scale)

@@ -40,6 +40,8 @@ def gpu_codes(codes, fmt, d):
         return rq.rq_prepare_sched(c16, d)
     if fmt == rq.U8:
         return rq.rq_pack8(c16, d)
+    if fmt == rq.ROT10:
+        return rq.rq_prepare_rot10(c16, d)
     return rq.rq_pack10(c16, d)
 
 
@@ -50,6 +52,8 @@ def fmt_applies(fmt, M, L, K):
         return K <= 1024 and (M * L) % 32 == 0
     if fmt == rq.U8:
         return K <= 256
+    if fmt == rq.ROT10:
+        return K <= 1024 and (M * L) % 64 == 0
     return True
 
 
@@ -92,7 +96,7 @@ CASES = [
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "V%d_D%d_M%d_L%d_K%d" % c)
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 13, 32, 33])
-@pytest.mark.parametrize("fmt", [0, 1, 2, 3], ids=["u16", "packed10", "sched", "u8"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3, 4], ids=["u16", "packed10", "sched", "u8", "rot10"])
 def test_logits_and_argmax(case, B, fmt):
     V, D, M, L, K = case
     if not fmt_applies(fmt, M, L, K):
@@ -198,9 +202,43 @@ def test_out_of_range_codes_stay_in_bounds():
         assert_logits_close(got.cpu().numpy(), ref)
 
 
+def unrotate10(buf, V, P):
+    """The RQ_CODES_PACKED10_ROT bytes back to uint16 codes [V, P], from the
+    layout's definition: V packed rows of 10 P / 8 bytes (code slot q at bits
+    [10q, 10q + 10), LSB first), then the rotations uint8 [P / 32][V]; slot j of
+    slice s holds pair 32 s + (j + r) mod 32."""
+    rb = P // 8 * 10
+    rows = np.asarray(buf[:V * rb], np.uint8).reshape(V, rb)
+    rot = np.asarray(buf[V * rb:V * rb + V * (P // 32)], np.uint8).reshape(P // 32, V) & 31
+    bits = np.unpackbits(rows, axis=1, bitorder="little").reshape(V, P, 10).astype(np.int64)
+    slots = (bits << np.arange(10)).sum(axis=2)                       # [V, P] by slot
+    out = np.empty((V, P), np.int64)
+    j = np.arange(32)
+    for sl in range(P // 32):
+        pair = 32 * sl + (j[None, :] + rot[sl][:, None].astype(np.int64)) % 32
+        np.put_along_axis(out, pair, slots[:, 32 * sl:32 * sl + 32], axis=1)
+    return out
+
+
+@pytest.mark.parametrize("V,P,K", [(4099, 64, 256), (1000, 128, 1024), (33, 192, 100)])
+def test_rotated_layout_holds_the_codes(V, P, K):
+    """rq_prepare_rot10 writes every row's codes, each slice rotated by its own
+    byte, and its rotations leave fewer bank passes than the plain order."""
+    codes = synth.codes(V, P // 2, 2, K, V)
+    d = rq.dims(V, 6 * (P // 2), P // 2, 2, K)
+    buf, (steps, passes) = rq.rq_prepare_rot10(dev(codes.reshape(V, -1)), d, stats=True)
+    assert buf.numel() == rq.rq_codes_bytes(d, rq.ROT10) == V * (P // 8 * 10 + P // 32)
+    got = unrotate10(buf.cpu().numpy(), V, P)
+    assert np.array_equal(got, codes.reshape(V, -1).astype(np.int64))
+    assert steps == 32 * ((V + 31) // 32) * (P // 32)
+    if K % 32 == 0 and V >= 1000:
+        # plain order: ~3.5 passes per step for random codes
+        assert passes / steps < 3.0
+
+
 # ------------------------------------------------------------ row decode
 
-@pytest.mark.parametrize("fmt", [0, 1, 2, 3], ids=["u16", "packed10", "sched", "u8"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3, 4], ids=["u16", "packed10", "sched", "u8", "rot10"])
 @pytest.mark.parametrize("shape", [(4096, 192, 32, 2, 256), (5000, 288, 48, 2, 1024),
                                    (300, 96, 16, 3, 100), (50, 9, 3, 1, 7)])
 def test_decode_rows_bit_exact(shape, fmt):
@@ -363,7 +401,7 @@ def test_prepare_sched_rejects_unsupported_shapes():
 # ------------------------------------------------------------ greedy step
 
 @pytest.mark.parametrize("B", [1, 3, 5, 33])
-@pytest.mark.parametrize("fmt", [0, 1, 2, 3], ids=["u16", "packed10", "sched", "u8"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3, 4], ids=["u16", "packed10", "sched", "u8", "rot10"])
 def test_greedy_step_rows_are_the_picked_tokens_rows(B, fmt):
     V, D, M, L, K = 3000, 192, 32, 2, 256
     C, codes, h = make_case(V, D, M, L, K, B, seed=B)
