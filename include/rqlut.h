@@ -69,6 +69,12 @@
  *                               time of RQ_CODES_U16 there, one stage of
  *                               codes in flight instead of two), other groups
  *                               read it in the generic lookup order.
+ *            RQ_CODES_PACKED10_ROT: uint8, the 10-bit rows (M*L % 64 == 0,
+ *                               K <= 1024) with each 32-code slice rotated,
+ *                               then one rotation byte per (slice, row),
+ *                               written by rq_prepare_rot10 (see there).
+ *                               Batch 1 and token groups read through L2
+ *                               take it; the decode paths do not.
  *   lut      float [M*L][K][Bs], Bs = rq_lut_token_stride(B): token b of
  *            table (p, k) at lut[(p*K + k)*Bs + b]
  *   logits   float [B][V]
