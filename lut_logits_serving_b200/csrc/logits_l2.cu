@@ -36,6 +36,25 @@ struct L2Args {
   int ssh;            // RQ_CODES_SCHED entry shift (table stride 2^ssh)
 };
 
+// 16-byte loads with an L2 eviction hint: the code stream is read once
+// (evict first), the group's tables are read throughout the pass (evict
+// last), so the stream does not push table lines out to DRAM.
+__device__ __forceinline__ uint4 ldg_u4_hint(const uint4 *p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ float4 ldg_f4_hint(const float *p, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
 template <int VW>
 __device__ __forceinline__ void add_vec(const float *e, float (&acc)[VW]) {
   if (VW == 1) {
@@ -45,7 +64,9 @@ __device__ __forceinline__ void add_vec(const float *e, float (&acc)[VW]) {
     acc[0] += t.x;
     acc[1] += t.y;
   } else {
-    const float4 t = __ldg(reinterpret_cast<const float4 *>(e));
+    // (the policy made at each load: measured faster than one kept in a
+    // register across the loop, 1394 vs 1490 us for a 32-token group)
+    const float4 t = ldg_f4_hint(e, l2_policy_evict_last());
     acc[0] += t.x;
     acc[1] += t.y;
     acc[2] += t.z;
@@ -56,6 +77,7 @@ __device__ __forceinline__ void add_vec(const float *e, float (&acc)[VW]) {
 template <int VW, int G, int FMT>
 __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
   griddep_wait();
+  const uint64_t pcode = l2_policy_evict_first();
   constexpr int RPW = 32 / G;     // rows per warp
   constexpr int RPB = 8 * RPW;    // rows per CTA step
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -87,7 +109,7 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         uint32_t wd[32];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint4 w = __ldg(crow + 8 * g + k);
+          const uint4 w = ldg_u4_hint(crow + 8 * g + k, pcode);
           wd[4 * k + 0] = w.x;
           wd[4 * k + 1] = w.y;
           wd[4 * k + 2] = w.z;
@@ -101,7 +123,7 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         }
       }
       for (int g = n64 * 8; g < a.P / 8; ++g) {
-        const uint4 w = __ldg(crow + g);
+        const uint4 w = ldg_u4_hint(crow + g, pcode);
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
         const float *tg = tl + (size_t)(8 * g) * K * Bs;
 #pragma unroll
@@ -120,7 +142,7 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         uint32_t wd[16];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint4 w = g + k < n16 ? __ldg(crow + g + k) : make_uint4(0, 0, 0, 0);
+          const uint4 w = g + k < n16 ? ldg_u4_hint(crow + g + k, pcode) : make_uint4(0, 0, 0, 0);
           wd[4 * k + 0] = w.x;
           wd[4 * k + 1] = w.y;
           wd[4 * k + 2] = w.z;
@@ -148,7 +170,7 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         uint32_t wd[16];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint4 w = __ldg(crow + k);
+          const uint4 w = ldg_u4_hint(crow + k, pcode);
           wd[4 * k + 0] = w.x;
           wd[4 * k + 1] = w.y;
           wd[4 * k + 2] = w.z;
@@ -180,7 +202,7 @@ __global__ void __launch_bounds__(256) logits_l2_kernel(const L2Args a) {
         uint32_t w[21];
 #pragma unroll
         for (int k = 0; k < 5; ++k) {
-          const uint4 x = __ldg(crow + 5 * g + k);
+          const uint4 x = ldg_u4_hint(crow + 5 * g + k, pcode);
           w[4 * k + 0] = x.x;
           w[4 * k + 1] = x.y;
           w[4 * k + 2] = x.z;
