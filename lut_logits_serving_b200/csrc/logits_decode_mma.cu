@@ -66,6 +66,17 @@ namespace rq {
 
 namespace {
 
+// Bulk copy global -> this CTA's shared memory (no multicast) with an L2
+// cache policy for the source lines.
+__device__ __forceinline__ void bulk_g2s_keep(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+      : "memory");
+}
+
 // Shape of one instance: NT tokens per group, FMT the code format.
 template <int NT, int FMT>
 struct DmShape {
@@ -423,7 +434,9 @@ __global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
   if (warp == DW + 1) {
     // ------------------------------------------------------------ copies
     if (lane == 0 && S > 0) {
-      const uint64_t pol_codes = l2_policy_evict_first();
+      // codes stream once (evict first); the codebooks (a few tens of MB) are
+      // read by every CTA on every pass and should stay in L2 (evict last)
+      const uint64_t pol_codes = l2_policy_evict_first(), pol_books = l2_policy_evict_last();
       int last_codes[ST], last_book[NB];
       for (int i = 0; i < ST; ++i) last_codes[i] = -1;
       for (int i = 0; i < NB; ++i) last_book[i] = -1;
@@ -454,7 +467,8 @@ __global__ void __launch_bounds__(DmShape<NT, FMT>::THREADS, 1)
         const int m = s % M;
         const uint32_t b = bar_at(kBarBook + s % NB);
         mbar_arrive_expect_tx(b, cbb + S_::HBYTES);
-        bulk_g2s(smem_addr(cb + (size_t)(s % NB) * cbs), a.C + (size_t)m * cbf, cbb, b);
+        bulk_g2s_keep(smem_addr(cb + (size_t)(s % NB) * cbs), a.C + (size_t)m * cbf, cbb, b,
+                      pol_books);
         bulk_g2s(smem_addr(hs + (s % kDmHSlots) * S_::HBYTES),
                  reinterpret_cast<const unsigned char *>(a.hop) + kDmHopHead +
                      (size_t)m * S_::HBYTES,
